@@ -1,0 +1,95 @@
+"""The pins catch plausible slips in the oracle.
+
+Each case copies the oracle's C source, plants one slip (a wrong rounding, a
+dropped term, a flipped sign, an off-by-one index, a wrong tie-break),
+builds it, and runs tests/test_oracle_pins.py against that copy in a child
+process.  The pins must fail for every mutant.  Nothing here touches a GPU.
+"""
+import os
+import shutil
+import subprocess
+import sys
+import tempfile
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "sq_oracle.c")
+
+MUTANTS = {
+    "round_floor_half_up": ("double r = round(t);", "double r = floor(t + 0.5);"),
+    "scale_divides_by_128": ("return (float)(a / 127.0);", "return (float)(a / 128.0);"),
+    "clip_to_minus_128": ("if (r < -127.0)\n        r = -127.0;", "if (r < -128.0)\n        r = -128.0;"),
+    "sign_of_zero_negative": ("(uint8_t)(w[j] >= 0.0f)", "(uint8_t)(w[j] > 0.0f)"),
+    "residual_adds_trunk": ("t = sign[row * K + j] ? (double)a : -(double)a;",
+                            "t = sign[row * K + j] ? -(double)a : (double)a;"),
+    "alpha_over_all_entries": ("            if (mask[row * K + j]) {\n                sum +=",
+                               "            if (1) {\n                sum +="),
+    "threshold_not_strict": ("(fabsf(w[j]) > tau)", "(fabsf(w[j]) >= tau)"),
+    "percentile_rank_off_by_one": ("((int64_t)P * K + 99) / 100", "((int64_t)P * K) / 100 + 1"),
+    "group_drops_last_channel": ("int64_t j1 = j0 + G < K ? j0 + G : K;",
+                                 "int64_t j1 = j0 + G < K ? j0 + G - 1 : K;"),
+    "act_absmax_includes_outliers": ("if (!is_out[j] && fabs((double)v[j]) > a)",
+                                     "if (fabs((double)v[j]) > a)"),
+    "outlier_term_dropped": ("out += dequant_weight(sign, mask, alpha, q, s, K, ng, G, r, idx[i]) *",
+                             "out += 0.0 * dequant_weight(sign, mask, alpha, q, s, K, ng, G, r, idx[i]) *"),
+    "outlier_weight_without_residual": ("return t + (double)s[r * ng + j / G] * (double)q[r * K + j];",
+                                        "return t;"),
+    "calibration_ties_to_higher_index": ("(best < 0 || mag[j] > mag[best])",
+                                         "(best < 0 || mag[j] >= mag[best])"),
+    "popcount_sign_plane_positive": ("int64_t c = p < 7 ? ((int64_t)1 << p) : -128;",
+                                     "int64_t c = p < 7 ? ((int64_t)1 << p) : 128;"),
+    "trunk_scale_missing": ("double inner = (double)alpha[r] * (double)T[t * N + r];",
+                            "double inner = (double)T[t * N + r];"),
+    "group_scale_index_shifted": ("inner += (double)s[r * ng + g] * (double)R[(t * N + r) * ng + g];",
+                                  "inner += (double)s[r * ng + (g + 1) % ng] * (double)R[(t * N + r) * ng + g];"),
+}
+
+
+def _build_mutant(tmp, name, old, new):
+    src = open(SRC, encoding="utf-8").read()
+    assert src.count(old) == 1, f"{name}: pattern must occur exactly once"
+    d = os.path.join(tmp, name)
+    os.makedirs(d)
+    shutil.copy(os.path.join(ROOT, "oracle", "sq_oracle.h"), d)
+    with open(os.path.join(d, "sq_oracle.c"), "w", encoding="utf-8") as f:
+        f.write(src.replace(old, new))
+    lib = os.path.join(d, "libmutant.so")
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fPIC", "-shared",
+                           "-o", lib, os.path.join(d, "sq_oracle.c"), "-lm"])
+    return lib
+
+
+def test_every_mutant_is_caught():
+    tmp = tempfile.mkdtemp(prefix="sq_mutants_")
+    try:
+        procs = {}
+        for name, (old, new) in MUTANTS.items():
+            lib = _build_mutant(tmp, name, old, new)
+            env = dict(os.environ, SQ_ORACLE_LIB=lib)
+            procs[name] = subprocess.Popen(
+                [sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
+                 os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                cwd=ROOT, env=env, stdout=subprocess.PIPE, stderr=subprocess.STDOUT)
+        survivors = []
+        for name, p in procs.items():
+            out, _ = p.communicate(timeout=600)
+            if p.returncode == 0:
+                survivors.append(name)
+        assert not survivors, f"mutants not caught by the pins: {survivors}"
+    finally:
+        shutil.rmtree(tmp, ignore_errors=True)
+
+
+def test_unmutated_copy_passes():
+    """Control: the same harness with no slip planted passes."""
+    tmp = tempfile.mkdtemp(prefix="sq_control_")
+    try:
+        lib = _build_mutant(tmp, "control", "#include <math.h>", "#include <math.h>")
+        env = dict(os.environ, SQ_ORACLE_LIB=lib)
+        r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
+                            os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                           cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+        assert r.returncode == 0, r.stdout[-2000:]
+    finally:
+        shutil.rmtree(tmp, ignore_errors=True)

@@ -1,0 +1,390 @@
+"""Pins of the CPU oracle to facts that do not come from the oracle itself.
+
+Each test ties one oracle function to a worked example printed on the pages
+(fixtures under tests/golden/, each with its citation), a closed form, an
+exact brute force, a library routine for a special case, or an independent
+second route.  A plausible slip in the oracle (dropped term, wrong sign,
+wrong index, wrong rounding, wrong tie-break) fails at least one of them;
+tests/test_oracle_mutants.py plants such slips in a copy of the oracle and
+checks that this file catches each.
+"""
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from synth import workloads as wl
+from conftest import read_golden
+
+
+def F(v):
+    return Fraction(float(v))
+
+
+# ---- quantizer ---------------------------------------------------------------
+
+def test_absmax_worked_example():
+    """2048ai.net s3.1: alpha=10.8 -> s=alpha/127; 3.08 and 3.02 -> 36 -> ~3.06."""
+    g = read_golden("absmax_worked_example.txt")
+    alpha = float(next(v for k, v in g if k == "alpha")[0])
+    s = oracle.scale_from_absmax(alpha)
+    # s is the float nearest to alpha/127 (closed form, exact rational check)
+    exact = Fraction(alpha) / 127
+    assert abs(F(s) - exact) <= abs(F(np.nextafter(s, np.float32(1))) - exact)
+    assert abs(F(s) - exact) <= abs(F(np.nextafter(s, np.float32(0))) - exact)
+    for key, vals in g:
+        if key == "code":
+            assert oracle.quantize(float(vals[0]), s) == int(vals[1]), vals
+        if key == "dequant":
+            q, expect, tol = int(vals[0]), float(vals[1]), float(vals[2])
+            assert abs(q * float(s) - expect) <= tol
+
+
+def test_range_is_symmetric_127():
+    """Visual guide: [-127, 127], not [-128, 127]; values beyond clip."""
+    s = oracle.scale_from_absmax(1.0)
+    assert oracle.quantize(1e6, s) == 127
+    assert oracle.quantize(-1e6, s) == -127
+    assert oracle.quantize(-1.0, s) == -127
+    assert oracle.quantize(1.0, s) == 127
+    assert oracle.quantize(0.3, 0.0) == 0       # zero scale -> zero code
+
+
+@pytest.mark.parametrize("v,s,q", [
+    (2.5, 1.0, 3), (-2.5, 1.0, -3), (0.5, 1.0, 1), (-0.5, 1.0, -1), (1.5, 1.0, 2),
+    (-1.5, 1.0, -2), (1.25, 0.5, 3), (0.49999999999999994, 1.0, 0), (126.5, 1.0, 127),
+    (-126.5, 1.0, -127), (0.0, 1.0, 0), (-0.0, 1.0, 0)])
+def test_round_half_away_from_zero(v, s, q):
+    assert oracle.quantize(v, s) == q
+
+
+def _brute_code(r: Fraction, s: Fraction) -> int:
+    """argmin over all 255 codes of |r - q*s|, ties to the larger |q|."""
+    best, best_err = 0, None
+    for q in range(-127, 128):
+        err = abs(r - q * s)
+        if best_err is None or err < best_err or (err == best_err and abs(q) > abs(best)):
+            best, best_err = q, err
+    return best
+
+
+def test_group_codes_brute_force_8x8():
+    rng = np.random.default_rng(7)
+    r = rng.laplace(0, 0.02, (8, 8))
+    r[3, :4] = 0.0                      # an all-zero group
+    r[5, 5] = 0.5 * r[5, 4]             # exact half-way structure
+    for row in r:
+        q, s = oracle.quantize_groups(row, 4)
+        for g in range(2):
+            blk = row[4 * g:4 * g + 4]
+            a = max(abs(float(v)) for v in blk)
+            assert (s[g] == 0) == (a == 0)
+            for j, v in enumerate(blk):
+                expect = 0 if s[g] == 0 else _brute_code(Fraction(float(v)), F(s[g]))
+                assert q[4 * g + j] == expect
+            if a > 0:  # the group maximum lands on the end of the range
+                jm = int(np.argmax(np.abs(blk)))
+                assert abs(int(q[4 * g + jm])) == 127
+
+
+def test_dequant_error_bound():
+    """Visual guide e_i = x_i - xhat_i; round-to-nearest bounds it by s/2."""
+    W = wl.config1().weights()[:64]
+    d = oracle.decompose(W, want_residual=True)
+    ng = d["s"].shape[1]
+    for r in range(W.shape[0]):
+        for g in range(ng):
+            s = float(d["s"][r, g])
+            blk = slice(128 * g, 128 * g + 128)
+            err = np.abs(d["res"][r, blk] - d["q"][r, blk].astype(np.float64) * s)
+            assert np.all(err <= s / 2)
+
+
+def test_group_scaling_example():
+    """Visual guide Q4_K section: two blocks of four beat one shared scale."""
+    g = dict(read_golden("group_scaling_example.txt"))
+    row = np.array([float(v) for v in g["row"]])
+    blk = int(g["block"][0])
+    qg, sg = oracle.quantize_groups(row, blk)
+    qs, ss = oracle.quantize_groups(row, len(row))
+    err_g = np.abs(row - qg * np.repeat(sg.astype(np.float64), blk))
+    err_s = np.abs(row - qs * float(ss[0]))
+    assert err_g.max() < err_s.max()
+    # the small-valued first block gains the most from its own scale
+    assert err_g[:blk].max() * 10 < err_s[:blk].max()
+    assert sg[0] < sg[1] and ss[0] == sg[1]
+
+
+# ---- threshold, sign and alpha -----------------------------------------------
+
+def test_threshold_is_smallest_value_reaching_the_percentile():
+    """Nearest-rank percentile = min{v in |w| : #(|w| <= v) * 100 >= P * K}."""
+    rng = np.random.default_rng(3)
+    for K in (1, 7, 100, 4096):
+        w = rng.laplace(0, 0.02, K).astype(np.float32)
+        w[: K // 7] = np.round(w[: K // 7], 2)          # some ties
+        a = np.abs(w)
+        for P in (1, 50, 60, 80, 100):
+            tau = oracle.trunk_threshold(w, P)
+            assert tau in a
+            assert int((a <= tau).sum()) * 100 >= P * K
+            below = a[a < tau]
+            if below.size:
+                assert int((a <= below.max()).sum()) * 100 < P * K, (K, P)
+
+
+def test_threshold_closed_form():
+    """|W| = 1..10, 60th percentile (nearest rank 6) -> tau 6, trunk {7..10}."""
+    w = np.array([1, -2, 3, -4, 5, -6, 7, -8, 9, -10], np.float32)
+    assert oracle.trunk_threshold(w, 60) == 6.0
+    d = oracle.decompose(w[None, :], G=32, P=60)
+    assert d["mask"][0].tolist() == [0] * 6 + [1] * 4
+    assert d["alpha"][0] == np.float32(8.5)
+
+
+def test_sign_tiebreak_zero_is_positive():
+    """BitNet weight binarization: non-negative -> +1 (both zeros)."""
+    w = np.array([[0.0, -0.0, 1.0, -1.0, 1e-30, -1e-30]], np.float32)
+    d = oracle.decompose(w, G=32)
+    assert d["sign"][0].tolist() == [1, 1, 1, 0, 1, 0]
+
+
+def test_alpha_closed_form_full_trunk():
+    w = np.array([[0.5, -1.5, 1.5, -0.5, 2.0, -0.0]], np.float32)
+    d = oracle.decompose(w, G=32)
+    assert d["alpha"][0] == np.float32(1.0)     # (0.5+1.5+1.5+0.5+2+0)/6
+    w2 = np.zeros((1, 40), np.float32)
+    assert oracle.decompose(w2, G=32)["alpha"][0] == 0.0
+
+
+def test_empty_trunk_at_100th_percentile():
+    w = np.array([[0.25, -0.5, 0.125, 0.5]], np.float32)
+    d = oracle.decompose(w, G=32, P=100)
+    assert d["mask"].sum() == 0 and d["alpha"][0] == 0.0
+    # everything is residual: codes of W itself
+    assert d["q"][0].tolist() == [64, -127, 32, 127]
+
+
+# ---- decomposition identity ----------------------------------------------------
+
+@pytest.mark.parametrize("P", [-1, 60])
+def test_residual_plus_trunk_is_W(P):
+    """m.lqnn.cn s2.1: W_res = W - alpha*sign(W), exactly, before rounding."""
+    W = wl.config1().weights()
+    d = oracle.decompose(W, P=P, want_residual=True)
+    trunk = d["mask"] * (2.0 * d["sign"] - 1.0) * d["alpha"].astype(np.float64)[:, None]
+    recon = d["res"] + trunk
+    ok = np.abs(W) >= 2.0 ** -29 * d["alpha"][:, None]
+    assert np.all(recon[ok] == W.astype(np.float64)[ok])
+    assert ok.all()
+
+
+# ---- exact end-to-end closed forms ---------------------------------------------
+
+def _exact_row(rng, K, big=None):
+    """A row whose decomposition is lossless: alpha exact, residual codes exact.
+
+    Trunk magnitudes come in pairs 1 +- c/1024 (mean exactly 1); every group
+    of 128 holds one |c| = 127 so its scale is exactly 2^-10.  With ``big``,
+    the trunk entries are ``big +- c/1024`` and the other half of the row
+    holds residual-only entries c/1024.
+    """
+    c = rng.integers(0, 128, K)
+    for g0 in range(0, K, 128):
+        c[g0] = 127
+    sgn = rng.choice([-1.0, 1.0], K)
+    w = np.zeros(K)
+    if big is None:
+        pm = np.ones(K)
+        pm[1::2] = -1.0
+        if K % 2:
+            c[-1] = 0 if K - 1 != (K - 1) // 128 * 128 else c[-1]
+            pm[-1] = 1.0 if c[-1] == 0 else pm[-1]
+        # pair (2i, 2i+1): +c and -c of the same c keep the mean at 1
+        c[1::2] = c[0:K - 1:2][:len(c[1::2])]
+        w = sgn * (1.0 + pm * c / 1024.0)
+    else:
+        in_trunk = np.zeros(K, bool)
+        in_trunk[K // 2:] = True
+        pm = np.ones(K)
+        pm[K // 2 + 1::2] = -1.0
+        ct = c.copy()
+        ct[K // 2 + 1::2] = ct[K // 2:K - 1:2][:len(ct[K // 2 + 1::2])]
+        w = np.where(in_trunk, sgn * (big + pm * ct / 1024.0), sgn * c / 1024.0)
+    return w.astype(np.float32)
+
+
+@pytest.mark.parametrize("K", [128, 130, 256, 384])
+def test_lossless_row_gives_exact_dot(K):
+    rng = np.random.default_rng(K)
+    N = 6
+    W = np.stack([_exact_row(rng, K) for _ in range(N)])
+    d = oracle.decompose(W, G=128)
+    assert np.all(d["alpha"] == 1.0)
+    ng = d["s"].shape[1]
+    # all groups hold a 127 code except possibly a short tail group
+    assert np.all(d["s"][:, :K // 128] == np.float32(2.0 ** -10))
+    x = rng.integers(-127, 128, (2, K)).astype(np.float32)
+    x[:, 5] = 127.0
+    idx = np.array([9, K - 1], np.int32)
+    x[0, 9], x[0, K - 1] = 1000.25, -333.5
+    x[1, 9], x[1, K - 1] = -4096.0, 0.75
+    xq, sx, xout = oracle.quantize_act(x, idx)
+    assert np.all(sx == 1.0)                    # absmax excludes the outliers
+    y = oracle.linear(d, xq, sx, xout, idx)
+    for t in range(2):
+        for r in range(N):
+            exact = sum(F(W[r, j]) * F(x[t, j]) for j in range(K))
+            assert Fraction(y[t, r]) == exact
+    assert ng == (K + 127) // 128
+
+
+def test_lossless_threshold_row_gives_exact_dot():
+    rng = np.random.default_rng(11)
+    K = 256
+    W = np.stack([_exact_row(rng, K, big=4.0) for _ in range(4)])
+    d = oracle.decompose(W, G=128, P=50)
+    assert np.all(d["mask"][:, K // 2:] == 1) and np.all(d["mask"][:, :K // 2] == 0)
+    assert np.all(d["alpha"] == 4.0)
+    x = rng.integers(-127, 128, (1, K)).astype(np.float32)
+    x[0, 0] = -127.0
+    idx = np.array([200], np.int32)
+    x[0, 200] = 77.125
+    xq, sx, xout = oracle.quantize_act(x, idx)
+    y = oracle.linear(d, xq, sx, xout, idx)
+    for r in range(4):
+        exact = sum(F(W[r, j]) * F(x[0, j]) for j in range(K))
+        assert Fraction(y[0, r]) == exact
+
+
+def test_ternary_select_example():
+    """2048ai.net s5.1: weights {+1,-1,-1,+1} give x0 - x1 - x2 + x3."""
+    wts = [float(v) for v in dict(read_golden("ternary_example.txt"))["weights"]]
+    K = 40
+    w = np.full(K, 0.001, np.float32)
+    w[1::2] = -0.001
+    w[:4] = np.array(wts, np.float32) * 5.0
+    d = oracle.decompose(w[None, :], G=32, P=90)   # the 4 large entries only
+    assert d["mask"][0, :4].tolist() == [1, 1, 1, 1] and d["mask"][0, 4:].sum() == 0
+    xq = np.random.default_rng(5).integers(-127, 128, (3, K)).astype(np.int8)
+    T, _ = oracle.accumulate(d, xq)
+    x = xq.astype(np.int64)
+    assert np.all(T[:, 0] == x[:, 0] - x[:, 1] - x[:, 2] + x[:, 3])
+
+
+def test_neuron_example_through_quantized_path():
+    """Visual guide: W=[0.6,-0.4], b=0.1: x=[2,-1] -> 1.7, x'=[0.2,3] -> -0.98,
+    reproduced through the separated path within the quantizers' error bound."""
+    g = read_golden("neuron_example.txt")
+    W = np.array([[float(v) for v in dict(g)["W"]]], np.float32)
+    b = float(dict(g)["b"][0])
+    d = oracle.decompose(W, G=32)
+    for key, vals in g:
+        if key != "case":
+            continue
+        x = np.array([[float(vals[0]), float(vals[1])]], np.float32)
+        z = float(vals[2])
+        xq, sx, xout = oracle.quantize_act(x, np.zeros(0, np.int32))
+        y = oracle.linear(d, xq, sx, xout, np.zeros(0, np.int32))[0, 0] + b
+        # |W.x - What.xhat| <= sum|W| sx/2 + sum|xhat| s_w/2
+        bound = np.abs(W).sum() * float(sx[0]) / 2 + np.abs(xq[0] * float(sx[0])).sum() * float(d["s"][0, 0]) / 2
+        assert abs(y - z) <= bound + 1e-12, (y, z, bound)
+
+
+# ---- trunk by popcount and the two output routes ------------------------------
+
+@pytest.mark.parametrize("K,P", [(33, -1), (100, 60), (128, -1), (300, 80)])
+def test_popcount_identity(K, P):
+    """m.lqnn.cn s2.3 bit trunk: 2*sum_{bit=1} xq - sum xq equals the +-1 sum."""
+    rng = np.random.default_rng(K + P)
+    W = rng.laplace(0, 0.02, (5, K)).astype(np.float32)
+    W[0, :3] = 0.0
+    d = oracle.decompose(W, G=32, P=P)
+    xq = rng.integers(-127, 128, (3, K)).astype(np.int8)
+    T, R = oracle.accumulate(d, xq)
+    assert np.array_equal(T, oracle.trunk_popcount(d, xq))
+    # and against a numpy +-1 product
+    pm = (d["mask"] * (2 * d["sign"].astype(np.int64) - 1))
+    assert np.array_equal(T, xq.astype(np.int64) @ pm.T)
+    qg = d["q"].astype(np.int64).reshape(5, -1)
+    for g in range(R.shape[2]):
+        sl = slice(32 * g, min(K, 32 * g + 32))
+        assert np.array_equal(R[:, :, g], xq[:, sl].astype(np.int64) @ qg[:, sl].T)
+
+
+@pytest.mark.parametrize("P", [-1, 60])
+def test_factored_equals_naive(P):
+    L = wl.config1()
+    W = L.weights()[:48]
+    x = L.activations(M=3)
+    idx = L.planted_channels()
+    d = oracle.decompose(W, P=P)
+    xq, sx, xout = oracle.quantize_act(x, idx)
+    y = oracle.linear(d, xq, sx, xout, idx)
+    yn = oracle.linear_naive(d, xq, sx, xout, idx)
+    scale = oracle.abs_dot(W, x)
+    assert np.all(np.abs(y - yn) <= 1e-12 * scale)
+    # and the dequantized product approximates the original W.x
+    ref = x.astype(np.float64) @ W.astype(np.float64).T
+    assert np.all(np.abs(y - ref) <= 0.05 * scale)
+
+
+# ---- calibration and activations ----------------------------------------------
+
+def test_calibration_recovers_planted_channels():
+    for L in (wl.config1(), wl.config2_layer(0, 0), wl.config2_layer(0, 3)):
+        X = L.calibration()
+        idx = oracle.calibrate(X, L.n_out)
+        assert np.array_equal(idx, L.planted_channels())
+
+
+def test_calibration_ties_and_library_order():
+    X = np.array([[3.0, -5.0, 5.0, 1.0], [0.0, 2.0, -5.0, -1.0]], np.float32)
+    assert oracle.calibrate(X, 1).tolist() == [1]
+    assert oracle.calibrate(X, 2).tolist() == [1, 2]
+    assert oracle.calibrate(X, 3).tolist() == [0, 1, 2]
+    rng = np.random.default_rng(2)
+    X = np.round(rng.standard_normal((16, 257)) * 4).astype(np.float32)  # many ties
+    mag = np.abs(X).max(axis=0)
+    order = np.lexsort((np.arange(257), -mag))
+    for k in (1, 5, 40, 257):
+        assert oracle.calibrate(X, k).tolist() == sorted(order[:k].tolist())
+
+
+def test_activation_split():
+    x = np.array([[1.0, -254.0, 0.5, 100.0, -0.25]], np.float32)
+    xq, sx, xout = oracle.quantize_act(x, np.array([3], np.int32))
+    assert sx[0] == np.float32(254.0 / 127.0)      # absmax without channel 3
+    assert xq[0].tolist() == [1, -127, 0, 0, 0]     # 0.5/2 = 0.25 -> 0; -0.125 -> 0
+    assert xout[0].tolist() == [100.0]
+    xq, sx, xout = oracle.quantize_act(np.zeros((2, 7), np.float32), np.array([0], np.int32))
+    assert np.all(sx == 0) and np.all(xq == 0)
+
+
+def test_nonfinite_and_bad_arguments():
+    W = np.ones((2, 40), np.float32)
+    W[1, 3] = np.nan
+    assert oracle.decompose(W, G=32)["status"] == 2
+    with pytest.raises(oracle.OracleError):
+        oracle.decompose(np.ones((1, 8), np.float32), G=32, P=0)
+    with pytest.raises(oracle.OracleError):
+        oracle.quantize_act(np.ones((1, 8), np.float32), np.array([3, 2], np.int32))
+    with pytest.raises(oracle.OracleError):
+        oracle.decompose(np.ones((1, 8), np.float32), G=48)
+
+
+def test_generator_statistics():
+    """The synthetic inputs have the stated distributions (sanity, not a pin)."""
+    W = wl.config1().weights()
+    assert abs(np.abs(W).mean() - 0.02) < 0.0005          # Laplace mean |W| = b
+    x = wl.config2_layer(0, 0).activations(M=64)
+    planted = wl.config2_layer(0, 0).planted_channels()
+    rest = np.delete(x, planted, axis=1)
+    assert abs(rest.std() - 1.0) < 0.02
+    assert abs(np.abs(x[:, planted]).mean() / np.abs(rest).mean() - 30.0) < 3.0
+    L3 = wl.config3()[0]
+    w3 = L3.weights(rows=np.arange(4))
+    heavy = np.abs(w3) > 6 * 0.015
+    assert 0.0003 < heavy.mean() < 0.003
