@@ -1,0 +1,503 @@
+#!/usr/bin/env python3
+"""Benchmark: batch-1 decode of the Llama-2-7B-shaped separated-quantization stack.
+
+One step = one token through 32 layers x {qkv 4096->12288, o 4096->4096,
+gate_up 4096->22016, down 11008->4096}: for each of the 128 linears the
+activation split (sq_quantize_act) and the fused linear (sq_linear), all in
+one CUDA graph with programmatic dependent launch.  Weights are packed once
+(offline) and resident in HBM; the 7.5 GB they take per step exceed the
+126 MB L2 many times over, so no flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl sq|reference]
+
+Prints ONE JSON line (rank 0).  With N > 1 (torchrun) every rank runs its own
+replica of the stack (weak scaling, no collective on the data path); the step
+time is the max over ranks.  ``--impl reference`` times the CPU oracle on a
+bounded sample of the same workload (host cores, no GPU).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode sq_linear HBM GB/s (% of 8 TB/s) and µs/token for 7B-shaped stack, batch 1"
+UNIT = "GB/s"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ---- algorithmic traffic ----------------------------------------------------------
+
+def bytes_per_weight(shares) -> float:
+    """Sum of share * bytes over the parts of a weight (the pages' accounting:
+    0.125 * 0.7 + 1 * 0.3 = 0.3875 for a 30 % 8-bit residual)."""
+    return sum(s * b for s, b in shares)
+
+
+def linear_weight_bytes(L) -> int:
+    """Packed-weight bytes the fused linear must read: sign (and mask) bits,
+    INT8 codes, fp32 group scales and the fp32 row scale."""
+    return L.packed_bytes
+
+
+def linear_act_bytes(L, M=1) -> int:
+    """Per call of the linear beyond the weights: xq, sx, x_out, idx in; y out."""
+    return M * (L.K + 4 + 4 * L.n_out + 4 * L.N) + 4 * L.n_out
+
+
+def quantize_bytes(L, M=1) -> int:
+    """Per call of the activation split: x and idx in; xq, sx, x_out out."""
+    return M * (4 * L.K + L.K + 4 + 4 * L.n_out) + 4 * L.n_out
+
+
+def step_bytes(layers, M=1) -> int:
+    return sum(linear_weight_bytes(L) + linear_act_bytes(L, M) + quantize_bytes(L, M) for L in layers)
+
+
+# ---- helpers ----------------------------------------------------------------------
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(prefix="sq_clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        return False
+
+    def summary(self):
+        rows = []
+        try:
+            with open(self.path) as f:
+                for line in f:
+                    parts = [p.strip() for p in line.split(",")]
+                    if len(parts) >= 9:
+                        rows.append(parts)
+        except OSError:
+            pass
+        finally:
+            try:
+                os.unlink(self.path)
+            except OSError:
+                pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+
+        def num(v):
+            try:
+                return float(v)
+            except ValueError:
+                return None
+
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        smax = [num(r[2]) for r in rows if num(r[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+# ---- CPU oracle baseline -----------------------------------------------------------
+
+def oracle_sample(rows: int = 256, layers_idx=(0,)):
+    """A bounded sample of the stack for the CPU oracle: the first `rows` rows of
+    each linear of the given layers (inputs generated on the host)."""
+    import numpy as np
+    from synth import workloads as wl
+    import oracle
+    sample = []
+    for l in layers_idx:
+        for mid in range(4):
+            L = wl.config2_layer(l, mid)
+            n = min(rows, L.N)
+            W = L.weights(rows=np.arange(n))
+            d = oracle.decompose(W)
+            sample.append((L, n, d, L.activations(), L.planted_channels()))
+    return sample
+
+
+def time_oracle(sample, min_seconds: float | None = None, passes: int | None = None):
+    """Times oracle.quantize_act + oracle.linear over the sample (one thread):
+    exactly `passes` passes, or as many as fill `min_seconds`."""
+    import oracle
+    done, t0 = 0, time.perf_counter()
+    while True:
+        for L, n, d, x, idx in sample:
+            xq, sx, xo = oracle.quantize_act(x, idx)
+            oracle.linear(d, xq, sx, xo, idx)
+        done += 1
+        el = time.perf_counter() - t0
+        if passes is not None and done >= passes:
+            break
+        if passes is None and el >= (min_seconds or 0.0):
+            break
+    per_pass = el / done
+    nbytes = 0
+    for L, n, d, x, idx in sample:
+        Ls = L.with_(N=n)
+        nbytes += linear_weight_bytes(Ls) + linear_act_bytes(Ls) + quantize_bytes(Ls)
+    return nbytes / per_pass / 1e9, per_pass, done, nbytes
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return 0
+    sample = oracle_sample(rows=args.oracle_rows)
+    time_oracle(sample, passes=args.warmup)
+    gbs, per_pass, passes, nbytes = time_oracle(sample, passes=args.steps)
+    desc = (f"first {args.oracle_rows} rows of each of the 4 linears of layer 0 "
+            f"({nbytes / 1e6:.1f} MB of algorithmic traffic per pass); quantize_act + linear, "
+            f"batch 1")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(per_pass * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int8+f64", "data": "synthetic",
+        "config": config_dict(args),
+        "cpu_baseline": {"value": round(gbs, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": round(gbs, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_dict(args):
+    return {"workload": "llama-2-7b-shaped decode linear stack, batch 1: "
+                        f"{args.layers} layers x {{qkv 4096->12288, o 4096->4096, "
+                        "gate_up 4096->22016, down 11008->4096}, W Laplace(0,0.02), "
+                        "x N(0,1) with 0.5% channels x30",
+            "layers": args.layers, "tokens": 1, "group_size": 128,
+            "l2": "inputs larger than L2 (packed weights of the stack, ~7.5 GB per step)",
+            "parallelism": "replicas" if args.gpus > 1 else "single"}
+
+
+# ---- GPU arm -----------------------------------------------------------------------
+
+class Stack:
+    def __init__(self, layers, device, pdl=True):
+        import torch
+        import decode_matvec_sq_b200 as sq
+        import synth
+        import synth.device as sdev
+        self.layers = layers
+        self.pdl = pdl
+        maxw = max(L.N * L.K for L in layers)
+        scratch = torch.empty(maxw, dtype=torch.float32, device=device)
+        cal = torch.empty(64 * max(L.K for L in layers), dtype=torch.float32, device=device)
+        st = torch.zeros(1, dtype=torch.int32, device=device)
+        self.status = st
+        self.pws, self.idx = [], []
+        xs_total = sum(L.K for L in layers)
+        ys_total = sum(L.N for L in layers)
+        # one contiguous x and y buffer each (e2e copies them in one transfer)
+        self.x_all = torch.empty(xs_total, dtype=torch.float32, device=device)
+        self.y_all = torch.empty(ys_total, dtype=torch.float32, device=device)
+        self.xs, self.ys, self.bufs = [], [], []
+        xo_, yo_ = 0, 0
+        for L in layers:
+            W = scratch[: L.N * L.K].view(L.N, L.K)
+            sdev.fill_weights(L, W)
+            self.pws.append(sq.decompose_pack(W, status=st))
+            X = cal[: 64 * L.K].view(64, L.K)
+            sdev.fill_activations(L, X, synth.STREAM_XCAL)
+            self.idx.append(sq.calibrate_outliers(X, L.n_out, status=st))
+            x = self.x_all[xo_: xo_ + L.K].view(1, L.K)
+            sdev.fill_activations(L, x)
+            self.xs.append(x)
+            self.ys.append(self.y_all[yo_: yo_ + L.N].view(1, L.N))
+            # keep every sub-buffer 16-byte aligned
+            assert (L.K * 4) % 16 == 0 and (L.N * 4) % 16 == 0
+            xo_ += L.K
+            yo_ += L.N
+            self.bufs.append(sq.quantize_act(x, self.idx[-1], status=st))
+        torch.cuda.synchronize()
+        del scratch, cal
+        if st.item() != 0:
+            raise RuntimeError(f"setup status {sq.STATUS.get(st.item())}")
+        self.ws = sq.new_workspace(max(self.pws, key=lambda p: p.N * 1000 + p.K), 1)
+        need = max(sq.workspace_bytes(p, 1) for p in self.pws)
+        if self.ws.numel() < need:
+            self.ws = torch.zeros(need, dtype=torch.uint8, device=device)
+
+    def step(self, pdl=None):
+        import decode_matvec_sq_b200 as sq
+        pdl = self.pdl if pdl is None else pdl
+        for pw, x, idx, (xq, sx, xo), y in zip(self.pws, self.xs, self.idx, self.bufs, self.ys):
+            sq.quantize_act(x, idx, xq=xq, sx=sx, x_out=xo, status=self.status, pdl=pdl)
+            sq.linear(pw, xq, sx, xo, idx, y=y, workspace=self.ws, status=self.status, pdl=pdl)
+
+    def capture(self):
+        import torch
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            self.step()  # warm every launch path once outside capture
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            self.step()
+        torch.cuda.synchronize()
+        return g
+
+    def time_linear_launches(self, reps: int):
+        """Average device duration of each fused-linear launch (events on the
+        launching stream), launched one by one without PDL."""
+        import torch
+        import decode_matvec_sq_b200 as sq
+        per_shape = {}
+        evs = []
+        stream = torch.cuda.current_stream()
+        for _ in range(reps):
+            for pw, idx, (xq, sx, xo), y, L in zip(self.pws, self.idx, self.bufs, self.ys, self.layers):
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                sq.linear(pw, xq, sx, xo, idx, y=y, workspace=self.ws, status=self.status)
+                b.record(stream)
+                evs.append((L, a, b))
+        torch.cuda.synchronize()
+        tot_ms, tot_bytes = 0.0, 0
+        for L, a, b in evs:
+            ms = a.elapsed_time(b)
+            key = L.name.split(".")[-1]
+            d = per_shape.setdefault(key, [0.0, 0, 0])
+            d[0] += ms
+            d[1] += 1
+            d[2] += linear_weight_bytes(L) + linear_act_bytes(L)
+            tot_ms += ms
+            tot_bytes += linear_weight_bytes(L) + linear_act_bytes(L)
+        shapes = {k: {"us": round(v[0] / v[1] * 1e3, 2),
+                      "gbs": round(v[2] / (v[0] * 1e-3) / 1e9, 1)} for k, v in per_shape.items()}
+        return tot_bytes / len(evs), tot_ms / len(evs), shapes
+
+
+def run_gpu(args, world, rank, local):
+    import torch
+    import torch.distributed as dist
+    import decode_matvec_sq_b200 as sq
+    from decode_matvec_sq_b200 import build
+    from synth import workloads as wl
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py: no CUDA device visible (the sq path has no CPU fallback)")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                device_id=device)
+    if rank == 0 or world == 1:
+        build.build_all()
+    if world > 1:
+        dist.barrier()
+    sq.device_check()
+
+    layers = wl.config2(args.layers)
+    stack = Stack(layers, device, pdl=not args.no_pdl)
+    graph = stack.capture()
+    nbytes = step_bytes(layers)
+    launches_per_step = 2 * len(layers)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+
+    # ---- headline: device-timed steps, inputs resident in HBM --------------------
+    with ClockSampler(local) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            graph.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ms_total = max_over_ranks(e0.elapsed_time(e1))
+    clocks = clk.summary()
+    ms_step = ms_total / args.steps
+    value = world * nbytes / (ms_step * 1e-3) / 1e9
+    if stack.status.item() != 0:
+        raise RuntimeError(f"device status {sq.STATUS.get(stack.status.item())}")
+
+    # ---- roofline of the dominant kernel: per-launch durations ------------------
+    bytes_launch, ms_launch, shapes = stack.time_linear_launches(max(1, args.steps))
+    peak, peak_kind = load_peaks()
+    achieved = bytes_launch / (ms_launch * 1e-3) / 1e9
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "linear_traffic.json")
+    if os.path.exists(tpath):
+        try:
+            with open(tpath) as f:
+                tr = json.load(f)
+            if tr.get("kernel_hash") == kernel_hash():
+                traffic = tr.get("dram_bytes_per_launch_stack_avg")
+        except Exception:
+            traffic = None
+
+    # ---- end to end through host buffers ---------------------------------------
+    e2e = None
+    if not args.no_e2e:
+        x_host = torch.empty_like(stack.x_all, device="cpu").pin_memory()
+        x_host.copy_(stack.x_all.cpu())
+        y_host = torch.empty_like(stack.y_all, device="cpu").pin_memory()
+        for _ in range(2):
+            stack.x_all.copy_(x_host, non_blocking=True)
+            graph.replay()
+            y_host.copy_(stack.y_all, non_blocking=True)
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            stack.x_all.copy_(x_host, non_blocking=True)
+            graph.replay()
+            y_host.copy_(stack.y_all, non_blocking=True)
+        b.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ms_e2e = max_over_ranks(a.elapsed_time(b)) / args.steps
+        e2e = {"value": round(world * nbytes / (ms_e2e * 1e-3) / 1e9, 1), "unit": UNIT,
+               "us_per_token": round(ms_e2e * 1e3, 2),
+               "h2d_bytes_per_step": int(stack.x_all.numel() * 4),
+               "d2h_bytes_per_step": int(stack.y_all.numel() * 4)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        sample = oracle_sample(rows=args.oracle_rows)
+        gbs, per_pass, passes, sbytes = time_oracle(sample, min_seconds=args.oracle_seconds)
+        cpu = {"value": round(gbs, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
+               "sample": f"first {args.oracle_rows} rows of each linear of layer 0 "
+                         f"({sbytes / 1e6:.1f} MB per pass, {passes} passes, "
+                         f"{per_pass * 1e3:.1f} ms per pass), quantize_act + linear"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+            "us_per_token": round(ms_step * 1e3, 2),
+            "pct_of_8tbs": round(100.0 * value / world / NOMINAL_HBM_GBS, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "int8", "data": "synthetic", "config": config_dict(argparse.Namespace(
+                layers=args.layers, gpus=world)),
+            "bytes_per_step": nbytes, "gpu_launches": launches_per_step * args.steps,
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                         "unit": "GB/s", "frac": round(achieved / peak, 4),
+                         "peak_kind": peak_kind, "traffic": traffic,
+                         "kernel": "k_linear (sq_linear decode)",
+                         "bytes_per_launch": int(bytes_launch),
+                         "us_per_launch": round(ms_launch * 1e3, 3), "per_shape": shapes},
+            "clocks": clocks,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    del graph
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def kernel_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("sq_linear.cu", "sq_common.cuh", "sq_internal.h"):
+        with open(os.path.join(ROOT, "decode_matvec_sq_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["sq", "reference"], default="sq")
+    ap.add_argument("--layers", type=int, default=32)
+    ap.add_argument("--no-pdl", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--oracle-rows", type=int, default=256)
+    ap.add_argument("--oracle-seconds", type=float, default=10.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        return run_reference(args, world, rank)
+    return run_gpu(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

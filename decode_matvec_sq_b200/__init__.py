@@ -1,0 +1,265 @@
+"""Python binding of libsq, the separated-quantization decode linear layer.
+
+Argument marshalling only: every step of the path runs in the CUDA kernels of
+``libsq.so`` (include/sq.h).  PyTorch provides device memory and the stream.
+There is no CPU fallback: importing works without a GPU (so the library can
+be inspected), but every call needs the built library and an sm_100 device,
+and fails loudly otherwise.
+
+Method (m.lqnn.cn/news/241359, sections 2.1-2.3): W ~ alpha_r*sign(W) + W_res
+with an INT8 group residual, activations split into cached fp32 outlier
+channels and per-token INT8 codes, and one fused kernel summing the trunk
+(bit operations), the residual (integer products) and the outliers.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG_DIR, "libsq.so")
+HEADER = os.path.join(os.path.dirname(PKG_DIR), "include", "sq.h")
+
+SQ_LAUNCH_PDL = 1
+
+STATUS = {
+    0: "SQ_OK", 1: "SQ_ERR_INVALID_ARG", 2: "SQ_ERR_SHAPE", 3: "SQ_ERR_ALIGN",
+    4: "SQ_ERR_UNSUPPORTED_DEVICE", 5: "SQ_ERR_CUDA", 6: "SQ_ERR_NONFINITE",
+    7: "SQ_ERR_TIMEOUT", 8: "SQ_ERR_WORKSPACE",
+}
+STATUS_CODE = {v: k for k, v in STATUS.items()}
+
+
+class SQError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        self.name = STATUS.get(code, f"status {code}")
+        super().__init__(f"{where}: {self.name}")
+
+
+class SqPackedWeight(ctypes.Structure):
+    _fields_ = [
+        ("N", ctypes.c_int32), ("K", ctypes.c_int32), ("group_size", ctypes.c_int32),
+        ("sign_stride", ctypes.c_int32), ("res_stride", ctypes.c_int32),
+        ("scale_stride", ctypes.c_int32),
+        ("sign_bits", ctypes.c_void_p), ("mask_bits", ctypes.c_void_p),
+        ("alpha", ctypes.c_void_p), ("res_q", ctypes.c_void_p), ("res_scale", ctypes.c_void_p),
+    ]
+
+
+_lib = None
+
+
+def lib():
+    """The loaded libsq.so; raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m decode_matvec_sq_b200.build` (nvcc, sm_100a)")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i32, u32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_uint32, ctypes.c_size_t
+    pw = ctypes.POINTER(SqPackedWeight)
+    sig = {
+        "sq_status_string": ([ctypes.c_int], ctypes.c_char_p),
+        "sq_device_check": ([], ctypes.c_int),
+        "sq_packed_bytes": ([i32, i32, i32, i32], sz),
+        "sq_packed_view": ([vp, i32, i32, i32, i32, pw], ctypes.c_int),
+        "sq_decompose_pack": ([vp, i32, i32, i32, pw, vp, vp], ctypes.c_int),
+        "sq_calibrate_outliers": ([vp, i32, i32, i32, vp, vp, vp], ctypes.c_int),
+        "sq_quantize_act": ([vp, i32, i32, vp, i32, vp, vp, vp, vp, u32, vp], ctypes.c_int),
+        "sq_linear_workspace_bytes": ([pw, i32], sz),
+        "sq_linear": ([pw, vp, vp, vp, vp, i32, i32, vp, vp, sz, vp, u32, vp], ctypes.c_int),
+        "sq_linear_accumulators": ([pw, vp, vp, vp, vp, i32, i32, vp, vp, vp, vp, sz, vp, vp],
+                                   ctypes.c_int),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(L, name)
+        fn.argtypes = args
+        fn.restype = res
+    _lib = L
+    return L
+
+
+def _ck(rc: int, where: str) -> None:
+    if rc != 0:
+        raise SQError(rc, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def ceil_div(a: int, b: int) -> int:
+    return -(-a // b)
+
+
+def round_up(a: int, b: int) -> int:
+    return ceil_div(a, b) * b
+
+
+def device_check() -> None:
+    _ck(lib().sq_device_check(), "sq_device_check")
+
+
+# ---- packed weights ------------------------------------------------------------
+
+@dataclass
+class PackedWeight:
+    """A packed weight in one device allocation (``buf``) with its C view."""
+    N: int
+    K: int
+    group_size: int
+    with_mask: bool
+    buf: object                 # torch.uint8 device tensor
+    view: SqPackedWeight
+
+    @property
+    def nbytes(self) -> int:
+        return int(self.buf.numel())
+
+    def _arr(self, field: str, dtype, shape):
+        import torch
+        base = self.buf.data_ptr()
+        off = getattr(self.view, field) - base
+        count = 1
+        for s in shape:
+            count *= s
+        itemsize = torch.empty(0, dtype=dtype).element_size()
+        return self.buf[off:off + count * itemsize].view(dtype).view(*shape)
+
+    def sign_bits(self):
+        import torch
+        return self._arr("sign_bits", torch.int32, (self.N, self.view.sign_stride))
+
+    def mask_bits(self):
+        import torch
+        if not self.with_mask:
+            return None
+        return self._arr("mask_bits", torch.int32, (self.N, self.view.sign_stride))
+
+    def alpha(self):
+        import torch
+        return self._arr("alpha", torch.float32, (self.N,))
+
+    def res_q(self):
+        import torch
+        return self._arr("res_q", torch.int8, (self.N, self.view.res_stride))
+
+    def res_scale(self):
+        import torch
+        return self._arr("res_scale", torch.float32, (self.N, self.view.scale_stride))
+
+
+def packed_bytes(N: int, K: int, group_size: int = 128, with_mask: bool = False) -> int:
+    return int(lib().sq_packed_bytes(N, K, group_size, int(with_mask)))
+
+
+def alloc_packed(N: int, K: int, group_size: int = 128, with_mask: bool = False,
+                 device=None) -> PackedWeight:
+    import torch
+    nbytes = packed_bytes(N, K, group_size, with_mask)
+    if nbytes == 0:
+        raise SQError(STATUS_CODE["SQ_ERR_SHAPE"], "sq_packed_bytes")
+    buf = torch.empty(nbytes, dtype=torch.uint8, device=device or "cuda")
+    v = SqPackedWeight()
+    _ck(lib().sq_packed_view(_ptr(buf), N, K, group_size, int(with_mask), ctypes.byref(v)),
+        "sq_packed_view")
+    return PackedWeight(N, K, group_size, with_mask, buf, v)
+
+
+def decompose_pack(W, trunk_percent: int = -1, group_size: int = 128, out: PackedWeight = None,
+                   status=None, stream=None) -> PackedWeight:
+    """Offline split of W[N][K] (float32, device) into the packed form."""
+    N, K = W.shape
+    if out is None:
+        out = alloc_packed(N, K, group_size, trunk_percent > 0, device=W.device)
+    _ck(lib().sq_decompose_pack(_ptr(W), N, K, trunk_percent, ctypes.byref(out.view),
+                                _ptr(status), _stream(stream)), "sq_decompose_pack")
+    return out
+
+
+def calibrate_outliers(X, k: int, out=None, status=None, stream=None):
+    """Top-k channels of X[T][K] by max |x| (ties: lower channel), ascending int32."""
+    import torch
+    T, K = X.shape
+    idx = out if out is not None else torch.empty(k, dtype=torch.int32, device=X.device)
+    _ck(lib().sq_calibrate_outliers(_ptr(X), T, K, k, _ptr(idx), _ptr(status), _stream(stream)),
+        "sq_calibrate_outliers")
+    return idx
+
+
+def quantize_act(x, idx, xq=None, sx=None, x_out=None, status=None, pdl: bool = False,
+                 stream=None):
+    """x[M][K] float32 -> (xq [M][roundup(K,16)] int8, sx [M], x_out [M][n_out])."""
+    import torch
+    M, K = x.shape
+    n = 0 if idx is None else int(idx.numel())
+    dev = x.device
+    if xq is None:
+        xq = torch.empty(M, round_up(K, 16), dtype=torch.int8, device=dev)
+    if sx is None:
+        sx = torch.empty(M, dtype=torch.float32, device=dev)
+    if x_out is None:
+        x_out = torch.empty(M, max(n, 1), dtype=torch.float32, device=dev)
+    _ck(lib().sq_quantize_act(_ptr(x), M, K, _ptr(idx) if n else None, n, _ptr(xq), _ptr(sx),
+                              _ptr(x_out) if n else None, _ptr(status),
+                              SQ_LAUNCH_PDL if pdl else 0, _stream(stream)), "sq_quantize_act")
+    return xq, sx, x_out
+
+
+def workspace_bytes(pw: PackedWeight, M: int = 1) -> int:
+    return int(lib().sq_linear_workspace_bytes(ctypes.byref(pw.view), M))
+
+
+def new_workspace(pw: PackedWeight, M: int = 1, device=None):
+    """A zero-filled workspace for sq_linear (zero once; calls keep it zeroed)."""
+    import torch
+    return torch.zeros(max(workspace_bytes(pw, M), 16), dtype=torch.uint8,
+                       device=device or pw.buf.device)
+
+
+def linear(pw: PackedWeight, xq, sx, x_out, idx, y=None, workspace=None, status=None,
+           pdl: bool = False, stream=None):
+    """y[M][N] = fused trunk + residual + outlier product (float32)."""
+    import torch
+    M = xq.shape[0]
+    n = 0 if idx is None else int(idx.numel())
+    if y is None:
+        y = torch.empty(M, pw.N, dtype=torch.float32, device=xq.device)
+    if workspace is None:
+        workspace = new_workspace(pw, M)
+    _ck(lib().sq_linear(ctypes.byref(pw.view), _ptr(xq), _ptr(sx), _ptr(x_out) if n else None,
+                        _ptr(idx) if n else None, n, M, _ptr(y), _ptr(workspace),
+                        workspace.numel(), _ptr(status), SQ_LAUNCH_PDL if pdl else 0,
+                        _stream(stream)), "sq_linear")
+    return y
+
+
+def linear_accumulators(pw: PackedWeight, xq, sx, x_out, idx, workspace=None, status=None,
+                        stream=None):
+    """(y, T [M][N] int32, R [M][N][ceil(K/G)] int32) from the decode kernel."""
+    import torch
+    M = xq.shape[0]
+    n = 0 if idx is None else int(idx.numel())
+    dev = xq.device
+    ng = ceil_div(pw.K, pw.group_size)
+    y = torch.empty(M, pw.N, dtype=torch.float32, device=dev)
+    T = torch.empty(M, pw.N, dtype=torch.int32, device=dev)
+    R = torch.empty(M, pw.N, ng, dtype=torch.int32, device=dev)
+    if workspace is None:
+        workspace = new_workspace(pw, M)
+    _ck(lib().sq_linear_accumulators(ctypes.byref(pw.view), _ptr(xq), _ptr(sx),
+                                     _ptr(x_out) if n else None, _ptr(idx) if n else None, n, M,
+                                     _ptr(y), _ptr(T), _ptr(R), _ptr(workspace),
+                                     workspace.numel(), _ptr(status), _stream(stream)),
+        "sq_linear_accumulators")
+    return y, T, R

@@ -1,0 +1,205 @@
+// sq_act.cu -- outlier calibration and the per-token activation split.
+//
+// Page: "1-bit量化不是玄学，以往掉点是机制问题" (m.lqnn.cn/news/241359),
+// section 2.2: outlier channels are found once, their indices cached and
+// looked up at run time; they stay at high precision while the remaining
+// channels are quantized to INT8.  Per-token runtime scale: visual guide to
+// LLM quantization, "动态量化" section.  Quantizer: symmetric absmax with
+// s = absmax/127 and q = round(x/s) in [-127, 127] (2048ai.net section 三.1).
+//
+// Built with -fmad=false.
+#include <stdint.h>
+
+#include "sq_common.cuh"
+#include "sq_internal.h"
+
+namespace sq {
+namespace {
+
+constexpr int kActThreads = 512;
+constexpr int kCalThreads = 1024;
+
+// round_half_away(|v| / s) decided exactly.  t = |v| * (1/s) is within far
+// less than 0.5 of the true quotient Q, so with k = floor(t) the exact test
+// Q >= k + 1/2  <=>  2|v| >= (2k+1)*s  (both sides exact in binary64: 2k+1
+// has at most 9 bits, s 24) yields the correctly rounded code whether Q lies
+// in [k, k+1) or just outside it.  Identical to rounding the exactly
+// rounded binary64 quotient v/s, which for float v and s never lands on the
+// wrong side of a midpoint.
+__device__ __forceinline__ int quantize_exact(float v, float s, double rinv) {
+  if (s == 0.0f) return 0;
+  const double av = fabs((double)v);
+  const double k = floor(av * rinv);
+  double q = (av + av >= (k + k + 1.0) * (double)s) ? k + 1.0 : k;
+  q = q < 127.0 ? q : 127.0;
+  const int qi = (int)q;
+  return v < 0.0f ? -qi : qi;
+}
+
+__global__ void __launch_bounds__(kActThreads) k_quantize_act(
+    const float* __restrict__ x, int M, int K, int K16, const int32_t* __restrict__ idx, int n_out,
+    int8_t* __restrict__ xq, float* __restrict__ sx, float* __restrict__ x_out,
+    int32_t* __restrict__ status, int pdl) {
+  extern __shared__ uint32_t is_out[];  // ceil(K/32) words
+  __shared__ float warp_max[kActThreads / 32];
+  if (pdl) {
+    pdl_launch_dependents();
+    pdl_wait();
+  }
+  const int t = blockIdx.x;
+  const int nw = (K + 31) / 32;
+  for (int i = threadIdx.x; i < nw; i += blockDim.x) is_out[i] = 0u;
+  __syncthreads();
+  const float* xt = x + (int64_t)t * K;
+  bool bad_idx = false;
+  for (int i = threadIdx.x; i < n_out; i += blockDim.x) {
+    const int j = idx[i];
+    const bool ok = j >= 0 && j < K && (i == 0 || idx[i - 1] < j);
+    bad_idx |= !ok;
+    if (j >= 0 && j < K) atomicOr(&is_out[j >> 5], 1u << (j & 31));
+    x_out[(int64_t)t * n_out + i] = (j >= 0 && j < K) ? xt[j] : 0.0f;
+  }
+  __syncthreads();
+
+  float a = 0.0f;
+  bool nonfinite = false;
+  for (int j = threadIdx.x; j < K; j += blockDim.x) {
+    const float v = xt[j];
+    nonfinite |= !isfinite(v);
+    if (!((is_out[j >> 5] >> (j & 31)) & 1u)) a = fmaxf(a, fabsf(v));
+  }
+  for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+  if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = a;
+  __syncthreads();
+  a = 0.0f;
+  for (int w = 0; w < kActThreads / 32; ++w) a = fmaxf(a, warp_max[w]);
+
+  const float s = (float)((double)a / 127.0);
+  const double rinv = s != 0.0f ? 1.0 / (double)s : 0.0;
+  if (threadIdx.x == 0) sx[t] = s;
+
+  // codes, four channels per 32-bit store; outlier slots and pads are 0
+  int8_t* qt = xq + (int64_t)t * K16;
+  for (int j0 = threadIdx.x * 4; j0 < K16; j0 += blockDim.x * 4) {
+    uint32_t word = 0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int j = j0 + k;
+      int q = 0;
+      if (j < K && !((is_out[j >> 5] >> (j & 31)) & 1u)) q = quantize_exact(xt[j], s, rinv);
+      word |= ((uint32_t)(uint8_t)(int8_t)q) << (8 * k);
+    }
+    *reinterpret_cast<uint32_t*>(qt + j0) = word;
+  }
+  if (nonfinite) set_status(status, SQ_ERR_NONFINITE);
+  if (bad_idx) set_status(status, SQ_ERR_INVALID_ARG);
+}
+
+// ---- calibration: per-channel max |X| over T tokens, top-k ------------------
+struct Cand {
+  float mag;
+  int j;
+};
+
+__device__ __forceinline__ bool better(const Cand& a, const Cand& b) {
+  return a.mag > b.mag || (a.mag == b.mag && a.j < b.j);
+}
+
+__global__ void __launch_bounds__(kCalThreads) k_calibrate(const float* __restrict__ X, int T,
+                                                           int K, int k,
+                                                           int32_t* __restrict__ idx_out,
+                                                           int32_t* __restrict__ status) {
+  extern __shared__ float mag[];  // [K] magnitudes, then [K] taken flags
+  uint8_t* taken = reinterpret_cast<uint8_t*>(mag + K);
+  __shared__ Cand warp_best[kCalThreads / 32];
+  __shared__ int counts[kCalThreads];
+  bool nonfinite = false;
+  for (int j = threadIdx.x; j < K; j += blockDim.x) {
+    float m = 0.0f;
+    for (int t = 0; t < T; ++t) {
+      const float v = X[(int64_t)t * K + j];
+      if (isfinite(v))
+        m = fmaxf(m, fabsf(v));
+      else
+        nonfinite = true;
+    }
+    mag[j] = m;
+    taken[j] = 0;
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int round = 0; round < k; ++round) {
+    Cand best{-1.0f, 0x7fffffff};
+    for (int j = threadIdx.x; j < K; j += blockDim.x) {
+      Cand c{taken[j] ? -1.0f : mag[j], j};
+      if (better(c, best)) best = c;
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+      Cand other{__shfl_xor_sync(0xffffffffu, best.mag, o), __shfl_xor_sync(0xffffffffu, best.j, o)};
+      if (better(other, best)) best = other;
+    }
+    if (lane == 0) warp_best[warp] = best;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      Cand b = warp_best[0];
+      for (int w = 1; w < kCalThreads / 32; ++w)
+        if (better(warp_best[w], b)) b = warp_best[w];
+      taken[b.j] = 1;
+    }
+    __syncthreads();
+  }
+  // ascending compaction: thread i owns channels [i*K/n, (i+1)*K/n)
+  const int n = blockDim.x;
+  const int j0 = (int)((int64_t)threadIdx.x * K / n), j1 = (int)((int64_t)(threadIdx.x + 1) * K / n);
+  int c = 0;
+  for (int j = j0; j < j1; ++j) c += taken[j];
+  counts[threadIdx.x] = c;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int run = 0;
+    for (int i = 0; i < n; ++i) {
+      const int v = counts[i];
+      counts[i] = run;
+      run += v;
+    }
+  }
+  __syncthreads();
+  int pos = counts[threadIdx.x];
+  for (int j = j0; j < j1; ++j)
+    if (taken[j]) idx_out[pos++] = j;
+  if (nonfinite) set_status(status, SQ_ERR_NONFINITE);
+}
+
+}  // namespace
+
+cudaError_t launch_quantize_act(const float* x, int M, int K, const int32_t* idx, int n_out,
+                                int8_t* xq, float* sx, float* x_out, int32_t* status, bool pdl,
+                                cudaStream_t stream) {
+  const int K16 = (int)round_up(K, 16);
+  const size_t smem = (size_t)ceil_div(K, 32) * sizeof(uint32_t);
+  cudaError_t e = ensure_smem_attr((const void*)k_quantize_act, (int)smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(M);
+  cfg.blockDim = dim3(kActThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, k_quantize_act, x, M, K, K16, idx, n_out, xq, sx, x_out, status,
+                            pdl ? 1 : 0);
+}
+
+cudaError_t launch_calibrate(const float* X, int T, int K, int k, int32_t* idx_out,
+                             int32_t* status, cudaStream_t stream) {
+  const size_t smem = (size_t)K * (sizeof(float) + 1);
+  cudaError_t e = ensure_smem_attr((const void*)k_calibrate, (int)smem);
+  if (e != cudaSuccess) return e;
+  k_calibrate<<<1, kCalThreads, smem, stream>>>(X, T, K, k, idx_out, status);
+  return cudaGetLastError();
+}
+
+}  // namespace sq

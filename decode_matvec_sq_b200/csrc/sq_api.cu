@@ -1,0 +1,287 @@
+// sq_api.cu -- the extern "C" entry points declared in include/sq.h:
+// host-side validation, device checks and launch orchestration.  No device
+// memory is allocated here.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "sq_internal.h"
+
+namespace sq {
+
+namespace {
+constexpr int kMaxDevices = 64;
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_mu;
+
+struct AttrEntry {
+  const void* fn;
+  int device;
+  int bytes;
+};
+AttrEntry g_attr[256];
+int g_attr_n = 0;
+}  // namespace
+
+bool current_device(DeviceInfo* out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (d.device != dev) {
+    DeviceInfo n;
+    n.device = dev;
+    if (cudaDeviceGetAttribute(&n.major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n.minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+            cudaSuccess)
+      return false;
+    d = n;
+  }
+  *out = d;
+  return true;
+}
+
+cudaError_t ensure_smem_attr(const void* func, int bytes) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(g_mu);
+  for (int i = 0; i < g_attr_n; ++i)
+    if (g_attr[i].fn == func && g_attr[i].device == dev) {
+      if (g_attr[i].bytes >= bytes) return cudaSuccess;
+      e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+      if (e == cudaSuccess) g_attr[i].bytes = bytes;
+      return e;
+    }
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && g_attr_n < 256) g_attr[g_attr_n++] = AttrEntry{func, dev, bytes};
+  return e;
+}
+
+}  // namespace sq
+
+using namespace sq;
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool valid_group(int g) { return g == 32 || g == 64 || g == 128; }
+
+// Shapes the library supports (int32 indexing of rows and channels).
+bool valid_shape(int64_t N, int64_t K) {
+  return N >= 1 && K >= 1 && N <= (1 << 28) && K <= (1 << 24) && N * round_up(K, 16) < (1ll << 40);
+}
+
+sq_status check_device(DeviceInfo* d) {
+  if (!current_device(d)) return SQ_ERR_CUDA;
+  if (d->major != 10 || d->minor != 0) return SQ_ERR_UNSUPPORTED_DEVICE;
+  return SQ_OK;
+}
+
+sq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? SQ_OK : SQ_ERR_CUDA; }
+
+int32_t sign_stride_of(int32_t K) { return (int32_t)round_up(ceil_div(K, 32), 4); }
+int32_t res_stride_of(int32_t K) { return (int32_t)round_up(K, 16); }
+int32_t scale_stride_of(int32_t K, int32_t G) { return (int32_t)round_up(ceil_div(K, G), 4); }
+
+sq_status check_weight(const sq_packed_weight* w) {
+  if (!w || !w->sign_bits || !w->alpha || !w->res_q || !w->res_scale) return SQ_ERR_INVALID_ARG;
+  if (!valid_group(w->group_size) || !valid_shape(w->N, w->K)) return SQ_ERR_SHAPE;
+  if (w->sign_stride != sign_stride_of(w->K) || w->res_stride != res_stride_of(w->K) ||
+      w->scale_stride != scale_stride_of(w->K, w->group_size))
+    return SQ_ERR_SHAPE;
+  if (!aligned16(w->sign_bits) || !aligned16(w->alpha) || !aligned16(w->res_q) ||
+      !aligned16(w->res_scale) || (w->mask_bits && !aligned16(w->mask_bits)))
+    return SQ_ERR_ALIGN;
+  return SQ_OK;
+}
+
+// Offsets of the five arrays inside one allocation, each 256-byte aligned.
+// alpha holds roundup(N, 8) floats so that whole 8-row blocks can be copied.
+struct Carve {
+  size_t sign, mask, alpha, res, scale, total;
+};
+
+Carve carve(int32_t N, int32_t K, int32_t G, int32_t with_mask) {
+  Carve c;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t at = off;
+    off = (size_t)round_up((int64_t)(off + bytes), 256);
+    return at;
+  };
+  c.sign = take((size_t)N * sign_stride_of(K) * 4);
+  c.mask = with_mask ? take((size_t)N * sign_stride_of(K) * 4) : 0;
+  c.alpha = take((size_t)round_up(N, 8) * 4);
+  c.res = take((size_t)N * res_stride_of(K));
+  c.scale = take((size_t)N * scale_stride_of(K, G) * 4);
+  c.total = off;
+  return c;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* sq_status_string(sq_status s) {
+  switch (s) {
+    case SQ_OK: return "ok";
+    case SQ_ERR_INVALID_ARG: return "invalid argument";
+    case SQ_ERR_SHAPE: return "unsupported shape";
+    case SQ_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case SQ_ERR_UNSUPPORTED_DEVICE: return "current device is not sm_100 (B200)";
+    case SQ_ERR_CUDA: return "CUDA runtime error";
+    case SQ_ERR_NONFINITE: return "non-finite input";
+    case SQ_ERR_TIMEOUT: return "bounded wait ran out";
+    case SQ_ERR_WORKSPACE: return "workspace missing or too small";
+  }
+  return "unknown status";
+}
+
+sq_status sq_device_check(void) {
+  DeviceInfo d;
+  return check_device(&d);
+}
+
+size_t sq_packed_bytes(int32_t N, int32_t K, int32_t group_size, int32_t with_mask) {
+  if (!valid_shape(N, K) || !valid_group(group_size)) return 0;
+  return carve(N, K, group_size, with_mask).total;
+}
+
+sq_status sq_packed_view(void* base, int32_t N, int32_t K, int32_t group_size, int32_t with_mask,
+                         sq_packed_weight* out) {
+  if (!base || !out) return SQ_ERR_INVALID_ARG;
+  if (!valid_shape(N, K) || !valid_group(group_size)) return SQ_ERR_SHAPE;
+  if ((reinterpret_cast<uintptr_t>(base) & 255u) != 0) return SQ_ERR_ALIGN;
+  const Carve c = carve(N, K, group_size, with_mask);
+  uint8_t* b = static_cast<uint8_t*>(base);
+  out->N = N;
+  out->K = K;
+  out->group_size = group_size;
+  out->sign_stride = sign_stride_of(K);
+  out->res_stride = res_stride_of(K);
+  out->scale_stride = scale_stride_of(K, group_size);
+  out->sign_bits = reinterpret_cast<uint32_t*>(b + c.sign);
+  out->mask_bits = with_mask ? reinterpret_cast<uint32_t*>(b + c.mask) : nullptr;
+  out->alpha = reinterpret_cast<float*>(b + c.alpha);
+  out->res_q = reinterpret_cast<int8_t*>(b + c.res);
+  out->res_scale = reinterpret_cast<float*>(b + c.scale);
+  return SQ_OK;
+}
+
+sq_status sq_decompose_pack(const float* W, int32_t N, int32_t K, int32_t trunk_percent,
+                            const sq_packed_weight* out, int32_t* dev_status, void* stream) {
+  if (!W || !out) return SQ_ERR_INVALID_ARG;
+  sq_status st = check_weight(out);
+  if (st != SQ_OK) return st;
+  if (out->N != N || out->K != K) return SQ_ERR_SHAPE;
+  if (trunk_percent == 0 || trunk_percent > 100) return SQ_ERR_INVALID_ARG;
+  if (trunk_percent > 0 && !out->mask_bits) return SQ_ERR_INVALID_ARG;
+  if (!aligned16(W) || (dev_status && (reinterpret_cast<uintptr_t>(dev_status) & 3u)))
+    return SQ_ERR_ALIGN;
+  DeviceInfo d;
+  if ((st = check_device(&d)) != SQ_OK) return st;
+  // full trunk with a mask array present: the mask is written all ones
+  sq_packed_weight pw = *out;
+  return from_cuda(launch_decompose_pack(W, N, K, trunk_percent, pw, dev_status,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+sq_status sq_calibrate_outliers(const float* X, int32_t T, int32_t K, int32_t k, int32_t* idx_out,
+                                int32_t* dev_status, void* stream) {
+  if (!X || !idx_out) return SQ_ERR_INVALID_ARG;
+  if (T < 1 || K < 1 || K > 40960 || k < 1 || k > K) return SQ_ERR_SHAPE;
+  if (!aligned16(X) || !aligned16(idx_out)) return SQ_ERR_ALIGN;
+  DeviceInfo d;
+  sq_status st = check_device(&d);
+  if (st != SQ_OK) return st;
+  return from_cuda(launch_calibrate(X, T, K, k, idx_out, dev_status, static_cast<cudaStream_t>(stream)));
+}
+
+sq_status sq_quantize_act(const float* x, int32_t M, int32_t K, const int32_t* idx, int32_t n_out,
+                          int8_t* xq, float* sx, float* x_out, int32_t* dev_status, uint32_t flags,
+                          void* stream) {
+  if (!x || !xq || !sx) return SQ_ERR_INVALID_ARG;
+  if (M < 1 || K < 1 || K > (1 << 24) || M > (1 << 24)) return SQ_ERR_SHAPE;
+  if (n_out < 0 || n_out > kMaxOutliers || n_out > K) return SQ_ERR_SHAPE;
+  if (n_out > 0 && (!idx || !x_out)) return SQ_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(xq) || !aligned16(sx) || (n_out > 0 && (!aligned16(idx) || !aligned16(x_out))))
+    return SQ_ERR_ALIGN;
+  if (flags & ~SQ_LAUNCH_PDL) return SQ_ERR_INVALID_ARG;
+  DeviceInfo d;
+  sq_status st = check_device(&d);
+  if (st != SQ_OK) return st;
+  return from_cuda(launch_quantize_act(x, M, K, idx, n_out, xq, sx, x_out, dev_status,
+                                       (flags & SQ_LAUNCH_PDL) != 0, static_cast<cudaStream_t>(stream)));
+}
+
+size_t sq_linear_workspace_bytes(const sq_packed_weight* w, int32_t M) {
+  if (!w || check_weight(w) != SQ_OK || M < 1) return 0;
+  DeviceInfo d;
+  if (!current_device(&d)) return 0;
+  return linear_workspace_bytes(*w, M, d.sm_count);
+}
+
+static sq_status linear_common(const sq_packed_weight* w, const int8_t* xq, const float* sx,
+                               const float* x_out, const int32_t* idx, int32_t n_out, int32_t M,
+                               float* y, int32_t* T_out, int32_t* R_out, void* workspace,
+                               size_t ws_bytes, int32_t* dev_status, uint32_t flags, void* stream) {
+  sq_status st = check_weight(w);
+  if (st != SQ_OK) return st;
+  if (!xq || !sx || !y) return SQ_ERR_INVALID_ARG;
+  if (M < 1 || M > (1 << 20)) return SQ_ERR_SHAPE;
+  if (n_out < 0 || n_out > kMaxOutliers || n_out > w->K) return SQ_ERR_SHAPE;
+  if (n_out > 0 && (!idx || !x_out)) return SQ_ERR_INVALID_ARG;
+  if (flags & ~SQ_LAUNCH_PDL) return SQ_ERR_INVALID_ARG;
+  if (!aligned16(xq) || !aligned16(sx) || !aligned16(y) ||
+      (n_out > 0 && (!aligned16(idx) || !aligned16(x_out))) || (workspace && !aligned16(workspace)))
+    return SQ_ERR_ALIGN;
+  DeviceInfo d;
+  if ((st = check_device(&d)) != SQ_OK) return st;
+  const size_t need = linear_workspace_bytes(*w, M, d.sm_count);
+  if (!workspace || ws_bytes < need) return SQ_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (T_out) {
+    cudaError_t e = cudaMemsetAsync(T_out, 0, (size_t)M * w->N * sizeof(int32_t), s);
+    if (e != cudaSuccess) return SQ_ERR_CUDA;
+  }
+  const int ng = (int)ceil_div(w->K, w->group_size);
+  for (int t0 = 0; t0 < M; t0 += kMaxTokensPerPass) {
+    const int m = std::min(kMaxTokensPerPass, M - t0);
+    LinearPlan plan;
+    if (!plan_linear(*w, m, n_out, d.sm_count, &plan)) return SQ_ERR_SHAPE;
+    if (plan.smem_bytes > d.smem_optin) return SQ_ERR_SHAPE;
+    cudaError_t e = launch_linear(
+        *w, plan, xq + (int64_t)t0 * w->res_stride, sx + t0, n_out ? x_out + (int64_t)t0 * n_out : nullptr,
+        idx, n_out, y + (int64_t)t0 * w->N, T_out ? T_out + (int64_t)t0 * w->N : nullptr,
+        R_out ? R_out + (int64_t)t0 * w->N * ng : nullptr, workspace, dev_status,
+        (flags & SQ_LAUNCH_PDL) != 0, s);
+    if (e != cudaSuccess) return SQ_ERR_CUDA;
+  }
+  return SQ_OK;
+}
+
+sq_status sq_linear(const sq_packed_weight* w, const int8_t* xq, const float* sx,
+                    const float* x_out, const int32_t* idx, int32_t n_out, int32_t M, float* y,
+                    void* workspace, size_t ws_bytes, int32_t* dev_status, uint32_t flags,
+                    void* stream) {
+  return linear_common(w, xq, sx, x_out, idx, n_out, M, y, nullptr, nullptr, workspace, ws_bytes,
+                       dev_status, flags, stream);
+}
+
+sq_status sq_linear_accumulators(const sq_packed_weight* w, const int8_t* xq, const float* sx,
+                                 const float* x_out, const int32_t* idx, int32_t n_out, int32_t M,
+                                 float* y, int32_t* T_out, int32_t* R_out, void* workspace,
+                                 size_t ws_bytes, int32_t* dev_status, void* stream) {
+  if (!T_out || !R_out) return SQ_ERR_INVALID_ARG;
+  if (!aligned16(T_out) || !aligned16(R_out)) return SQ_ERR_ALIGN;
+  return linear_common(w, xq, sx, x_out, idx, n_out, M, y, T_out, R_out, workspace, ws_bytes,
+                       dev_status, 0u, stream);
+}
+
+}  // extern "C"

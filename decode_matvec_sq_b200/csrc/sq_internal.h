@@ -1,0 +1,69 @@
+// sq_internal.h -- launchers shared between the C-ABI layer and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/sq.h"
+
+namespace sq {
+
+struct DeviceInfo {
+  int device = -1;
+  int major = 0, minor = 0;
+  int sm_count = 0;
+  int smem_optin = 0;  // max dynamic shared memory per block (opt-in)
+};
+
+// Properties of the current device (cached per device).  false on CUDA error.
+bool current_device(DeviceInfo* out);
+
+// Sets the kernel's max dynamic shared memory once per device.
+cudaError_t ensure_smem_attr(const void* func, int bytes);
+
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
+
+// ---- launchers ---------------------------------------------------------------
+cudaError_t launch_decompose_pack(const float* W, int N, int K, int P, const sq_packed_weight& pw,
+                                  int32_t* status, cudaStream_t stream);
+
+cudaError_t launch_calibrate(const float* X, int T, int K, int k, int32_t* idx_out,
+                             int32_t* status, cudaStream_t stream);
+
+cudaError_t launch_quantize_act(const float* x, int M, int K, const int32_t* idx, int n_out,
+                                int8_t* xq, float* sx, float* x_out, int32_t* status, bool pdl,
+                                cudaStream_t stream);
+
+struct LinearPlan {
+  int M = 1;           // tokens in this pass (1..kMaxTokensPerPass)
+  int Kc = 0;          // channels per chunk
+  int n_c = 0;         // chunks per row
+  int n_rb = 0;        // row blocks
+  int U = 0;           // work units = n_rb * n_c
+  int grid = 0;        // CTAs
+  int S = 0;           // pipeline stages
+  int stage_bytes = 0;
+  int off_sign = 0, off_mask = 0, off_scale = 0, off_alpha = 0;
+  int hdr_bytes = 0;   // shared memory before the stages
+  int smem_bytes = 0;
+  size_t ws_cnt_bytes = 0;
+  size_t ws_part_bytes = 0;
+};
+
+constexpr int kRowsPerBlock = 8;   // one consumer warp per row of a row block
+constexpr int kMaxTokensPerPass = 4;
+constexpr int kMaxOutliers = 4096;
+
+// Plans a decode launch for M tokens (M <= kMaxTokensPerPass) on the current device.
+bool plan_linear(const sq_packed_weight& w, int M, int n_out, int sm_count, LinearPlan* plan);
+
+size_t linear_workspace_bytes(const sq_packed_weight& w, int M, int sm_count);
+
+cudaError_t launch_linear(const sq_packed_weight& w, const LinearPlan& plan, const int8_t* xq,
+                          const float* sx, const float* x_out, const int32_t* idx, int n_out,
+                          float* y, int32_t* T_out, int32_t* R_out, void* workspace,
+                          int32_t* status, bool pdl, cudaStream_t stream);
+
+}  // namespace sq

@@ -1,0 +1,204 @@
+// sq_pack.cu -- offline decomposition of W into the packed separated form.
+//
+// Page: "1-bit量化不是玄学，以往掉点是机制问题" (m.lqnn.cn/news/241359):
+//   section 2.1  W ~ alpha*sign(W) + W_res,  W_res = W - alpha*sign(W),
+//                residual re-quantized to 8 bits; trunk limited to |W| > threshold;
+//   section 5.2  threshold from a percentile of |W|;
+//   section 5.3  the split is done once, offline, and reused by every inference;
+//   section 6.2  one scale and one threshold per output row.
+// Quantizer: symmetric absmax, [-127, 127], s = absmax/127, q = round(r/s)
+// (visual guide "对称量化以零为中心"; 2048ai.net section 三.1).
+//
+// Built with -fmad=false: every floating-point step below is a single IEEE
+// operation in a fixed order, so the results are identical to any other
+// implementation of the same sequence (binary64 sum of |W| in ascending
+// channel order, one binary64 division for alpha and for each quotient).
+#include <stdint.h>
+
+#include "sq_common.cuh"
+#include "sq_internal.h"
+
+namespace sq {
+namespace {
+
+constexpr int kPackRows = 128;  // rows per CTA, one thread per row
+constexpr int kTile = 32;       // columns per shared-memory tile
+
+// ---- per-row nearest-rank threshold (MSB-first radix select) ---------------
+// tau_r = the rank-th smallest |W[r][:]|, rank = ceil(P*K/100).  |W| as the
+// float's bit pattern with the sign bit cleared orders like the value.
+__global__ void __launch_bounds__(256) k_threshold(const float* __restrict__ W, int N, int K,
+                                                   int P, float* __restrict__ tau_out) {
+  __shared__ uint32_t hist[256];
+  __shared__ uint32_t s_prefix, s_remaining;
+  const int row = blockIdx.x;
+  if (row >= N) return;
+  const uint32_t* w = reinterpret_cast<const uint32_t*>(W + (int64_t)row * K);
+  if (threadIdx.x == 0) {
+    s_prefix = 0;
+    s_remaining = (uint32_t)(((int64_t)P * K + 99) / 100);
+  }
+  uint32_t hi_mask = 0;
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    const uint32_t prefix = s_prefix;
+    for (int j = threadIdx.x; j < K; j += blockDim.x) {
+      uint32_t key = __ldg(w + j) & 0x7FFFFFFFu;
+      if ((key & hi_mask) == prefix) atomicAdd(&hist[(key >> shift) & 0xFFu], 1u);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      uint32_t rem = s_remaining, cum = 0;
+      int b = 0;
+      for (; b < 255; ++b) {
+        if (cum + hist[b] >= rem) break;
+        cum += hist[b];
+      }
+      s_remaining = rem - cum;
+      s_prefix = prefix | ((uint32_t)b << shift);
+    }
+    hi_mask |= 0xFFu << shift;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) tau_out[row] = __uint_as_float(s_prefix);
+}
+
+__device__ __forceinline__ int quantize_q(double r, float s) {
+  if (s == 0.0f) return 0;
+  double t = r / (double)s;  // IEEE binary64 division
+  double q = round(t);       // half away from zero
+  q = q > 127.0 ? 127.0 : q;
+  q = q < -127.0 ? -127.0 : q;
+  return (int)q;
+}
+
+// Loads columns [c0, c0 + ncols) of rows [r0, r0 + kPackRows) into tile[row][col].
+__device__ __forceinline__ void load_tile(float* tile, int pitch, const float* __restrict__ W,
+                                          int N, int K, int r0, int c0, int ncols) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  for (int rr = warp; rr < kPackRows; rr += nwarps) {
+    const int row = r0 + rr;
+    for (int cc = lane; cc < ncols; cc += 32) {
+      const int col = c0 + cc;
+      tile[rr * pitch + cc] = (row < N && col < K) ? __ldg(W + (int64_t)row * K + col) : 0.0f;
+    }
+  }
+}
+
+// ---- sign / mask bitplanes, alpha, residual codes and group scales --------
+__global__ void __launch_bounds__(kPackRows) k_pack(const float* __restrict__ W, int N, int K,
+                                                    int P, int G, sq_packed_weight pw,
+                                                    int32_t* __restrict__ status) {
+  extern __shared__ float tile[];  // [kPackRows][G + 1]
+  const int r0 = blockIdx.x * kPackRows;
+  const int row = r0 + threadIdx.x;
+  const bool valid = row < N;
+  const int nwords = (K + 31) / 32;
+  const int ng = (K + G - 1) / G;
+  const float tau = (valid && P > 0) ? pw.alpha[row] : -1.0f;  // k_threshold wrote it here
+  bool nonfinite = false;
+
+  // pass 1: bits, trunk sum, count
+  double sum = 0.0;
+  int64_t cnt = 0;
+  const int pitch1 = kTile + 1;
+  for (int c0 = 0; c0 < K; c0 += kTile) {
+    load_tile(tile, pitch1, W, N, K, r0, c0, kTile);
+    __syncthreads();
+    if (valid) {
+      uint32_t sbits = 0, mbits = 0;
+      const int ncols = min(kTile, K - c0);
+      for (int j = 0; j < ncols; ++j) {
+        const float v = tile[threadIdx.x * pitch1 + j];
+        nonfinite |= !isfinite(v);
+        if (v >= 0.0f) sbits |= 1u << j;
+        const bool m = P < 0 ? true : (fabsf(v) > tau);
+        if (m) {
+          mbits |= 1u << j;
+          sum += fabs((double)v);
+          cnt += 1;
+        }
+      }
+      pw.sign_bits[(int64_t)row * pw.sign_stride + c0 / 32] = sbits;
+      if (pw.mask_bits) pw.mask_bits[(int64_t)row * pw.sign_stride + c0 / 32] = mbits;
+    }
+    __syncthreads();
+  }
+  float alpha = 0.0f;
+  if (valid) {
+    alpha = cnt ? (float)(sum / (double)cnt) : 0.0f;
+    for (int w = nwords; w < pw.sign_stride; ++w) {
+      pw.sign_bits[(int64_t)row * pw.sign_stride + w] = 0u;
+      if (pw.mask_bits) pw.mask_bits[(int64_t)row * pw.sign_stride + w] = 0u;
+    }
+  }
+  __syncthreads();  // every thread has read its tau before alpha overwrites it
+  if (valid) pw.alpha[row] = alpha;
+
+  // pass 2: residual per group, absmax scale, codes
+  const int pitch2 = G + 1;
+  for (int g = 0; g < ng; ++g) {
+    const int c0 = g * G;
+    load_tile(tile, pitch2, W, N, K, r0, c0, G);
+    __syncthreads();
+    if (valid) {
+      const int ncols = min(G, K - c0);
+      const float* t = tile + threadIdx.x * pitch2;
+      double a = 0.0;
+      for (int j = 0; j < ncols; ++j) {
+        const float v = t[j];
+        const bool m = P < 0 ? true : (fabsf(v) > tau);
+        const double tr = m ? (v >= 0.0f ? (double)alpha : -(double)alpha) : 0.0;
+        const double r = (double)v - tr;
+        a = fabs(r) > a ? fabs(r) : a;
+      }
+      const float s = (float)(a / 127.0);
+      pw.res_scale[(int64_t)row * pw.scale_stride + g] = s;
+      int8_t* qrow = pw.res_q + (int64_t)row * pw.res_stride + c0;
+      for (int j0 = 0; j0 < ncols; j0 += 4) {
+        uint32_t word = 0;
+        for (int j = j0; j < j0 + 4 && j < ncols; ++j) {
+          const float v = t[j];
+          const bool m = P < 0 ? true : (fabsf(v) > tau);
+          const double tr = m ? (v >= 0.0f ? (double)alpha : -(double)alpha) : 0.0;
+          const int q = quantize_q((double)v - tr, s);
+          word |= ((uint32_t)(uint8_t)(int8_t)q) << (8 * (j - j0));
+        }
+        *reinterpret_cast<uint32_t*>(qrow + j0) = word;
+      }
+    }
+    __syncthreads();
+  }
+  if (valid) {
+    // pads: codes K..res_stride (the word loop above already covered up to
+    // roundup(K, 4)), scales ng..scale_stride
+    int8_t* qrow = pw.res_q + (int64_t)row * pw.res_stride;
+    for (int j = (K + 3) / 4 * 4; j < pw.res_stride; j += 4)
+      *reinterpret_cast<uint32_t*>(qrow + j) = 0u;
+    for (int g = ng; g < pw.scale_stride; ++g)
+      pw.res_scale[(int64_t)row * pw.scale_stride + g] = 0.0f;
+    if (nonfinite) set_status(status, SQ_ERR_NONFINITE);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_decompose_pack(const float* W, int N, int K, int P, const sq_packed_weight& pw,
+                                  int32_t* status, cudaStream_t stream) {
+  if (P > 0) {
+    k_threshold<<<N, 256, 0, stream>>>(W, N, K, P, pw.alpha);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  const int G = pw.group_size;
+  const size_t smem = (size_t)kPackRows * (G + 1) * sizeof(float);
+  cudaError_t e = ensure_smem_attr((const void*)k_pack, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int blocks = (N + kPackRows - 1) / kPackRows;
+  k_pack<<<blocks, kPackRows, smem, stream>>>(W, N, K, P, G, pw, status);
+  return cudaGetLastError();
+}
+
+}  // namespace sq

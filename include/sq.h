@@ -1,0 +1,196 @@
+/*
+ * sq.h -- C ABI of the separated-quantization decode linear layer on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The method (Chinese-language web page "1-bit量化不是玄学，以往掉点是机制问题",
+ * m.lqnn.cn/news/241359, sections 2.1-2.3, 3.3, 5.2, 5.3 and 6.2):
+ *   W ~ alpha_r * sign(W) + W_res        one 1-bit sign trunk, one scale per row
+ *   W_res = W - alpha_r * sign(W)       re-quantized to INT8 (groups along K)
+ *   x -> fp32 outlier channels + INT8 per-token codes on the other channels
+ *   y = (trunk product by bit operations) + (residual integer product)
+ *       + (outlier channels at full precision), all in one kernel.
+ * The symmetric INT8 quantizer follows the "对称量化以零为中心" (absmax) section of
+ * the visual guide to LLM quantization (puppylpg.github.io) and the divide
+ * convention s = absmax/127, q = round(x/s) of the 2048ai.net explainer,
+ * section 三.1; the sign of zero follows the BitNet "权重量化" paragraph of the
+ * visual guide (non-negative -> +1).
+ *
+ * Conventions for every call:
+ *  - All pointers are DEVICE pointers owned by the caller, unless stated.
+ *    The library never allocates device memory; sizes are queryable.
+ *  - Every call is asynchronous on the caller's stream ("stream" is a
+ *    cudaStream_t; NULL = the legacy default stream).  The return value only
+ *    covers host-side validation and the launch itself.
+ *  - Device-side findings (non-finite input, a wait that ran out) are written
+ *    to the optional caller-owned int32 word "dev_status" (device memory): it
+ *    is left untouched on success and set to a sq_status code otherwise.
+ *  - Pointers must be 16-byte aligned (else SQ_ERR_ALIGN).
+ *  - The current device must be an sm_100 (B200-class) GPU, else
+ *    SQ_ERR_UNSUPPORTED_DEVICE.  There is no CPU fallback.
+ *  - Calls on one stream are ordered; calls that share output or workspace
+ *    buffers on different streams must be ordered by the caller.
+ */
+#ifndef SQ_H
+#define SQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SQ_OK = 0,
+  SQ_ERR_INVALID_ARG = 1,        /* NULL pointer, bad enum, unsorted index list */
+  SQ_ERR_SHAPE = 2,              /* size out of the supported range */
+  SQ_ERR_ALIGN = 3,              /* a pointer is not 16-byte aligned */
+  SQ_ERR_UNSUPPORTED_DEVICE = 4, /* current device is not sm_100 */
+  SQ_ERR_CUDA = 5,               /* a CUDA runtime call or launch failed */
+  SQ_ERR_NONFINITE = 6,          /* (device status) NaN or Inf in an input */
+  SQ_ERR_TIMEOUT = 7,            /* (device status) a bounded wait ran out */
+  SQ_ERR_WORKSPACE = 8           /* workspace missing or too small */
+} sq_status;
+
+/* Launch flags (bit set). */
+#define SQ_LAUNCH_PDL 1u
+/* SQ_LAUNCH_PDL: launch with programmatic dependent launch.  The kernel may
+ * start while the previous kernel in the stream is still running and begins
+ * streaming the packed weights at once; it reads every other input and writes
+ * every output only after the previous kernel has completed.  Set it only if
+ * no earlier work still in flight on the stream writes the packed weights. */
+
+/*
+ * Packed weight of one linear layer (N output rows, K input channels).
+ * Layout in device memory, all row-major, all rows 16-byte aligned:
+ *   sign_bits [N][sign_stride] u32  bit (j % 32) of word (j / 32) is 1 iff
+ *                                   W[r][j] >= 0 (so both zeros give 1);
+ *                                   pad bits and pad words are 0
+ *   mask_bits [N][sign_stride] u32  trunk membership, same bit layout; NULL
+ *                                   means every element is in the trunk
+ *   alpha     [N]              f32  per-row trunk scale
+ *   res_q     [N][res_stride]  i8   residual codes in [-127, 127]; pad 0
+ *   res_scale [N][scale_stride] f32 residual scale of group g = channels
+ *                                   [g*G, g*G + G); pad 0
+ * sign_stride  = roundup(ceil(K/32), 4) words
+ * res_stride   = roundup(K, 16) bytes
+ * scale_stride = roundup(ceil(K/G), 4) floats
+ * The arrays may live in one allocation carved by sq_packed_view().
+ */
+typedef struct {
+  int32_t N, K, group_size;  /* group_size G: 32, 64 or 128 */
+  int32_t sign_stride;       /* u32 words per row of sign_bits / mask_bits */
+  int32_t res_stride;        /* bytes per row of res_q */
+  int32_t scale_stride;      /* floats per row of res_scale */
+  uint32_t *sign_bits;
+  uint32_t *mask_bits;       /* NULL = full trunk */
+  float *alpha;
+  int8_t *res_q;
+  float *res_scale;
+} sq_packed_weight;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *sq_status_string(sq_status s);
+
+/* Checks that the current device is sm_100.  SQ_OK or SQ_ERR_UNSUPPORTED_DEVICE. */
+sq_status sq_device_check(void);
+
+/* Bytes of one allocation that holds a packed weight of this shape (the five
+ * arrays, each 256-byte aligned inside it).  0 for an unsupported shape. */
+size_t sq_packed_bytes(int32_t N, int32_t K, int32_t group_size, int32_t with_mask);
+
+/* Fills *out with the strides and with pointers into "base" (device memory of
+ * at least sq_packed_bytes() bytes, 256-byte aligned).  Host-only; no device
+ * work.  with_mask = 0 leaves mask_bits NULL. */
+sq_status sq_packed_view(void *base, int32_t N, int32_t K, int32_t group_size,
+                         int32_t with_mask, sq_packed_weight *out);
+
+/*
+ * Offline decomposition ("分离阶段（离线完成）", m.lqnn.cn section 5.3; the split of
+ * section 2.1; the per-row threshold of sections 5.2 and 6.2).
+ *   W             [N][K] f32 row-major, device, read only
+ *   trunk_percent < 0: every element is in the trunk (out->mask_bits may be
+ *                 NULL).  1..100: per row, tau_r = the ceil(P*K/100)-th
+ *                 smallest |W[r][j]| (nearest rank) and the trunk is
+ *                 |W| > tau_r (out->mask_bits must be set).
+ *   out           strides and pointers as from sq_packed_view(); written in
+ *                 full, pads included.
+ * alpha_r = float(S / cnt), S the binary64 sum of |W| over the trunk members
+ * in ascending channel order, cnt their number (0 -> alpha 0).  Residual
+ * r = double(W) - m*(+-alpha) in binary64; group scale s = float(absmax/127);
+ * code = clip(round_half_away(r / s), +-127) with a binary64 quotient (s == 0
+ * gives 0).  Non-finite W sets SQ_ERR_NONFINITE in dev_status.
+ */
+sq_status sq_decompose_pack(const float *W, int32_t N, int32_t K, int32_t trunk_percent,
+                            const sq_packed_weight *out, int32_t *dev_status, void *stream);
+
+/*
+ * Outlier calibration (m.lqnn.cn section 2.2: detect the outlier channels once,
+ * cache their indices, look them up at run time).
+ *   X        [T][K] f32 calibration activations, device
+ *   k        number of channels to keep, 1 <= k <= K
+ *   idx_out  [k] i32, device: the k channels with the largest max_t |X[t][j]|
+ *            (ties: the lower channel first), sorted ascending.
+ * K <= 57344.  Non-finite X counts as magnitude 0 and sets SQ_ERR_NONFINITE.
+ */
+sq_status sq_calibrate_outliers(const float *X, int32_t T, int32_t K, int32_t k,
+                                int32_t *idx_out, int32_t *dev_status, void *stream);
+
+/*
+ * Per-token activation split (m.lqnn.cn section 2.2; dynamic per-token scale
+ * of the visual guide's "动态量化" section).
+ *   x      [M][K] f32 activations, device
+ *   idx    [n_out] i32 outlier channels, strictly ascending in [0, K)
+ *          (host-checked only for n_out; the caller guarantees the order,
+ *          as produced by sq_calibrate_outliers)
+ *   xq     [M][roundup(K,16)] i8 out: codes, 0 on outlier channels and pads
+ *   sx     [M] f32 out: absmax over the non-outlier channels / 127
+ *   x_out  [M][n_out] f32 out: the outlier channels, copied
+ * 0 <= n_out <= 4096.  Non-finite x sets SQ_ERR_NONFINITE.
+ */
+sq_status sq_quantize_act(const float *x, int32_t M, int32_t K, const int32_t *idx,
+                          int32_t n_out, int8_t *xq, float *sx, float *x_out,
+                          int32_t *dev_status, uint32_t flags, void *stream);
+
+/* Workspace bytes sq_linear() needs for this weight and token count (split
+ * rows: per-CTA partial sums and per-row arrival counters).  The workspace
+ * must be zero-filled once before its first use; every call leaves it
+ * zero-filled again. */
+size_t sq_linear_workspace_bytes(const sq_packed_weight *w, int32_t M);
+
+/*
+ * Fused separated-quantization linear layer (m.lqnn.cn sections 2.3 and 3.3:
+ * trunk by bit operations, residual by integer products, summed in one
+ * kernel; the outlier channels of section 2.2 at full precision).
+ *   w           packed weight (device arrays)
+ *   xq, sx, x_out, idx, n_out   as written by sq_quantize_act
+ *   M           tokens, 1 <= M; the decode kernel takes M <= 16 per pass
+ *   y           [M][N] f32 out
+ *   workspace   device, ws_bytes >= sq_linear_workspace_bytes(w, M)
+ * For every token t and row r:
+ *   T  = sum_j m*(2b-1)*xq  = 2*sum_{m and b} xq - sum_m xq   (exact int32)
+ *   R_g = sum_{j in g} q*xq                                     (exact int32)
+ *   y  = sx*(alpha*T + sum_g s_g*R_g) + sum_i What[r][idx_i]*x_out[i]
+ * with What = m*(+-alpha) + s_g*q the dequantized weight, in fp32.
+ */
+sq_status sq_linear(const sq_packed_weight *w, const int8_t *xq, const float *sx,
+                    const float *x_out, const int32_t *idx, int32_t n_out, int32_t M,
+                    float *y, void *workspace, size_t ws_bytes, int32_t *dev_status,
+                    uint32_t flags, void *stream);
+
+/*
+ * Same kernel as sq_linear, additionally writing its exact integer
+ * accumulators for inspection:
+ *   T_out [M][N] i32, R_out [M][N][ceil(K/G)] i32.
+ * y is written as by sq_linear.  Intended for tests; not on the hot path.
+ */
+sq_status sq_linear_accumulators(const sq_packed_weight *w, const int8_t *xq,
+                                 const float *sx, const float *x_out, const int32_t *idx,
+                                 int32_t n_out, int32_t M, float *y, int32_t *T_out,
+                                 int32_t *R_out, void *workspace, size_t ws_bytes,
+                                 int32_t *dev_status, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SQ_H */

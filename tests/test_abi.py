@@ -1,0 +1,116 @@
+"""C-ABI checks that need no GPU: the libraries load, every function declared
+in include/sq.h is exported, the host-only layout calls agree with the
+documented strides, and host-side validation rejects bad arguments before
+any device work."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import decode_matvec_sq_b200 as sq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared(header):
+    text = open(header, encoding="utf-8").read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"\b(sq_[a-z_0-9]+)\s*\(", text)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def L():
+    import torch  # noqa: F401  (loads the CUDA runtime the library links against)
+    from decode_matvec_sq_b200 import build
+    build.build_libsq()
+    return sq.lib()
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = _declared(os.path.join(ROOT, "include", "sq.h"))
+    assert {"sq_decompose_pack", "sq_calibrate_outliers", "sq_quantize_act", "sq_linear"} <= set(names)
+    for n in names:
+        assert hasattr(L, n), f"{n} declared in include/sq.h but not exported"
+
+
+def test_oracle_exports_its_header():
+    import oracle
+    oracle.build()
+    lib = ctypes.CDLL(os.path.join(ROOT, "oracle", "libsq_oracle.so"))
+    for n in re.findall(r"\b(sqo_[a-z_0-9]+)\s*\(", open(os.path.join(ROOT, "oracle", "sq_oracle.h")).read()):
+        assert hasattr(lib, n)
+
+
+def test_status_strings(L):
+    for code in range(9):
+        assert L.sq_status_string(code)
+    assert L.sq_status_string(99) == b"unknown status"
+
+
+@pytest.mark.parametrize("N,K,G,mask", [(1, 1, 128, 0), (7, 33, 32, 1), (512, 512, 128, 0),
+                                        (12288, 4096, 128, 0), (8192, 28672, 64, 1)])
+def test_packed_view_layout(L, N, K, G, mask):
+    nbytes = L.sq_packed_bytes(N, K, G, mask)
+    assert nbytes > 0
+    base = 1 << 40  # a fake 256-aligned address: the view call does not touch memory
+    v = sq.SqPackedWeight()
+    assert L.sq_packed_view(ctypes.c_void_p(base), N, K, G, mask, ctypes.byref(v)) == 0
+    assert v.sign_stride == sq.round_up(sq.ceil_div(K, 32), 4)
+    assert v.res_stride == sq.round_up(K, 16)
+    assert v.scale_stride == sq.round_up(sq.ceil_div(K, G), 4)
+    spans = [(v.sign_bits, N * v.sign_stride * 4), (v.alpha, sq.round_up(N, 8) * 4),
+             (v.res_q, N * v.res_stride), (v.res_scale, N * v.scale_stride * 4)]
+    if mask:
+        spans.append((v.mask_bits, N * v.sign_stride * 4))
+    else:
+        assert v.mask_bits is None
+    spans.sort()
+    for (a, la), (b, _) in zip(spans, spans[1:]):
+        assert a % 256 == 0 and a + la <= b
+    assert spans[-1][0] + spans[-1][1] <= base + nbytes
+
+
+def test_packed_view_rejects(L):
+    v = sq.SqPackedWeight()
+    assert L.sq_packed_view(ctypes.c_void_p((1 << 40) + 16), 8, 8, 128, 0, ctypes.byref(v)) == 3
+    assert L.sq_packed_view(ctypes.c_void_p(1 << 40), 8, 8, 48, 0, ctypes.byref(v)) == 2
+    assert L.sq_packed_view(ctypes.c_void_p(1 << 40), 0, 8, 128, 0, ctypes.byref(v)) == 2
+    assert L.sq_packed_view(None, 8, 8, 128, 0, ctypes.byref(v)) == 1
+    assert L.sq_packed_bytes(8, 8, 100, 0) == 0
+
+
+def test_host_validation_before_device_work(L):
+    """Each of these returns from the host checks; no kernel is launched."""
+    v = sq.SqPackedWeight()
+    L.sq_packed_view(ctypes.c_void_p(1 << 40), 64, 256, 128, 0, ctypes.byref(v))
+    p = ctypes.c_void_p(1 << 41)
+    bad = ctypes.c_void_p((1 << 41) + 4)
+    assert L.sq_linear(None, p, p, p, p, 1, 1, p, p, 1 << 20, None, 0, None) == 1
+    assert L.sq_linear(ctypes.byref(v), None, p, p, p, 1, 1, p, p, 1 << 20, None, 0, None) == 1
+    assert L.sq_linear(ctypes.byref(v), p, p, p, p, 1, 0, p, p, 1 << 20, None, 0, None) == 2
+    assert L.sq_linear(ctypes.byref(v), bad, p, p, p, 1, 1, p, p, 1 << 20, None, 0, None) == 3
+    assert L.sq_linear(ctypes.byref(v), p, p, p, p, 1, 1, p, p, 1 << 20, None, 8, None) == 1
+    assert L.sq_linear(ctypes.byref(v), p, p, None, p, 1, 1, p, p, 1 << 20, None, 0, None) == 1
+    w2 = sq.SqPackedWeight.from_buffer_copy(v)
+    w2.res_stride = 100
+    assert L.sq_linear(ctypes.byref(w2), p, p, p, p, 1, 1, p, p, 1 << 20, None, 0, None) == 2
+    assert L.sq_decompose_pack(None, 64, 256, -1, ctypes.byref(v), None, None) == 1
+    assert L.sq_decompose_pack(p, 64, 256, 0, ctypes.byref(v), None, None) == 1
+    assert L.sq_decompose_pack(p, 64, 256, 60, ctypes.byref(v), None, None) == 1  # no mask array
+    assert L.sq_decompose_pack(p, 65, 256, -1, ctypes.byref(v), None, None) == 2
+    assert L.sq_quantize_act(p, 1, 256, p, -1, p, p, p, None, 0, None) == 2
+    assert L.sq_quantize_act(p, 1, 256, None, 3, p, p, p, None, 0, None) == 1
+    assert L.sq_calibrate_outliers(p, 64, 256, 0, p, None, None) == 2
+    assert L.sq_calibrate_outliers(p, 64, 256, 300, p, None, None) == 2
+
+
+def test_product_path_does_not_import_oracle():
+    """The package and its native sources never reach into oracle/."""
+    pkg = os.path.join(ROOT, "decode_matvec_sq_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                text = open(os.path.join(dirpath, f), encoding="utf-8").read()
+                assert "oracle" not in text.replace("no CPU fallback", ""), f

@@ -1,0 +1,403 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Integer and byte outputs (sign and mask bits, alpha, residual codes and
+scales, activation codes, outlier indices, the int32 trunk and group
+accumulators) must match bit for bit.  The float output y must satisfy
+|y - y_ref| <= 1e-5 * sum_j |W_rj * x_j| (original fp32 W and x), per element.
+Small shapes compare every element; full-size workloads compare sampled rows
+that the oracle recomputes from regenerated inputs.
+"""
+import numpy as np
+import pytest
+import torch
+
+import decode_matvec_sq_b200 as sq
+import oracle
+import synth
+import synth.device as sdev
+from synth import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+TOL = 1e-5
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built(cuda_device):
+    from decode_matvec_sq_b200 import build
+    build.build_all()
+    sq.device_check()
+    yield
+
+
+def unpack_words(words: torch.Tensor, K: int):
+    a = words.cpu().numpy().astype(np.int32).view(np.uint8)
+    bits = np.unpackbits(a, axis=1, bitorder="little")
+    return bits[:, :K], bits[:, K:]
+
+
+def check_packed(pw: sq.PackedWeight, d: dict, rows=None):
+    """GPU packed weight (optionally only `rows`) == oracle decomposition d."""
+    K = pw.K
+    sl = slice(None) if rows is None else torch.as_tensor(rows, device="cuda")
+    sign, sign_pad = unpack_words(pw.sign_bits()[sl], K)
+    assert np.array_equal(sign, d["sign"]), "sign bits"
+    assert not sign_pad.any(), "sign pad bits"
+    if pw.with_mask:
+        mask, mask_pad = unpack_words(pw.mask_bits()[sl], K)
+        assert np.array_equal(mask, d["mask"]), "mask bits"
+        assert not mask_pad.any()
+    else:
+        assert d["mask"].all()
+    alpha = pw.alpha()[sl].cpu().numpy()
+    assert np.array_equal(alpha.view(np.uint32), d["alpha"].view(np.uint32)), "alpha"
+    q = pw.res_q()[sl].cpu().numpy()
+    assert np.array_equal(q[:, :K], d["q"]), "residual codes"
+    assert not q[:, K:].any()
+    s = pw.res_scale()[sl].cpu().numpy()
+    ng = d["s"].shape[1]
+    assert np.array_equal(s[:, :ng].view(np.uint32), d["s"].view(np.uint32)), "group scales"
+    assert not s[:, ng:].any()
+
+
+def check_y(y, y_ref, bound, what="y"):
+    err = np.abs(y.astype(np.float64) - y_ref)
+    ok = err <= TOL * bound
+    assert ok.all(), f"{what}: {int((~ok).sum())} of {ok.size} outside tolerance; worst " \
+                     f"{float((err / np.maximum(bound, 1e-300)).max()):.3e}"
+
+
+def run_path(W: np.ndarray, x: np.ndarray, idx: np.ndarray, P=-1, G=128, pdl=False):
+    Wd = torch.from_numpy(W).cuda()
+    xd = torch.from_numpy(x).cuda()
+    idxd = torch.from_numpy(idx.astype(np.int32)).cuda()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pw = sq.decompose_pack(Wd, trunk_percent=P, group_size=G, status=status)
+    xq, sx, xo = sq.quantize_act(xd, idxd, status=status, pdl=pdl)
+    y, T, R = sq.linear_accumulators(pw, xq, sx, xo, idxd, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    return pw, (xq, sx, xo), (y, T, R)
+
+
+def full_compare(W, x, idx, P=-1, G=128):
+    pw, (xq, sx, xo), (y, T, R) = run_path(W, x, idx, P, G)
+    d = oracle.decompose(W, G=G, P=P)
+    check_packed(pw, d)
+    oxq, osx, oxo = oracle.quantize_act(x, idx)
+    K = W.shape[1]
+    assert np.array_equal(xq.cpu().numpy()[:, :K], oxq)
+    assert not xq.cpu().numpy()[:, K:].any()
+    assert np.array_equal(sx.cpu().numpy().view(np.uint32), osx.view(np.uint32))
+    if len(idx):
+        assert np.array_equal(xo.cpu().numpy()[:, :len(idx)], oxo)
+    oT, oR = oracle.accumulate(d, oxq)
+    assert np.array_equal(T.cpu().numpy().astype(np.int64), oT), "trunk accumulators"
+    assert np.array_equal(R.cpu().numpy().astype(np.int64), oR), "group accumulators"
+    y_ref = oracle.linear(d, oxq, osx, oxo, idx)
+    check_y(y.cpu().numpy(), y_ref, oracle.abs_dot(W, x))
+    return pw, y
+
+
+# ---- generators ------------------------------------------------------------------
+
+def test_device_generator_matches_host():
+    L1 = wl.config1()
+    Wd = sdev.fill_weights(L1, torch.empty(L1.N, L1.K, device="cuda"))
+    assert np.array_equal(Wd.cpu().numpy().view(np.uint32), L1.weights().view(np.uint32))
+    L3 = wl.config3()[1]
+    Wd = sdev.fill_weights(L3, torch.empty(16, L3.K, device="cuda"), row0=100)
+    assert np.array_equal(Wd.cpu().numpy().view(np.uint32),
+                          L3.weights(rows=np.arange(100, 116)).view(np.uint32))
+    L2 = wl.config2_layer(3, 3)
+    xd = sdev.fill_activations(L2, torch.empty(4, L2.K, device="cuda"))
+    assert np.array_equal(xd.cpu().numpy().view(np.uint32), L2.activations(M=4).view(np.uint32))
+    Xd = sdev.fill_activations(L2, torch.empty(wl.CAL_TOKENS, L2.K, device="cuda"), synth.STREAM_XCAL)
+    assert np.array_equal(Xd.cpu().numpy().view(np.uint32), L2.calibration().view(np.uint32))
+
+
+# ---- offline pack ------------------------------------------------------------------
+
+@pytest.mark.parametrize("N,K", [(1, 8), (7, 33), (8, 100), (13, 128), (9, 129), (64, 512),
+                                 (513, 300), (16, 4096), (3, 1000)])
+@pytest.mark.parametrize("G", [32, 64, 128])
+@pytest.mark.parametrize("P", [-1, 60])
+def test_pack_parity_shapes(N, K, G, P):
+    rng = np.random.default_rng(N * 1000 + K + G + P)
+    W = rng.laplace(0, 0.02, (N, K)).astype(np.float32)
+    W[0, : min(K, 5)] = np.array([0.0, -0.0, 1e-30, -1e-30, 0.5], np.float32)[: min(K, 5)]
+    if N > 2:
+        W[1] = 0.0                                   # all-zero row: alpha 0, codes 0
+        W[2, : K // 2] = np.round(W[2, : K // 2], 2)  # ties for the percentile
+    pw = sq.decompose_pack(torch.from_numpy(W).cuda(), trunk_percent=P, group_size=G)
+    torch.cuda.synchronize()
+    check_packed(pw, oracle.decompose(W, G=G, P=P))
+
+
+@pytest.mark.parametrize("P", [1, 50, 99, 100])
+def test_pack_threshold_percentiles(P):
+    rng = np.random.default_rng(P)
+    W = rng.laplace(0, 0.02, (37, 777)).astype(np.float32)
+    W[5] = np.round(W[5], 3)
+    pw = sq.decompose_pack(torch.from_numpy(W).cuda(), trunk_percent=P)
+    torch.cuda.synchronize()
+    check_packed(pw, oracle.decompose(W, P=P))
+
+
+def test_pack_nonfinite_status():
+    W = np.ones((4, 64), np.float32)
+    W[2, 7] = np.inf
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    sq.decompose_pack(torch.from_numpy(W).cuda(), status=st)
+    torch.cuda.synchronize()
+    assert st.item() == sq.STATUS_CODE["SQ_ERR_NONFINITE"]
+
+
+# ---- calibration and activation split ----------------------------------------------
+
+@pytest.mark.parametrize("layer", [wl.config1(), wl.config2_layer(0, 0), wl.config2_layer(0, 3),
+                                   wl.config3()[1]])
+def test_calibrate_parity(layer):
+    X = layer.calibration()
+    idx = sq.calibrate_outliers(torch.from_numpy(X).cuda(), layer.n_out)
+    torch.cuda.synchronize()
+    ref = oracle.calibrate(X, layer.n_out)
+    assert np.array_equal(idx.cpu().numpy(), ref)
+    assert np.array_equal(ref, layer.planted_channels())
+
+
+def test_calibrate_ties():
+    rng = np.random.default_rng(9)
+    X = np.round(rng.standard_normal((16, 1000)) * 3).astype(np.float32)
+    for k in (1, 7, 100, 1000):
+        idx = sq.calibrate_outliers(torch.from_numpy(X).cuda(), k)
+        torch.cuda.synchronize()
+        assert np.array_equal(idx.cpu().numpy(), oracle.calibrate(X, k)), k
+
+
+@pytest.mark.parametrize("M,K,n", [(1, 512, 4), (3, 100, 0), (2, 33, 5), (5, 4096, 20),
+                                   (1, 11008, 55), (16, 8192, 20), (1, 1, 0)])
+def test_quantize_act_parity(M, K, n):
+    rng = np.random.default_rng(M * K + n)
+    x = rng.standard_normal((M, K)).astype(np.float32)
+    idx = np.sort(rng.choice(K, n, replace=False)).astype(np.int32)
+    x[:, idx] *= 40.0
+    if M > 1:
+        x[1] = 0.0                                  # zero token
+    if K >= 8:
+        # exact midpoints: absmax 127 gives s = 1, values k + 0.5 tie
+        x[0, :8] = np.array([127.0, 2.5, -2.5, 0.5, -0.5, 126.5, -126.5, 1.5], np.float32)
+        x[0, idx] = np.where(idx < 8, 0.0, x[0, idx])
+    xq, sx, xo = sq.quantize_act(torch.from_numpy(x).cuda(),
+                                 torch.from_numpy(idx).cuda() if n else None)
+    torch.cuda.synchronize()
+    oxq, osx, oxo = oracle.quantize_act(x, idx)
+    assert np.array_equal(xq.cpu().numpy()[:, :K], oxq)
+    assert not xq.cpu().numpy()[:, K:].any()
+    assert np.array_equal(sx.cpu().numpy().view(np.uint32), osx.view(np.uint32))
+    if n:
+        assert np.array_equal(xo.cpu().numpy(), oxo)
+
+
+def test_quantize_act_random_midpoints():
+    """Values on exact half-steps of many different scales."""
+    rng = np.random.default_rng(4)
+    M, K = 64, 256
+    a = rng.uniform(0.1, 100.0, M).astype(np.float32)
+    s = (a.astype(np.float64) / 127.0).astype(np.float32)
+    k = rng.integers(0, 127, (M, K))
+    x = ((k + 0.5) * s[:, None].astype(np.float64)).astype(np.float32)
+    x *= rng.choice([-1, 1], (M, K)).astype(np.float32)
+    x[:, 0] = a
+    xq, sx, _ = sq.quantize_act(torch.from_numpy(x).cuda(), None)
+    torch.cuda.synchronize()
+    oxq, osx, _ = oracle.quantize_act(x, np.zeros(0, np.int32))
+    assert np.array_equal(sx.cpu().numpy(), osx)
+    assert np.array_equal(xq.cpu().numpy()[:, :K], oxq)
+
+
+# ---- fused linear: small shapes, every element --------------------------------------
+
+@pytest.mark.parametrize("N,K,M,n", [(1, 8, 1, 0), (7, 33, 1, 2), (8, 100, 2, 3), (513, 300, 1, 6),
+                                     (64, 512, 3, 4), (16, 4096, 4, 20), (33, 1000, 5, 9),
+                                     (40, 129, 8, 1), (24, 11008, 1, 55), (8, 28672, 1, 72),
+                                     (100, 2048, 16, 10)])
+@pytest.mark.parametrize("P", [-1, 60])
+def test_linear_parity_small(N, K, M, n, P):
+    rng = np.random.default_rng(N + K + M + n + P)
+    W = rng.laplace(0, 0.02, (N, K)).astype(np.float32)
+    x = rng.standard_normal((M, K)).astype(np.float32)
+    idx = np.sort(rng.choice(K, n, replace=False)).astype(np.int32)
+    x[:, idx] *= 30.0
+    full_compare(W, x, idx, P=P)
+
+
+@pytest.mark.parametrize("G", [32, 64])
+def test_linear_parity_group_sizes(G):
+    rng = np.random.default_rng(G)
+    W = rng.laplace(0, 0.02, (50, 1500)).astype(np.float32)
+    x = rng.standard_normal((2, 1500)).astype(np.float32)
+    idx = np.array([0, 31, 32, 700, 1499], np.int32)
+    full_compare(W, x, idx, G=G)
+
+
+def test_linear_degenerate():
+    rng = np.random.default_rng(0)
+    W = np.zeros((9, 64), np.float32)
+    x = rng.standard_normal((1, 64)).astype(np.float32)
+    full_compare(W, x, np.array([3], np.int32))          # zero weights: y = 0
+    W = rng.laplace(0, 0.02, (9, 64)).astype(np.float32)
+    full_compare(W, np.zeros((2, 64), np.float32), np.array([3], np.int32))  # zero tokens
+    x = np.zeros((1, 64), np.float32)
+    x[0, 3] = 7.0                                         # only the outlier channel is live
+    full_compare(W, x, np.array([3], np.int32))
+    full_compare(W[:1, :1], np.ones((1, 1), np.float32), np.zeros(0, np.int32))
+
+
+def test_linear_deterministic_and_split_rows():
+    """N=8, K=28672: one 8-row block split over 14 CTAs (stream of partials)."""
+    rng = np.random.default_rng(1)
+    W = rng.laplace(0, 0.02, (8, 28672)).astype(np.float32)
+    x = rng.standard_normal((1, 28672)).astype(np.float32)
+    idx = np.sort(rng.choice(28672, 72, replace=False)).astype(np.int32)
+    Wd, xd, idxd = (torch.from_numpy(a).cuda() for a in (W, x, idx))
+    pw = sq.decompose_pack(Wd)
+    xq, sx, xo = sq.quantize_act(xd, idxd)
+    ws = sq.new_workspace(pw, 1)
+    ys = [sq.linear(pw, xq, sx, xo, idxd, workspace=ws).cpu().numpy() for _ in range(5)]
+    torch.cuda.synchronize()
+    for y in ys[1:]:
+        assert np.array_equal(y.view(np.uint32), ys[0].view(np.uint32))
+    assert not ws.any().item(), "workspace left zero-filled"
+    d = oracle.decompose(W)
+    oxq, osx, oxo = oracle.quantize_act(x, idx)
+    check_y(ys[0], oracle.linear(d, oxq, osx, oxo, idx), oracle.abs_dot(W, x))
+
+
+def test_linear_errors():
+    W = torch.randn(16, 256, device="cuda")
+    pw = sq.decompose_pack(W)
+    xq, sx, xo = sq.quantize_act(torch.randn(1, 256, device="cuda"), None)
+    small = torch.zeros(16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(sq.SQError) as e:
+        sq.linear(pw, xq, sx, xo, None, workspace=small)
+    assert e.value.name == "SQ_ERR_WORKSPACE"
+    y = torch.empty(2, 17, device="cuda")
+    with pytest.raises(sq.SQError) as e:
+        sq.linear(pw, xq, sx, xo, None, y=y.view(-1)[1:17].view(1, 16))
+    assert e.value.name == "SQ_ERR_ALIGN"
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    x = torch.randn(1, 256, device="cuda")
+    x[0, 5] = float("nan")
+    sq.quantize_act(x, None, status=st)
+    torch.cuda.synchronize()
+    assert st.item() == sq.STATUS_CODE["SQ_ERR_NONFINITE"]
+    st.zero_()
+    bad_idx = torch.tensor([5, 3], dtype=torch.int32, device="cuda")
+    sq.quantize_act(torch.randn(1, 256, device="cuda"), bad_idx, status=st)
+    torch.cuda.synchronize()
+    assert st.item() == sq.STATUS_CODE["SQ_ERR_INVALID_ARG"]
+
+
+# ---- the five workloads ------------------------------------------------------------
+
+def test_config1_full_pipeline():
+    """512 x 512, batch 1, top-4 calibrated outliers: every output element."""
+    L = wl.config1()
+    X = torch.from_numpy(L.calibration()).cuda()
+    idx = sq.calibrate_outliers(X, L.n_out)
+    W, x = L.weights(), L.activations()
+    torch.cuda.synchronize()
+    assert np.array_equal(idx.cpu().numpy(), L.planted_channels())
+    full_compare(W, x, idx.cpu().numpy())
+
+
+def test_config4_threshold_full():
+    """4096 -> 14336 threshold trunk (per-row 60th percentile), batch 1, every row."""
+    L = wl.config4()
+    W, x, idx = L.weights(), L.activations(), L.planted_channels()
+    full_compare(W, x, idx, P=L.trunk_percent)
+
+
+def _sampled_layer(L, M, rows, pdl=False):
+    """Full-size layer generated on the device; oracle on sampled rows."""
+    Wd = sdev.fill_weights(L, torch.empty(L.N, L.K, device="cuda"))
+    Xc = sdev.fill_activations(L, torch.empty(wl.CAL_TOKENS, L.K, device="cuda"), synth.STREAM_XCAL)
+    xd = sdev.fill_activations(L, torch.empty(M, L.K, device="cuda"))
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pw = sq.decompose_pack(Wd, trunk_percent=L.trunk_percent, status=st)
+    del Wd
+    idx = sq.calibrate_outliers(Xc, L.n_out, status=st)
+    xq, sx, xo = sq.quantize_act(xd, idx, status=st, pdl=pdl)
+    y, T, R = sq.linear_accumulators(pw, xq, sx, xo, idx, status=st)
+    y2 = sq.linear(pw, xq, sx, xo, idx, status=st, pdl=pdl)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    assert torch.equal(y, y2)
+    idx_h = idx.cpu().numpy()
+    assert np.array_equal(idx_h, oracle.calibrate(L.calibration(), L.n_out))
+    Wr = L.weights(rows=rows)
+    x = L.activations(M=M)
+    d = oracle.decompose(Wr, P=L.trunk_percent)
+    check_packed(pw, d, rows=rows)
+    oxq, osx, oxo = oracle.quantize_act(x, idx_h)
+    assert np.array_equal(xq.cpu().numpy()[:, :L.K], oxq)
+    oT, oR = oracle.accumulate(d, oxq)
+    rt = torch.as_tensor(rows, device="cuda")
+    assert np.array_equal(T[:, rt].cpu().numpy().astype(np.int64), oT)
+    assert np.array_equal(R[:, rt].cpu().numpy().astype(np.int64), oR)
+    check_y(y[:, rt].cpu().numpy(), oracle.linear(d, oxq, osx, oxo, idx_h), oracle.abs_dot(Wr, x))
+
+
+def _rows(N, n=96, seed=0):
+    rng = np.random.default_rng(seed)
+    r = set(rng.choice(N, n, replace=False).tolist()) | {0, 1, 7, 8, N // 2, N - 9, N - 8, N - 1}
+    return np.array(sorted(r))
+
+
+@pytest.mark.parametrize("M", [1, 2, 4, 8, 16])
+@pytest.mark.parametrize("which", [0, 1])
+def test_config3_batch_sweep_sampled(M, which):
+    L = wl.config3(M)[which]
+    _sampled_layer(L, M, _rows(L.N, seed=M + which))
+
+
+@pytest.mark.parametrize("layer", [0, 31])
+@pytest.mark.parametrize("mid", [0, 1, 2, 3])
+def test_config2_stack_layers_sampled(layer, mid):
+    L = wl.config2_layer(layer, mid)
+    _sampled_layer(L, 1, _rows(L.N, seed=layer * 4 + mid), pdl=True)
+
+
+# ---- launch modes ----------------------------------------------------------------
+
+def test_pdl_chain_in_cuda_graph_matches_plain():
+    """quantize -> linear pairs launched with PDL inside a captured graph."""
+    layers = [wl.config2_layer(0, m) for m in range(4)] + [wl.config1()]
+    pws, xs, idxs, ys_plain = [], [], [], []
+    for L in layers:
+        Wd = sdev.fill_weights(L, torch.empty(L.N, L.K, device="cuda"))
+        pws.append(sq.decompose_pack(Wd))
+        xs.append(sdev.fill_activations(L, torch.empty(1, L.K, device="cuda")))
+        idxs.append(torch.from_numpy(L.planted_channels()).cuda())
+    ws = sq.new_workspace(max(pws, key=lambda p: p.N), 1)
+    bufs = [sq.quantize_act(x, i) for x, i in zip(xs, idxs)]
+    ys = [torch.empty(1, p.N, device="cuda") for p in pws]
+    for p, (xq, sx, xo), i, y in zip(pws, bufs, idxs, ys):
+        ys_plain.append(sq.linear(p, xq, sx, xo, i, workspace=ws).clone())
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            for p, x, i, (xq, sx, xo), y in zip(pws, xs, idxs, bufs, ys):
+                sq.quantize_act(x, i, xq=xq, sx=sx, x_out=xo, pdl=True)
+                sq.linear(p, xq, sx, xo, i, y=y, workspace=ws, pdl=True)
+    for _ in range(3):
+        for y in ys:
+            y.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        for y, yp in zip(ys, ys_plain):
+            assert torch.equal(y, yp)
+    assert not ws.any().item()
