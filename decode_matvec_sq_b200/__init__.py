@@ -220,6 +220,12 @@ def workspace_bytes(pw: PackedWeight, M: int = 1) -> int:
     return int(lib().sq_linear_workspace_bytes(ctypes.byref(pw.view), M))
 
 
+def workspace_counters(ws, pw: PackedWeight, M: int = 1):
+    """The per-row arrival counters inside a workspace (they end every call at zero)."""
+    base = workspace_bytes(pw, M) - round_up(4 * pw.N, 256)
+    return ws[base: base + 4 * pw.N]
+
+
 def new_workspace(pw: PackedWeight, M: int = 1, device=None):
     """A zero-filled workspace for sq_linear (zero once; calls keep it zeroed)."""
     import torch
@@ -252,7 +258,7 @@ def linear_accumulators(pw: PackedWeight, xq, sx, x_out, idx, workspace=None, st
     n = 0 if idx is None else int(idx.numel())
     dev = xq.device
     ng = ceil_div(pw.K, pw.group_size)
-    y = torch.empty(M, pw.N, dtype=torch.float32, device=dev)
+    y = torch.full((M, pw.N), float("nan"), dtype=torch.float32, device=dev)
     T = torch.empty(M, pw.N, dtype=torch.int32, device=dev)
     R = torch.empty(M, pw.N, ng, dtype=torch.int32, device=dev)
     if workspace is None:

@@ -68,7 +68,8 @@ typedef enum {
  *                                   pad bits and pad words are 0
  *   mask_bits [N][sign_stride] u32  trunk membership, same bit layout; NULL
  *                                   means every element is in the trunk
- *   alpha     [N]              f32  per-row trunk scale
+ *   alpha     [roundup(N,4)]   f32  per-row trunk scale (entries past N are
+ *                                   read as padding of 8-row blocks, never used)
  *   res_q     [N][res_stride]  i8   residual codes in [-127, 127]; pad 0
  *   res_scale [N][scale_stride] f32 residual scale of group g = channels
  *                                   [g*G, g*G + G); pad 0
@@ -131,7 +132,7 @@ sq_status sq_decompose_pack(const float *W, int32_t N, int32_t K, int32_t trunk_
  *   k        number of channels to keep, 1 <= k <= K
  *   idx_out  [k] i32, device: the k channels with the largest max_t |X[t][j]|
  *            (ties: the lower channel first), sorted ascending.
- * K <= 57344.  Non-finite X counts as magnitude 0 and sets SQ_ERR_NONFINITE.
+ * K <= 40960.  Non-finite X counts as magnitude 0 and sets SQ_ERR_NONFINITE.
  */
 sq_status sq_calibrate_outliers(const float *X, int32_t T, int32_t K, int32_t k,
                                 int32_t *idx_out, int32_t *dev_status, void *stream);
@@ -152,10 +153,13 @@ sq_status sq_quantize_act(const float *x, int32_t M, int32_t K, const int32_t *i
                           int32_t n_out, int8_t *xq, float *sx, float *x_out,
                           int32_t *dev_status, uint32_t flags, void *stream);
 
-/* Workspace bytes sq_linear() needs for this weight and token count (split
- * rows: per-CTA partial sums and per-row arrival counters).  The workspace
- * must be zero-filled once before its first use; every call leaves it
- * zero-filled again. */
+/* Workspace bytes sq_linear() needs for this weight and token count on the
+ * current device.  Layout: a partial-sum area whose size depends only on the
+ * device (for rows split between warps), then one int32 arrival counter per
+ * row (the last roundup(4*N, 256) bytes).  Zero-fill the workspace once
+ * before its first use; every call leaves the counters zero again (the
+ * partial sums are scratch).  One workspace may serve calls on different
+ * weights, in stream order, if it is at least as large as each call needs. */
 size_t sq_linear_workspace_bytes(const sq_packed_weight *w, int32_t M);
 
 /*

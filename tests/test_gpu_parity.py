@@ -264,11 +264,14 @@ def test_linear_deterministic_and_split_rows():
     pw = sq.decompose_pack(Wd)
     xq, sx, xo = sq.quantize_act(xd, idxd)
     ws = sq.new_workspace(pw, 1)
-    ys = [sq.linear(pw, xq, sx, xo, idxd, workspace=ws).cpu().numpy() for _ in range(5)]
+    ys = []
+    for _ in range(5):
+        y = torch.full((1, 8), float("nan"), device="cuda")
+        ys.append(sq.linear(pw, xq, sx, xo, idxd, y=y, workspace=ws).cpu().numpy())
     torch.cuda.synchronize()
     for y in ys[1:]:
         assert np.array_equal(y.view(np.uint32), ys[0].view(np.uint32))
-    assert not ws.any().item(), "workspace left zero-filled"
+    assert not sq.workspace_counters(ws, pw).any().item(), "arrival counters left zero-filled"
     d = oracle.decompose(W)
     oxq, osx, oxo = oracle.quantize_act(x, idx)
     check_y(ys[0], oracle.linear(d, oxq, osx, oxo, idx), oracle.abs_dot(W, x))
@@ -330,7 +333,8 @@ def _sampled_layer(L, M, rows, pdl=False):
     idx = sq.calibrate_outliers(Xc, L.n_out, status=st)
     xq, sx, xo = sq.quantize_act(xd, idx, status=st, pdl=pdl)
     y, T, R = sq.linear_accumulators(pw, xq, sx, xo, idx, status=st)
-    y2 = sq.linear(pw, xq, sx, xo, idx, status=st, pdl=pdl)
+    y2 = torch.full_like(y, float("nan"))
+    sq.linear(pw, xq, sx, xo, idx, y=y2, status=st, pdl=pdl)
     torch.cuda.synchronize()
     assert st.item() == 0
     assert torch.equal(y, y2)
@@ -384,7 +388,8 @@ def test_pdl_chain_in_cuda_graph_matches_plain():
     bufs = [sq.quantize_act(x, i) for x, i in zip(xs, idxs)]
     ys = [torch.empty(1, p.N, device="cuda") for p in pws]
     for p, (xq, sx, xo), i, y in zip(pws, bufs, idxs, ys):
-        ys_plain.append(sq.linear(p, xq, sx, xo, i, workspace=ws).clone())
+        y.fill_(float("nan"))
+        ys_plain.append(sq.linear(p, xq, sx, xo, i, y=y, workspace=ws).clone())
     torch.cuda.synchronize()
     g = torch.cuda.CUDAGraph()
     s = torch.cuda.Stream()
@@ -395,9 +400,47 @@ def test_pdl_chain_in_cuda_graph_matches_plain():
                 sq.linear(p, xq, sx, xo, i, y=y, workspace=ws, pdl=True)
     for _ in range(3):
         for y in ys:
-            y.zero_()
+            y.fill_(float("nan"))
         g.replay()
         torch.cuda.synchronize()
         for y, yp in zip(ys, ys_plain):
             assert torch.equal(y, yp)
-    assert not ws.any().item()
+    for p in pws:
+        assert not sq.workspace_counters(ws, p).any().item()
+
+
+def test_shared_workspace_across_shapes():
+    """One workspace serving layers of different N, called in interleaved
+    order: every row is written every time and matches the oracle."""
+    layers = [wl.config2_layer(1, m) for m in (0, 2, 1, 3)] + [wl.config1()]
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    items = []
+    for L in layers:
+        Wd = sdev.fill_weights(L, torch.empty(L.N, L.K, device="cuda"))
+        pw = sq.decompose_pack(Wd)
+        del Wd
+        idx = torch.from_numpy(L.planted_channels()).cuda()
+        x = sdev.fill_activations(L, torch.empty(1, L.K, device="cuda"))
+        items.append((L, pw, idx, sq.quantize_act(x, idx, status=st)))
+    ws = torch.zeros(max(sq.workspace_bytes(pw, 1) for _, pw, _, _ in items), dtype=torch.uint8,
+                     device="cuda")
+    outs = {}
+    for rep in range(3):
+        for L, pw, idx, (xq, sx, xo) in items[::(1 if rep % 2 == 0 else -1)]:
+            y = torch.full((1, L.N), float("nan"), device="cuda")
+            sq.linear(pw, xq, sx, xo, idx, y=y, workspace=ws, status=st)
+            torch.cuda.synchronize()
+            assert not torch.isnan(y).any().item(), f"{L.name}: rows not written"
+            if L.name in outs:
+                assert torch.equal(outs[L.name], y), f"{L.name}: not reproducible"
+            outs[L.name] = y
+    assert st.item() == 0
+    for L, pw, idx, _ in items:
+        assert not sq.workspace_counters(ws, pw).any().item()
+        rows = _rows(L.N, n=48, seed=L.N)
+        Wr, x = L.weights(rows=rows), L.activations()
+        d = oracle.decompose(Wr)
+        oxq, osx, oxo = oracle.quantize_act(x, L.planted_channels())
+        y_ref = oracle.linear(d, oxq, osx, oxo, L.planted_channels())
+        check_y(outs[L.name][:, torch.as_tensor(rows, device="cuda")].cpu().numpy(), y_ref,
+                oracle.abs_dot(Wr, x), L.name)
