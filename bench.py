@@ -276,9 +276,10 @@ class Stack:
     def step(self, pdl=None):
         import decode_matvec_sq_b200 as sq
         pdl = self.pdl if pdl is None else pdl
-        for pw, x, idx, (xq, sx, xo), y in zip(self.pws, self.xs, self.idx, self.bufs, self.ys):
-            sq.quantize_act(x, idx, xq=xq, sx=sx, x_out=xo, status=self.status, pdl=pdl)
-            sq.linear(pw, xq, sx, xo, idx, y=y, workspace=self.ws, status=self.status, pdl=pdl)
+        for pw, x, idx, a, y in zip(self.pws, self.xs, self.idx, self.bufs, self.ys):
+            sq.quantize_act(x, idx, xq=a[0], sx=a[1], x_out=a[2], status=self.status, pdl=pdl)
+            sq.linear(pw, a[0], a[1], a[2], idx, y=y, workspace=self.ws, status=self.status,
+                      pdl=pdl)
 
     def capture(self):
         import torch
@@ -303,11 +304,12 @@ class Stack:
         evs = []
         stream = torch.cuda.current_stream()
         for _ in range(reps):
-            for pw, idx, (xq, sx, xo), y, L in zip(self.pws, self.idx, self.bufs, self.ys, self.layers):
+            for pw, idx, act, y, L in zip(self.pws, self.idx, self.bufs, self.ys, self.layers):
                 a = torch.cuda.Event(enable_timing=True)
                 b = torch.cuda.Event(enable_timing=True)
                 a.record(stream)
-                sq.linear(pw, xq, sx, xo, idx, y=y, workspace=self.ws, status=self.status)
+                sq.linear(pw, act[0], act[1], act[2], idx, y=y, workspace=self.ws,
+                          status=self.status)
                 b.record(stream)
                 evs.append((L, a, b))
         torch.cuda.synchronize()

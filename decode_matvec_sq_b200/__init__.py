@@ -22,6 +22,7 @@ LIB_PATH = os.path.join(PKG_DIR, "libsq.so")
 HEADER = os.path.join(os.path.dirname(PKG_DIR), "include", "sq.h")
 
 SQ_LAUNCH_PDL = 1
+SQ_LAUNCH_CUDA_CORES = 2
 
 STATUS = {
     0: "SQ_OK", 1: "SQ_ERR_INVALID_ARG", 2: "SQ_ERR_SHAPE", 3: "SQ_ERR_ALIGN",
@@ -72,7 +73,7 @@ def lib():
         "sq_quantize_act": ([vp, i32, i32, vp, i32, vp, vp, vp, vp, u32, vp], ctypes.c_int),
         "sq_linear_workspace_bytes": ([pw, i32], sz),
         "sq_linear": ([pw, vp, vp, vp, vp, i32, i32, vp, vp, sz, vp, u32, vp], ctypes.c_int),
-        "sq_linear_accumulators": ([pw, vp, vp, vp, vp, i32, i32, vp, vp, vp, vp, sz, vp, vp],
+        "sq_linear_accumulators": ([pw, vp, vp, vp, vp, i32, i32, vp, vp, vp, vp, sz, vp, u32, vp],
                                    ctypes.c_int),
     }
     for name, (args, res) in sig.items():
@@ -233,9 +234,14 @@ def new_workspace(pw: PackedWeight, M: int = 1, device=None):
                        device=device or pw.buf.device)
 
 
+def _flags(pdl: bool, cuda_cores: bool) -> int:
+    return (SQ_LAUNCH_PDL if pdl else 0) | (SQ_LAUNCH_CUDA_CORES if cuda_cores else 0)
+
+
 def linear(pw: PackedWeight, xq, sx, x_out, idx, y=None, workspace=None, status=None,
-           pdl: bool = False, stream=None):
-    """y[M][N] = fused trunk + residual + outlier product (float32)."""
+           pdl: bool = False, cuda_cores: bool = False, stream=None):
+    """y[M][N] = fused trunk + residual + outlier product (float32).
+    ``cuda_cores`` selects the dp4a kernel instead of the tensor-core one."""
     import torch
     M = xq.shape[0]
     n = 0 if idx is None else int(idx.numel())
@@ -245,13 +251,13 @@ def linear(pw: PackedWeight, xq, sx, x_out, idx, y=None, workspace=None, status=
         workspace = new_workspace(pw, M)
     _ck(lib().sq_linear(ctypes.byref(pw.view), _ptr(xq), _ptr(sx), _ptr(x_out) if n else None,
                         _ptr(idx) if n else None, n, M, _ptr(y), _ptr(workspace),
-                        workspace.numel(), _ptr(status), SQ_LAUNCH_PDL if pdl else 0,
+                        workspace.numel(), _ptr(status), _flags(pdl, cuda_cores),
                         _stream(stream)), "sq_linear")
     return y
 
 
 def linear_accumulators(pw: PackedWeight, xq, sx, x_out, idx, workspace=None, status=None,
-                        stream=None):
+                        cuda_cores: bool = False, stream=None):
     """(y, T [M][N] int32, R [M][N][ceil(K/G)] int32) from the decode kernel."""
     import torch
     M = xq.shape[0]
@@ -266,6 +272,6 @@ def linear_accumulators(pw: PackedWeight, xq, sx, x_out, idx, workspace=None, st
     _ck(lib().sq_linear_accumulators(ctypes.byref(pw.view), _ptr(xq), _ptr(sx),
                                      _ptr(x_out) if n else None, _ptr(idx) if n else None, n, M,
                                      _ptr(y), _ptr(T), _ptr(R), _ptr(workspace),
-                                     workspace.numel(), _ptr(status), _stream(stream)),
-        "sq_linear_accumulators")
+                                     workspace.numel(), _ptr(status), _flags(False, cuda_cores),
+                                     _stream(stream)), "sq_linear_accumulators")
     return y, T, R

@@ -33,6 +33,7 @@ SOURCES = [
     ("sq_pack.cu", ["-fmad=false"]),
     ("sq_act.cu", ["-fmad=false"]),
     ("sq_linear.cu", []),
+    ("sq_linear_tc.cu", []),
 ]
 
 

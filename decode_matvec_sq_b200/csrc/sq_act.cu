@@ -16,7 +16,7 @@
 namespace sq {
 namespace {
 
-constexpr int kActThreads = 512;
+constexpr int kActThreads = 1024;
 constexpr int kCalThreads = 1024;
 
 // round_half_away(|v| / s) decided exactly.  t = |v| * (1/s) is within far
@@ -36,6 +36,15 @@ __device__ __forceinline__ int quantize_exact(float v, float s, double rinv) {
   return v < 0.0f ? -qi : qi;
 }
 
+// One CTA per token; warp w handles the 32-channel chunks w, w + 32, ...
+// with one channel per lane, keeping its x values in registers between the
+// absmax pass and the code pass (one global round trip).
+constexpr int kActRegs = 28;  // chunks per warp kept in registers: K <= 32*32*28
+
+__device__ __forceinline__ bool outlier_bit(const uint32_t* is_out, int j) {
+  return (is_out[j >> 5] >> (j & 31)) & 1u;
+}
+
 __global__ void __launch_bounds__(kActThreads) k_quantize_act(
     const float* __restrict__ x, int M, int K, int K16, const int32_t* __restrict__ idx, int n_out,
     int8_t* __restrict__ xq, float* __restrict__ sx, float* __restrict__ x_out,
@@ -47,10 +56,18 @@ __global__ void __launch_bounds__(kActThreads) k_quantize_act(
     pdl_wait();
   }
   const int t = blockIdx.x;
-  const int nw = (K + 31) / 32;
-  for (int i = threadIdx.x; i < nw; i += blockDim.x) is_out[i] = 0u;
-  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nchunk = (K + 31) >> 5;  // also ceil(K16 / 32)
   const float* xt = x + (int64_t)t * K;
+  // x into registers (issued before anything else)
+  float v[kActRegs];
+#pragma unroll
+  for (int i = 0; i < kActRegs; ++i) {
+    const int j = (warp + 32 * i) * 32 + lane;
+    v[i] = j < K ? __ldg(xt + j) : 0.0f;
+  }
+  for (int i = threadIdx.x; i < nchunk; i += blockDim.x) is_out[i] = 0u;
+  __syncthreads();
   bool bad_idx = false;
   for (int i = threadIdx.x; i < n_out; i += blockDim.x) {
     const int j = idx[i];
@@ -63,33 +80,52 @@ __global__ void __launch_bounds__(kActThreads) k_quantize_act(
 
   float a = 0.0f;
   bool nonfinite = false;
-  for (int j = threadIdx.x; j < K; j += blockDim.x) {
-    const float v = xt[j];
-    nonfinite |= !isfinite(v);
-    if (!((is_out[j >> 5] >> (j & 31)) & 1u)) a = fmaxf(a, fabsf(v));
+  const bool big = nchunk > 32 * kActRegs;  // more chunks than registers: re-read x
+#pragma unroll
+  for (int i = 0; i < kActRegs; ++i) {
+    const int j = (warp + 32 * i) * 32 + lane;
+    if (j < K) {
+      nonfinite |= !isfinite(v[i]);
+      if (!outlier_bit(is_out, j)) a = fmaxf(a, fabsf(v[i]));
+    }
+  }
+  if (big) {
+    for (int c = warp + 32 * kActRegs; c < nchunk; c += 32) {
+      const int j = c * 32 + lane;
+      if (j < K) {
+        const float u = xt[j];
+        nonfinite |= !isfinite(u);
+        if (!outlier_bit(is_out, j)) a = fmaxf(a, fabsf(u));
+      }
+    }
   }
   for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-  if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = a;
+  if (lane == 0) warp_max[warp] = a;
   __syncthreads();
-  a = 0.0f;
-  for (int w = 0; w < kActThreads / 32; ++w) a = fmaxf(a, warp_max[w]);
+  a = warp_max[lane];
+  for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
 
   const float s = (float)((double)a / 127.0);
   const double rinv = s != 0.0f ? 1.0 / (double)s : 0.0;
   if (threadIdx.x == 0) sx[t] = s;
 
-  // codes, four channels per 32-bit store; outlier slots and pads are 0
   int8_t* qt = xq + (int64_t)t * K16;
-  for (int j0 = threadIdx.x * 4; j0 < K16; j0 += blockDim.x * 4) {
-    uint32_t word = 0;
+  auto emit = [&](int c, float u) {
+    const int j = c * 32 + lane;
+    int q = 0;
+    if (j < K && !outlier_bit(is_out, j)) q = quantize_exact(u, s, rinv);
+    if (j < K16) qt[j] = (int8_t)q;
+  };
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int j = j0 + k;
-      int q = 0;
-      if (j < K && !((is_out[j >> 5] >> (j & 31)) & 1u)) q = quantize_exact(xt[j], s, rinv);
-      word |= ((uint32_t)(uint8_t)(int8_t)q) << (8 * k);
+  for (int i = 0; i < kActRegs; ++i) {
+    const int c = warp + 32 * i;
+    if (c < nchunk) emit(c, v[i]);
+  }
+  if (big) {
+    for (int c = warp + 32 * kActRegs; c < nchunk; c += 32) {
+      const int j = c * 32 + lane;
+      emit(c, j < K ? xt[j] : 0.0f);
     }
-    *reinterpret_cast<uint32_t*>(qt + j0) = word;
   }
   if (nonfinite) set_status(status, SQ_ERR_NONFINITE);
   if (bad_idx) set_status(status, SQ_ERR_INVALID_ARG);

@@ -237,7 +237,7 @@ static sq_status linear_common(const sq_packed_weight* w, const int8_t* xq, cons
   if (M < 1 || M > (1 << 20)) return SQ_ERR_SHAPE;
   if (n_out < 0 || n_out > kMaxOutliers || n_out > w->K) return SQ_ERR_SHAPE;
   if (n_out > 0 && (!idx || !x_out)) return SQ_ERR_INVALID_ARG;
-  if (flags & ~SQ_LAUNCH_PDL) return SQ_ERR_INVALID_ARG;
+  if (flags & ~(SQ_LAUNCH_PDL | SQ_LAUNCH_CUDA_CORES)) return SQ_ERR_INVALID_ARG;
   if (!aligned16(xq) || !aligned16(sx) || !aligned16(y) ||
       (n_out > 0 && (!aligned16(idx) || !aligned16(x_out))) || (workspace && !aligned16(workspace)))
     return SQ_ERR_ALIGN;
@@ -245,22 +245,33 @@ static sq_status linear_common(const sq_packed_weight* w, const int8_t* xq, cons
   if ((st = check_device(&d)) != SQ_OK) return st;
   const size_t need = linear_workspace_bytes(*w, M, d.sm_count);
   if (!workspace || ws_bytes < need) return SQ_ERR_WORKSPACE;
+  const size_t part = linear_part_bytes(d.sm_count);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (T_out) {
     cudaError_t e = cudaMemsetAsync(T_out, 0, (size_t)M * w->N * sizeof(int32_t), s);
     if (e != cudaSuccess) return SQ_ERR_CUDA;
   }
   const int ng = (int)ceil_div(w->K, w->group_size);
-  for (int t0 = 0; t0 < M; t0 += kMaxTokensPerPass) {
-    const int m = std::min(kMaxTokensPerPass, M - t0);
-    LinearPlan plan;
-    if (!plan_linear(*w, m, n_out, d.sm_count, &plan)) return SQ_ERR_SHAPE;
-    if (plan.smem_bytes > d.smem_optin) return SQ_ERR_SHAPE;
-    cudaError_t e = launch_linear(
-        *w, plan, xq + (int64_t)t0 * w->res_stride, sx + t0, n_out ? x_out + (int64_t)t0 * n_out : nullptr,
-        idx, n_out, y + (int64_t)t0 * w->N, T_out ? T_out + (int64_t)t0 * w->N : nullptr,
-        R_out ? R_out + (int64_t)t0 * w->N * ng : nullptr, workspace, dev_status,
-        (flags & SQ_LAUNCH_PDL) != 0, s);
+  const bool tc = !(flags & SQ_LAUNCH_CUDA_CORES) && linear_tc_supported(*w);
+  const int per_pass = tc ? kMaxTokensPerPassTc : kMaxTokensPerPass;
+  for (int t0 = 0; t0 < M; t0 += per_pass) {
+    const int m = std::min(per_pass, M - t0);
+    const int8_t* xq_t = xq + (int64_t)t0 * w->res_stride;
+    const float* xo_t = n_out ? x_out + (int64_t)t0 * n_out : nullptr;
+    float* y_t = y + (int64_t)t0 * w->N;
+    int32_t* T_t = T_out ? T_out + (int64_t)t0 * w->N : nullptr;
+    int32_t* R_t = R_out ? R_out + (int64_t)t0 * w->N * ng : nullptr;
+    cudaError_t e;
+    if (tc) {
+      e = launch_linear_tc(*w, m, xq_t, sx + t0, xo_t, idx, n_out, y_t, T_t, R_t, workspace, part,
+                           d.sm_count, (flags & SQ_LAUNCH_PDL) != 0, s);
+    } else {
+      LinearPlan plan;
+      if (!plan_linear(*w, m, n_out, d.sm_count, &plan)) return SQ_ERR_SHAPE;
+      if (plan.smem_bytes > d.smem_optin) return SQ_ERR_SHAPE;
+      e = launch_linear(*w, plan, xq_t, sx + t0, xo_t, idx, n_out, y_t, T_t, R_t, workspace, part,
+                        dev_status, (flags & SQ_LAUNCH_PDL) != 0, s);
+    }
     if (e != cudaSuccess) return SQ_ERR_CUDA;
   }
   return SQ_OK;
@@ -277,11 +288,13 @@ sq_status sq_linear(const sq_packed_weight* w, const int8_t* xq, const float* sx
 sq_status sq_linear_accumulators(const sq_packed_weight* w, const int8_t* xq, const float* sx,
                                  const float* x_out, const int32_t* idx, int32_t n_out, int32_t M,
                                  float* y, int32_t* T_out, int32_t* R_out, void* workspace,
-                                 size_t ws_bytes, int32_t* dev_status, void* stream) {
+                                 size_t ws_bytes, int32_t* dev_status, uint32_t flags,
+                                 void* stream) {
   if (!T_out || !R_out) return SQ_ERR_INVALID_ARG;
   if (!aligned16(T_out) || !aligned16(R_out)) return SQ_ERR_ALIGN;
+  if (flags & SQ_LAUNCH_PDL) return SQ_ERR_INVALID_ARG;
   return linear_common(w, xq, sx, x_out, idx, n_out, M, y, T_out, R_out, workspace, ws_bytes,
-                       dev_status, 0u, stream);
+                       dev_status, flags, stream);
 }
 
 }  // extern "C"

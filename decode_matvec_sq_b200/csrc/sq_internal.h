@@ -52,18 +52,30 @@ struct LinearPlan {
   size_t ws_part_bytes = 0;
 };
 
-constexpr int kRowsPerBlock = 8;   // one consumer warp per row of a row block
-constexpr int kMaxTokensPerPass = 4;
+constexpr int kMaxTokensPerPass = 4;     // CUDA-core decode kernel
+constexpr int kMaxTokensPerPassTc = 8;   // tensor-core decode kernel
 constexpr int kMaxOutliers = 4096;
 
 // Plans a decode launch for M tokens (M <= kMaxTokensPerPass) on the current device.
 bool plan_linear(const sq_packed_weight& w, int M, int n_out, int sm_count, LinearPlan* plan);
 
+// Workspace: [partial sums of rows shared by warps: linear_part_bytes()]
+// [one int32 arrival counter per row].  The first area depends only on the
+// device, so one workspace can serve weights of any N and both kernels.
+size_t linear_part_bytes(int sm_count);
 size_t linear_workspace_bytes(const sq_packed_weight& w, int M, int sm_count);
 
 cudaError_t launch_linear(const sq_packed_weight& w, const LinearPlan& plan, const int8_t* xq,
                           const float* sx, const float* x_out, const int32_t* idx, int n_out,
                           float* y, int32_t* T_out, int32_t* R_out, void* workspace,
-                          int32_t* status, bool pdl, cudaStream_t stream);
+                          size_t part_bytes, int32_t* status, bool pdl, cudaStream_t stream);
+
+// Tensor-core decode kernel (group size 128), up to kMaxTokensPerPassTc tokens.
+bool linear_tc_supported(const sq_packed_weight& w);
+size_t linear_tc_part_bytes(int sm_count);
+cudaError_t launch_linear_tc(const sq_packed_weight& w, int M, const int8_t* xq, const float* sx,
+                             const float* x_out, const int32_t* idx, int n_out, float* y,
+                             int32_t* T_out, int32_t* R_out, void* workspace, size_t part_bytes,
+                             int sm_count, bool pdl, cudaStream_t stream);
 
 }  // namespace sq

@@ -14,22 +14,27 @@
 //   y   = sx*(alpha*T + sum_g s_g*R_g) + U
 //
 // Design (B200): the layer moves 1.156 bytes per weight and does a few
-// integer operations per byte, so it is an HBM stream.  Measured on this
-// part, plain 128-bit loads with enough bytes in flight reach ~7.1 TB/s,
-// while a ring of bulk asynchronous copies sustains only about one stage per
-// ~0.55 us per CTA (it needs >= 32 KB stages, too coarse to balance the small
-// layers).  So every lane loads its own weight bytes with LDG.128 straight
-// into a register ring that keeps kDepth 512-channel pieces in flight per
-// warp (~110 KB per SM), the trunk bits are expanded to bytes and dotted with
-// dp4a, the residual codes are dotted with dp4a per 16-channel segment and
-// scaled once per segment, and the outlier channels are taken from the
-// lane's own registers.  Work = 512-channel pieces of the row-major weight,
-// split evenly over all warps of a grid of kBlocksPerSm CTAs per SM; a row
-// shared by two warps is finished by its last contributor from per-warp
-// partials in a fixed order (deterministic, no spin-wait).  With programmatic
-// dependent launch each warp issues its first weight loads before the
-// previous kernel has finished; every other input is read, and every output
-// written, only after it has completed.
+// integer operations per byte, so it is an HBM stream whose instruction
+// budget is tight (~70 warp-instructions per KiB of codes at 7 TB/s).
+// Measured on this part, plain wide loads with enough bytes in flight reach
+// ~7.1 TB/s, while a ring of bulk asynchronous copies into shared memory
+// sustains only about one stage per ~0.55 us per CTA (it needs >= 32 KB
+// stages, too coarse to balance the small layers).  So:
+//   * the weight is cut into 1024-channel pieces of one row; lane l of a warp
+//     owns channels [32l, 32l+32) of a piece: one 256-bit load of codes, one
+//     sign word, one group scale (a lane never spans two groups, G >= 32);
+//   * each warp streams a contiguous range of pieces (split evenly over all
+//     warps) through a register ring of kDepth pieces in flight, pointers
+//     advanced incrementally;
+//   * the trunk bits are expanded four at a time to 0/1 bytes and dotted
+//     with xq by dp4a; the residual codes are dotted by dp4a and scaled once
+//     per lane and piece; sum xq comes precomputed per piece;
+//   * outlier channels are taken from the lane's own registers;
+//   * a row shared by two warps is finished by its last contributor from
+//     per-warp partials, summed in warp order (deterministic, no spin-wait).
+// With programmatic dependent launch each warp issues its first weight loads
+// before the previous kernel has finished; every other input is read, and
+// every output written, only after it has completed.
 #include <stdint.h>
 
 #include <algorithm>
@@ -43,16 +48,14 @@ namespace {
 
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
-// Pieces in flight per warp and CTAs per SM, per tokens per pass: keep
-// ~100+ KB of weight loads in flight per SM without register spills.
-constexpr int kDepth1 = 6, kBps1 = 3;
-constexpr int kDepth2 = 4, kBps2 = 3;
-constexpr int kDepth4 = 4, kBps4 = 2;
-constexpr int kBlocksPerSm = 3;  // the largest of the kBps*
+constexpr int kPiece = 1024;  // channels per piece: 32 per lane
+// Pieces in flight per warp and CTAs per SM, per tokens per pass.
+constexpr int kDepth1 = 5, kBps1 = 2;
+constexpr int kDepth2 = 4, kBps2 = 2;
+constexpr int kDepth4 = 3, kBps4 = 2;
+constexpr int kBlocksPerSm = 2;  // the largest of the kBps*
 
 int blocks_per_sm(int M) { return M == 1 ? kBps1 : (M == 2 ? kBps2 : kBps4); }
-constexpr int kPiece = 512;  // channels per piece: 16 per lane
-constexpr int kMaxPiecesPerRow = (1 << 24) / kPiece;
 
 struct Params {
   const uint32_t* sign;
@@ -61,9 +64,9 @@ struct Params {
   const int8_t* res;
   const float* scale;
   int N, K, K16, log2G, ng, sign_stride, res_stride, scale_stride;
-  int ppr;          // pieces per row = ceil(K16 / 512)
+  int ppr;          // pieces per row = ceil(K16 / 1024)
   int P;            // total pieces = N * ppr (< 2^31)
-  int warps_total;  // gridDim.x * kWarps
+  int warps_total;  // warps that own pieces: min(gridDim.x * kWarps, P); the rest idle
   const int8_t* xq;
   const float* sx;
   const float* xout;
@@ -78,11 +81,12 @@ struct Params {
   int pdl;
 };
 
-// One 512-channel piece as seen by one lane: 16 codes, 16 sign bits (and 16
-// mask bits), the scale of the lane's group.
+// One piece as seen by one lane: 32 codes, 32 sign bits (32 mask bits), the
+// lane's group scale.
 struct Piece {
-  int4 q;
-  uint32_t bm;  // sign bits (low 16) and mask bits (high 16)
+  int q[8];
+  uint32_t b;
+  uint32_t m;
   float s;
 };
 
@@ -94,73 +98,148 @@ __device__ __forceinline__ int piece_owner(int g, const Params& p) {
   return (int)(((int64_t)(g + 1) * p.warps_total + p.P - 1) / p.P) - 1;
 }
 
-template <bool MASK>
-__device__ __forceinline__ void load_piece(Piece& pc, const Params& p, int row, int c, int lane,
-                                           bool live) {
-  const int k = c * kPiece + lane * 16;
-  if (live && k < p.K16) {
-    pc.q = ldg_nc_v4(p.res + (int64_t)row * p.res_stride + k);
-    const uint16_t* sg = reinterpret_cast<const uint16_t*>(p.sign + (int64_t)row * p.sign_stride);
-    pc.bm = __ldg(sg + (k >> 4));
-    if (MASK)
-      pc.bm |= (uint32_t)__ldg(reinterpret_cast<const uint16_t*>(p.mask + (int64_t)row * p.sign_stride) +
-                               (k >> 4)) << 16;
-    pc.s = __ldg(p.scale + (int64_t)row * p.scale_stride + (k >> p.log2G));
+__device__ __forceinline__ void ld32B_v4x2(int* v, const int8_t* p) {
+  const int4 a = ldg_nc_v4(p), b = ldg_nc_v4(p + 16);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+// 32 streamed bytes (read once): 32-byte aligned when V8, else 16.
+template <bool V8>
+__device__ __forceinline__ void ld32B_stream(int* v, const int8_t* p) {
+  if (V8) {
+    asm volatile("ld.global.nc.L1::no_allocate.v8.s32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]),
+                   "=r"(v[6]), "=r"(v[7])
+                 : "l"(p));
   } else {
-    pc.q = make_int4(0, 0, 0, 0);
-    pc.bm = 0;
+    ld32B_v4x2(v, p);
+  }
+}
+
+// 32 bytes of activation codes: reused by every row, so they stay in L1.
+template <bool V8>
+__device__ __forceinline__ void ld32B_cached(int* v, const int8_t* p) {
+  if (V8) {
+    asm volatile("ld.global.nc.v8.s32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]),
+                   "=r"(v[6]), "=r"(v[7])
+                 : "l"(p));
+  } else {
+    ld32B_v4x2(v, p);
+  }
+}
+
+// Streaming position of one lane: row, piece in row, and its pointers.
+struct Cursor {
+  int row, pc;
+  const int8_t* res;
+  const uint32_t* sign;
+  const uint32_t* mask;
+  const float* scale;
+};
+
+__device__ __forceinline__ void cursor_seek(Cursor& c, const Params& p, int row, int pc, int lane) {
+  c.row = row;
+  c.pc = pc;
+  const int k = pc * kPiece + lane * 32;
+  c.res = p.res + (int64_t)row * p.res_stride + k;
+  c.sign = p.sign + (int64_t)row * p.sign_stride + (k >> 5);
+  c.mask = p.mask + (int64_t)row * p.sign_stride + (k >> 5);  // unused without a mask
+  c.scale = p.scale + (int64_t)row * p.scale_stride + (k >> p.log2G);
+}
+
+__device__ __forceinline__ void cursor_next(Cursor& c, const Params& p, int lane) {
+  if (++c.pc == p.ppr) {
+    cursor_seek(c, p, c.row + 1, 0, lane);
+  } else {
+    c.res += kPiece;
+    c.sign += kPiece / 32;
+    c.mask += kPiece / 32;
+    c.scale += kPiece >> p.log2G;
+  }
+}
+
+template <bool MASK, bool V8>
+__device__ __forceinline__ void load_piece(Piece& pc, const Cursor& c, const Params& p, int lane,
+                                           bool live) {
+  const int k = c.pc * kPiece + lane * 32;
+  if (live && k < p.K16) {
+    if (k + 32 <= p.K16) {
+      ld32B_stream<V8>(pc.q, c.res);
+    } else {  // last 16 bytes of a row whose stride is 16 mod 32
+      const int4 a = ldg_nc_v4(c.res);
+      pc.q[0] = a.x; pc.q[1] = a.y; pc.q[2] = a.z; pc.q[3] = a.w;
+      pc.q[4] = pc.q[5] = pc.q[6] = pc.q[7] = 0;
+    }
+    pc.b = __ldg(c.sign);
+    pc.m = MASK ? __ldg(c.mask) : 0xFFFFFFFFu;
+    pc.s = __ldg(c.scale);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) pc.q[i] = 0;
+    pc.b = 0;
+    pc.m = 0;
     pc.s = 0.0f;
   }
 }
 
-template <int M, int D, int BPS, bool MASK, bool EMIT>
+__device__ __forceinline__ int pick_word(const int* q, int w) {
+  // register select (no dynamically indexed local array)
+  const int a = (w & 1) ? q[1] : q[0], b = (w & 1) ? q[3] : q[2];
+  const int c = (w & 1) ? q[5] : q[4], d = (w & 1) ? q[7] : q[6];
+  const int ab = (w & 2) ? b : a, cd = (w & 2) ? d : c;
+  return (w & 4) ? cd : ab;
+}
+
+template <int M, int D, int BPS, bool MASK, bool EMIT, bool V8>
 __global__ void __launch_bounds__(kThreads, BPS) k_linear(const Params p) {
   extern __shared__ __align__(16) uint8_t smem[];
-  // shared layout: Sx[M][ppr] int, omask[roundup(K16/16, 2)] u16 (outlier
-  //                channel bits per 16-channel segment), idx[n_pad] int,
-  //                xo[M][n_pad] f32, sx[M] f32
-  const int nseg = p.K16 >> 4;
-  const int nseg2 = (nseg + 1) & ~1;
+  // shared: Sx[M][ppr] i32 | omask[nw] u32 (outlier bits per 32 channels) |
+  //         obase[nw] i32 (first outlier of the word) | xo[M][n_pad] f32 | sx[M] f32
+  const int nw = (p.K16 + 31) >> 5;
   int* sx_sum = reinterpret_cast<int*>(smem);
-  uint16_t* omask = reinterpret_cast<uint16_t*>(sx_sum + M * p.ppr);
+  uint32_t* omask = reinterpret_cast<uint32_t*>(sx_sum + M * p.ppr);
+  int* obase = reinterpret_cast<int*>(omask + nw);
   const int n_pad = (p.n_out + 3) & ~3;
-  int* idx_s = reinterpret_cast<int*>(omask + nseg2);
-  float* xo_s = reinterpret_cast<float*>(idx_s + n_pad);
+  float* xo_s = reinterpret_cast<float*>(obase + nw);
   float* sx_s = xo_s + M * n_pad;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gw = blockIdx.x * kWarps + warp;
-  const int g0 = warp_begin(gw, p), g1 = warp_begin(gw + 1, p);
+  // every owning warp has >= 1 piece, so the owners of a row are consecutive
+  const int g0 = gw < p.warps_total ? warp_begin(gw, p) : p.P;
+  const int g1 = gw < p.warps_total ? warp_begin(gw + 1, p) : p.P;
 
   // ---- prefetch the first D pieces (weights only; allowed before the wait)
   Piece buf[D];
-  int irow = g0 / p.ppr;
-  int ic = (int)(g0 - irow * p.ppr);
+  Cursor ic;
+  cursor_seek(ic, p, g0 / p.ppr, g0 % p.ppr, lane);
 #pragma unroll
   for (int d = 0; d < D; ++d) {
-    load_piece<MASK>(buf[d], p, irow, ic, lane, g0 + d < g1);
-    if (++ic == p.ppr) {
-      ic = 0;
-      ++irow;
-    }
+    load_piece<MASK, V8>(buf[d], ic, p, lane, g0 + d < g1);
+    if (g0 + d + 1 < g1) cursor_next(ic, p, lane);
   }
 
   if (p.pdl) pdl_wait();
 
   // ---- per-block tables (after the previous kernel completed) -------------
-  for (int i = threadIdx.x; i < nseg2; i += kThreads) omask[i] = 0;
+  for (int i = threadIdx.x; i < nw; i += kThreads) omask[i] = 0u;
   for (int i = threadIdx.x; i < M * p.ppr; i += kThreads) sx_sum[i] = 0;
   __syncthreads();
   for (int i = threadIdx.x; i < p.n_out; i += kThreads) {
     const int j = p.idx[i];
-    idx_s[i] = j;
-    if (j >= 0 && j < p.K) atomicOr(reinterpret_cast<unsigned int*>(omask) + (j >> 5), 1u << (j & 31));
+    if (j >= 0 && j < p.K) {
+      atomicOr(&omask[j >> 5], 1u << (j & 31));
+      // the first outlier of each 32-channel word (the list is ascending)
+      if (i == 0 || (p.idx[i - 1] >> 5) != (j >> 5)) obase[j >> 5] = i;
+    }
 #pragma unroll
     for (int t = 0; t < M; ++t) xo_s[t * n_pad + i] = p.xout[(int64_t)t * p.n_out + i];
   }
   if (threadIdx.x < M) sx_s[threadIdx.x] = p.sx[threadIdx.x];
-  // per-piece sums of xq (for T = 2*P - S without a mask)
-  if (!MASK) {
+  if (!MASK) {  // per-piece sums of xq for T = 2*P - S
+    const int nseg = p.K16 >> 4;
     for (int t = 0; t < M; ++t)
       for (int seg = threadIdx.x; seg < nseg; seg += kThreads) {
         const int4 x = ldg_nc_v4(p.xq + (int64_t)t * p.K16 + seg * 16);
@@ -168,7 +247,7 @@ __global__ void __launch_bounds__(kThreads, BPS) k_linear(const Params p) {
         s = __dp4a(x.y, 0x01010101, s);
         s = __dp4a(x.z, 0x01010101, s);
         s = __dp4a(x.w, 0x01010101, s);
-        atomicAdd(&sx_sum[t * p.ppr + (seg >> 5)], s);
+        atomicAdd(&sx_sum[t * p.ppr + (seg >> 6)], s);
       }
   }
   __syncthreads();
@@ -186,43 +265,57 @@ __global__ void __launch_bounds__(kThreads, BPS) k_linear(const Params p) {
     accUr[t] = 0.0f;
   }
   int crow = g0 / p.ppr;
-  int cc = (int)(g0 - crow * p.ppr);
+  int cc = g0 - crow * p.ppr;
   float row_alpha = (g0 < g1) ? __ldg(p.alpha + crow) : 0.0f;
-  bool row_head = true;  // the current row started inside this warp's range?
-  row_head = (cc == 0);
+  bool row_head = (cc == 0);  // the current row started inside this warp's range
+  const int8_t* xq_lane = p.xq + lane * 32;
 
   for (int g = g0; g < g1; g += D) {
 #pragma unroll
     for (int d = 0; d < D; ++d) {
       if (g + d < g1) {
         Piece& pc = buf[d];
-        const int seg = cc * 32 + lane;  // 16-channel segment index in the row
-        const int k = seg * 16;
+        const int k = cc * kPiece + lane * 32;
         const bool act = k < p.K16;
-        const uint32_t pb_ = pc.bm & 0xFFFFu, pm_ = MASK ? (pc.bm >> 16) : 0xFFFFu;
-        const uint32_t mb = pb_ & pm_;
-        const int e0 = expand_nibble(mb), e1 = expand_nibble(mb >> 4), e2 = expand_nibble(mb >> 8),
-                  e3 = expand_nibble(mb >> 12);
-        int f0 = 0, f1 = 0, f2 = 0, f3 = 0;
-        if (MASK) {
-          f0 = expand_nibble(pm_);
-          f1 = expand_nibble(pm_ >> 4);
-          f2 = expand_nibble(pm_ >> 8);
-          f3 = expand_nibble(pm_ >> 12);
+        const uint32_t mb = pc.b & pc.m;
+        int e[8], f[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          e[i] = expand_nibble(mb >> (4 * i));
+          if (MASK) f[i] = expand_nibble(pc.m >> (4 * i));
         }
 #pragma unroll
         for (int t = 0; t < M; ++t) {
-          int4 x = make_int4(0, 0, 0, 0);
-          if (act) x = ldg_nc_v4(p.xq + (int64_t)t * p.K16 + k);
-          int R = __dp4a(pc.q.x, x.x, 0);
-          R = __dp4a(pc.q.y, x.y, R);
-          R = __dp4a(pc.q.z, x.z, R);
-          R = __dp4a(pc.q.w, x.w, R);
+          int x[8];
+          if (act) {
+            const int8_t* xp = xq_lane + (int64_t)t * p.K16 + cc * kPiece;
+            if (k + 32 <= p.K16) {
+              ld32B_cached<V8>(x, xp);
+            } else {
+              const int4 a = ldg_nc_v4(xp);
+              x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+              x[4] = x[5] = x[6] = x[7] = 0;
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) x[i] = 0;
+          }
+          int R = 0, Pt = accP[t];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            R = __dp4a(pc.q[i], x[i], R);
+            Pt = __dp4a(e[i], x[i], Pt);
+          }
+          accP[t] = Pt;
+          if (MASK) {
+            int St = accS[t];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) St = __dp4a(f[i], x[i], St);
+            accS[t] = St;
+          }
           accF[t] = fmaf(pc.s, (float)R, accF[t]);
-          accP[t] = __dp4a(e0, x.x, __dp4a(e1, x.y, __dp4a(e2, x.z, __dp4a(e3, x.w, accP[t]))));
-          if (MASK) accS[t] = __dp4a(f0, x.x, __dp4a(f1, x.y, __dp4a(f2, x.z, __dp4a(f3, x.w, accS[t]))));
           if (EMIT) {
-            const int sh = p.log2G - 4;  // segments per group = 2^sh
+            const int sh = p.log2G - 5;  // lanes per group = 2^sh
             for (int o = 1; o < (1 << sh); o <<= 1) R += __shfl_xor_sync(0xffffffffu, R, o);
             if (act && (lane & ((1 << sh) - 1)) == 0)
               p.R_out[((int64_t)t * p.N + crow) * p.ng + (k >> p.log2G)] = R;
@@ -232,54 +325,44 @@ __global__ void __launch_bounds__(kThreads, BPS) k_linear(const Params p) {
 #pragma unroll
           for (int t = 0; t < M; ++t) accS[t] += sx_sum[t * p.ppr + cc];
         }
-        // outlier channels among this lane's 16
-        uint32_t om = act ? omask[seg] : 0u;
+        // outlier channels among this lane's 32
+        uint32_t om = act ? omask[k >> 5] : 0u;
         if (om) {
-          // position of the segment's first outlier in the ascending list
-          int pos = 0, hi = p.n_out;
-          while (pos < hi) {
-            const int mid = (pos + hi) >> 1;
-            if (idx_s[mid] < k)
-              pos = mid + 1;
-            else
-              hi = mid;
-          }
+          int pos = obase[k >> 5];
           do {
             const int bit = __ffs(om) - 1;
             om &= om - 1;
-            const int wsel = bit >> 2;
-            const int word = wsel == 0 ? pc.q.x : (wsel == 1 ? pc.q.y : (wsel == 2 ? pc.q.z : pc.q.w));
-            const int qv = (int)(int8_t)(word >> (8 * (bit & 3)));
-            const bool in_trunk = MASK ? ((pm_ >> bit) & 1u) : true;
-            const float sgn = ((pb_ >> bit) & 1u) ? 1.0f : -1.0f;
+            const int qv = (int)(int8_t)(pick_word(pc.q, bit >> 2) >> (8 * (bit & 3)));
+            const bool in_trunk = (pc.m >> bit) & 1u;
+            const float sgn = ((pc.b >> bit) & 1u) ? 1.0f : -1.0f;
             const float rq = pc.s * (float)qv;
+            // (an index list that is not strictly ascending cannot push pos
+            // past the staged values)
+            if (pos >= 0 && pos < p.n_out) {
 #pragma unroll
-            for (int t = 0; t < M; ++t) {
-              // (an index list that is not strictly ascending cannot push
-              // pos past the staged values)
-              const float xv = pos < p.n_out ? xo_s[t * n_pad + pos] : 0.0f;
-              if (in_trunk) accUt[t] = fmaf(sgn, xv, accUt[t]);
-              accUr[t] = fmaf(rq, xv, accUr[t]);
+              for (int t = 0; t < M; ++t) {
+                const float xv = xo_s[t * n_pad + pos];
+                if (in_trunk) accUt[t] = fmaf(sgn, xv, accUt[t]);
+                accUr[t] = fmaf(rq, xv, accUr[t]);
+              }
             }
             ++pos;
           } while (om);
         }
 
         // refill this slot with the piece D ahead
-        load_piece<MASK>(buf[d], p, irow, ic, lane, g + d + D < g1);
-        if (++ic == p.ppr) {
-          ic = 0;
-          ++irow;
-        }
+        const bool live = g + d + D < g1;
+        load_piece<MASK, V8>(buf[d], ic, p, lane, live);
+        if (live) cursor_next(ic, p, lane);
 
         // end of a row, or end of this warp's range
-        const bool row_end = (cc == p.ppr - 1) || (g + d + 1 == g1);
-        if (row_end) {
+        if (cc == p.ppr - 1 || g + d + 1 == g1) {
 #pragma unroll
           for (int t = 0; t < M; ++t) {
+#pragma unroll
             for (int o = 16; o > 0; o >>= 1) {
               accP[t] += __shfl_xor_sync(0xffffffffu, accP[t], o);
-              accS[t] += __shfl_xor_sync(0xffffffffu, accS[t], o);
+              if (MASK) accS[t] += __shfl_xor_sync(0xffffffffu, accS[t], o);
               accF[t] += __shfl_xor_sync(0xffffffffu, accF[t], o);
               accUt[t] += __shfl_xor_sync(0xffffffffu, accUt[t], o);
               accUr[t] += __shfl_xor_sync(0xffffffffu, accUr[t], o);
@@ -292,8 +375,7 @@ __global__ void __launch_bounds__(kThreads, BPS) k_linear(const Params p) {
               T[t] = 2 * accP[t] - accS[t];
               if (EMIT) atomicAdd(&p.T_out[(int64_t)t * p.N + crow], T[t]);
             }
-            const bool whole = row_head && cc == p.ppr - 1;
-            if (whole) {
+            if (row_head && cc == p.ppr - 1) {
 #pragma unroll
               for (int t = 0; t < M; ++t) {
                 const float inner = fmaf(row_alpha, (float)T[t], accF[t]);
@@ -371,9 +453,9 @@ __global__ void __launch_bounds__(kThreads, BPS) k_linear(const Params p) {
   }
 }
 
-template <int M, int D, int BPS, bool MASK, bool EMIT>
+template <int M, int D, int BPS, bool MASK, bool EMIT, bool V8>
 cudaError_t launch_one(const Params& p, const LinearPlan& plan, bool pdl, cudaStream_t stream) {
-  auto* fn = k_linear<M, D, BPS, MASK, EMIT>;
+  auto* fn = k_linear<M, D, BPS, MASK, EMIT, V8>;
   cudaError_t e = ensure_smem_attr((const void*)fn, plan.smem_bytes);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -389,15 +471,22 @@ cudaError_t launch_one(const Params& p, const LinearPlan& plan, bool pdl, cudaSt
   return cudaLaunchKernelEx(&cfg, fn, p);
 }
 
-template <bool MASK, bool EMIT>
+template <bool MASK, bool EMIT, bool V8>
 cudaError_t dispatch_m(int M, const Params& p, const LinearPlan& plan, bool pdl, cudaStream_t st) {
   switch (M) {
-    case 1: return launch_one<1, kDepth1, kBps1, MASK, EMIT>(p, plan, pdl, st);
-    case 2: return launch_one<2, kDepth2, kBps2, MASK, EMIT>(p, plan, pdl, st);
-    case 3: return launch_one<3, kDepth4, kBps4, MASK, EMIT>(p, plan, pdl, st);
-    case 4: return launch_one<4, kDepth4, kBps4, MASK, EMIT>(p, plan, pdl, st);
+    case 1: return launch_one<1, kDepth1, kBps1, MASK, EMIT, V8>(p, plan, pdl, st);
+    case 2: return launch_one<2, kDepth2, kBps2, MASK, EMIT, V8>(p, plan, pdl, st);
+    case 3: return launch_one<3, kDepth4, kBps4, MASK, EMIT, V8>(p, plan, pdl, st);
+    case 4: return launch_one<4, kDepth4, kBps4, MASK, EMIT, V8>(p, plan, pdl, st);
     default: return cudaErrorInvalidValue;
   }
+}
+
+template <bool MASK, bool EMIT>
+cudaError_t dispatch_v8(bool v8, int M, const Params& p, const LinearPlan& plan, bool pdl,
+                        cudaStream_t st) {
+  return v8 ? dispatch_m<MASK, EMIT, true>(M, p, plan, pdl, st)
+            : dispatch_m<MASK, EMIT, false>(M, p, plan, pdl, st);
 }
 
 int log2_exact(int v) {
@@ -414,28 +503,28 @@ bool plan_linear(const sq_packed_weight& w, int M, int n_out, int sm_count, Line
   pl.M = M;
   const int64_t K16 = round_up(w.K, 16);
   const int64_t ppr = ceil_div(K16, kPiece);
-  if (ppr > kMaxPiecesPerRow) return false;
   const int64_t P = (int64_t)w.N * ppr;
   if (P >= INT32_MAX) return false;
-  // at least ~4 pieces per warp, at most kBlocksPerSm CTAs per SM
+  // about two pieces per warp at least, at most blocks_per_sm(M) CTAs per SM
   const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((int64_t)sm_count * blocks_per_sm(M),
-                                                                ceil_div(P, 4 * kWarps)));
+                                                                ceil_div(P, 2 * kWarps)));
   pl.grid = (int)blocks;
   pl.Kc = kPiece;
   pl.n_c = (int)ppr;
-  pl.U = (int)std::min<int64_t>(P, INT32_MAX);
-  const int nseg = (int)(K16 / 16);
-  const int n_pad = (int)round_up(n_out, 4);
-  size_t smem = (size_t)M * ppr * 4 + (size_t)round_up(nseg, 2) * 2 + (size_t)n_pad * 4 +
-                (size_t)M * n_pad * 4 + (size_t)M * 4 + 16;
-  pl.smem_bytes = (int)round_up((int64_t)smem, 16);
-  // workspace: [partial sums, sized for the largest grid on this device]
-  //            [per-row arrival counters]; the first area does not depend on
-  //            the weight, so one workspace can serve weights of any N
-  pl.ws_part_bytes = (size_t)sm_count * kBlocksPerSm * kWarps * 2 * kMaxTokensPerPass * 4 * sizeof(float);
+  pl.U = (int)P;
+  const int64_t nw = ceil_div(K16, 32);
+  const int64_t n_pad = round_up(n_out, 4);
+  const int64_t smem = (int64_t)M * ppr * 4 + nw * 4 + nw * 4 + (int64_t)M * n_pad * 4 + M * 4 + 16;
+  pl.smem_bytes = (int)round_up(smem, 16);
+  pl.ws_part_bytes = linear_part_bytes(sm_count);
   pl.ws_cnt_bytes = (size_t)round_up((int64_t)w.N * 4, 256);
   *plan = pl;
   return true;
+}
+
+size_t linear_part_bytes(int sm_count) {
+  const size_t core = (size_t)sm_count * kBlocksPerSm * kWarps * 2 * kMaxTokensPerPass * 4 * sizeof(float);
+  return (size_t)round_up((int64_t)std::max(core, linear_tc_part_bytes(sm_count)), 256);
 }
 
 size_t linear_workspace_bytes(const sq_packed_weight& w, int M, int sm_count) {
@@ -447,7 +536,7 @@ size_t linear_workspace_bytes(const sq_packed_weight& w, int M, int sm_count) {
 cudaError_t launch_linear(const sq_packed_weight& w, const LinearPlan& plan, const int8_t* xq,
                           const float* sx, const float* x_out, const int32_t* idx, int n_out,
                           float* y, int32_t* T_out, int32_t* R_out, void* workspace,
-                          int32_t* status, bool pdl, cudaStream_t stream) {
+                          size_t part_bytes, int32_t* status, bool pdl, cudaStream_t stream) {
   Params p;
   p.sign = w.sign_bits;
   p.mask = w.mask_bits;
@@ -464,7 +553,7 @@ cudaError_t launch_linear(const sq_packed_weight& w, const LinearPlan& plan, con
   p.scale_stride = w.scale_stride;
   p.ppr = plan.n_c;
   p.P = w.N * plan.n_c;
-  p.warps_total = plan.grid * kWarps;
+  p.warps_total = std::min(plan.grid * kWarps, p.P);
   p.xq = xq;
   p.sx = sx;
   p.xout = x_out;
@@ -474,16 +563,19 @@ cudaError_t launch_linear(const sq_packed_weight& w, const LinearPlan& plan, con
   p.T_out = T_out;
   p.R_out = R_out;
   p.ws_part = reinterpret_cast<float*>(workspace);
-  p.ws_cnt = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(workspace) + plan.ws_part_bytes);
+  p.ws_cnt = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(workspace) + part_bytes);
   p.status = status;
   p.pdl = pdl ? 1 : 0;
+  // 256-bit loads need 32-byte aligned rows of codes and of activation codes
+  const bool v8 = (w.res_stride % 32) == 0 && (reinterpret_cast<uintptr_t>(w.res_q) % 32) == 0 &&
+                  (reinterpret_cast<uintptr_t>(xq) % 32) == 0;
   const bool mask = w.mask_bits != nullptr;
   const bool emit = T_out != nullptr;
   if (mask)
-    return emit ? dispatch_m<true, true>(plan.M, p, plan, pdl, stream)
-                : dispatch_m<true, false>(plan.M, p, plan, pdl, stream);
-  return emit ? dispatch_m<false, true>(plan.M, p, plan, pdl, stream)
-              : dispatch_m<false, false>(plan.M, p, plan, pdl, stream);
+    return emit ? dispatch_v8<true, true>(v8, plan.M, p, plan, pdl, stream)
+                : dispatch_v8<true, false>(v8, plan.M, p, plan, pdl, stream);
+  return emit ? dispatch_v8<false, true>(v8, plan.M, p, plan, pdl, stream)
+              : dispatch_v8<false, false>(v8, plan.M, p, plan, pdl, stream);
 }
 
 }  // namespace sq

@@ -59,6 +59,10 @@ typedef enum {
  * streaming the packed weights at once; it reads every other input and writes
  * every output only after the previous kernel has completed.  Set it only if
  * no earlier work still in flight on the stream writes the packed weights. */
+#define SQ_LAUNCH_CUDA_CORES 2u
+/* SQ_LAUNCH_CUDA_CORES (sq_linear only): run the CUDA-core kernel (dp4a)
+ * instead of the tensor-core kernel; same results.  The CUDA-core kernel is
+ * also the one used for group sizes 32 and 64. */
 
 /*
  * Packed weight of one linear layer (N output rows, K input channels).
@@ -140,13 +144,12 @@ sq_status sq_calibrate_outliers(const float *X, int32_t T, int32_t K, int32_t k,
 /*
  * Per-token activation split (m.lqnn.cn section 2.2; dynamic per-token scale
  * of the visual guide's "动态量化" section).
- *   x      [M][K] f32 activations, device
- *   idx    [n_out] i32 outlier channels, strictly ascending in [0, K)
- *          (host-checked only for n_out; the caller guarantees the order,
- *          as produced by sq_calibrate_outliers)
- *   xq     [M][roundup(K,16)] i8 out: codes, 0 on outlier channels and pads
- *   sx     [M] f32 out: absmax over the non-outlier channels / 127
- *   x_out  [M][n_out] f32 out: the outlier channels, copied
+ *   x          [M][K] f32 activations, device
+ *   idx        [n_out] i32 outlier channels, strictly ascending in [0, K)
+ *              (checked on the device: a violation sets SQ_ERR_INVALID_ARG)
+ *   xq         [M][roundup(K,16)] i8 out: codes, 0 on outlier channels and pads
+ *   sx         [M] f32 out: absmax over the non-outlier channels / 127
+ *   x_out      [M][n_out] f32 out: the outlier channels, copied
  * 0 <= n_out <= 4096.  Non-finite x sets SQ_ERR_NONFINITE.
  */
 sq_status sq_quantize_act(const float *x, int32_t M, int32_t K, const int32_t *idx,
@@ -168,7 +171,12 @@ size_t sq_linear_workspace_bytes(const sq_packed_weight *w, int32_t M);
  * kernel; the outlier channels of section 2.2 at full precision).
  *   w           packed weight (device arrays)
  *   xq, sx, x_out, idx, n_out   as written by sq_quantize_act
- *   M           tokens, 1 <= M; the decode kernel takes M <= 16 per pass
+ *   M           tokens, M >= 1.  Group size 128 runs on the tensor cores
+ *               (INT8 MMAs for the residual codes and for the trunk bits
+ *               expanded to 0/1 bytes), in passes of up to 8 tokens; group
+ *               sizes 32 and 64, or SQ_LAUNCH_CUDA_CORES, run on the CUDA
+ *               cores (dp4a), in passes of up to 4 tokens.  The results are
+ *               the same.
  *   y           [M][N] f32 out
  *   workspace   device, ws_bytes >= sq_linear_workspace_bytes(w, M)
  * For every token t and row r:
@@ -178,21 +186,22 @@ size_t sq_linear_workspace_bytes(const sq_packed_weight *w, int32_t M);
  * with What = m*(+-alpha) + s_g*q the dequantized weight, in fp32.
  */
 sq_status sq_linear(const sq_packed_weight *w, const int8_t *xq, const float *sx,
-                    const float *x_out, const int32_t *idx, int32_t n_out, int32_t M,
-                    float *y, void *workspace, size_t ws_bytes, int32_t *dev_status,
-                    uint32_t flags, void *stream);
+                    const float *x_out, const int32_t *idx, int32_t n_out, int32_t M, float *y,
+                    void *workspace, size_t ws_bytes, int32_t *dev_status, uint32_t flags,
+                    void *stream);
 
 /*
- * Same kernel as sq_linear, additionally writing its exact integer
+ * Same kernels as sq_linear, additionally writing the exact integer
  * accumulators for inspection:
  *   T_out [M][N] i32, R_out [M][N][ceil(K/G)] i32.
- * y is written as by sq_linear.  Intended for tests; not on the hot path.
+ * y is written as by sq_linear.  flags: 0 or SQ_LAUNCH_CUDA_CORES.  Intended
+ * for tests; not on the hot path.
  */
-sq_status sq_linear_accumulators(const sq_packed_weight *w, const int8_t *xq,
-                                 const float *sx, const float *x_out, const int32_t *idx,
-                                 int32_t n_out, int32_t M, float *y, int32_t *T_out,
-                                 int32_t *R_out, void *workspace, size_t ws_bytes,
-                                 int32_t *dev_status, void *stream);
+sq_status sq_linear_accumulators(const sq_packed_weight *w, const int8_t *xq, const float *sx,
+                                 const float *x_out, const int32_t *idx, int32_t n_out,
+                                 int32_t M, float *y, int32_t *T_out, int32_t *R_out,
+                                 void *workspace, size_t ws_bytes, int32_t *dev_status,
+                                 uint32_t flags, void *stream);
 
 #ifdef __cplusplus
 }

@@ -87,6 +87,7 @@ def test_host_validation_before_device_work(L):
     L.sq_packed_view(ctypes.c_void_p(1 << 40), 64, 256, 128, 0, ctypes.byref(v))
     p = ctypes.c_void_p(1 << 41)
     bad = ctypes.c_void_p((1 << 41) + 4)
+    # sq_linear(w, xq, sx, x_out, idx, n_out, M, y, ws, ws_bytes, status, flags, stream)
     assert L.sq_linear(None, p, p, p, p, 1, 1, p, p, 1 << 20, None, 0, None) == 1
     assert L.sq_linear(ctypes.byref(v), None, p, p, p, 1, 1, p, p, 1 << 20, None, 0, None) == 1
     assert L.sq_linear(ctypes.byref(v), p, p, p, p, 1, 0, p, p, 1 << 20, None, 0, None) == 2
@@ -96,12 +97,17 @@ def test_host_validation_before_device_work(L):
     w2 = sq.SqPackedWeight.from_buffer_copy(v)
     w2.res_stride = 100
     assert L.sq_linear(ctypes.byref(w2), p, p, p, p, 1, 1, p, p, 1 << 20, None, 0, None) == 2
+    # accumulators: PDL is not accepted
+    assert L.sq_linear_accumulators(ctypes.byref(v), p, p, p, p, 1, 1, p, p, p, p, 1 << 20, None,
+                                    1, None) == 1
     assert L.sq_decompose_pack(None, 64, 256, -1, ctypes.byref(v), None, None) == 1
     assert L.sq_decompose_pack(p, 64, 256, 0, ctypes.byref(v), None, None) == 1
     assert L.sq_decompose_pack(p, 64, 256, 60, ctypes.byref(v), None, None) == 1  # no mask array
     assert L.sq_decompose_pack(p, 65, 256, -1, ctypes.byref(v), None, None) == 2
+    # sq_quantize_act(x, M, K, idx, n_out, xq, sx, x_out, status, flags, stream)
     assert L.sq_quantize_act(p, 1, 256, p, -1, p, p, p, None, 0, None) == 2
     assert L.sq_quantize_act(p, 1, 256, None, 3, p, p, p, None, 0, None) == 1
+    assert L.sq_quantize_act(p, 1, 256, p, 3, bad, p, p, None, 0, None) == 3
     assert L.sq_calibrate_outliers(p, 64, 256, 0, p, None, None) == 2
     assert L.sq_calibrate_outliers(p, 64, 256, 300, p, None, None) == 2
 

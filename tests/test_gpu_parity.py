@@ -67,21 +67,23 @@ def check_y(y, y_ref, bound, what="y"):
                      f"{float((err / np.maximum(bound, 1e-300)).max()):.3e}"
 
 
-def run_path(W: np.ndarray, x: np.ndarray, idx: np.ndarray, P=-1, G=128, pdl=False):
+def run_path(W: np.ndarray, x: np.ndarray, idx: np.ndarray, P=-1, G=128, pdl=False, tc=True):
     Wd = torch.from_numpy(W).cuda()
     xd = torch.from_numpy(x).cuda()
     idxd = torch.from_numpy(idx.astype(np.int32)).cuda()
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     pw = sq.decompose_pack(Wd, trunk_percent=P, group_size=G, status=status)
-    xq, sx, xo = sq.quantize_act(xd, idxd, status=status, pdl=pdl)
-    y, T, R = sq.linear_accumulators(pw, xq, sx, xo, idxd, status=status)
+    act = sq.quantize_act(xd, idxd, status=status, pdl=pdl)
+    xq, sx, xo = act
+    y, T, R = sq.linear_accumulators(pw, xq, sx, xo, idxd, status=status, cuda_cores=not tc)
     torch.cuda.synchronize()
     assert status.item() == 0
-    return pw, (xq, sx, xo), (y, T, R)
+    return pw, act, (y, T, R)
 
 
-def full_compare(W, x, idx, P=-1, G=128):
-    pw, (xq, sx, xo), (y, T, R) = run_path(W, x, idx, P, G)
+def full_compare(W, x, idx, P=-1, G=128, tc=True):
+    pw, act, (y, T, R) = run_path(W, x, idx, P, G, tc=tc)
+    xq, sx, xo = act
     d = oracle.decompose(W, G=G, P=P)
     check_packed(pw, d)
     oxq, osx, oxo = oracle.quantize_act(x, idx)
@@ -199,6 +201,18 @@ def test_quantize_act_parity(M, K, n):
         assert np.array_equal(xo.cpu().numpy(), oxo)
 
 
+def test_quantize_act_large_k():
+    """K beyond the range the kernel keeps in registers (re-read path)."""
+    rng = np.random.default_rng(12)
+    K = 40000
+    x = rng.standard_normal((2, K)).astype(np.float32)
+    idx = np.sort(rng.choice(K, 50, replace=False)).astype(np.int32)
+    act = sq.quantize_act(torch.from_numpy(x).cuda(), torch.from_numpy(idx).cuda())
+    torch.cuda.synchronize()
+    oxq, osx, _ = oracle.quantize_act(x, idx)
+    assert np.array_equal(act[0].cpu().numpy()[:, :K], oxq)
+
+
 def test_quantize_act_random_midpoints():
     """Values on exact half-steps of many different scales."""
     rng = np.random.default_rng(4)
@@ -220,16 +234,17 @@ def test_quantize_act_random_midpoints():
 
 @pytest.mark.parametrize("N,K,M,n", [(1, 8, 1, 0), (7, 33, 1, 2), (8, 100, 2, 3), (513, 300, 1, 6),
                                      (64, 512, 3, 4), (16, 4096, 4, 20), (33, 1000, 5, 9),
-                                     (40, 129, 8, 1), (24, 11008, 1, 55), (8, 28672, 1, 72),
+                                     (40, 129, 8, 1), (20, 300, 8, 3), (24, 11008, 1, 55), (8, 28672, 1, 72),
                                      (100, 2048, 16, 10)])
 @pytest.mark.parametrize("P", [-1, 60])
-def test_linear_parity_small(N, K, M, n, P):
+@pytest.mark.parametrize("tc", [False, True])
+def test_linear_parity_small(N, K, M, n, P, tc):
     rng = np.random.default_rng(N + K + M + n + P)
     W = rng.laplace(0, 0.02, (N, K)).astype(np.float32)
     x = rng.standard_normal((M, K)).astype(np.float32)
     idx = np.sort(rng.choice(K, n, replace=False)).astype(np.int32)
     x[:, idx] *= 30.0
-    full_compare(W, x, idx, P=P)
+    full_compare(W, x, idx, P=P, tc=tc)
 
 
 @pytest.mark.parametrize("G", [32, 64])
@@ -241,33 +256,37 @@ def test_linear_parity_group_sizes(G):
     full_compare(W, x, idx, G=G)
 
 
-def test_linear_degenerate():
+@pytest.mark.parametrize("tc", [False, True])
+def test_linear_degenerate(tc):
     rng = np.random.default_rng(0)
     W = np.zeros((9, 64), np.float32)
     x = rng.standard_normal((1, 64)).astype(np.float32)
-    full_compare(W, x, np.array([3], np.int32))          # zero weights: y = 0
+    full_compare(W, x, np.array([3], np.int32), tc=tc)          # zero weights: y = 0
     W = rng.laplace(0, 0.02, (9, 64)).astype(np.float32)
-    full_compare(W, np.zeros((2, 64), np.float32), np.array([3], np.int32))  # zero tokens
+    full_compare(W, np.zeros((2, 64), np.float32), np.array([3], np.int32), tc=tc)  # zero tokens
     x = np.zeros((1, 64), np.float32)
     x[0, 3] = 7.0                                         # only the outlier channel is live
-    full_compare(W, x, np.array([3], np.int32))
-    full_compare(W[:1, :1], np.ones((1, 1), np.float32), np.zeros(0, np.int32))
+    full_compare(W, x, np.array([3], np.int32), tc=tc)
+    full_compare(W[:1, :1], np.ones((1, 1), np.float32), np.zeros(0, np.int32), tc=tc)
 
 
-def test_linear_deterministic_and_split_rows():
-    """N=8, K=28672: one 8-row block split over 14 CTAs (stream of partials)."""
+@pytest.mark.parametrize("tc", [False, True])
+def test_linear_deterministic_and_split_rows(tc):
+    """N=8, K=28672: one row block split over many warps (partials + fixup)."""
     rng = np.random.default_rng(1)
     W = rng.laplace(0, 0.02, (8, 28672)).astype(np.float32)
     x = rng.standard_normal((1, 28672)).astype(np.float32)
     idx = np.sort(rng.choice(28672, 72, replace=False)).astype(np.int32)
     Wd, xd, idxd = (torch.from_numpy(a).cuda() for a in (W, x, idx))
     pw = sq.decompose_pack(Wd)
-    xq, sx, xo = sq.quantize_act(xd, idxd)
+    act = sq.quantize_act(xd, idxd)
+    xq, sx, xo = act
     ws = sq.new_workspace(pw, 1)
     ys = []
     for _ in range(5):
         y = torch.full((1, 8), float("nan"), device="cuda")
-        ys.append(sq.linear(pw, xq, sx, xo, idxd, y=y, workspace=ws).cpu().numpy())
+        ys.append(sq.linear(pw, xq, sx, xo, idxd, y=y, workspace=ws,
+                            cuda_cores=not tc).cpu().numpy())
     torch.cuda.synchronize()
     for y in ys[1:]:
         assert np.array_equal(y.view(np.uint32), ys[0].view(np.uint32))
@@ -304,7 +323,8 @@ def test_linear_errors():
 
 # ---- the five workloads ------------------------------------------------------------
 
-def test_config1_full_pipeline():
+@pytest.mark.parametrize("tc", [False, True])
+def test_config1_full_pipeline(tc):
     """512 x 512, batch 1, top-4 calibrated outliers: every output element."""
     L = wl.config1()
     X = torch.from_numpy(L.calibration()).cuda()
@@ -312,17 +332,18 @@ def test_config1_full_pipeline():
     W, x = L.weights(), L.activations()
     torch.cuda.synchronize()
     assert np.array_equal(idx.cpu().numpy(), L.planted_channels())
-    full_compare(W, x, idx.cpu().numpy())
+    full_compare(W, x, idx.cpu().numpy(), tc=tc)
 
 
-def test_config4_threshold_full():
+@pytest.mark.parametrize("tc", [False, True])
+def test_config4_threshold_full(tc):
     """4096 -> 14336 threshold trunk (per-row 60th percentile), batch 1, every row."""
     L = wl.config4()
     W, x, idx = L.weights(), L.activations(), L.planted_channels()
-    full_compare(W, x, idx, P=L.trunk_percent)
+    full_compare(W, x, idx, P=L.trunk_percent, tc=tc)
 
 
-def _sampled_layer(L, M, rows, pdl=False):
+def _sampled_layer(L, M, rows, pdl=False, tc=True):
     """Full-size layer generated on the device; oracle on sampled rows."""
     Wd = sdev.fill_weights(L, torch.empty(L.N, L.K, device="cuda"))
     Xc = sdev.fill_activations(L, torch.empty(wl.CAL_TOKENS, L.K, device="cuda"), synth.STREAM_XCAL)
@@ -332,9 +353,9 @@ def _sampled_layer(L, M, rows, pdl=False):
     del Wd
     idx = sq.calibrate_outliers(Xc, L.n_out, status=st)
     xq, sx, xo = sq.quantize_act(xd, idx, status=st, pdl=pdl)
-    y, T, R = sq.linear_accumulators(pw, xq, sx, xo, idx, status=st)
+    y, T, R = sq.linear_accumulators(pw, xq, sx, xo, idx, status=st, cuda_cores=not tc)
     y2 = torch.full_like(y, float("nan"))
-    sq.linear(pw, xq, sx, xo, idx, y=y2, status=st, pdl=pdl)
+    sq.linear(pw, xq, sx, xo, idx, y=y2, status=st, pdl=pdl, cuda_cores=not tc)
     torch.cuda.synchronize()
     assert st.item() == 0
     assert torch.equal(y, y2)
@@ -361,16 +382,18 @@ def _rows(N, n=96, seed=0):
 
 @pytest.mark.parametrize("M", [1, 2, 4, 8, 16])
 @pytest.mark.parametrize("which", [0, 1])
-def test_config3_batch_sweep_sampled(M, which):
+@pytest.mark.parametrize("tc", [False, True])
+def test_config3_batch_sweep_sampled(M, which, tc):
     L = wl.config3(M)[which]
-    _sampled_layer(L, M, _rows(L.N, seed=M + which))
+    _sampled_layer(L, M, _rows(L.N, seed=M + which), tc=tc)
 
 
 @pytest.mark.parametrize("layer", [0, 31])
 @pytest.mark.parametrize("mid", [0, 1, 2, 3])
-def test_config2_stack_layers_sampled(layer, mid):
+@pytest.mark.parametrize("tc", [False, True])
+def test_config2_stack_layers_sampled(layer, mid, tc):
     L = wl.config2_layer(layer, mid)
-    _sampled_layer(L, 1, _rows(L.N, seed=layer * 4 + mid), pdl=True)
+    _sampled_layer(L, 1, _rows(L.N, seed=layer * 4 + mid), pdl=True, tc=tc)
 
 
 # ---- launch modes ----------------------------------------------------------------
@@ -387,17 +410,17 @@ def test_pdl_chain_in_cuda_graph_matches_plain():
     ws = sq.new_workspace(max(pws, key=lambda p: p.N), 1)
     bufs = [sq.quantize_act(x, i) for x, i in zip(xs, idxs)]
     ys = [torch.empty(1, p.N, device="cuda") for p in pws]
-    for p, (xq, sx, xo), i, y in zip(pws, bufs, idxs, ys):
+    for p, a, i, y in zip(pws, bufs, idxs, ys):
         y.fill_(float("nan"))
-        ys_plain.append(sq.linear(p, xq, sx, xo, i, y=y, workspace=ws).clone())
+        ys_plain.append(sq.linear(p, a[0], a[1], a[2], i, y=y, workspace=ws).clone())
     torch.cuda.synchronize()
     g = torch.cuda.CUDAGraph()
     s = torch.cuda.Stream()
     with torch.cuda.stream(s):
         with torch.cuda.graph(g, stream=s):
-            for p, x, i, (xq, sx, xo), y in zip(pws, xs, idxs, bufs, ys):
-                sq.quantize_act(x, i, xq=xq, sx=sx, x_out=xo, pdl=True)
-                sq.linear(p, xq, sx, xo, i, y=y, workspace=ws, pdl=True)
+            for p, x, i, a, y in zip(pws, xs, idxs, bufs, ys):
+                sq.quantize_act(x, i, xq=a[0], sx=a[1], x_out=a[2], pdl=True)
+                sq.linear(p, a[0], a[1], a[2], i, y=y, workspace=ws, pdl=True)
     for _ in range(3):
         for y in ys:
             y.fill_(float("nan"))
@@ -409,7 +432,8 @@ def test_pdl_chain_in_cuda_graph_matches_plain():
         assert not sq.workspace_counters(ws, p).any().item()
 
 
-def test_shared_workspace_across_shapes():
+@pytest.mark.parametrize("tc", [False, True])
+def test_shared_workspace_across_shapes(tc):
     """One workspace serving layers of different N, called in interleaved
     order: every row is written every time and matches the oracle."""
     layers = [wl.config2_layer(1, m) for m in (0, 2, 1, 3)] + [wl.config1()]
@@ -426,9 +450,10 @@ def test_shared_workspace_across_shapes():
                      device="cuda")
     outs = {}
     for rep in range(3):
-        for L, pw, idx, (xq, sx, xo) in items[::(1 if rep % 2 == 0 else -1)]:
+        for L, pw, idx, a in items[::(1 if rep % 2 == 0 else -1)]:
             y = torch.full((1, L.N), float("nan"), device="cuda")
-            sq.linear(pw, xq, sx, xo, idx, y=y, workspace=ws, status=st)
+            sq.linear(pw, a[0], a[1], a[2], idx, y=y, workspace=ws, status=st,
+                      cuda_cores=not tc)
             torch.cuda.synchronize()
             assert not torch.isnan(y).any().item(), f"{L.name}: rows not written"
             if L.name in outs:
@@ -444,3 +469,25 @@ def test_shared_workspace_across_shapes():
         y_ref = oracle.linear(d, oxq, osx, oxo, L.planted_channels())
         check_y(outs[L.name][:, torch.as_tensor(rows, device="cuda")].cpu().numpy(), y_ref,
                 oracle.abs_dot(Wr, x), L.name)
+
+
+@pytest.mark.parametrize("tc", [False, True])
+@pytest.mark.parametrize("N,K", [(16, 129), (40, 256), (3, 3000), (17, 2048)])
+def test_fewer_work_units_than_warps(N, K, tc):
+    """Tiny layers: more warps than units of work; rows split between warps
+    must still be finished on every call (two calls in a row, NaN-prefilled)."""
+    rng = np.random.default_rng(N * K)
+    W = rng.laplace(0, 0.02, (N, K)).astype(np.float32)
+    x = rng.standard_normal((2, K)).astype(np.float32)
+    pw = sq.decompose_pack(torch.from_numpy(W).cuda())
+    act = sq.quantize_act(torch.from_numpy(x).cuda(), None)
+    ws = sq.new_workspace(pw, 2)
+    d = oracle.decompose(W)
+    oxq, osx, oxo = oracle.quantize_act(x, np.zeros(0, np.int32))
+    y_ref = oracle.linear(d, oxq, osx, oxo, np.zeros(0, np.int32))
+    for _ in range(2):
+        y = torch.full((2, N), float("nan"), device="cuda")
+        sq.linear(pw, act[0], act[1], act[2], None, y=y, workspace=ws, cuda_cores=not tc)
+        torch.cuda.synchronize()
+        check_y(y.cpu().numpy(), y_ref, oracle.abs_dot(W, x))
+        assert not sq.workspace_counters(ws, pw, 2).any().item()
