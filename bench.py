@@ -149,6 +149,24 @@ def dist_setup():
     return world, rank, local
 
 
+def barrier(world: int) -> None:
+    """Every rank reaches this point before any goes on (no-op on one rank)."""
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int, device) -> float:
+    """The largest of the ranks' values (the step time of the slowest rank)."""
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 # ---- CPU oracle baseline -----------------------------------------------------------
 
 def oracle_sample(rows: int = 256, layers_idx=(0,)):
@@ -355,17 +373,6 @@ def run_gpu(args, world, rank, local):
     nbytes = step_bytes(layers)
     launches_per_step = 2 * len(layers)
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
     stream = torch.cuda.current_stream()
     for _ in range(args.warmup):
         graph.replay()
@@ -373,7 +380,7 @@ def run_gpu(args, world, rank, local):
 
     # ---- headline: device-timed steps, inputs resident in HBM --------------------
     with ClockSampler(local) as clk:
-        barrier()
+        barrier(world)
         torch.cuda.synchronize()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
@@ -382,8 +389,8 @@ def run_gpu(args, world, rank, local):
             graph.replay()
         e1.record(stream)
         torch.cuda.synchronize()
-        barrier()
-        ms_total = max_over_ranks(e0.elapsed_time(e1))
+        barrier(world)
+        ms_total = max_over_ranks(e0.elapsed_time(e1), world, device)
     clocks = clk.summary()
     ms_step = ms_total / args.steps
     value = world * nbytes / (ms_step * 1e-3) / 1e9
@@ -416,7 +423,7 @@ def run_gpu(args, world, rank, local):
             graph.replay()
             y_host.copy_(stack.y_all, non_blocking=True)
         torch.cuda.synchronize()
-        barrier()
+        barrier(world)
         torch.cuda.synchronize()
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
@@ -427,8 +434,8 @@ def run_gpu(args, world, rank, local):
             y_host.copy_(stack.y_all, non_blocking=True)
         b.record(stream)
         torch.cuda.synchronize()
-        barrier()
-        ms_e2e = max_over_ranks(a.elapsed_time(b)) / args.steps
+        barrier(world)
+        ms_e2e = max_over_ranks(a.elapsed_time(b), world, device) / args.steps
         e2e = {"value": round(world * nbytes / (ms_e2e * 1e-3) / 1e9, 1), "unit": UNIT,
                "us_per_token": round(ms_e2e * 1e3, 2),
                "h2d_bytes_per_step": int(stack.x_all.numel() * 4),
@@ -456,7 +463,7 @@ def run_gpu(args, world, rank, local):
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                          "unit": "GB/s", "frac": round(achieved / peak, 4),
                          "peak_kind": peak_kind, "traffic": traffic,
-                         "kernel": "k_linear (sq_linear decode)",
+                         "kernel": "k_linear_tc (sq_linear decode, tensor cores)",
                          "bytes_per_launch": int(bytes_launch),
                          "us_per_launch": round(ms_launch * 1e3, 3), "per_shape": shapes},
             "clocks": clocks,
@@ -474,7 +481,7 @@ def run_gpu(args, world, rank, local):
 def kernel_hash() -> str:
     import hashlib
     h = hashlib.sha256()
-    for f in ("sq_linear.cu", "sq_common.cuh", "sq_internal.h"):
+    for f in ("sq_linear_tc.cu", "sq_common.cuh", "sq_internal.h"):
         with open(os.path.join(ROOT, "decode_matvec_sq_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]

@@ -1,0 +1,92 @@
+"""Host-side logic of bench.py that needs no GPU: the algorithmic byte
+accounting, the rank helpers on a world-size-2 gloo group, and the CPU
+reference arm launched the way the multi-GPU bench is (torchrun, 2 ranks)."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from synth import workloads as wl  # noqa: E402
+from tests.conftest import read_golden  # noqa: E402
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def test_bytes_per_weight_matches_page_example():
+    # m.lqnn.cn/news/241359, section 3.2: 0.125 * 0.7 + 1 * 0.3 = 0.3875 byte
+    rows = read_golden("bytes_per_weight_example.txt")
+    shares = [(float(v[0]), float(v[1])) for k, v in rows if k == "share"]
+    assert len(shares) == 2
+    assert bench.bytes_per_weight(shares) == pytest.approx(0.3875, abs=1e-12)
+
+
+def test_stack_step_bytes():
+    """Packed weights of the 7B-shaped stack: 1/8 + 1 + 4/128 + 4/K bytes per
+    weight; plus per token xq, sx, x_out, idx, y and the activation split."""
+    layers = wl.config2(32)
+    shapes = {(4096, 12288, 20), (4096, 4096, 20), (4096, 22016, 20), (11008, 4096, 55)}
+    assert {(L.K, L.N, L.n_out) for L in layers} == shapes
+    w = sum(L.N * L.K for L in layers)
+    assert w == 32 * (4096 * 12288 + 4096 * 4096 + 4096 * 22016 + 11008 * 4096)
+    packed = sum(bench.linear_weight_bytes(L) for L in layers)
+    closed = sum(L.N * (L.K / 8 + L.K + 4 * L.K / 128 + 4) for L in layers)
+    assert packed == pytest.approx(closed, rel=1e-9)  # K multiple of 128: no padding
+    total = bench.step_bytes(layers)
+    assert 7.49e9 < packed < total < 7.52e9
+
+
+def _gloo_worker(rank, world, port, out_dir):
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        bench.barrier(world)
+        m = bench.max_over_ranks(1.5 * (rank + 1), world, "cpu")
+        bench.barrier(world)
+        with open(os.path.join(out_dir, f"r{rank}.txt"), "w") as f:
+            f.write(repr(m))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_gloo(tmp_path):
+    import torch.multiprocessing as mp
+    mp.start_processes(_gloo_worker, args=(2, _free_port(), str(tmp_path)), nprocs=2,
+                       start_method="spawn", join=True)
+    for r in range(2):
+        assert float(open(tmp_path / f"r{r}.txt").read()) == 3.0
+
+
+def test_max_over_ranks_single_rank_is_identity():
+    assert bench.max_over_ranks(2.25, 1, "cpu") == 2.25
+    bench.barrier(1)
+
+
+def test_reference_arm_under_torchrun_two_ranks():
+    """Rank 0 alone times the oracle and prints one JSON line; rank 1 exits 0
+    without work."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(_free_port()),
+           os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
+           "--steps", "1", "--warmup", "3", "--oracle-rows", "4"]
+    env = dict(os.environ, OMP_NUM_THREADS="1")
+    p = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=600, env=env)
+    assert p.returncode == 0, p.stderr[-2000:]
+    lines = [l for l in p.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, p.stdout
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["unit"] == "GB/s" and d["n_gpus"] == 2
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] == 1
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"] > 0
+    assert d["metric"] == bench.METRIC and d["higher_is_better"] is True
