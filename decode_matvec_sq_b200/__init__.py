@@ -75,6 +75,7 @@ def lib():
         "sq_linear": ([pw, vp, vp, vp, vp, i32, i32, vp, vp, sz, vp, u32, vp], ctypes.c_int),
         "sq_linear_accumulators": ([pw, vp, vp, vp, vp, i32, i32, vp, vp, vp, vp, sz, vp, u32, vp],
                                    ctypes.c_int),
+        "sq_linear_noalloc": ([pw, vp, vp, vp, vp, i32, i32, vp, vp, u32, vp], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -253,6 +254,24 @@ def linear(pw: PackedWeight, xq, sx, x_out, idx, y=None, workspace=None, status=
                         _ptr(idx) if n else None, n, M, _ptr(y), _ptr(workspace),
                         workspace.numel(), _ptr(status), _flags(pdl, cuda_cores),
                         _stream(stream)), "sq_linear")
+    return y
+
+
+# the fixed scratch size of sq_linear_noalloc (include/sq.h)
+NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def linear_noalloc(pw: PackedWeight, xq, sx, x_out, idx, y, status=None, pdl: bool = False,
+                   cuda_cores: bool = False, stream=None):
+    """sq_linear with the library's fixed device scratch instead of a workspace
+    (for callers that cannot allocate device memory at call time).  y [M][N]
+    float32 is the caller's.  Calls on one device must not overlap in time."""
+    M = xq.shape[0]
+    n = 0 if idx is None else int(idx.numel())
+    _ck(lib().sq_linear_noalloc(ctypes.byref(pw.view), _ptr(xq), _ptr(sx),
+                                _ptr(x_out) if n else None, _ptr(idx) if n else None, n, M,
+                                _ptr(y), _ptr(status), _flags(pdl, cuda_cores), _stream(stream)),
+        "sq_linear_noalloc")
     return y
 
 

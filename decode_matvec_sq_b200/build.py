@@ -34,6 +34,7 @@ SOURCES = [
     ("sq_act.cu", ["-fmad=false"]),
     ("sq_linear.cu", []),
     ("sq_linear_tc.cu", []),
+    ("sq_noalloc.cu", []),
 ]
 
 

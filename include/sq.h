@@ -203,6 +203,30 @@ sq_status sq_linear_accumulators(const sq_packed_weight *w, const int8_t *xq, co
                                  void *workspace, size_t ws_bytes, int32_t *dev_status,
                                  uint32_t flags, void *stream);
 
+/*
+ * sq_linear without a caller workspace, for callers that cannot allocate
+ * device memory at call time.  This entry point has no counterpart on the
+ * pages: it only changes where the scratch lives.
+ *   Scratch: one file-scope device array of SQ_LINEAR_NOALLOC_SCRATCH_BYTES
+ *   (16 MiB) per device, inside this library.  Nothing is allocated.
+ *   Limit: a call whose sq_linear_workspace_bytes(w, M) exceeds that size
+ *   returns SQ_ERR_WORKSPACE before any device work (on a 148-SM B200: more
+ *   than 1,769,472 rows).
+ *   First call on each device: looks up the array's device address
+ *   (cudaGetSymbolAddress, with that device current) and zero-fills the
+ *   array on `stream` before its launch, because the per-row arrival
+ *   counters in it must start at zero.  Make that first call before any
+ *   stream capture.  Every call leaves the counters zero again.
+ *   Overlapping calls race: all calls on a device share the array, so two
+ *   calls whose kernels may run at the same time (other streams, other host
+ *   threads) give wrong results.  Order them on one stream or by events.
+ * Arguments, flags and results are those of sq_linear.
+ */
+#define SQ_LINEAR_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+sq_status sq_linear_noalloc(const sq_packed_weight *w, const int8_t *xq, const float *sx,
+                            const float *x_out, const int32_t *idx, int32_t n_out, int32_t M,
+                            float *y, int32_t *dev_status, uint32_t flags, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -1,0 +1,73 @@
+"""sq_linear_noalloc: the decode linear layer with the library's fixed device
+scratch instead of a caller workspace.  Two calls in a row must agree with
+sq_linear on the same inputs within the y tolerance (1e-5 * sum_j |W_rj x_j|);
+the second call also shows that the first left the arrival counters zero.
+Self-contained: passes alone in a fresh process and after the other tests."""
+import ctypes
+
+import numpy as np
+import pytest
+
+import decode_matvec_sq_b200 as sq
+
+torch = pytest.importorskip("torch")
+
+TOL = 1e-5
+
+
+def _inputs(N, K, M, n_out, seed):
+    rng = np.random.default_rng(seed)
+    W = rng.laplace(0.0, 0.02, (N, K)).astype(np.float32)
+    x = rng.standard_normal((M, K)).astype(np.float32)
+    idx = np.sort(rng.choice(K, n_out, replace=False)).astype(np.int32)
+    x[:, idx] *= 30.0
+    return W, x, idx
+
+
+def _bound(W, x):
+    return np.abs(x.astype(np.float64)) @ np.abs(W.astype(np.float64)).T  # [M][N]
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("N,K,M,n_out,P,cuda_cores", [
+    (512, 512, 1, 4, -1, False),       # the single-layer workload's shape
+    (4096, 4096, 1, 20, -1, False),    # rows shared between warps (counters used)
+    (1000, 1000, 3, 9, 60, False),     # threshold trunk, ragged K, 3 tokens
+    (777, 2048, 5, 10, -1, True),      # CUDA-core kernel, two passes of tokens
+])
+def test_noalloc_matches_sq_linear_twice(cuda_device, N, K, M, n_out, P, cuda_cores):
+    W, x, idx = _inputs(N, K, M, n_out, seed=N + K + M)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pw = sq.decompose_pack(torch.from_numpy(W).cuda(), trunk_percent=P, status=st)
+    idxd = torch.from_numpy(idx).cuda()
+    xq, sx, xo = sq.quantize_act(torch.from_numpy(x).cuda(), idxd, status=st)
+    y_ref = sq.linear(pw, xq, sx, xo, idxd, status=st, cuda_cores=cuda_cores)
+    ys = []
+    for _ in range(2):
+        y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+        sq.linear_noalloc(pw, xq, sx, xo, idxd, y, status=st, cuda_cores=cuda_cores)
+        ys.append(y)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    ref = y_ref.cpu().numpy().astype(np.float64)
+    bound = _bound(W, x)
+    for y in ys:
+        err = np.abs(y.cpu().numpy().astype(np.float64) - ref)
+        assert np.isfinite(err).all()
+        assert (err <= TOL * bound).all(), float((err / bound).max())
+
+
+@pytest.mark.gpu
+def test_noalloc_rejects_problems_beyond_its_scratch(cuda_device):
+    """More rows than the fixed scratch has counters for: SQ_ERR_WORKSPACE from
+    the host checks, before any device work (the view's pointers are never
+    dereferenced)."""
+    L = sq.lib()
+    N, K = 4_000_000, 128
+    v = sq.SqPackedWeight()
+    assert L.sq_packed_view(ctypes.c_void_p(1 << 40), N, K, 128, 0, ctypes.byref(v)) == 0
+    need = L.sq_linear_workspace_bytes(ctypes.byref(v), 1)
+    assert need > sq.NOALLOC_SCRATCH_BYTES
+    p = ctypes.c_void_p(1 << 41)
+    rc = L.sq_linear_noalloc(ctypes.byref(v), p, p, None, None, 0, 1, p, None, 0, None)
+    assert rc == 8 and L.sq_status_string(rc)  # SQ_ERR_WORKSPACE
