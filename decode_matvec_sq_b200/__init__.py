@@ -22,7 +22,8 @@ LIB_PATH = os.path.join(PKG_DIR, "libsq.so")
 HEADER = os.path.join(os.path.dirname(PKG_DIR), "include", "sq.h")
 
 SQ_LAUNCH_PDL = 1
-SQ_LAUNCH_CUDA_CORES = 2
+SQ_LAYOUT_ROWS = 0
+SQ_LAYOUT_TILES = 1
 
 STATUS = {
     0: "SQ_OK", 1: "SQ_ERR_INVALID_ARG", 2: "SQ_ERR_SHAPE", 3: "SQ_ERR_ALIGN",
@@ -42,7 +43,7 @@ class SQError(RuntimeError):
 class SqPackedWeight(ctypes.Structure):
     _fields_ = [
         ("N", ctypes.c_int32), ("K", ctypes.c_int32), ("group_size", ctypes.c_int32),
-        ("sign_stride", ctypes.c_int32), ("res_stride", ctypes.c_int32),
+        ("layout", ctypes.c_int32), ("sign_stride", ctypes.c_int32), ("res_stride", ctypes.c_int32),
         ("scale_stride", ctypes.c_int32),
         ("sign_bits", ctypes.c_void_p), ("mask_bits", ctypes.c_void_p),
         ("alpha", ctypes.c_void_p), ("res_q", ctypes.c_void_p), ("res_scale", ctypes.c_void_p),
@@ -66,8 +67,8 @@ def lib():
     sig = {
         "sq_status_string": ([ctypes.c_int], ctypes.c_char_p),
         "sq_device_check": ([], ctypes.c_int),
-        "sq_packed_bytes": ([i32, i32, i32, i32], sz),
-        "sq_packed_view": ([vp, i32, i32, i32, i32, pw], ctypes.c_int),
+        "sq_packed_bytes": ([i32, i32, i32, i32, i32], sz),
+        "sq_packed_view": ([vp, i32, i32, i32, i32, i32, pw], ctypes.c_int),
         "sq_decompose_pack": ([vp, i32, i32, i32, pw, vp, vp], ctypes.c_int),
         "sq_calibrate_outliers": ([vp, i32, i32, i32, vp, vp, vp], ctypes.c_int),
         "sq_quantize_act": ([vp, i32, i32, vp, i32, vp, vp, vp, vp, u32, vp], ctypes.c_int),
@@ -114,19 +115,32 @@ def device_check() -> None:
 
 # ---- packed weights ------------------------------------------------------------
 
+def default_layout(group_size: int) -> int:
+    """The tensor-core layout for group size 128, the row layout otherwise."""
+    return SQ_LAYOUT_TILES if group_size == 128 else SQ_LAYOUT_ROWS
+
+
 @dataclass
 class PackedWeight:
-    """A packed weight in one device allocation (``buf``) with its C view."""
+    """A packed weight in one device allocation (``buf``) with its C view.
+    The array accessors return the raw arrays in the weight's layout
+    (include/sq.h documents both layouts)."""
     N: int
     K: int
     group_size: int
     with_mask: bool
+    layout: int
     buf: object                 # torch.uint8 device tensor
     view: SqPackedWeight
 
     @property
     def nbytes(self) -> int:
         return int(self.buf.numel())
+
+    @property
+    def rows(self) -> int:
+        """Rows of every array: N, or N padded to 16 in the tiled layout."""
+        return round_up(self.N, 16) if self.layout == SQ_LAYOUT_TILES else self.N
 
     def _arr(self, field: str, dtype, shape):
         import torch
@@ -140,50 +154,56 @@ class PackedWeight:
 
     def sign_bits(self):
         import torch
-        return self._arr("sign_bits", torch.int32, (self.N, self.view.sign_stride))
+        return self._arr("sign_bits", torch.int32, (self.rows, self.view.sign_stride))
 
     def mask_bits(self):
         import torch
         if not self.with_mask:
             return None
-        return self._arr("mask_bits", torch.int32, (self.N, self.view.sign_stride))
+        return self._arr("mask_bits", torch.int32, (self.rows, self.view.sign_stride))
 
     def alpha(self):
         import torch
-        return self._arr("alpha", torch.float32, (self.N,))
+        return self._arr("alpha", torch.float32, (self.rows,))[:self.N]
 
     def res_q(self):
         import torch
-        return self._arr("res_q", torch.int8, (self.N, self.view.res_stride))
+        return self._arr("res_q", torch.int8, (self.rows, self.view.res_stride))
 
     def res_scale(self):
         import torch
-        return self._arr("res_scale", torch.float32, (self.N, self.view.scale_stride))
+        return self._arr("res_scale", torch.float32, (self.rows, self.view.scale_stride))
 
 
-def packed_bytes(N: int, K: int, group_size: int = 128, with_mask: bool = False) -> int:
-    return int(lib().sq_packed_bytes(N, K, group_size, int(with_mask)))
+def packed_bytes(N: int, K: int, group_size: int = 128, with_mask: bool = False,
+                 layout: int = None) -> int:
+    if layout is None:
+        layout = default_layout(group_size)
+    return int(lib().sq_packed_bytes(N, K, group_size, int(with_mask), layout))
 
 
 def alloc_packed(N: int, K: int, group_size: int = 128, with_mask: bool = False,
-                 device=None) -> PackedWeight:
+                 layout: int = None, device=None) -> PackedWeight:
     import torch
-    nbytes = packed_bytes(N, K, group_size, with_mask)
+    if layout is None:
+        layout = default_layout(group_size)
+    nbytes = packed_bytes(N, K, group_size, with_mask, layout)
     if nbytes == 0:
         raise SQError(STATUS_CODE["SQ_ERR_SHAPE"], "sq_packed_bytes")
     buf = torch.empty(nbytes, dtype=torch.uint8, device=device or "cuda")
     v = SqPackedWeight()
-    _ck(lib().sq_packed_view(_ptr(buf), N, K, group_size, int(with_mask), ctypes.byref(v)),
-        "sq_packed_view")
-    return PackedWeight(N, K, group_size, with_mask, buf, v)
+    _ck(lib().sq_packed_view(_ptr(buf), N, K, group_size, int(with_mask), layout,
+                             ctypes.byref(v)), "sq_packed_view")
+    return PackedWeight(N, K, group_size, with_mask, layout, buf, v)
 
 
-def decompose_pack(W, trunk_percent: int = -1, group_size: int = 128, out: PackedWeight = None,
-                   status=None, stream=None) -> PackedWeight:
-    """Offline split of W[N][K] (float32, device) into the packed form."""
+def decompose_pack(W, trunk_percent: int = -1, group_size: int = 128, layout: int = None,
+                   out: PackedWeight = None, status=None, stream=None) -> PackedWeight:
+    """Offline split of W[N][K] (float32, device) into the packed form
+    (default layout: tiles for group size 128, rows otherwise)."""
     N, K = W.shape
     if out is None:
-        out = alloc_packed(N, K, group_size, trunk_percent > 0, device=W.device)
+        out = alloc_packed(N, K, group_size, trunk_percent > 0, layout, device=W.device)
     _ck(lib().sq_decompose_pack(_ptr(W), N, K, trunk_percent, ctypes.byref(out.view),
                                 _ptr(status), _stream(stream)), "sq_decompose_pack")
     return out
@@ -201,13 +221,13 @@ def calibrate_outliers(X, k: int, out=None, status=None, stream=None):
 
 def quantize_act(x, idx, xq=None, sx=None, x_out=None, status=None, pdl: bool = False,
                  stream=None):
-    """x[M][K] float32 -> (xq [M][roundup(K,16)] int8, sx [M], x_out [M][n_out])."""
+    """x[M][K] float32 -> (xq [M][roundup(K,128)] int8, sx [M], x_out [M][n_out])."""
     import torch
     M, K = x.shape
     n = 0 if idx is None else int(idx.numel())
     dev = x.device
     if xq is None:
-        xq = torch.empty(M, round_up(K, 16), dtype=torch.int8, device=dev)
+        xq = torch.empty(M, round_up(K, 128), dtype=torch.int8, device=dev)
     if sx is None:
         sx = torch.empty(M, dtype=torch.float32, device=dev)
     if x_out is None:
@@ -235,14 +255,14 @@ def new_workspace(pw: PackedWeight, M: int = 1, device=None):
                        device=device or pw.buf.device)
 
 
-def _flags(pdl: bool, cuda_cores: bool) -> int:
-    return (SQ_LAUNCH_PDL if pdl else 0) | (SQ_LAUNCH_CUDA_CORES if cuda_cores else 0)
+def _flags(pdl: bool) -> int:
+    return SQ_LAUNCH_PDL if pdl else 0
 
 
 def linear(pw: PackedWeight, xq, sx, x_out, idx, y=None, workspace=None, status=None,
-           pdl: bool = False, cuda_cores: bool = False, stream=None):
+           pdl: bool = False, stream=None):
     """y[M][N] = fused trunk + residual + outlier product (float32).
-    ``cuda_cores`` selects the dp4a kernel instead of the tensor-core one."""
+    The weight's layout picks the kernel: tiles -> tensor cores, rows -> dp4a."""
     import torch
     M = xq.shape[0]
     n = 0 if idx is None else int(idx.numel())
@@ -252,7 +272,7 @@ def linear(pw: PackedWeight, xq, sx, x_out, idx, y=None, workspace=None, status=
         workspace = new_workspace(pw, M)
     _ck(lib().sq_linear(ctypes.byref(pw.view), _ptr(xq), _ptr(sx), _ptr(x_out) if n else None,
                         _ptr(idx) if n else None, n, M, _ptr(y), _ptr(workspace),
-                        workspace.numel(), _ptr(status), _flags(pdl, cuda_cores),
+                        workspace.numel(), _ptr(status), _flags(pdl),
                         _stream(stream)), "sq_linear")
     return y
 
@@ -262,7 +282,7 @@ NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 def linear_noalloc(pw: PackedWeight, xq, sx, x_out, idx, y, status=None, pdl: bool = False,
-                   cuda_cores: bool = False, stream=None):
+                   stream=None):
     """sq_linear with the library's fixed device scratch instead of a workspace
     (for callers that cannot allocate device memory at call time).  y [M][N]
     float32 is the caller's.  Calls on one device must not overlap in time."""
@@ -270,13 +290,13 @@ def linear_noalloc(pw: PackedWeight, xq, sx, x_out, idx, y, status=None, pdl: bo
     n = 0 if idx is None else int(idx.numel())
     _ck(lib().sq_linear_noalloc(ctypes.byref(pw.view), _ptr(xq), _ptr(sx),
                                 _ptr(x_out) if n else None, _ptr(idx) if n else None, n, M,
-                                _ptr(y), _ptr(status), _flags(pdl, cuda_cores), _stream(stream)),
+                                _ptr(y), _ptr(status), _flags(pdl), _stream(stream)),
         "sq_linear_noalloc")
     return y
 
 
 def linear_accumulators(pw: PackedWeight, xq, sx, x_out, idx, workspace=None, status=None,
-                        cuda_cores: bool = False, stream=None):
+                        stream=None):
     """(y, T [M][N] int32, R [M][N][ceil(K/G)] int32) from the decode kernel."""
     import torch
     M = xq.shape[0]
@@ -291,6 +311,6 @@ def linear_accumulators(pw: PackedWeight, xq, sx, x_out, idx, workspace=None, st
     _ck(lib().sq_linear_accumulators(ctypes.byref(pw.view), _ptr(xq), _ptr(sx),
                                      _ptr(x_out) if n else None, _ptr(idx) if n else None, n, M,
                                      _ptr(y), _ptr(T), _ptr(R), _ptr(workspace),
-                                     workspace.numel(), _ptr(status), _flags(False, cuda_cores),
+                                     workspace.numel(), _ptr(status), _flags(False),
                                      _stream(stream)), "sq_linear_accumulators")
     return y, T, R

@@ -46,7 +46,7 @@ __device__ __forceinline__ bool outlier_bit(const uint32_t* is_out, int j) {
 }
 
 __global__ void __launch_bounds__(kActThreads) k_quantize_act(
-    const float* __restrict__ x, int M, int K, int K16, const int32_t* __restrict__ idx, int n_out,
+    const float* __restrict__ x, int M, int K, int Kx, const int32_t* __restrict__ idx, int n_out,
     int8_t* __restrict__ xq, float* __restrict__ sx, float* __restrict__ x_out,
     int32_t* __restrict__ status, int pdl) {
   extern __shared__ uint32_t is_out[];  // ceil(K/32) words
@@ -57,7 +57,7 @@ __global__ void __launch_bounds__(kActThreads) k_quantize_act(
   }
   const int t = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nchunk = (K + 31) >> 5;  // also ceil(K16 / 32)
+  const int nchunk = (K + 31) >> 5;
   const float* xt = x + (int64_t)t * K;
   // x into registers (issued before anything else)
   float v[kActRegs];
@@ -109,12 +109,12 @@ __global__ void __launch_bounds__(kActThreads) k_quantize_act(
   const double rinv = s != 0.0f ? 1.0 / (double)s : 0.0;
   if (threadIdx.x == 0) sx[t] = s;
 
-  int8_t* qt = xq + (int64_t)t * K16;
+  int8_t* qt = xq + (int64_t)t * Kx;
   auto emit = [&](int c, float u) {
     const int j = c * 32 + lane;
     int q = 0;
     if (j < K && !outlier_bit(is_out, j)) q = quantize_exact(u, s, rinv);
-    if (j < K16) qt[j] = (int8_t)q;
+    qt[j] = (int8_t)q;  // j < 32 * nchunk <= Kx
   };
 #pragma unroll
   for (int i = 0; i < kActRegs; ++i) {
@@ -127,6 +127,8 @@ __global__ void __launch_bounds__(kActThreads) k_quantize_act(
       emit(c, j < K ? xt[j] : 0.0f);
     }
   }
+  // pad chunks up to the row stride (a multiple of 128 channels)
+  for (int c = nchunk + warp; c < (Kx >> 5); c += 32) qt[c * 32 + lane] = 0;
   if (nonfinite) set_status(status, SQ_ERR_NONFINITE);
   if (bad_idx) set_status(status, SQ_ERR_INVALID_ARG);
 }
@@ -211,7 +213,7 @@ __global__ void __launch_bounds__(kCalThreads) k_calibrate(const float* __restri
 cudaError_t launch_quantize_act(const float* x, int M, int K, const int32_t* idx, int n_out,
                                 int8_t* xq, float* sx, float* x_out, int32_t* status, bool pdl,
                                 cudaStream_t stream) {
-  const int K16 = (int)round_up(K, 16);
+  const int Kx = (int)xq_stride_of(K);
   const size_t smem = (size_t)ceil_div(K, 32) * sizeof(uint32_t);
   cudaError_t e = ensure_smem_attr((const void*)k_quantize_act, (int)smem);
   if (e != cudaSuccess) return e;
@@ -225,7 +227,7 @@ cudaError_t launch_quantize_act(const float* x, int M, int K, const int32_t* idx
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, k_quantize_act, x, M, K, K16, idx, n_out, xq, sx, x_out, status,
+  return cudaLaunchKernelEx(&cfg, k_quantize_act, x, M, K, Kx, idx, n_out, xq, sx, x_out, status,
                             pdl ? 1 : 0);
 }
 

@@ -8,6 +8,7 @@
 #include <mutex>
 
 #include "sq_internal.h"
+#include "sq_layout.h"
 
 namespace sq {
 
@@ -85,15 +86,38 @@ sq_status check_device(DeviceInfo* d) {
 
 sq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? SQ_OK : SQ_ERR_CUDA; }
 
-int32_t sign_stride_of(int32_t K) { return (int32_t)round_up(ceil_div(K, 32), 4); }
-int32_t res_stride_of(int32_t K) { return (int32_t)round_up(K, 16); }
-int32_t scale_stride_of(int32_t K, int32_t G) { return (int32_t)round_up(ceil_div(K, G), 4); }
+// Largest K of the tiled layout (the decode kernel keeps a bitmap of the
+// outlier channels of a whole row in shared memory).
+constexpr int32_t kMaxTiledK = 131072;
+
+bool valid_layout(int32_t layout, int32_t G, int32_t K) {
+  if (layout == SQ_LAYOUT_ROWS) return true;
+  return layout == SQ_LAYOUT_TILES && G == kTileK && K <= kMaxTiledK;
+}
+
+int32_t sign_stride_of(int32_t K, int32_t layout) {
+  return layout == SQ_LAYOUT_TILES ? (int32_t)(tiles_cols(K) / 32) : (int32_t)round_up(ceil_div(K, 32), 4);
+}
+int32_t res_stride_of(int32_t K, int32_t layout) {
+  return layout == SQ_LAYOUT_TILES ? (int32_t)tiles_cols(K) : (int32_t)round_up(K, 16);
+}
+int32_t scale_stride_of(int32_t K, int32_t G, int32_t layout) {
+  return layout == SQ_LAYOUT_TILES ? (int32_t)(tiles_cols(K) / kTileK)
+                                   : (int32_t)round_up(ceil_div(K, G), 4);
+}
+// Rows of every array (the tiled layout pads N to a multiple of 16).
+int64_t rows_of(int32_t N, int32_t layout) {
+  return layout == SQ_LAYOUT_TILES ? tiles_rows(N) : (int64_t)N;
+}
 
 sq_status check_weight(const sq_packed_weight* w) {
   if (!w || !w->sign_bits || !w->alpha || !w->res_q || !w->res_scale) return SQ_ERR_INVALID_ARG;
   if (!valid_group(w->group_size) || !valid_shape(w->N, w->K)) return SQ_ERR_SHAPE;
-  if (w->sign_stride != sign_stride_of(w->K) || w->res_stride != res_stride_of(w->K) ||
-      w->scale_stride != scale_stride_of(w->K, w->group_size))
+  if (w->layout != SQ_LAYOUT_ROWS && w->layout != SQ_LAYOUT_TILES) return SQ_ERR_INVALID_ARG;
+  if (!valid_layout(w->layout, w->group_size, w->K)) return SQ_ERR_SHAPE;
+  if (w->sign_stride != sign_stride_of(w->K, w->layout) ||
+      w->res_stride != res_stride_of(w->K, w->layout) ||
+      w->scale_stride != scale_stride_of(w->K, w->group_size, w->layout))
     return SQ_ERR_SHAPE;
   if (!aligned16(w->sign_bits) || !aligned16(w->alpha) || !aligned16(w->res_q) ||
       !aligned16(w->res_scale) || (w->mask_bits && !aligned16(w->mask_bits)))
@@ -102,12 +126,12 @@ sq_status check_weight(const sq_packed_weight* w) {
 }
 
 // Offsets of the five arrays inside one allocation, each 256-byte aligned.
-// alpha holds roundup(N, 8) floats so that whole 8-row blocks can be copied.
+// alpha holds roundup(N, 8) (rows) or N16 (tiles) floats.
 struct Carve {
   size_t sign, mask, alpha, res, scale, total;
 };
 
-Carve carve(int32_t N, int32_t K, int32_t G, int32_t with_mask) {
+Carve carve(int32_t N, int32_t K, int32_t G, int32_t with_mask, int32_t layout) {
   Carve c;
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -115,11 +139,12 @@ Carve carve(int32_t N, int32_t K, int32_t G, int32_t with_mask) {
     off = (size_t)round_up((int64_t)(off + bytes), 256);
     return at;
   };
-  c.sign = take((size_t)N * sign_stride_of(K) * 4);
-  c.mask = with_mask ? take((size_t)N * sign_stride_of(K) * 4) : 0;
-  c.alpha = take((size_t)round_up(N, 8) * 4);
-  c.res = take((size_t)N * res_stride_of(K));
-  c.scale = take((size_t)N * scale_stride_of(K, G) * 4);
+  const int64_t rows = rows_of(N, layout);
+  c.sign = take((size_t)rows * sign_stride_of(K, layout) * 4);
+  c.mask = with_mask ? take((size_t)rows * sign_stride_of(K, layout) * 4) : 0;
+  c.alpha = take((size_t)round_up(rows, 8) * 4);
+  c.res = take((size_t)rows * res_stride_of(K, layout));
+  c.scale = take((size_t)rows * scale_stride_of(K, G, layout) * 4);
   c.total = off;
   return c;
 }
@@ -148,24 +173,30 @@ sq_status sq_device_check(void) {
   return check_device(&d);
 }
 
-size_t sq_packed_bytes(int32_t N, int32_t K, int32_t group_size, int32_t with_mask) {
+size_t sq_packed_bytes(int32_t N, int32_t K, int32_t group_size, int32_t with_mask,
+                       int32_t layout) {
   if (!valid_shape(N, K) || !valid_group(group_size)) return 0;
-  return carve(N, K, group_size, with_mask).total;
+  if (layout != SQ_LAYOUT_ROWS && layout != SQ_LAYOUT_TILES) return 0;
+  if (!valid_layout(layout, group_size, K)) return 0;
+  return carve(N, K, group_size, with_mask, layout).total;
 }
 
 sq_status sq_packed_view(void* base, int32_t N, int32_t K, int32_t group_size, int32_t with_mask,
-                         sq_packed_weight* out) {
+                         int32_t layout, sq_packed_weight* out) {
   if (!base || !out) return SQ_ERR_INVALID_ARG;
+  if (layout != SQ_LAYOUT_ROWS && layout != SQ_LAYOUT_TILES) return SQ_ERR_INVALID_ARG;
   if (!valid_shape(N, K) || !valid_group(group_size)) return SQ_ERR_SHAPE;
+  if (!valid_layout(layout, group_size, K)) return SQ_ERR_SHAPE;
   if ((reinterpret_cast<uintptr_t>(base) & 255u) != 0) return SQ_ERR_ALIGN;
-  const Carve c = carve(N, K, group_size, with_mask);
+  const Carve c = carve(N, K, group_size, with_mask, layout);
   uint8_t* b = static_cast<uint8_t*>(base);
   out->N = N;
   out->K = K;
   out->group_size = group_size;
-  out->sign_stride = sign_stride_of(K);
-  out->res_stride = res_stride_of(K);
-  out->scale_stride = scale_stride_of(K, group_size);
+  out->layout = layout;
+  out->sign_stride = sign_stride_of(K, layout);
+  out->res_stride = res_stride_of(K, layout);
+  out->scale_stride = scale_stride_of(K, group_size, layout);
   out->sign_bits = reinterpret_cast<uint32_t*>(b + c.sign);
   out->mask_bits = with_mask ? reinterpret_cast<uint32_t*>(b + c.mask) : nullptr;
   out->alpha = reinterpret_cast<float*>(b + c.alpha);
@@ -237,7 +268,7 @@ static sq_status linear_common(const sq_packed_weight* w, const int8_t* xq, cons
   if (M < 1 || M > (1 << 20)) return SQ_ERR_SHAPE;
   if (n_out < 0 || n_out > kMaxOutliers || n_out > w->K) return SQ_ERR_SHAPE;
   if (n_out > 0 && (!idx || !x_out)) return SQ_ERR_INVALID_ARG;
-  if (flags & ~(SQ_LAUNCH_PDL | SQ_LAUNCH_CUDA_CORES)) return SQ_ERR_INVALID_ARG;
+  if (flags & ~SQ_LAUNCH_PDL) return SQ_ERR_INVALID_ARG;
   if (!aligned16(xq) || !aligned16(sx) || !aligned16(y) ||
       (n_out > 0 && (!aligned16(idx) || !aligned16(x_out))) || (workspace && !aligned16(workspace)))
     return SQ_ERR_ALIGN;
@@ -252,11 +283,12 @@ static sq_status linear_common(const sq_packed_weight* w, const int8_t* xq, cons
     if (e != cudaSuccess) return SQ_ERR_CUDA;
   }
   const int ng = (int)ceil_div(w->K, w->group_size);
-  const bool tc = !(flags & SQ_LAUNCH_CUDA_CORES) && linear_tc_supported(*w);
+  const bool tc = w->layout == SQ_LAYOUT_TILES;
   const int per_pass = tc ? kMaxTokensPerPassTc : kMaxTokensPerPass;
+  const int64_t xs = xq_stride_of(w->K);
   for (int t0 = 0; t0 < M; t0 += per_pass) {
     const int m = std::min(per_pass, M - t0);
-    const int8_t* xq_t = xq + (int64_t)t0 * w->res_stride;
+    const int8_t* xq_t = xq + (int64_t)t0 * xs;
     const float* xo_t = n_out ? x_out + (int64_t)t0 * n_out : nullptr;
     float* y_t = y + (int64_t)t0 * w->N;
     int32_t* T_t = T_out ? T_out + (int64_t)t0 * w->N : nullptr;

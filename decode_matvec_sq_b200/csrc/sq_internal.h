@@ -25,6 +25,10 @@ cudaError_t ensure_smem_attr(const void* func, int bytes);
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
 
+// Row stride of the activation codes xq: roundup(K, 128) bytes, zero padded,
+// so that the decode kernels read whole 128-channel groups.
+inline int64_t xq_stride_of(int64_t K) { return round_up(K, 128); }
+
 // ---- launchers ---------------------------------------------------------------
 cudaError_t launch_decompose_pack(const float* W, int N, int K, int P, const sq_packed_weight& pw,
                                   int32_t* status, cudaStream_t stream);
@@ -36,17 +40,13 @@ cudaError_t launch_quantize_act(const float* x, int M, int K, const int32_t* idx
                                 int8_t* xq, float* sx, float* x_out, int32_t* status, bool pdl,
                                 cudaStream_t stream);
 
+// Launch plan of the CUDA-core decode kernel (SQ_LAYOUT_ROWS).
 struct LinearPlan {
   int M = 1;           // tokens in this pass (1..kMaxTokensPerPass)
-  int Kc = 0;          // channels per chunk
-  int n_c = 0;         // chunks per row
-  int n_rb = 0;        // row blocks
-  int U = 0;           // work units = n_rb * n_c
+  int Kc = 0;          // channels per piece
+  int n_c = 0;         // pieces per row
+  int U = 0;           // work units = N * n_c
   int grid = 0;        // CTAs
-  int S = 0;           // pipeline stages
-  int stage_bytes = 0;
-  int off_sign = 0, off_mask = 0, off_scale = 0, off_alpha = 0;
-  int hdr_bytes = 0;   // shared memory before the stages
   int smem_bytes = 0;
   size_t ws_cnt_bytes = 0;
   size_t ws_part_bytes = 0;
@@ -70,8 +70,7 @@ cudaError_t launch_linear(const sq_packed_weight& w, const LinearPlan& plan, con
                           float* y, int32_t* T_out, int32_t* R_out, void* workspace,
                           size_t part_bytes, int32_t* status, bool pdl, cudaStream_t stream);
 
-// Tensor-core decode kernel (group size 128), up to kMaxTokensPerPassTc tokens.
-bool linear_tc_supported(const sq_packed_weight& w);
+// Tensor-core decode kernel (SQ_LAYOUT_TILES), up to kMaxTokensPerPassTc tokens.
 size_t linear_tc_part_bytes(int sm_count);
 cudaError_t launch_linear_tc(const sq_packed_weight& w, int M, const int8_t* xq, const float* sx,
                              const float* x_out, const int32_t* idx, int n_out, float* y,

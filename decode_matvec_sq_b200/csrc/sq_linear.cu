@@ -64,6 +64,7 @@ struct Params {
   const int8_t* res;
   const float* scale;
   int N, K, K16, log2G, ng, sign_stride, res_stride, scale_stride;
+  int xs;            // row stride of xq (roundup(K, 128))
   int ppr;          // pieces per row = ceil(K16 / 1024)
   int P;            // total pieces = N * ppr (< 2^31)
   int warps_total;  // warps that own pieces: min(gridDim.x * kWarps, P); the rest idle
@@ -242,7 +243,7 @@ __global__ void __launch_bounds__(kThreads, BPS) k_linear(const Params p) {
     const int nseg = p.K16 >> 4;
     for (int t = 0; t < M; ++t)
       for (int seg = threadIdx.x; seg < nseg; seg += kThreads) {
-        const int4 x = ldg_nc_v4(p.xq + (int64_t)t * p.K16 + seg * 16);
+        const int4 x = ldg_nc_v4(p.xq + (int64_t)t * p.xs + seg * 16);
         int s = __dp4a(x.x, 0x01010101, 0);
         s = __dp4a(x.y, 0x01010101, s);
         s = __dp4a(x.z, 0x01010101, s);
@@ -288,7 +289,7 @@ __global__ void __launch_bounds__(kThreads, BPS) k_linear(const Params p) {
         for (int t = 0; t < M; ++t) {
           int x[8];
           if (act) {
-            const int8_t* xp = xq_lane + (int64_t)t * p.K16 + cc * kPiece;
+            const int8_t* xp = xq_lane + (int64_t)t * p.xs + cc * kPiece;
             if (k + 32 <= p.K16) {
               ld32B_cached<V8>(x, xp);
             } else {
@@ -546,6 +547,7 @@ cudaError_t launch_linear(const sq_packed_weight& w, const LinearPlan& plan, con
   p.N = w.N;
   p.K = w.K;
   p.K16 = w.res_stride;
+  p.xs = (int)xq_stride_of(w.K);
   p.log2G = log2_exact(w.group_size);
   p.ng = (int)ceil_div(w.K, w.group_size);
   p.sign_stride = w.sign_stride;

@@ -17,6 +17,7 @@
 
 #include "sq_common.cuh"
 #include "sq_internal.h"
+#include "sq_layout.h"
 
 namespace sq {
 namespace {
@@ -88,28 +89,43 @@ __device__ __forceinline__ void load_tile(float* tile, int pitch, const float* _
 }
 
 // ---- sign / mask bitplanes, alpha, residual codes and group scales --------
+// One thread per row.  TILED writes SQ_LAYOUT_TILES (rows padded to a
+// multiple of 16 and channels to a multiple of 128, pads zero); otherwise
+// SQ_LAYOUT_ROWS.
+template <bool TILED>
 __global__ void __launch_bounds__(kPackRows) k_pack(const float* __restrict__ W, int N, int K,
                                                     int P, int G, sq_packed_weight pw,
                                                     int32_t* __restrict__ status) {
   extern __shared__ float tile[];  // [kPackRows][G + 1]
   const int r0 = blockIdx.x * kPackRows;
   const int row = r0 + threadIdx.x;
-  const bool valid = row < N;
+  const bool valid = row < N;  // a row of W
+  // rows written: the rows of W, plus the zero pad rows of the tiled layout
+  const bool live = TILED ? row < (int)tiles_rows(N) : valid;
+  const int Kp = TILED ? (int)tiles_cols(K) : K;  // channels written
+  const int tpr = Kp / kTileK;                    // tiles per row block (tiled)
   const int nwords = (K + 31) / 32;
   const int ng = (K + G - 1) / G;
   const float tau = (valid && P > 0) ? pw.alpha[row] : -1.0f;  // k_threshold wrote it here
   bool nonfinite = false;
 
+  auto store_bits = [&](uint32_t* base, int word, uint32_t bits) {
+    if (TILED)
+      base[tiled_bits_word(row, word, tpr)] = tiled_bits_from_row_order(bits);
+    else
+      base[(int64_t)row * pw.sign_stride + word] = bits;
+  };
+
   // pass 1: bits, trunk sum, count
   double sum = 0.0;
   int64_t cnt = 0;
   const int pitch1 = kTile + 1;
-  for (int c0 = 0; c0 < K; c0 += kTile) {
-    load_tile(tile, pitch1, W, N, K, r0, c0, kTile);
+  for (int c0 = 0; c0 < Kp; c0 += kTile) {
+    if (c0 < K) load_tile(tile, pitch1, W, N, K, r0, c0, kTile);
     __syncthreads();
-    if (valid) {
+    if (live) {
       uint32_t sbits = 0, mbits = 0;
-      const int ncols = min(kTile, K - c0);
+      const int ncols = valid ? max(0, min(kTile, K - c0)) : 0;
       for (int j = 0; j < ncols; ++j) {
         const float v = tile[threadIdx.x * pitch1 + j];
         nonfinite |= !isfinite(v);
@@ -121,21 +137,21 @@ __global__ void __launch_bounds__(kPackRows) k_pack(const float* __restrict__ W,
           cnt += 1;
         }
       }
-      pw.sign_bits[(int64_t)row * pw.sign_stride + c0 / 32] = sbits;
-      if (pw.mask_bits) pw.mask_bits[(int64_t)row * pw.sign_stride + c0 / 32] = mbits;
+      store_bits(pw.sign_bits, c0 / 32, sbits);
+      if (pw.mask_bits) store_bits(pw.mask_bits, c0 / 32, mbits);
     }
     __syncthreads();
   }
   float alpha = 0.0f;
-  if (valid) {
-    alpha = cnt ? (float)(sum / (double)cnt) : 0.0f;
+  if (valid) alpha = cnt ? (float)(sum / (double)cnt) : 0.0f;
+  if (!TILED && valid) {
     for (int w = nwords; w < pw.sign_stride; ++w) {
       pw.sign_bits[(int64_t)row * pw.sign_stride + w] = 0u;
       if (pw.mask_bits) pw.mask_bits[(int64_t)row * pw.sign_stride + w] = 0u;
     }
   }
   __syncthreads();  // every thread has read its tau before alpha overwrites it
-  if (valid) pw.alpha[row] = alpha;
+  if (live) pw.alpha[row] = alpha;
 
   // pass 2: residual per group, absmax scale, codes
   const int pitch2 = G + 1;
@@ -143,8 +159,8 @@ __global__ void __launch_bounds__(kPackRows) k_pack(const float* __restrict__ W,
     const int c0 = g * G;
     load_tile(tile, pitch2, W, N, K, r0, c0, G);
     __syncthreads();
-    if (valid) {
-      const int ncols = min(G, K - c0);
+    if (live) {
+      const int ncols = valid ? min(G, K - c0) : 0;
       const float* t = tile + threadIdx.x * pitch2;
       double a = 0.0;
       for (int j = 0; j < ncols; ++j) {
@@ -155,9 +171,13 @@ __global__ void __launch_bounds__(kPackRows) k_pack(const float* __restrict__ W,
         a = fabs(r) > a ? fabs(r) : a;
       }
       const float s = (float)(a / 127.0);
-      pw.res_scale[(int64_t)row * pw.scale_stride + g] = s;
-      int8_t* qrow = pw.res_q + (int64_t)row * pw.res_stride + c0;
-      for (int j0 = 0; j0 < ncols; j0 += 4) {
+      if (TILED)
+        pw.res_scale[tiled_scale_index(row, g, tpr)] = s;
+      else
+        pw.res_scale[(int64_t)row * pw.scale_stride + g] = s;
+      // tiled: whole 128-channel groups (codes past K are 0)
+      const int nwr = TILED ? G : ncols;
+      for (int j0 = 0; j0 < nwr; j0 += 4) {
         uint32_t word = 0;
         for (int j = j0; j < j0 + 4 && j < ncols; ++j) {
           const float v = t[j];
@@ -166,12 +186,15 @@ __global__ void __launch_bounds__(kPackRows) k_pack(const float* __restrict__ W,
           const int q = quantize_q((double)v - tr, s);
           word |= ((uint32_t)(uint8_t)(int8_t)q) << (8 * (j - j0));
         }
-        *reinterpret_cast<uint32_t*>(qrow + j0) = word;
+        if (TILED)
+          *reinterpret_cast<uint32_t*>(pw.res_q + tiled_code_offset(row, c0 + j0, tpr)) = word;
+        else
+          *reinterpret_cast<uint32_t*>(pw.res_q + (int64_t)row * pw.res_stride + c0 + j0) = word;
       }
     }
     __syncthreads();
   }
-  if (valid) {
+  if (!TILED && valid) {
     // pads: codes K..res_stride (the word loop above already covered up to
     // roundup(K, 4)), scales ng..scale_stride
     int8_t* qrow = pw.res_q + (int64_t)row * pw.res_stride;
@@ -179,8 +202,8 @@ __global__ void __launch_bounds__(kPackRows) k_pack(const float* __restrict__ W,
       *reinterpret_cast<uint32_t*>(qrow + j) = 0u;
     for (int g = ng; g < pw.scale_stride; ++g)
       pw.res_scale[(int64_t)row * pw.scale_stride + g] = 0.0f;
-    if (nonfinite) set_status(status, SQ_ERR_NONFINITE);
   }
+  if (valid && nonfinite) set_status(status, SQ_ERR_NONFINITE);
 }
 
 }  // namespace
@@ -193,11 +216,17 @@ cudaError_t launch_decompose_pack(const float* W, int N, int K, int P, const sq_
     if (e != cudaSuccess) return e;
   }
   const int G = pw.group_size;
+  const bool tiled = pw.layout == SQ_LAYOUT_TILES;
   const size_t smem = (size_t)kPackRows * (G + 1) * sizeof(float);
-  cudaError_t e = ensure_smem_attr((const void*)k_pack, (int)smem);
+  const void* fn = tiled ? (const void*)k_pack<true> : (const void*)k_pack<false>;
+  cudaError_t e = ensure_smem_attr(fn, (int)smem);
   if (e != cudaSuccess) return e;
-  const int blocks = (N + kPackRows - 1) / kPackRows;
-  k_pack<<<blocks, kPackRows, smem, stream>>>(W, N, K, P, G, pw, status);
+  const int64_t rows = tiled ? tiles_rows(N) : N;
+  const int blocks = (int)ceil_div(rows, kPackRows);
+  if (tiled)
+    k_pack<true><<<blocks, kPackRows, smem, stream>>>(W, N, K, P, G, pw, status);
+  else
+    k_pack<false><<<blocks, kPackRows, smem, stream>>>(W, N, K, P, G, pw, status);
   return cudaGetLastError();
 }
 

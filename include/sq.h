@@ -59,31 +59,49 @@ typedef enum {
  * streaming the packed weights at once; it reads every other input and writes
  * every output only after the previous kernel has completed.  Set it only if
  * no earlier work still in flight on the stream writes the packed weights. */
-#define SQ_LAUNCH_CUDA_CORES 2u
-/* SQ_LAUNCH_CUDA_CORES (sq_linear only): run the CUDA-core kernel (dp4a)
- * instead of the tensor-core kernel; same results.  The CUDA-core kernel is
- * also the one used for group sizes 32 and 64. */
+
+/* Packed-weight layouts (sq_packed_weight.layout). */
+#define SQ_LAYOUT_ROWS 0
+#define SQ_LAYOUT_TILES 1
 
 /*
  * Packed weight of one linear layer (N output rows, K input channels).
- * Layout in device memory, all row-major, all rows 16-byte aligned:
- *   sign_bits [N][sign_stride] u32  bit (j % 32) of word (j / 32) is 1 iff
- *                                   W[r][j] >= 0 (so both zeros give 1);
- *                                   pad bits and pad words are 0
- *   mask_bits [N][sign_stride] u32  trunk membership, same bit layout; NULL
- *                                   means every element is in the trunk
- *   alpha     [roundup(N,4)]   f32  per-row trunk scale (entries past N are
- *                                   read as padding of 8-row blocks, never used)
- *   res_q     [N][res_stride]  i8   residual codes in [-127, 127]; pad 0
- *   res_scale [N][scale_stride] f32 residual scale of group g = channels
- *                                   [g*G, g*G + G); pad 0
- * sign_stride  = roundup(ceil(K/32), 4) words
- * res_stride   = roundup(K, 16) bytes
- * scale_stride = roundup(ceil(K/G), 4) floats
+ * The content is the same in both layouts: sign bit b = [W[r][j] >= 0] (so
+ * both zeros give 1), trunk mask bit, per-row trunk scale alpha, residual
+ * code in [-127, 127] and residual scale of group g = channels [g*G, g*G+G).
+ * Pads (bits, codes, scales, alpha) are 0.
+ *
+ * SQ_LAYOUT_ROWS (any G; decoded on the CUDA cores), row-major:
+ *   sign_bits [N][sign_stride] u32  bit (j % 32) of word (j / 32) = channel j
+ *   mask_bits [N][sign_stride] u32  same bit layout; NULL = full trunk
+ *   alpha     [roundup(N,8)]   f32
+ *   res_q     [N][res_stride]  i8
+ *   res_scale [N][scale_stride] f32
+ *   sign_stride = roundup(ceil(K/32), 4), res_stride = roundup(K, 16),
+ *   scale_stride = roundup(ceil(K/G), 4).
+ *
+ * SQ_LAYOUT_TILES (G = 128 only; decoded on the tensor cores): the order in
+ * which the decode kernel streams the weight.  Rows are padded to
+ * N16 = roundup(N, 16) and channels to K128 = roundup(K, 128); tile
+ * t = rb*tpr + g (tpr = K128/128) covers rows [16rb, 16rb+16) and channels
+ * [128g, 128g+128).  Within a tile, lane L = 4*gid + q owns rows
+ * r0 = 16rb + gid, r1 = r0 + 8 and channels 128g + 32q + j (j = 0..31);
+ * word w = j/4 holds channels 4w..4w+3.
+ *   res_q     tile t at byte 2048*t, lane L at +64*L: four 16-byte groups
+ *             m = 0..3 of words {r0 w=2m, r1 w=2m, r0 w=2m+1, r1 w=2m+1}
+ *   sign_bits tile t at word 64*t; lane L: word 2L (row r0), 2L+1 (row r1);
+ *             channel j of the lane's 32 at bit 8*(j%4) + j/4
+ *   mask_bits same as sign_bits; NULL = full trunk
+ *   res_scale tile t at float 16*t, one per row of the row block
+ *   alpha     [N16] f32
+ *   sign_stride = K128/32, res_stride = K128, scale_stride = K128/128
+ *   (the padded row lengths).  K <= 131072.
+ *
  * The arrays may live in one allocation carved by sq_packed_view().
  */
 typedef struct {
   int32_t N, K, group_size;  /* group_size G: 32, 64 or 128 */
+  int32_t layout;            /* SQ_LAYOUT_ROWS or SQ_LAYOUT_TILES */
   int32_t sign_stride;       /* u32 words per row of sign_bits / mask_bits */
   int32_t res_stride;        /* bytes per row of res_q */
   int32_t scale_stride;      /* floats per row of res_scale */
@@ -100,15 +118,17 @@ const char *sq_status_string(sq_status s);
 /* Checks that the current device is sm_100.  SQ_OK or SQ_ERR_UNSUPPORTED_DEVICE. */
 sq_status sq_device_check(void);
 
-/* Bytes of one allocation that holds a packed weight of this shape (the five
- * arrays, each 256-byte aligned inside it).  0 for an unsupported shape. */
-size_t sq_packed_bytes(int32_t N, int32_t K, int32_t group_size, int32_t with_mask);
+/* Bytes of one allocation that holds a packed weight of this shape and
+ * layout (the five arrays, each 256-byte aligned inside it).  0 for an
+ * unsupported shape, group size or layout. */
+size_t sq_packed_bytes(int32_t N, int32_t K, int32_t group_size, int32_t with_mask,
+                       int32_t layout);
 
 /* Fills *out with the strides and with pointers into "base" (device memory of
  * at least sq_packed_bytes() bytes, 256-byte aligned).  Host-only; no device
  * work.  with_mask = 0 leaves mask_bits NULL. */
 sq_status sq_packed_view(void *base, int32_t N, int32_t K, int32_t group_size,
-                         int32_t with_mask, sq_packed_weight *out);
+                         int32_t with_mask, int32_t layout, sq_packed_weight *out);
 
 /*
  * Offline decomposition ("分离阶段（离线完成）", m.lqnn.cn section 5.3; the split of
@@ -147,7 +167,7 @@ sq_status sq_calibrate_outliers(const float *X, int32_t T, int32_t K, int32_t k,
  *   x          [M][K] f32 activations, device
  *   idx        [n_out] i32 outlier channels, strictly ascending in [0, K)
  *              (checked on the device: a violation sets SQ_ERR_INVALID_ARG)
- *   xq         [M][roundup(K,16)] i8 out: codes, 0 on outlier channels and pads
+ *   xq         [M][roundup(K,128)] i8 out: codes, 0 on outlier channels and pads
  *   sx         [M] f32 out: absmax over the non-outlier channels / 127
  *   x_out      [M][n_out] f32 out: the outlier channels, copied
  * 0 <= n_out <= 4096.  Non-finite x sets SQ_ERR_NONFINITE.
@@ -171,12 +191,11 @@ size_t sq_linear_workspace_bytes(const sq_packed_weight *w, int32_t M);
  * kernel; the outlier channels of section 2.2 at full precision).
  *   w           packed weight (device arrays)
  *   xq, sx, x_out, idx, n_out   as written by sq_quantize_act
- *   M           tokens, M >= 1.  Group size 128 runs on the tensor cores
- *               (INT8 MMAs for the residual codes and for the trunk bits
- *               expanded to 0/1 bytes), in passes of up to 8 tokens; group
- *               sizes 32 and 64, or SQ_LAUNCH_CUDA_CORES, run on the CUDA
- *               cores (dp4a), in passes of up to 4 tokens.  The results are
- *               the same.
+ *   M           tokens, M >= 1.  A weight in SQ_LAYOUT_TILES runs on the
+ *               tensor cores (INT8 MMAs for the residual codes and for the
+ *               trunk bits expanded to 0/-1 bytes), in passes of up to 8
+ *               tokens; SQ_LAYOUT_ROWS runs on the CUDA cores (dp4a), in
+ *               passes of up to 4 tokens.  The results are the same.
  *   y           [M][N] f32 out
  *   workspace   device, ws_bytes >= sq_linear_workspace_bytes(w, M)
  * For every token t and row r:
@@ -194,8 +213,8 @@ sq_status sq_linear(const sq_packed_weight *w, const int8_t *xq, const float *sx
  * Same kernels as sq_linear, additionally writing the exact integer
  * accumulators for inspection:
  *   T_out [M][N] i32, R_out [M][N][ceil(K/G)] i32.
- * y is written as by sq_linear.  flags: 0 or SQ_LAUNCH_CUDA_CORES.  Intended
- * for tests; not on the hot path.
+ * y is written as by sq_linear.  flags: 0.  Intended for tests; not on the
+ * hot path.
  */
 sq_status sq_linear_accumulators(const sq_packed_weight *w, const int8_t *xq, const float *sx,
                                  const float *x_out, const int32_t *idx, int32_t n_out,
@@ -211,7 +230,7 @@ sq_status sq_linear_accumulators(const sq_packed_weight *w, const int8_t *xq, co
  *   (16 MiB) per device, inside this library.  Nothing is allocated.
  *   Limit: a call whose sq_linear_workspace_bytes(w, M) exceeds that size
  *   returns SQ_ERR_WORKSPACE before any device work (on a 148-SM B200: more
- *   than 1,769,472 rows).
+ *   than 3,891,200 rows).
  *   First call on each device: looks up the array's device address
  *   (cudaGetSymbolAddress, with that device current) and zero-fills the
  *   array on `stream` before its launch, because the per-row arrival

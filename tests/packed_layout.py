@@ -1,0 +1,95 @@
+"""Reads a packed weight back in row order, for comparison with the oracle.
+
+Independent of the library's code: the index maps below follow the layout as
+include/sq.h documents it.  Row layout: the arrays are row-major already.
+Tiled layout (group size 128): rows padded to 16 and channels to 128; tile
+t = rb * tpr + g; lane L = 4 * (row % 8) + (channel % 128) / 32 of the tile;
+codes: 64 bytes per lane, four groups of words {r0 w=2m, r1 w=2m, r0 w=2m+1,
+r1 w=2m+1}; sign / mask: two words per lane (row r0, row r1), channel j of the
+lane's 32 at bit 8*(j%4) + j/4; scales: 16 per tile (one per row).
+"""
+import numpy as np
+import torch
+
+import decode_matvec_sq_b200 as sq
+
+
+def _tiled_code_offsets(rows: np.ndarray, K128: int) -> np.ndarray:
+    tpr = K128 // 128
+    r = rows.astype(np.int64)[:, None]
+    c = np.arange(K128, dtype=np.int64)[None, :]
+    t = (r >> 4) * tpr + (c >> 7)
+    rr, cc = r & 15, c & 127
+    lane = (rr & 7) * 4 + (cc >> 5)
+    j = cc & 31
+    w = j >> 2
+    return (t * 32 + lane) * 64 + (w >> 1) * 16 + ((w & 1) * 2 + (rr >> 3)) * 4 + (j & 3)
+
+
+def _tiled_word_index(rows: np.ndarray, nwords: int) -> np.ndarray:
+    tpr = nwords // 4
+    r = rows.astype(np.int64)[:, None]
+    word = np.arange(nwords, dtype=np.int64)[None, :]
+    t = (r >> 4) * tpr + (word >> 2)
+    rr = r & 15
+    return (t * 32 + (rr & 7) * 4 + (word & 3)) * 2 + (rr >> 3)
+
+
+def _to_row_bit_order(words: np.ndarray) -> np.ndarray:
+    """Tiled bit order (channel j at bit 8*(j%4) + j/4) -> bit j = channel j."""
+    w = words.astype(np.uint32)
+    out = np.zeros_like(w)
+    for j in range(32):
+        out |= ((w >> np.uint32(8 * (j % 4) + j // 4)) & np.uint32(1)) << np.uint32(j)
+    return out
+
+
+def _gather(flat: torch.Tensor, index: np.ndarray) -> np.ndarray:
+    ix = torch.from_numpy(index.reshape(-1)).to(flat.device)
+    return flat[ix].cpu().numpy().reshape(index.shape)
+
+
+def unpack(pw: "sq.PackedWeight", rows=None) -> dict:
+    """Row-order arrays of the given rows (default: all N rows, plus the pad
+    rows of the tiled layout under key 'pad_rows'):
+      sign, mask: uint32 [n][words] (bit j of word w = channel 32w + j)
+      alpha [n] float32, q [n][Kp] int8, s [n][groups] float32."""
+    if rows is None:
+        rows = np.arange(pw.N)
+    rows = np.asarray(rows, dtype=np.int64)
+    if pw.layout == sq.SQ_LAYOUT_ROWS:
+        sl = torch.as_tensor(rows, device=pw.buf.device)
+        out = {
+            "sign": pw.sign_bits()[sl].cpu().numpy().view(np.uint32),
+            "mask": None if not pw.with_mask else pw.mask_bits()[sl].cpu().numpy().view(np.uint32),
+            "alpha": pw.alpha()[sl].cpu().numpy(),
+            "q": pw.res_q()[sl].cpu().numpy(),
+            "s": pw.res_scale()[sl].cpu().numpy(),
+        }
+        return out
+    K128 = pw.view.res_stride
+    nwords = pw.view.sign_stride
+    code_flat = pw.res_q().reshape(-1)
+    sign_flat = pw.sign_bits().reshape(-1)
+    scale_flat = pw.res_scale().reshape(-1)
+    alpha_all = pw._arr("alpha", torch.float32, (pw.rows,))
+    q = _gather(code_flat, _tiled_code_offsets(rows, K128))
+    wi = _tiled_word_index(rows, nwords)
+    sign = _to_row_bit_order(_gather(sign_flat, wi).view(np.uint32))
+    mask = None
+    if pw.with_mask:
+        mask = _to_row_bit_order(_gather(pw.mask_bits().reshape(-1), wi).view(np.uint32))
+    tpr = K128 // 128
+    si = ((rows[:, None] >> 4) * tpr + np.arange(tpr)[None, :]) * 16 + (rows[:, None] & 15)
+    s = _gather(scale_flat, si)
+    alpha = _gather(alpha_all, rows)
+    return {"sign": sign, "mask": mask, "alpha": alpha, "q": q, "s": s}
+
+
+def pad_rows_are_zero(pw: "sq.PackedWeight") -> bool:
+    """The tiled layout's rows N..roundup(N,16) hold only zeros."""
+    if pw.layout != sq.SQ_LAYOUT_TILES or pw.rows == pw.N:
+        return True
+    u = unpack(pw, rows=np.arange(pw.N, pw.rows))
+    parts = [u["sign"], u["alpha"], u["q"], u["s"]] + ([u["mask"]] if pw.with_mask else [])
+    return all(not np.asarray(a).view(np.uint8).any() for a in parts)

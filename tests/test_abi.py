@@ -49,21 +49,30 @@ def test_status_strings(L):
     assert L.sq_status_string(99) == b"unknown status"
 
 
-@pytest.mark.parametrize("N,K,G,mask", [(1, 1, 128, 0), (7, 33, 32, 1), (512, 512, 128, 0),
-                                        (12288, 4096, 128, 0), (8192, 28672, 64, 1)])
-def test_packed_view_layout(L, N, K, G, mask):
-    nbytes = L.sq_packed_bytes(N, K, G, mask)
+@pytest.mark.parametrize("N,K,G,mask,layout", [
+    (1, 1, 128, 0, 0), (7, 33, 32, 1, 0), (512, 512, 128, 0, 0), (12288, 4096, 128, 0, 0),
+    (8192, 28672, 64, 1, 0), (1, 1, 128, 0, 1), (7, 33, 128, 1, 1), (12288, 4096, 128, 0, 1),
+    (4096, 11008, 128, 1, 1), (8192, 28672, 128, 0, 1)])
+def test_packed_view_layout(L, N, K, G, mask, layout):
+    nbytes = L.sq_packed_bytes(N, K, G, mask, layout)
     assert nbytes > 0
     base = 1 << 40  # a fake 256-aligned address: the view call does not touch memory
     v = sq.SqPackedWeight()
-    assert L.sq_packed_view(ctypes.c_void_p(base), N, K, G, mask, ctypes.byref(v)) == 0
-    assert v.sign_stride == sq.round_up(sq.ceil_div(K, 32), 4)
-    assert v.res_stride == sq.round_up(K, 16)
-    assert v.scale_stride == sq.round_up(sq.ceil_div(K, G), 4)
-    spans = [(v.sign_bits, N * v.sign_stride * 4), (v.alpha, sq.round_up(N, 8) * 4),
-             (v.res_q, N * v.res_stride), (v.res_scale, N * v.scale_stride * 4)]
+    assert L.sq_packed_view(ctypes.c_void_p(base), N, K, G, mask, layout, ctypes.byref(v)) == 0
+    assert v.layout == layout
+    if layout == sq.SQ_LAYOUT_ROWS:
+        rows = N
+        assert v.sign_stride == sq.round_up(sq.ceil_div(K, 32), 4)
+        assert v.res_stride == sq.round_up(K, 16)
+        assert v.scale_stride == sq.round_up(sq.ceil_div(K, G), 4)
+    else:
+        rows = sq.round_up(N, 16)
+        assert v.res_stride == sq.round_up(K, 128)
+        assert v.sign_stride == v.res_stride // 32 and v.scale_stride == v.res_stride // 128
+    spans = [(v.sign_bits, rows * v.sign_stride * 4), (v.alpha, sq.round_up(rows, 8) * 4),
+             (v.res_q, rows * v.res_stride), (v.res_scale, rows * v.scale_stride * 4)]
     if mask:
-        spans.append((v.mask_bits, N * v.sign_stride * 4))
+        spans.append((v.mask_bits, rows * v.sign_stride * 4))
     else:
         assert v.mask_bits is None
     spans.sort()
@@ -74,17 +83,22 @@ def test_packed_view_layout(L, N, K, G, mask):
 
 def test_packed_view_rejects(L):
     v = sq.SqPackedWeight()
-    assert L.sq_packed_view(ctypes.c_void_p((1 << 40) + 16), 8, 8, 128, 0, ctypes.byref(v)) == 3
-    assert L.sq_packed_view(ctypes.c_void_p(1 << 40), 8, 8, 48, 0, ctypes.byref(v)) == 2
-    assert L.sq_packed_view(ctypes.c_void_p(1 << 40), 0, 8, 128, 0, ctypes.byref(v)) == 2
-    assert L.sq_packed_view(None, 8, 8, 128, 0, ctypes.byref(v)) == 1
-    assert L.sq_packed_bytes(8, 8, 100, 0) == 0
+    assert L.sq_packed_view(ctypes.c_void_p((1 << 40) + 16), 8, 8, 128, 0, 0, ctypes.byref(v)) == 3
+    assert L.sq_packed_view(ctypes.c_void_p(1 << 40), 8, 8, 48, 0, 0, ctypes.byref(v)) == 2
+    assert L.sq_packed_view(ctypes.c_void_p(1 << 40), 0, 8, 128, 0, 0, ctypes.byref(v)) == 2
+    assert L.sq_packed_view(None, 8, 8, 128, 0, 0, ctypes.byref(v)) == 1
+    assert L.sq_packed_view(ctypes.c_void_p(1 << 40), 8, 8, 128, 0, 2, ctypes.byref(v)) == 1
+    # the tiled layout: group size 128 only, K <= 131072
+    assert L.sq_packed_view(ctypes.c_void_p(1 << 40), 8, 8, 64, 0, 1, ctypes.byref(v)) == 2
+    assert L.sq_packed_view(ctypes.c_void_p(1 << 40), 8, 131073, 128, 0, 1, ctypes.byref(v)) == 2
+    assert L.sq_packed_bytes(8, 8, 100, 0, 0) == 0
+    assert L.sq_packed_bytes(8, 8, 64, 0, 1) == 0
 
 
 def test_host_validation_before_device_work(L):
     """Each of these returns from the host checks; no kernel is launched."""
     v = sq.SqPackedWeight()
-    L.sq_packed_view(ctypes.c_void_p(1 << 40), 64, 256, 128, 0, ctypes.byref(v))
+    L.sq_packed_view(ctypes.c_void_p(1 << 40), 64, 256, 128, 0, 1, ctypes.byref(v))
     p = ctypes.c_void_p(1 << 41)
     bad = ctypes.c_void_p((1 << 41) + 4)
     # sq_linear(w, xq, sx, x_out, idx, n_out, M, y, ws, ws_bytes, status, flags, stream)
@@ -93,6 +107,10 @@ def test_host_validation_before_device_work(L):
     assert L.sq_linear(ctypes.byref(v), p, p, p, p, 1, 0, p, p, 1 << 20, None, 0, None) == 2
     assert L.sq_linear(ctypes.byref(v), bad, p, p, p, 1, 1, p, p, 1 << 20, None, 0, None) == 3
     assert L.sq_linear(ctypes.byref(v), p, p, p, p, 1, 1, p, p, 1 << 20, None, 8, None) == 1
+    assert L.sq_linear(ctypes.byref(v), p, p, p, p, 1, 1, p, p, 1 << 20, None, 2, None) == 1
+    w3 = sq.SqPackedWeight.from_buffer_copy(v)
+    w3.layout = 5
+    assert L.sq_linear(ctypes.byref(w3), p, p, p, p, 1, 1, p, p, 1 << 20, None, 0, None) == 1
     assert L.sq_linear(ctypes.byref(v), p, p, None, p, 1, 1, p, p, 1 << 20, None, 0, None) == 1
     w2 = sq.SqPackedWeight.from_buffer_copy(v)
     w2.res_stride = 100

@@ -13,6 +13,7 @@ import torch
 
 import decode_matvec_sq_b200 as sq
 import oracle
+from tests import packed_layout
 import synth
 import synth.device as sdev
 from synth import workloads as wl
@@ -30,34 +31,38 @@ def built(cuda_device):
     yield
 
 
-def unpack_words(words: torch.Tensor, K: int):
-    a = words.cpu().numpy().astype(np.int32).view(np.uint8)
-    bits = np.unpackbits(a, axis=1, bitorder="little")
+def _bits(words: np.ndarray, K: int):
+    """uint32 words in row bit order -> (bits of channels < K, pad bits)."""
+    bits = np.unpackbits(np.ascontiguousarray(words).view(np.uint8), axis=1, bitorder="little")
     return bits[:, :K], bits[:, K:]
 
 
+def _layout(tc: bool, G: int = 128) -> int:
+    return sq.SQ_LAYOUT_TILES if (tc and G == 128) else sq.SQ_LAYOUT_ROWS
+
+
 def check_packed(pw: sq.PackedWeight, d: dict, rows=None):
-    """GPU packed weight (optionally only `rows`) == oracle decomposition d."""
+    """GPU packed weight (optionally only `rows`) == oracle decomposition d,
+    read back in row order from either layout; pads are zero."""
     K = pw.K
-    sl = slice(None) if rows is None else torch.as_tensor(rows, device="cuda")
-    sign, sign_pad = unpack_words(pw.sign_bits()[sl], K)
+    u = packed_layout.unpack(pw, rows)
+    sign, sign_pad = _bits(u["sign"], K)
     assert np.array_equal(sign, d["sign"]), "sign bits"
     assert not sign_pad.any(), "sign pad bits"
     if pw.with_mask:
-        mask, mask_pad = unpack_words(pw.mask_bits()[sl], K)
+        mask, mask_pad = _bits(u["mask"], K)
         assert np.array_equal(mask, d["mask"]), "mask bits"
         assert not mask_pad.any()
     else:
         assert d["mask"].all()
-    alpha = pw.alpha()[sl].cpu().numpy()
-    assert np.array_equal(alpha.view(np.uint32), d["alpha"].view(np.uint32)), "alpha"
-    q = pw.res_q()[sl].cpu().numpy()
-    assert np.array_equal(q[:, :K], d["q"]), "residual codes"
-    assert not q[:, K:].any()
-    s = pw.res_scale()[sl].cpu().numpy()
+    assert np.array_equal(u["alpha"].view(np.uint32), d["alpha"].view(np.uint32)), "alpha"
+    assert np.array_equal(u["q"][:, :K], d["q"]), "residual codes"
+    assert not u["q"][:, K:].any()
     ng = d["s"].shape[1]
-    assert np.array_equal(s[:, :ng].view(np.uint32), d["s"].view(np.uint32)), "group scales"
-    assert not s[:, ng:].any()
+    assert np.array_equal(u["s"][:, :ng].view(np.uint32), d["s"].view(np.uint32)), "group scales"
+    assert not u["s"][:, ng:].any()
+    if rows is None:
+        assert packed_layout.pad_rows_are_zero(pw), "pad rows of the tiled layout"
 
 
 def check_y(y, y_ref, bound, what="y"):
@@ -72,10 +77,10 @@ def run_path(W: np.ndarray, x: np.ndarray, idx: np.ndarray, P=-1, G=128, pdl=Fal
     xd = torch.from_numpy(x).cuda()
     idxd = torch.from_numpy(idx.astype(np.int32)).cuda()
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    pw = sq.decompose_pack(Wd, trunk_percent=P, group_size=G, status=status)
+    pw = sq.decompose_pack(Wd, trunk_percent=P, group_size=G, layout=_layout(tc, G), status=status)
     act = sq.quantize_act(xd, idxd, status=status, pdl=pdl)
     xq, sx, xo = act
-    y, T, R = sq.linear_accumulators(pw, xq, sx, xo, idxd, status=status, cuda_cores=not tc)
+    y, T, R = sq.linear_accumulators(pw, xq, sx, xo, idxd, status=status)
     torch.cuda.synchronize()
     assert status.item() == 0
     return pw, act, (y, T, R)
@@ -122,16 +127,16 @@ def test_device_generator_matches_host():
 
 @pytest.mark.parametrize("N,K", [(1, 8), (7, 33), (8, 100), (13, 128), (9, 129), (64, 512),
                                  (513, 300), (16, 4096), (3, 1000)])
-@pytest.mark.parametrize("G", [32, 64, 128])
+@pytest.mark.parametrize("G,layout", [(32, 0), (64, 0), (128, 0), (128, 1)])
 @pytest.mark.parametrize("P", [-1, 60])
-def test_pack_parity_shapes(N, K, G, P):
+def test_pack_parity_shapes(N, K, G, layout, P):
     rng = np.random.default_rng(N * 1000 + K + G + P)
     W = rng.laplace(0, 0.02, (N, K)).astype(np.float32)
     W[0, : min(K, 5)] = np.array([0.0, -0.0, 1e-30, -1e-30, 0.5], np.float32)[: min(K, 5)]
     if N > 2:
         W[1] = 0.0                                   # all-zero row: alpha 0, codes 0
         W[2, : K // 2] = np.round(W[2, : K // 2], 2)  # ties for the percentile
-    pw = sq.decompose_pack(torch.from_numpy(W).cuda(), trunk_percent=P, group_size=G)
+    pw = sq.decompose_pack(torch.from_numpy(W).cuda(), trunk_percent=P, group_size=G, layout=layout)
     torch.cuda.synchronize()
     check_packed(pw, oracle.decompose(W, G=G, P=P))
 
@@ -278,15 +283,14 @@ def test_linear_deterministic_and_split_rows(tc):
     x = rng.standard_normal((1, 28672)).astype(np.float32)
     idx = np.sort(rng.choice(28672, 72, replace=False)).astype(np.int32)
     Wd, xd, idxd = (torch.from_numpy(a).cuda() for a in (W, x, idx))
-    pw = sq.decompose_pack(Wd)
+    pw = sq.decompose_pack(Wd, layout=_layout(tc))
     act = sq.quantize_act(xd, idxd)
     xq, sx, xo = act
     ws = sq.new_workspace(pw, 1)
     ys = []
     for _ in range(5):
         y = torch.full((1, 8), float("nan"), device="cuda")
-        ys.append(sq.linear(pw, xq, sx, xo, idxd, y=y, workspace=ws,
-                            cuda_cores=not tc).cpu().numpy())
+        ys.append(sq.linear(pw, xq, sx, xo, idxd, y=y, workspace=ws).cpu().numpy())
     torch.cuda.synchronize()
     for y in ys[1:]:
         assert np.array_equal(y.view(np.uint32), ys[0].view(np.uint32))
@@ -349,13 +353,13 @@ def _sampled_layer(L, M, rows, pdl=False, tc=True):
     Xc = sdev.fill_activations(L, torch.empty(wl.CAL_TOKENS, L.K, device="cuda"), synth.STREAM_XCAL)
     xd = sdev.fill_activations(L, torch.empty(M, L.K, device="cuda"))
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
-    pw = sq.decompose_pack(Wd, trunk_percent=L.trunk_percent, status=st)
+    pw = sq.decompose_pack(Wd, trunk_percent=L.trunk_percent, layout=_layout(tc), status=st)
     del Wd
     idx = sq.calibrate_outliers(Xc, L.n_out, status=st)
     xq, sx, xo = sq.quantize_act(xd, idx, status=st, pdl=pdl)
-    y, T, R = sq.linear_accumulators(pw, xq, sx, xo, idx, status=st, cuda_cores=not tc)
+    y, T, R = sq.linear_accumulators(pw, xq, sx, xo, idx, status=st)
     y2 = torch.full_like(y, float("nan"))
-    sq.linear(pw, xq, sx, xo, idx, y=y2, status=st, pdl=pdl, cuda_cores=not tc)
+    sq.linear(pw, xq, sx, xo, idx, y=y2, status=st, pdl=pdl)
     torch.cuda.synchronize()
     assert st.item() == 0
     assert torch.equal(y, y2)
@@ -441,7 +445,7 @@ def test_shared_workspace_across_shapes(tc):
     items = []
     for L in layers:
         Wd = sdev.fill_weights(L, torch.empty(L.N, L.K, device="cuda"))
-        pw = sq.decompose_pack(Wd)
+        pw = sq.decompose_pack(Wd, layout=_layout(tc))
         del Wd
         idx = torch.from_numpy(L.planted_channels()).cuda()
         x = sdev.fill_activations(L, torch.empty(1, L.K, device="cuda"))
@@ -452,8 +456,7 @@ def test_shared_workspace_across_shapes(tc):
     for rep in range(3):
         for L, pw, idx, a in items[::(1 if rep % 2 == 0 else -1)]:
             y = torch.full((1, L.N), float("nan"), device="cuda")
-            sq.linear(pw, a[0], a[1], a[2], idx, y=y, workspace=ws, status=st,
-                      cuda_cores=not tc)
+            sq.linear(pw, a[0], a[1], a[2], idx, y=y, workspace=ws, status=st)
             torch.cuda.synchronize()
             assert not torch.isnan(y).any().item(), f"{L.name}: rows not written"
             if L.name in outs:
@@ -479,7 +482,7 @@ def test_fewer_work_units_than_warps(N, K, tc):
     rng = np.random.default_rng(N * K)
     W = rng.laplace(0, 0.02, (N, K)).astype(np.float32)
     x = rng.standard_normal((2, K)).astype(np.float32)
-    pw = sq.decompose_pack(torch.from_numpy(W).cuda())
+    pw = sq.decompose_pack(torch.from_numpy(W).cuda(), layout=_layout(tc))
     act = sq.quantize_act(torch.from_numpy(x).cuda(), None)
     ws = sq.new_workspace(pw, 2)
     d = oracle.decompose(W)
@@ -487,7 +490,7 @@ def test_fewer_work_units_than_warps(N, K, tc):
     y_ref = oracle.linear(d, oxq, osx, oxo, np.zeros(0, np.int32))
     for _ in range(2):
         y = torch.full((2, N), float("nan"), device="cuda")
-        sq.linear(pw, act[0], act[1], act[2], None, y=y, workspace=ws, cuda_cores=not tc)
+        sq.linear(pw, act[0], act[1], act[2], None, y=y, workspace=ws)
         torch.cuda.synchronize()
         check_y(y.cpu().numpy(), y_ref, oracle.abs_dot(W, x))
         assert not sq.workspace_counters(ws, pw, 2).any().item()

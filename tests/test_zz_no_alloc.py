@@ -29,23 +29,23 @@ def _bound(W, x):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("N,K,M,n_out,P,cuda_cores", [
-    (512, 512, 1, 4, -1, False),       # the single-layer workload's shape
-    (4096, 4096, 1, 20, -1, False),    # rows shared between warps (counters used)
-    (1000, 1000, 3, 9, 60, False),     # threshold trunk, ragged K, 3 tokens
-    (777, 2048, 5, 10, -1, True),      # CUDA-core kernel, two passes of tokens
+@pytest.mark.parametrize("N,K,M,n_out,P,layout", [
+    (512, 512, 1, 4, -1, 1),           # the single-layer workload's shape
+    (4096, 4096, 1, 20, -1, 1),        # rows shared between warps and CTAs
+    (1000, 1000, 3, 9, 60, 1),         # threshold trunk, ragged K, 3 tokens
+    (777, 2048, 5, 10, -1, 0),         # row layout: CUDA-core kernel, two passes
 ])
-def test_noalloc_matches_sq_linear_twice(cuda_device, N, K, M, n_out, P, cuda_cores):
+def test_noalloc_matches_sq_linear_twice(cuda_device, N, K, M, n_out, P, layout):
     W, x, idx = _inputs(N, K, M, n_out, seed=N + K + M)
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
-    pw = sq.decompose_pack(torch.from_numpy(W).cuda(), trunk_percent=P, status=st)
+    pw = sq.decompose_pack(torch.from_numpy(W).cuda(), trunk_percent=P, layout=layout, status=st)
     idxd = torch.from_numpy(idx).cuda()
     xq, sx, xo = sq.quantize_act(torch.from_numpy(x).cuda(), idxd, status=st)
-    y_ref = sq.linear(pw, xq, sx, xo, idxd, status=st, cuda_cores=cuda_cores)
+    y_ref = sq.linear(pw, xq, sx, xo, idxd, status=st)
     ys = []
     for _ in range(2):
         y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
-        sq.linear_noalloc(pw, xq, sx, xo, idxd, y, status=st, cuda_cores=cuda_cores)
+        sq.linear_noalloc(pw, xq, sx, xo, idxd, y, status=st)
         ys.append(y)
     torch.cuda.synchronize()
     assert st.item() == 0
@@ -63,9 +63,9 @@ def test_noalloc_rejects_problems_beyond_its_scratch(cuda_device):
     the host checks, before any device work (the view's pointers are never
     dereferenced)."""
     L = sq.lib()
-    N, K = 4_000_000, 128
+    N, K = 8_000_000, 128
     v = sq.SqPackedWeight()
-    assert L.sq_packed_view(ctypes.c_void_p(1 << 40), N, K, 128, 0, ctypes.byref(v)) == 0
+    assert L.sq_packed_view(ctypes.c_void_p(1 << 40), N, K, 128, 0, 1, ctypes.byref(v)) == 0
     need = L.sq_linear_workspace_bytes(ctypes.byref(v), 1)
     assert need > sq.NOALLOC_SCRATCH_BYTES
     p = ctypes.c_void_p(1 << 41)
