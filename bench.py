@@ -3,8 +3,9 @@
 
 One step = one token through 32 layers x {qkv 4096->12288, o 4096->4096,
 gate_up 4096->22016, down 11008->4096}: for each of the 128 linears the
-activation split (sq_quantize_act) and the fused linear (sq_linear), all in
-one CUDA graph with programmatic dependent launch.  Weights are packed once
+activation split and the linear layer in one kernel (sq_quantize_linear;
+--two-kernels: sq_quantize_act then sq_linear), all in one CUDA graph with
+programmatic dependent launch.  Weights are packed once
 (offline) and resident in HBM; the 7.5 GB they take per step exceed the
 126 MB L2 many times over, so no flush is needed between steps.
 
@@ -246,13 +247,14 @@ def config_dict(args):
 # ---- GPU arm -----------------------------------------------------------------------
 
 class Stack:
-    def __init__(self, layers, device, pdl=True):
+    def __init__(self, layers, device, pdl=True, fused=True):
         import torch
         import decode_matvec_sq_b200 as sq
         import synth
         import synth.device as sdev
         self.layers = layers
         self.pdl = pdl
+        self.fused = fused
         maxw = max(L.N * L.K for L in layers)
         scratch = torch.empty(maxw, dtype=torch.float32, device=device)
         cal = torch.empty(64 * max(L.K for L in layers), dtype=torch.float32, device=device)
@@ -291,13 +293,22 @@ class Stack:
         if self.ws.numel() < need:
             self.ws = torch.zeros(need, dtype=torch.uint8, device=device)
 
+    @property
+    def launches_per_step(self) -> int:
+        return len(self.layers) * (1 if self.fused else 2)
+
     def step(self, pdl=None):
+        """One token through the stack: per linear, the activation split and the
+        fused linear layer (one kernel, or two with fused=False)."""
         import decode_matvec_sq_b200 as sq
         pdl = self.pdl if pdl is None else pdl
         for pw, x, idx, a, y in zip(self.pws, self.xs, self.idx, self.bufs, self.ys):
-            sq.quantize_act(x, idx, xq=a[0], sx=a[1], x_out=a[2], status=self.status, pdl=pdl)
-            sq.linear(pw, a[0], a[1], a[2], idx, y=y, workspace=self.ws, status=self.status,
-                      pdl=pdl)
+            if self.fused:
+                sq.quantize_linear(pw, x, idx, y=y, workspace=self.ws, status=self.status, pdl=pdl)
+            else:
+                sq.quantize_act(x, idx, xq=a[0], sx=a[1], x_out=a[2], status=self.status, pdl=pdl)
+                sq.linear(pw, a[0], a[1], a[2], idx, y=y, workspace=self.ws, status=self.status,
+                          pdl=pdl)
 
     def capture(self):
         import torch
@@ -314,36 +325,55 @@ class Stack:
         return g
 
     def time_linear_launches(self, reps: int):
-        """Average device duration of each fused-linear launch (events on the
-        launching stream), launched one by one without PDL."""
+        """Average device duration of the linear-layer kernel per shape: for each
+        shape, a CUDA graph of its launches over all layers (different weights,
+        no PDL), replayed `reps` times between events on the replay stream."""
         import torch
         import decode_matvec_sq_b200 as sq
+        groups = {}
+        for i, L in enumerate(self.layers):
+            groups.setdefault(L.name.split(".")[-1], []).append(i)
+        s = torch.cuda.Stream()
         per_shape = {}
-        evs = []
-        stream = torch.cuda.current_stream()
-        for _ in range(reps):
-            for pw, idx, act, y, L in zip(self.pws, self.idx, self.bufs, self.ys, self.layers):
+        tot_ms, tot_bytes = 0.0, 0
+        for key, ids in groups.items():
+            def launch():
+                for i in ids:
+                    if self.fused:
+                        sq.quantize_linear(self.pws[i], self.xs[i], self.idx[i], y=self.ys[i],
+                                           workspace=self.ws, status=self.status)
+                    else:
+                        a = self.bufs[i]
+                        sq.linear(self.pws[i], a[0], a[1], a[2], self.idx[i], y=self.ys[i],
+                                  workspace=self.ws, status=self.status)
+            s.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(s):
+                launch()
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=s):
+                launch()
+            with torch.cuda.stream(s):
+                g.replay()
                 a = torch.cuda.Event(enable_timing=True)
                 b = torch.cuda.Event(enable_timing=True)
-                a.record(stream)
-                sq.linear(pw, act[0], act[1], act[2], idx, y=y, workspace=self.ws,
-                          status=self.status)
-                b.record(stream)
-                evs.append((L, a, b))
-        torch.cuda.synchronize()
-        tot_ms, tot_bytes = 0.0, 0
-        for L, a, b in evs:
+                a.record(s)
+                for _ in range(reps):
+                    g.replay()
+                b.record(s)
+            torch.cuda.synchronize()
             ms = a.elapsed_time(b)
-            key = L.name.split(".")[-1]
-            d = per_shape.setdefault(key, [0.0, 0, 0])
-            d[0] += ms
-            d[1] += 1
-            d[2] += linear_weight_bytes(L) + linear_act_bytes(L)
+            n = reps * len(ids)
+            nbytes = sum(linear_weight_bytes(self.layers[i]) + linear_act_bytes(self.layers[i])
+                         for i in ids) * reps
+            per_shape[key] = [ms, n, nbytes]
             tot_ms += ms
-            tot_bytes += linear_weight_bytes(L) + linear_act_bytes(L)
+            tot_bytes += nbytes
+            del g
         shapes = {k: {"us": round(v[0] / v[1] * 1e3, 2),
                       "gbs": round(v[2] / (v[0] * 1e-3) / 1e9, 1)} for k, v in per_shape.items()}
-        return tot_bytes / len(evs), tot_ms / len(evs), shapes
+        n_launch = sum(v[1] for v in per_shape.values())
+        return tot_bytes / n_launch, tot_ms / n_launch, shapes
 
 
 def run_gpu(args, world, rank, local):
@@ -368,10 +398,10 @@ def run_gpu(args, world, rank, local):
     sq.device_check()
 
     layers = wl.config2(args.layers)
-    stack = Stack(layers, device, pdl=not args.no_pdl)
+    stack = Stack(layers, device, pdl=not args.no_pdl, fused=not args.two_kernels)
     graph = stack.capture()
     nbytes = step_bytes(layers)
-    launches_per_step = 2 * len(layers)
+    launches_per_step = stack.launches_per_step
 
     stream = torch.cuda.current_stream()
     for _ in range(args.warmup):
@@ -463,7 +493,8 @@ def run_gpu(args, world, rank, local):
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                          "unit": "GB/s", "frac": round(achieved / peak, 4),
                          "peak_kind": peak_kind, "traffic": traffic,
-                         "kernel": "k_linear_tc (sq_linear decode, tensor cores)",
+                         "kernel": "k_linear_tc (activation split + decode linear, tensor cores)"
+                                   if stack.fused else "k_linear_tc (decode linear, tensor cores)",
                          "bytes_per_launch": int(bytes_launch),
                          "us_per_launch": round(ms_launch * 1e3, 3), "per_shape": shapes},
             "clocks": clocks,
@@ -481,7 +512,7 @@ def run_gpu(args, world, rank, local):
 def kernel_hash() -> str:
     import hashlib
     h = hashlib.sha256()
-    for f in ("sq_linear_tc.cu", "sq_common.cuh", "sq_internal.h"):
+    for f in ("sq_linear_tc.cu", "sq_common.cuh", "sq_internal.h", "sq_quant.cuh", "sq_layout.h"):
         with open(os.path.join(ROOT, "decode_matvec_sq_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -495,6 +526,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["sq", "reference"], default="sq")
     ap.add_argument("--layers", type=int, default=32)
     ap.add_argument("--no-pdl", action="store_true")
+    ap.add_argument("--two-kernels", action="store_true",
+                    help="activation split and linear layer as two kernels per linear")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--oracle-rows", type=int, default=256)

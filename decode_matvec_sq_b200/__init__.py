@@ -77,6 +77,7 @@ def lib():
         "sq_linear_accumulators": ([pw, vp, vp, vp, vp, i32, i32, vp, vp, vp, vp, sz, vp, u32, vp],
                                    ctypes.c_int),
         "sq_linear_noalloc": ([pw, vp, vp, vp, vp, i32, i32, vp, vp, u32, vp], ctypes.c_int),
+        "sq_quantize_linear": ([pw, vp, i32, vp, i32, vp, vp, sz, vp, u32, vp], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -274,6 +275,23 @@ def linear(pw: PackedWeight, xq, sx, x_out, idx, y=None, workspace=None, status=
                         _ptr(idx) if n else None, n, M, _ptr(y), _ptr(workspace),
                         workspace.numel(), _ptr(status), _flags(pdl),
                         _stream(stream)), "sq_linear")
+    return y
+
+
+def quantize_linear(pw: PackedWeight, x, idx, y=None, workspace=None, status=None,
+                    pdl: bool = False, stream=None):
+    """y[M][N] from fp32 activations x[M][K]: the activation split and the
+    linear layer in one kernel (tiled layout)."""
+    import torch
+    M = x.shape[0]
+    n = 0 if idx is None else int(idx.numel())
+    if y is None:
+        y = torch.empty(M, pw.N, dtype=torch.float32, device=x.device)
+    if workspace is None:
+        workspace = new_workspace(pw, M)
+    _ck(lib().sq_quantize_linear(ctypes.byref(pw.view), _ptr(x), M, _ptr(idx) if n else None, n,
+                                 _ptr(y), _ptr(workspace), workspace.numel(), _ptr(status),
+                                 _flags(pdl), _stream(stream)), "sq_quantize_linear")
     return y
 
 

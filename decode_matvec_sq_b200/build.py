@@ -35,6 +35,7 @@ SOURCES = [
     ("sq_linear.cu", []),
     ("sq_linear_tc.cu", []),
     ("sq_noalloc.cu", []),
+    ("sq_prefill.cu", []),
 ]
 
 

@@ -12,29 +12,13 @@
 
 #include "sq_common.cuh"
 #include "sq_internal.h"
+#include "sq_quant.cuh"
 
 namespace sq {
 namespace {
 
 constexpr int kActThreads = 1024;
 constexpr int kCalThreads = 1024;
-
-// round_half_away(|v| / s) decided exactly.  t = |v| * (1/s) is within far
-// less than 0.5 of the true quotient Q, so with k = floor(t) the exact test
-// Q >= k + 1/2  <=>  2|v| >= (2k+1)*s  (both sides exact in binary64: 2k+1
-// has at most 9 bits, s 24) yields the correctly rounded code whether Q lies
-// in [k, k+1) or just outside it.  Identical to rounding the exactly
-// rounded binary64 quotient v/s, which for float v and s never lands on the
-// wrong side of a midpoint.
-__device__ __forceinline__ int quantize_exact(float v, float s, double rinv) {
-  if (s == 0.0f) return 0;
-  const double av = fabs((double)v);
-  const double k = floor(av * rinv);
-  double q = (av + av >= (k + k + 1.0) * (double)s) ? k + 1.0 : k;
-  q = q < 127.0 ? q : 127.0;
-  const int qi = (int)q;
-  return v < 0.0f ? -qi : qi;
-}
 
 // One CTA per token; warp w handles the 32-channel chunks w, w + 32, ...
 // with one channel per lane, keeping its x values in registers between the
@@ -105,8 +89,8 @@ __global__ void __launch_bounds__(kActThreads) k_quantize_act(
   a = warp_max[lane];
   for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
 
-  const float s = (float)((double)a / 127.0);
-  const double rinv = s != 0.0f ? 1.0 / (double)s : 0.0;
+  const float s = act_scale(a);
+  const double rinv = act_rinv(s);
   if (threadIdx.x == 0) sx[t] = s;
 
   int8_t* qt = xq + (int64_t)t * Kx;

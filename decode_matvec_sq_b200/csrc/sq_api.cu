@@ -283,6 +283,12 @@ static sq_status linear_common(const sq_packed_weight* w, const int8_t* xq, cons
     if (e != cudaSuccess) return SQ_ERR_CUDA;
   }
   const int ng = (int)ceil_div(w->K, w->group_size);
+  if (w->layout == SQ_LAYOUT_ROWS && M >= kPrefillMinTokens && prefill_supported(*w)) {
+    // many tokens: one tcgen05 GEMM-shaped launch over all of them
+    const cudaError_t e = launch_prefill(*w, M, xq, sx, x_out, idx, n_out, y, T_out, R_out,
+                                         dev_status, s);
+    return e == cudaSuccess ? SQ_OK : SQ_ERR_CUDA;
+  }
   const bool tc = w->layout == SQ_LAYOUT_TILES;
   const int per_pass = tc ? kMaxTokensPerPassTc : kMaxTokensPerPass;
   const int64_t xs = xq_stride_of(w->K);
@@ -295,8 +301,8 @@ static sq_status linear_common(const sq_packed_weight* w, const int8_t* xq, cons
     int32_t* R_t = R_out ? R_out + (int64_t)t0 * w->N * ng : nullptr;
     cudaError_t e;
     if (tc) {
-      e = launch_linear_tc(*w, m, xq_t, sx + t0, xo_t, idx, n_out, y_t, T_t, R_t, workspace, part,
-                           d.sm_count, (flags & SQ_LAUNCH_PDL) != 0, s);
+      e = launch_linear_tc(*w, m, xq_t, sx + t0, xo_t, nullptr, idx, n_out, y_t, T_t, R_t,
+                           workspace, part, d.sm_count, dev_status, (flags & SQ_LAUNCH_PDL) != 0, s);
     } else {
       LinearPlan plan;
       if (!plan_linear(*w, m, n_out, d.sm_count, &plan)) return SQ_ERR_SHAPE;
@@ -327,6 +333,38 @@ sq_status sq_linear_accumulators(const sq_packed_weight* w, const int8_t* xq, co
   if (flags & SQ_LAUNCH_PDL) return SQ_ERR_INVALID_ARG;
   return linear_common(w, xq, sx, x_out, idx, n_out, M, y, T_out, R_out, workspace, ws_bytes,
                        dev_status, flags, stream);
+}
+
+sq_status sq_quantize_linear(const sq_packed_weight* w, const float* x, int32_t M,
+                             const int32_t* idx, int32_t n_out, float* y, void* workspace,
+                             size_t ws_bytes, int32_t* dev_status, uint32_t flags, void* stream) {
+  sq_status st = check_weight(w);
+  if (st != SQ_OK) return st;
+  if (!x || !y) return SQ_ERR_INVALID_ARG;
+  if (w->layout != SQ_LAYOUT_TILES) return SQ_ERR_SHAPE;
+  if (M < 1 || M > (1 << 20)) return SQ_ERR_SHAPE;
+  if (n_out < 0 || n_out > kMaxOutliers || n_out > w->K) return SQ_ERR_SHAPE;
+  if (n_out > 0 && !idx) return SQ_ERR_INVALID_ARG;
+  if (flags & ~SQ_LAUNCH_PDL) return SQ_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(y) || (n_out > 0 && !aligned16(idx)) ||
+      (workspace && !aligned16(workspace)))
+    return SQ_ERR_ALIGN;
+  const int per_pass = linear_tc_fused_tokens(*w, n_out);
+  if (per_pass < 1) return SQ_ERR_SHAPE;
+  DeviceInfo d;
+  if ((st = check_device(&d)) != SQ_OK) return st;
+  const size_t need = linear_workspace_bytes(*w, M, d.sm_count);
+  if (!workspace || ws_bytes < need) return SQ_ERR_WORKSPACE;
+  const size_t part = linear_part_bytes(d.sm_count);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  for (int t0 = 0; t0 < M; t0 += per_pass) {
+    const int m = std::min(per_pass, M - t0);
+    cudaError_t e = launch_linear_tc(*w, m, nullptr, nullptr, nullptr, x + (int64_t)t0 * w->K, idx,
+                                     n_out, y + (int64_t)t0 * w->N, nullptr, nullptr, workspace,
+                                     part, d.sm_count, dev_status, (flags & SQ_LAUNCH_PDL) != 0, s);
+    if (e != cudaSuccess) return SQ_ERR_CUDA;
+  }
+  return SQ_OK;
 }
 
 }  // extern "C"

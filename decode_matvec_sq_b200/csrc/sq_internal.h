@@ -71,10 +71,22 @@ cudaError_t launch_linear(const sq_packed_weight& w, const LinearPlan& plan, con
                           size_t part_bytes, int32_t* status, bool pdl, cudaStream_t stream);
 
 // Tensor-core decode kernel (SQ_LAYOUT_TILES), up to kMaxTokensPerPassTc tokens.
+// With x != NULL (fused mode) it performs the activation split of x itself
+// (xq, sx, x_out unused) for at most linear_tc_fused_tokens() tokens.
 size_t linear_tc_part_bytes(int sm_count);
+int linear_tc_fused_tokens(const sq_packed_weight& w, int n_out);
 cudaError_t launch_linear_tc(const sq_packed_weight& w, int M, const int8_t* xq, const float* sx,
-                             const float* x_out, const int32_t* idx, int n_out, float* y,
-                             int32_t* T_out, int32_t* R_out, void* workspace, size_t part_bytes,
-                             int sm_count, bool pdl, cudaStream_t stream);
+                             const float* x_out, const float* x, const int32_t* idx, int n_out,
+                             float* y, int32_t* T_out, int32_t* R_out, void* workspace,
+                             size_t part_bytes, int sm_count, int32_t* status, bool pdl,
+                             cudaStream_t stream);
+
+// Prefill kernel (SQ_LAYOUT_ROWS, group size 128, many tokens): tcgen05 int8
+// MMAs with TMEM accumulators.  T_out / R_out optional (both or neither).
+constexpr int kPrefillMinTokens = 64;
+bool prefill_supported(const sq_packed_weight& w);
+cudaError_t launch_prefill(const sq_packed_weight& w, int M, const int8_t* xq, const float* sx,
+                           const float* x_out, const int32_t* idx, int n_out, float* y,
+                           int32_t* T_out, int32_t* R_out, int32_t* status, cudaStream_t stream);
 
 }  // namespace sq

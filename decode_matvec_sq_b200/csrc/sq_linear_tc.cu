@@ -28,6 +28,11 @@
 // barrier; one shared by CTAs is summed by its last arriving CTA from per-CTA
 // partials in global memory.  Partial sums are added in tile order, so the
 // results do not depend on timing.
+// Fused mode (sq_quantize_linear): the kernel takes the fp32 activations and
+// performs the activation split itself after the weight prefetch: every CTA
+// forms the per-token scale (absmax over the non-outlier channels), the INT8
+// codes and the outlier values in shared memory with the same arithmetic as
+// the activation split kernel, and the main loop reads its codes from there.
 #include <stdint.h>
 
 #include <algorithm>
@@ -36,6 +41,7 @@
 #include "sq_common.cuh"
 #include "sq_internal.h"
 #include "sq_layout.h"
+#include "sq_quant.cuh"
 
 namespace sq {
 namespace {
@@ -68,6 +74,11 @@ struct Params {
   float4* ws_part;  // [CTA][slot 0/1][cell 0..3][lane] {T bits, F, Ut, Ur}
   int32_t* ws_cnt;  // [row block] arrival counters
   int pdl;
+  // fused mode
+  const float* x;     // [M][K] activations
+  int32_t* status;    // device status word (non-finite x, bad index list)
+  int n_pad;          // x_out row stride in shared memory
+  int off_xq, off_xo, off_sx, off_red;  // shared-memory offsets (bytes)
 };
 
 // First tile of warp w (w >= warps_total: T, an empty range).
@@ -220,7 +231,56 @@ __device__ __forceinline__ void write_y(const Params& p, int rb, int gid, int ti
   }
 }
 
-template <bool MASK, bool EMIT>
+// Fused mode: the activation split of the pass's tokens into shared memory
+// (codes [M][K128], outlier values [M][n_pad], scales [M]); outlier channels
+// are those marked in omask.  Same arithmetic as the activation split kernel.
+__device__ __forceinline__ void split_activations(const Params& p, const uint32_t* omask,
+                                                  int8_t* xq_s, float* xo_s, float* sx_s,
+                                                  float* red_s) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int K128 = p.xs;
+  bool nonfinite = false;
+  for (int t = 0; t < p.M; ++t) {
+    const float* xt = p.x + (int64_t)t * p.K;
+    float a = 0.0f;
+    for (int j = threadIdx.x; j < p.K; j += kThreads) {
+      const float v = xt[j];
+      nonfinite |= !isfinite(v);
+      if (!((omask[j >> 5] >> (j & 31)) & 1u)) a = fmaxf(a, fabsf(v));
+    }
+    for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    if (lane == 0) red_s[warp * kCols + t] = a;
+  }
+  __syncthreads();
+  if (threadIdx.x < p.M) {
+    float a = 0.0f;
+    for (int w = 0; w < kWarps; ++w) a = fmaxf(a, red_s[w * kCols + threadIdx.x]);
+    sx_s[threadIdx.x] = act_scale(a);
+  }
+  __syncthreads();
+  bool bad_idx = false;
+  for (int t = 0; t < p.M; ++t) {
+    const float* xt = p.x + (int64_t)t * p.K;
+    const float s = sx_s[t];
+    const double rinv = act_rinv(s);
+    for (int j = threadIdx.x; j < K128; j += kThreads) {
+      int q = 0;
+      if (j < p.K && !((omask[j >> 5] >> (j & 31)) & 1u)) q = quantize_exact(xt[j], s, rinv);
+      xq_s[t * K128 + j] = (int8_t)q;
+    }
+    for (int i = threadIdx.x; i < p.n_out; i += kThreads) {
+      const int j = p.idx[i];
+      const bool in = j >= 0 && j < p.K;
+      bad_idx |= !in || (i > 0 && p.idx[i - 1] >= j);
+      xo_s[t * p.n_pad + i] = in ? xt[j] : 0.0f;
+    }
+  }
+  if (nonfinite) set_status(p.status, SQ_ERR_NONFINITE);
+  if (bad_idx) set_status(p.status, SQ_ERR_INVALID_ARG);
+  __syncthreads();
+}
+
+template <bool MASK, bool EMIT, bool FUSED>
 __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
   extern __shared__ __align__(16) uint8_t smem[];
   // shared: part[kWarps][2][4][32] float4 | omask[nw] u32 | obase[nw] i32
@@ -270,13 +330,25 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
     pdl_wait();
     pdl_launch_dependents();
   }
+  int8_t* xq_s = reinterpret_cast<int8_t*>(smem + p.off_xq);
+  float* xo_s = reinterpret_cast<float*>(smem + p.off_xo);
+  float* sx_s = reinterpret_cast<float*>(smem + p.off_sx);
+  if constexpr (FUSED)
+    split_activations(p, omask, xq_s, xo_s, sx_s, reinterpret_cast<float*>(smem + p.off_red));
 
   // tokens of this lane's accumulator columns; the B operand of this lane
   // (MMA column gid) is token min(gid, M - 1): columns past M are not written
   const int tk0 = 2 * tid4, tk1 = tk0 + 1;
-  const float sx0 = tk0 < p.M ? __ldg(p.sx + tk0) : 0.0f;
-  const float sx1 = tk1 < p.M ? __ldg(p.sx + tk1) : 0.0f;
-  const int8_t* xrow = p.xq + (int64_t)min(gid, p.M - 1) * p.xs + tid4 * 32;
+  float sx0, sx1;
+  if constexpr (FUSED) {
+    sx0 = tk0 < p.M ? sx_s[tk0] : 0.0f;
+    sx1 = tk1 < p.M ? sx_s[tk1] : 0.0f;
+  } else {
+    sx0 = tk0 < p.M ? __ldg(p.sx + tk0) : 0.0f;
+    sx1 = tk1 < p.M ? __ldg(p.sx + tk1) : 0.0f;
+  }
+  const int tok = min(gid, p.M - 1);
+  const int8_t* xrow = (FUSED ? xq_s + tok * p.xs : p.xq + (int64_t)tok * p.xs) + tid4 * 32;
 
   Acc acc;
   acc_zero(acc);
@@ -297,8 +369,15 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
         // activation codes of this lane's 32 channels for its MMA column
         uint32_t xw[8];
         {
-          const int4 a = __ldg(reinterpret_cast<const int4*>(xrow + cg * kTileK));
-          const int4 b = __ldg(reinterpret_cast<const int4*>(xrow + cg * kTileK + 16));
+          const int4* xp = reinterpret_cast<const int4*>(xrow + cg * kTileK);
+          int4 a, b;
+          if constexpr (FUSED) {
+            a = xp[0];
+            b = xp[1];
+          } else {
+            a = __ldg(xp);
+            b = __ldg(xp + 1);
+          }
           xw[0] = a.x; xw[1] = a.y; xw[2] = a.z; xw[3] = a.w;
           xw[4] = b.x; xw[5] = b.y; xw[6] = b.z; xw[7] = b.w;
         }
@@ -365,8 +444,14 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
             // (an index list that is not strictly ascending cannot push pos
             // past the list)
             if (pos >= 0 && pos < p.n_out) {
-              const float x0 = tk0 < p.M ? __ldg(p.xout + (int64_t)tk0 * p.n_out + pos) : 0.0f;
-              const float x1 = tk1 < p.M ? __ldg(p.xout + (int64_t)tk1 * p.n_out + pos) : 0.0f;
+              float x0, x1;
+              if constexpr (FUSED) {
+                x0 = tk0 < p.M ? xo_s[tk0 * p.n_pad + pos] : 0.0f;
+                x1 = tk1 < p.M ? xo_s[tk1 * p.n_pad + pos] : 0.0f;
+              } else {
+                x0 = tk0 < p.M ? __ldg(p.xout + (int64_t)tk0 * p.n_out + pos) : 0.0f;
+                x1 = tk1 < p.M ? __ldg(p.xout + (int64_t)tk1 * p.n_out + pos) : 0.0f;
+              }
               acc.Ut[0] = fmaf(u0, x0, acc.Ut[0]);
               acc.Ut[1] = fmaf(u0, x1, acc.Ut[1]);
               acc.Ut[2] = fmaf(u1, x0, acc.Ut[2]);
@@ -515,9 +600,9 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
   }
 }
 
-template <bool MASK, bool EMIT>
+template <bool MASK, bool EMIT, bool FUSED>
 cudaError_t launch_one(const Params& p, int grid, int smem, bool pdl, cudaStream_t stream) {
-  auto* fn = k_linear_tc<MASK, EMIT>;
+  auto* fn = k_linear_tc<MASK, EMIT, FUSED>;
   cudaError_t e = ensure_smem_attr((const void*)fn, smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -540,11 +625,32 @@ size_t linear_tc_part_bytes(int sm_count) {
   return (size_t)sm_count * kBps * 2 * 4 * 32 * sizeof(float4);
 }
 
+namespace {
+constexpr int kSmemPart = kWarps * 2 * 4 * 32 * (int)sizeof(float4);
+// Shared memory of one CTA stays within this so that kBps CTAs fit an SM.
+constexpr int kSmemBudget = 100 * 1024;
+
+int outlier_table_bytes(const sq_packed_weight& w) { return (int)(tiles_cols(w.K) / 32) * 8; }
+int fused_token_bytes(const sq_packed_weight& w, int n_out) {
+  return (int)tiles_cols(w.K) + (int)round_up(n_out, 4) * 4;
+}
+}  // namespace
+
+int linear_tc_fused_tokens(const sq_packed_weight& w, int n_out) {
+  const int fixed = kSmemPart + outlier_table_bytes(w) + kCols * 4 + kWarps * kCols * 4 + 64;
+  const int per = fused_token_bytes(w, n_out);
+  const int m = (kSmemBudget - fixed) / per;
+  return m < 0 ? 0 : std::min(m, kCols);
+}
+
 cudaError_t launch_linear_tc(const sq_packed_weight& w, int M, const int8_t* xq, const float* sx,
-                             const float* x_out, const int32_t* idx, int n_out, float* y,
-                             int32_t* T_out, int32_t* R_out, void* workspace, size_t part_bytes,
-                             int sm_count, bool pdl, cudaStream_t stream) {
+                             const float* x_out, const float* x, const int32_t* idx, int n_out,
+                             float* y, int32_t* T_out, int32_t* R_out, void* workspace,
+                             size_t part_bytes, int sm_count, int32_t* status, bool pdl,
+                             cudaStream_t stream) {
   if (M < 1 || M > kCols || w.layout != SQ_LAYOUT_TILES) return cudaErrorInvalidValue;
+  const bool fused = x != nullptr;
+  if (fused && (T_out || M > linear_tc_fused_tokens(w, n_out))) return cudaErrorInvalidValue;
   Params p;
   p.res = w.res_q;
   p.sign = w.sign_bits;
@@ -573,16 +679,33 @@ cudaError_t launch_linear_tc(const sq_packed_weight& w, int M, const int8_t* xq,
   p.ws_part = reinterpret_cast<float4*>(workspace);
   p.ws_cnt = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(workspace) + part_bytes);
   p.pdl = pdl ? 1 : 0;
-  const int nw = p.tpr * 4;
-  const int smem = kWarps * 2 * 4 * 32 * (int)sizeof(float4) + nw * 8;
+  p.x = x;
+  p.status = status;
+  p.n_pad = (int)round_up(n_out, 4);
+  int smem = kSmemPart + outlier_table_bytes(w);
+  p.off_xq = p.off_xo = p.off_sx = p.off_red = 0;
+  if (fused) {
+    p.off_xq = smem;
+    smem += M * p.xs;
+    p.off_xo = smem;
+    smem += M * p.n_pad * 4;
+    p.off_sx = smem;
+    smem += kCols * 4;
+    p.off_red = smem;
+    smem += kWarps * kCols * 4;
+  }
+  smem = (int)round_up(smem, 16);
   const bool mask = w.mask_bits != nullptr;
   const bool emit = T_out != nullptr;
   const int grid = (int)blocks;
+  if (fused)
+    return mask ? launch_one<true, false, true>(p, grid, smem, pdl, stream)
+                : launch_one<false, false, true>(p, grid, smem, pdl, stream);
   if (mask)
-    return emit ? launch_one<true, true>(p, grid, smem, pdl, stream)
-                : launch_one<true, false>(p, grid, smem, pdl, stream);
-  return emit ? launch_one<false, true>(p, grid, smem, pdl, stream)
-              : launch_one<false, false>(p, grid, smem, pdl, stream);
+    return emit ? launch_one<true, true, false>(p, grid, smem, pdl, stream)
+                : launch_one<true, false, false>(p, grid, smem, pdl, stream);
+  return emit ? launch_one<false, true, false>(p, grid, smem, pdl, stream)
+              : launch_one<false, false, false>(p, grid, smem, pdl, stream);
 }
 
 }  // namespace sq

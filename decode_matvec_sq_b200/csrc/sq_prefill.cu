@@ -1,0 +1,493 @@
+// sq_prefill.cu -- the separated-quantization linear layer for many tokens
+// (prefill) on the 5th-generation tensor cores: tcgen05.mma kind::i8 with the
+// accumulators in tensor memory, operands staged by TMA.
+//
+// Page: "1-bit量化不是玄学，以往掉点是机制问题" (m.lqnn.cn/news/241359),
+// section 2.3: the trunk product and the residual product side by side,
+// summed; at prefill the activation matrix is a dense operand, so both are
+// int8 GEMMs: xq [M][K] against the trunk as +-1 (0 outside the mask) bytes
+// and against the residual codes.
+//
+// Same results as the decode kernels: exact int32 T and R_g, fp32 y.
+//   CTA tile: 128 tokens (MMA M, one TMEM lane each) x 64 weight rows (MMA N),
+//   looping over the 128-channel groups g (MMA K = 32, four per group).
+//   Warp 0 (one lane): TMA loads of the activation codes, residual codes and
+//     sign / mask words of group g into a 3-stage ring (128-byte swizzle).
+//   Warps 2-3: expand the sign (and mask) bits of the stage into +-1 / 0
+//     bytes, written in the same swizzled K-major layout.
+//   Warp 1 (one lane): four MMAs of the residual into accumulator R[g % 2]
+//     and four of the trunk into T (accumulating over all K).
+//   Warps 4-7: read R[g % 2] (tcgen05.ld), promote it with the group scales
+//     (F += s_g * R_g) and free the buffer; at the end read T and write
+//     y = sx * (alpha * T + F) + sum_i What[r][idx_i] * x_out[i].
+// Two CTAs share an SM (256 of the 512 TMEM columns each), so one CTA's
+// epilogue overlaps the other's MMAs.  Every wait is bounded: a wait that
+// runs out sets SQ_ERR_TIMEOUT in the status word and the CTA winds down.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <stdint.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "sq_common.cuh"
+#include "sq_internal.h"
+
+namespace sq {
+namespace {
+
+constexpr int BM = 128;        // tokens per CTA
+constexpr int BN = 64;         // weight rows per CTA
+constexpr int BK = 128;        // channels per group
+constexpr int kStages = 3;
+constexpr int kThreads = 256;  // 8 warps
+constexpr uint32_t kTmemCols = 256;  // T [0,64), R0 [64,128), R1 [128,192)
+
+constexpr int kBytesA = BM * BK;  // 16 KB
+constexpr int kBytesB = BN * BK;  // 8 KB
+constexpr int kBytesE = BN * BK;  // 8 KB
+constexpr int kBytesBits = BN * 16;  // 4 words per row
+constexpr int kOffA = 0, kOffB = kOffA + kBytesA, kOffE = kOffB + kBytesB;
+constexpr int kOffS = kOffE + kBytesE, kOffM = kOffS + kBytesBits;
+constexpr int kStageBytes = kOffM + kBytesBits;  // 34 KB, a multiple of 1024
+static_assert(kStageBytes % 1024 == 0, "stages must stay 1024-byte aligned");
+
+// small shared state after the stages
+struct Aux {
+  uint64_t full[kStages], tready[kStages], empty[kStages];
+  uint64_t accf[2], acce[2], tdone;
+  uint32_t tmem_base;
+  int abort;
+  float scl[2][BN];  // group scales of the CTA's rows, double buffered
+  float alpha[BN];
+};
+constexpr int kSmemBytes = kStages * kStageBytes + (int)sizeof(Aux) + 1024;  // + alignment slack
+
+struct Params {
+  int M, N, K, nk;  // nk = ceil(K / 128) groups
+  const float* alpha;
+  const float* scale;
+  int scale_stride;
+  const int8_t* res;  // row layout, for the outlier weights
+  int res_stride;
+  const uint32_t* sign;
+  const uint32_t* mask;
+  int sign_stride;
+  const float* sx;
+  const float* xout;
+  const int32_t* idx;
+  int n_out;
+  float* y;
+  int32_t* T_out;
+  int32_t* R_out;
+  int32_t* status;
+};
+
+// ---- PTX wrappers ---------------------------------------------------------------
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+      "%3}], [%4];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// K-major operand with 128-byte swizzle: rows of 128 bytes, 8-row atoms 1024
+// bytes apart (stride byte offset), leading byte offset 1 (unused by this
+// mode), descriptor version 1, layout type 2.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t addr) {
+  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// D (s32) += A (s8, K-major) * B (s8, K-major), M = 128, N = 64.
+constexpr uint32_t kIdesc = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                            ((uint32_t)(BM >> 4) << 24);
+
+__device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t a, uint64_t b, bool acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(kIdesc), "r"(acc ? 1 : 0));
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// 32 consecutive TMEM columns of this thread's lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, int (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+      "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void named_sync_epi() {
+  asm volatile("bar.sync 1, 128;" ::: "memory");  // the four epilogue warps
+}
+
+// Waits on an mbarrier phase; on a timeout records it and asks the CTA to stop.
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Aux* aux,
+                                              int32_t* status) {
+  if (mbar_wait(bar, parity)) return true;
+  set_status(status, SQ_ERR_TIMEOUT);
+  atomicExch(&aux->abort, 1);
+  return false;
+}
+__device__ __forceinline__ bool aborted(const Aux* aux) {
+  return *reinterpret_cast<const volatile int*>(&aux->abort) != 0;
+}
+
+// +-1 (or 0 outside the mask) bytes of channels 4n .. 4n+3 from the nibble of
+// sign bits (and mask bits): byte = 0x01 if b, 0xFF if not, 0 if m = 0.
+template <bool MASK>
+__device__ __forceinline__ uint32_t trunk_bytes(uint32_t snib, uint32_t mnib) {
+  const uint32_t eb = ((snib & 0xFu) * 0x00204081u) & 0x01010101u;  // 0/1 per byte
+  uint32_t pm = ~(eb * 0xFEu);                                      // 0x01 / 0xFF
+  if (MASK) pm &= (((mnib & 0xFu) * 0x00204081u) & 0x01010101u) * 0xFFu;
+  return pm;
+}
+
+template <bool MASK, bool EMIT>
+__global__ void __launch_bounds__(kThreads, 2)
+    k_prefill(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+              const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmM,
+              const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Aux* aux = reinterpret_cast<Aux*>(smem + kStages * kStageBytes);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nt_m = (p.M + BM - 1) / BM;
+  const int m0 = (blockIdx.x % nt_m) * BM, n0 = (blockIdx.x / nt_m) * BN;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&aux->full[s], 1);
+      mbar_init(&aux->tready[s], 64);
+      mbar_init(&aux->empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&aux->accf[b], 1);
+      mbar_init(&aux->acce[b], 128);
+    }
+    mbar_init(&aux->tdone, 1);
+    aux->abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&aux->tmem_base)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  if (threadIdx.x >= 128 && threadIdx.x < 128 + BN) {
+    const int n = n0 + threadIdx.x - 128;
+    aux->alpha[threadIdx.x - 128] = n < p.N ? __ldg(p.alpha + n) : 0.0f;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = aux->tmem_base;
+
+  if (warp == 0) {
+    // ---- TMA producer
+    if (lane == 0) {
+      for (int kb = 0; kb < p.nk; ++kb) {
+        const int s = kb % kStages;
+        const uint32_t use = (uint32_t)(kb / kStages);
+        if (kb >= kStages && !wait_or_abort(&aux->empty[s], (use & 1u) ^ 1u, aux, p.status)) break;
+        if (aborted(aux)) break;
+        uint8_t* st = smem + s * kStageBytes;
+        mbar_arrive_expect_tx(&aux->full[s],
+                              kBytesA + kBytesB + kBytesBits + (MASK ? kBytesBits : 0));
+        tma_load_2d(st + kOffA, &tmA, kb * BK, m0, &aux->full[s]);
+        tma_load_2d(st + kOffB, &tmB, kb * BK, n0, &aux->full[s]);
+        tma_load_2d(st + kOffS, &tmS, kb * 4, n0, &aux->full[s]);
+        if (MASK) tma_load_2d(st + kOffM, &tmM, kb * 4, n0, &aux->full[s]);
+      }
+    }
+  } else if (warp == 1) {
+    // ---- MMA issuer
+    if (lane == 0) {
+      for (int kb = 0; kb < p.nk; ++kb) {
+        const int s = kb % kStages, b = kb & 1;
+        const uint32_t use = (uint32_t)(kb / kStages);
+        if (!wait_or_abort(&aux->full[s], use & 1u, aux, p.status)) break;
+        if (!wait_or_abort(&aux->tready[s], use & 1u, aux, p.status)) break;
+        if (kb >= 2 && !wait_or_abort(&aux->acce[b], ((uint32_t)(kb >> 1) & 1u) ^ 1u, aux, p.status))
+          break;
+        tc_fence_after();
+        const uint32_t st = smem_u32(smem + s * kStageBytes);
+#pragma unroll
+        for (int kk = 0; kk < BK / 32; ++kk) {
+          const uint64_t da = sw128_desc(st + kOffA + kk * 32);
+          const uint64_t db = sw128_desc(st + kOffB + kk * 32);
+          const uint64_t de = sw128_desc(st + kOffE + kk * 32);
+          mma_i8(tmem + 64 + 64 * b, da, db, kk > 0);
+          mma_i8(tmem, da, de, kb > 0 || kk > 0);
+        }
+        mma_commit(&aux->empty[s]);
+        mma_commit(&aux->accf[b]);
+      }
+      mma_commit(&aux->tdone);
+    }
+  } else if (warp < 4) {
+    // ---- trunk expansion: one weight row per thread
+    const int r = threadIdx.x - 64;
+    for (int kb = 0; kb < p.nk; ++kb) {
+      const int s = kb % kStages;
+      if (!wait_or_abort(&aux->full[s], (uint32_t)(kb / kStages) & 1u, aux, p.status)) break;
+      uint8_t* st = smem + s * kStageBytes;
+      const uint4 sw = *reinterpret_cast<const uint4*>(st + kOffS + r * 16);
+      uint4 mw = make_uint4(0u, 0u, 0u, 0u);
+      if (MASK) mw = *reinterpret_cast<const uint4*>(st + kOffM + r * 16);
+      const uint32_t sv[4] = {sw.x, sw.y, sw.z, sw.w};
+      const uint32_t mv[4] = {mw.x, mw.y, mw.z, mw.w};
+      uint8_t* row = st + kOffE + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {  // 16-byte chunk c = channels 16c .. 16c+15
+        const uint32_t s16 = sv[c >> 1] >> (16 * (c & 1));
+        const uint32_t m16 = mv[c >> 1] >> (16 * (c & 1));
+        uint4 v;
+        v.x = trunk_bytes<MASK>(s16, m16);
+        v.y = trunk_bytes<MASK>(s16 >> 4, m16 >> 4);
+        v.z = trunk_bytes<MASK>(s16 >> 8, m16 >> 8);
+        v.w = trunk_bytes<MASK>(s16 >> 12, m16 >> 12);
+        *reinterpret_cast<uint4*>(row + ((c ^ (r & 7)) * 16)) = v;
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive(&aux->tready[s]);
+    }
+  } else {
+    // ---- epilogue: one token (TMEM lane) per thread
+    const int et = threadIdx.x - 128;
+    const int lb = 32 * (warp & 3);  // TMEM lanes of this warp
+    const int t = m0 + lb + lane;
+    float F[BN];
+#pragma unroll
+    for (int n = 0; n < BN; ++n) F[n] = 0.0f;
+    const int ng = p.nk;
+    // Every epilogue thread runs every iteration and meets every named
+    // barrier; whether a warp reads TMEM is decided per warp (tcgen05.ld is
+    // warp-collective), and after a timeout the rest is skipped.
+    for (int kb = 0; kb < p.nk; ++kb) {
+      const int b = kb & 1;
+      if (et < BN) {
+        const int n = n0 + et;
+        aux->scl[b][et] = n < p.N ? __ldg(p.scale + (int64_t)n * p.scale_stride + kb) : 0.0f;
+      }
+      named_sync_epi();
+      bool ok = !aborted(aux) && wait_or_abort(&aux->accf[b], (uint32_t)(kb >> 1) & 1u, aux, p.status);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) continue;
+      tc_fence_after();
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        int r[32];
+        tmem_ld32(tmem + ((uint32_t)lb << 16) + 64 + 64 * b + 32 * h, r);
+        if (h == 1) {
+          tc_fence_before();
+          mbar_arrive(&aux->acce[b]);
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) F[32 * h + i] = fmaf(aux->scl[b][32 * h + i], (float)r[i], F[32 * h + i]);
+        if (EMIT && t < p.M) {
+          for (int i = 0; i < 32; ++i) {
+            const int n = n0 + 32 * h + i;
+            if (n < p.N) p.R_out[((int64_t)t * p.N + n) * ng + kb] = r[i];
+          }
+        }
+      }
+    }
+    bool fin = !aborted(aux) && wait_or_abort(&aux->tdone, 0u, aux, p.status);
+    named_sync_epi();  // a timeout anywhere is now visible to all epilogue threads
+    fin = fin && !aborted(aux);
+    if (__any_sync(0xffffffffu, !fin)) fin = false;
+    named_sync_epi();
+    fin = !aborted(aux) && fin;
+    if (fin) {
+      tc_fence_after();
+      const float sxt = t < p.M ? __ldg(p.sx + t) : 0.0f;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        int r[32];
+        tmem_ld32(tmem + ((uint32_t)lb << 16) + 32 * h, r);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int n = 32 * h + i;
+          F[n] = sxt * fmaf(aux->alpha[n], (float)r[i], F[n]);
+        }
+        if (EMIT && t < p.M) {
+          for (int i = 0; i < 32; ++i) {
+            const int n = n0 + 32 * h + i;
+            if (n < p.N) p.T_out[(int64_t)t * p.N + n] = r[i];
+          }
+        }
+      }
+      // outlier channels: y += sum_i What[n][idx_i] * x_out[t][i], What from
+      // the packed row (the dequantized weight); table in the free stage memory
+      float* wo = reinterpret_cast<float*>(smem);  // [64 outliers][BN]
+      for (int i0 = 0; i0 < p.n_out; i0 += 64) {
+        const int ni = min(64, p.n_out - i0);
+        named_sync_epi();
+        for (int e = et; e < ni * BN; e += 128) {
+          const int i = e / BN, nn = e - i * BN, n = n0 + nn;
+          const int j = p.idx[i0 + i];
+          float w = 0.0f;
+          if (n < p.N && j >= 0 && j < p.K) {
+            const uint32_t bit = 1u << (j & 31);
+            const bool sgn = (p.sign[(int64_t)n * p.sign_stride + (j >> 5)] & bit) != 0;
+            const bool m = MASK ? (p.mask[(int64_t)n * p.sign_stride + (j >> 5)] & bit) != 0 : true;
+            const float al = aux->alpha[nn];
+            const float tr = m ? (sgn ? al : -al) : 0.0f;
+            w = fmaf(p.scale[(int64_t)n * p.scale_stride + (j >> 7)],
+                     (float)p.res[(int64_t)n * p.res_stride + j], tr);
+          }
+          wo[i * BN + nn] = w;
+        }
+        named_sync_epi();
+        if (t < p.M) {
+          for (int i = 0; i < ni; ++i) {
+            const float xv = __ldg(p.xout + (int64_t)t * p.n_out + i0 + i);
+#pragma unroll
+            for (int n = 0; n < BN; ++n) F[n] = fmaf(wo[i * BN + n], xv, F[n]);
+          }
+        }
+      }
+      if (t < p.M) {
+        float* yr = p.y + (int64_t)t * p.N + n0;
+        if (n0 + BN <= p.N && (p.N & 3) == 0) {
+#pragma unroll
+          for (int n = 0; n < BN; n += 4)
+            *reinterpret_cast<float4*>(yr + n) = make_float4(F[n], F[n + 1], F[n + 2], F[n + 3]);
+        } else {
+          for (int n = 0; n < BN; ++n)
+            if (n0 + n < p.N) yr[n] = F[n];
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+// ---- host: tensor maps -------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int esize, const void* base, uint64_t inner,
+              uint64_t rows, uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows,
+              CUtensorMapSwizzle sw) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_rows};
+  const cuuint32_t es[2] = {1, 1};
+  (void)esize;
+  return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <bool MASK, bool EMIT>
+cudaError_t launch_prefill_t(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& s,
+                             const CUtensorMap& m, const Params& p, int grid, cudaStream_t stream) {
+  auto* fn = k_prefill<MASK, EMIT>;
+  cudaError_t e = ensure_smem_attr((const void*)fn, kSmemBytes);
+  if (e != cudaSuccess) return e;
+  fn<<<grid, kThreads, kSmemBytes, stream>>>(a, b, s, m, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool prefill_supported(const sq_packed_weight& w) {
+  return w.layout == SQ_LAYOUT_ROWS && w.group_size == BK && encode_fn() != nullptr;
+}
+
+cudaError_t launch_prefill(const sq_packed_weight& w, int M, const int8_t* xq, const float* sx,
+                           const float* x_out, const int32_t* idx, int n_out, float* y,
+                           int32_t* T_out, int32_t* R_out, int32_t* status, cudaStream_t stream) {
+  if (!prefill_supported(w) || M < 1) return cudaErrorInvalidValue;
+  const int64_t K128 = xq_stride_of(w.K);
+  CUtensorMap ma, mb, ms, mm;
+  if (!make_map(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, xq, (uint64_t)K128, (uint64_t)M,
+                (uint64_t)K128, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&mb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w.res_q, (uint64_t)w.res_stride,
+                (uint64_t)w.N, (uint64_t)w.res_stride, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&ms, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, w.sign_bits, (uint64_t)w.sign_stride,
+                (uint64_t)w.N, (uint64_t)w.sign_stride * 4, 4, BN, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
+  if (w.mask_bits) {
+    if (!make_map(&mm, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, w.mask_bits, (uint64_t)w.sign_stride,
+                  (uint64_t)w.N, (uint64_t)w.sign_stride * 4, 4, BN, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return cudaErrorInvalidValue;
+  } else {
+    mm = ms;
+  }
+  Params p;
+  p.M = M;
+  p.N = w.N;
+  p.K = w.K;
+  p.nk = (int)ceil_div(w.K, BK);
+  p.alpha = w.alpha;
+  p.scale = w.res_scale;
+  p.scale_stride = w.scale_stride;
+  p.res = w.res_q;
+  p.res_stride = w.res_stride;
+  p.sign = w.sign_bits;
+  p.mask = w.mask_bits;
+  p.sign_stride = w.sign_stride;
+  p.sx = sx;
+  p.xout = x_out;
+  p.idx = idx;
+  p.n_out = n_out;
+  p.y = y;
+  p.T_out = T_out;
+  p.R_out = R_out;
+  p.status = status;
+  const int64_t grid = ceil_div(M, BM) * ceil_div(w.N, BN);
+  if (grid >= INT32_MAX) return cudaErrorInvalidValue;
+  const bool mask = w.mask_bits != nullptr, emit = T_out != nullptr;
+  if (mask)
+    return emit ? launch_prefill_t<true, true>(ma, mb, ms, mm, p, (int)grid, stream)
+                : launch_prefill_t<true, false>(ma, mb, ms, mm, p, (int)grid, stream);
+  return emit ? launch_prefill_t<false, true>(ma, mb, ms, mm, p, (int)grid, stream)
+              : launch_prefill_t<false, false>(ma, mb, ms, mm, p, (int)grid, stream);
+}
+
+}  // namespace sq

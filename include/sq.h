@@ -223,6 +223,29 @@ sq_status sq_linear_accumulators(const sq_packed_weight *w, const int8_t *xq, co
                                  uint32_t flags, void *stream);
 
 /*
+ * The activation split and the linear layer in one kernel (m.lqnn.cn
+ * sections 2.2, 2.3 and 3.3: the split, the two products and their sum in a
+ * single fused step).  For a weight in SQ_LAYOUT_TILES.
+ *   x           [M][K] f32 activations, device
+ *   idx, n_out  outlier channels, strictly ascending in [0, K) (checked on
+ *               the device: a violation sets SQ_ERR_INVALID_ARG)
+ *   y           [M][N] f32 out
+ *   workspace   as for sq_linear (sq_linear_workspace_bytes(w, M))
+ * Every CTA forms the per-token scale, codes and outlier values of x in its
+ * shared memory with the same arithmetic as sq_quantize_act, then runs the
+ * decode of sq_linear: y is bit-identical to sq_quantize_act followed by
+ * sq_linear.  Non-finite x sets SQ_ERR_NONFINITE.  Tokens are processed in
+ * passes of up to 8 that fit the shared memory: roundup(K,128) +
+ * 4*roundup(n_out,4) bytes per token; SQ_ERR_SHAPE if not even one token
+ * fits (K above about 60000).  flags: 0 or SQ_LAUNCH_PDL (the kernel then
+ * reads x, idx and y-independent data only after the previous kernel
+ * completes; the packed weights are streamed before).
+ */
+sq_status sq_quantize_linear(const sq_packed_weight *w, const float *x, int32_t M,
+                             const int32_t *idx, int32_t n_out, float *y, void *workspace,
+                             size_t ws_bytes, int32_t *dev_status, uint32_t flags, void *stream);
+
+/*
  * sq_linear without a caller workspace, for callers that cannot allocate
  * device memory at call time.  This entry point has no counterpart on the
  * pages: it only changes where the scratch lives.

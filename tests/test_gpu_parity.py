@@ -494,3 +494,143 @@ def test_fewer_work_units_than_warps(N, K, tc):
         torch.cuda.synchronize()
         check_y(y.cpu().numpy(), y_ref, oracle.abs_dot(W, x))
         assert not sq.workspace_counters(ws, pw, 2).any().item()
+
+
+# ---- fused activation split + linear --------------------------------------------
+
+def _fused_vs_two_step(W, x, idx, P=-1, pdl=False):
+    """sq_quantize_linear == sq_quantize_act + sq_linear bit for bit, and
+    within the tolerance of the oracle."""
+    Wd, xd = torch.from_numpy(W).cuda(), torch.from_numpy(x).cuda()
+    idxd = torch.from_numpy(idx.astype(np.int32)).cuda() if len(idx) else None
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pw = sq.decompose_pack(Wd, trunk_percent=P, layout=sq.SQ_LAYOUT_TILES, status=st)
+    xq, sx, xo = sq.quantize_act(xd, idxd, status=st)
+    ws = sq.new_workspace(pw, x.shape[0])
+    y2 = torch.full((x.shape[0], W.shape[0]), float("nan"), device="cuda")
+    sq.linear(pw, xq, sx, xo, idxd, y=y2, workspace=ws, status=st)
+    for _ in range(2):  # twice: the arrival counters are left zero
+        y1 = torch.full_like(y2, float("nan"))
+        sq.quantize_linear(pw, xd, idxd, y=y1, workspace=ws, status=st, pdl=pdl)
+        torch.cuda.synchronize()
+        assert st.item() == 0
+        assert np.array_equal(y1.cpu().numpy().view(np.uint32), y2.cpu().numpy().view(np.uint32))
+    assert not sq.workspace_counters(ws, pw, x.shape[0]).any().item()
+    d = oracle.decompose(W, P=P)
+    oxq, osx, oxo = oracle.quantize_act(x, idx)
+    check_y(y1.cpu().numpy(), oracle.linear(d, oxq, osx, oxo, idx), oracle.abs_dot(W, x))
+
+
+@pytest.mark.parametrize("N,K,M,n", [(1, 8, 1, 0), (7, 33, 1, 2), (40, 129, 8, 1), (20, 300, 3, 3),
+                                     (513, 300, 1, 6), (64, 4096, 1, 20), (24, 11008, 1, 55),
+                                     (8, 28672, 2, 72), (100, 2048, 16, 10), (33, 1000, 13, 9)])
+@pytest.mark.parametrize("P", [-1, 60])
+def test_quantize_linear_parity(N, K, M, n, P):
+    rng = np.random.default_rng(7 * N + K + M + n + P)
+    W = rng.laplace(0, 0.02, (N, K)).astype(np.float32)
+    x = rng.standard_normal((M, K)).astype(np.float32)
+    idx = np.sort(rng.choice(K, n, replace=False)).astype(np.int32)
+    x[:, idx] *= 30.0
+    if M > 1:
+        x[1] = 0.0  # a zero token
+    _fused_vs_two_step(W, x, idx, P=P)
+
+
+def test_quantize_linear_config2_layers():
+    """Full-size stack shapes, batch 1, with PDL."""
+    for mid in range(4):
+        L = wl.config2_layer(2, mid)
+        rows = _rows(L.N, n=64, seed=mid)
+        Wd = sdev.fill_weights(L, torch.empty(L.N, L.K, device="cuda"))
+        pw = sq.decompose_pack(Wd)
+        del Wd
+        x = L.activations()
+        idx = L.planted_channels()
+        xd, idxd = torch.from_numpy(x).cuda(), torch.from_numpy(idx).cuda()
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        y = sq.quantize_linear(pw, xd, idxd, status=st, pdl=True)
+        xq, sx, xo = sq.quantize_act(xd, idxd, status=st)
+        y2 = sq.linear(pw, xq, sx, xo, idxd, status=st)
+        torch.cuda.synchronize()
+        assert st.item() == 0 and torch.equal(y, y2)
+        Wr = L.weights(rows=rows)
+        d = oracle.decompose(Wr)
+        oxq, osx, oxo = oracle.quantize_act(x, idx)
+        check_y(y[:, torch.as_tensor(rows, device="cuda")].cpu().numpy(),
+                oracle.linear(d, oxq, osx, oxo, idx), oracle.abs_dot(Wr, x), L.name)
+
+
+def test_quantize_linear_status_and_errors():
+    W = torch.randn(32, 256, device="cuda")
+    pw = sq.decompose_pack(W)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    x = torch.randn(2, 256, device="cuda")
+    x[1, 9] = float("inf")
+    sq.quantize_linear(pw, x, None, status=st)
+    torch.cuda.synchronize()
+    assert st.item() == sq.STATUS_CODE["SQ_ERR_NONFINITE"]
+    st.zero_()
+    sq.quantize_linear(pw, torch.randn(1, 256, device="cuda"),
+                       torch.tensor([7, 7], dtype=torch.int32, device="cuda"), status=st)
+    torch.cuda.synchronize()
+    assert st.item() == sq.STATUS_CODE["SQ_ERR_INVALID_ARG"]
+    pr = sq.decompose_pack(W, layout=sq.SQ_LAYOUT_ROWS)
+    with pytest.raises(sq.SQError) as e:
+        sq.quantize_linear(pr, torch.randn(1, 256, device="cuda"), None)
+    assert e.value.name == "SQ_ERR_SHAPE"
+
+
+# ---- prefill: many tokens on tcgen05 (row layout, M >= 64) --------------------------
+
+@pytest.mark.parametrize("N,K,M,n,P", [(64, 128, 128, 2, -1), (100, 300, 200, 5, -1), (64, 129, 64, 1, 60),
+                                       (130, 1024, 257, 9, -1), (64, 4096, 128, 20, 60),
+                                       (192, 2048, 384, 70, -1)])
+def test_prefill_parity(N, K, M, n, P):
+    """Exact T and R_g, y within tolerance, on ragged tokens, rows and channels."""
+    rng = np.random.default_rng(N * 7 + K + M + n)
+    W = rng.laplace(0, 0.02, (N, K)).astype(np.float32)
+    x = rng.standard_normal((M, K)).astype(np.float32)
+    idx = np.sort(rng.choice(K, n, replace=False)).astype(np.int32)
+    x[:, idx] *= 30.0
+    x[3] = 0.0  # a zero token
+    Wd, xd, idxd = (torch.from_numpy(a).cuda() for a in (W, x, idx))
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pw = sq.decompose_pack(Wd, trunk_percent=P, layout=sq.SQ_LAYOUT_ROWS, status=st)
+    xq, sx, xo = sq.quantize_act(xd, idxd, status=st)
+    y, T, R = sq.linear_accumulators(pw, xq, sx, xo, idxd, status=st)
+    y2 = sq.linear(pw, xq, sx, xo, idxd, status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0, sq.STATUS.get(st.item())
+    d = oracle.decompose(W, P=P)
+    oxq, osx, oxo = oracle.quantize_act(x, idx)
+    oT, oR = oracle.accumulate(d, oxq)
+    assert np.array_equal(T.cpu().numpy().astype(np.int64), oT), "trunk accumulators"
+    assert np.array_equal(R.cpu().numpy().astype(np.int64), oR), "group accumulators"
+    y_ref = oracle.linear(d, oxq, osx, oxo, idx)
+    bound = oracle.abs_dot(W, x)
+    check_y(y.cpu().numpy(), y_ref, bound)
+    check_y(y2.cpu().numpy(), y_ref, bound)
+
+
+def test_prefill_config5_sampled():
+    """M = 2048 tokens x 4096 -> 14336 (the prefill workload): every token of
+    sampled rows against the oracle."""
+    L = wl.config5()
+    Wd = sdev.fill_weights(L, torch.empty(L.N, L.K, device="cuda"))
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pw = sq.decompose_pack(Wd, layout=sq.SQ_LAYOUT_ROWS, status=st)
+    del Wd
+    xd = sdev.fill_activations(L, torch.empty(L.M, L.K, device="cuda"))
+    idx = torch.from_numpy(L.planted_channels()).cuda()
+    xq, sx, xo = sq.quantize_act(xd, idx, status=st)
+    y = sq.linear(pw, xq, sx, xo, idx, status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    rows = _rows(L.N, n=40, seed=5)
+    Wr = L.weights(rows=rows)
+    x = L.activations(M=L.M)
+    d = oracle.decompose(Wr)
+    oxq, osx, oxo = oracle.quantize_act(x, L.planted_channels())
+    assert np.array_equal(xq.cpu().numpy()[:, :L.K], oxq)
+    check_y(y[:, torch.as_tensor(rows, device="cuda")].cpu().numpy(),
+            oracle.linear(d, oxq, osx, oxo, L.planted_channels()), oracle.abs_dot(Wr, x))
