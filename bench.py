@@ -76,6 +76,22 @@ def load_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+FALLBACK_BF16_TFLOPS = 1590.0
+INT8_PER_BF16 = 2.0  # nominal dense int8 : bf16 tensor throughput (4.5 : 2.25 P/s)
+
+
+def load_int8_peak():
+    """Dense int8 tensor peak in T int-ops/s: the measured cuBLAS bf16 burst
+    figure times the nominal int8/bf16 ratio."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]) * INT8_PER_BF16, "measured bf16 x nominal int8/bf16 ratio"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS * INT8_PER_BF16, "fallback bf16 x nominal int8/bf16 ratio"
+
+
 class ClockSampler:
     """nvidia-smi samples of SM clock and throttle reasons during a region."""
 
@@ -376,6 +392,95 @@ class Stack:
         return tot_bytes / n_launch, tot_ms / n_launch, shapes
 
 
+def run_prefill(args, world, rank, local):
+    """Prefill-sized linear layer: M = 2048 tokens x 4096 -> 14336 (row layout,
+    tcgen05 kernel).  One step = the activation split of the 2048 tokens and
+    the linear layer.  Tensor-bound: reported in T int-ops/s, where the work
+    is the trunk and residual products, 4*M*N*K int-ops."""
+    import torch
+    import torch.distributed as dist
+    import decode_matvec_sq_b200 as sq
+    from decode_matvec_sq_b200 import build
+    import synth.device as sdev
+    from synth import workloads as wl
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py: no CUDA device visible (the sq path has no CPU fallback)")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=device)
+    if rank == 0 or world == 1:
+        build.build_all()
+    barrier(world)
+    sq.device_check()
+    L = wl.config5()
+    W = sdev.fill_weights(L, torch.empty(L.N, L.K, device=device))
+    st = torch.zeros(1, dtype=torch.int32, device=device)
+    pw = sq.decompose_pack(W, layout=sq.SQ_LAYOUT_ROWS, status=st)
+    del W
+    x = sdev.fill_activations(L, torch.empty(L.M, L.K, device=device))
+    idx = torch.from_numpy(L.planted_channels()).to(device)
+    xq, sx, xo = sq.quantize_act(x, idx, status=st)
+    y = torch.empty(L.M, L.N, device=device)
+    ws = sq.new_workspace(pw, L.M)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)  # > L2, written between steps
+
+    def step():
+        sq.quantize_act(x, idx, xq=xq, sx=sx, x_out=xo, status=st)
+        sq.linear(pw, xq, sx, xo, idx, y=y, workspace=ws, status=st)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    ops = 4 * L.M * L.N * L.K
+    with ClockSampler(local) as clk:
+        barrier(world)
+        ev = []
+        for _ in range(args.steps):
+            flush.fill_(1)
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            c = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            sq.quantize_act(x, idx, xq=xq, sx=sx, x_out=xo, status=st)
+            b.record(stream)
+            sq.linear(pw, xq, sx, xo, idx, y=y, workspace=ws, status=st)
+            c.record(stream)
+            ev.append((a, b, c))
+        torch.cuda.synchronize()
+        barrier(world)
+    clocks = clk.summary()
+    ms_step = max_over_ranks(sum(a.elapsed_time(c) for a, b, c in ev) / len(ev), world, device)
+    ms_lin = max_over_ranks(sum(b.elapsed_time(c) for a, b, c in ev) / len(ev), world, device)
+    if st.item() != 0:
+        raise RuntimeError(f"device status {sq.STATUS.get(st.item())}")
+    peak, kind = load_int8_peak()
+    value = world * ops / (ms_step * 1e-3) / 1e12
+    achieved = ops / (ms_lin * 1e-3) / 1e12
+    if rank == 0:
+        print(json.dumps({
+            "metric": "prefill sq_linear int8 tensor T int-ops/s, 2048 tokens x 4096 -> 14336",
+            "value": round(value, 1), "unit": "T int-ops/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+            "config": {"workload": "prefill 2048 tokens x 4096 -> 14336, W Laplace(0,0.02), "
+                                   "x N(0,1) with 0.5% channels x30",
+                       "l2": "a 256 MB buffer written between steps"},
+            "gpu_launches": 2 * args.steps,
+            "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak, 1),
+                         "unit": "T int-ops/s", "frac": round(achieved / peak, 4), "peak_kind": kind,
+                         "traffic": None, "kernel": "k_prefill (tcgen05 kind::i8)",
+                         "us_per_launch": round(ms_lin * 1e3, 2)},
+            "clocks": clocks,
+        }), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
 def run_gpu(args, world, rank, local):
     import torch
     import torch.distributed as dist
@@ -525,6 +630,9 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["sq", "reference"], default="sq")
     ap.add_argument("--layers", type=int, default=32)
+    ap.add_argument("--workload", choices=["decode", "prefill"], default="decode",
+                    help="decode: the 7B-shaped stack at batch 1 (default); prefill: "
+                         "2048 tokens x 4096 -> 14336 on the tcgen05 kernel")
     ap.add_argument("--no-pdl", action="store_true")
     ap.add_argument("--two-kernels", action="store_true",
                     help="activation split and linear layer as two kernels per linear")
@@ -538,6 +646,8 @@ def main(argv=None):
     world, rank, local = dist_setup()
     if args.impl == "reference":
         return run_reference(args, world, rank)
+    if args.workload == "prefill":
+        return run_prefill(args, world, rank, local)
     return run_gpu(args, world, rank, local)
 
 

@@ -90,6 +90,15 @@ __device__ __forceinline__ int tile_warp(int t, const Params& p) {
   return (int)(((int64_t)(t + 1) * p.warps_total + p.T - 1) / p.T) - 1;
 }
 
+// Arrival on a row block's counter: release orders this warp's partial-sum
+// stores (made visible to lane 0 by __syncwarp) before the increment; acquire
+// orders the finisher's loads of the other CTAs' partials after it.
+__device__ __forceinline__ int arrive_acq_rel(int32_t* cnt) {
+  int prev;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;" : "=r"(prev) : "l"(cnt) : "memory");
+  return prev;
+}
+
 __device__ __forceinline__ void mma_s8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                        uint32_t a3, uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -234,19 +243,53 @@ __device__ __forceinline__ void write_y(const Params& p, int rb, int gid, int ti
 // Fused mode: the activation split of the pass's tokens into shared memory
 // (codes [M][K128], outlier values [M][n_pad], scales [M]); outlier channels
 // are those marked in omask.  Same arithmetic as the activation split kernel.
+// x is read as float4 (when rows are 16-byte aligned), eight loads in flight
+// per thread, so the two passes take few memory round trips.
+constexpr int kSplitUnroll = 8;
+
+__device__ __forceinline__ uint32_t omask_nibble(const uint32_t* omask, int j4) {
+  return (omask[j4 >> 3] >> ((j4 & 7) * 4)) & 0xFu;  // outlier bits of channels 4*j4 .. 4*j4+3
+}
+
 __device__ __forceinline__ void split_activations(const Params& p, const uint32_t* omask,
                                                   int8_t* xq_s, float* xo_s, float* sx_s,
                                                   float* red_s) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int K128 = p.xs;
+  const bool vec = (p.K & 3) == 0 && (reinterpret_cast<uintptr_t>(p.x) & 15u) == 0;
+  const int K4 = p.K >> 2;
   bool nonfinite = false;
   for (int t = 0; t < p.M; ++t) {
     const float* xt = p.x + (int64_t)t * p.K;
     float a = 0.0f;
-    for (int j = threadIdx.x; j < p.K; j += kThreads) {
-      const float v = xt[j];
-      nonfinite |= !isfinite(v);
-      if (!((omask[j >> 5] >> (j & 31)) & 1u)) a = fmaxf(a, fabsf(v));
+    if (vec) {
+      const float4* x4 = reinterpret_cast<const float4*>(xt);
+      for (int j0 = threadIdx.x; j0 < K4; j0 += kThreads * kSplitUnroll) {
+        float4 v[kSplitUnroll];
+#pragma unroll
+        for (int u = 0; u < kSplitUnroll; ++u) {
+          const int j4 = j0 + u * kThreads;
+          v[u] = j4 < K4 ? x4[j4] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        }
+#pragma unroll
+        for (int u = 0; u < kSplitUnroll; ++u) {
+          const int j4 = j0 + u * kThreads;
+          if (j4 < K4) {
+            const uint32_t om = omask_nibble(omask, j4);
+            nonfinite |= !isfinite(v[u].x) || !isfinite(v[u].y) || !isfinite(v[u].z) || !isfinite(v[u].w);
+            if (!(om & 1u)) a = fmaxf(a, fabsf(v[u].x));
+            if (!(om & 2u)) a = fmaxf(a, fabsf(v[u].y));
+            if (!(om & 4u)) a = fmaxf(a, fabsf(v[u].z));
+            if (!(om & 8u)) a = fmaxf(a, fabsf(v[u].w));
+          }
+        }
+      }
+    } else {
+      for (int j = threadIdx.x; j < p.K; j += kThreads) {
+        const float v = xt[j];
+        nonfinite |= !isfinite(v);
+        if (!((omask[j >> 5] >> (j & 31)) & 1u)) a = fmaxf(a, fabsf(v));
+      }
     }
     for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
     if (lane == 0) red_s[warp * kCols + t] = a;
@@ -263,10 +306,36 @@ __device__ __forceinline__ void split_activations(const Params& p, const uint32_
     const float* xt = p.x + (int64_t)t * p.K;
     const float s = sx_s[t];
     const double rinv = act_rinv(s);
-    for (int j = threadIdx.x; j < K128; j += kThreads) {
-      int q = 0;
-      if (j < p.K && !((omask[j >> 5] >> (j & 31)) & 1u)) q = quantize_exact(xt[j], s, rinv);
-      xq_s[t * K128 + j] = (int8_t)q;
+    uint32_t* q4 = reinterpret_cast<uint32_t*>(xq_s + t * K128);
+    if (vec) {
+      const float4* x4 = reinterpret_cast<const float4*>(xt);
+      for (int j0 = threadIdx.x; j0 < K128 / 4; j0 += kThreads * kSplitUnroll) {
+        float4 v[kSplitUnroll];
+#pragma unroll
+        for (int u = 0; u < kSplitUnroll; ++u) {
+          const int j4 = j0 + u * kThreads;
+          v[u] = j4 < K4 ? x4[j4] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        }
+#pragma unroll
+        for (int u = 0; u < kSplitUnroll; ++u) {
+          const int j4 = j0 + u * kThreads;
+          if (j4 < K128 / 4) {
+            const uint32_t om = j4 < K4 ? omask_nibble(omask, j4) : 0xFu;
+            const int q0 = (om & 1u) ? 0 : quantize_exact(v[u].x, s, rinv);
+            const int q1 = (om & 2u) ? 0 : quantize_exact(v[u].y, s, rinv);
+            const int q2 = (om & 4u) ? 0 : quantize_exact(v[u].z, s, rinv);
+            const int q3 = (om & 8u) ? 0 : quantize_exact(v[u].w, s, rinv);
+            q4[j4] = (uint32_t)(q0 & 0xFF) | ((uint32_t)(q1 & 0xFF) << 8) |
+                     ((uint32_t)(q2 & 0xFF) << 16) | ((uint32_t)(q3 & 0xFF) << 24);
+          }
+        }
+      }
+    } else {
+      for (int j = threadIdx.x; j < K128; j += kThreads) {
+        int q = 0;
+        if (j < p.K && !((omask[j >> 5] >> (j & 31)) & 1u)) q = quantize_exact(xt[j], s, rinv);
+        xq_s[t * K128 + j] = (int8_t)q;
+      }
     }
     for (int i = threadIdx.x; i < p.n_out; i += kThreads) {
       const int j = p.idx[i];
@@ -509,11 +578,18 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
   }
 
   // ---- row blocks shared by warps ---------------------------------------------
-  __syncthreads();
-  if (t0 >= t1) return;
   const int cta_w0 = blockIdx.x * kWarps;
   const int T0c = warp_begin(cta_w0, p);
   const int T1c = warp_begin(cta_w0 + kWarps, p);
+  // row scales of the row block this CTA continues (warp 0 finishes it),
+  // loaded while the CTA's other warps finish their ranges
+  float ah0 = 0.0f, ah1 = 0.0f;
+  if (warp == 0 && t0 < t1 && T0c % p.tpr != 0) {
+    ah0 = __ldg(p.alpha + (T0c / p.tpr) * kTileRows + gid);
+    ah1 = __ldg(p.alpha + (T0c / p.tpr) * kTileRows + gid + 8);
+  }
+  __syncthreads();
+  if (t0 >= t1) return;
   const int last_w = tile_warp(T1c - 1, p) - cta_w0;  // last warp of this CTA with tiles
 
   // Sums, in warp order, the shared-memory parts of warps [w_lo, w_hi] of
@@ -529,19 +605,17 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
 
   // Publishes this CTA's part of row block r (global slot `slot`) and, if
   // this CTA is the last of those sharing r to arrive, finishes r.
-  auto arrive = [&](int r, int slot, float4 (&v)[4]) {
+  auto arrive = [&](int r, int slot, float4 (&v)[4], float a0, float a1) {
     float4* mine = p.ws_part + ((size_t)blockIdx.x * 2 + slot) * 4 * 32 + lane;
 #pragma unroll
     for (int i = 0; i < 4; ++i) __stcg(mine + i * 32, v[i]);
-    __threadfence();
     __syncwarp();
     const int b_first = tile_warp(r * p.tpr, p) / kWarps;
     const int b_last = tile_warp(r * p.tpr + p.tpr - 1, p) / kWarps;
     int prev = 0;
-    if (lane == 0) prev = atomicAdd(&p.ws_cnt[r], 1);
-    prev = __shfl_sync(0xffffffffu, prev, 0);
+    if (lane == 0) prev = arrive_acq_rel(&p.ws_cnt[r]);
+    prev = __shfl_sync(0xffffffffu, prev, 0);  // also orders the lanes' loads below
     if (prev != b_last - b_first) return;
-    __threadfence();
     // the CTAs' parts in CTA order, loaded in batches before they are added
     constexpr int kBatch = 4;
     const int n = b_last - b_first + 1;
@@ -570,8 +644,7 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
         }
       }
     }
-    write_y(p, r, gid, tid4, v, __ldg(p.alpha + r * kTileRows + gid),
-            __ldg(p.alpha + r * kTileRows + gid + 8), sx0, sx1);
+    write_y(p, r, gid, tid4, v, a0, a1, sx0, sx1);
     if (lane == 0) p.ws_cnt[r] = 0;
   };
 
@@ -581,9 +654,10 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
     const int w_hi = tile_warp(min((r + 1) * p.tpr, T1c) - 1, p) - cta_w0;
     float4 v[4];
     sum_smem(v, 0, 0, w_hi);
-    arrive(r, 0, v);
+    arrive(r, 0, v, ah0, ah1);
   }
-  // the row block whose first tile is in this warp's range and whose end lies past it
+  // the row block whose first tile is in this warp's range and whose end lies
+  // past it (al0 / al1 still hold its row scales)
   const int rb_last = (t1 - 1) / p.tpr;
   if (rb_last * p.tpr >= t0 && t1 % p.tpr != 0) {
     const int r = rb_last;
@@ -591,11 +665,10 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
     float4 v[4];
     if (end <= T1c) {
       sum_smem(v, warp, 1, tile_warp(end - 1, p) - cta_w0);
-      write_y(p, r, gid, tid4, v, __ldg(p.alpha + r * kTileRows + gid),
-              __ldg(p.alpha + r * kTileRows + gid + 8), sx0, sx1);
+      write_y(p, r, gid, tid4, v, al0, al1, sx0, sx1);
     } else {
       sum_smem(v, warp, 1, last_w);
-      arrive(r, 1, v);
+      arrive(r, 1, v, al0, al1);
     }
   }
 }

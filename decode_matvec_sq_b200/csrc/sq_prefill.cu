@@ -58,7 +58,7 @@ struct Aux {
   uint64_t accf[2], acce[2], tdone;
   uint32_t tmem_base;
   int abort;
-  float scl[2][BN];  // group scales of the CTA's rows, double buffered
+  float scl[4][BN];  // group scales of the CTA's rows: a ring, loaded two groups ahead
   float alpha[BN];
 };
 constexpr int kSmemBytes = kStages * kStageBytes + (int)sizeof(Aux) + 1024;  // + alignment slack
@@ -286,14 +286,22 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
     for (int n = 0; n < BN; ++n) F[n] = 0.0f;
     const int ng = p.nk;
+    // group scales: thread et < BN owns row n0 + et; the scale of group kb + 2
+    // is loaded while group kb is promoted and stored one group ahead
+    const int sn = n0 + et;
+    const bool srow = et < BN && sn < p.N;
+    const float* srow_p = p.scale + (int64_t)(srow ? sn : 0) * p.scale_stride;
+    if (et < BN) aux->scl[0][et] = srow ? __ldg(srow_p) : 0.0f;
+    float s_next = (srow && p.nk > 1) ? __ldg(srow_p + 1) : 0.0f;
     // Every epilogue thread runs every iteration and meets every named
     // barrier; whether a warp reads TMEM is decided per warp (tcgen05.ld is
     // warp-collective), and after a timeout the rest is skipped.
     for (int kb = 0; kb < p.nk; ++kb) {
       const int b = kb & 1;
-      if (et < BN) {
-        const int n = n0 + et;
-        aux->scl[b][et] = n < p.N ? __ldg(p.scale + (int64_t)n * p.scale_stride + kb) : 0.0f;
+      const float* scl = aux->scl[kb & 3];
+      if (et < BN && kb + 1 < p.nk) {
+        aux->scl[(kb + 1) & 3][et] = s_next;
+        s_next = (srow && kb + 2 < p.nk) ? __ldg(srow_p + kb + 2) : 0.0f;
       }
       named_sync_epi();
       bool ok = !aborted(aux) && wait_or_abort(&aux->accf[b], (uint32_t)(kb >> 1) & 1u, aux, p.status);
@@ -309,7 +317,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           mbar_arrive(&aux->acce[b]);
         }
 #pragma unroll
-        for (int i = 0; i < 32; ++i) F[32 * h + i] = fmaf(aux->scl[b][32 * h + i], (float)r[i], F[32 * h + i]);
+        for (int i = 0; i < 32; ++i) F[32 * h + i] = fmaf(scl[32 * h + i], (float)r[i], F[32 * h + i]);
         if (EMIT && t < p.M) {
           for (int i = 0; i < 32; ++i) {
             const int n = n0 + 32 * h + i;
