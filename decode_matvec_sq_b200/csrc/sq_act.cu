@@ -90,14 +90,15 @@ __global__ void __launch_bounds__(kActThreads) k_quantize_act(
   for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
 
   const float s = act_scale(a);
-  const double rinv = act_rinv(s);
+  const float rinv = act_rinv(s);
   if (threadIdx.x == 0) sx[t] = s;
 
   int8_t* qt = xq + (int64_t)t * Kx;
+  const bool fast = quantize_fast_ok(s, a);  // one branch per token
   auto emit = [&](int c, float u) {
     const int j = c * 32 + lane;
     int q = 0;
-    if (j < K && !outlier_bit(is_out, j)) q = quantize_exact(u, s, rinv);
+    if (j < K && !outlier_bit(is_out, j)) q = fast ? quantize_fast(u, s, rinv) : quantize_exact(u, s, rinv);
     qt[j] = (int8_t)q;  // j < 32 * nchunk <= Kx
   };
 #pragma unroll

@@ -50,6 +50,10 @@ constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
 constexpr int kBps = 2;    // CTAs per SM
 constexpr int kDepth = 3;  // tiles in flight per warp
+// Fused mode: tiles prefetched before the activation split.  The split's
+// loads of x must not queue behind a full ring of weight loads, so only the
+// first tile is in flight while it runs; the rest follow it.
+constexpr int kDepthEarly = 1;
 constexpr int kCols = 8;   // tokens per pass (MMA N)
 
 struct Params {
@@ -60,7 +64,7 @@ struct Params {
   const float* scale;
   int N, K, tpr;    // rows, channels, tiles per row block
   int T;            // tiles = ceil(N / 16) * tpr
-  int warps_total;  // warps that own tiles: min(gridDim.x * kWarps, T)
+  int n_rb;         // row blocks = ceil(N / 16); CTA b owns [b*n_rb/grid, (b+1)*n_rb/grid)
   int M;            // tokens in this pass (<= 8)
   const int8_t* xq;
   int xs;           // row stride of xq (roundup(K, 128))
@@ -71,8 +75,6 @@ struct Params {
   float* y;
   int32_t* T_out;
   int32_t* R_out;
-  float4* ws_part;  // [CTA][slot 0/1][cell 0..3][lane] {T bits, F, Ut, Ur}
-  int32_t* ws_cnt;  // [row block] arrival counters
   int pdl;
   // fused mode
   const float* x;     // [M][K] activations
@@ -81,22 +83,20 @@ struct Params {
   int off_xq, off_xo, off_sx, off_red;  // shared-memory offsets (bytes)
 };
 
-// First tile of warp w (w >= warps_total: T, an empty range).
-__device__ __forceinline__ int warp_begin(int w, const Params& p) {
-  return w >= p.warps_total ? p.T : (int)((int64_t)w * p.T / p.warps_total);
+// Work split: CTA b owns whole row blocks [b*n_rb/grid, (b+1)*n_rb/grid), so
+// no row block is shared between CTAs; its tiles are split evenly over its
+// warps (a row block may be shared by warps of the CTA).
+__device__ __forceinline__ int cta_first_tile(int b, const Params& p) {
+  return (int)((int64_t)b * p.n_rb / gridDim.x) * p.tpr;
 }
-// The warp whose range holds tile t.
-__device__ __forceinline__ int tile_warp(int t, const Params& p) {
-  return (int)(((int64_t)(t + 1) * p.warps_total + p.T - 1) / p.T) - 1;
+// First tile of warp i of the CTA whose tiles are [T0, T1).
+__device__ __forceinline__ int warp_first_tile(int i, int T0, int T1) {
+  return T0 + (int)((int64_t)i * (T1 - T0) / kWarps);
 }
-
-// Arrival on a row block's counter: release orders this warp's partial-sum
-// stores (made visible to lane 0 by __syncwarp) before the increment; acquire
-// orders the finisher's loads of the other CTAs' partials after it.
-__device__ __forceinline__ int arrive_acq_rel(int32_t* cnt) {
-  int prev;
-  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;" : "=r"(prev) : "l"(cnt) : "memory");
-  return prev;
+// The warp of that CTA whose range holds tile t.
+__device__ __forceinline__ int tile_warp(int t, int T0, int T1) {
+  const int len = T1 - T0;
+  return (int)(((int64_t)(t - T0 + 1) * kWarps + len - 1) / len) - 1;
 }
 
 __device__ __forceinline__ void mma_s8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
@@ -243,47 +243,87 @@ __device__ __forceinline__ void write_y(const Params& p, int rb, int gid, int ti
 // Fused mode: the activation split of the pass's tokens into shared memory
 // (codes [M][K128], outlier values [M][n_pad], scales [M]); outlier channels
 // are those marked in omask.  Same arithmetic as the activation split kernel.
-// x is read as float4 (when rows are 16-byte aligned), eight loads in flight
-// per thread, so the two passes take few memory round trips.
-constexpr int kSplitUnroll = 8;
+// Latency is what counts here (the weight stream waits for the codes): for
+// K <= 16384 each thread keeps its share of a token's x in registers (float4,
+// all loads in flight at once), so a token costs one memory round trip and
+// one barrier; the outlier values are gathered with the same round trip.
+constexpr int kXRegs = 16;  // float4 per thread kept in registers: K <= 16384
 
 __device__ __forceinline__ uint32_t omask_nibble(const uint32_t* omask, int j4) {
   return (omask[j4 >> 3] >> ((j4 & 7) * 4)) & 0xFu;  // outlier bits of channels 4*j4 .. 4*j4+3
 }
 
+template <bool FAST>
+__device__ __forceinline__ int qcode(float v, float s, float rinv) {
+  return FAST ? quantize_fast(v, s, rinv) : quantize_exact(v, s, rinv);
+}
+template <bool FAST>
+__device__ __forceinline__ uint32_t pack_codes(float4 v, uint32_t om, float s, float rinv) {
+  const int q0 = (om & 1u) ? 0 : qcode<FAST>(v.x, s, rinv);
+  const int q1 = (om & 2u) ? 0 : qcode<FAST>(v.y, s, rinv);
+  const int q2 = (om & 4u) ? 0 : qcode<FAST>(v.z, s, rinv);
+  const int q3 = (om & 8u) ? 0 : qcode<FAST>(v.w, s, rinv);
+  return (uint32_t)(q0 & 0xFF) | ((uint32_t)(q1 & 0xFF) << 8) | ((uint32_t)(q2 & 0xFF) << 16) |
+         ((uint32_t)(q3 & 0xFF) << 24);
+}
+
+__device__ __forceinline__ float absmax4(float4 v, uint32_t om, float a, bool& nonfinite) {
+  nonfinite |= !isfinite(v.x) || !isfinite(v.y) || !isfinite(v.z) || !isfinite(v.w);
+  if (!(om & 1u)) a = fmaxf(a, fabsf(v.x));
+  if (!(om & 2u)) a = fmaxf(a, fabsf(v.y));
+  if (!(om & 4u)) a = fmaxf(a, fabsf(v.z));
+  if (!(om & 8u)) a = fmaxf(a, fabsf(v.w));
+  return a;
+}
+
+// jv, jp: this thread's entry of the outlier list and the one before it
+// (threads < n_out, loaded in the prologue).
 __device__ __forceinline__ void split_activations(const Params& p, const uint32_t* omask,
                                                   int8_t* xq_s, float* xo_s, float* sx_s,
-                                                  float* red_s) {
+                                                  float* red_s, int jv, int jp) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int K128 = p.xs;
+  const int K4 = p.K >> 2, Kq = K128 >> 2;
   const bool vec = (p.K & 3) == 0 && (reinterpret_cast<uintptr_t>(p.x) & 15u) == 0;
-  const int K4 = p.K >> 2;
+  const bool in_regs = vec && Kq <= kXRegs * kThreads;
   bool nonfinite = false;
+  bool bad_idx = false;
+  // the index list is checked once (strictly ascending, inside [0, K))
+  for (int i = threadIdx.x; i < p.n_out; i += kThreads) {
+    const int j = i < kThreads ? jv : p.idx[i];
+    const int jq = i < kThreads ? jp : p.idx[i - 1];
+    bad_idx |= j < 0 || j >= p.K || (i > 0 && jq >= j);
+  }
   for (int t = 0; t < p.M; ++t) {
     const float* xt = p.x + (int64_t)t * p.K;
+    uint32_t* q4 = reinterpret_cast<uint32_t*>(xq_s + t * K128);
+    // outlier values of this token, loaded alongside x
+    if (threadIdx.x < p.n_out)
+      xo_s[t * p.n_pad + threadIdx.x] = (jv >= 0 && jv < p.K) ? xt[jv] : 0.0f;
+    for (int i = threadIdx.x + kThreads; i < p.n_out; i += kThreads) {
+      const int j = p.idx[i];
+      xo_s[t * p.n_pad + i] = (j >= 0 && j < p.K) ? xt[j] : 0.0f;
+    }
     float a = 0.0f;
-    if (vec) {
+    float4 xr[kXRegs];
+    if (in_regs) {
       const float4* x4 = reinterpret_cast<const float4*>(xt);
-      for (int j0 = threadIdx.x; j0 < K4; j0 += kThreads * kSplitUnroll) {
-        float4 v[kSplitUnroll];
+      // (every loop over u stops at a bound that is the same for the whole CTA)
 #pragma unroll
-        for (int u = 0; u < kSplitUnroll; ++u) {
-          const int j4 = j0 + u * kThreads;
-          v[u] = j4 < K4 ? x4[j4] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-        }
-#pragma unroll
-        for (int u = 0; u < kSplitUnroll; ++u) {
-          const int j4 = j0 + u * kThreads;
-          if (j4 < K4) {
-            const uint32_t om = omask_nibble(omask, j4);
-            nonfinite |= !isfinite(v[u].x) || !isfinite(v[u].y) || !isfinite(v[u].z) || !isfinite(v[u].w);
-            if (!(om & 1u)) a = fmaxf(a, fabsf(v[u].x));
-            if (!(om & 2u)) a = fmaxf(a, fabsf(v[u].y));
-            if (!(om & 4u)) a = fmaxf(a, fabsf(v[u].z));
-            if (!(om & 8u)) a = fmaxf(a, fabsf(v[u].w));
-          }
-        }
+      for (int u = 0; u < kXRegs; ++u) {
+        if (u * kThreads >= K4) break;
+        const int j4 = threadIdx.x + u * kThreads;
+        xr[u] = j4 < K4 ? x4[j4] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
       }
+#pragma unroll
+      for (int u = 0; u < kXRegs; ++u) {
+        if (u * kThreads >= K4) break;
+        const int j4 = threadIdx.x + u * kThreads;
+        if (j4 < K4) a = absmax4(xr[u], omask_nibble(omask, j4), a, nonfinite);
+      }
+    } else if (vec) {
+      const float4* x4 = reinterpret_cast<const float4*>(xt);
+      for (int j4 = threadIdx.x; j4 < K4; j4 += kThreads) a = absmax4(x4[j4], omask_nibble(omask, j4), a, nonfinite);
     } else {
       for (int j = threadIdx.x; j < p.K; j += kThreads) {
         const float v = xt[j];
@@ -292,56 +332,40 @@ __device__ __forceinline__ void split_activations(const Params& p, const uint32_
       }
     }
     for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-    if (lane == 0) red_s[warp * kCols + t] = a;
-  }
-  __syncthreads();
-  if (threadIdx.x < p.M) {
-    float a = 0.0f;
-    for (int w = 0; w < kWarps; ++w) a = fmaxf(a, red_s[w * kCols + threadIdx.x]);
-    sx_s[threadIdx.x] = act_scale(a);
-  }
-  __syncthreads();
-  bool bad_idx = false;
-  for (int t = 0; t < p.M; ++t) {
-    const float* xt = p.x + (int64_t)t * p.K;
-    const float s = sx_s[t];
-    const double rinv = act_rinv(s);
-    uint32_t* q4 = reinterpret_cast<uint32_t*>(xq_s + t * K128);
-    if (vec) {
-      const float4* x4 = reinterpret_cast<const float4*>(xt);
-      for (int j0 = threadIdx.x; j0 < K128 / 4; j0 += kThreads * kSplitUnroll) {
-        float4 v[kSplitUnroll];
+    if (lane == 0) red_s[(t & 1) * kWarps + warp] = a;  // two buffers: token t+1 may start early
+    __syncthreads();
+    a = 0.0f;
 #pragma unroll
-        for (int u = 0; u < kSplitUnroll; ++u) {
-          const int j4 = j0 + u * kThreads;
-          v[u] = j4 < K4 ? x4[j4] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-        }
+    for (int w = 0; w < kWarps; ++w) a = fmaxf(a, red_s[(t & 1) * kWarps + w]);
+    const float s = act_scale(a);
+    const float rinv = act_rinv(s);
+    if (threadIdx.x == 0) sx_s[t] = s;
+    // one branch per token: the common range needs no per-element test
+    const bool fast = quantize_fast_ok(s, a);
+    if (in_regs && fast) {
 #pragma unroll
-        for (int u = 0; u < kSplitUnroll; ++u) {
-          const int j4 = j0 + u * kThreads;
-          if (j4 < K128 / 4) {
-            const uint32_t om = j4 < K4 ? omask_nibble(omask, j4) : 0xFu;
-            const int q0 = (om & 1u) ? 0 : quantize_exact(v[u].x, s, rinv);
-            const int q1 = (om & 2u) ? 0 : quantize_exact(v[u].y, s, rinv);
-            const int q2 = (om & 4u) ? 0 : quantize_exact(v[u].z, s, rinv);
-            const int q3 = (om & 8u) ? 0 : quantize_exact(v[u].w, s, rinv);
-            q4[j4] = (uint32_t)(q0 & 0xFF) | ((uint32_t)(q1 & 0xFF) << 8) |
-                     ((uint32_t)(q2 & 0xFF) << 16) | ((uint32_t)(q3 & 0xFF) << 24);
-          }
-        }
+      for (int u = 0; u < kXRegs; ++u) {
+        if (u * kThreads >= Kq) break;
+        const int j4 = threadIdx.x + u * kThreads;
+        if (j4 < Kq) q4[j4] = j4 < K4 ? pack_codes<true>(xr[u], omask_nibble(omask, j4), s, rinv) : 0u;
       }
+    } else if (in_regs) {
+#pragma unroll
+      for (int u = 0; u < kXRegs; ++u) {
+        if (u * kThreads >= Kq) break;
+        const int j4 = threadIdx.x + u * kThreads;
+        if (j4 < Kq) q4[j4] = j4 < K4 ? pack_codes<false>(xr[u], omask_nibble(omask, j4), s, rinv) : 0u;
+      }
+    } else if (vec) {
+      const float4* x4 = reinterpret_cast<const float4*>(xt);
+      for (int j4 = threadIdx.x; j4 < Kq; j4 += kThreads)
+        q4[j4] = j4 < K4 ? pack_codes<false>(x4[j4], omask_nibble(omask, j4), s, rinv) : 0u;
     } else {
       for (int j = threadIdx.x; j < K128; j += kThreads) {
         int q = 0;
         if (j < p.K && !((omask[j >> 5] >> (j & 31)) & 1u)) q = quantize_exact(xt[j], s, rinv);
         xq_s[t * K128 + j] = (int8_t)q;
       }
-    }
-    for (int i = threadIdx.x; i < p.n_out; i += kThreads) {
-      const int j = p.idx[i];
-      const bool in = j >= 0 && j < p.K;
-      bad_idx |= !in || (i > 0 && p.idx[i - 1] >= j);
-      xo_s[t * p.n_pad + i] = in ? xt[j] : 0.0f;
     }
   }
   if (nonfinite) set_status(p.status, SQ_ERR_NONFINITE);
@@ -360,8 +384,8 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gid = lane >> 2, tid4 = lane & 3;
-  const int gw = blockIdx.x * kWarps + warp;
-  const int t0 = warp_begin(gw, p), t1 = warp_begin(gw + 1, p);
+  const int T0c = cta_first_tile(blockIdx.x, p), T1c = cta_first_tile(blockIdx.x + 1, p);
+  const int t0 = warp_first_tile(warp, T0c, T1c), t1 = warp_first_tile(warp + 1, T0c, T1c);
 
   // ---- the outlier index list first (small loads ahead of the stream)
   const int my_i = threadIdx.x;
@@ -379,8 +403,9 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
     cur.scale = p.scale + (int64_t)t0 * 16 + gid;
   }
   Tile<MASK> buf[kDepth];
+  constexpr int kEarly = FUSED ? kDepthEarly : kDepth;
 #pragma unroll
-  for (int d = 0; d < kDepth; ++d) {
+  for (int d = 0; d < kEarly; ++d) {
     if (t0 + d < t1) load_tile<MASK>(buf[d], cur);
     cur.advance();
   }
@@ -402,8 +427,14 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
   int8_t* xq_s = reinterpret_cast<int8_t*>(smem + p.off_xq);
   float* xo_s = reinterpret_cast<float*>(smem + p.off_xo);
   float* sx_s = reinterpret_cast<float*>(smem + p.off_sx);
-  if constexpr (FUSED)
-    split_activations(p, omask, xq_s, xo_s, sx_s, reinterpret_cast<float*>(smem + p.off_red));
+  if constexpr (FUSED) {
+    split_activations(p, omask, xq_s, xo_s, sx_s, reinterpret_cast<float*>(smem + p.off_red), jv, jp);
+#pragma unroll
+    for (int d = kEarly; d < kDepth; ++d) {
+      if (t0 + d < t1) load_tile<MASK>(buf[d], cur);
+      cur.advance();
+    }
+  }
 
   // tokens of this lane's accumulator columns; the B operand of this lane
   // (MMA column gid) is token min(gid, M - 1): columns past M are not written
@@ -577,99 +608,25 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
     }
   }
 
-  // ---- row blocks shared by warps ---------------------------------------------
-  const int cta_w0 = blockIdx.x * kWarps;
-  const int T0c = warp_begin(cta_w0, p);
-  const int T1c = warp_begin(cta_w0 + kWarps, p);
-  // row scales of the row block this CTA continues (warp 0 finishes it),
-  // loaded while the CTA's other warps finish their ranges
-  float ah0 = 0.0f, ah1 = 0.0f;
-  if (warp == 0 && t0 < t1 && T0c % p.tpr != 0) {
-    ah0 = __ldg(p.alpha + (T0c / p.tpr) * kTileRows + gid);
-    ah1 = __ldg(p.alpha + (T0c / p.tpr) * kTileRows + gid + 8);
-  }
+  // ---- row blocks shared by warps of this CTA ---------------------------------
   __syncthreads();
   if (t0 >= t1) return;
-  const int last_w = tile_warp(T1c - 1, p) - cta_w0;  // last warp of this CTA with tiles
-
-  // Sums, in warp order, the shared-memory parts of warps [w_lo, w_hi] of
-  // this CTA for one row block; warp w_lo contributes slot s_lo, the rest
-  // slot 0 (their ranges start inside the row block).
-  auto sum_smem = [&](float4 (&v)[4], int w_lo, int s_lo, int w_hi) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) v[i] = part_s[((w_lo * 2 + s_lo) * 4 + i) * 32 + lane];
-    for (int w = w_lo + 1; w <= w_hi; ++w)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) cell_add(v[i], part_s[((w * 2) * 4 + i) * 32 + lane]);
-  };
-
-  // Publishes this CTA's part of row block r (global slot `slot`) and, if
-  // this CTA is the last of those sharing r to arrive, finishes r.
-  auto arrive = [&](int r, int slot, float4 (&v)[4], float a0, float a1) {
-    float4* mine = p.ws_part + ((size_t)blockIdx.x * 2 + slot) * 4 * 32 + lane;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) __stcg(mine + i * 32, v[i]);
-    __syncwarp();
-    const int b_first = tile_warp(r * p.tpr, p) / kWarps;
-    const int b_last = tile_warp(r * p.tpr + p.tpr - 1, p) / kWarps;
-    int prev = 0;
-    if (lane == 0) prev = arrive_acq_rel(&p.ws_cnt[r]);
-    prev = __shfl_sync(0xffffffffu, prev, 0);  // also orders the lanes' loads below
-    if (prev != b_last - b_first) return;
-    // the CTAs' parts in CTA order, loaded in batches before they are added
-    constexpr int kBatch = 4;
-    const int n = b_last - b_first + 1;
-    for (int c0 = 0; c0 < n; c0 += kBatch) {
-      float4 got[kBatch][4];
-#pragma unroll
-      for (int k = 0; k < kBatch; ++k) {
-        if (c0 + k < n) {
-          const int b = b_first + c0 + k;
-          const int s = warp_begin(b * kWarps, p) > r * p.tpr ? 0 : 1;
-          const float4* src = p.ws_part + ((size_t)b * 2 + s) * 4 * 32 + lane;
-#pragma unroll
-          for (int i = 0; i < 4; ++i) got[k][i] = __ldcg(src + i * 32);
-        }
-      }
-#pragma unroll
-      for (int k = 0; k < kBatch; ++k) {
-        if (c0 + k < n) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            if (c0 + k == 0)
-              v[i] = got[k][i];
-            else
-              cell_add(v[i], got[k][i]);
-          }
-        }
-      }
-    }
-    write_y(p, r, gid, tid4, v, a0, a1, sx0, sx1);
-    if (lane == 0) p.ws_cnt[r] = 0;
-  };
-
-  // the row block this CTA continues from an earlier CTA: warp 0 gathers it
-  if (warp == 0 && T0c % p.tpr != 0) {
-    const int r = T0c / p.tpr;
-    const int w_hi = tile_warp(min((r + 1) * p.tpr, T1c) - 1, p) - cta_w0;
-    float4 v[4];
-    sum_smem(v, 0, 0, w_hi);
-    arrive(r, 0, v, ah0, ah1);
-  }
   // the row block whose first tile is in this warp's range and whose end lies
-  // past it (al0 / al1 still hold its row scales)
+  // past it: this warp adds the parts of the CTA's later warps, in warp order
+  // (al0 / al1 still hold its row scales)
   const int rb_last = (t1 - 1) / p.tpr;
   if (rb_last * p.tpr >= t0 && t1 % p.tpr != 0) {
-    const int r = rb_last;
-    const int end = (r + 1) * p.tpr;
+    const int w_hi = tile_warp((rb_last + 1) * p.tpr - 1, T0c, T1c);
     float4 v[4];
-    if (end <= T1c) {
-      sum_smem(v, warp, 1, tile_warp(end - 1, p) - cta_w0);
-      write_y(p, r, gid, tid4, v, al0, al1, sx0, sx1);
-    } else {
-      sum_smem(v, warp, 1, last_w);
-      arrive(r, 1, v, al0, al1);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = part_s[((warp * 2 + 1) * 4 + i) * 32 + lane];
+    for (int w = warp + 1; w <= w_hi; ++w) {
+      // a CTA with fewer tiles than warps has empty warps between its owners
+      if (warp_first_tile(w, T0c, T1c) == warp_first_tile(w + 1, T0c, T1c)) continue;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) cell_add(v[i], part_s[((w * 2) * 4 + i) * 32 + lane]);
     }
+    write_y(p, rb_last, gid, tid4, v, al0, al1, sx0, sx1);
   }
 }
 
@@ -693,9 +650,9 @@ cudaError_t launch_one(const Params& p, int grid, int smem, bool pdl, cudaStream
 
 }  // namespace
 
-size_t linear_tc_part_bytes(int sm_count) {
-  // per CTA: two slots of 4 cells x 32 lanes x float4
-  return (size_t)sm_count * kBps * 2 * 4 * 32 * sizeof(float4);
+size_t linear_tc_part_bytes(int) {
+  // no row block is shared between CTAs: the workspace is not used
+  return 0;
 }
 
 namespace {
@@ -736,9 +693,8 @@ cudaError_t launch_linear_tc(const sq_packed_weight& w, int M, const int8_t* xq,
   const int64_t T = ceil_div(w.N, kTileRows) * (int64_t)p.tpr;
   if (T >= INT32_MAX / 2) return cudaErrorInvalidValue;
   p.T = (int)T;
-  const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((int64_t)sm_count * kBps,
-                                                                ceil_div(T, 2 * kWarps)));
-  p.warps_total = (int)std::min<int64_t>(blocks * kWarps, T);
+  p.n_rb = (int)ceil_div(w.N, kTileRows);
+  const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((int64_t)sm_count * kBps, p.n_rb));
   p.M = M;
   p.xq = xq;
   p.xs = (int)xq_stride_of(w.K);
@@ -749,8 +705,8 @@ cudaError_t launch_linear_tc(const sq_packed_weight& w, int M, const int8_t* xq,
   p.y = y;
   p.T_out = T_out;
   p.R_out = R_out;
-  p.ws_part = reinterpret_cast<float4*>(workspace);
-  p.ws_cnt = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(workspace) + part_bytes);
+  (void)workspace;
+  (void)part_bytes;
   p.pdl = pdl ? 1 : 0;
   p.x = x;
   p.status = status;
