@@ -253,7 +253,7 @@ sq_status sq_quantize_linear(const sq_packed_weight *w, const float *x, int32_t 
  *   (16 MiB) per device, inside this library.  Nothing is allocated.
  *   Limit: a call whose sq_linear_workspace_bytes(w, M) exceeds that size
  *   returns SQ_ERR_WORKSPACE before any device work (on a 148-SM B200: more
- *   than 4,156,416 rows).
+ *   than 4,118,528 rows).
  *   First call on each device: looks up the array's device address
  *   (cudaGetSymbolAddress, with that device current) and zero-fills the
  *   array on `stream` before its launch, because the per-row arrival
