@@ -419,6 +419,14 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
   };
   if (my_i < p.n_out) add_outlier(my_i, jv, jp);
   for (int i = my_i + kThreads; i < p.n_out; i += kThreads) add_outlier(i, p.idx[i], p.idx[i - 1]);
+  if (FUSED && p.pdl) {
+    // warm L2 with the activations while the previous kernel finishes (a
+    // prefetch moves no data to the SM, so it cannot return stale values)
+    const char* xb = reinterpret_cast<const char*>(p.x);
+    const int64_t xbytes = (int64_t)p.M * p.K * 4;
+    for (int64_t o = (int64_t)threadIdx.x * 128; o < xbytes; o += kThreads * 128)
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(xb + o));
+  }
   __syncthreads();
   if (p.pdl) {
     pdl_wait();

@@ -41,13 +41,16 @@ __device__ __forceinline__ float act_rinv(float s) { return s != 0.0f ? __frcp_r
 __device__ __forceinline__ bool quantize_fast_ok(float s, float absmax) {
   return s > 0x1p-100f && absmax < 0x1p100f;
 }
+// floor(t) for 0 <= t < 2^22 without a conversion instruction: t + 2^23
+// rounded down is 2^23 + floor(t) exactly, whose low mantissa bits are the
+// integer.
 __device__ __forceinline__ int quantize_fast(float v, float s, float rinv) {
   const float av = fabsf(v);
-  const float k = floorf(__fmul_rn(av, rinv));
-  float q = fmaf(k + 0.5f, s, -av) <= 0.0f ? k + 1.0f : k;
-  q = q < 127.0f ? q : 127.0f;
-  const int qi = (int)q;
-  return v < 0.0f ? -qi : qi;
+  const float f = __fadd_rd(__fmul_rn(av, rinv), 8388608.0f);  // 2^23 + k
+  const float k = __fsub_rn(f, 8388608.0f);
+  int q = (__float_as_int(f) - 0x4B000000) + (fmaf(k + 0.5f, s, -av) <= 0.0f ? 1 : 0);
+  q = min(q, 127);
+  return v < 0.0f ? -q : q;
 }
 
 __device__ __forceinline__ int quantize_exact(float v, float s, float rinv) {
