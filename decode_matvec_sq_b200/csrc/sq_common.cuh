@@ -1,8 +1,8 @@
 // sq_common.cuh -- device helpers shared by the kernels of libsq (sm_100a).
 //
-// Thin wrappers over PTX: shared-memory mbarriers, the bulk (non-tensor) TMA
-// copy global -> shared, L2 eviction policies, programmatic dependent launch
-// control and a wall-clock bound for every wait.
+// Thin wrappers over PTX: shared-memory mbarriers with a wall-clock bound on
+// every wait, programmatic dependent launch control, status reporting and a
+// few load / bit helpers.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -67,40 +67,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   return true;
 }
 
-__device__ __forceinline__ uint64_t l2_evict_first_policy() {
-  uint64_t p;
-  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
-  return p;
-}
-
-__device__ __forceinline__ uint64_t l2_evict_last_policy() {
-  uint64_t p;
-  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
-  return p;
-}
-
-// Bulk copy of `bytes` (multiple of 16, both addresses 16-byte aligned) from
-// global to this CTA's shared memory; completion is signalled on `bar` as
-// transaction bytes.  No cluster multicast.
-__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes,
-                                         uint64_t* bar, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(dst)),
-      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
-      : "memory");
-}
-
 // Programmatic dependent launch: wait for the preceding grid (and its memory),
 // and allow the next grid in the stream to begin launching.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-
-// Named barrier over `count` threads (a multiple of 32), id 1..15.
-__device__ __forceinline__ void named_sync(uint32_t id, uint32_t count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 __device__ __forceinline__ void set_status(int32_t* st, int32_t code) {

@@ -523,7 +523,8 @@ def _fused_vs_two_step(W, x, idx, P=-1, pdl=False):
 
 @pytest.mark.parametrize("N,K,M,n", [(1, 8, 1, 0), (7, 33, 1, 2), (40, 129, 8, 1), (20, 300, 3, 3),
                                      (513, 300, 1, 6), (64, 4096, 1, 20), (24, 11008, 1, 55),
-                                     (8, 28672, 2, 72), (100, 2048, 16, 10), (33, 1000, 13, 9)])
+                                     (8, 28672, 2, 72), (16, 28672, 5, 72), (100, 2048, 16, 10),
+                                     (33, 1000, 13, 9)])
 @pytest.mark.parametrize("P", [-1, 60])
 def test_quantize_linear_parity(N, K, M, n, P):
     rng = np.random.default_rng(7 * N + K + M + n + P)
