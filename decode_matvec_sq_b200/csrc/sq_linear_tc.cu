@@ -46,9 +46,9 @@
 namespace sq {
 namespace {
 
-constexpr int kWarps = 8;
+constexpr int kWarps = 16;
 constexpr int kThreads = kWarps * 32;
-constexpr int kBps = 2;    // CTAs per SM
+constexpr int kBps = 1;    // CTAs per SM
 constexpr int kDepth = 3;  // tiles in flight per warp
 // Fused mode: tiles prefetched before the activation split.  The split's
 // loads of x must not queue behind a full ring of weight loads, so only the
@@ -666,7 +666,7 @@ size_t linear_tc_part_bytes(int) {
 namespace {
 constexpr int kSmemPart = kWarps * 2 * 4 * 32 * (int)sizeof(float4);
 // Shared memory of one CTA stays within this so that kBps CTAs fit an SM.
-constexpr int kSmemBudget = 100 * 1024;
+constexpr int kSmemBudget = 200 * 1024;
 
 int outlier_table_bytes(const sq_packed_weight& w) { return (int)(tiles_cols(w.K) / 32) * 8; }
 int fused_token_bytes(const sq_packed_weight& w, int n_out) {
