@@ -49,11 +49,14 @@ namespace {
 constexpr int kWarps = 16;
 constexpr int kThreads = kWarps * 32;
 constexpr int kBps = 1;    // CTAs per SM
-constexpr int kDepth = 3;  // tiles in flight per warp
-// Fused mode: tiles prefetched before the activation split.  The split's
-// loads of x must not queue behind a full ring of weight loads, so only the
-// first tile is in flight while it runs; the rest follow it.
+// Fused mode: tiles copied before the activation split.  The split's loads
+// of x must not queue behind a full ring of weight loads, so only the first
+// tile is in flight while it runs; the rest follow it.
 constexpr int kDepthEarly = 1;
+// Tiles in flight per warp (the shared-memory ring).  Deeper rings measured
+// slower: two tiles per warp keep enough bytes in flight at batch <= 2, three
+// above it, where a tile takes longer to consume.
+constexpr int kDeep = 3, kShallow = 2;
 constexpr int kCols = 8;   // tokens per pass (MMA N)
 
 struct Params {
@@ -81,6 +84,7 @@ struct Params {
   int32_t* status;    // device status word (non-finite x, bad index list)
   int n_pad;          // x_out row stride in shared memory
   int off_xq, off_xo, off_sx, off_red;  // shared-memory offsets (bytes)
+  int off_ring, off_omask;
 };
 
 // Work split: CTA b owns whole row blocks [b*n_rb/grid, (b+1)*n_rb/grid), so
@@ -120,23 +124,6 @@ __device__ __forceinline__ uint32_t bits_word(uint32_t bits, int w) {
   return sign_bytes(bits << (7 - w));
 }
 
-__device__ __forceinline__ void ld_stream_v8(uint32_t* v, const void* p) {
-  asm volatile("ld.global.nc.L1::no_allocate.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-               : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]),
-                 "=r"(v[6]), "=r"(v[7])
-               : "l"(p));
-}
-__device__ __forceinline__ void ld_stream_v2(uint32_t* v, const void* p) {
-  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];"
-               : "=r"(v[0]), "=r"(v[1])
-               : "l"(p));
-}
-__device__ __forceinline__ float ld_stream_f32(const float* p) {
-  float v;
-  asm volatile("ld.global.nc.L1::no_allocate.f32 %0, [%1];" : "=f"(v) : "l"(p));
-  return v;
-}
-
 // One tile as seen by one lane.
 template <bool MASK>
 struct Tile {
@@ -146,12 +133,12 @@ struct Tile {
   float c[2];      // group scales of rows r0, r1
 };
 
-// Streaming position of one lane: the next tile to load.
+// Streaming position of one lane: its part of the next tile to copy.
 struct Cursor {
-  const uint8_t* code;   // + 2048 bytes per tile
-  const uint32_t* sign;  // + 64 words per tile
+  const uint8_t* code;   // the lane's 64 code bytes; + 2048 per tile
+  const uint32_t* sign;  // the lane's two sign words; + 64 words per tile
   const uint32_t* mask;
-  const float* scale;    // + 16 floats per tile
+  const float* scale;    // the scale of row r0 (r1: + 8); + 16 floats per tile
   __device__ __forceinline__ void advance() {
     code += 2048;
     sign += 64;
@@ -160,14 +147,76 @@ struct Cursor {
   }
 };
 
+// ---- shared-memory tile ring ------------------------------------------------------
+// Each warp streams its tiles through a ring of D slots filled by cp.async
+// (global -> shared without registers), D tiles ahead of use.  A lane copies,
+// and later reads back, only its own bytes, so the warp needs no
+// synchronisation around a slot.  Slot layout: 32 lanes x 64 code bytes, then
+// 32 x 8 sign bytes (then 32 x 8 mask bytes), then 32 x 8 bytes of the lane's
+// two scales.  Code chunk j (16 bytes) of lane L sits at L*64 + ((j + L/2) % 4)
+// * 16, so the 16-byte reads of eight consecutive lanes hit eight different
+// bank groups.  The codes bypass L1; the small sign, mask and scale copies go
+// through it, where neighbouring lanes' requests coalesce (copies of 16 bytes
+// that bypass L1 measured slower for these).
 template <bool MASK>
-__device__ __forceinline__ void load_tile(Tile<MASK>& t, const Cursor& c) {
-  ld_stream_v8(t.q, c.code);
-  ld_stream_v8(t.q + 8, c.code + 32);
-  ld_stream_v2(t.s, c.sign);
-  if constexpr (MASK) ld_stream_v2(t.m, c.mask);
-  t.c[0] = ld_stream_f32(c.scale);
-  t.c[1] = ld_stream_f32(c.scale + 8);
+struct Slot {
+  static constexpr int kSign = 2048;
+  static constexpr int kMask = kSign + 256;  // (MASK only)
+  static constexpr int kScale = MASK ? kMask + 256 : kMask;
+  static constexpr int kBytes = MASK ? 2816 : 2560;
+};
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async8(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+// All but the newest N groups of this thread's copies are complete.
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+template <bool MASK>
+__device__ __forceinline__ void copy_tile(uint32_t slot, const Cursor& c, int lane) {
+  const uint32_t cb = slot + lane * 64;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) cp_async16(cb + (((j + (lane >> 1)) & 3) << 4), c.code + 16 * j);
+  cp_async8(slot + Slot<MASK>::kSign + lane * 8, c.sign);
+  if constexpr (MASK) cp_async8(slot + Slot<MASK>::kMask + lane * 8, c.mask);
+  cp_async4(slot + Slot<MASK>::kScale + lane * 8, c.scale);
+  cp_async4(slot + Slot<MASK>::kScale + lane * 8 + 4, c.scale + 8);
+}
+
+template <bool MASK>
+__device__ __forceinline__ void read_tile(Tile<MASK>& t, const uint8_t* slot, int lane) {
+  const uint8_t* cb = slot + lane * 64;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint4 v = *reinterpret_cast<const uint4*>(cb + (((j + (lane >> 1)) & 3) << 4));
+    t.q[4 * j] = v.x;
+    t.q[4 * j + 1] = v.y;
+    t.q[4 * j + 2] = v.z;
+    t.q[4 * j + 3] = v.w;
+  }
+  const uint2 sv = *reinterpret_cast<const uint2*>(slot + Slot<MASK>::kSign + lane * 8);
+  t.s[0] = sv.x;
+  t.s[1] = sv.y;
+  if constexpr (MASK) {
+    const uint2 mv = *reinterpret_cast<const uint2*>(slot + Slot<MASK>::kMask + lane * 8);
+    t.m[0] = mv.x;
+    t.m[1] = mv.y;
+  }
+  const float2 cv = *reinterpret_cast<const float2*>(slot + Slot<MASK>::kScale + lane * 8);
+  t.c[0] = cv.x;
+  t.c[1] = cv.y;
 }
 
 // Code of channel j (0..31) of row R (0: r0, 1: r1) held in a tile's A
@@ -373,13 +422,14 @@ __device__ __forceinline__ void split_activations(const Params& p, const uint32_
   __syncthreads();
 }
 
-template <bool MASK, bool EMIT, bool FUSED>
+template <bool MASK, bool EMIT, bool FUSED, int D>
 __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
   extern __shared__ __align__(16) uint8_t smem[];
-  // shared: part[kWarps][2][4][32] float4 | omask[nw] u32 | obase[nw] i32
+  // shared: part [kWarps][2 slots][16 rows][M tokens] float4 | omask[nw] u32 |
+  // obase[nw] i32 | fused-mode buffers | ring [kWarps][D slots]
   float4* part_s = reinterpret_cast<float4*>(smem);
   const int nw = p.tpr * 4;  // 32-channel words of a padded row
-  uint32_t* omask = reinterpret_cast<uint32_t*>(part_s + kWarps * 2 * 4 * 32);
+  uint32_t* omask = reinterpret_cast<uint32_t*>(smem + p.off_omask);
   int* obase = reinterpret_cast<int*>(omask + nw);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -393,7 +443,7 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
   const int jp = (my_i < p.n_out && my_i > 0) ? __ldg(p.idx + my_i - 1) : -1;
   for (int i = threadIdx.x; i < nw; i += kThreads) omask[i] = 0u;
 
-  // ---- prefetch the first kDepth tiles (weights only: allowed before the wait)
+  // ---- copy the first D tiles (weights only: allowed before the wait)
   Cursor cur;
   {
     const int64_t lt = (int64_t)t0 * 32 + lane;
@@ -402,11 +452,13 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
     cur.mask = MASK ? p.mask + lt * 2 : p.sign;
     cur.scale = p.scale + (int64_t)t0 * 16 + gid;
   }
-  Tile<MASK> buf[kDepth];
-  constexpr int kEarly = FUSED ? kDepthEarly : kDepth;
+  uint8_t* ring_w = smem + p.off_ring + warp * D * Slot<MASK>::kBytes;
+  const uint32_t ring_u = smem_u32(ring_w);
+  constexpr int kEarly = FUSED ? kDepthEarly : D;
 #pragma unroll
-  for (int d = 0; d < kEarly; ++d) {
-    if (t0 + d < t1) load_tile<MASK>(buf[d], cur);
+  for (int d = 0; d < kEarly; ++d) {  // one commit group per tile, empty past the range
+    if (t0 + d < t1) copy_tile<MASK>(ring_u + d * Slot<MASK>::kBytes, cur, lane);
+    cp_async_commit();
     cur.advance();
   }
 
@@ -438,8 +490,9 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
   if constexpr (FUSED) {
     split_activations(p, omask, xq_s, xo_s, sx_s, reinterpret_cast<float*>(smem + p.off_red), jv, jp);
 #pragma unroll
-    for (int d = kEarly; d < kDepth; ++d) {
-      if (t0 + d < t1) load_tile<MASK>(buf[d], cur);
+    for (int d = kEarly; d < D; ++d) {
+      if (t0 + d < t1) copy_tile<MASK>(ring_u + d * Slot<MASK>::kBytes, cur, lane);
+      cp_async_commit();
       cur.advance();
     }
   }
@@ -469,150 +522,153 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
   }
   const uint32_t kOnes = 0x01010101u;
 
-  for (int t = t0; t < t1; t += kDepth) {
+  int slot_i = 0;
+  for (int t = t0; t < t1; ++t) {
+    cp_async_wait<D - 1>();  // this lane's copies of the tile have landed
+    Tile<MASK> tl;
+    read_tile<MASK>(tl, ring_w + slot_i * Slot<MASK>::kBytes, lane);
+    // activation codes of this lane's 32 channels for its MMA column
+    uint32_t xw[8];
+    {
+      const int4* xp = reinterpret_cast<const int4*>(xrow + cg * kTileK);
+      int4 a, b;
+      if constexpr (FUSED) {
+        a = xp[0];
+        b = xp[1];
+      } else {
+        a = __ldg(xp);
+        b = __ldg(xp + 1);
+      }
+      xw[0] = a.x; xw[1] = a.y; xw[2] = a.z; xw[3] = a.w;
+      xw[4] = b.x; xw[5] = b.y; xw[6] = b.z; xw[7] = b.w;
+    }
+    const uint32_t pb0 = MASK ? (tl.s[0] & tl.m[0]) : tl.s[0];
+    const uint32_t pb1 = MASK ? (tl.s[1] & tl.m[1]) : tl.s[1];
+    int R[4] = {0, 0, 0, 0};
 #pragma unroll
-    for (int d = 0; d < kDepth; ++d) {
-      if (t + d < t1) {
-        Tile<MASK>& tl = buf[d];
-        // activation codes of this lane's 32 channels for its MMA column
-        uint32_t xw[8];
-        {
-          const int4* xp = reinterpret_cast<const int4*>(xrow + cg * kTileK);
-          int4 a, b;
+    for (int m = 0; m < 4; ++m) {
+      const uint32_t b0 = xw[2 * m], b1 = xw[2 * m + 1];
+      mma_s8(R, tl.q[4 * m], tl.q[4 * m + 1], tl.q[4 * m + 2], tl.q[4 * m + 3], b0, b1);
+      mma_s8(acc.Pn, bits_word(pb0, 2 * m), bits_word(pb1, 2 * m), bits_word(pb0, 2 * m + 1),
+             bits_word(pb1, 2 * m + 1), b0, b1);
+      if constexpr (MASK)
+        mma_s8(acc.S, bits_word(tl.m[0], 2 * m), bits_word(tl.m[1], 2 * m),
+               bits_word(tl.m[0], 2 * m + 1), bits_word(tl.m[1], 2 * m + 1), b0, b1);
+      else
+        mma_s8(acc.S, kOnes, kOnes, kOnes, kOnes, b0, b1);
+    }
+    // promote the group sums: R[0..1] row r0, R[2..3] row r1
+    acc.F[0] = fmaf(tl.c[0], (float)R[0], acc.F[0]);
+    acc.F[1] = fmaf(tl.c[0], (float)R[1], acc.F[1]);
+    acc.F[2] = fmaf(tl.c[1], (float)R[2], acc.F[2]);
+    acc.F[3] = fmaf(tl.c[1], (float)R[3], acc.F[3]);
+    if (EMIT) {
+      const int ng = p.tpr;
+      const int r0 = rb * kTileRows + gid, r1 = r0 + 8;
+      if (tk0 < p.M) {
+        if (r0 < p.N) p.R_out[((int64_t)tk0 * p.N + r0) * ng + cg] = R[0];
+        if (r1 < p.N) p.R_out[((int64_t)tk0 * p.N + r1) * ng + cg] = R[2];
+      }
+      if (tk1 < p.M) {
+        if (r0 < p.N) p.R_out[((int64_t)tk1 * p.N + r0) * ng + cg] = R[1];
+        if (r1 < p.N) p.R_out[((int64_t)tk1 * p.N + r1) * ng + cg] = R[3];
+      }
+    }
+    // outlier channels of this tile (the same for every row): the lane
+    // holding the channel forms the dequantized weight of its two rows;
+    // the four lanes of its row group take it by shuffle
+    const uint32_t om = omask[cg * 4 + tid4];
+    uint32_t any = __ballot_sync(0xffffffffu, om != 0u) & 0xFu;  // lanes 0..3 = chunks 0..3
+    while (any) {
+      const int src = __ffs(any) - 1;
+      any &= any - 1;
+      uint32_t bits = __shfl_sync(0xffffffffu, om, src);
+      int pos = __shfl_sync(0xffffffffu, obase[cg * 4 + tid4], src);
+      const int owner = gid * 4 + src;
+      while (bits) {
+        const int j = __ffs(bits) - 1;
+        bits &= bits - 1;
+        float w0 = 0.0f, w1 = 0.0f, u0 = 0.0f, u1 = 0.0f;
+        if (tid4 == src) {
+          const int bit = tiled_bit_of(j);
+          const uint32_t m0 = MASK ? (tl.m[0] >> bit) & 1u : 1u;
+          const uint32_t m1 = MASK ? (tl.m[1] >> bit) & 1u : 1u;
+          u0 = m0 ? (((tl.s[0] >> bit) & 1u) ? 1.0f : -1.0f) : 0.0f;
+          u1 = m1 ? (((tl.s[1] >> bit) & 1u) ? 1.0f : -1.0f) : 0.0f;
+          w0 = tl.c[0] * (float)tile_code<0>(tl.q, j);
+          w1 = tl.c[1] * (float)tile_code<1>(tl.q, j);
+        }
+        w0 = __shfl_sync(0xffffffffu, w0, owner);
+        w1 = __shfl_sync(0xffffffffu, w1, owner);
+        u0 = __shfl_sync(0xffffffffu, u0, owner);
+        u1 = __shfl_sync(0xffffffffu, u1, owner);
+        // (an index list that is not strictly ascending cannot push pos
+        // past the list)
+        if (pos >= 0 && pos < p.n_out) {
+          float x0, x1;
           if constexpr (FUSED) {
-            a = xp[0];
-            b = xp[1];
+            x0 = tk0 < p.M ? xo_s[tk0 * p.n_pad + pos] : 0.0f;
+            x1 = tk1 < p.M ? xo_s[tk1 * p.n_pad + pos] : 0.0f;
           } else {
-            a = __ldg(xp);
-            b = __ldg(xp + 1);
+            x0 = tk0 < p.M ? __ldg(p.xout + (int64_t)tk0 * p.n_out + pos) : 0.0f;
+            x1 = tk1 < p.M ? __ldg(p.xout + (int64_t)tk1 * p.n_out + pos) : 0.0f;
           }
-          xw[0] = a.x; xw[1] = a.y; xw[2] = a.z; xw[3] = a.w;
-          xw[4] = b.x; xw[5] = b.y; xw[6] = b.z; xw[7] = b.w;
+          acc.Ut[0] = fmaf(u0, x0, acc.Ut[0]);
+          acc.Ut[1] = fmaf(u0, x1, acc.Ut[1]);
+          acc.Ut[2] = fmaf(u1, x0, acc.Ut[2]);
+          acc.Ut[3] = fmaf(u1, x1, acc.Ut[3]);
+          acc.Ur[0] = fmaf(w0, x0, acc.Ur[0]);
+          acc.Ur[1] = fmaf(w0, x1, acc.Ur[1]);
+          acc.Ur[2] = fmaf(w1, x0, acc.Ur[2]);
+          acc.Ur[3] = fmaf(w1, x1, acc.Ur[3]);
         }
-        const uint32_t pb0 = MASK ? (tl.s[0] & tl.m[0]) : tl.s[0];
-        const uint32_t pb1 = MASK ? (tl.s[1] & tl.m[1]) : tl.s[1];
-        int R[4] = {0, 0, 0, 0};
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          const uint32_t b0 = xw[2 * m], b1 = xw[2 * m + 1];
-          mma_s8(R, tl.q[4 * m], tl.q[4 * m + 1], tl.q[4 * m + 2], tl.q[4 * m + 3], b0, b1);
-          mma_s8(acc.Pn, bits_word(pb0, 2 * m), bits_word(pb1, 2 * m), bits_word(pb0, 2 * m + 1),
-                 bits_word(pb1, 2 * m + 1), b0, b1);
-          if constexpr (MASK)
-            mma_s8(acc.S, bits_word(tl.m[0], 2 * m), bits_word(tl.m[1], 2 * m),
-                   bits_word(tl.m[0], 2 * m + 1), bits_word(tl.m[1], 2 * m + 1), b0, b1);
-          else
-            mma_s8(acc.S, kOnes, kOnes, kOnes, kOnes, b0, b1);
-        }
-        // promote the group sums: R[0..1] row r0, R[2..3] row r1
-        acc.F[0] = fmaf(tl.c[0], (float)R[0], acc.F[0]);
-        acc.F[1] = fmaf(tl.c[0], (float)R[1], acc.F[1]);
-        acc.F[2] = fmaf(tl.c[1], (float)R[2], acc.F[2]);
-        acc.F[3] = fmaf(tl.c[1], (float)R[3], acc.F[3]);
-        if (EMIT) {
-          const int ng = p.tpr;
-          const int r0 = rb * kTileRows + gid, r1 = r0 + 8;
-          if (tk0 < p.M) {
-            if (r0 < p.N) p.R_out[((int64_t)tk0 * p.N + r0) * ng + cg] = R[0];
-            if (r1 < p.N) p.R_out[((int64_t)tk0 * p.N + r1) * ng + cg] = R[2];
-          }
-          if (tk1 < p.M) {
-            if (r0 < p.N) p.R_out[((int64_t)tk1 * p.N + r0) * ng + cg] = R[1];
-            if (r1 < p.N) p.R_out[((int64_t)tk1 * p.N + r1) * ng + cg] = R[3];
-          }
-        }
-        // outlier channels of this tile (the same for every row): the lane
-        // holding the channel forms the dequantized weight of its two rows;
-        // the four lanes of its row group take it by shuffle
-        const uint32_t om = omask[cg * 4 + tid4];
-        uint32_t any = __ballot_sync(0xffffffffu, om != 0u) & 0xFu;  // lanes 0..3 = chunks 0..3
-        while (any) {
-          const int src = __ffs(any) - 1;
-          any &= any - 1;
-          uint32_t bits = __shfl_sync(0xffffffffu, om, src);
-          int pos = __shfl_sync(0xffffffffu, obase[cg * 4 + tid4], src);
-          const int owner = gid * 4 + src;
-          while (bits) {
-            const int j = __ffs(bits) - 1;
-            bits &= bits - 1;
-            float w0 = 0.0f, w1 = 0.0f, u0 = 0.0f, u1 = 0.0f;
-            if (tid4 == src) {
-              const int bit = tiled_bit_of(j);
-              const uint32_t m0 = MASK ? (tl.m[0] >> bit) & 1u : 1u;
-              const uint32_t m1 = MASK ? (tl.m[1] >> bit) & 1u : 1u;
-              u0 = m0 ? (((tl.s[0] >> bit) & 1u) ? 1.0f : -1.0f) : 0.0f;
-              u1 = m1 ? (((tl.s[1] >> bit) & 1u) ? 1.0f : -1.0f) : 0.0f;
-              w0 = tl.c[0] * (float)tile_code<0>(tl.q, j);
-              w1 = tl.c[1] * (float)tile_code<1>(tl.q, j);
-            }
-            w0 = __shfl_sync(0xffffffffu, w0, owner);
-            w1 = __shfl_sync(0xffffffffu, w1, owner);
-            u0 = __shfl_sync(0xffffffffu, u0, owner);
-            u1 = __shfl_sync(0xffffffffu, u1, owner);
-            // (an index list that is not strictly ascending cannot push pos
-            // past the list)
-            if (pos >= 0 && pos < p.n_out) {
-              float x0, x1;
-              if constexpr (FUSED) {
-                x0 = tk0 < p.M ? xo_s[tk0 * p.n_pad + pos] : 0.0f;
-                x1 = tk1 < p.M ? xo_s[tk1 * p.n_pad + pos] : 0.0f;
-              } else {
-                x0 = tk0 < p.M ? __ldg(p.xout + (int64_t)tk0 * p.n_out + pos) : 0.0f;
-                x1 = tk1 < p.M ? __ldg(p.xout + (int64_t)tk1 * p.n_out + pos) : 0.0f;
-              }
-              acc.Ut[0] = fmaf(u0, x0, acc.Ut[0]);
-              acc.Ut[1] = fmaf(u0, x1, acc.Ut[1]);
-              acc.Ut[2] = fmaf(u1, x0, acc.Ut[2]);
-              acc.Ut[3] = fmaf(u1, x1, acc.Ut[3]);
-              acc.Ur[0] = fmaf(w0, x0, acc.Ur[0]);
-              acc.Ur[1] = fmaf(w0, x1, acc.Ur[1]);
-              acc.Ur[2] = fmaf(w1, x0, acc.Ur[2]);
-              acc.Ur[3] = fmaf(w1, x1, acc.Ur[3]);
-            }
-            ++pos;
-          }
-        }
+        ++pos;
+      }
+    }
 
-        // refill this slot with the tile kDepth ahead
-        if (t + d + kDepth < t1) load_tile<MASK>(tl, cur);
-        cur.advance();
+    // refill this slot with the tile D ahead (this lane has read its bytes)
+    if (t + D < t1) copy_tile<MASK>(ring_u + slot_i * Slot<MASK>::kBytes, cur, lane);
+    cp_async_commit();
+    cur.advance();
+    if (++slot_i == D) slot_i = 0;
 
-        // end of a row block, or end of this warp's range
-        if (cg == p.tpr - 1 || t + d + 1 == t1) {
-          float4 v[4];
+    // end of a row block, or end of this warp's range
+    if (cg == p.tpr - 1 || t + 1 == t1) {
+      float4 v[4];
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            v[i] = cell(trunk_T<MASK>(acc, i), acc.F[i], acc.Ut[i], acc.Ur[i]);
-          if (EMIT) {
-            const int r0 = rb * kTileRows + gid, r1 = r0 + 8;
-            if (tk0 < p.M && r0 < p.N) atomicAdd(&p.T_out[(int64_t)tk0 * p.N + r0], trunk_T<MASK>(acc, 0));
-            if (tk1 < p.M && r0 < p.N) atomicAdd(&p.T_out[(int64_t)tk1 * p.N + r0], trunk_T<MASK>(acc, 1));
-            if (tk0 < p.M && r1 < p.N) atomicAdd(&p.T_out[(int64_t)tk0 * p.N + r1], trunk_T<MASK>(acc, 2));
-            if (tk1 < p.M && r1 < p.N) atomicAdd(&p.T_out[(int64_t)tk1 * p.N + r1], trunk_T<MASK>(acc, 3));
-          }
-          if (rb_head && cg == p.tpr - 1) {
-            write_y(p, rb, gid, tid4, v, al0, al1, sx0, sx1);
-          } else {
-            // a shared row block: slot 1 if this piece starts the row block
-            // (this range ends inside it), slot 0 if it continues one begun
-            // before this range
-            const int slot = rb_head ? 1 : 0;
+      for (int i = 0; i < 4; ++i)
+        v[i] = cell(trunk_T<MASK>(acc, i), acc.F[i], acc.Ut[i], acc.Ur[i]);
+      if (EMIT) {
+        const int r0 = rb * kTileRows + gid, r1 = r0 + 8;
+        if (tk0 < p.M && r0 < p.N) atomicAdd(&p.T_out[(int64_t)tk0 * p.N + r0], trunk_T<MASK>(acc, 0));
+        if (tk1 < p.M && r0 < p.N) atomicAdd(&p.T_out[(int64_t)tk1 * p.N + r0], trunk_T<MASK>(acc, 1));
+        if (tk0 < p.M && r1 < p.N) atomicAdd(&p.T_out[(int64_t)tk0 * p.N + r1], trunk_T<MASK>(acc, 2));
+        if (tk1 < p.M && r1 < p.N) atomicAdd(&p.T_out[(int64_t)tk1 * p.N + r1], trunk_T<MASK>(acc, 3));
+      }
+      if (rb_head && cg == p.tpr - 1) {
+        write_y(p, rb, gid, tid4, v, al0, al1, sx0, sx1);
+      } else {
+        // a shared row block: slot 1 if this piece starts the row block
+        // (this range ends inside it), slot 0 if it continues one begun
+        // before this range
+        const int slot = rb_head ? 1 : 0;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) part_s[((warp * 2 + slot) * 4 + i) * 32 + lane] = v[i];
-          }
-          acc_zero(acc);
-          rb_head = true;
-          if (cg == p.tpr - 1 && t + d + 1 < t1) {
-            // the next row block starts: its row scales, needed at its end
-            al0 = __ldg(p.alpha + (rb + 1) * kTileRows + gid);
-            al1 = __ldg(p.alpha + (rb + 1) * kTileRows + gid + 8);
-          }
-        }
-        if (++cg == p.tpr) {
-          cg = 0;
-          ++rb;
+        for (int i = 0; i < 4; ++i) {
+          const int tk = (i & 1) ? tk1 : tk0;
+          if (tk < p.M) part_s[((warp * 2 + slot) * 16 + (i >> 1) * 8 + gid) * p.M + tk] = v[i];
         }
       }
+      acc_zero(acc);
+      rb_head = true;
+      if (cg == p.tpr - 1 && t + 1 < t1) {
+        // the next row block starts: its row scales, needed at its end
+        al0 = __ldg(p.alpha + (rb + 1) * kTileRows + gid);
+        al1 = __ldg(p.alpha + (rb + 1) * kTileRows + gid + 8);
+      }
+    }
+    if (++cg == p.tpr) {
+      cg = 0;
+      ++rb;
     }
   }
 
@@ -625,22 +681,27 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
   const int rb_last = (t1 - 1) / p.tpr;
   if (rb_last * p.tpr >= t0 && t1 % p.tpr != 0) {
     const int w_hi = tile_warp((rb_last + 1) * p.tpr - 1, T0c, T1c);
+    // (cells of tokens past M were never stored and are not written)
+    auto cell_at = [&](int w, int slot, int i) -> const float4& {
+      const int tk = min((i & 1) ? tk1 : tk0, p.M - 1);
+      return part_s[((w * 2 + slot) * 16 + (i >> 1) * 8 + gid) * p.M + tk];
+    };
     float4 v[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) v[i] = part_s[((warp * 2 + 1) * 4 + i) * 32 + lane];
+    for (int i = 0; i < 4; ++i) v[i] = cell_at(warp, 1, i);
     for (int w = warp + 1; w <= w_hi; ++w) {
       // a CTA with fewer tiles than warps has empty warps between its owners
       if (warp_first_tile(w, T0c, T1c) == warp_first_tile(w + 1, T0c, T1c)) continue;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) cell_add(v[i], part_s[((w * 2) * 4 + i) * 32 + lane]);
+      for (int i = 0; i < 4; ++i) cell_add(v[i], cell_at(w, 0, i));
     }
     write_y(p, rb_last, gid, tid4, v, al0, al1, sx0, sx1);
   }
 }
 
-template <bool MASK, bool EMIT, bool FUSED>
+template <bool MASK, bool EMIT, bool FUSED, int D>
 cudaError_t launch_one(const Params& p, int grid, int smem, bool pdl, cudaStream_t stream) {
-  auto* fn = k_linear_tc<MASK, EMIT, FUSED>;
+  auto* fn = k_linear_tc<MASK, EMIT, FUSED, D>;
   cudaError_t e = ensure_smem_attr((const void*)fn, smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -656,6 +717,27 @@ cudaError_t launch_one(const Params& p, int grid, int smem, bool pdl, cudaStream
   return cudaLaunchKernelEx(&cfg, fn, p);
 }
 
+template <bool MASK, bool FUSED, int D>
+cudaError_t launch_plain(const Params& p, int grid, int smem, bool pdl, cudaStream_t stream) {
+  return launch_one<MASK, false, FUSED, D>(p, grid, smem, pdl, stream);
+}
+
+// Non-accumulator launch with a ring depth chosen at run time among Ds.
+template <int D0, int... Ds>
+cudaError_t launch_depth(int depth, bool mask, bool fused, const Params& p, int grid, int smem,
+                         bool pdl, cudaStream_t stream) {
+  if (depth == D0 || sizeof...(Ds) == 0) {
+    if (fused)
+      return mask ? launch_plain<true, true, D0>(p, grid, smem, pdl, stream)
+                  : launch_plain<false, true, D0>(p, grid, smem, pdl, stream);
+    return mask ? launch_plain<true, false, D0>(p, grid, smem, pdl, stream)
+                : launch_plain<false, false, D0>(p, grid, smem, pdl, stream);
+  }
+  if constexpr (sizeof...(Ds) > 0)
+    return launch_depth<Ds...>(depth, mask, fused, p, grid, smem, pdl, stream);
+  return cudaErrorInvalidValue;
+}
+
 }  // namespace
 
 size_t linear_tc_part_bytes(int) {
@@ -664,20 +746,26 @@ size_t linear_tc_part_bytes(int) {
 }
 
 namespace {
-constexpr int kSmemPart = kWarps * 2 * 4 * 32 * (int)sizeof(float4);
-// Shared memory of one CTA stays within this so that kBps CTAs fit an SM.
-constexpr int kSmemBudget = 200 * 1024;
+// Partial sums of one token: kWarps warps x 2 slots x 16 rows.
+constexpr int kSmemPartPerToken = kWarps * 2 * 16 * (int)sizeof(float4);
+// Largest dynamic shared memory of one CTA on sm_100 (227 KiB, opt-in).
+constexpr int kSmemMax = 227 * 1024;
 
 int outlier_table_bytes(const sq_packed_weight& w) { return (int)(tiles_cols(w.K) / 32) * 8; }
 int fused_token_bytes(const sq_packed_weight& w, int n_out) {
   return (int)tiles_cols(w.K) + (int)round_up(n_out, 4) * 4;
 }
+int ring_bytes(bool mask, int depth) {
+  return kWarps * depth * (mask ? Slot<true>::kBytes : Slot<false>::kBytes);
+}
 }  // namespace
 
 int linear_tc_fused_tokens(const sq_packed_weight& w, int n_out) {
-  const int fixed = kSmemPart + outlier_table_bytes(w) + kCols * 4 + kWarps * kCols * 4 + 64;
-  const int per = fused_token_bytes(w, n_out);
-  const int m = (kSmemBudget - fixed) / per;
+  // counted with the shallow ring; the deep one is used when it fits
+  const int fixed = ring_bytes(w.mask_bits != nullptr, kShallow) + outlier_table_bytes(w) +
+                    kCols * 4 + kWarps * kCols * 4 + 64;
+  const int per = fused_token_bytes(w, n_out) + kSmemPartPerToken;
+  const int m = (kSmemMax - fixed) / per;
   return m < 0 ? 0 : std::min(m, kCols);
 }
 
@@ -719,7 +807,11 @@ cudaError_t launch_linear_tc(const sq_packed_weight& w, int M, const int8_t* xq,
   p.x = x;
   p.status = status;
   p.n_pad = (int)round_up(n_out, 4);
-  int smem = kSmemPart + outlier_table_bytes(w);
+  const bool mask = w.mask_bits != nullptr;
+  const bool emit = T_out != nullptr;
+  int smem = kSmemPartPerToken * M;
+  p.off_omask = smem;
+  smem += outlier_table_bytes(w);
   p.off_xq = p.off_xo = p.off_sx = p.off_red = 0;
   if (fused) {
     p.off_xq = smem;
@@ -732,17 +824,17 @@ cudaError_t launch_linear_tc(const sq_packed_weight& w, int M, const int8_t* xq,
     smem += kWarps * kCols * 4;
   }
   smem = (int)round_up(smem, 16);
-  const bool mask = w.mask_bits != nullptr;
-  const bool emit = T_out != nullptr;
+  p.off_ring = smem;
+  // three tiles per warp above batch 2 where they fit, else two (the
+  // accumulator mode, used to check the kernel, always takes two)
+  const int depth = (!emit && M > 2 && smem + ring_bytes(mask, kDeep) <= kSmemMax) ? kDeep : kShallow;
+  smem += ring_bytes(mask, depth);
+  if (smem > kSmemMax) return cudaErrorInvalidValue;
   const int grid = (int)blocks;
-  if (fused)
-    return mask ? launch_one<true, false, true>(p, grid, smem, pdl, stream)
-                : launch_one<false, false, true>(p, grid, smem, pdl, stream);
-  if (mask)
-    return emit ? launch_one<true, true, false>(p, grid, smem, pdl, stream)
-                : launch_one<true, false, false>(p, grid, smem, pdl, stream);
-  return emit ? launch_one<false, true, false>(p, grid, smem, pdl, stream)
-              : launch_one<false, false, false>(p, grid, smem, pdl, stream);
+  if (emit)
+    return mask ? launch_one<true, true, false, kShallow>(p, grid, smem, pdl, stream)
+                : launch_one<false, true, false, kShallow>(p, grid, smem, pdl, stream);
+  return launch_depth<kDeep, kShallow>(depth, mask, fused, p, grid, smem, pdl, stream);
 }
 
 }  // namespace sq
