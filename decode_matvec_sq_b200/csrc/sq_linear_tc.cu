@@ -135,7 +135,7 @@ struct Tile {
 
 // Streaming position of one lane: its part of the next tile to copy.
 struct Cursor {
-  const uint8_t* code;   // the lane's 64 code bytes; + 2048 per tile
+  const uint8_t* code;   // the tile's code bytes + 16 * lane; + 2048 per tile
   const uint32_t* sign;  // the lane's two sign words; + 64 words per tile
   const uint32_t* mask;
   const float* scale;    // the scale of row r0 (r1: + 8); + 16 floats per tile
@@ -149,15 +149,18 @@ struct Cursor {
 
 // ---- shared-memory tile ring ------------------------------------------------------
 // Each warp streams its tiles through a ring of D slots filled by cp.async
-// (global -> shared without registers), D tiles ahead of use.  A lane copies,
-// and later reads back, only its own bytes, so the warp needs no
-// synchronisation around a slot.  Slot layout: 32 lanes x 64 code bytes, then
-// 32 x 8 sign bytes (then 32 x 8 mask bytes), then 32 x 8 bytes of the lane's
-// two scales.  Code chunk j (16 bytes) of lane L sits at L*64 + ((j + L/2) % 4)
-// * 16, so the 16-byte reads of eight consecutive lanes hit eight different
-// bank groups.  The codes bypass L1; the small sign, mask and scale copies go
-// through it, where neighbouring lanes' requests coalesce (copies of 16 bytes
-// that bypass L1 measured slower for these).
+// (global -> shared without registers), D tiles ahead of use.  Slot layout:
+// 32 lanes x 64 code bytes, then 32 x 8 sign bytes (then 32 x 8 mask bytes),
+// then 32 x 8 bytes of the lane's two scales.  Code chunk j (16 bytes) of lane
+// L sits at L*64 + ((j + L/2) % 4) * 16, so the 16-byte reads of eight
+// consecutive lanes hit eight different bank groups.
+// The codes are copied in four warp-wide instructions of 512 contiguous bytes
+// (whole 32-byte sectors, each requested once), 16 bytes per lane, into their
+// owners' places, so the warp synchronises after the wait (the owner reads
+// other lanes' copies) and before a refill (no lane may still read the slot).
+// They bypass L1.  A lane copies its own sign, mask and scale words, through
+// L1, where neighbouring lanes' requests coalesce (16-byte copies that bypass
+// L1 measured slower for these).
 template <bool MASK>
 struct Slot {
   static constexpr int kSign = 2048;
@@ -186,9 +189,11 @@ __device__ __forceinline__ void cp_async_wait() {
 
 template <bool MASK>
 __device__ __forceinline__ void copy_tile(uint32_t slot, const Cursor& c, int lane) {
-  const uint32_t cb = slot + lane * 64;
 #pragma unroll
-  for (int j = 0; j < 4; ++j) cp_async16(cb + (((j + (lane >> 1)) & 3) << 4), c.code + 16 * j);
+  for (int j = 0; j < 4; ++j) {
+    const int lo = j * 8 + (lane >> 2), ch = lane & 3;  // owner lane, its chunk
+    cp_async16(slot + lo * 64 + (((ch + (lo >> 1)) & 3) << 4), c.code + 512 * j);
+  }
   cp_async8(slot + Slot<MASK>::kSign + lane * 8, c.sign);
   if constexpr (MASK) cp_async8(slot + Slot<MASK>::kMask + lane * 8, c.mask);
   cp_async4(slot + Slot<MASK>::kScale + lane * 8, c.scale);
@@ -447,7 +452,7 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
   Cursor cur;
   {
     const int64_t lt = (int64_t)t0 * 32 + lane;
-    cur.code = reinterpret_cast<const uint8_t*>(p.res) + lt * 64;
+    cur.code = reinterpret_cast<const uint8_t*>(p.res) + (int64_t)t0 * 2048 + lane * 16;
     cur.sign = p.sign + lt * 2;
     cur.mask = MASK ? p.mask + lt * 2 : p.sign;
     cur.scale = p.scale + (int64_t)t0 * 16 + gid;
@@ -525,6 +530,7 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
   int slot_i = 0;
   for (int t = t0; t < t1; ++t) {
     cp_async_wait<D - 1>();  // this lane's copies of the tile have landed
+    __syncwarp();             // ... and every lane's
     Tile<MASK> tl;
     read_tile<MASK>(tl, ring_w + slot_i * Slot<MASK>::kBytes, lane);
     // activation codes of this lane's 32 channels for its MMA column
@@ -626,7 +632,8 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
       }
     }
 
-    // refill this slot with the tile D ahead (this lane has read its bytes)
+    // refill this slot with the tile D ahead, once no lane reads it
+    __syncwarp();
     if (t + D < t1) copy_tile<MASK>(ring_u + slot_i * Slot<MASK>::kBytes, cur, lane);
     cp_async_commit();
     cur.advance();
