@@ -481,6 +481,161 @@ def run_prefill(args, world, rank, local):
     return 0
 
 
+L2_BYTES = 126 << 20
+
+
+def _time_calls(launch, replays: int) -> float:
+    """Device ms per replay of a CUDA graph of launch(), on a side stream."""
+    import torch
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        launch()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        launch()
+    with torch.cuda.stream(s):
+        for _ in range(3):
+            g.replay()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(s)
+        for _ in range(replays):
+            g.replay()
+        b.record(s)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / replays
+    del g
+    return ms
+
+
+def layer_cases(workload: str):
+    """(label, layer, M, weight copies) of a single-layer workload.  Cold cases
+    rotate over enough copies of the packed weight that every call reads it
+    from HBM; the hot case of the 512 x 512 layer reads one L2-resident copy."""
+    from synth import workloads as wl
+    if workload == "single":
+        L = wl.config1()
+        cold = -(-2 * L2_BYTES // L.packed_bytes)
+        return [("512x512 hot (L2-resident)", L, 1, 1), ("512x512 cold", L, 1, cold)]
+    if workload == "mlp70b":
+        out = []
+        for M in (1, 2, 4, 8, 16):
+            for L in wl.config3(M):
+                out.append((f"{L.K}->{L.N} M={M}", L, M, 2))
+        return out
+    if workload == "threshold":
+        L = wl.config4()
+        return [("4096->14336 threshold trunk P=60", L, 1, -(-2 * L2_BYTES // L.packed_bytes))]
+    raise ValueError(workload)
+
+
+def _fused_launches(pw, M: int, L) -> int:
+    """Launches of one sq_quantize_linear call with a fused_workspace_bytes
+    workspace: the staged route (split + linear passes of 8) when M > 1 and
+    M * roundup(K, 128) > 16 KiB or when fused passes outnumber passes of 8,
+    else one fused launch per pass."""
+    import ctypes
+    import decode_matvec_sq_b200 as sq
+    kx = -(-L.K // 128) * 128
+    per_pass = int(sq.lib().sq_quantize_linear_tokens_per_pass(ctypes.byref(pw.view), L.n_out))
+    staged = M > 1 and (M * kx > (16 << 10) or -(-M // per_pass) > -(-M // 8))
+    return 1 + -(-M // 8) if staged else -(-M // per_pass)
+
+
+def run_layers(args, world, rank, local):
+    """Single-layer workloads beside the stack: the 512 x 512 layer (hot and
+    cold), the 70B-shaped MLP pair at batch 1..16 and the threshold-trunk layer.
+    Each call is the one-launch fused entry point (activation split + linear;
+    batches above 8 take one launch per 8 tokens), timed as a CUDA graph of
+    calls rotating over the weight copies.  GB/s = algorithmic bytes (packed
+    weights once + activations + y) / device time."""
+    import torch
+    import decode_matvec_sq_b200 as sq
+    from decode_matvec_sq_b200 import build
+    import synth.device as sdev
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py: no CUDA device visible (the sq path has no CPU fallback)")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=device)
+    if rank == 0 or world == 1:
+        build.build_all()
+    barrier(world)
+    sq.device_check()
+    st = torch.zeros(1, dtype=torch.int32, device=device)
+    cases = []
+    tot_ms, tot_bytes, tot_launch = 0.0, 0, 0
+    with ClockSampler(local) as clk:
+        for label, L, M, copies in layer_cases(args.workload):
+            W = sdev.fill_weights(L, torch.empty(L.N, L.K, device=device))
+            pw = sq.decompose_pack(W, trunk_percent=L.trunk_percent, status=st)
+            del W
+            pws = [pw]
+            for _ in range(copies - 1):
+                c = sq.alloc_packed(L.N, L.K, 128, pw.with_mask, pw.layout, device=device)
+                c.buf.copy_(pw.buf)
+                pws.append(c)
+            idx = torch.from_numpy(L.planted_channels()).to(device)
+            x = sdev.fill_activations(L, torch.empty(M, L.K, device=device))
+            y = torch.empty(M, L.N, device=device)
+            ws = sq.new_fused_workspace(pw, M, L.n_out)
+            calls = max(copies, 20)
+
+            def launch():
+                for r in range(calls):
+                    sq.quantize_linear(pws[r % copies], x, idx, y=y, workspace=ws, status=st)
+
+            for _ in range(args.warmup):
+                launch()
+            barrier(world)
+            ms = max_over_ranks(_time_calls(launch, max(1, args.steps)) / calls, world, device)
+            nbytes = linear_weight_bytes(L) + M * (4 * L.K + 4 * L.N) + 4 * L.n_out
+            launches = _fused_launches(pw, M, L)
+            cases.append({"case": label, "M": M, "us": round(ms * 1e3, 2),
+                          "gbs": round(nbytes / (ms * 1e-3) / 1e9, 1), "launches_per_call": launches})
+            tot_ms += ms
+            tot_bytes += nbytes
+            tot_launch += launches
+            del pws, pw, ws
+            torch.cuda.empty_cache()
+    clocks = clk.summary()
+    if st.item() != 0:
+        raise RuntimeError(f"device status {sq.STATUS.get(st.item())}")
+    peak, kind = load_peaks()
+    achieved = tot_bytes / (tot_ms * 1e-3) / 1e9
+    names = {"single": "512x512 layer, batch 1, W Laplace(0,0.02), x N(0,1) with 4 channels x50",
+             "mlp70b": "70B-shaped MLP pair 8192->28672 and 28672->8192, batch 1..16, "
+                       "W N(0,0.015^2) with 0.1% entries x10, x N(0,1) with 0.25% channels x40",
+             "threshold": "4096->14336, batch 1, per-row 60th-percentile trunk mask, "
+                          "W Laplace(0,0.02), x N(0,1) with 0.5% channels x30"}
+    if rank == 0:
+        print(json.dumps({
+            "metric": f"single-layer sq_quantize_linear HBM GB/s ({args.workload})",
+            "value": round(world * achieved, 1), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(tot_ms, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+            "config": {"workload": names[args.workload],
+                       "l2": "cold cases rotate over copies of the weight totalling >= 2x L2"},
+            "gpu_launches": tot_launch,
+            "cases": cases,
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": round(peak, 1),
+                         "unit": "GB/s", "frac": round(achieved / peak, 4), "peak_kind": kind,
+                         "traffic": None, "kernel": "k_linear_tc (activation split + decode linear)"},
+            "clocks": clocks,
+        }), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
 def run_gpu(args, world, rank, local):
     import torch
     import torch.distributed as dist
@@ -630,9 +785,12 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["sq", "reference"], default="sq")
     ap.add_argument("--layers", type=int, default=32)
-    ap.add_argument("--workload", choices=["decode", "prefill"], default="decode",
+    ap.add_argument("--workload", choices=["decode", "prefill", "single", "mlp70b", "threshold"],
+                    default="decode",
                     help="decode: the 7B-shaped stack at batch 1 (default); prefill: "
-                         "2048 tokens x 4096 -> 14336 on the tcgen05 kernel")
+                         "2048 tokens x 4096 -> 14336 on the tcgen05 kernel; single, mlp70b, "
+                         "threshold: single-layer workloads (512x512 hot/cold, the 70B-shaped "
+                         "MLP pair at batch 1..16, the threshold-trunk layer)")
     ap.add_argument("--no-pdl", action="store_true")
     ap.add_argument("--two-kernels", action="store_true",
                     help="activation split and linear layer as two kernels per linear")
@@ -648,6 +806,8 @@ def main(argv=None):
         return run_reference(args, world, rank)
     if args.workload == "prefill":
         return run_prefill(args, world, rank, local)
+    if args.workload in ("single", "mlp70b", "threshold"):
+        return run_layers(args, world, rank, local)
     return run_gpu(args, world, rank, local)
 
 

@@ -73,6 +73,8 @@ def lib():
         "sq_calibrate_outliers": ([vp, i32, i32, i32, vp, vp, vp], ctypes.c_int),
         "sq_quantize_act": ([vp, i32, i32, vp, i32, vp, vp, vp, vp, u32, vp], ctypes.c_int),
         "sq_linear_workspace_bytes": ([pw, i32], sz),
+        "sq_quantize_linear_workspace_bytes": ([pw, i32, i32], sz),
+        "sq_quantize_linear_tokens_per_pass": ([pw, i32], i32),
         "sq_linear": ([pw, vp, vp, vp, vp, i32, i32, vp, vp, sz, vp, u32, vp], ctypes.c_int),
         "sq_linear_accumulators": ([pw, vp, vp, vp, vp, i32, i32, vp, vp, vp, vp, sz, vp, u32, vp],
                                    ctypes.c_int),
@@ -256,6 +258,19 @@ def new_workspace(pw: PackedWeight, M: int = 1, device=None):
                        device=device or pw.buf.device)
 
 
+def fused_workspace_bytes(pw: PackedWeight, M: int = 1, n_out: int = 0) -> int:
+    """Workspace with which quantize_linear may run the activation split once
+    and the linear layer on its codes (where that is faster)."""
+    return int(lib().sq_quantize_linear_workspace_bytes(ctypes.byref(pw.view), M, n_out))
+
+
+def new_fused_workspace(pw: PackedWeight, M: int = 1, n_out: int = 0, device=None):
+    """A zero-filled workspace of fused_workspace_bytes."""
+    import torch
+    return torch.zeros(max(fused_workspace_bytes(pw, M, n_out), 16), dtype=torch.uint8,
+                       device=device or pw.buf.device)
+
+
 def _flags(pdl: bool) -> int:
     return SQ_LAUNCH_PDL if pdl else 0
 
@@ -281,14 +296,15 @@ def linear(pw: PackedWeight, xq, sx, x_out, idx, y=None, workspace=None, status=
 def quantize_linear(pw: PackedWeight, x, idx, y=None, workspace=None, status=None,
                     pdl: bool = False, stream=None):
     """y[M][N] from fp32 activations x[M][K]: the activation split and the
-    linear layer in one kernel (tiled layout)."""
+    linear layer in one kernel (tiled layout), or, for larger M * K with a
+    workspace of fused_workspace_bytes, the split once and the linear layer."""
     import torch
     M = x.shape[0]
     n = 0 if idx is None else int(idx.numel())
     if y is None:
         y = torch.empty(M, pw.N, dtype=torch.float32, device=x.device)
     if workspace is None:
-        workspace = new_workspace(pw, M)
+        workspace = new_fused_workspace(pw, M, n)
     _ck(lib().sq_quantize_linear(ctypes.byref(pw.view), _ptr(x), M, _ptr(idx) if n else None, n,
                                  _ptr(y), _ptr(workspace), workspace.numel(), _ptr(status),
                                  _flags(pdl), _stream(stream)), "sq_quantize_linear")

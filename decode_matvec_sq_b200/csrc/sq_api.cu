@@ -335,6 +335,36 @@ sq_status sq_linear_accumulators(const sq_packed_weight* w, const int8_t* xq, co
                        dev_status, flags, stream);
 }
 
+// The staged route of sq_quantize_linear: the activation split once
+// (k_quantize_act into the workspace), then the decode kernel on its codes.
+// Measured on B200 (70B-shaped MLP, 8192 <-> 28672): every CTA of the fused
+// kernel quantizes all M tokens of x, which costs more than a separate split
+// once M > 1 and M * roundup(K, 128) > 16 KiB (8192 -> 28672 at M = 4: 62.3
+// against 60.0 us); and where the codes of M tokens do not fit one pass of
+// the fused kernel, it reads the weights once per pass (28672 -> 8192 at
+// M = 8: 215.8 against 69.9 us).
+constexpr int64_t kFusedMaxCodeBytes = 16 << 10;
+
+static size_t stage_bytes(const sq_packed_weight& w, int M, int n_out) {
+  return (size_t)round_up((int64_t)M * xq_stride_of(w.K), 256) + (size_t)round_up(4 * (int64_t)M, 256) +
+         (size_t)round_up(4 * (int64_t)M * n_out, 256);
+}
+
+size_t sq_quantize_linear_workspace_bytes(const sq_packed_weight* w, int32_t M, int32_t n_out) {
+  if (!w || check_weight(w) != SQ_OK || M < 1 || n_out < 0 || n_out > kMaxOutliers) return 0;
+  DeviceInfo d;
+  if (!current_device(&d)) return 0;
+  const size_t need = linear_workspace_bytes(*w, M, d.sm_count);
+  if (need == 0) return 0;
+  return (size_t)round_up((int64_t)need, 256) + stage_bytes(*w, M, n_out);
+}
+
+int32_t sq_quantize_linear_tokens_per_pass(const sq_packed_weight* w, int32_t n_out) {
+  if (!w || check_weight(w) != SQ_OK || w->layout != SQ_LAYOUT_TILES) return 0;
+  if (n_out < 0 || n_out > kMaxOutliers || n_out > w->K) return 0;
+  return linear_tc_fused_tokens(*w, n_out);
+}
+
 sq_status sq_quantize_linear(const sq_packed_weight* w, const float* x, int32_t M,
                              const int32_t* idx, int32_t n_out, float* y, void* workspace,
                              size_t ws_bytes, int32_t* dev_status, uint32_t flags, void* stream) {
@@ -357,6 +387,19 @@ sq_status sq_quantize_linear(const sq_packed_weight* w, const float* x, int32_t 
   if (!workspace || ws_bytes < need) return SQ_ERR_WORKSPACE;
   const size_t part = linear_part_bytes(d.sm_count);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool staged_faster = M > 1 && ((int64_t)M * xq_stride_of(w->K) > kFusedMaxCodeBytes ||
+                                       ceil_div(M, per_pass) > ceil_div(M, kMaxTokensPerPassTc));
+  const size_t base = (size_t)round_up((int64_t)need, 256);
+  if (staged_faster && ws_bytes >= base + stage_bytes(*w, M, n_out)) {
+    int8_t* xq = static_cast<int8_t*>(workspace) + base;
+    float* sx = reinterpret_cast<float*>(xq + round_up((int64_t)M * xq_stride_of(w->K), 256));
+    float* xo = n_out > 0 ? sx + round_up(4 * (int64_t)M, 256) / 4 : nullptr;
+    const cudaError_t e = launch_quantize_act(x, M, w->K, idx, n_out, xq, sx, xo, dev_status,
+                                              (flags & SQ_LAUNCH_PDL) != 0, s);
+    if (e != cudaSuccess) return SQ_ERR_CUDA;
+    return linear_common(w, xq, sx, xo, idx, n_out, M, y, nullptr, nullptr, workspace, need,
+                         dev_status, flags, stream);
+  }
   for (int t0 = 0; t0 < M; t0 += per_pass) {
     const int m = std::min(per_pass, M - t0);
     cudaError_t e = launch_linear_tc(*w, m, nullptr, nullptr, nullptr, x + (int64_t)t0 * w->K, idx,

@@ -301,7 +301,7 @@ __device__ __forceinline__ void write_y(const Params& p, int rb, int gid, int ti
 // K <= 16384 each thread keeps its share of a token's x in registers (float4,
 // all loads in flight at once), so a token costs one memory round trip and
 // one barrier; the outlier values are gathered with the same round trip.
-constexpr int kXRegs = 16;  // float4 per thread kept in registers: K <= 16384
+constexpr int kXRegs = 16;  // float4 per thread kept in registers: K <= 32768
 
 __device__ __forceinline__ uint32_t omask_nibble(const uint32_t* omask, int j4) {
   return (omask[j4 >> 3] >> ((j4 & 7) * 4)) & 0xFu;  // outlier bits of channels 4*j4 .. 4*j4+3

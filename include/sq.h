@@ -230,20 +230,45 @@ sq_status sq_linear_accumulators(const sq_packed_weight *w, const int8_t *xq, co
  *   idx, n_out  outlier channels, strictly ascending in [0, K) (checked on
  *               the device: a violation sets SQ_ERR_INVALID_ARG)
  *   y           [M][N] f32 out
- *   workspace   as for sq_linear (sq_linear_workspace_bytes(w, M))
+ *   workspace   at least sq_linear_workspace_bytes(w, M) bytes, 16-byte
+ *               aligned, zero-filled before its first use (as for
+ *               sq_linear); with sq_quantize_linear_workspace_bytes(w, M,
+ *               n_out) bytes the staged route below may be taken
  * Every CTA forms the per-token scale, codes and outlier values of x in its
  * shared memory with the same arithmetic as sq_quantize_act, then runs the
  * decode of sq_linear: y is bit-identical to sq_quantize_act followed by
  * sq_linear.  Non-finite x sets SQ_ERR_NONFINITE.  Tokens are processed in
- * passes of up to 8 that fit the shared memory: roundup(K,128) +
- * 4*roundup(n_out,4) bytes per token; SQ_ERR_SHAPE if not even one token
- * fits (K above about 60000).  flags: 0 or SQ_LAUNCH_PDL (the kernel then
- * reads x, idx and y-independent data only after the previous kernel
- * completes; the packed weights are streamed before).
+ * passes of up to 8 that fit the shared memory (roundup(K,128) +
+ * 4*roundup(n_out,4) + 8192 bytes per token beside a fixed part); SQ_ERR_SHAPE
+ * if not even one token fits (K above about 100000).
+ * Staged route: when M > 1 and M*roundup(K,128) > 16384, or the tokens need
+ * more fused passes than the decode kernel's passes of 8, and the workspace
+ * is large enough, the call runs sq_quantize_act once into the workspace and
+ * then sq_linear on its codes (two launches; y is the same bit for bit).
+ * flags: 0 or SQ_LAUNCH_PDL (the kernel then reads x, idx and y-independent
+ * data only after the previous kernel completes; the packed weights are
+ * streamed before).
  */
 sq_status sq_quantize_linear(const sq_packed_weight *w, const float *x, int32_t M,
                              const int32_t *idx, int32_t n_out, float *y, void *workspace,
                              size_t ws_bytes, int32_t *dev_status, uint32_t flags, void *stream);
+
+/*
+ * Workspace bytes with which sq_quantize_linear may take its staged route:
+ * sq_linear_workspace_bytes(w, M) rounded up to 256, then the activation
+ * codes [M][roundup(K,128)] i8, the token scales [M] f32 and the outlier
+ * values [M][n_out] f32, each 256-byte aligned.  Only the leading
+ * sq_linear_workspace_bytes part must be zero-filled.  0 for an invalid
+ * weight, M < 1, n_out out of range or no usable device.
+ */
+size_t sq_quantize_linear_workspace_bytes(const sq_packed_weight *w, int32_t M, int32_t n_out);
+
+/*
+ * Tokens per launch of sq_quantize_linear's fused kernel for this weight and
+ * outlier count (1..8; 0 if not even one token fits, or for an invalid
+ * weight or a weight not in SQ_LAYOUT_TILES).
+ */
+int32_t sq_quantize_linear_tokens_per_pass(const sq_packed_weight *w, int32_t n_out);
 
 /*
  * sq_linear without a caller workspace, for callers that cannot allocate

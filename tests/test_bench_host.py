@@ -90,3 +90,19 @@ def test_reference_arm_under_torchrun_two_ranks():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] == 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"] > 0
     assert d["metric"] == bench.METRIC and d["higher_is_better"] is True
+
+
+def test_single_layer_workload_cases():
+    """The single-layer workloads cover the 512 x 512 layer hot and cold, the
+    70B-shaped pair at every batch of its sweep, and the threshold layer; every
+    cold case rotates over at least twice the L2 capacity of weights."""
+    single = bench.layer_cases("single")
+    assert [c[3] for c in single][0] == 1
+    L, copies = single[1][1], single[1][3]
+    assert copies * L.packed_bytes >= 2 * bench.L2_BYTES
+    mlp = bench.layer_cases("mlp70b")
+    assert sorted({c[2] for c in mlp}) == [1, 2, 4, 8, 16]
+    assert {(c[1].K, c[1].N) for c in mlp} == {(8192, 28672), (28672, 8192)}
+    assert all(c[3] * c[1].packed_bytes >= 2 * bench.L2_BYTES for c in mlp)
+    (label, L, M, copies), = bench.layer_cases("threshold")
+    assert L.trunk_percent == 60 and M == 1 and copies * L.packed_bytes >= 2 * bench.L2_BYTES

@@ -506,16 +506,21 @@ def _fused_vs_two_step(W, x, idx, P=-1, pdl=False):
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     pw = sq.decompose_pack(Wd, trunk_percent=P, layout=sq.SQ_LAYOUT_TILES, status=st)
     xq, sx, xo = sq.quantize_act(xd, idxd, status=st)
-    ws = sq.new_workspace(pw, x.shape[0])
-    y2 = torch.full((x.shape[0], W.shape[0]), float("nan"), device="cuda")
+    M, n = x.shape[0], len(idx)
+    ws = sq.new_workspace(pw, M)
+    y2 = torch.full((M, W.shape[0]), float("nan"), device="cuda")
     sq.linear(pw, xq, sx, xo, idxd, y=y2, workspace=ws, status=st)
-    for _ in range(2):  # twice: the arrival counters are left zero
-        y1 = torch.full_like(y2, float("nan"))
-        sq.quantize_linear(pw, xd, idxd, y=y1, workspace=ws, status=st, pdl=pdl)
-        torch.cuda.synchronize()
-        assert st.item() == 0
-        assert np.array_equal(y1.cpu().numpy().view(np.uint32), y2.cpu().numpy().view(np.uint32))
-    assert not sq.workspace_counters(ws, pw, x.shape[0]).any().item()
+    # the fused kernel (a workspace for sq_linear), then with a workspace that
+    # also lets the call take the staged route (split once + linear)
+    assert sq.fused_workspace_bytes(pw, M, n) > sq.workspace_bytes(pw, M)
+    for ws in (ws, sq.new_fused_workspace(pw, M, n)):
+        for _ in range(2):  # twice: the arrival counters are left zero
+            y1 = torch.full_like(y2, float("nan"))
+            sq.quantize_linear(pw, xd, idxd, y=y1, workspace=ws, status=st, pdl=pdl)
+            torch.cuda.synchronize()
+            assert st.item() == 0
+            assert np.array_equal(y1.cpu().numpy().view(np.uint32), y2.cpu().numpy().view(np.uint32))
+        assert not sq.workspace_counters(ws, pw, M).any().item()
     d = oracle.decompose(W, P=P)
     oxq, osx, oxo = oracle.quantize_act(x, idx)
     check_y(y1.cpu().numpy(), oracle.linear(d, oxq, osx, oxo, idx), oracle.abs_dot(W, x))
