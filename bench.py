@@ -601,7 +601,7 @@ def run_layers(args, world, rank, local):
                           "gbs": round(nbytes / (ms * 1e-3) / 1e9, 1), "launches_per_call": launches})
             tot_ms += ms
             tot_bytes += nbytes
-            tot_launch += launches
+            tot_launch += max(1, args.steps) * calls * launches  # inside the timed replays
             del pws, pw, ws
             torch.cuda.empty_cache()
     clocks = clk.summary()

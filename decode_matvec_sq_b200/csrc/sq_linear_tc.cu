@@ -10,8 +10,8 @@
 //   * residual: four int8 MMAs (mma.sync m16n8k32) per tile of 16 rows x 128
 //     channels give the exact group sums R_g; each lane's 64 bytes of the
 //     tile are already its four A fragments (the packed layout is the MMA's
-//     operand order), so they go from two 256-bit loads straight into the
-//     MMAs;
+//     operand order), so they go from the warp's shared-memory ring straight
+//     into the MMAs;
 //   * trunk: the sign bits are stored so that the four bits of one 4-channel
 //     word are the top bits of the four bytes of (bits << (7 - w)); a
 //     sign-replicating byte permute (prmt) turns them into 0 / -1 bytes, one
@@ -20,14 +20,13 @@
 //     all-ones (or the mask's) operand; T = 2P - S.  (A binary AND/popcount
 //     MMA would read the bits directly, but sm_100 runs it emulated at ~69
 //     instructions per m16n8k128, ten times the int8 MMA.)
-// Work: the tiles in row-block-major order are split evenly over all warps;
-// the packed tiles lie in memory in that same order, so each warp streams one
-// contiguous range with no edge cases (rows and channels are zero padded).
-// A row block finished inside one warp is written at once.  A row block
-// shared by warps of one CTA is summed from shared memory after one CTA
-// barrier; one shared by CTAs is summed by its last arriving CTA from per-CTA
-// partials in global memory.  Partial sums are added in tile order, so the
-// results do not depend on timing.
+// Work: one CTA of 16 warps per SM owns whole row blocks; its tiles, in
+// row-block-major order, are split evenly over its warps.  The packed tiles
+// lie in memory in that same order, so each warp streams one contiguous range
+// (through a per-warp cp.async ring in shared memory) with no edge cases: rows
+// and channels are zero padded.  A row block finished inside one warp is
+// written at once; one shared by warps of the CTA is summed from shared memory
+// after one CTA barrier, in warp order, so the results do not depend on timing.
 // Fused mode (sq_quantize_linear): the kernel takes the fp32 activations and
 // performs the activation split itself after the weight prefetch: every CTA
 // forms the per-token scale (absmax over the non-outlier channels), the INT8
@@ -84,6 +83,7 @@ struct Params {
   int32_t* status;    // device status word (non-finite x, bad index list)
   int n_pad;          // x_out row stride in shared memory
   int off_xq, off_xo, off_sx, off_red;  // shared-memory offsets (bytes)
+  // shared-memory offsets of the tile rings and the outlier bitmap (bytes)
   int off_ring, off_omask;
 };
 
@@ -298,7 +298,7 @@ __device__ __forceinline__ void write_y(const Params& p, int rb, int gid, int ti
 // (codes [M][K128], outlier values [M][n_pad], scales [M]); outlier channels
 // are those marked in omask.  Same arithmetic as the activation split kernel.
 // Latency is what counts here (the weight stream waits for the codes): for
-// K <= 16384 each thread keeps its share of a token's x in registers (float4,
+// K <= 32768 each thread keeps its share of a token's x in registers (float4,
 // all loads in flight at once), so a token costs one memory round trip and
 // one barrier; the outlier values are gathered with the same round trip.
 constexpr int kXRegs = 16;  // float4 per thread kept in registers: K <= 32768

@@ -7,6 +7,8 @@ accumulators) must match bit for bit.  The float output y must satisfy
 Small shapes compare every element; full-size workloads compare sampled rows
 that the oracle recomputes from regenerated inputs.
 """
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -584,6 +586,50 @@ def test_quantize_linear_status_and_errors():
     with pytest.raises(sq.SQError) as e:
         sq.quantize_linear(pr, torch.randn(1, 256, device="cuda"), None)
     assert e.value.name == "SQ_ERR_SHAPE"
+
+
+def test_quantize_linear_staged_route_status():
+    """The staged route (M * roundup(K,128) > 16 KiB) reports the same device
+    findings as the fused kernel: non-finite x, a bad index list."""
+    W = torch.randn(48, 8192, device="cuda")
+    pw = sq.decompose_pack(W)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ws = sq.new_fused_workspace(pw, 4, 2)
+    x = torch.randn(4, 8192, device="cuda")
+    x[3, 100] = float("nan")
+    sq.quantize_linear(pw, x, torch.tensor([5, 9], dtype=torch.int32, device="cuda"), workspace=ws,
+                       status=st)
+    torch.cuda.synchronize()
+    assert st.item() == sq.STATUS_CODE["SQ_ERR_NONFINITE"]
+    st.zero_()
+    sq.quantize_linear(pw, torch.randn(4, 8192, device="cuda"),
+                       torch.tensor([9, 5], dtype=torch.int32, device="cuda"), workspace=ws, status=st)
+    torch.cuda.synchronize()
+    assert st.item() == sq.STATUS_CODE["SQ_ERR_INVALID_ARG"]
+
+
+def test_fused_pass_and_workspace_queries():
+    """Tokens per fused pass and the staged-route workspace follow the shared
+    memory and workspace arithmetic of include/sq.h."""
+    L = sq.lib()
+    def tiles(N, K, mask=False):
+        v = sq.SqPackedWeight()
+        assert L.sq_packed_view(ctypes.c_void_p(1 << 40), N, K, 128, int(mask), 1, ctypes.byref(v)) == 0
+        return v
+    # ring of two 2560-byte slots per warp, 16 warps; outlier table K/32*8; per
+    # token roundup(K,128) + 4*roundup(n,4) + 8192; 227 KiB in all
+    for K, n, mask, want in [(4096, 20, False, 8), (11008, 55, False, 7), (28672, 72, False, 3),
+                             (28672, 72, True, 3), (65536, 0, False, 1), (131072, 0, False, 0)]:
+        assert L.sq_quantize_linear_tokens_per_pass(ctypes.byref(tiles(64, K, mask)), n) == want, (K, n)
+    v = sq.SqPackedWeight()
+    assert L.sq_packed_view(ctypes.c_void_p(1 << 40), 64, 4096, 128, 0, 0, ctypes.byref(v)) == 0
+    assert L.sq_quantize_linear_tokens_per_pass(ctypes.byref(v), 20) == 0  # row layout
+    r = lambda a: -(-a // 256) * 256
+    for M, n in [(1, 0), (4, 20), (16, 72)]:
+        w = tiles(300, 8192)
+        got = L.sq_quantize_linear_workspace_bytes(ctypes.byref(w), M, n)
+        assert got == r(L.sq_linear_workspace_bytes(ctypes.byref(w), M)) + r(M * 8192) + r(4 * M) + r(4 * M * n)
+    assert L.sq_quantize_linear_workspace_bytes(ctypes.byref(tiles(300, 8192)), 0, 0) == 0
 
 
 # ---- prefill: many tokens on tcgen05 (row layout, M >= 64) --------------------------
