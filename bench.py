@@ -528,7 +528,23 @@ def layer_cases(workload: str):
     if workload == "threshold":
         L = wl.config4()
         return [("4096->14336 threshold trunk P=60", L, 1, -(-2 * L2_BYTES // L.packed_bytes))]
+    if workload == "trunk":
+        out = []
+        for mid in range(4):
+            L = wl.config2_layer(0, mid)
+            out.append((f"{L.name.split('.')[-1]} {L.K}->{L.N} trunk only", L, 1,
+                        -(-2 * L2_BYTES // trunk_weight_bytes(L))))
+        return out
     raise ValueError(workload)
+
+
+def trunk_weight_bytes(L) -> int:
+    """Bytes the trunk-only mode reads of a tiled packed weight: the sign (and
+    mask) bits and the row scales of the padded rows."""
+    rows = -(-L.N // 16) * 16
+    words = -(-L.K // 128) * 4
+    planes = 2 if L.trunk_percent >= 0 else 1
+    return rows * (4 * words * planes + 4)
 
 
 def _fused_launches(pw, M: int, L) -> int:
@@ -587,15 +603,19 @@ def run_layers(args, world, rank, local):
             ws = sq.new_fused_workspace(pw, M, L.n_out)
             calls = max(copies, 20)
 
+            trunk = args.workload == "trunk"
+
             def launch():
                 for r in range(calls):
-                    sq.quantize_linear(pws[r % copies], x, idx, y=y, workspace=ws, status=st)
+                    sq.quantize_linear(pws[r % copies], x, idx, y=y, workspace=ws, status=st,
+                                       trunk_only=trunk)
 
             for _ in range(args.warmup):
                 launch()
             barrier(world)
             ms = max_over_ranks(_time_calls(launch, max(1, args.steps)) / calls, world, device)
-            nbytes = linear_weight_bytes(L) + M * (4 * L.K + 4 * L.N) + 4 * L.n_out
+            wbytes = trunk_weight_bytes(L) if trunk else linear_weight_bytes(L)
+            nbytes = wbytes + M * (4 * L.K + 4 * L.N) + 4 * L.n_out
             launches = _fused_launches(pw, M, L)
             cases.append({"case": label, "M": M, "us": round(ms * 1e3, 2),
                           "gbs": round(nbytes / (ms * 1e-3) / 1e9, 1), "launches_per_call": launches})
@@ -613,7 +633,9 @@ def run_layers(args, world, rank, local):
              "mlp70b": "70B-shaped MLP pair 8192->28672 and 28672->8192, batch 1..16, "
                        "W N(0,0.015^2) with 0.1% entries x10, x N(0,1) with 0.25% channels x40",
              "threshold": "4096->14336, batch 1, per-row 60th-percentile trunk mask, "
-                          "W Laplace(0,0.02), x N(0,1) with 0.5% channels x30"}
+                          "W Laplace(0,0.02), x N(0,1) with 0.5% channels x30",
+             "trunk": "trunk-only mode (residual path skipped) of the 7B-shaped stack's four "
+                      "linears, batch 1, W Laplace(0,0.02), x N(0,1) with 0.5% channels x30"}
     if rank == 0:
         print(json.dumps({
             "metric": f"single-layer sq_quantize_linear HBM GB/s ({args.workload})",
@@ -785,12 +807,14 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["sq", "reference"], default="sq")
     ap.add_argument("--layers", type=int, default=32)
-    ap.add_argument("--workload", choices=["decode", "prefill", "single", "mlp70b", "threshold"],
+    ap.add_argument("--workload", choices=["decode", "prefill", "single", "mlp70b", "threshold",
+                                           "trunk"],
                     default="decode",
                     help="decode: the 7B-shaped stack at batch 1 (default); prefill: "
                          "2048 tokens x 4096 -> 14336 on the tcgen05 kernel; single, mlp70b, "
                          "threshold: single-layer workloads (512x512 hot/cold, the 70B-shaped "
-                         "MLP pair at batch 1..16, the threshold-trunk layer)")
+                         "MLP pair at batch 1..16, the threshold-trunk layer); trunk: the "
+                         "stack's four linears in the trunk-only mode")
     ap.add_argument("--no-pdl", action="store_true")
     ap.add_argument("--two-kernels", action="store_true",
                     help="activation split and linear layer as two kernels per linear")
@@ -806,7 +830,7 @@ def main(argv=None):
         return run_reference(args, world, rank)
     if args.workload == "prefill":
         return run_prefill(args, world, rank, local)
-    if args.workload in ("single", "mlp70b", "threshold"):
+    if args.workload in ("single", "mlp70b", "threshold", "trunk"):
         return run_layers(args, world, rank, local)
     return run_gpu(args, world, rank, local)
 

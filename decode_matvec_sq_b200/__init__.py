@@ -22,6 +22,7 @@ LIB_PATH = os.path.join(PKG_DIR, "libsq.so")
 HEADER = os.path.join(os.path.dirname(PKG_DIR), "include", "sq.h")
 
 SQ_LAUNCH_PDL = 1
+SQ_TRUNK_ONLY = 2
 SQ_LAYOUT_ROWS = 0
 SQ_LAYOUT_TILES = 1
 
@@ -271,14 +272,15 @@ def new_fused_workspace(pw: PackedWeight, M: int = 1, n_out: int = 0, device=Non
                        device=device or pw.buf.device)
 
 
-def _flags(pdl: bool) -> int:
-    return SQ_LAUNCH_PDL if pdl else 0
+def _flags(pdl: bool, trunk_only: bool = False) -> int:
+    return (SQ_LAUNCH_PDL if pdl else 0) | (SQ_TRUNK_ONLY if trunk_only else 0)
 
 
 def linear(pw: PackedWeight, xq, sx, x_out, idx, y=None, workspace=None, status=None,
-           pdl: bool = False, stream=None):
+           pdl: bool = False, stream=None, trunk_only: bool = False):
     """y[M][N] = fused trunk + residual + outlier product (float32).
-    The weight's layout picks the kernel: tiles -> tensor cores, rows -> dp4a."""
+    The weight's layout picks the kernel: tiles -> tensor cores, rows -> dp4a.
+    trunk_only (tiles): the residual path skipped."""
     import torch
     M = xq.shape[0]
     n = 0 if idx is None else int(idx.numel())
@@ -288,13 +290,13 @@ def linear(pw: PackedWeight, xq, sx, x_out, idx, y=None, workspace=None, status=
         workspace = new_workspace(pw, M)
     _ck(lib().sq_linear(ctypes.byref(pw.view), _ptr(xq), _ptr(sx), _ptr(x_out) if n else None,
                         _ptr(idx) if n else None, n, M, _ptr(y), _ptr(workspace),
-                        workspace.numel(), _ptr(status), _flags(pdl),
+                        workspace.numel(), _ptr(status), _flags(pdl, trunk_only),
                         _stream(stream)), "sq_linear")
     return y
 
 
 def quantize_linear(pw: PackedWeight, x, idx, y=None, workspace=None, status=None,
-                    pdl: bool = False, stream=None):
+                    pdl: bool = False, stream=None, trunk_only: bool = False):
     """y[M][N] from fp32 activations x[M][K]: the activation split and the
     linear layer in one kernel (tiled layout), or, for larger M * K with a
     workspace of fused_workspace_bytes, the split once and the linear layer."""
@@ -307,7 +309,7 @@ def quantize_linear(pw: PackedWeight, x, idx, y=None, workspace=None, status=Non
         workspace = new_fused_workspace(pw, M, n)
     _ck(lib().sq_quantize_linear(ctypes.byref(pw.view), _ptr(x), M, _ptr(idx) if n else None, n,
                                  _ptr(y), _ptr(workspace), workspace.numel(), _ptr(status),
-                                 _flags(pdl), _stream(stream)), "sq_quantize_linear")
+                                 _flags(pdl, trunk_only), _stream(stream)), "sq_quantize_linear")
     return y
 
 

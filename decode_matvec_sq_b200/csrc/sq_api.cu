@@ -268,7 +268,9 @@ static sq_status linear_common(const sq_packed_weight* w, const int8_t* xq, cons
   if (M < 1 || M > (1 << 20)) return SQ_ERR_SHAPE;
   if (n_out < 0 || n_out > kMaxOutliers || n_out > w->K) return SQ_ERR_SHAPE;
   if (n_out > 0 && (!idx || !x_out)) return SQ_ERR_INVALID_ARG;
-  if (flags & ~SQ_LAUNCH_PDL) return SQ_ERR_INVALID_ARG;
+  if (flags & ~(SQ_LAUNCH_PDL | SQ_TRUNK_ONLY)) return SQ_ERR_INVALID_ARG;
+  const bool trunk_only = (flags & SQ_TRUNK_ONLY) != 0;
+  if (trunk_only && (w->layout != SQ_LAYOUT_TILES || T_out || R_out)) return SQ_ERR_INVALID_ARG;
   if (!aligned16(xq) || !aligned16(sx) || !aligned16(y) ||
       (n_out > 0 && (!aligned16(idx) || !aligned16(x_out))) || (workspace && !aligned16(workspace)))
     return SQ_ERR_ALIGN;
@@ -302,7 +304,8 @@ static sq_status linear_common(const sq_packed_weight* w, const int8_t* xq, cons
     cudaError_t e;
     if (tc) {
       e = launch_linear_tc(*w, m, xq_t, sx + t0, xo_t, nullptr, idx, n_out, y_t, T_t, R_t,
-                           workspace, part, d.sm_count, dev_status, (flags & SQ_LAUNCH_PDL) != 0, s);
+                           workspace, part, d.sm_count, dev_status, (flags & SQ_LAUNCH_PDL) != 0,
+                           trunk_only, s);
     } else {
       LinearPlan plan;
       if (!plan_linear(*w, m, n_out, d.sm_count, &plan)) return SQ_ERR_SHAPE;
@@ -330,7 +333,7 @@ sq_status sq_linear_accumulators(const sq_packed_weight* w, const int8_t* xq, co
                                  void* stream) {
   if (!T_out || !R_out) return SQ_ERR_INVALID_ARG;
   if (!aligned16(T_out) || !aligned16(R_out)) return SQ_ERR_ALIGN;
-  if (flags & SQ_LAUNCH_PDL) return SQ_ERR_INVALID_ARG;
+  if (flags & (SQ_LAUNCH_PDL | SQ_TRUNK_ONLY)) return SQ_ERR_INVALID_ARG;
   return linear_common(w, xq, sx, x_out, idx, n_out, M, y, T_out, R_out, workspace, ws_bytes,
                        dev_status, flags, stream);
 }
@@ -375,7 +378,7 @@ sq_status sq_quantize_linear(const sq_packed_weight* w, const float* x, int32_t 
   if (M < 1 || M > (1 << 20)) return SQ_ERR_SHAPE;
   if (n_out < 0 || n_out > kMaxOutliers || n_out > w->K) return SQ_ERR_SHAPE;
   if (n_out > 0 && !idx) return SQ_ERR_INVALID_ARG;
-  if (flags & ~SQ_LAUNCH_PDL) return SQ_ERR_INVALID_ARG;
+  if (flags & ~(SQ_LAUNCH_PDL | SQ_TRUNK_ONLY)) return SQ_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(y) || (n_out > 0 && !aligned16(idx)) ||
       (workspace && !aligned16(workspace)))
     return SQ_ERR_ALIGN;
@@ -404,7 +407,8 @@ sq_status sq_quantize_linear(const sq_packed_weight* w, const float* x, int32_t 
     const int m = std::min(per_pass, M - t0);
     cudaError_t e = launch_linear_tc(*w, m, nullptr, nullptr, nullptr, x + (int64_t)t0 * w->K, idx,
                                      n_out, y + (int64_t)t0 * w->N, nullptr, nullptr, workspace,
-                                     part, d.sm_count, dev_status, (flags & SQ_LAUNCH_PDL) != 0, s);
+                                     part, d.sm_count, dev_status, (flags & SQ_LAUNCH_PDL) != 0,
+                                     (flags & SQ_TRUNK_ONLY) != 0, s);
     if (e != cudaSuccess) return SQ_ERR_CUDA;
   }
   return SQ_OK;

@@ -79,7 +79,7 @@ cudaError_t launch_linear_tc(const sq_packed_weight& w, int M, const int8_t* xq,
                              const float* x_out, const float* x, const int32_t* idx, int n_out,
                              float* y, int32_t* T_out, int32_t* R_out, void* workspace,
                              size_t part_bytes, int sm_count, int32_t* status, bool pdl,
-                             cudaStream_t stream);
+                             bool trunk_only, cudaStream_t stream);
 
 // Prefill kernel (SQ_LAYOUT_ROWS, group size 128, many tokens): tcgen05 int8
 // MMAs with TMEM accumulators.  T_out / R_out optional (both or neither).

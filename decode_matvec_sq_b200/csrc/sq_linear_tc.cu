@@ -187,29 +187,36 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-template <bool MASK>
+// RES = false (trunk only): the codes and scales are neither copied nor read.
+template <bool MASK, bool RES>
 __device__ __forceinline__ void copy_tile(uint32_t slot, const Cursor& c, int lane) {
+  if constexpr (RES) {
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const int lo = j * 8 + (lane >> 2), ch = lane & 3;  // owner lane, its chunk
-    cp_async16(slot + lo * 64 + (((ch + (lo >> 1)) & 3) << 4), c.code + 512 * j);
+    for (int j = 0; j < 4; ++j) {
+      const int lo = j * 8 + (lane >> 2), ch = lane & 3;  // owner lane, its chunk
+      cp_async16(slot + lo * 64 + (((ch + (lo >> 1)) & 3) << 4), c.code + 512 * j);
+    }
   }
   cp_async8(slot + Slot<MASK>::kSign + lane * 8, c.sign);
   if constexpr (MASK) cp_async8(slot + Slot<MASK>::kMask + lane * 8, c.mask);
-  cp_async4(slot + Slot<MASK>::kScale + lane * 8, c.scale);
-  cp_async4(slot + Slot<MASK>::kScale + lane * 8 + 4, c.scale + 8);
+  if constexpr (RES) {
+    cp_async4(slot + Slot<MASK>::kScale + lane * 8, c.scale);
+    cp_async4(slot + Slot<MASK>::kScale + lane * 8 + 4, c.scale + 8);
+  }
 }
 
-template <bool MASK>
+template <bool MASK, bool RES>
 __device__ __forceinline__ void read_tile(Tile<MASK>& t, const uint8_t* slot, int lane) {
-  const uint8_t* cb = slot + lane * 64;
+  if constexpr (RES) {
+    const uint8_t* cb = slot + lane * 64;
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const uint4 v = *reinterpret_cast<const uint4*>(cb + (((j + (lane >> 1)) & 3) << 4));
-    t.q[4 * j] = v.x;
-    t.q[4 * j + 1] = v.y;
-    t.q[4 * j + 2] = v.z;
-    t.q[4 * j + 3] = v.w;
+    for (int j = 0; j < 4; ++j) {
+      const uint4 v = *reinterpret_cast<const uint4*>(cb + (((j + (lane >> 1)) & 3) << 4));
+      t.q[4 * j] = v.x;
+      t.q[4 * j + 1] = v.y;
+      t.q[4 * j + 2] = v.z;
+      t.q[4 * j + 3] = v.w;
+    }
   }
   const uint2 sv = *reinterpret_cast<const uint2*>(slot + Slot<MASK>::kSign + lane * 8);
   t.s[0] = sv.x;
@@ -219,9 +226,11 @@ __device__ __forceinline__ void read_tile(Tile<MASK>& t, const uint8_t* slot, in
     t.m[0] = mv.x;
     t.m[1] = mv.y;
   }
-  const float2 cv = *reinterpret_cast<const float2*>(slot + Slot<MASK>::kScale + lane * 8);
-  t.c[0] = cv.x;
-  t.c[1] = cv.y;
+  if constexpr (RES) {
+    const float2 cv = *reinterpret_cast<const float2*>(slot + Slot<MASK>::kScale + lane * 8);
+    t.c[0] = cv.x;
+    t.c[1] = cv.y;
+  }
 }
 
 // Code of channel j (0..31) of row R (0: r0, 1: r1) held in a tile's A
@@ -427,7 +436,9 @@ __device__ __forceinline__ void split_activations(const Params& p, const uint32_
   __syncthreads();
 }
 
-template <bool MASK, bool EMIT, bool FUSED, int D>
+// RES = false: the trunk-only mode (the residual path skipped: no codes or
+// scales read, no residual MMAs, outlier channels take the trunk weight).
+template <bool MASK, bool EMIT, bool FUSED, int D, bool RES>
 __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
   extern __shared__ __align__(16) uint8_t smem[];
   // shared: part [kWarps][2 slots][16 rows][M tokens] float4 | omask[nw] u32 |
@@ -462,7 +473,7 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
   constexpr int kEarly = FUSED ? kDepthEarly : D;
 #pragma unroll
   for (int d = 0; d < kEarly; ++d) {  // one commit group per tile, empty past the range
-    if (t0 + d < t1) copy_tile<MASK>(ring_u + d * Slot<MASK>::kBytes, cur, lane);
+    if (t0 + d < t1) copy_tile<MASK, RES>(ring_u + d * Slot<MASK>::kBytes, cur, lane);
     cp_async_commit();
     cur.advance();
   }
@@ -496,7 +507,7 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
     split_activations(p, omask, xq_s, xo_s, sx_s, reinterpret_cast<float*>(smem + p.off_red), jv, jp);
 #pragma unroll
     for (int d = kEarly; d < D; ++d) {
-      if (t0 + d < t1) copy_tile<MASK>(ring_u + d * Slot<MASK>::kBytes, cur, lane);
+      if (t0 + d < t1) copy_tile<MASK, RES>(ring_u + d * Slot<MASK>::kBytes, cur, lane);
       cp_async_commit();
       cur.advance();
     }
@@ -532,7 +543,7 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
     cp_async_wait<D - 1>();  // this lane's copies of the tile have landed
     __syncwarp();             // ... and every lane's
     Tile<MASK> tl;
-    read_tile<MASK>(tl, ring_w + slot_i * Slot<MASK>::kBytes, lane);
+    read_tile<MASK, RES>(tl, ring_w + slot_i * Slot<MASK>::kBytes, lane);
     // activation codes of this lane's 32 channels for its MMA column
     uint32_t xw[8];
     {
@@ -554,7 +565,8 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
       const uint32_t b0 = xw[2 * m], b1 = xw[2 * m + 1];
-      mma_s8(R, tl.q[4 * m], tl.q[4 * m + 1], tl.q[4 * m + 2], tl.q[4 * m + 3], b0, b1);
+      if constexpr (RES)
+        mma_s8(R, tl.q[4 * m], tl.q[4 * m + 1], tl.q[4 * m + 2], tl.q[4 * m + 3], b0, b1);
       mma_s8(acc.Pn, bits_word(pb0, 2 * m), bits_word(pb1, 2 * m), bits_word(pb0, 2 * m + 1),
              bits_word(pb1, 2 * m + 1), b0, b1);
       if constexpr (MASK)
@@ -564,10 +576,12 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
         mma_s8(acc.S, kOnes, kOnes, kOnes, kOnes, b0, b1);
     }
     // promote the group sums: R[0..1] row r0, R[2..3] row r1
-    acc.F[0] = fmaf(tl.c[0], (float)R[0], acc.F[0]);
-    acc.F[1] = fmaf(tl.c[0], (float)R[1], acc.F[1]);
-    acc.F[2] = fmaf(tl.c[1], (float)R[2], acc.F[2]);
-    acc.F[3] = fmaf(tl.c[1], (float)R[3], acc.F[3]);
+    if constexpr (RES) {
+      acc.F[0] = fmaf(tl.c[0], (float)R[0], acc.F[0]);
+      acc.F[1] = fmaf(tl.c[0], (float)R[1], acc.F[1]);
+      acc.F[2] = fmaf(tl.c[1], (float)R[2], acc.F[2]);
+      acc.F[3] = fmaf(tl.c[1], (float)R[3], acc.F[3]);
+    }
     if (EMIT) {
       const int ng = p.tpr;
       const int r0 = rb * kTileRows + gid, r1 = r0 + 8;
@@ -601,8 +615,10 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
           const uint32_t m1 = MASK ? (tl.m[1] >> bit) & 1u : 1u;
           u0 = m0 ? (((tl.s[0] >> bit) & 1u) ? 1.0f : -1.0f) : 0.0f;
           u1 = m1 ? (((tl.s[1] >> bit) & 1u) ? 1.0f : -1.0f) : 0.0f;
-          w0 = tl.c[0] * (float)tile_code<0>(tl.q, j);
-          w1 = tl.c[1] * (float)tile_code<1>(tl.q, j);
+          if constexpr (RES) {
+            w0 = tl.c[0] * (float)tile_code<0>(tl.q, j);
+            w1 = tl.c[1] * (float)tile_code<1>(tl.q, j);
+          }
         }
         w0 = __shfl_sync(0xffffffffu, w0, owner);
         w1 = __shfl_sync(0xffffffffu, w1, owner);
@@ -634,7 +650,7 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
 
     // refill this slot with the tile D ahead, once no lane reads it
     __syncwarp();
-    if (t + D < t1) copy_tile<MASK>(ring_u + slot_i * Slot<MASK>::kBytes, cur, lane);
+    if (t + D < t1) copy_tile<MASK, RES>(ring_u + slot_i * Slot<MASK>::kBytes, cur, lane);
     cp_async_commit();
     cur.advance();
     if (++slot_i == D) slot_i = 0;
@@ -706,9 +722,9 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
   }
 }
 
-template <bool MASK, bool EMIT, bool FUSED, int D>
+template <bool MASK, bool EMIT, bool FUSED, int D, bool RES = true>
 cudaError_t launch_one(const Params& p, int grid, int smem, bool pdl, cudaStream_t stream) {
-  auto* fn = k_linear_tc<MASK, EMIT, FUSED, D>;
+  auto* fn = k_linear_tc<MASK, EMIT, FUSED, D, RES>;
   cudaError_t e = ensure_smem_attr((const void*)fn, smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -725,23 +741,25 @@ cudaError_t launch_one(const Params& p, int grid, int smem, bool pdl, cudaStream
 }
 
 template <bool MASK, bool FUSED, int D>
-cudaError_t launch_plain(const Params& p, int grid, int smem, bool pdl, cudaStream_t stream) {
-  return launch_one<MASK, false, FUSED, D>(p, grid, smem, pdl, stream);
+cudaError_t launch_plain(const Params& p, bool res, int grid, int smem, bool pdl,
+                         cudaStream_t stream) {
+  return res ? launch_one<MASK, false, FUSED, D, true>(p, grid, smem, pdl, stream)
+             : launch_one<MASK, false, FUSED, D, false>(p, grid, smem, pdl, stream);
 }
 
 // Non-accumulator launch with a ring depth chosen at run time among Ds.
 template <int D0, int... Ds>
-cudaError_t launch_depth(int depth, bool mask, bool fused, const Params& p, int grid, int smem,
-                         bool pdl, cudaStream_t stream) {
+cudaError_t launch_depth(int depth, bool mask, bool fused, bool res, const Params& p, int grid,
+                         int smem, bool pdl, cudaStream_t stream) {
   if (depth == D0 || sizeof...(Ds) == 0) {
     if (fused)
-      return mask ? launch_plain<true, true, D0>(p, grid, smem, pdl, stream)
-                  : launch_plain<false, true, D0>(p, grid, smem, pdl, stream);
-    return mask ? launch_plain<true, false, D0>(p, grid, smem, pdl, stream)
-                : launch_plain<false, false, D0>(p, grid, smem, pdl, stream);
+      return mask ? launch_plain<true, true, D0>(p, res, grid, smem, pdl, stream)
+                  : launch_plain<false, true, D0>(p, res, grid, smem, pdl, stream);
+    return mask ? launch_plain<true, false, D0>(p, res, grid, smem, pdl, stream)
+                : launch_plain<false, false, D0>(p, res, grid, smem, pdl, stream);
   }
   if constexpr (sizeof...(Ds) > 0)
-    return launch_depth<Ds...>(depth, mask, fused, p, grid, smem, pdl, stream);
+    return launch_depth<Ds...>(depth, mask, fused, res, p, grid, smem, pdl, stream);
   return cudaErrorInvalidValue;
 }
 
@@ -780,8 +798,9 @@ cudaError_t launch_linear_tc(const sq_packed_weight& w, int M, const int8_t* xq,
                              const float* x_out, const float* x, const int32_t* idx, int n_out,
                              float* y, int32_t* T_out, int32_t* R_out, void* workspace,
                              size_t part_bytes, int sm_count, int32_t* status, bool pdl,
-                             cudaStream_t stream) {
+                             bool trunk_only, cudaStream_t stream) {
   if (M < 1 || M > kCols || w.layout != SQ_LAYOUT_TILES) return cudaErrorInvalidValue;
+  if (trunk_only && T_out) return cudaErrorInvalidValue;
   const bool fused = x != nullptr;
   if (fused && (T_out || M > linear_tc_fused_tokens(w, n_out))) return cudaErrorInvalidValue;
   Params p;
@@ -841,7 +860,7 @@ cudaError_t launch_linear_tc(const sq_packed_weight& w, int M, const int8_t* xq,
   if (emit)
     return mask ? launch_one<true, true, false, kShallow>(p, grid, smem, pdl, stream)
                 : launch_one<false, true, false, kShallow>(p, grid, smem, pdl, stream);
-  return launch_depth<kDeep, kShallow>(depth, mask, fused, p, grid, smem, pdl, stream);
+  return launch_depth<kDeep, kShallow>(depth, mask, fused, !trunk_only, p, grid, smem, pdl, stream);
 }
 
 }  // namespace sq

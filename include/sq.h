@@ -54,6 +54,16 @@ typedef enum {
 
 /* Launch flags (bit set). */
 #define SQ_LAUNCH_PDL 1u
+#define SQ_TRUNK_ONLY 2u
+/* SQ_TRUNK_ONLY (sq_linear, sq_quantize_linear, sq_linear_noalloc; weights in
+ * SQ_LAYOUT_TILES only, else SQ_ERR_INVALID_ARG): the residual path is
+ * skipped (m.lqnn.cn section 3.3: the 1-bit trunk first, the residual added
+ * on demand; a request that tolerates a rougher answer skips it).  The
+ * residual codes and scales are not read:
+ *   y_tr = sx_t * alpha_r * T_tr + sum_i Wt_{r,idx_i} * x_out_ti,
+ *   Wt_rj = m_rj * alpha_r * (2 b_rj - 1)
+ * (outlier channels take the trunk weight).  Not accepted by
+ * sq_linear_accumulators. */
 /* SQ_LAUNCH_PDL: launch with programmatic dependent launch.  The kernel may
  * start while the previous kernel in the stream is still running and begins
  * streaming the packed weights at once; it reads every other input and writes
@@ -203,6 +213,7 @@ size_t sq_linear_workspace_bytes(const sq_packed_weight *w, int32_t M);
  *   R_g = sum_{j in g} q*xq                                     (exact int32)
  *   y  = sx*(alpha*T + sum_g s_g*R_g) + sum_i What[r][idx_i]*x_out[i]
  * with What = m*(+-alpha) + s_g*q the dequantized weight, in fp32.
+ * flags: SQ_LAUNCH_PDL and/or SQ_TRUNK_ONLY (the residual terms dropped).
  */
 sq_status sq_linear(const sq_packed_weight *w, const int8_t *xq, const float *sx,
                     const float *x_out, const int32_t *idx, int32_t n_out, int32_t M, float *y,
@@ -245,9 +256,9 @@ sq_status sq_linear_accumulators(const sq_packed_weight *w, const int8_t *xq, co
  * more fused passes than the decode kernel's passes of 8, and the workspace
  * is large enough, the call runs sq_quantize_act once into the workspace and
  * then sq_linear on its codes (two launches; y is the same bit for bit).
- * flags: 0 or SQ_LAUNCH_PDL (the kernel then reads x, idx and y-independent
- * data only after the previous kernel completes; the packed weights are
- * streamed before).
+ * flags: SQ_LAUNCH_PDL (the kernel then reads x, idx and y-independent data
+ * only after the previous kernel completes; the packed weights are streamed
+ * before) and/or SQ_TRUNK_ONLY.
  */
 sq_status sq_quantize_linear(const sq_packed_weight *w, const float *x, int32_t M,
                              const int32_t *idx, int32_t n_out, float *y, void *workspace,

@@ -66,10 +66,12 @@ def _load():
             lin = [i64, i64, i64, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp]
             lib.sqo_linear.argtypes = lin
             lib.sqo_linear_naive.argtypes = lin
+            lib.sqo_linear_trunk.argtypes = [i64, i64, i64, vp, vp, vp, vp, vp, vp, vp, i32, vp]
             lib.sqo_abs_dot.argtypes = [i64, i64, i64, vp, vp, vp]
             for name in ("sqo_quantize_groups", "sqo_trunk_threshold", "sqo_decompose",
                          "sqo_calibrate", "sqo_quantize_act", "sqo_accumulate",
-                         "sqo_trunk_popcount", "sqo_linear", "sqo_linear_naive", "sqo_abs_dot"):
+                         "sqo_trunk_popcount", "sqo_linear", "sqo_linear_naive", "sqo_linear_trunk",
+                         "sqo_abs_dot"):
                 getattr(lib, name).restype = i32
             _lib = lib
     return _lib
@@ -219,6 +221,23 @@ def linear(d, xq, sx, xout, idx):
 def linear_naive(d, xq, sx, xout, idx):
     """Second route: y = sum_j What_j * xhat_j (binary64)."""
     return _linear(_load().sqo_linear_naive, d, xq, sx, xout, idx)
+
+
+def linear_trunk(d, xq, sx, xout, idx):
+    """Trunk-only y = sx*alpha*T + sum_i Wt*xout, Wt = m*alpha*(2b-1): the
+    residual path skipped ([P1] s3.3, binary64)."""
+    xq = _c(xq, np.int8)
+    M, K = xq.shape
+    N = d["sign"].shape[0]
+    idx = _c(idx, np.int32)
+    n = idx.shape[0]
+    sx = _c(sx, np.float32)
+    xout = _c(xout, np.float32).reshape(M, n) if n else np.zeros((M, 1), np.float32)
+    y = np.zeros((M, N), np.float64)
+    _ck(_load().sqo_linear_trunk(M, N, K, _p(d["sign"]), _p(d["mask"]), _p(d["alpha"]), _p(xq),
+                                 _p(sx), _p(xout), _p(idx) if n else None, n, _p(y)),
+        "linear_trunk")
+    return y
 
 
 def abs_dot(W, x):

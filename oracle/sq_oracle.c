@@ -351,6 +351,31 @@ int sqo_linear(int64_t M, int64_t N, int64_t K, int G, const uint8_t *sign,
     return SQO_OK;
 }
 
+int sqo_linear_trunk(int64_t M, int64_t N, int64_t K, const uint8_t *sign,
+                     const uint8_t *mask, const float *alpha, const int8_t *xq,
+                     const float *sx, const float *xout, const int32_t *idx, int n_out,
+                     double *y)
+{
+    if (M < 1 || N < 1 || K < 1 || !sign || !mask || !alpha || !xq || !sx || !y ||
+        !check_idx(idx, n_out, K) || (n_out > 0 && !xout))
+        return SQO_BAD_ARG;
+    for (int64_t t = 0; t < M; ++t)
+        for (int64_t r = 0; r < N; ++r) {
+            int64_t T = 0;  /* the direct +-1 sum over the trunk */
+            for (int64_t j = 0; j < K; ++j)
+                if (mask[r * K + j])
+                    T += (sign[r * K + j] ? 1 : -1) * (int64_t)xq[t * K + j];
+            double out = (double)sx[t] * ((double)alpha[r] * (double)T);
+            for (int i = 0; i < n_out; ++i) {
+                int64_t j = idx[i];
+                double wt = mask[r * K + j] ? (sign[r * K + j] ? (double)alpha[r] : -(double)alpha[r]) : 0.0;
+                out += wt * (double)xout[t * n_out + i];
+            }
+            y[t * N + r] = out;
+        }
+    return SQO_OK;
+}
+
 int sqo_linear_naive(int64_t M, int64_t N, int64_t K, int G, const uint8_t *sign,
                      const uint8_t *mask, const float *alpha, const int8_t *q,
                      const float *s, const int8_t *xq, const float *sx,

@@ -120,6 +120,16 @@ int sqo_linear(int64_t M, int64_t N, int64_t K, int G, const uint8_t *sign,
                const float *s, const int8_t *xq, const float *sx,
                const float *xout, const int32_t *idx, int n_out, double *y);
 
+/* Trunk-only output (m.lqnn.cn news 241359, section 3.3: the 1-bit trunk is
+ * computed first and the residual added on demand; a request may skip the
+ * residual path).  The residual arrays are not read:
+ *   y_tr = sx_t*alpha_r*T_tr + sum_i Wt_{r,idx_i}*xout_ti,
+ *   Wt_rj = mask*alpha*(2*sign-1).  All binary64. */
+int sqo_linear_trunk(int64_t M, int64_t N, int64_t K, const uint8_t *sign,
+                     const uint8_t *mask, const float *alpha, const int8_t *xq,
+                     const float *sx, const float *xout, const int32_t *idx, int n_out,
+                     double *y);
+
 /* Naive second route: y_tr = sum_j What_rj * xhat_tj with
  * xhat = xq*sx off the outlier set and x itself on it. */
 int sqo_linear_naive(int64_t M, int64_t N, int64_t K, int G, const uint8_t *sign,

@@ -107,7 +107,12 @@ def test_host_validation_before_device_work(L):
     assert L.sq_linear(ctypes.byref(v), p, p, p, p, 1, 0, p, p, 1 << 20, None, 0, None) == 2
     assert L.sq_linear(ctypes.byref(v), bad, p, p, p, 1, 1, p, p, 1 << 20, None, 0, None) == 3
     assert L.sq_linear(ctypes.byref(v), p, p, p, p, 1, 1, p, p, 1 << 20, None, 8, None) == 1
-    assert L.sq_linear(ctypes.byref(v), p, p, p, p, 1, 1, p, p, 1 << 20, None, 2, None) == 1
+    assert L.sq_linear(ctypes.byref(v), p, p, p, p, 1, 1, p, p, 1 << 20, None, 4, None) == 1
+    # SQ_TRUNK_ONLY (2) needs the tiled layout
+    vr = sq.SqPackedWeight()
+    L.sq_packed_view(ctypes.c_void_p(1 << 40), 64, 256, 128, 0, 0, ctypes.byref(vr))
+    assert L.sq_linear(ctypes.byref(vr), p, p, p, p, 1, 1, p, p, 1 << 20, None, 2, None) == 1
+    assert L.sq_linear(ctypes.byref(vr), p, p, p, p, 1, 1, p, p, 1 << 20, None, 3, None) == 1
     w3 = sq.SqPackedWeight.from_buffer_copy(v)
     w3.layout = 5
     assert L.sq_linear(ctypes.byref(w3), p, p, p, p, 1, 1, p, p, 1 << 20, None, 0, None) == 1
@@ -115,9 +120,12 @@ def test_host_validation_before_device_work(L):
     w2 = sq.SqPackedWeight.from_buffer_copy(v)
     w2.res_stride = 100
     assert L.sq_linear(ctypes.byref(w2), p, p, p, p, 1, 1, p, p, 1 << 20, None, 0, None) == 2
-    # accumulators: PDL is not accepted
-    assert L.sq_linear_accumulators(ctypes.byref(v), p, p, p, p, 1, 1, p, p, p, p, 1 << 20, None,
-                                    1, None) == 1
+    # accumulators: neither PDL nor the trunk-only mode is accepted
+    for flags in (1, 2):
+        assert L.sq_linear_accumulators(ctypes.byref(v), p, p, p, p, 1, 1, p, p, p, p, 1 << 20, None,
+                                        flags, None) == 1
+    # sq_quantize_linear(w, x, M, idx, n_out, y, ws, ws_bytes, status, flags, stream): unknown flag
+    assert L.sq_quantize_linear(ctypes.byref(v), p, 1, p, 1, p, p, 1 << 20, None, 4, None) == 1
     assert L.sq_decompose_pack(None, 64, 256, -1, ctypes.byref(v), None, None) == 1
     assert L.sq_decompose_pack(p, 64, 256, 0, ctypes.byref(v), None, None) == 1
     assert L.sq_decompose_pack(p, 64, 256, 60, ctypes.byref(v), None, None) == 1  # no mask array

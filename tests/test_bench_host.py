@@ -106,3 +106,14 @@ def test_single_layer_workload_cases():
     assert all(c[3] * c[1].packed_bytes >= 2 * bench.L2_BYTES for c in mlp)
     (label, L, M, copies), = bench.layer_cases("threshold")
     assert L.trunk_percent == 60 and M == 1 and copies * L.packed_bytes >= 2 * bench.L2_BYTES
+
+
+def test_trunk_workload_cases():
+    """The trunk-only workload covers the stack's four shapes at batch 1, each
+    rotating over at least twice the L2 capacity of sign bits and row scales."""
+    cases = bench.layer_cases("trunk")
+    assert [(c[1].K, c[1].N) for c in cases] == [(4096, 12288), (4096, 4096), (4096, 22016), (11008, 4096)]
+    for label, L, M, copies in cases:
+        assert M == 1 and copies * bench.trunk_weight_bytes(L) >= 2 * bench.L2_BYTES
+        # sign bits (1/8 byte per weight of the padded tile grid) + 4 bytes per padded row
+        assert bench.trunk_weight_bytes(L) == (-(-L.N // 16) * 16) * (-(-L.K // 128) * 16 + 4)

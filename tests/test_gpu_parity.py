@@ -588,6 +588,54 @@ def test_quantize_linear_status_and_errors():
     assert e.value.name == "SQ_ERR_SHAPE"
 
 
+# ---- trunk-only mode (residual path skipped) ------------------------------------
+
+@pytest.mark.parametrize("N,K,M,n,P", [(1, 8, 1, 0, -1), (40, 129, 8, 1, -1), (20, 300, 3, 3, 60),
+                                       (513, 300, 1, 6, -1), (64, 4096, 2, 20, 60),
+                                       (24, 11008, 1, 55, -1), (16, 28672, 4, 72, -1)])
+def test_trunk_only_parity(N, K, M, n, P):
+    """sq_linear with SQ_TRUNK_ONLY against the oracle's trunk-only output,
+    and sq_quantize_linear (fused kernel and staged route) bit for bit
+    against it."""
+    rng = np.random.default_rng(3 * N + K + 5 * M + n + P)
+    W = rng.laplace(0, 0.02, (N, K)).astype(np.float32)
+    x = rng.standard_normal((M, K)).astype(np.float32)
+    idx = np.sort(rng.choice(K, n, replace=False)).astype(np.int32)
+    x[:, idx] *= 30.0
+    Wd, xd = torch.from_numpy(W).cuda(), torch.from_numpy(x).cuda()
+    idxd = torch.from_numpy(idx).cuda() if n else None
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pw = sq.decompose_pack(Wd, trunk_percent=P, layout=sq.SQ_LAYOUT_TILES, status=st)
+    xq, sx, xo = sq.quantize_act(xd, idxd, status=st)
+    y = sq.linear(pw, xq, sx, xo, idxd, status=st, trunk_only=True)
+    for ws in (sq.new_workspace(pw, M), sq.new_fused_workspace(pw, M, n)):
+        y1 = torch.full_like(y, float("nan"))
+        sq.quantize_linear(pw, xd, idxd, y=y1, workspace=ws, status=st, trunk_only=True)
+        torch.cuda.synchronize()
+        assert np.array_equal(y1.cpu().numpy().view(np.uint32), y.cpu().numpy().view(np.uint32))
+    assert st.item() == 0
+    d = oracle.decompose(W, P=P)
+    oxq, osx, oxo = oracle.quantize_act(x, idx)
+    ref = oracle.linear_trunk(d, oxq, osx, oxo, idx)
+    xh = oxq.astype(np.float64) * osx.astype(np.float64)[:, None]
+    xh[:, idx] = x[:, idx]
+    trunk_hat = d["mask"] * d["alpha"].astype(np.float64)[:, None]
+    bound = np.abs(xh) @ trunk_hat.T
+    err = np.abs(y.cpu().numpy().astype(np.float64) - ref)
+    assert np.all(err <= 1e-5 * bound + 1e-30), float((err / np.maximum(bound, 1e-30)).max())
+    # the full output differs from it by the residual path
+    assert not torch.equal(y, sq.linear(pw, xq, sx, xo, idxd, status=st)) or not d["q"].any()
+
+
+def test_trunk_only_rejected_for_row_layout():
+    W = torch.randn(32, 256, device="cuda")
+    pr = sq.decompose_pack(W, layout=sq.SQ_LAYOUT_ROWS)
+    xq, sx, xo = sq.quantize_act(torch.randn(1, 256, device="cuda"), None)
+    with pytest.raises(sq.SQError) as e:
+        sq.linear(pr, xq, sx, xo, None, trunk_only=True)
+    assert e.value.name == "SQ_ERR_INVALID_ARG"
+
+
 def test_quantize_linear_staged_route_status():
     """The staged route (M * roundup(K,128) > 16 KiB) reports the same device
     findings as the fused kernel: non-finite x, a bad index list."""

@@ -43,6 +43,16 @@ MUTANTS = {
                             "double inner = (double)T[t * N + r];"),
     "group_scale_index_shifted": ("inner += (double)s[r * ng + g] * (double)R[(t * N + r) * ng + g];",
                                   "inner += (double)s[r * ng + (g + 1) % ng] * (double)R[(t * N + r) * ng + g];"),
+    "trunk_only_ignores_mask": ("                if (mask[r * K + j])\n                    T +=",
+                                "                if (1)\n                    T +="),
+    "trunk_only_sign_flipped": ("T += (sign[r * K + j] ? 1 : -1) * (int64_t)xq[t * K + j];",
+                                "T += (sign[r * K + j] ? -1 : 1) * (int64_t)xq[t * K + j];"),
+    "trunk_only_outliers_dropped": ("out += wt * (double)xout[t * n_out + i];",
+                                    "out += 0.0 * wt * (double)xout[t * n_out + i];"),
+    "trunk_only_outlier_weight_unmasked": ("double wt = mask[r * K + j] ? (sign[r * K + j]",
+                                           "double wt = 1 ? (sign[r * K + j]"),
+    "trunk_only_scale_missing": ("double out = (double)sx[t] * ((double)alpha[r] * (double)T);",
+                                 "double out = (double)alpha[r] * (double)T;"),
 }
 
 

@@ -331,6 +331,60 @@ def test_factored_equals_naive(P):
     assert np.all(np.abs(y - ref) <= 0.05 * scale)
 
 
+# ---- trunk-only output (residual path skipped, [P1] s3.3) -----------------------
+
+def _xhat(x, xq, sx, idx):
+    """Dequantized activations: xq*sx off the outlier set, x itself on it."""
+    xh = xq.astype(np.float64) * sx.astype(np.float64)[:, None]
+    xh[:, idx] = x[:, idx].astype(np.float64)
+    return xh
+
+
+def test_trunk_only_binary_weights_is_the_exact_product():
+    """Rows whose entries are all +-c_r: alpha_r = c_r, the residual vanishes,
+    and the trunk-only output is the full output and the plain product W.xhat."""
+    rng = np.random.default_rng(41)
+    N, K = 24, 700
+    c = (rng.integers(1, 64, N) / 1024.0).astype(np.float32)
+    W = (np.where(rng.random((N, K)) < 0.5, -1.0, 1.0) * c[:, None]).astype(np.float32)
+    x = rng.standard_normal((3, K)).astype(np.float32)
+    idx = np.array([5, 311, 699], np.int32)
+    x[:, idx] *= 40.0
+    d = oracle.decompose(W)
+    assert np.array_equal(d["alpha"], c) and not d["q"].any()
+    xq, sx, xout = oracle.quantize_act(x, idx)
+    yt = oracle.linear_trunk(d, xq, sx, xout, idx)
+    ref = _xhat(x, xq, sx, idx) @ W.astype(np.float64).T
+    scale = np.abs(_xhat(x, xq, sx, idx)) @ np.abs(W.astype(np.float64)).T
+    assert np.all(np.abs(yt - ref) <= 1e-12 * scale)
+    assert np.all(np.abs(yt - oracle.linear(d, xq, sx, xout, idx)) <= 1e-12 * scale)
+
+
+@pytest.mark.parametrize("P", [-1, 60])
+def test_trunk_only_plus_residual_path_is_the_full_output(P):
+    """y - y_trunk is the residual path alone: the dense dequantized residual
+    s_{r,g(j)} * q_rj times xhat, formed here with numpy."""
+    L = wl.config1()
+    W = L.weights()[:40]
+    x = L.activations(M=2)
+    idx = L.planted_channels()
+    d = oracle.decompose(W, P=P)
+    xq, sx, xout = oracle.quantize_act(x, idx)
+    xh = _xhat(x, xq, sx, idx)
+    y = oracle.linear(d, xq, sx, xout, idx)
+    yt = oracle.linear_trunk(d, xq, sx, xout, idx)
+    G = d["G"]
+    res_hat = d["s"].astype(np.float64)[:, np.arange(W.shape[1]) // G] * d["q"].astype(np.float64)
+    trunk_hat = d["mask"] * np.where(d["sign"] == 1, 1.0, -1.0) * d["alpha"].astype(np.float64)[:, None]
+    scale = np.abs(xh) @ (np.abs(res_hat) + np.abs(trunk_hat)).T
+    assert np.all(np.abs((y - yt) - xh @ res_hat.T) <= 1e-12 * scale)
+    # the trunk-only output is the dense trunk weight times xhat: the mask
+    # removes entries, outlier channels take the trunk weight, not the full one
+    assert np.all(np.abs(yt - xh @ trunk_hat.T) <= 1e-12 * scale)
+    if P > 0:
+        assert (d["mask"] == 0).any()
+
+
 # ---- calibration and activations ----------------------------------------------
 
 def test_calibration_recovers_planted_channels():
