@@ -318,7 +318,7 @@ NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 def linear_noalloc(pw: PackedWeight, xq, sx, x_out, idx, y, status=None, pdl: bool = False,
-                   stream=None):
+                   stream=None, trunk_only: bool = False):
     """sq_linear with the library's fixed device scratch instead of a workspace
     (for callers that cannot allocate device memory at call time).  y [M][N]
     float32 is the caller's.  Calls on one device must not overlap in time."""
@@ -326,7 +326,7 @@ def linear_noalloc(pw: PackedWeight, xq, sx, x_out, idx, y, status=None, pdl: bo
     n = 0 if idx is None else int(idx.numel())
     _ck(lib().sq_linear_noalloc(ctypes.byref(pw.view), _ptr(xq), _ptr(sx),
                                 _ptr(x_out) if n else None, _ptr(idx) if n else None, n, M,
-                                _ptr(y), _ptr(status), _flags(pdl), _stream(stream)),
+                                _ptr(y), _ptr(status), _flags(pdl, trunk_only), _stream(stream)),
         "sq_linear_noalloc")
     return y
 

@@ -71,3 +71,19 @@ def test_noalloc_rejects_problems_beyond_its_scratch(cuda_device):
     p = ctypes.c_void_p(1 << 41)
     rc = L.sq_linear_noalloc(ctypes.byref(v), p, p, None, None, 0, 1, p, None, 0, None)
     assert rc == 8 and L.sq_status_string(rc)  # SQ_ERR_WORKSPACE
+
+
+@pytest.mark.gpu
+def test_noalloc_trunk_only_matches_sq_linear(cuda_device):
+    """The trunk-only flag passes through the no-allocation entry point."""
+    W, x, idx = _inputs(1000, 1000, 3, 9, seed=5)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pw = sq.decompose_pack(torch.from_numpy(W).cuda(), layout=1, status=st)
+    idxd = torch.from_numpy(idx).cuda()
+    xq, sx, xo = sq.quantize_act(torch.from_numpy(x).cuda(), idxd, status=st)
+    y_ref = sq.linear(pw, xq, sx, xo, idxd, status=st, trunk_only=True)
+    y = torch.full((3, 1000), float("nan"), dtype=torch.float32, device="cuda")
+    sq.linear_noalloc(pw, xq, sx, xo, idxd, y, status=st, trunk_only=True)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    assert torch.equal(y, y_ref)
