@@ -146,3 +146,20 @@ def test_product_path_does_not_import_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
                 text = open(os.path.join(dirpath, f), encoding="utf-8").read()
                 assert "oracle" not in text.replace("no CPU fallback", ""), f
+
+
+def test_fused_tokens_per_pass(L):
+    """Tokens per fused pass follow the shared-memory arithmetic of
+    include/sq.h: a ring of two 2560-byte slots (2816 with a mask) per warp,
+    16 warps; an outlier table of K/32*8 bytes; per token roundup(K,128) +
+    4*roundup(n,4) + 8192 bytes; 227 KiB in all.  Host-only: no device."""
+    def view(N, K, mask=False, layout=1):
+        v = sq.SqPackedWeight()
+        assert L.sq_packed_view(ctypes.c_void_p(1 << 40), N, K, 128, int(mask), layout, ctypes.byref(v)) == 0
+        return v
+    for K, n, mask, want in [(4096, 20, False, 8), (11008, 55, False, 7), (28672, 72, False, 3),
+                             (28672, 72, True, 3), (65536, 0, False, 1), (131072, 0, False, 0)]:
+        assert L.sq_quantize_linear_tokens_per_pass(ctypes.byref(view(64, K, mask)), n) == want, (K, n)
+    assert L.sq_quantize_linear_tokens_per_pass(ctypes.byref(view(64, 4096, layout=0)), 20) == 0
+    assert L.sq_quantize_linear_tokens_per_pass(ctypes.byref(view(64, 4096)), -1) == 0
+    assert L.sq_quantize_linear_tokens_per_pass(None, 0) == 0

@@ -656,28 +656,16 @@ def test_quantize_linear_staged_route_status():
     assert st.item() == sq.STATUS_CODE["SQ_ERR_INVALID_ARG"]
 
 
-def test_fused_pass_and_workspace_queries():
-    """Tokens per fused pass and the staged-route workspace follow the shared
-    memory and workspace arithmetic of include/sq.h."""
+def test_fused_workspace_query():
+    """The staged-route workspace follows the arithmetic of include/sq.h."""
     L = sq.lib()
-    def tiles(N, K, mask=False):
-        v = sq.SqPackedWeight()
-        assert L.sq_packed_view(ctypes.c_void_p(1 << 40), N, K, 128, int(mask), 1, ctypes.byref(v)) == 0
-        return v
-    # ring of two 2560-byte slots per warp, 16 warps; outlier table K/32*8; per
-    # token roundup(K,128) + 4*roundup(n,4) + 8192; 227 KiB in all
-    for K, n, mask, want in [(4096, 20, False, 8), (11008, 55, False, 7), (28672, 72, False, 3),
-                             (28672, 72, True, 3), (65536, 0, False, 1), (131072, 0, False, 0)]:
-        assert L.sq_quantize_linear_tokens_per_pass(ctypes.byref(tiles(64, K, mask)), n) == want, (K, n)
-    v = sq.SqPackedWeight()
-    assert L.sq_packed_view(ctypes.c_void_p(1 << 40), 64, 4096, 128, 0, 0, ctypes.byref(v)) == 0
-    assert L.sq_quantize_linear_tokens_per_pass(ctypes.byref(v), 20) == 0  # row layout
     r = lambda a: -(-a // 256) * 256
+    w = sq.SqPackedWeight()
+    assert L.sq_packed_view(ctypes.c_void_p(1 << 40), 300, 8192, 128, 0, 1, ctypes.byref(w)) == 0
     for M, n in [(1, 0), (4, 20), (16, 72)]:
-        w = tiles(300, 8192)
         got = L.sq_quantize_linear_workspace_bytes(ctypes.byref(w), M, n)
         assert got == r(L.sq_linear_workspace_bytes(ctypes.byref(w), M)) + r(M * 8192) + r(4 * M) + r(4 * M * n)
-    assert L.sq_quantize_linear_workspace_bytes(ctypes.byref(tiles(300, 8192)), 0, 0) == 0
+    assert L.sq_quantize_linear_workspace_bytes(ctypes.byref(w), 0, 0) == 0
 
 
 # ---- prefill: many tokens on tcgen05 (row layout, M >= 64) --------------------------
