@@ -67,11 +67,12 @@ def _load():
             lib.sqo_linear.argtypes = lin
             lib.sqo_linear_naive.argtypes = lin
             lib.sqo_linear_trunk.argtypes = [i64, i64, i64, vp, vp, vp, vp, vp, vp, vp, i32, vp]
+            lib.sqo_sparsify_residual.argtypes = [vp, i64, i32, i32, vp, vp, vp]
             lib.sqo_abs_dot.argtypes = [i64, i64, i64, vp, vp, vp]
             for name in ("sqo_quantize_groups", "sqo_trunk_threshold", "sqo_decompose",
                          "sqo_calibrate", "sqo_quantize_act", "sqo_accumulate",
                          "sqo_trunk_popcount", "sqo_linear", "sqo_linear_naive", "sqo_linear_trunk",
-                         "sqo_abs_dot"):
+                         "sqo_sparsify_residual", "sqo_abs_dot"):
                 getattr(lib, name).restype = i32
             _lib = lib
     return _lib
@@ -151,6 +152,33 @@ def decompose(W, G: int = 128, P: int = -1, want_residual: bool = False):
 
 
 # ---- calibration and activations ([P1] s2.2, [P2] dynamic quantization) -----
+
+def sparsify_residual(r, G: int, Ps: int):
+    """One residual row r[K] (float64): drop the entries at or below the
+    nearest-rank Ps-th percentile of |r| (strict > keeps), quantize the kept
+    ones by groups ([P1] s3.3, sparse residual).  Returns keep, q, s."""
+    r = _c(r, np.float64)
+    K = r.shape[0]
+    keep = np.zeros(K, np.uint8)
+    q = np.zeros(K, np.int8)
+    s = np.zeros(n_groups(K, G), np.float32)
+    _ck(_load().sqo_sparsify_residual(_p(r), K, G, Ps, _p(keep), _p(q), _p(s)), "sparsify_residual")
+    return keep, q, s
+
+
+def decompose_sparse(W, G: int = 128, P: int = -1, Ps: int = 60):
+    """decompose() with the residual sparsified row by row (keys as
+    decompose, plus keep [N][K] uint8)."""
+    d = decompose(W, G=G, P=P, want_residual=True)
+    N, K = d["res"].shape
+    keep = np.zeros((N, K), np.uint8)
+    q = np.zeros_like(d["q"])
+    s = np.zeros_like(d["s"])
+    for r in range(N):
+        keep[r], q[r], s[r] = sparsify_residual(d["res"][r], G, Ps)
+    d = dict(d, q=q, s=s, keep=keep)
+    return d
+
 
 def calibrate(X, k: int) -> np.ndarray:
     X = _c(X, np.float32)

@@ -351,6 +351,42 @@ int sqo_linear(int64_t M, int64_t N, int64_t K, int G, const uint8_t *sign,
     return SQO_OK;
 }
 
+static int cmp_double(const void *a, const void *b)
+{
+    double x = *(const double *)a, y = *(const double *)b;
+    return (x > y) - (x < y);
+}
+
+int sqo_sparsify_residual(const double *r, int64_t K, int G, int Ps, uint8_t *keep,
+                          int8_t *q, float *s)
+{
+    if (!r || !keep || !q || !s || K < 1 || !valid_group(G) || Ps < 0 || Ps > 99)
+        return SQO_BAD_ARG;
+    double *a = (double *)malloc((size_t)K * sizeof(double));
+    double *kept = (double *)malloc((size_t)K * sizeof(double));
+    if (!a || !kept) {
+        free(a);
+        free(kept);
+        return SQO_BAD_ARG;
+    }
+    for (int64_t j = 0; j < K; ++j)
+        a[j] = fabs(r[j]);
+    double theta = -1.0; /* Ps = 0: nothing dropped */
+    if (Ps > 0) {
+        qsort(a, (size_t)K, sizeof(double), cmp_double);
+        int64_t rank = ((int64_t)Ps * K + 99) / 100; /* ceil(Ps*K/100), >= 1 */
+        theta = a[rank - 1];
+    }
+    for (int64_t j = 0; j < K; ++j) {
+        keep[j] = (uint8_t)(fabs(r[j]) > theta);
+        kept[j] = keep[j] ? r[j] : 0.0;
+    }
+    int rc = sqo_quantize_groups(kept, K, G, q, s);
+    free(a);
+    free(kept);
+    return rc;
+}
+
 int sqo_linear_trunk(int64_t M, int64_t N, int64_t K, const uint8_t *sign,
                      const uint8_t *mask, const float *alpha, const int8_t *xq,
                      const float *sx, const float *xout, const int32_t *idx, int n_out,

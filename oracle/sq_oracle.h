@@ -120,6 +120,16 @@ int sqo_linear(int64_t M, int64_t N, int64_t K, int G, const uint8_t *sign,
                const float *s, const int8_t *xq, const float *sx,
                const float *xout, const int32_t *idx, int n_out, double *y);
 
+/* Sparse residual (m.lqnn.cn news 241359, section 3.3, second point: a small
+ * threshold zeroes the residual entries near zero, typically 50-70 % of
+ * them, which are then stored in a sparse form).  For one residual row r[K]
+ * (binary64): theta = the ceil(Ps*K/100)-th smallest |r_j| (nearest rank,
+ * 1 <= Ps <= 99; Ps = 0 keeps every entry); keep[j] = (|r_j| > theta)
+ * (strict: ties at theta are dropped); then the kept entries (the dropped
+ * ones as 0) are quantized by groups of G exactly as sqo_quantize_groups. */
+int sqo_sparsify_residual(const double *r, int64_t K, int G, int Ps, uint8_t *keep,
+                          int8_t *q, float *s);
+
 /* Trunk-only output (m.lqnn.cn news 241359, section 3.3: the 1-bit trunk is
  * computed first and the residual added on demand; a request may skip the
  * residual path).  The residual arrays are not read:

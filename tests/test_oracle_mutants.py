@@ -53,6 +53,12 @@ MUTANTS = {
                                            "double wt = 1 ? (sign[r * K + j]"),
     "trunk_only_scale_missing": ("double out = (double)sx[t] * ((double)alpha[r] * (double)T);",
                                  "double out = (double)alpha[r] * (double)T;"),
+    "sparse_keeps_ties": ("keep[j] = (uint8_t)(fabs(r[j]) > theta);",
+                          "keep[j] = (uint8_t)(fabs(r[j]) >= theta);"),
+    "sparse_rank_floor_plus_one": ("int64_t rank = ((int64_t)Ps * K + 99) / 100;",
+                                   "int64_t rank = ((int64_t)Ps * K) / 100 + 1;"),
+    "sparse_quantizes_dropped_entries": ("kept[j] = keep[j] ? r[j] : 0.0;", "kept[j] = r[j];"),
+    "sparse_theta_next_rank": ("theta = a[rank - 1];", "theta = a[rank < K ? rank : K - 1];"),
 }
 
 

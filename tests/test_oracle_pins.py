@@ -385,6 +385,73 @@ def test_trunk_only_plus_residual_path_is_the_full_output(P):
         assert (d["mask"] == 0).any()
 
 
+# ---- sparse residual ([P1] s3.3, second point) -----------------------------------
+
+@pytest.mark.parametrize("K,Ps", [(300, 60), (128, 50), (1000, 70), (97, 1), (64, 99)])
+def test_sparse_residual_keeps_the_largest_entries(K, Ps):
+    """Exactly the K - ceil(Ps*K/100) largest |r| survive (continuous values:
+    no ties), checked against a sort."""
+    r = np.random.default_rng(K + Ps).laplace(0, 0.02, K)
+    keep, q, s = oracle.sparsify_residual(r, 32, Ps)
+    rank = -(-Ps * K // 100)
+    expect = np.zeros(K, np.uint8)
+    expect[np.argsort(np.abs(r), kind="stable")[rank:]] = 1
+    assert np.array_equal(keep, expect)
+    assert not q[keep == 0].any()
+
+
+def test_sparse_residual_ties_at_the_threshold_are_dropped():
+    """|r| sorted: 0.25 x8, 0.5 x8, 1.0 x32, 2.0 x8, 3.0 x8.  Ps = 50 puts the
+    rank (32) inside the run of 1.0s: theta = 1.0 and every 1.0 is dropped."""
+    r = np.array([0.5, -1.0, 1.0, 1.0, -1.0, 2.0, 3.0, -0.25] * 8)
+    keep, q, s = oracle.sparsify_residual(r, 32, 50)
+    assert np.array_equal(keep, (np.abs(r) > 1.0).astype(np.uint8)) and keep.sum() == 16
+
+
+def test_sparse_residual_codes_brute_force():
+    """Kept entries take the brute-force nearest code under s = (binary32)
+    (max kept |r| / 127); dropped ones 0; a group dropped whole gets s = 0."""
+    rng = np.random.default_rng(52)
+    r = rng.laplace(0, 0.02, 64)
+    r[:32] = np.sign(r[:32]) * (0.01 + np.abs(r[:32]))  # every |r| of group 0 exceeds 0.01
+    r[32:] *= 1e-3 / max(1.0, float(np.abs(r[32:]).max()) / 0.005)  # group 1 wholly below
+    keep, q, s = oracle.sparsify_residual(r, 32, 50)
+    assert not keep[32:].any() and s[1] == 0 and not q[32:].any()
+    a = max(abs(float(v)) for v, k in zip(r[:32], keep[:32]) if k)
+    assert s[0] == np.float32(a / 127.0)
+    for j in range(32):
+        assert q[j] == (_brute_code(Fraction(float(r[j])), F(s[0])) if keep[j] else 0)
+
+
+def test_sparse_residual_at_zero_percent_is_the_dense_quantizer():
+    r = np.random.default_rng(53).laplace(0, 0.02, 300)
+    keep, q, s = oracle.sparsify_residual(r, 128, 0)
+    q2, s2 = oracle.quantize_groups(r, 128)
+    assert keep.all() and np.array_equal(q, q2) and np.array_equal(s, s2)
+
+
+@pytest.mark.parametrize("Ps", [50, 70])
+def test_sparse_residual_sparsity_and_output(Ps):
+    """[P1] s3.3 quotes 50-70 % residual sparsity: on the stack's weights at
+    least that share of the codes is zero (a few more round to zero); the
+    output is the dense (trunk + sparse residual) weight times xhat."""
+    L = wl.config2_layer(0, 1)
+    W = L.weights()[:24]
+    x = L.activations(M=2)
+    idx = L.planted_channels()
+    d = oracle.decompose_sparse(W, Ps=Ps)
+    zero = float((d["q"] == 0).mean())
+    assert Ps / 100 <= zero <= Ps / 100 + 0.1, zero
+    xq, sx, xout = oracle.quantize_act(x, idx)
+    xh = _xhat(x, xq, sx, idx)
+    G = d["G"]
+    res_hat = d["s"].astype(np.float64)[:, np.arange(W.shape[1]) // G] * d["q"].astype(np.float64)
+    trunk_hat = d["mask"] * np.where(d["sign"] == 1, 1.0, -1.0) * d["alpha"].astype(np.float64)[:, None]
+    y = oracle.linear(d, xq, sx, xout, idx)
+    scale = np.abs(xh) @ (np.abs(res_hat) + np.abs(trunk_hat)).T
+    assert np.all(np.abs(y - xh @ (trunk_hat + res_hat).T) <= 1e-12 * scale)
+
+
 # ---- calibration and activations ----------------------------------------------
 
 def test_calibration_recovers_planted_channels():
