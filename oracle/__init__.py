@@ -68,11 +68,15 @@ def _load():
             lib.sqo_linear_naive.argtypes = lin
             lib.sqo_linear_trunk.argtypes = [i64, i64, i64, vp, vp, vp, vp, vp, vp, vp, i32, vp]
             lib.sqo_sparsify_residual.argtypes = [vp, i64, i32, i32, vp, vp, vp]
+            lib.sqo_quantize_groups_asym.argtypes = [vp, i64, i32, vp, vp, vp]
+            lib.sqo_linear_asym.argtypes = [i64, i64, i64, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                            vp, i32, vp]
             lib.sqo_abs_dot.argtypes = [i64, i64, i64, vp, vp, vp]
             for name in ("sqo_quantize_groups", "sqo_trunk_threshold", "sqo_decompose",
                          "sqo_calibrate", "sqo_quantize_act", "sqo_accumulate",
                          "sqo_trunk_popcount", "sqo_linear", "sqo_linear_naive", "sqo_linear_trunk",
-                         "sqo_sparsify_residual", "sqo_abs_dot"):
+                         "sqo_sparsify_residual", "sqo_quantize_groups_asym", "sqo_linear_asym",
+                         "sqo_abs_dot"):
                 getattr(lib, name).restype = i32
             _lib = lib
     return _lib
@@ -178,6 +182,45 @@ def decompose_sparse(W, G: int = 128, P: int = -1, Ps: int = 60):
         keep[r], q[r], s[r] = sparsify_residual(d["res"][r], G, Ps)
     d = dict(d, q=q, s=s, keep=keep)
     return d
+
+
+def quantize_groups_asym(r, G: int):
+    """One residual row, asymmetric INT8 per group: own min/max, scale and
+    zero-point ([P1] s2 pitfalls, [P3] asymmetric quantization).  q, s, z."""
+    r = _c(r, np.float64)
+    K = r.shape[0]
+    q = np.zeros(K, np.int8)
+    s = np.zeros(n_groups(K, G), np.float32)
+    z = np.zeros(n_groups(K, G), np.int32)
+    _ck(_load().sqo_quantize_groups_asym(_p(r), K, G, _p(q), _p(s), _p(z)), "quantize_groups_asym")
+    return q, s, z
+
+
+def decompose_asym(W, G: int = 128, P: int = -1):
+    """decompose() with asymmetric residual groups (keys as decompose, plus z)."""
+    d = decompose(W, G=G, P=P, want_residual=True)
+    N = d["res"].shape[0]
+    q, s = np.zeros_like(d["q"]), np.zeros_like(d["s"])
+    z = np.zeros(d["s"].shape, np.int32)
+    for r in range(N):
+        q[r], s[r], z[r] = quantize_groups_asym(d["res"][r], G)
+    return dict(d, q=q, s=s, z=z)
+
+
+def linear_asym(d, xq, sx, xout, idx):
+    """y = sx*(alpha*T + sum_g s_g*(R_g - z_g*S_g)) + sum_i What*xout (binary64)."""
+    xq = _c(xq, np.int8)
+    M, K = xq.shape
+    N = d["sign"].shape[0]
+    idx = _c(idx, np.int32)
+    n = idx.shape[0]
+    sx = _c(sx, np.float32)
+    xout = _c(xout, np.float32).reshape(M, n) if n else np.zeros((M, 1), np.float32)
+    y = np.zeros((M, N), np.float64)
+    _ck(_load().sqo_linear_asym(M, N, K, d["G"], _p(d["sign"]), _p(d["mask"]), _p(d["alpha"]),
+                                _p(d["q"]), _p(d["s"]), _p(_c(d["z"], np.int32)), _p(xq), _p(sx),
+                                _p(xout), _p(idx) if n else None, n, _p(y)), "linear_asym")
+    return y
 
 
 def calibrate(X, k: int) -> np.ndarray:

@@ -351,6 +351,79 @@ int sqo_linear(int64_t M, int64_t N, int64_t K, int G, const uint8_t *sign,
     return SQO_OK;
 }
 
+int sqo_quantize_groups_asym(const double *r, int64_t K, int G, int8_t *q, float *s,
+                             int32_t *z)
+{
+    if (!r || !q || !s || !z || K < 1 || !valid_group(G))
+        return SQO_BAD_ARG;
+    for (int64_t g = 0; g * G < K; ++g) {
+        int64_t j0 = g * G;
+        int64_t j1 = K < j0 + G ? K : j0 + G;
+        double lo = r[j0], hi = r[j0];
+        for (int64_t j = j0; j < j1; ++j) {
+            if (r[j] < lo)
+                lo = r[j];
+            if (r[j] > hi)
+                hi = r[j];
+        }
+        s[g] = (float)((hi - lo) / 255.0);
+        if (s[g] == 0.0f) {
+            z[g] = 0;
+            for (int64_t j = j0; j < j1; ++j)
+                q[j] = 0;
+            continue;
+        }
+        double sd = (double)s[g];
+        z[g] = (int32_t)round(-lo / sd - 128.0);
+        for (int64_t j = j0; j < j1; ++j) {
+            double v = round(r[j] / sd + (double)z[g]);
+            if (v > 127.0)
+                v = 127.0;
+            if (v < -128.0)
+                v = -128.0;
+            q[j] = (int8_t)v;
+        }
+    }
+    return SQO_OK;
+}
+
+int sqo_linear_asym(int64_t M, int64_t N, int64_t K, int G, const uint8_t *sign,
+                    const uint8_t *mask, const float *alpha, const int8_t *q, const float *s,
+                    const int32_t *z, const int8_t *xq, const float *sx, const float *xout,
+                    const int32_t *idx, int n_out, double *y)
+{
+    if (M < 1 || N < 1 || K < 1 || !valid_group(G) || !sign || !mask || !alpha || !q || !s ||
+        !z || !xq || !sx || !y || !check_idx(idx, n_out, K) || (n_out > 0 && !xout))
+        return SQO_BAD_ARG;
+    int64_t ng = n_groups(K, G);
+    for (int64_t t = 0; t < M; ++t)
+        for (int64_t r = 0; r < N; ++r) {
+            int64_t T = 0;
+            double inner = 0.0;
+            for (int64_t g = 0; g < ng; ++g) {
+                int64_t j0 = g * G, j1 = j0 + G < K ? j0 + G : K;
+                int64_t R = 0, S = 0;
+                for (int64_t j = j0; j < j1; ++j) {
+                    int64_t x = xq[t * K + j];
+                    if (mask[r * K + j])
+                        T += sign[r * K + j] ? x : -x;
+                    R += (int64_t)q[r * K + j] * x;
+                    S += x;
+                }
+                inner += (double)s[r * ng + g] * (double)(R - (int64_t)z[r * ng + g] * S);
+            }
+            double out = (double)sx[t] * ((double)alpha[r] * (double)T + inner);
+            for (int i = 0; i < n_out; ++i) {
+                int64_t j = idx[i], g = j / G;
+                double w = mask[r * K + j] ? (sign[r * K + j] ? (double)alpha[r] : -(double)alpha[r]) : 0.0;
+                w += (double)s[r * ng + g] * (double)((int64_t)q[r * K + j] - z[r * ng + g]);
+                out += w * (double)xout[t * n_out + i];
+            }
+            y[t * N + r] = out;
+        }
+    return SQO_OK;
+}
+
 static int cmp_double(const void *a, const void *b)
 {
     double x = *(const double *)a, y = *(const double *)b;

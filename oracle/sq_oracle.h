@@ -130,6 +130,25 @@ int sqo_linear(int64_t M, int64_t N, int64_t K, int G, const uint8_t *sign,
 int sqo_sparsify_residual(const double *r, int64_t K, int G, int Ps, uint8_t *keep,
                           int8_t *q, float *s);
 
+/* Asymmetric residual groups ([P1] section 2 pitfalls: the residual gets its
+ * own min/max, scale and zero-point; [P3] asymmetric quantization, divide
+ * form; INT8 range [-128, 127]).  Per group of G entries of r (binary64),
+ * beta = min, alpha = max:
+ *   s = (float)((alpha - beta) / 255)
+ *   z = round(-beta / s - 128)            (half away from zero; any int)
+ *   q = clip(round(r / s + z), -128, 127),  dequantized (q - z) * s;
+ * alpha == beta (a constant group) gives s = 0, z = 0, q = 0. */
+int sqo_quantize_groups_asym(const double *r, int64_t K, int G, int8_t *q, float *s,
+                             int32_t *z);
+
+/* Output with asymmetric residual groups:
+ *   y_tr = sx_t*(alpha_r*T_tr + sum_g s_rg*(R_trg - z_rg*S_tg)) + sum_i What_{r,idx_i}*xout_ti
+ * S_tg = sum_{j in g} xq_tj (exact), What_rj = trunk + s_{r,g(j)}*(q_rj - z_{r,g(j)}). */
+int sqo_linear_asym(int64_t M, int64_t N, int64_t K, int G, const uint8_t *sign,
+                    const uint8_t *mask, const float *alpha, const int8_t *q, const float *s,
+                    const int32_t *z, const int8_t *xq, const float *sx, const float *xout,
+                    const int32_t *idx, int n_out, double *y);
+
 /* Trunk-only output (m.lqnn.cn news 241359, section 3.3: the 1-bit trunk is
  * computed first and the residual added on demand; a request may skip the
  * residual path).  The residual arrays are not read:

@@ -59,6 +59,18 @@ MUTANTS = {
                                    "int64_t rank = ((int64_t)Ps * K) / 100 + 1;"),
     "sparse_quantizes_dropped_entries": ("kept[j] = keep[j] ? r[j] : 0.0;", "kept[j] = r[j];"),
     "sparse_theta_next_rank": ("theta = a[rank - 1];", "theta = a[rank < K ? rank : K - 1];"),
+    "asym_group_drops_last_channel": ("int64_t j1 = K < j0 + G ? K : j0 + G;",
+                                      "int64_t j1 = K < j0 + G ? K : j0 + G - 1;"),
+    "asym_zero_point_floor": ("z[g] = (int32_t)round(-lo / sd - 128.0);",
+                              "z[g] = (int32_t)floor(-lo / sd - 128.0);"),
+    "asym_zero_point_sign": ("z[g] = (int32_t)round(-lo / sd - 128.0);",
+                             "z[g] = (int32_t)round(lo / sd - 128.0);"),
+    "asym_range_254": ("s[g] = (float)((hi - lo) / 255.0);", "s[g] = (float)((hi - lo) / 254.0);"),
+    "asym_clip_minus_127": ("            if (v < -128.0)\n                v = -128.0;",
+                            "            if (v < -127.0)\n                v = -127.0;"),
+    "asym_linear_drops_zero_point": ("(double)(R - (int64_t)z[r * ng + g] * S);", "(double)R;"),
+    "asym_outlier_weight_drops_zero_point": ("(double)((int64_t)q[r * K + j] - z[r * ng + g]);",
+                                             "(double)q[r * K + j];"),
 }
 
 

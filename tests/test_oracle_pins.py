@@ -452,6 +452,91 @@ def test_sparse_residual_sparsity_and_output(Ps):
     assert np.all(np.abs(y - xh @ (trunk_hat + res_hat).T) <= 1e-12 * scale)
 
 
+# ---- asymmetric residual groups ([P1] s2 pitfalls, [P3] asymmetric quantization) --
+
+def _asym_groups(rng):
+    """Groups of 32: centred, all positive, all negative, skewed, with an exact 0."""
+    out = [rng.laplace(0, 0.02, 32), rng.uniform(0.1, 0.9, 32), -rng.uniform(0.1, 0.9, 32),
+           np.concatenate([rng.uniform(-0.01, 0, 8), rng.uniform(0, 1, 24)])]
+    g = rng.laplace(0, 0.02, 32)
+    g[7] = 0.0
+    out.append(g)
+    return out
+
+
+def test_asym_range_ends_and_zero_point():
+    """The group minimum and maximum land on -128 and 127; an exact 0.0 in a
+    group that straddles zero lands on the zero-point and dequantizes to 0."""
+    rng = np.random.default_rng(61)
+    for trial in range(40):
+        for g in _asym_groups(rng):
+            q, s, z = oracle.quantize_groups_asym(g, 32)
+            assert q[int(np.argmin(g))] == -128 and q[int(np.argmax(g))] == 127
+            for j in np.flatnonzero(g == 0.0):
+                if g.min() <= 0.0 <= g.max():
+                    assert q[j] == z[0] and (int(q[j]) - int(z[0])) * float(s[0]) == 0.0
+
+
+def test_asym_range_example():
+    """The pages' range [-7.59, 10.8]: s = (10.8 + 7.59) / 255, z = round(7.59/s - 128)
+    = -23 (exact rational arithmetic on the binary32 s)."""
+    r = np.zeros(32)
+    r[0], r[1] = -7.59, 10.8
+    q, s, z = oracle.quantize_groups_asym(r, 32)
+    assert s[0] == np.float32((10.8 + 7.59) / 255.0)
+    t = Fraction(7.59) / F(s[0]) - 128  # = -22.76...
+    assert z[0] == -23 and abs(t - z[0]) < Fraction(1, 2)
+    assert q[0] == -128 and q[1] == 127
+
+
+def test_asym_codes_are_nearest_levels():
+    """Each code is a nearest of the 256 levels (q - z) * s (brute force over
+    rationals), and a constant group gives s = 0, z = 0, q = 0."""
+    rng = np.random.default_rng(62)
+    for g in _asym_groups(rng):
+        q, s, z = oracle.quantize_groups_asym(g, 32)
+        S, Z = F(s[0]), int(z[0])
+        for v, c in zip(g, q):
+            R = Fraction(float(v))
+            best = min(abs(R - (k - Z) * S) for k in range(-128, 128))
+            assert abs(R - (int(c) - Z) * S) == best
+    q, s, z = oracle.quantize_groups_asym(np.full(32, 0.37), 32)
+    assert s[0] == 0 and z[0] == 0 and not q.any()
+
+
+def test_asym_halves_the_error_on_a_skewed_group():
+    """[P3]: the asymmetric form fits a one-sided group better; on values in
+    [0, 1] its step is (max - min)/255 against max/127."""
+    g = np.random.default_rng(63).uniform(0, 1, 128)
+    qa, sa, za = oracle.quantize_groups_asym(g, 128)
+    qs, ss = oracle.quantize_groups(g, 128)
+    ea = np.abs(g - (qa.astype(np.float64) - za[0]) * sa[0]).max()
+    es = np.abs(g - qs.astype(np.float64) * ss[0]).max()
+    assert ea <= 0.55 * es
+
+
+@pytest.mark.parametrize("P", [-1, 60])
+def test_asym_linear_is_the_dense_product(P):
+    """y = sx*(alpha*T + sum_g s_g*(R_g - z_g*S_g)) + outliers equals the dense
+    (trunk + (q - z)*s) weight times xhat, formed with numpy."""
+    L = wl.config2_layer(0, 1)
+    W = L.weights()[:24]
+    x = L.activations(M=2)
+    idx = L.planted_channels()
+    d = oracle.decompose_asym(W, P=P)
+    xq, sx, xout = oracle.quantize_act(x, idx)
+    xh = _xhat(x, xq, sx, idx)
+    g = np.arange(W.shape[1]) // d["G"]
+    res_hat = d["s"].astype(np.float64)[:, g] * (d["q"].astype(np.float64) - d["z"][:, g])
+    trunk_hat = d["mask"] * np.where(d["sign"] == 1, 1.0, -1.0) * d["alpha"].astype(np.float64)[:, None]
+    y = oracle.linear_asym(d, xq, sx, xout, idx)
+    scale = np.abs(xh) @ (np.abs(res_hat) + np.abs(trunk_hat)).T
+    assert np.all(np.abs(y - xh @ (trunk_hat + res_hat).T) <= 1e-12 * scale)
+    # and it stays within the symmetric residual's accuracy of the original product
+    ref = x.astype(np.float64) @ W.astype(np.float64).T
+    assert np.all(np.abs(y - ref) <= 0.05 * oracle.abs_dot(W, x))
+
+
 # ---- calibration and activations ----------------------------------------------
 
 def test_calibration_recovers_planted_channels():
