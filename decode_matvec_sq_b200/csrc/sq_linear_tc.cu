@@ -161,13 +161,17 @@ struct Cursor {
 // They bypass L1.  A lane copies its own sign, mask and scale words, through
 // L1, where neighbouring lanes' requests coalesce (16-byte copies that bypass
 // L1 measured slower for these).
-template <bool MASK>
+// In the trunk-only mode (RES = false) a slot holds only the 256 sign bytes
+// (then the 256 mask bytes), and the ring is kTrunkDepth slots deep.
+template <bool MASK, bool RES = true>
 struct Slot {
-  static constexpr int kSign = 2048;
+  static constexpr int kSign = RES ? 2048 : 0;
   static constexpr int kMask = kSign + 256;  // (MASK only)
-  static constexpr int kScale = MASK ? kMask + 256 : kMask;
-  static constexpr int kBytes = MASK ? 2816 : 2560;
+  static constexpr int kScale = MASK ? kMask + 256 : kMask;  // (RES only)
+  static constexpr int kBytes = kScale + (RES ? 256 : 0);
 };
+// Tiles in flight per warp in the trunk-only mode (small slots).
+constexpr int kTrunkDepth = 6;
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
@@ -197,11 +201,11 @@ __device__ __forceinline__ void copy_tile(uint32_t slot, const Cursor& c, int la
       cp_async16(slot + lo * 64 + (((ch + (lo >> 1)) & 3) << 4), c.code + 512 * j);
     }
   }
-  cp_async8(slot + Slot<MASK>::kSign + lane * 8, c.sign);
-  if constexpr (MASK) cp_async8(slot + Slot<MASK>::kMask + lane * 8, c.mask);
+  cp_async8(slot + Slot<MASK, RES>::kSign + lane * 8, c.sign);
+  if constexpr (MASK) cp_async8(slot + Slot<MASK, RES>::kMask + lane * 8, c.mask);
   if constexpr (RES) {
-    cp_async4(slot + Slot<MASK>::kScale + lane * 8, c.scale);
-    cp_async4(slot + Slot<MASK>::kScale + lane * 8 + 4, c.scale + 8);
+    cp_async4(slot + Slot<MASK, RES>::kScale + lane * 8, c.scale);
+    cp_async4(slot + Slot<MASK, RES>::kScale + lane * 8 + 4, c.scale + 8);
   }
 }
 
@@ -218,16 +222,16 @@ __device__ __forceinline__ void read_tile(Tile<MASK>& t, const uint8_t* slot, in
       t.q[4 * j + 3] = v.w;
     }
   }
-  const uint2 sv = *reinterpret_cast<const uint2*>(slot + Slot<MASK>::kSign + lane * 8);
+  const uint2 sv = *reinterpret_cast<const uint2*>(slot + Slot<MASK, RES>::kSign + lane * 8);
   t.s[0] = sv.x;
   t.s[1] = sv.y;
   if constexpr (MASK) {
-    const uint2 mv = *reinterpret_cast<const uint2*>(slot + Slot<MASK>::kMask + lane * 8);
+    const uint2 mv = *reinterpret_cast<const uint2*>(slot + Slot<MASK, RES>::kMask + lane * 8);
     t.m[0] = mv.x;
     t.m[1] = mv.y;
   }
   if constexpr (RES) {
-    const float2 cv = *reinterpret_cast<const float2*>(slot + Slot<MASK>::kScale + lane * 8);
+    const float2 cv = *reinterpret_cast<const float2*>(slot + Slot<MASK, RES>::kScale + lane * 8);
     t.c[0] = cv.x;
     t.c[1] = cv.y;
   }
@@ -468,12 +472,12 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
     cur.mask = MASK ? p.mask + lt * 2 : p.sign;
     cur.scale = p.scale + (int64_t)t0 * 16 + gid;
   }
-  uint8_t* ring_w = smem + p.off_ring + warp * D * Slot<MASK>::kBytes;
+  uint8_t* ring_w = smem + p.off_ring + warp * D * Slot<MASK, RES>::kBytes;
   const uint32_t ring_u = smem_u32(ring_w);
   constexpr int kEarly = FUSED ? kDepthEarly : D;
 #pragma unroll
   for (int d = 0; d < kEarly; ++d) {  // one commit group per tile, empty past the range
-    if (t0 + d < t1) copy_tile<MASK, RES>(ring_u + d * Slot<MASK>::kBytes, cur, lane);
+    if (t0 + d < t1) copy_tile<MASK, RES>(ring_u + d * Slot<MASK, RES>::kBytes, cur, lane);
     cp_async_commit();
     cur.advance();
   }
@@ -507,7 +511,7 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
     split_activations(p, omask, xq_s, xo_s, sx_s, reinterpret_cast<float*>(smem + p.off_red), jv, jp);
 #pragma unroll
     for (int d = kEarly; d < D; ++d) {
-      if (t0 + d < t1) copy_tile<MASK, RES>(ring_u + d * Slot<MASK>::kBytes, cur, lane);
+      if (t0 + d < t1) copy_tile<MASK, RES>(ring_u + d * Slot<MASK, RES>::kBytes, cur, lane);
       cp_async_commit();
       cur.advance();
     }
@@ -543,7 +547,7 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
     cp_async_wait<D - 1>();  // this lane's copies of the tile have landed
     __syncwarp();             // ... and every lane's
     Tile<MASK> tl;
-    read_tile<MASK, RES>(tl, ring_w + slot_i * Slot<MASK>::kBytes, lane);
+    read_tile<MASK, RES>(tl, ring_w + slot_i * Slot<MASK, RES>::kBytes, lane);
     // activation codes of this lane's 32 channels for its MMA column
     uint32_t xw[8];
     {
@@ -650,7 +654,7 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
 
     // refill this slot with the tile D ahead, once no lane reads it
     __syncwarp();
-    if (t + D < t1) copy_tile<MASK, RES>(ring_u + slot_i * Slot<MASK>::kBytes, cur, lane);
+    if (t + D < t1) copy_tile<MASK, RES>(ring_u + slot_i * Slot<MASK, RES>::kBytes, cur, lane);
     cp_async_commit();
     cur.advance();
     if (++slot_i == D) slot_i = 0;
@@ -744,7 +748,7 @@ template <bool MASK, bool FUSED, int D>
 cudaError_t launch_plain(const Params& p, bool res, int grid, int smem, bool pdl,
                          cudaStream_t stream) {
   return res ? launch_one<MASK, false, FUSED, D, true>(p, grid, smem, pdl, stream)
-             : launch_one<MASK, false, FUSED, D, false>(p, grid, smem, pdl, stream);
+             : launch_one<MASK, false, FUSED, kTrunkDepth, false>(p, grid, smem, pdl, stream);
 }
 
 // Non-accumulator launch with a ring depth chosen at run time among Ds.
@@ -782,6 +786,9 @@ int fused_token_bytes(const sq_packed_weight& w, int n_out) {
 }
 int ring_bytes(bool mask, int depth) {
   return kWarps * depth * (mask ? Slot<true>::kBytes : Slot<false>::kBytes);
+}
+int trunk_ring_bytes(bool mask) {
+  return kWarps * kTrunkDepth * (mask ? Slot<true, false>::kBytes : Slot<false, false>::kBytes);
 }
 }  // namespace
 
@@ -854,7 +861,7 @@ cudaError_t launch_linear_tc(const sq_packed_weight& w, int M, const int8_t* xq,
   // three tiles per warp above batch 2 where they fit, else two (the
   // accumulator mode, used to check the kernel, always takes two)
   const int depth = (!emit && M > 2 && smem + ring_bytes(mask, kDeep) <= kSmemMax) ? kDeep : kShallow;
-  smem += ring_bytes(mask, depth);
+  smem += trunk_only ? trunk_ring_bytes(mask) : ring_bytes(mask, depth);
   if (smem > kSmemMax) return cudaErrorInvalidValue;
   const int grid = (int)blocks;
   if (emit)
