@@ -163,3 +163,30 @@ def test_fused_tokens_per_pass(L):
     assert L.sq_quantize_linear_tokens_per_pass(ctypes.byref(view(64, 4096, layout=0)), 20) == 0
     assert L.sq_quantize_linear_tokens_per_pass(ctypes.byref(view(64, 4096)), -1) == 0
     assert L.sq_quantize_linear_tokens_per_pass(None, 0) == 0
+
+
+def test_missing_library_fails_loudly():
+    """Without the built CUDA library every entry point raises: there is no
+    CPU fallback.  Run in a child process so this process keeps its loaded
+    library."""
+    import subprocess
+    import sys
+    code = ("import decode_matvec_sq_b200 as sq\n"
+            "sq.LIB_PATH = '/nonexistent/libsq.so'\n"
+            "sq._lib = None\n"
+            "try:\n"
+            "    sq.packed_bytes(64, 256)\n"
+            "except ImportError as e:\n"
+            "    print('raised', 'missing' in str(e))\n")
+    r = subprocess.run([sys.executable, "-c", code], cwd=os.path.dirname(os.path.dirname(__file__)),
+                       capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0 and r.stdout.strip() == "raised True", r.stdout + r.stderr
+
+
+def test_device_entry_points_refuse_without_a_device(L):
+    """On a machine with no usable sm_100 device the device check fails with
+    a status, not a silent fallback (this CPU machine has none)."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a device is visible")
+    assert L.sq_device_check() != 0
