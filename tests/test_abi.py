@@ -190,3 +190,40 @@ def test_device_entry_points_refuse_without_a_device(L):
     if torch.cuda.is_available():
         pytest.skip("a device is visible")
     assert L.sq_device_check() != 0
+
+
+C_PROGRAM = r"""
+#include <stdio.h>
+#include "sq.h"
+int main(void) {
+  sq_packed_weight v;
+  size_t b = sq_packed_bytes(64, 256, 128, 0, SQ_LAYOUT_TILES);
+  int rc = sq_packed_view((void *)(1ull << 40), 64, 256, 128, 0, SQ_LAYOUT_TILES, &v);
+  int bad = sq_linear(NULL, NULL, NULL, NULL, NULL, 0, 1, NULL, NULL, 0, NULL, 0u, NULL);
+  printf("%zu %d %d %d %s\n", b, rc, v.layout, bad, sq_status_string(SQ_ERR_INVALID_ARG));
+  return 0;
+}
+"""
+
+
+def test_header_is_plain_c_and_links(tmp_path):
+    """include/sq.h compiles as pedantic C11 with warnings as errors, and a C
+    host program links against libsq.so and makes host-only calls."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc not available")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    src = tmp_path / "t.c"
+    src.write_text(C_PROGRAM)
+    exe = tmp_path / "t"
+    libdir = os.path.dirname(sq.LIB_PATH)
+    subprocess.run(["gcc", "-std=c11", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                    "-I" + os.path.join(root, "include"), str(src), "-L" + libdir, "-lsq",
+                    "-Wl,-rpath," + libdir, "-o", str(exe)], check=True, capture_output=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
+    assert int(out[0]) == L_bytes() and out[1] == "0" and out[2] == "1" and out[3] == "1"
+
+
+def L_bytes() -> int:
+    return sq.packed_bytes(64, 256, 128, False, sq.SQ_LAYOUT_TILES)
