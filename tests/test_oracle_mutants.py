@@ -71,6 +71,11 @@ MUTANTS = {
     "asym_linear_drops_zero_point": ("(double)(R - (int64_t)z[r * ng + g] * S);", "(double)R;"),
     "asym_outlier_weight_drops_zero_point": ("(double)((int64_t)q[r * K + j] - z[r * ng + g]);",
                                              "(double)q[r * K + j];"),
+    "abs_dot_drops_fabs": ("acc += fabs((double)W[r * K + j] * (double)x[t * K + j]);",
+                           "acc += (double)W[r * K + j] * (double)x[t * K + j];"),
+    "abs_dot_doubles_term": ("acc += fabs((double)W[r * K + j] * (double)x[t * K + j]);",
+                             "acc += 2.0 * fabs((double)W[r * K + j] * (double)x[t * K + j]);"),
+    "abs_dot_transposes_output": ("out[t * N + r] = acc;", "out[r * M + t] = acc;"),
 }
 
 

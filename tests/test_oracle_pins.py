@@ -581,6 +581,38 @@ def test_nonfinite_and_bad_arguments():
         oracle.decompose(np.ones((1, 8), np.float32), G=48)
 
 
+# ---- tolerance scale ------------------------------------------------------------
+
+def test_abs_dot_closed_form():
+    """sum_j |W_rj x_tj| on weights +-c and activations +-d with random signs
+    is K*c*d exactly (every product and partial sum is exact in binary64)."""
+    rng = np.random.default_rng(11)
+    K, c, d = 37, 0.75, 1.5
+    W = (c * rng.choice([-1.0, 1.0], size=(5, K))).astype(np.float32)
+    x = (d * rng.choice([-1.0, 1.0], size=(3, K))).astype(np.float32)
+    out = oracle.abs_dot(W, x)
+    assert out.shape == (3, 5)
+    assert np.all(out == K * c * d)
+
+
+def test_abs_dot_hand_computed():
+    """A 2 x 3 weight and two tokens, summed by hand: [[6, 4.5], [5.5, 5]]."""
+    W = np.array([[1.0, -2.0, 3.0], [0.5, 0.0, -4.0]], np.float32)
+    x = np.array([[1.0, 1.0, 1.0], [-2.0, 0.25, 1.0]], np.float32)
+    assert np.array_equal(oracle.abs_dot(W, x), np.array([[6.0, 4.5], [5.5, 5.0]]))
+
+
+def test_abs_dot_matches_absolute_matrix_product():
+    """Second route: the product of the element-wise absolute values (numpy,
+    binary64) on the stack's weights and activations, to 1e-12 relative."""
+    L = wl.config2_layer(0, 1)
+    W = L.weights(rows=np.arange(24))
+    x = L.activations(M=2)
+    ref = np.abs(x.astype(np.float64)) @ np.abs(W.astype(np.float64)).T
+    got = oracle.abs_dot(W, x)
+    assert np.allclose(got, ref, rtol=1e-12, atol=0.0)
+
+
 def test_generator_statistics():
     """The synthetic inputs have the stated distributions (sanity, not a pin)."""
     W = wl.config1().weights()
