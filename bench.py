@@ -60,6 +60,11 @@ def quantize_bytes(L, M=1) -> int:
     return M * (4 * L.K + L.K + 4 + 4 * L.n_out) + 4 * L.n_out
 
 
+def fused_launch_bytes(L, M=1) -> int:
+    """One launch of the fused kernel: packed weights, x and idx in, y out."""
+    return L.packed_bytes + M * (4 * L.K + 4 * L.N) + 4 * L.n_out
+
+
 def step_bytes(layers, M=1) -> int:
     return sum(linear_weight_bytes(L) + linear_act_bytes(L, M) + quantize_bytes(L, M) for L in layers)
 
@@ -199,7 +204,7 @@ def oracle_sample(rows: int = 256, layers_idx=(0,)):
             n = min(rows, L.N)
             W = L.weights(rows=np.arange(n))
             d = oracle.decompose(W)
-            sample.append((L, n, d, L.activations(), L.planted_channels()))
+            sample.append((L, n, d, L.activations(), L.planted_channels(), W))
     return sample
 
 
@@ -209,7 +214,7 @@ def time_oracle(sample, min_seconds: float | None = None, passes: int | None = N
     import oracle
     done, t0 = 0, time.perf_counter()
     while True:
-        for L, n, d, x, idx in sample:
+        for L, n, d, x, idx, _ in sample:
             xq, sx, xo = oracle.quantize_act(x, idx)
             oracle.linear(d, xq, sx, xo, idx)
         done += 1
@@ -220,10 +225,27 @@ def time_oracle(sample, min_seconds: float | None = None, passes: int | None = N
             break
     per_pass = el / done
     nbytes = 0
-    for L, n, d, x, idx in sample:
+    for L, n, d, x, idx, _ in sample:
         Ls = L.with_(N=n)
         nbytes += linear_weight_bytes(Ls) + linear_act_bytes(Ls) + quantize_bytes(Ls)
     return nbytes / per_pass / 1e9, per_pass, done, nbytes
+
+
+def oracle_parity(sample, ys):
+    """The oracle's y for the sampled rows against the GPU's y of the same
+    linears (ys[i] [1][N], device): max |y - y_ref| / sum_j |W_rj x_j| and
+    whether it is within the 1e-5 tolerance."""
+    import numpy as np
+    import oracle
+    worst, rows = 0.0, 0
+    for (L, n, d, x, idx, W), y in zip(sample, ys):
+        xq, sx, xo = oracle.quantize_act(x, idx)
+        ref = oracle.linear(d, xq, sx, xo, idx)
+        bound = oracle.abs_dot(W, x)
+        got = y[:, :n].cpu().numpy().astype(np.float64)
+        worst = max(worst, float((np.abs(got - ref) / np.maximum(bound, 1e-300)).max()))
+        rows += n
+    return {"rows": rows, "max_err_over_bound": worst, "tolerance": 1e-5, "ok": worst <= 1e-5}
 
 
 def run_reference(args, world, rank):
@@ -339,57 +361,6 @@ class Stack:
             self.step()
         torch.cuda.synchronize()
         return g
-
-    def time_linear_launches(self, reps: int):
-        """Average device duration of the linear-layer kernel per shape: for each
-        shape, a CUDA graph of its launches over all layers (different weights,
-        no PDL), replayed `reps` times between events on the replay stream."""
-        import torch
-        import decode_matvec_sq_b200 as sq
-        groups = {}
-        for i, L in enumerate(self.layers):
-            groups.setdefault(L.name.split(".")[-1], []).append(i)
-        s = torch.cuda.Stream()
-        per_shape = {}
-        tot_ms, tot_bytes = 0.0, 0
-        for key, ids in groups.items():
-            def launch():
-                for i in ids:
-                    if self.fused:
-                        sq.quantize_linear(self.pws[i], self.xs[i], self.idx[i], y=self.ys[i],
-                                           workspace=self.ws, status=self.status)
-                    else:
-                        a = self.bufs[i]
-                        sq.linear(self.pws[i], a[0], a[1], a[2], self.idx[i], y=self.ys[i],
-                                  workspace=self.ws, status=self.status)
-            s.wait_stream(torch.cuda.current_stream())
-            with torch.cuda.stream(s):
-                launch()
-            torch.cuda.synchronize()
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=s):
-                launch()
-            with torch.cuda.stream(s):
-                g.replay()
-                a = torch.cuda.Event(enable_timing=True)
-                b = torch.cuda.Event(enable_timing=True)
-                a.record(s)
-                for _ in range(reps):
-                    g.replay()
-                b.record(s)
-            torch.cuda.synchronize()
-            ms = a.elapsed_time(b)
-            n = reps * len(ids)
-            nbytes = sum(linear_weight_bytes(self.layers[i]) + linear_act_bytes(self.layers[i])
-                         for i in ids) * reps
-            per_shape[key] = [ms, n, nbytes]
-            tot_ms += ms
-            tot_bytes += nbytes
-            del g
-        shapes = {k: {"us": round(v[0] / v[1] * 1e3, 2),
-                      "gbs": round(v[2] / (v[0] * 1e-3) / 1e9, 1)} for k, v in per_shape.items()}
-        n_launch = sum(v[1] for v in per_shape.values())
-        return tot_bytes / n_launch, tot_ms / n_launch, shapes
 
 
 def run_prefill(args, world, rank, local):
@@ -560,6 +531,119 @@ def _fused_launches(pw, M: int, L) -> int:
     return 1 + -(-M // 8) if staged else -(-M // per_pass)
 
 
+def time_layer_case(L, M, copies, trunk, st, device, warmup, reps):
+    """Device ms per sq_quantize_linear call of layer L at M tokens, as a CUDA
+    graph of calls rotating over `copies` copies of the packed weight (enough
+    copies that every call reads its weight from HBM, unless one), and the
+    call's algorithmic bytes, launches per call and calls per graph."""
+    import torch
+    import decode_matvec_sq_b200 as sq
+    import synth.device as sdev
+    W = sdev.fill_weights(L, torch.empty(L.N, L.K, device=device))
+    pw = sq.decompose_pack(W, trunk_percent=L.trunk_percent, status=st)
+    del W
+    pws = [pw]
+    for _ in range(copies - 1):
+        c = sq.alloc_packed(L.N, L.K, 128, pw.with_mask, pw.layout, device=device)
+        c.buf.copy_(pw.buf)
+        pws.append(c)
+    idx = torch.from_numpy(L.planted_channels()).to(device)
+    x = sdev.fill_activations(L, torch.empty(M, L.K, device=device))
+    y = torch.empty(M, L.N, device=device)
+    ws = sq.new_fused_workspace(pw, M, L.n_out)
+    calls = max(copies, 20)
+
+    def launch():
+        for r in range(calls):
+            sq.quantize_linear(pws[r % copies], x, idx, y=y, workspace=ws, status=st,
+                               trunk_only=trunk)
+
+    for _ in range(warmup):
+        launch()
+    ms = _time_calls(launch, reps) / calls
+    wbytes = trunk_weight_bytes(L) if trunk else linear_weight_bytes(L)
+    nbytes = wbytes + M * (4 * L.K + 4 * L.N) + 4 * L.n_out
+    launches = _fused_launches(pw, M, L)
+    del pws, pw, ws
+    torch.cuda.empty_cache()
+    return ms, nbytes, launches, calls
+
+
+def time_prefill_case(st, device, warmup, steps):
+    """The prefill workload (2048 tokens x 4096 -> 14336, row layout): device
+    ms of the activation split + linear step and of the linear alone, with a
+    256 MB buffer written between steps (cold L2)."""
+    import torch
+    import decode_matvec_sq_b200 as sq
+    import synth.device as sdev
+    from synth import workloads as wl
+    L = wl.config5()
+    W = sdev.fill_weights(L, torch.empty(L.N, L.K, device=device))
+    pw = sq.decompose_pack(W, layout=sq.SQ_LAYOUT_ROWS, status=st)
+    del W
+    x = sdev.fill_activations(L, torch.empty(L.M, L.K, device=device))
+    idx = torch.from_numpy(L.planted_channels()).to(device)
+    xq, sx, xo = sq.quantize_act(x, idx, status=st)
+    y = torch.empty(L.M, L.N, device=device)
+    ws = sq.new_workspace(pw, L.M)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        sq.quantize_act(x, idx, xq=xq, sx=sx, x_out=xo, status=st)
+        sq.linear(pw, xq, sx, xo, idx, y=y, workspace=ws, status=st)
+    torch.cuda.synchronize()
+    ev = []
+    for _ in range(steps):
+        flush.fill_(1)
+        a, b, c = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        a.record(stream)
+        sq.quantize_act(x, idx, xq=xq, sx=sx, x_out=xo, status=st)
+        b.record(stream)
+        sq.linear(pw, xq, sx, xo, idx, y=y, workspace=ws, status=st)
+        c.record(stream)
+        ev.append((a, b, c))
+    torch.cuda.synchronize()
+    ms_step = sum(a.elapsed_time(c) for a, b, c in ev) / len(ev)
+    ms_lin = sum(b.elapsed_time(c) for a, b, c in ev) / len(ev)
+    del pw, ws, flush, x, xq, y
+    torch.cuda.empty_cache()
+    return ms_step, ms_lin, 4 * L.M * L.N * L.K
+
+
+def side_configs(device, warmup=3, reps=10):
+    """Compact measurements of the other workloads, outside the headline's
+    timed region: the 512 x 512 layer (hot and cold), the 70B-shaped MLP pair
+    at batch 1..16, the threshold-trunk layer and the prefill workload."""
+    import torch
+    st = torch.zeros(1, dtype=torch.int32, device=device)
+    out = {}
+    single = {}
+    for label, L, M, copies in layer_cases("single"):
+        ms, nbytes, _, _ = time_layer_case(L, M, copies, False, st, device, warmup, reps)
+        single["us_hot" if copies == 1 else "us_cold"] = round(ms * 1e3, 2)
+    out["single_512x512_batch1"] = single
+    mlp = {}
+    for label, L, M, copies in layer_cases("mlp70b"):
+        ms, nbytes, _, _ = time_layer_case(L, M, copies, False, st, device, warmup, reps)
+        mlp.setdefault(f"M={M}", {})[f"{L.K}->{L.N}"] = {"us": round(ms * 1e3, 2),
+                                                           "gbs": round(nbytes / (ms * 1e-3) / 1e9, 1)}
+    out["mlp70b_batch_sweep"] = mlp
+    for label, L, M, copies in layer_cases("threshold"):
+        ms, nbytes, _, _ = time_layer_case(L, M, copies, False, st, device, warmup, reps)
+        out["threshold_4096x14336_batch1"] = {"us": round(ms * 1e3, 2),
+                                              "gbs": round(nbytes / (ms * 1e-3) / 1e9, 1)}
+    ms_step, ms_lin, ops = time_prefill_case(st, device, warmup, reps)
+    peak, kind = load_int8_peak()
+    out["prefill_2048x4096x14336"] = {"us_step": round(ms_step * 1e3, 1),
+                                       "us_linear": round(ms_lin * 1e3, 1),
+                                       "t_intops_linear": round(ops / (ms_lin * 1e-3) / 1e12, 1),
+                                       "frac_of_int8_peak": round(ops / (ms_lin * 1e-3) / 1e12 / peak, 4),
+                                       "int8_peak_kind": kind}
+    if st.item() != 0:
+        raise RuntimeError(f"side configurations: device status {st.item()}")
+    return out
+
+
 def run_layers(args, world, rank, local):
     """Single-layer workloads beside the stack: the 512 x 512 layer (hot and
     cold), the 70B-shaped MLP pair at batch 1..16 and the threshold-trunk layer.
@@ -570,7 +654,6 @@ def run_layers(args, world, rank, local):
     import torch
     import decode_matvec_sq_b200 as sq
     from decode_matvec_sq_b200 import build
-    import synth.device as sdev
 
     if not torch.cuda.is_available():
         raise SystemExit("bench.py: no CUDA device visible (the sq path has no CPU fallback)")
@@ -589,41 +672,16 @@ def run_layers(args, world, rank, local):
     tot_ms, tot_bytes, tot_launch = 0.0, 0, 0
     with ClockSampler(local) as clk:
         for label, L, M, copies in layer_cases(args.workload):
-            W = sdev.fill_weights(L, torch.empty(L.N, L.K, device=device))
-            pw = sq.decompose_pack(W, trunk_percent=L.trunk_percent, status=st)
-            del W
-            pws = [pw]
-            for _ in range(copies - 1):
-                c = sq.alloc_packed(L.N, L.K, 128, pw.with_mask, pw.layout, device=device)
-                c.buf.copy_(pw.buf)
-                pws.append(c)
-            idx = torch.from_numpy(L.planted_channels()).to(device)
-            x = sdev.fill_activations(L, torch.empty(M, L.K, device=device))
-            y = torch.empty(M, L.N, device=device)
-            ws = sq.new_fused_workspace(pw, M, L.n_out)
-            calls = max(copies, 20)
-
             trunk = args.workload == "trunk"
-
-            def launch():
-                for r in range(calls):
-                    sq.quantize_linear(pws[r % copies], x, idx, y=y, workspace=ws, status=st,
-                                       trunk_only=trunk)
-
-            for _ in range(args.warmup):
-                launch()
             barrier(world)
-            ms = max_over_ranks(_time_calls(launch, max(1, args.steps)) / calls, world, device)
-            wbytes = trunk_weight_bytes(L) if trunk else linear_weight_bytes(L)
-            nbytes = wbytes + M * (4 * L.K + 4 * L.N) + 4 * L.n_out
-            launches = _fused_launches(pw, M, L)
+            ms, nbytes, launches, calls = time_layer_case(L, M, copies, trunk, st, device,
+                                                          args.warmup, max(1, args.steps))
+            ms = max_over_ranks(ms, world, device)
             cases.append({"case": label, "M": M, "us": round(ms * 1e3, 2),
                           "gbs": round(nbytes / (ms * 1e-3) / 1e9, 1), "launches_per_call": launches})
             tot_ms += ms
             tot_bytes += nbytes
             tot_launch += max(1, args.steps) * calls * launches  # inside the timed replays
-            del pws, pw, ws
-            torch.cuda.empty_cache()
     clocks = clk.summary()
     if st.item() != 0:
         raise RuntimeError(f"device status {sq.STATUS.get(st.item())}")
@@ -709,10 +767,22 @@ def run_gpu(args, world, rank, local):
     if stack.status.item() != 0:
         raise RuntimeError(f"device status {sq.STATUS.get(stack.status.item())}")
 
-    # ---- roofline of the dominant kernel: per-launch durations ------------------
-    bytes_launch, ms_launch, shapes = stack.time_linear_launches(max(1, args.steps))
+    # ---- roofline of the dominant kernel ---------------------------------------
+    # Every launch of the timed graph is the decode kernel (fused: activation
+    # split + linear; two-kernel mode: the linear, with the split beside it),
+    # so its average duration inside the timed step is the step time divided
+    # by the launches; the algorithmic bytes per launch are its own reads and
+    # writes.
     peak, peak_kind = load_peaks()
-    achieved = bytes_launch / (ms_launch * 1e-3) / 1e9
+    if stack.fused:
+        kbytes = sum(fused_launch_bytes(L) for L in layers)
+        n_kernel = len(layers)
+    else:
+        kbytes = sum(linear_weight_bytes(L) + linear_act_bytes(L) + quantize_bytes(L) for L in layers)
+        n_kernel = 2 * len(layers)
+    bytes_launch = kbytes / len(layers)
+    ms_launch = ms_step / n_kernel
+    achieved = kbytes / (ms_step * 1e-3) / 1e9
     traffic = None
     tpath = os.path.join(ROOT, "profiles", "linear_traffic.json")
     if os.path.exists(tpath):
@@ -723,6 +793,8 @@ def run_gpu(args, world, rank, local):
                 traffic = tr.get("dram_bytes_per_launch_stack_avg")
         except Exception:
             traffic = None
+
+    y_checked = [y.clone() for y in stack.ys[:4]]  # layer 0's outputs of the timed steps
 
     # ---- end to end through host buffers ---------------------------------------
     e2e = None
@@ -753,7 +825,7 @@ def run_gpu(args, world, rank, local):
                "h2d_bytes_per_step": int(stack.x_all.numel() * 4),
                "d2h_bytes_per_step": int(stack.y_all.numel() * 4)}
 
-    cpu = None
+    cpu, parity = None, None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         sample = oracle_sample(rows=args.oracle_rows)
         gbs, per_pass, passes, sbytes = time_oracle(sample, min_seconds=args.oracle_seconds)
@@ -761,6 +833,12 @@ def run_gpu(args, world, rank, local):
                "sample": f"first {args.oracle_rows} rows of each linear of layer 0 "
                          f"({sbytes / 1e6:.1f} MB per pass, {passes} passes, "
                          f"{per_pass * 1e3:.1f} ms per pass), quantize_act + linear"}
+        # the oracle's outputs for that sample against the timed graph's y
+        parity = oracle_parity(sample, y_checked[:len(sample)])
+
+    side = None
+    if rank == 0 and not args.no_side_configs:
+        side = side_configs(device)
 
     if rank == 0:
         line = {
@@ -778,10 +856,13 @@ def run_gpu(args, world, rank, local):
                          "kernel": "k_linear_tc (activation split + decode linear, tensor cores)"
                                    if stack.fused else "k_linear_tc (decode linear, tensor cores)",
                          "bytes_per_launch": int(bytes_launch),
-                         "us_per_launch": round(ms_launch * 1e3, 3), "per_shape": shapes},
+                         "us_per_launch": round(ms_launch * 1e3, 3),
+                         "timing": "timed PDL graph: step time / launches per step"},
             "clocks": clocks,
             "e2e": e2e,
             "cpu_baseline": cpu,
+            "parity_check": parity,
+            "other_workloads": side,
         }
         print(json.dumps(line), flush=True)
     del graph
@@ -820,6 +901,9 @@ def main(argv=None):
                     help="activation split and linear layer as two kernels per linear")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-side-configs", action="store_true",
+                    help="skip the compact measurements of the other workloads (512x512, "
+                         "70B-shaped MLP batch sweep, threshold trunk, prefill)")
     ap.add_argument("--oracle-rows", type=int, default=256)
     ap.add_argument("--oracle-seconds", type=float, default=10.0)
     args = ap.parse_args(argv)

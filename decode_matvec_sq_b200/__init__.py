@@ -81,6 +81,8 @@ def lib():
                                    ctypes.c_int),
         "sq_linear_noalloc": ([pw, vp, vp, vp, vp, i32, i32, vp, vp, u32, vp], ctypes.c_int),
         "sq_quantize_linear": ([pw, vp, i32, vp, i32, vp, vp, sz, vp, u32, vp], ctypes.c_int),
+        "sq_testing_prefill_stalled": ([pw, vp, vp, vp, vp, i32, i32, vp, i32, ctypes.c_uint64, vp,
+                                        vp], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -328,6 +330,21 @@ def linear_noalloc(pw: PackedWeight, xq, sx, x_out, idx, y, status=None, pdl: bo
                                 _ptr(x_out) if n else None, _ptr(idx) if n else None, n, M,
                                 _ptr(y), _ptr(status), _flags(pdl, trunk_only), _stream(stream)),
         "sq_linear_noalloc")
+    return y
+
+
+def testing_prefill_stalled(pw: PackedWeight, xq, sx, x_out, idx, y, skip_group: int,
+                            wait_ns: int, status=None, stream=None):
+    """include/sq_testing.h: the prefill kernel with its waits limited to
+    wait_ns and channel group skip_group's operands never requested (-1:
+    none), so that its bounded waits run out (tests of the wind-down path)."""
+    M = xq.shape[0]
+    n = 0 if idx is None else int(idx.numel())
+    _ck(lib().sq_testing_prefill_stalled(ctypes.byref(pw.view), _ptr(xq), _ptr(sx),
+                                         _ptr(x_out) if n else None, _ptr(idx) if n else None, n,
+                                         M, _ptr(y), skip_group, wait_ns, _ptr(status),
+                                         _stream(stream)),
+        "sq_testing_prefill_stalled")
     return y
 
 

@@ -415,3 +415,31 @@ sq_status sq_quantize_linear(const sq_packed_weight* w, const float* x, int32_t 
 }
 
 }  // extern "C"
+
+// ---- failure injection for the tests (include/sq_testing.h) -----------------------
+#include "../../include/sq_testing.h"
+
+extern "C" sq_status sq_testing_prefill_stalled(const sq_packed_weight* w, const int8_t* xq,
+                                                const float* sx, const float* x_out,
+                                                const int32_t* idx, int32_t n_out, int32_t M,
+                                                float* y, int32_t skip_group, uint64_t wait_ns,
+                                                int32_t* dev_status, void* stream) {
+  sq_status st = check_weight(w);
+  if (st != SQ_OK) return st;
+  if (!xq || !sx || !y) return SQ_ERR_INVALID_ARG;
+  if (w->layout != SQ_LAYOUT_ROWS || w->group_size != kTileK || M < kPrefillMinTokens ||
+      M > (1 << 20))
+    return SQ_ERR_SHAPE;
+  if (n_out < 0 || n_out > kMaxOutliers || n_out > w->K) return SQ_ERR_SHAPE;
+  if (n_out > 0 && (!idx || !x_out)) return SQ_ERR_INVALID_ARG;
+  if (skip_group < -1 || skip_group >= (int32_t)ceil_div(w->K, kTileK)) return SQ_ERR_INVALID_ARG;
+  if (wait_ns < 1 || wait_ns > 1000000000ull) return SQ_ERR_INVALID_ARG;
+  if (!aligned16(xq) || !aligned16(sx) || !aligned16(y) ||
+      (n_out > 0 && (!aligned16(idx) || !aligned16(x_out))))
+    return SQ_ERR_ALIGN;
+  DeviceInfo d;
+  if ((st = check_device(&d)) != SQ_OK) return st;
+  if (!prefill_supported(*w)) return SQ_ERR_UNSUPPORTED_DEVICE;
+  return from_cuda(launch_prefill(*w, M, xq, sx, x_out, idx, n_out, y, nullptr, nullptr, dev_status,
+                                  static_cast<cudaStream_t>(stream), wait_ns, skip_group));
+}

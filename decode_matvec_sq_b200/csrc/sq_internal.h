@@ -85,8 +85,11 @@ cudaError_t launch_linear_tc(const sq_packed_weight& w, int M, const int8_t* xq,
 // MMAs with TMEM accumulators.  T_out / R_out optional (both or neither).
 constexpr int kPrefillMinTokens = 64;
 bool prefill_supported(const sq_packed_weight& w);
+// wait_ns bounds every wait of the kernel; skip_group >= 0 (tests only) never
+// requests that channel group's operands, so the kernel's waits run out.
 cudaError_t launch_prefill(const sq_packed_weight& w, int M, const int8_t* xq, const float* sx,
                            const float* x_out, const int32_t* idx, int n_out, float* y,
-                           int32_t* T_out, int32_t* R_out, int32_t* status, cudaStream_t stream);
+                           int32_t* T_out, int32_t* R_out, int32_t* status, cudaStream_t stream,
+                           uint64_t wait_ns = 1000000000ull, int skip_group = -1);
 
 }  // namespace sq

@@ -311,10 +311,12 @@ __device__ __forceinline__ void write_y(const Params& p, int rb, int gid, int ti
 // (codes [M][K128], outlier values [M][n_pad], scales [M]); outlier channels
 // are those marked in omask.  Same arithmetic as the activation split kernel.
 // Latency is what counts here (the weight stream waits for the codes): for
-// K <= 32768 each thread keeps its share of a token's x in registers (float4,
+// K <= 16384 each thread keeps its share of a token's x in registers (float4,
 // all loads in flight at once), so a token costs one memory round trip and
 // one barrier; the outlier values are gathered with the same round trip.
-constexpr int kXRegs = 16;  // float4 per thread kept in registers: K <= 32768
+// float4 per thread kept in registers: K <= 16384 (16 per thread made the
+// compiler spill registers in the fused kernels)
+constexpr int kXRegs = 8;
 
 __device__ __forceinline__ uint32_t omask_nibble(const uint32_t* omask, int j4) {
   return (omask[j4 >> 3] >> ((j4 & 7) * 4)) & 0xFu;  // outlier bits of channels 4*j4 .. 4*j4+3
@@ -398,12 +400,20 @@ __device__ __forceinline__ void split_activations(const Params& p, const uint32_
         if (!((omask[j >> 5] >> (j & 31)) & 1u)) a = fmaxf(a, fabsf(v));
       }
     }
-    for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    // a >= 0 (or +inf): the order of non-negative floats is that of their bits
+    a = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(a)));
     if (lane == 0) red_s[(t & 1) * kWarps + warp] = a;  // two buffers: token t+1 may start early
     __syncthreads();
-    a = 0.0f;
+    {
+      const uint4* r4 = reinterpret_cast<const uint4*>(red_s + (t & 1) * kWarps);
+      uint32_t m = 0u;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) a = fmaxf(a, red_s[(t & 1) * kWarps + w]);
+      for (int w = 0; w < kWarps / 4; ++w) {
+        const uint4 v = r4[w];
+        m = max(m, max(max(v.x, v.y), max(v.z, v.w)));
+      }
+      a = __uint_as_float(m);
+    }
     const float s = act_scale(a);
     const float rinv = act_rinv(s);
     if (threadIdx.x == 0) sx_s[t] = s;

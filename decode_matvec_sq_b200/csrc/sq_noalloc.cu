@@ -67,6 +67,15 @@ extern "C" sq_status sq_linear_noalloc(const sq_packed_weight* w, const int8_t* 
   if (need == 0)
     return sq_linear(w, xq, sx, x_out, idx, n_out, M, y, nullptr, 0, dev_status, flags, stream);
   if (need > kScratchBytes) return SQ_ERR_WORKSPACE;
+  // the scratch is the current device's; a stream of another device would
+  // make the kernel use (and race on) the wrong array
+  if (stream) {
+    int sdev = -1, cur = -1;
+    if (cudaStreamGetDevice(static_cast<cudaStream_t>(stream), &sdev) != cudaSuccess ||
+        cudaGetDevice(&cur) != cudaSuccess)
+      return SQ_ERR_CUDA;
+    if (sdev != cur) return SQ_ERR_INVALID_ARG;
+  }
   void* ws = nullptr;
   const sq_status st = scratch_of_current_device(static_cast<cudaStream_t>(stream), &ws);
   if (st != SQ_OK) return st;

@@ -23,6 +23,11 @@
 // Two CTAs share an SM (256 of the 512 TMEM columns each), so one CTA's
 // epilogue overlaps the other's MMAs.  Every wait is bounded: a wait that
 // runs out sets SQ_ERR_TIMEOUT in the status word and the CTA winds down.
+// Winding down drains the asynchronous work first: the TMA producer waits
+// (bounded) until every stage it requested has landed, and the MMA issuer
+// commits to a last barrier and waits (bounded) until its MMAs are done, so
+// no copy still writes shared memory and no MMA still writes tensor memory
+// when the CTA frees it and exits.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <stdint.h>
@@ -83,6 +88,8 @@ struct Params {
   int32_t* T_out;
   int32_t* R_out;
   int32_t* status;
+  uint64_t wait_ns;  // limit of every bounded wait
+  int skip_group;    // failure injection for tests: this group's operands are never requested (-1: none)
 };
 
 // ---- PTX wrappers ---------------------------------------------------------------
@@ -154,9 +161,9 @@ __device__ __forceinline__ void named_sync_epi() {
 
 // Waits on an mbarrier phase; on a timeout records it and asks the CTA to stop.
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Aux* aux,
-                                              int32_t* status) {
-  if (mbar_wait(bar, parity)) return true;
-  set_status(status, SQ_ERR_TIMEOUT);
+                                              const Params& p) {
+  if (mbar_wait(bar, parity, p.wait_ns)) return true;
+  set_status(p.status, SQ_ERR_TIMEOUT);
   atomicExch(&aux->abort, 1);
   return false;
 }
@@ -220,11 +227,15 @@ __global__ void __launch_bounds__(kThreads, 2)
   if (warp == 0) {
     // ---- TMA producer
     if (lane == 0) {
+      int last_use[kStages];  // the last use of each stage requested (-1: none)
+#pragma unroll
+      for (int s = 0; s < kStages; ++s) last_use[s] = -1;
       for (int kb = 0; kb < p.nk; ++kb) {
         const int s = kb % kStages;
         const uint32_t use = (uint32_t)(kb / kStages);
-        if (kb >= kStages && !wait_or_abort(&aux->empty[s], (use & 1u) ^ 1u, aux, p.status)) break;
+        if (kb >= kStages && !wait_or_abort(&aux->empty[s], (use & 1u) ^ 1u, aux, p)) break;
         if (aborted(aux)) break;
+        if (kb == p.skip_group) continue;  // (tests only) never requested: its waits run out
         uint8_t* st = smem + s * kStageBytes;
         mbar_arrive_expect_tx(&aux->full[s],
                               kBytesA + kBytesB + kBytesBits + (MASK ? kBytesBits : 0));
@@ -232,6 +243,14 @@ __global__ void __launch_bounds__(kThreads, 2)
         tma_load_2d(st + kOffB, &tmB, kb * BK, n0, &aux->full[s]);
         tma_load_2d(st + kOffS, &tmS, kb * 4, n0, &aux->full[s]);
         if (MASK) tma_load_2d(st + kOffM, &tmM, kb * 4, n0, &aux->full[s]);
+        last_use[s] = (int)use;
+      }
+      // winding down after a timeout: every requested stage must have landed
+      // before the CTA's shared memory is released
+      if (aborted(aux)) {
+#pragma unroll
+        for (int s = 0; s < kStages; ++s)
+          if (last_use[s] >= 0) (void)mbar_wait(&aux->full[s], (uint32_t)last_use[s] & 1u, p.wait_ns);
       }
     }
   } else if (warp == 1) {
@@ -240,10 +259,10 @@ __global__ void __launch_bounds__(kThreads, 2)
       for (int kb = 0; kb < p.nk; ++kb) {
         const int s = kb % kStages, b = kb % kAccBufs;
         const uint32_t use = (uint32_t)(kb / kStages);
-        if (!wait_or_abort(&aux->full[s], use & 1u, aux, p.status)) break;
-        if (!wait_or_abort(&aux->tready[s], use & 1u, aux, p.status)) break;
+        if (!wait_or_abort(&aux->full[s], use & 1u, aux, p)) break;
+        if (!wait_or_abort(&aux->tready[s], use & 1u, aux, p)) break;
         if (kb >= kAccBufs &&
-            !wait_or_abort(&aux->acce[b], ((uint32_t)(kb / kAccBufs) & 1u) ^ 1u, aux, p.status))
+            !wait_or_abort(&aux->acce[b], ((uint32_t)(kb / kAccBufs) & 1u) ^ 1u, aux, p))
           break;
         tc_fence_after();
         const uint32_t st = smem_u32(smem + s * kStageBytes);
@@ -259,6 +278,9 @@ __global__ void __launch_bounds__(kThreads, 2)
         mma_commit(&aux->accf[b]);
       }
       mma_commit(&aux->tdone);
+      // winding down after a timeout: the MMAs issued must be done before the
+      // tensor memory is freed (in a normal run the epilogue waited for this)
+      if (aborted(aux)) (void)mbar_wait(&aux->tdone, 0u, p.wait_ns);
     }
   } else if (warp < 4) {
     // ---- trunk expansion: one weight row per thread; the same thread puts
@@ -274,7 +296,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       s_cur = s_next;
       s_next = (srow && kb + 2 < p.nk) ? __ldg(srow_p + kb + 2) : 0.0f;
       mbar_arrive(&aux->sready[kb & 7]);
-      if (!wait_or_abort(&aux->full[s], (uint32_t)(kb / kStages) & 1u, aux, p.status)) break;
+      if (!wait_or_abort(&aux->full[s], (uint32_t)(kb / kStages) & 1u, aux, p)) break;
       uint8_t* st = smem + s * kStageBytes;
       const uint4 sw = *reinterpret_cast<const uint4*>(st + kOffS + r * 16);
       uint4 mw = make_uint4(0u, 0u, 0u, 0u);
@@ -312,8 +334,8 @@ __global__ void __launch_bounds__(kThreads, 2)
       const int b = kb % kAccBufs;
       const float4* scl4 = reinterpret_cast<const float4*>(aux->scl[kb & 7]);
       bool ok = !aborted(aux) &&
-                wait_or_abort(&aux->sready[kb & 7], (uint32_t)(kb >> 3) & 1u, aux, p.status) &&
-                wait_or_abort(&aux->accf[b], (uint32_t)(kb / kAccBufs) & 1u, aux, p.status);
+                wait_or_abort(&aux->sready[kb & 7], (uint32_t)(kb >> 3) & 1u, aux, p) &&
+                wait_or_abort(&aux->accf[b], (uint32_t)(kb / kAccBufs) & 1u, aux, p);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) continue;
       tc_fence_after();
@@ -342,7 +364,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
       }
     }
-    bool fin = !aborted(aux) && wait_or_abort(&aux->tdone, 0u, aux, p.status);
+    bool fin = !aborted(aux) && wait_or_abort(&aux->tdone, 0u, aux, p);
     named_sync_epi();  // a timeout anywhere is now visible to all epilogue threads
     fin = fin && !aborted(aux);
     if (__any_sync(0xffffffffu, !fin)) fin = false;
@@ -465,7 +487,8 @@ bool prefill_supported(const sq_packed_weight& w) {
 
 cudaError_t launch_prefill(const sq_packed_weight& w, int M, const int8_t* xq, const float* sx,
                            const float* x_out, const int32_t* idx, int n_out, float* y,
-                           int32_t* T_out, int32_t* R_out, int32_t* status, cudaStream_t stream) {
+                           int32_t* T_out, int32_t* R_out, int32_t* status, cudaStream_t stream,
+                           uint64_t wait_ns, int skip_group) {
   if (!prefill_supported(w) || M < 1) return cudaErrorInvalidValue;
   const int64_t K128 = xq_stride_of(w.K);
   CUtensorMap ma, mb, ms, mm;
@@ -504,6 +527,8 @@ cudaError_t launch_prefill(const sq_packed_weight& w, int M, const int8_t* xq, c
   p.T_out = T_out;
   p.R_out = R_out;
   p.status = status;
+  p.wait_ns = wait_ns;
+  p.skip_group = skip_group;
   const int64_t grid = ceil_div(M, BM) * ceil_div(w.N, BN);
   if (grid >= INT32_MAX) return cudaErrorInvalidValue;
   const bool mask = w.mask_bits != nullptr, emit = T_out != nullptr;

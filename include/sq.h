@@ -65,10 +65,12 @@ typedef enum {
  * (outlier channels take the trunk weight).  Not accepted by
  * sq_linear_accumulators. */
 /* SQ_LAUNCH_PDL: launch with programmatic dependent launch.  The kernel may
- * start while the previous kernel in the stream is still running and begins
- * streaming the packed weights at once; it reads every other input and writes
+ * start while the previous kernel in the stream is still running: it begins
+ * streaming the packed weights and reads the outlier index list (both fixed
+ * once a layer is set up) at once, and reads every other input and writes
  * every output only after the previous kernel has completed.  Set it only if
- * no earlier work still in flight on the stream writes the packed weights. */
+ * no earlier work still in flight on the stream writes the packed weights or
+ * the index list. */
 
 /* Packed-weight layouts (sq_packed_weight.layout). */
 #define SQ_LAYOUT_ROWS 0
@@ -298,6 +300,8 @@ int32_t sq_quantize_linear_tokens_per_pass(const sq_packed_weight *w, int32_t n_
  *   Overlapping calls race: all calls on a device share the array, so two
  *   calls whose kernels may run at the same time (other streams, other host
  *   threads) give wrong results.  Order them on one stream or by events.
+ *   The stream must belong to the current device (else SQ_ERR_INVALID_ARG):
+ *   the array used is the current device's.
  * Arguments, flags and results are those of sq_linear.
  */
 #define SQ_LINEAR_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)

@@ -29,7 +29,11 @@ def L():
 
 
 def test_every_declared_symbol_is_exported(L):
-    names = _declared(os.path.join(ROOT, "include", "sq.h"))
+    import glob
+    names = []
+    for h in sorted(glob.glob(os.path.join(ROOT, "include", "*.h"))):
+        names += _declared(h)
+    assert "sq_testing_prefill_stalled" in names
     assert {"sq_decompose_pack", "sq_calibrate_outliers", "sq_quantize_act", "sq_linear"} <= set(names)
     for n in names:
         assert hasattr(L, n), f"{n} declared in include/sq.h but not exported"

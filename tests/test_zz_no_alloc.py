@@ -55,6 +55,56 @@ def test_noalloc_matches_sq_linear_twice(cuda_device, N, K, M, n_out, P, layout)
         err = np.abs(y.cpu().numpy().astype(np.float64) - ref)
         assert np.isfinite(err).all()
         assert (err <= TOL * bound).all(), float((err / bound).max())
+        # the same kernel on the same inputs: the scratch must not change the sums
+        assert torch.equal(y, y_ref)
+
+
+@pytest.mark.gpu
+def test_noalloc_reuse_across_sizes_is_exact(cuda_device):
+    """The row layout (CUDA-core kernel, rows split between CTAs finished
+    through per-row counters in the scratch): a large layer, a small one, then
+    the large one again through the one shared array, each bit-equal to
+    sq_linear with a workspace of its own.  A counter left non-zero by one
+    call would change the next call's finishing order or sums."""
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    cases = {}
+    for name, (N, K, M, n_out) in {"large": (6000, 4096, 2, 20), "small": (40, 512, 1, 3)}.items():
+        W, x, idx = _inputs(N, K, M, n_out, seed=N + 7)
+        pw = sq.decompose_pack(torch.from_numpy(W).cuda(), layout=0, status=st)
+        idxd = torch.from_numpy(idx).cuda()
+        act = sq.quantize_act(torch.from_numpy(x).cuda(), idxd, status=st)
+        cases[name] = (pw, idxd, act, sq.linear(pw, *act, idxd, status=st), (M, N))
+    for name in ("large", "small", "large", "small"):
+        pw, idxd, act, y_ref, shape = cases[name]
+        y = torch.full(shape, float("nan"), dtype=torch.float32, device="cuda")
+        sq.linear_noalloc(pw, *act, idxd, y, status=st)
+        torch.cuda.synchronize()
+        assert st.item() == 0
+        assert torch.equal(y, y_ref), name
+
+
+@pytest.mark.gpu
+def test_noalloc_rejects_a_stream_of_another_device(cuda_device):
+    """Only checkable with two devices; on one it checks the same-device path
+    with an explicit (non-default) stream."""
+    W, x, idx = _inputs(64, 256, 1, 2, seed=3)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pw = sq.decompose_pack(torch.from_numpy(W).cuda(), layout=1, status=st)
+    idxd = torch.from_numpy(idx).cuda()
+    act = sq.quantize_act(torch.from_numpy(x).cuda(), idxd, status=st)
+    y_ref = sq.linear(pw, *act, idxd, status=st)
+    s = torch.cuda.Stream()
+    y = torch.full((1, 64), float("nan"), dtype=torch.float32, device="cuda")
+    with torch.cuda.stream(s):
+        sq.linear_noalloc(pw, *act, idxd, y, status=st)
+    torch.cuda.synchronize()
+    assert torch.equal(y, y_ref)
+    if torch.cuda.device_count() > 1:
+        with torch.cuda.device(1):
+            other = torch.cuda.Stream()
+        with pytest.raises(sq.SQError) as e:
+            sq.linear_noalloc(pw, *act, idxd, y, status=st, stream=other)
+        assert e.value.name == "SQ_ERR_INVALID_ARG"
 
 
 @pytest.mark.gpu
