@@ -72,11 +72,13 @@ def _load():
             lib.sqo_linear_asym.argtypes = [i64, i64, i64, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                             vp, i32, vp]
             lib.sqo_abs_dot.argtypes = [i64, i64, i64, vp, vp, vp]
+            lib.sqo_layer_sq_error.argtypes = [i64, i64, i32, vp, vp, vp, vp, vp, vp, vp, vp]
+            lib.sqo_plain_sq_error.argtypes = [i64, i64, i32, vp, vp]
             for name in ("sqo_quantize_groups", "sqo_trunk_threshold", "sqo_decompose",
                          "sqo_calibrate", "sqo_quantize_act", "sqo_accumulate",
                          "sqo_trunk_popcount", "sqo_linear", "sqo_linear_naive", "sqo_linear_trunk",
                          "sqo_sparsify_residual", "sqo_quantize_groups_asym", "sqo_linear_asym",
-                         "sqo_abs_dot"):
+                         "sqo_abs_dot", "sqo_layer_sq_error", "sqo_plain_sq_error"):
                 getattr(lib, name).restype = i32
             _lib = lib
     return _lib
@@ -330,3 +332,34 @@ def reference_forward(W, x, idx, G: int = 128, P: int = -1):
     xq, sx, xout = quantize_act(x, idx)
     y = linear(d, xq, sx, xout, idx)
     return d, (xq, sx, xout), y
+
+
+def layer_sq_error(d, W) -> float:
+    """sum over the layer of (W - What)^2 for decomposition d (symmetric, or
+    asymmetric when d has "z"), binary64 ([P1] s2.3: the fallback measure)."""
+    W = _c(W, np.float32)
+    N, K = W.shape
+    z = d.get("z")
+    out = np.zeros(1, np.float64)
+    _ck(_load().sqo_layer_sq_error(N, K, d["G"], _p(W), _p(_c(d["sign"], np.uint8)),
+                                   _p(_c(d["mask"], np.uint8)), _p(_c(d["alpha"], np.float32)),
+                                   _p(_c(d["q"], np.int8)), _p(_c(d["s"], np.float32)),
+                                   None if z is None else _p(_c(z, np.int32)), _p(out)),
+        "layer_sq_error")
+    return float(out[0])
+
+
+def plain_sq_error(W, G: int = 128) -> float:
+    """The same error for plain symmetric INT8 groups of W (no trunk)."""
+    W = _c(W, np.float32)
+    N, K = W.shape
+    out = np.zeros(1, np.float64)
+    _ck(_load().sqo_plain_sq_error(N, K, G, _p(W), _p(out)), "plain_sq_error")
+    return float(out[0])
+
+
+def choose_fallback(W, P: int = -1, G: int = 128) -> bool:
+    """The per-layer rule ([P1] s2.3, last paragraph: a layer that gains
+    nothing from the split falls back to plain 8-bit): fall back when plain
+    INT8 groups reconstruct W at least as well as the split does."""
+    return plain_sq_error(W, G) <= layer_sq_error(decompose(W, G=G, P=P), W)

@@ -528,3 +528,55 @@ int sqo_abs_dot(int64_t M, int64_t N, int64_t K, const float *W,
         }
     return SQO_OK;
 }
+
+/* ---- per-layer fallback measure ([P1] s2.3, last paragraph) ------------- */
+
+int sqo_layer_sq_error(int64_t N, int64_t K, int G, const float *W, const uint8_t *sign,
+                       const uint8_t *mask, const float *alpha, const int8_t *q,
+                       const float *s, const int32_t *z, double *err)
+{
+    if (N < 1 || K < 1 || !valid_group(G) || !W || !sign || !mask || !alpha || !q || !s || !err)
+        return SQO_BAD_ARG;
+    int64_t ng = n_groups(K, G);
+    double total = 0.0;
+    for (int64_t r = 0; r < N; ++r) {
+        double e = 0.0;
+        for (int64_t j = 0; j < K; ++j) {
+            int64_t g = j / G;
+            double t = mask[r * K + j] ? (sign[r * K + j] ? (double)alpha[r] : -(double)alpha[r]) : 0.0;
+            int64_t zz = z ? (int64_t)z[r * ng + g] : 0;
+            double what = t + (double)s[r * ng + g] * (double)((int64_t)q[r * K + j] - zz);
+            double d = (double)W[r * K + j] - what;
+            e += d * d;
+        }
+        total += e;
+    }
+    *err = total;
+    return SQO_OK;
+}
+
+int sqo_plain_sq_error(int64_t N, int64_t K, int G, const float *W, double *err)
+{
+    if (N < 1 || K < 1 || !valid_group(G) || !W || !err)
+        return SQO_BAD_ARG;
+    double total = 0.0;
+    for (int64_t r = 0; r < N; ++r) {
+        double e = 0.0;
+        for (int64_t j0 = 0; j0 < K; j0 += G) {
+            const int64_t jend = (j0 + G < K) ? (j0 + G) : K;
+            double a = 0.0;
+            for (int64_t j = j0; j < jend; ++j)
+                if (fabs((double)W[r * K + j]) > a)
+                    a = fabs((double)W[r * K + j]);
+            float sg = sqo_scale_from_absmax(a);
+            for (int64_t j = j0; j < jend; ++j) {
+                double w = (double)W[r * K + j];
+                double d = w - (double)sg * (double)sqo_quantize(w, sg);
+                e += d * d;
+            }
+        }
+        total += e;
+    }
+    *err = total;
+    return SQO_OK;
+}

@@ -166,6 +166,21 @@ int sqo_linear_naive(int64_t M, int64_t N, int64_t K, int G, const uint8_t *sign
                      const float *s, const int8_t *xq, const float *sx,
                      const float *xout, const int32_t *idx, int n_out, double *y);
 
+/* Reconstruction error of a decomposition over a layer (m.lqnn.cn news
+ * 241359, section 2.3, last paragraph: a layer that gains nothing from the
+ * split falls back to plain 8-bit; this is the measure compared):
+ *   E = sum_r e_r,  e_r = sum_j (W_rj - What_rj)^2 in ascending j,
+ *   What = mask*(sign ? alpha : -alpha) + s_g*(q - z_g)
+ * with z = NULL for a symmetric residual (z_g = 0).  Binary64, rows in
+ * order. */
+int sqo_layer_sq_error(int64_t N, int64_t K, int G, const float *W, const uint8_t *sign,
+                       const uint8_t *mask, const float *alpha, const int8_t *q,
+                       const float *s, const int32_t *z, double *err);
+
+/* The same error for plain symmetric INT8 groups of W itself (no trunk):
+ * What = s_g*Q(W, s_g), s_g = float(absmax_g |W| / 127). */
+int sqo_plain_sq_error(int64_t N, int64_t K, int G, const float *W, double *err);
+
 /* Tolerance scale sum_j |W_rj * x_tj| from the original fp32 W and x, [M][N]. */
 int sqo_abs_dot(int64_t M, int64_t N, int64_t K, const float *W,
                 const float *x, double *out);

@@ -76,6 +76,13 @@ MUTANTS = {
     "abs_dot_doubles_term": ("acc += fabs((double)W[r * K + j] * (double)x[t * K + j]);",
                              "acc += 2.0 * fabs((double)W[r * K + j] * (double)x[t * K + j]);"),
     "abs_dot_transposes_output": ("out[t * N + r] = acc;", "out[r * M + t] = acc;"),
+    "layer_error_not_squared": ("            e += d * d;\n        }\n        total += e;\n    }\n    *err = total;\n    return SQO_OK;\n}\n\nint sqo_plain_sq_error",
+                                "            e += fabs(d);\n        }\n        total += e;\n    }\n    *err = total;\n    return SQO_OK;\n}\n\nint sqo_plain_sq_error"),
+    "layer_error_drops_zero_point": ("int64_t zz = z ? (int64_t)z[r * ng + g] : 0;", "int64_t zz = 0;"),
+    "layer_error_trunk_sign_flipped": ("double t = mask[r * K + j] ? (sign[r * K + j] ? (double)alpha[r] : -(double)alpha[r]) : 0.0;\n            int64_t zz",
+                                       "double t = mask[r * K + j] ? (sign[r * K + j] ? -(double)alpha[r] : (double)alpha[r]) : 0.0;\n            int64_t zz"),
+    "plain_error_without_quantizer_clip": ("double d = w - (double)sg * (double)sqo_quantize(w, sg);",
+                                           "double d = w - (double)sg * round(w / (double)sg * 1.001);"),
 }
 
 

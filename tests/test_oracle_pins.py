@@ -581,6 +581,76 @@ def test_nonfinite_and_bad_arguments():
         oracle.decompose(np.ones((1, 8), np.float32), G=48)
 
 
+# ---- per-layer fallback to plain INT8 ---------------------------------------------
+
+def test_fallback_errors_on_binary_rows():
+    """Rows of +-c_r: the split is lossless (alpha = c_r, residual 0).  With
+    c_r = 127 * 2^-e plain INT8 is lossless too (s = 2^-e exactly, codes
+    +-127): both errors are exactly 0, the split gains nothing, and the rule
+    falls back.  With c_r = 0.5 the plain scale 0.5/127 rounds, so plain
+    INT8 leaves a small error and the split is kept."""
+    rng = np.random.default_rng(21)
+    signs = rng.choice([-1.0, 1.0], size=(3, 300))
+    c = (127.0 * np.array([2.0 ** -8, 2.0 ** -10, 2.0 ** -6]))[:, None]
+    W = (c * signs).astype(np.float32)
+    assert oracle.layer_sq_error(oracle.decompose(W), W) == 0.0
+    assert oracle.plain_sq_error(W) == 0.0
+    assert oracle.choose_fallback(W)
+    W2 = (0.5 * signs).astype(np.float32)
+    assert oracle.layer_sq_error(oracle.decompose(W2), W2) == 0.0
+    assert 0.0 < oracle.plain_sq_error(W2) < 1e-12
+    assert not oracle.choose_fallback(W2)
+
+
+def test_fallback_on_grid_aligned_weights():
+    """Weights on every group's own INT8 grid (w = s_g * k, |k| <= 127, each
+    group reaching 127): plain INT8 is exact, the split is not -> fall back."""
+    rng = np.random.default_rng(22)
+    N, K, G = 4, 256, 128
+    k = rng.integers(-127, 128, size=(N, K))
+    k[:, 0] = 127
+    k[:, G] = -127
+    sg = np.repeat(rng.uniform(1e-3, 1e-2, size=(N, K // G)), G, axis=1)
+    W = (sg * k).astype(np.float32)
+    # on the grid up to the rounding of s_g*k and of the quantizer's scale
+    assert oracle.plain_sq_error(W) < 1e-12 * float((W.astype(np.float64) ** 2).sum())
+    assert oracle.layer_sq_error(oracle.decompose(W), W) > 0.0
+    assert oracle.choose_fallback(W)
+
+
+def test_no_fallback_on_the_stack_weights():
+    """Laplace weights of the 7B-shaped stack: the residual has the smaller
+    range, so the split reconstructs W better and is kept."""
+    for mid in range(4):
+        W = wl.config2_layer(0, mid).weights(rows=np.arange(8))
+        assert oracle.layer_sq_error(oracle.decompose(W), W) < oracle.plain_sq_error(W)
+        assert not oracle.choose_fallback(W)
+
+
+@pytest.mark.parametrize("P", [-1, 60])
+def test_fallback_errors_second_route(P):
+    """Second route with numpy: What formed from the decomposition's arrays,
+    the squared error summed row by row (1e-12 relative); plain INT8 equals
+    the split with an empty trunk (100th percentile) bit for bit."""
+    rng = np.random.default_rng(23 + P)
+    W = rng.laplace(0, 0.02, (7, 300)).astype(np.float32)
+    d = oracle.decompose(W, P=P)
+    G = 128
+    s = np.repeat(d["s"].astype(np.float64), G, axis=1)[:, :300]
+    what = d["mask"] * np.where(d["sign"] == 1, 1.0, -1.0) * d["alpha"].astype(np.float64)[:, None] \
+        + s * d["q"].astype(np.float64)
+    ref = float(((W.astype(np.float64) - what) ** 2).sum(axis=1).sum())
+    assert abs(oracle.layer_sq_error(d, W) - ref) <= 1e-12 * ref
+    assert oracle.plain_sq_error(W) == oracle.layer_sq_error(oracle.decompose(W, P=100), W)
+    da = oracle.decompose_asym(W, P=P)
+    sa = np.repeat(da["s"].astype(np.float64), G, axis=1)[:, :300]
+    za = np.repeat(da["z"].astype(np.float64), G, axis=1)[:, :300]
+    what_a = da["mask"] * np.where(da["sign"] == 1, 1.0, -1.0) * da["alpha"].astype(np.float64)[:, None] \
+        + sa * (da["q"].astype(np.float64) - za)
+    ref_a = float(((W.astype(np.float64) - what_a) ** 2).sum(axis=1).sum())
+    assert abs(oracle.layer_sq_error(da, W) - ref_a) <= 1e-12 * ref_a
+
+
 # ---- tolerance scale ------------------------------------------------------------
 
 def test_abs_dot_closed_form():
