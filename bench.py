@@ -499,6 +499,15 @@ def layer_cases(workload: str):
     if workload == "threshold":
         L = wl.config4()
         return [("4096->14336 threshold trunk P=60", L, 1, -(-2 * L2_BYTES // L.packed_bytes))]
+    if workload == "sparse":
+        out = []
+        for Ps in (50, 60, 70):
+            for mid in range(4):
+                L = wl.config2_layer(0, mid)
+                out.append((f"{L.name.split('.')[-1]} {L.K}->{L.N} sparse residual Ps={Ps}",
+                            L.with_(residual_percent=Ps), 1,
+                            -(-2 * L2_BYTES // int(L.packed_bytes * (1.2 - Ps / 100.0)))))
+        return out
     if workload == "trunk":
         out = []
         for mid in range(4):
@@ -516,6 +525,16 @@ def trunk_weight_bytes(L) -> int:
     words = -(-L.K // 128) * 4
     planes = 2 if L.trunk_percent >= 0 else 1
     return rows * (4 * words * planes + 4)
+
+
+def sparse_weight_bytes(pw) -> int:
+    """Bytes the decode kernel reads of a sparse-residual weight: sign (and
+    mask) and keep bits, each tile's packed kept codes (padded to 16), the
+    group scales, the row scales and the per-tile byte counts."""
+    rows, words, groups = pw.rows, pw.view.sign_stride, pw.view.scale_stride
+    planes = 3 if pw.with_mask else 2
+    nb = pw.res_bytes()
+    return rows * (4 * words * planes + 4 * groups + 4) + int(nb.sum().item()) + 4 * nb.numel()
 
 
 def _fused_launches(pw, M: int, L) -> int:
@@ -540,7 +559,11 @@ def time_layer_case(L, M, copies, trunk, st, device, warmup, reps):
     import decode_matvec_sq_b200 as sq
     import synth.device as sdev
     W = sdev.fill_weights(L, torch.empty(L.N, L.K, device=device))
-    pw = sq.decompose_pack(W, trunk_percent=L.trunk_percent, status=st)
+    Ps = getattr(L, "residual_percent", None)
+    if Ps:
+        pw = sq.decompose_pack_sparse(W, Ps, trunk_percent=L.trunk_percent, status=st)
+    else:
+        pw = sq.decompose_pack(W, trunk_percent=L.trunk_percent, status=st)
     del W
     pws = [pw]
     for _ in range(copies - 1):
@@ -561,7 +584,7 @@ def time_layer_case(L, M, copies, trunk, st, device, warmup, reps):
     for _ in range(warmup):
         launch()
     ms = _time_calls(launch, reps) / calls
-    wbytes = trunk_weight_bytes(L) if trunk else linear_weight_bytes(L)
+    wbytes = trunk_weight_bytes(L) if trunk else (sparse_weight_bytes(pw) if Ps else linear_weight_bytes(L))
     nbytes = wbytes + M * (4 * L.K + 4 * L.N) + 4 * L.n_out
     launches = _fused_launches(pw, M, L)
     del pws, pw, ws
@@ -693,7 +716,10 @@ def run_layers(args, world, rank, local):
              "threshold": "4096->14336, batch 1, per-row 60th-percentile trunk mask, "
                           "W Laplace(0,0.02), x N(0,1) with 0.5% channels x30",
              "trunk": "trunk-only mode (residual path skipped) of the 7B-shaped stack's four "
-                      "linears, batch 1, W Laplace(0,0.02), x N(0,1) with 0.5% channels x30"}
+                      "linears, batch 1, W Laplace(0,0.02), x N(0,1) with 0.5% channels x30",
+             "sparse": "sparse residual (per-row Ps-th percentile of |r| dropped, Ps 50/60/70) on "
+                       "the 7B-shaped stack's four linears, batch 1, W Laplace(0,0.02), "
+                       "x N(0,1) with 0.5% channels x30; GB/s on the bytes the kernel reads"}
     if rank == 0:
         print(json.dumps({
             "metric": f"single-layer sq_quantize_linear HBM GB/s ({args.workload})",
@@ -889,7 +915,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["sq", "reference"], default="sq")
     ap.add_argument("--layers", type=int, default=32)
     ap.add_argument("--workload", choices=["decode", "prefill", "single", "mlp70b", "threshold",
-                                           "trunk"],
+                                           "trunk", "sparse"],
                     default="decode",
                     help="decode: the 7B-shaped stack at batch 1 (default); prefill: "
                          "2048 tokens x 4096 -> 14336 on the tcgen05 kernel; single, mlp70b, "
@@ -914,7 +940,7 @@ def main(argv=None):
         return run_reference(args, world, rank)
     if args.workload == "prefill":
         return run_prefill(args, world, rank, local)
-    if args.workload in ("single", "mlp70b", "threshold", "trunk"):
+    if args.workload in ("single", "mlp70b", "threshold", "trunk", "sparse"):
         return run_layers(args, world, rank, local)
     return run_gpu(args, world, rank, local)
 

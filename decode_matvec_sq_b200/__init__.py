@@ -25,6 +25,7 @@ SQ_LAUNCH_PDL = 1
 SQ_TRUNK_ONLY = 2
 SQ_LAYOUT_ROWS = 0
 SQ_LAYOUT_TILES = 1
+SQ_LAYOUT_TILES_SPARSE = 2
 
 STATUS = {
     0: "SQ_OK", 1: "SQ_ERR_INVALID_ARG", 2: "SQ_ERR_SHAPE", 3: "SQ_ERR_ALIGN",
@@ -48,6 +49,7 @@ class SqPackedWeight(ctypes.Structure):
         ("scale_stride", ctypes.c_int32),
         ("sign_bits", ctypes.c_void_p), ("mask_bits", ctypes.c_void_p),
         ("alpha", ctypes.c_void_p), ("res_q", ctypes.c_void_p), ("res_scale", ctypes.c_void_p),
+        ("keep_bits", ctypes.c_void_p), ("res_bytes", ctypes.c_void_p),
     ]
 
 
@@ -71,6 +73,7 @@ def lib():
         "sq_packed_bytes": ([i32, i32, i32, i32, i32], sz),
         "sq_packed_view": ([vp, i32, i32, i32, i32, i32, pw], ctypes.c_int),
         "sq_decompose_pack": ([vp, i32, i32, i32, pw, vp, vp], ctypes.c_int),
+        "sq_decompose_pack_sparse": ([vp, i32, i32, i32, i32, pw, vp, vp], ctypes.c_int),
         "sq_calibrate_outliers": ([vp, i32, i32, i32, vp, vp, vp], ctypes.c_int),
         "sq_quantize_act": ([vp, i32, i32, vp, i32, vp, vp, vp, vp, u32, vp], ctypes.c_int),
         "sq_linear_workspace_bytes": ([pw, i32], sz),
@@ -144,9 +147,13 @@ class PackedWeight:
         return int(self.buf.numel())
 
     @property
+    def tiled(self) -> bool:
+        return self.layout in (SQ_LAYOUT_TILES, SQ_LAYOUT_TILES_SPARSE)
+
+    @property
     def rows(self) -> int:
-        """Rows of every array: N, or N padded to 16 in the tiled layout."""
-        return round_up(self.N, 16) if self.layout == SQ_LAYOUT_TILES else self.N
+        """Rows of every array: N, or N padded to 16 in the tiled layouts."""
+        return round_up(self.N, 16) if self.tiled else self.N
 
     def _arr(self, field: str, dtype, shape):
         import torch
@@ -180,6 +187,20 @@ class PackedWeight:
         import torch
         return self._arr("res_scale", torch.float32, (self.rows, self.view.scale_stride))
 
+    def keep_bits(self):
+        import torch
+        if self.layout != SQ_LAYOUT_TILES_SPARSE:
+            return None
+        return self._arr("keep_bits", torch.int32, (self.rows, self.view.sign_stride))
+
+    def res_bytes(self):
+        """Packed code bytes of every tile (sparse layout)."""
+        import torch
+        if self.layout != SQ_LAYOUT_TILES_SPARSE:
+            return None
+        tiles = (self.rows // 16) * (self.view.res_stride // 128)
+        return self._arr("res_bytes", torch.int32, (tiles,))
+
 
 def packed_bytes(N: int, K: int, group_size: int = 128, with_mask: bool = False,
                  layout: int = None) -> int:
@@ -212,6 +233,19 @@ def decompose_pack(W, trunk_percent: int = -1, group_size: int = 128, layout: in
         out = alloc_packed(N, K, group_size, trunk_percent > 0, layout, device=W.device)
     _ck(lib().sq_decompose_pack(_ptr(W), N, K, trunk_percent, ctypes.byref(out.view),
                                 _ptr(status), _stream(stream)), "sq_decompose_pack")
+    return out
+
+
+def decompose_pack_sparse(W, residual_percent: int, trunk_percent: int = -1,
+                          out: PackedWeight = None, status=None, stream=None) -> PackedWeight:
+    """sq_decompose_pack with the residual entries at or below the per-row
+    residual_percent-th percentile of |r| dropped, into SQ_LAYOUT_TILES_SPARSE."""
+    N, K = W.shape
+    if out is None:
+        out = alloc_packed(N, K, 128, trunk_percent > 0, SQ_LAYOUT_TILES_SPARSE, device=W.device)
+    _ck(lib().sq_decompose_pack_sparse(_ptr(W), N, K, trunk_percent, residual_percent,
+                                       ctypes.byref(out.view), _ptr(status), _stream(stream)),
+        "sq_decompose_pack_sparse")
     return out
 
 

@@ -90,31 +90,41 @@ sq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? SQ_OK : SQ_ERR_CU
 // outlier channels of a whole row in shared memory).
 constexpr int32_t kMaxTiledK = 131072;
 
+bool known_layout(int32_t layout) {
+  return layout == SQ_LAYOUT_ROWS || layout == SQ_LAYOUT_TILES || layout == SQ_LAYOUT_TILES_SPARSE;
+}
+bool tiled(int32_t layout) { return layout == SQ_LAYOUT_TILES || layout == SQ_LAYOUT_TILES_SPARSE; }
+
 bool valid_layout(int32_t layout, int32_t G, int32_t K) {
   if (layout == SQ_LAYOUT_ROWS) return true;
-  return layout == SQ_LAYOUT_TILES && G == kTileK && K <= kMaxTiledK;
+  return tiled(layout) && G == kTileK && K <= kMaxTiledK;
 }
 
 int32_t sign_stride_of(int32_t K, int32_t layout) {
-  return layout == SQ_LAYOUT_TILES ? (int32_t)(tiles_cols(K) / 32) : (int32_t)round_up(ceil_div(K, 32), 4);
+  return tiled(layout) ? (int32_t)(tiles_cols(K) / 32) : (int32_t)round_up(ceil_div(K, 32), 4);
 }
 int32_t res_stride_of(int32_t K, int32_t layout) {
-  return layout == SQ_LAYOUT_TILES ? (int32_t)tiles_cols(K) : (int32_t)round_up(K, 16);
+  return tiled(layout) ? (int32_t)tiles_cols(K) : (int32_t)round_up(K, 16);
 }
 int32_t scale_stride_of(int32_t K, int32_t G, int32_t layout) {
-  return layout == SQ_LAYOUT_TILES ? (int32_t)(tiles_cols(K) / kTileK)
-                                   : (int32_t)round_up(ceil_div(K, G), 4);
+  return tiled(layout) ? (int32_t)(tiles_cols(K) / kTileK) : (int32_t)round_up(ceil_div(K, G), 4);
 }
-// Rows of every array (the tiled layout pads N to a multiple of 16).
+// Rows of every array (the tiled layouts pad N to a multiple of 16).
 int64_t rows_of(int32_t N, int32_t layout) {
-  return layout == SQ_LAYOUT_TILES ? tiles_rows(N) : (int64_t)N;
+  return tiled(layout) ? tiles_rows(N) : (int64_t)N;
 }
+// Tiles of a tiled layout.
+int64_t tiles_of(int32_t N, int32_t K) { return tiles_rows(N) / kTileRows * (tiles_cols(K) / kTileK); }
 
 sq_status check_weight(const sq_packed_weight* w) {
   if (!w || !w->sign_bits || !w->alpha || !w->res_q || !w->res_scale) return SQ_ERR_INVALID_ARG;
   if (!valid_group(w->group_size) || !valid_shape(w->N, w->K)) return SQ_ERR_SHAPE;
-  if (w->layout != SQ_LAYOUT_ROWS && w->layout != SQ_LAYOUT_TILES) return SQ_ERR_INVALID_ARG;
+  if (!known_layout(w->layout)) return SQ_ERR_INVALID_ARG;
   if (!valid_layout(w->layout, w->group_size, w->K)) return SQ_ERR_SHAPE;
+  if (w->layout == SQ_LAYOUT_TILES_SPARSE) {
+    if (!w->keep_bits || !w->res_bytes) return SQ_ERR_INVALID_ARG;
+    if (!aligned16(w->keep_bits) || !aligned16(w->res_bytes)) return SQ_ERR_ALIGN;
+  }
   if (w->sign_stride != sign_stride_of(w->K, w->layout) ||
       w->res_stride != res_stride_of(w->K, w->layout) ||
       w->scale_stride != scale_stride_of(w->K, w->group_size, w->layout))
@@ -128,7 +138,7 @@ sq_status check_weight(const sq_packed_weight* w) {
 // Offsets of the five arrays inside one allocation, each 256-byte aligned.
 // alpha holds roundup(N, 8) (rows) or N16 (tiles) floats.
 struct Carve {
-  size_t sign, mask, alpha, res, scale, total;
+  size_t sign, mask, alpha, res, scale, keep, count, total;
 };
 
 Carve carve(int32_t N, int32_t K, int32_t G, int32_t with_mask, int32_t layout) {
@@ -145,6 +155,11 @@ Carve carve(int32_t N, int32_t K, int32_t G, int32_t with_mask, int32_t layout) 
   c.alpha = take((size_t)round_up(rows, 8) * 4);
   c.res = take((size_t)rows * res_stride_of(K, layout));
   c.scale = take((size_t)rows * scale_stride_of(K, G, layout) * 4);
+  c.keep = c.count = 0;
+  if (layout == SQ_LAYOUT_TILES_SPARSE) {
+    c.keep = take((size_t)rows * sign_stride_of(K, layout) * 4);
+    c.count = take((size_t)tiles_of(N, K) * 4);
+  }
   c.total = off;
   return c;
 }
@@ -176,7 +191,7 @@ sq_status sq_device_check(void) {
 size_t sq_packed_bytes(int32_t N, int32_t K, int32_t group_size, int32_t with_mask,
                        int32_t layout) {
   if (!valid_shape(N, K) || !valid_group(group_size)) return 0;
-  if (layout != SQ_LAYOUT_ROWS && layout != SQ_LAYOUT_TILES) return 0;
+  if (!known_layout(layout)) return 0;
   if (!valid_layout(layout, group_size, K)) return 0;
   return carve(N, K, group_size, with_mask, layout).total;
 }
@@ -184,7 +199,7 @@ size_t sq_packed_bytes(int32_t N, int32_t K, int32_t group_size, int32_t with_ma
 sq_status sq_packed_view(void* base, int32_t N, int32_t K, int32_t group_size, int32_t with_mask,
                          int32_t layout, sq_packed_weight* out) {
   if (!base || !out) return SQ_ERR_INVALID_ARG;
-  if (layout != SQ_LAYOUT_ROWS && layout != SQ_LAYOUT_TILES) return SQ_ERR_INVALID_ARG;
+  if (!known_layout(layout)) return SQ_ERR_INVALID_ARG;
   if (!valid_shape(N, K) || !valid_group(group_size)) return SQ_ERR_SHAPE;
   if (!valid_layout(layout, group_size, K)) return SQ_ERR_SHAPE;
   if ((reinterpret_cast<uintptr_t>(base) & 255u) != 0) return SQ_ERR_ALIGN;
@@ -202,6 +217,9 @@ sq_status sq_packed_view(void* base, int32_t N, int32_t K, int32_t group_size, i
   out->alpha = reinterpret_cast<float*>(b + c.alpha);
   out->res_q = reinterpret_cast<int8_t*>(b + c.res);
   out->res_scale = reinterpret_cast<float*>(b + c.scale);
+  const bool sparse = layout == SQ_LAYOUT_TILES_SPARSE;
+  out->keep_bits = sparse ? reinterpret_cast<uint32_t*>(b + c.keep) : nullptr;
+  out->res_bytes = sparse ? reinterpret_cast<int32_t*>(b + c.count) : nullptr;
   return SQ_OK;
 }
 
@@ -211,6 +229,7 @@ sq_status sq_decompose_pack(const float* W, int32_t N, int32_t K, int32_t trunk_
   sq_status st = check_weight(out);
   if (st != SQ_OK) return st;
   if (out->N != N || out->K != K) return SQ_ERR_SHAPE;
+  if (out->layout == SQ_LAYOUT_TILES_SPARSE) return SQ_ERR_INVALID_ARG;  // sq_decompose_pack_sparse
   if (trunk_percent == 0 || trunk_percent > 100) return SQ_ERR_INVALID_ARG;
   if (trunk_percent > 0 && !out->mask_bits) return SQ_ERR_INVALID_ARG;
   if (!aligned16(W) || (dev_status && (reinterpret_cast<uintptr_t>(dev_status) & 3u)))
@@ -221,6 +240,31 @@ sq_status sq_decompose_pack(const float* W, int32_t N, int32_t K, int32_t trunk_
   sq_packed_weight pw = *out;
   return from_cuda(launch_decompose_pack(W, N, K, trunk_percent, pw, dev_status,
                                          static_cast<cudaStream_t>(stream)));
+}
+
+sq_status sq_decompose_pack_sparse(const float* W, int32_t N, int32_t K, int32_t trunk_percent,
+                                   int32_t residual_percent, const sq_packed_weight* out,
+                                   int32_t* dev_status, void* stream) {
+  if (!W || !out) return SQ_ERR_INVALID_ARG;
+  sq_status st = check_weight(out);
+  if (st != SQ_OK) return st;
+  if (out->layout != SQ_LAYOUT_TILES_SPARSE) return SQ_ERR_INVALID_ARG;
+  if (out->N != N || out->K != K) return SQ_ERR_SHAPE;
+  if (trunk_percent == 0 || trunk_percent > 100) return SQ_ERR_INVALID_ARG;
+  if (trunk_percent > 0 && !out->mask_bits) return SQ_ERR_INVALID_ARG;
+  if (residual_percent < 1 || residual_percent > 99) return SQ_ERR_INVALID_ARG;
+  if (!aligned16(W) || (dev_status && (reinterpret_cast<uintptr_t>(dev_status) & 3u)))
+    return SQ_ERR_ALIGN;
+  DeviceInfo d;
+  if ((st = check_device(&d)) != SQ_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // the dense tiled decomposition first (trunk, alpha, codes), then the
+  // sparse residual over it
+  sq_packed_weight dense = *out;
+  dense.layout = SQ_LAYOUT_TILES;
+  cudaError_t e = launch_decompose_pack(W, N, K, trunk_percent, dense, dev_status, s);
+  if (e != cudaSuccess) return SQ_ERR_CUDA;
+  return from_cuda(launch_sparsify_residual(W, N, K, residual_percent, *out, s));
 }
 
 sq_status sq_calibrate_outliers(const float* X, int32_t T, int32_t K, int32_t k, int32_t* idx_out,
@@ -270,7 +314,7 @@ static sq_status linear_common(const sq_packed_weight* w, const int8_t* xq, cons
   if (n_out > 0 && (!idx || !x_out)) return SQ_ERR_INVALID_ARG;
   if (flags & ~(SQ_LAUNCH_PDL | SQ_TRUNK_ONLY)) return SQ_ERR_INVALID_ARG;
   const bool trunk_only = (flags & SQ_TRUNK_ONLY) != 0;
-  if (trunk_only && (w->layout != SQ_LAYOUT_TILES || T_out || R_out)) return SQ_ERR_INVALID_ARG;
+  if (trunk_only && (!tiled(w->layout) || T_out || R_out)) return SQ_ERR_INVALID_ARG;
   if (!aligned16(xq) || !aligned16(sx) || !aligned16(y) ||
       (n_out > 0 && (!aligned16(idx) || !aligned16(x_out))) || (workspace && !aligned16(workspace)))
     return SQ_ERR_ALIGN;
@@ -291,7 +335,7 @@ static sq_status linear_common(const sq_packed_weight* w, const int8_t* xq, cons
                                          dev_status, s);
     return e == cudaSuccess ? SQ_OK : SQ_ERR_CUDA;
   }
-  const bool tc = w->layout == SQ_LAYOUT_TILES;
+  const bool tc = tiled(w->layout);
   const int per_pass = tc ? kMaxTokensPerPassTc : kMaxTokensPerPass;
   const int64_t xs = xq_stride_of(w->K);
   for (int t0 = 0; t0 < M; t0 += per_pass) {
@@ -363,7 +407,7 @@ size_t sq_quantize_linear_workspace_bytes(const sq_packed_weight* w, int32_t M, 
 }
 
 int32_t sq_quantize_linear_tokens_per_pass(const sq_packed_weight* w, int32_t n_out) {
-  if (!w || check_weight(w) != SQ_OK || w->layout != SQ_LAYOUT_TILES) return 0;
+  if (!w || check_weight(w) != SQ_OK || !tiled(w->layout)) return 0;
   if (n_out < 0 || n_out > kMaxOutliers || n_out > w->K) return 0;
   return linear_tc_fused_tokens(*w, n_out);
 }
@@ -374,7 +418,7 @@ sq_status sq_quantize_linear(const sq_packed_weight* w, const float* x, int32_t 
   sq_status st = check_weight(w);
   if (st != SQ_OK) return st;
   if (!x || !y) return SQ_ERR_INVALID_ARG;
-  if (w->layout != SQ_LAYOUT_TILES) return SQ_ERR_SHAPE;
+  if (!tiled(w->layout)) return SQ_ERR_SHAPE;
   if (M < 1 || M > (1 << 20)) return SQ_ERR_SHAPE;
   if (n_out < 0 || n_out > kMaxOutliers || n_out > w->K) return SQ_ERR_SHAPE;
   if (n_out > 0 && !idx) return SQ_ERR_INVALID_ARG;

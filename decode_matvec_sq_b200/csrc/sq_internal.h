@@ -33,6 +33,11 @@ inline int64_t xq_stride_of(int64_t K) { return round_up(K, 128); }
 cudaError_t launch_decompose_pack(const float* W, int N, int K, int P, const sq_packed_weight& pw,
                                   int32_t* status, cudaStream_t stream);
 
+// The sparse residual over a tiled decomposition already in pw's arrays:
+// per-row threshold, re-quantized groups, keep bits, packed codes, byte counts.
+cudaError_t launch_sparsify_residual(const float* W, int N, int K, int Ps, const sq_packed_weight& pw,
+                                     cudaStream_t stream);
+
 cudaError_t launch_calibrate(const float* X, int T, int K, int k, int32_t* idx_out,
                              int32_t* status, cudaStream_t stream);
 

@@ -64,6 +64,8 @@ struct Params {
   const uint32_t* mask;
   const float* alpha;
   const float* scale;
+  const uint32_t* keep;    // keep bits of a sparse residual (SQ_LAYOUT_TILES_SPARSE)
+  const int32_t* nbytes;   // packed code bytes per tile (sparse)
   int N, K, tpr;    // rows, channels, tiles per row block
   int T;            // tiles = ceil(N / 16) * tpr
   int n_rb;         // row blocks = ceil(N / 16); CTA b owns [b*n_rb/grid, (b+1)*n_rb/grid)
@@ -139,11 +141,23 @@ struct Cursor {
   const uint32_t* sign;  // the lane's two sign words; + 64 words per tile
   const uint32_t* mask;
   const float* scale;    // the scale of row r0 (r1: + 8); + 16 floats per tile
+  // sparse residual: the lane's two keep words, and the packed code bytes of
+  // the cursor's tile (loaded one tile ahead, 0 past the last tile)
+  const uint32_t* keep;
+  const int32_t* nbytes;
+  int nb, t, T;
+  template <bool SPARSE>
   __device__ __forceinline__ void advance() {
     code += 2048;
     sign += 64;
     mask += 64;
     scale += 16;
+    if constexpr (SPARSE) {
+      keep += 64;
+      ++nbytes;
+      ++t;
+      nb = t < T ? __ldg(nbytes) : 0;
+    }
   }
 };
 
@@ -163,11 +177,14 @@ struct Cursor {
 // L1 measured slower for these).
 // In the trunk-only mode (RES = false) a slot holds only the 256 sign bytes
 // (then the 256 mask bytes), and the ring is kTrunkDepth slots deep.
-template <bool MASK, bool RES = true>
+// A sparse residual (SPARSE) keeps the tile's packed codes, as they lie in
+// memory, in the code area and its keep words after the bit planes.
+template <bool MASK, bool RES = true, bool SPARSE = false>
 struct Slot {
   static constexpr int kSign = RES ? 2048 : 0;
   static constexpr int kMask = kSign + 256;  // (MASK only)
-  static constexpr int kScale = MASK ? kMask + 256 : kMask;  // (RES only)
+  static constexpr int kKeep = MASK ? kMask + 256 : kMask;  // (SPARSE only)
+  static constexpr int kScale = SPARSE ? kKeep + 256 : kKeep;  // (RES only)
   static constexpr int kBytes = kScale + (RES ? 256 : 0);
 };
 // Tiles in flight per warp in the trunk-only mode (small slots).
@@ -192,26 +209,78 @@ __device__ __forceinline__ void cp_async_wait() {
 }
 
 // RES = false (trunk only): the codes and scales are neither copied nor read.
-template <bool MASK, bool RES>
+// SPARSE: only the tile's c.nb packed code bytes are copied, as they lie.
+template <bool MASK, bool RES, bool SPARSE = false>
 __device__ __forceinline__ void copy_tile(uint32_t slot, const Cursor& c, int lane) {
-  if constexpr (RES) {
+  using SL = Slot<MASK, RES, SPARSE>;
+  if constexpr (RES && SPARSE) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if ((lane + 32 * j) * 16 < c.nb) cp_async16(slot + lane * 16 + 512 * j, c.code + 512 * j);
+    cp_async8(slot + SL::kKeep + lane * 8, c.keep);
+  } else if constexpr (RES) {
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int lo = j * 8 + (lane >> 2), ch = lane & 3;  // owner lane, its chunk
       cp_async16(slot + lo * 64 + (((ch + (lo >> 1)) & 3) << 4), c.code + 512 * j);
     }
   }
-  cp_async8(slot + Slot<MASK, RES>::kSign + lane * 8, c.sign);
-  if constexpr (MASK) cp_async8(slot + Slot<MASK, RES>::kMask + lane * 8, c.mask);
+  cp_async8(slot + SL::kSign + lane * 8, c.sign);
+  if constexpr (MASK) cp_async8(slot + SL::kMask + lane * 8, c.mask);
   if constexpr (RES) {
-    cp_async4(slot + Slot<MASK, RES>::kScale + lane * 8, c.scale);
-    cp_async4(slot + Slot<MASK, RES>::kScale + lane * 8 + 4, c.scale + 8);
+    cp_async4(slot + SL::kScale + lane * 8, c.scale);
+    cp_async4(slot + SL::kScale + lane * 8 + 4, c.scale + 8);
   }
 }
 
-template <bool MASK, bool RES>
-__device__ __forceinline__ void read_tile(Tile<MASK>& t, const uint8_t* slot, int lane) {
-  if constexpr (RES) {
+// Sparse residual: the lane's codes from the tile's packed stream.  Its
+// place in the stream is the count of kept codes of the lanes before it (a
+// warp scan of the keep-bit counts); each 4-channel word (row r0's 32
+// channels, then row r1's) takes the next popc(keep nibble) bytes, spread to
+// its kept channels by one byte permute whose selector comes from a 16-entry
+// table (sel_lut[n]: byte c from stream byte popc(n & ((1 << c) - 1)) if bit
+// c of n is set, else 0).  (Forming the 16 words independently, each from its
+// own popcount offset, measured slower: the reads of shared memory, not their
+// latency, bound this expansion.)
+__device__ __forceinline__ void expand_sparse(uint32_t (&q)[16], const uint8_t* slot, uint32_t k0,
+                                              uint32_t k1, int lane, const uint32_t* sel_lut) {
+  const int n = __popc(k0) + __popc(k1);
+  int incl = n;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  int pos = incl - n;
+  const uint32_t* cw = reinterpret_cast<const uint32_t*>(slot);
+  uint32_t lo = cw[pos >> 2], hi = cw[(pos >> 2) + 1];
+#pragma unroll
+  for (int R = 0; R < 2; ++R) {
+    const uint32_t kb = R ? k1 : k0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      // keep bits 8c + w of the word are channels 4w + c
+      const uint32_t nib = (((kb >> w) & 0x01010101u) * 0x01020408u) >> 24;
+      const uint32_t bytes = __funnelshift_r(lo, hi, (pos & 3) * 8);
+      q[4 * (w >> 1) + 2 * (w & 1) + R] = __byte_perm(bytes, 0u, sel_lut[nib]);
+      const int np = pos + __popc(nib);
+      if ((np >> 2) != (pos >> 2)) {
+        lo = hi;
+        hi = cw[(np >> 2) + 1];
+      }
+      pos = np;
+    }
+  }
+}
+
+template <bool MASK, bool RES, bool SPARSE = false>
+__device__ __forceinline__ void read_tile(Tile<MASK>& t, const uint8_t* slot, int lane,
+                                          const uint32_t* sel_lut = nullptr) {
+  using SL = Slot<MASK, RES, SPARSE>;
+  if constexpr (RES && SPARSE) {
+    const uint2 kv = *reinterpret_cast<const uint2*>(slot + SL::kKeep + lane * 8);
+    expand_sparse(t.q, slot, kv.x, kv.y, lane, sel_lut);
+  } else if constexpr (RES) {
     const uint8_t* cb = slot + lane * 64;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -222,16 +291,16 @@ __device__ __forceinline__ void read_tile(Tile<MASK>& t, const uint8_t* slot, in
       t.q[4 * j + 3] = v.w;
     }
   }
-  const uint2 sv = *reinterpret_cast<const uint2*>(slot + Slot<MASK, RES>::kSign + lane * 8);
+  const uint2 sv = *reinterpret_cast<const uint2*>(slot + SL::kSign + lane * 8);
   t.s[0] = sv.x;
   t.s[1] = sv.y;
   if constexpr (MASK) {
-    const uint2 mv = *reinterpret_cast<const uint2*>(slot + Slot<MASK, RES>::kMask + lane * 8);
+    const uint2 mv = *reinterpret_cast<const uint2*>(slot + SL::kMask + lane * 8);
     t.m[0] = mv.x;
     t.m[1] = mv.y;
   }
   if constexpr (RES) {
-    const float2 cv = *reinterpret_cast<const float2*>(slot + Slot<MASK, RES>::kScale + lane * 8);
+    const float2 cv = *reinterpret_cast<const float2*>(slot + SL::kScale + lane * 8);
     t.c[0] = cv.x;
     t.c[1] = cv.y;
   }
@@ -452,9 +521,12 @@ __device__ __forceinline__ void split_activations(const Params& p, const uint32_
 
 // RES = false: the trunk-only mode (the residual path skipped: no codes or
 // scales read, no residual MMAs, outlier channels take the trunk weight).
-template <bool MASK, bool EMIT, bool FUSED, int D, bool RES>
+// SPARSE: the weight is in SQ_LAYOUT_TILES_SPARSE (packed kept codes).
+template <bool MASK, bool EMIT, bool FUSED, int D, bool RES, bool SPARSE>
 __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
+  using SL = Slot<MASK, RES, SPARSE>;
   extern __shared__ __align__(16) uint8_t smem[];
+  __shared__ uint32_t sel_lut[16];  // byte-permute selectors of the sparse expansion
   // shared: part [kWarps][2 slots][16 rows][M tokens] float4 | omask[nw] u32 |
   // obase[nw] i32 | fused-mode buffers | ring [kWarps][D slots]
   float4* part_s = reinterpret_cast<float4*>(smem);
@@ -481,18 +553,32 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
     cur.sign = p.sign + lt * 2;
     cur.mask = MASK ? p.mask + lt * 2 : p.sign;
     cur.scale = p.scale + (int64_t)t0 * 16 + gid;
+    if constexpr (SPARSE) {
+      cur.keep = p.keep + lt * 2;
+      cur.nbytes = p.nbytes + t0;
+      cur.t = t0;
+      cur.T = p.T;
+      cur.nb = t0 < p.T ? __ldg(cur.nbytes) : 0;
+    }
   }
-  uint8_t* ring_w = smem + p.off_ring + warp * D * Slot<MASK, RES>::kBytes;
+  if (SPARSE && threadIdx.x < 16) {
+    const uint32_t n = threadIdx.x;
+    uint32_t sel = 0;
+    for (int c = 0; c < 4; ++c)
+      sel |= (((n >> c) & 1u) ? (uint32_t)__popc(n & ((1u << c) - 1u)) : 4u) << (4 * c);
+    sel_lut[n] = sel;
+  }
+  uint8_t* ring_w = smem + p.off_ring + warp * D * SL::kBytes;
   const uint32_t ring_u = smem_u32(ring_w);
   constexpr int kEarly = FUSED ? kDepthEarly : D;
 #pragma unroll
   for (int d = 0; d < kEarly; ++d) {  // one commit group per tile, empty past the range
-    if (t0 + d < t1) copy_tile<MASK, RES>(ring_u + d * Slot<MASK, RES>::kBytes, cur, lane);
+    if (t0 + d < t1) copy_tile<MASK, RES, SPARSE>(ring_u + d * SL::kBytes, cur, lane);
     cp_async_commit();
-    cur.advance();
+    cur.advance<SPARSE>();
   }
 
-  __syncthreads();  // omask zeroed
+  __syncthreads();  // omask zeroed (and the selector table written)
   auto add_outlier = [&](int i, int j, int jprev) {
     if (j >= 0 && j < p.K) {
       atomicOr(&omask[j >> 5], 1u << (j & 31));
@@ -521,9 +607,9 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
     split_activations(p, omask, xq_s, xo_s, sx_s, reinterpret_cast<float*>(smem + p.off_red), jv, jp);
 #pragma unroll
     for (int d = kEarly; d < D; ++d) {
-      if (t0 + d < t1) copy_tile<MASK, RES>(ring_u + d * Slot<MASK, RES>::kBytes, cur, lane);
+      if (t0 + d < t1) copy_tile<MASK, RES, SPARSE>(ring_u + d * SL::kBytes, cur, lane);
       cp_async_commit();
-      cur.advance();
+      cur.advance<SPARSE>();
     }
   }
 
@@ -557,7 +643,7 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
     cp_async_wait<D - 1>();  // this lane's copies of the tile have landed
     __syncwarp();             // ... and every lane's
     Tile<MASK> tl;
-    read_tile<MASK, RES>(tl, ring_w + slot_i * Slot<MASK, RES>::kBytes, lane);
+    read_tile<MASK, RES, SPARSE>(tl, ring_w + slot_i * SL::kBytes, lane, sel_lut);
     // activation codes of this lane's 32 channels for its MMA column
     uint32_t xw[8];
     {
@@ -664,9 +750,9 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
 
     // refill this slot with the tile D ahead, once no lane reads it
     __syncwarp();
-    if (t + D < t1) copy_tile<MASK, RES>(ring_u + slot_i * Slot<MASK, RES>::kBytes, cur, lane);
+    if (t + D < t1) copy_tile<MASK, RES, SPARSE>(ring_u + slot_i * SL::kBytes, cur, lane);
     cp_async_commit();
-    cur.advance();
+    cur.advance<SPARSE>();
     if (++slot_i == D) slot_i = 0;
 
     // end of a row block, or end of this warp's range
@@ -736,9 +822,9 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
   }
 }
 
-template <bool MASK, bool EMIT, bool FUSED, int D, bool RES = true>
+template <bool MASK, bool EMIT, bool FUSED, int D, bool RES = true, bool SPARSE = false>
 cudaError_t launch_one(const Params& p, int grid, int smem, bool pdl, cudaStream_t stream) {
-  auto* fn = k_linear_tc<MASK, EMIT, FUSED, D, RES>;
+  auto* fn = k_linear_tc<MASK, EMIT, FUSED, D, RES, SPARSE>;
   cudaError_t e = ensure_smem_attr((const void*)fn, smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -755,25 +841,26 @@ cudaError_t launch_one(const Params& p, int grid, int smem, bool pdl, cudaStream
 }
 
 template <bool MASK, bool FUSED, int D>
-cudaError_t launch_plain(const Params& p, bool res, int grid, int smem, bool pdl,
+cudaError_t launch_plain(const Params& p, bool res, bool sparse, int grid, int smem, bool pdl,
                          cudaStream_t stream) {
-  return res ? launch_one<MASK, false, FUSED, D, true>(p, grid, smem, pdl, stream)
-             : launch_one<MASK, false, FUSED, kTrunkDepth, false>(p, grid, smem, pdl, stream);
+  if (!res) return launch_one<MASK, false, FUSED, kTrunkDepth, false>(p, grid, smem, pdl, stream);
+  return sparse ? launch_one<MASK, false, FUSED, D, true, true>(p, grid, smem, pdl, stream)
+                : launch_one<MASK, false, FUSED, D, true, false>(p, grid, smem, pdl, stream);
 }
 
 // Non-accumulator launch with a ring depth chosen at run time among Ds.
 template <int D0, int... Ds>
-cudaError_t launch_depth(int depth, bool mask, bool fused, bool res, const Params& p, int grid,
-                         int smem, bool pdl, cudaStream_t stream) {
+cudaError_t launch_depth(int depth, bool mask, bool fused, bool res, bool sparse, const Params& p,
+                         int grid, int smem, bool pdl, cudaStream_t stream) {
   if (depth == D0 || sizeof...(Ds) == 0) {
     if (fused)
-      return mask ? launch_plain<true, true, D0>(p, res, grid, smem, pdl, stream)
-                  : launch_plain<false, true, D0>(p, res, grid, smem, pdl, stream);
-    return mask ? launch_plain<true, false, D0>(p, res, grid, smem, pdl, stream)
-                : launch_plain<false, false, D0>(p, res, grid, smem, pdl, stream);
+      return mask ? launch_plain<true, true, D0>(p, res, sparse, grid, smem, pdl, stream)
+                  : launch_plain<false, true, D0>(p, res, sparse, grid, smem, pdl, stream);
+    return mask ? launch_plain<true, false, D0>(p, res, sparse, grid, smem, pdl, stream)
+                : launch_plain<false, false, D0>(p, res, sparse, grid, smem, pdl, stream);
   }
   if constexpr (sizeof...(Ds) > 0)
-    return launch_depth<Ds...>(depth, mask, fused, res, p, grid, smem, pdl, stream);
+    return launch_depth<Ds...>(depth, mask, fused, res, sparse, p, grid, smem, pdl, stream);
   return cudaErrorInvalidValue;
 }
 
@@ -787,15 +874,18 @@ size_t linear_tc_part_bytes(int) {
 namespace {
 // Partial sums of one token: kWarps warps x 2 slots x 16 rows.
 constexpr int kSmemPartPerToken = kWarps * 2 * 16 * (int)sizeof(float4);
-// Largest dynamic shared memory of one CTA on sm_100 (227 KiB, opt-in).
-constexpr int kSmemMax = 227 * 1024;
+// Largest dynamic shared memory of one CTA on sm_100: 227 KiB (opt-in) less
+// the kernel's static shared memory.
+constexpr int kSmemMax = 227 * 1024 - 256;
 
 int outlier_table_bytes(const sq_packed_weight& w) { return (int)(tiles_cols(w.K) / 32) * 8; }
 int fused_token_bytes(const sq_packed_weight& w, int n_out) {
   return (int)tiles_cols(w.K) + (int)round_up(n_out, 4) * 4;
 }
-int ring_bytes(bool mask, int depth) {
-  return kWarps * depth * (mask ? Slot<true>::kBytes : Slot<false>::kBytes);
+int ring_bytes(bool mask, int depth, bool sparse = false) {
+  const int slot = sparse ? (mask ? Slot<true, true, true>::kBytes : Slot<false, true, true>::kBytes)
+                          : (mask ? Slot<true>::kBytes : Slot<false>::kBytes);
+  return kWarps * depth * slot;
 }
 int trunk_ring_bytes(bool mask) {
   return kWarps * kTrunkDepth * (mask ? Slot<true, false>::kBytes : Slot<false, false>::kBytes);
@@ -804,7 +894,8 @@ int trunk_ring_bytes(bool mask) {
 
 int linear_tc_fused_tokens(const sq_packed_weight& w, int n_out) {
   // counted with the shallow ring; the deep one is used when it fits
-  const int fixed = ring_bytes(w.mask_bits != nullptr, kShallow) + outlier_table_bytes(w) +
+  const int fixed = ring_bytes(w.mask_bits != nullptr, kShallow, w.layout == SQ_LAYOUT_TILES_SPARSE) +
+                    outlier_table_bytes(w) +
                     kCols * 4 + kWarps * kCols * 4 + 64;
   const int per = fused_token_bytes(w, n_out) + kSmemPartPerToken;
   const int m = (kSmemMax - fixed) / per;
@@ -816,7 +907,9 @@ cudaError_t launch_linear_tc(const sq_packed_weight& w, int M, const int8_t* xq,
                              float* y, int32_t* T_out, int32_t* R_out, void* workspace,
                              size_t part_bytes, int sm_count, int32_t* status, bool pdl,
                              bool trunk_only, cudaStream_t stream) {
-  if (M < 1 || M > kCols || w.layout != SQ_LAYOUT_TILES) return cudaErrorInvalidValue;
+  const bool sparse = w.layout == SQ_LAYOUT_TILES_SPARSE;
+  if (M < 1 || M > kCols || (w.layout != SQ_LAYOUT_TILES && !sparse)) return cudaErrorInvalidValue;
+  if (sparse && (!w.keep_bits || !w.res_bytes)) return cudaErrorInvalidValue;
   if (trunk_only && T_out) return cudaErrorInvalidValue;
   const bool fused = x != nullptr;
   if (fused && (T_out || M > linear_tc_fused_tokens(w, n_out))) return cudaErrorInvalidValue;
@@ -826,6 +919,8 @@ cudaError_t launch_linear_tc(const sq_packed_weight& w, int M, const int8_t* xq,
   p.mask = w.mask_bits;
   p.alpha = w.alpha;
   p.scale = w.res_scale;
+  p.keep = w.keep_bits;
+  p.nbytes = w.res_bytes;
   p.N = w.N;
   p.K = w.K;
   p.tpr = (int)(tiles_cols(w.K) / kTileK);
@@ -870,14 +965,20 @@ cudaError_t launch_linear_tc(const sq_packed_weight& w, int M, const int8_t* xq,
   p.off_ring = smem;
   // three tiles per warp above batch 2 where they fit, else two (the
   // accumulator mode, used to check the kernel, always takes two)
-  const int depth = (!emit && M > 2 && smem + ring_bytes(mask, kDeep) <= kSmemMax) ? kDeep : kShallow;
-  smem += trunk_only ? trunk_ring_bytes(mask) : ring_bytes(mask, depth);
+  const int depth =
+      (!emit && M > 2 && smem + ring_bytes(mask, kDeep, sparse) <= kSmemMax) ? kDeep : kShallow;
+  smem += trunk_only ? trunk_ring_bytes(mask) : ring_bytes(mask, depth, sparse);
   if (smem > kSmemMax) return cudaErrorInvalidValue;
   const int grid = (int)blocks;
-  if (emit)
+  if (emit) {
+    if (sparse)
+      return mask ? launch_one<true, true, false, kShallow, true, true>(p, grid, smem, pdl, stream)
+                  : launch_one<false, true, false, kShallow, true, true>(p, grid, smem, pdl, stream);
     return mask ? launch_one<true, true, false, kShallow>(p, grid, smem, pdl, stream)
                 : launch_one<false, true, false, kShallow>(p, grid, smem, pdl, stream);
-  return launch_depth<kDeep, kShallow>(depth, mask, fused, !trunk_only, p, grid, smem, pdl, stream);
+  }
+  return launch_depth<kDeep, kShallow>(depth, mask, fused, !trunk_only, sparse, p, grid, smem, pdl,
+                                       stream);
 }
 
 }  // namespace sq

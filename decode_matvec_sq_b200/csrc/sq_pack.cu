@@ -206,7 +206,154 @@ __global__ void __launch_bounds__(kPackRows) k_pack(const float* __restrict__ W,
   if (valid && nonfinite) set_status(status, SQ_ERR_NONFINITE);
 }
 
+// ---- sparse residual (SQ_LAYOUT_TILES_SPARSE) -----------------------------------
+// m.lqnn.cn section 3.3: residual entries near zero are dropped and the rest
+// stored sparsely.  Over a tiled decomposition already written by k_pack
+// (sign / mask bits, alpha, dense codes): one CTA per (padded) row re-forms
+// r in binary64 exactly as k_pack does, finds theta_r = the rank-th smallest
+// |r| (rank = ceil(Ps*K/100)) by an MSB-first radix select on the binary64
+// bit patterns (non-negative doubles order like their bits), keeps |r| >
+// theta_r and re-quantizes every group from its kept entries.
+__global__ void __launch_bounds__(256) k_sparse_residual(const float* __restrict__ W, int N, int K,
+                                                         int Ps, sq_packed_weight pw) {
+  __shared__ uint32_t hist[256];
+  __shared__ unsigned long long s_prefix;
+  __shared__ uint32_t s_remaining;
+  const int row = blockIdx.x;
+  const int tpr = (int)(tiles_cols(K) / kTileK);
+  const int nw = tpr * 4;  // 32-channel words of a padded row
+  if (row >= N) {
+    // pad rows of the tiled layout: nothing kept (their codes and scales are 0)
+    for (int w = threadIdx.x; w < nw; w += blockDim.x) pw.keep_bits[tiled_bits_word(row, w, tpr)] = 0u;
+    return;
+  }
+  const float alpha = pw.alpha[row];
+  const float* wr = W + (int64_t)row * K;
+  auto resid = [&](int j) -> double {
+    const float v = __ldg(wr + j);
+    bool m = true;
+    if (pw.mask_bits) m = (pw.mask_bits[tiled_bits_word(row, j >> 5, tpr)] >> tiled_bit_of(j & 31)) & 1u;
+    const double tr = m ? (v >= 0.0f ? (double)alpha : -(double)alpha) : 0.0;
+    return (double)v - tr;
+  };
+  if (threadIdx.x == 0) {
+    s_prefix = 0ull;
+    s_remaining = (uint32_t)(((int64_t)Ps * K + 99) / 100);
+  }
+  unsigned long long hi_mask = 0ull;
+  for (int pass = 0; pass < 8; ++pass) {
+    const int shift = 56 - 8 * pass;
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0u;
+    __syncthreads();
+    const unsigned long long prefix = s_prefix;
+    for (int j = threadIdx.x; j < K; j += blockDim.x) {
+      const unsigned long long key = (unsigned long long)__double_as_longlong(fabs(resid(j)));
+      if ((key & hi_mask) == prefix) atomicAdd(&hist[(key >> shift) & 0xFFull], 1u);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      uint32_t rem = s_remaining, cum = 0;
+      int b = 0;
+      for (; b < 255; ++b) {
+        if (cum + hist[b] >= rem) break;
+        cum += hist[b];
+      }
+      s_remaining = rem - cum;
+      s_prefix = prefix | ((unsigned long long)b << shift);
+    }
+    hi_mask |= 0xFFull << shift;
+    __syncthreads();
+  }
+  const double theta = __longlong_as_double((long long)s_prefix);
+  // groups of 128 channels: scale from the kept entries, codes of the kept ones
+  for (int g = threadIdx.x; g < tpr; g += blockDim.x) {
+    const int c0 = g * kTileK, c1 = min(K, c0 + kTileK);
+    double a = 0.0;
+    for (int j = c0; j < c1; ++j) {
+      const double r = resid(j);
+      if (fabs(r) > theta) a = fabs(r) > a ? fabs(r) : a;
+    }
+    const float sc = (float)(a / 127.0);
+    pw.res_scale[tiled_scale_index(row, g, tpr)] = sc;
+    for (int j0 = c0; j0 < c0 + kTileK; j0 += 4) {
+      uint32_t word = 0;
+      for (int j = j0; j < j0 + 4 && j < c1; ++j) {
+        const double r = resid(j);
+        const int q = fabs(r) > theta ? quantize_q(r, sc) : 0;
+        word |= ((uint32_t)(uint8_t)(int8_t)q) << (8 * (j - j0));
+      }
+      *reinterpret_cast<uint32_t*>(pw.res_q + tiled_code_offset(row, j0, tpr)) = word;
+    }
+  }
+  // keep bits, tiled order
+  for (int w = threadIdx.x; w < nw; w += blockDim.x) {
+    uint32_t bits = 0;
+    for (int b = 0; b < 32; ++b) {
+      const int j = 32 * w + b;
+      if (j < K && fabs(resid(j)) > theta) bits |= 1u << b;
+    }
+    pw.keep_bits[tiled_bits_word(row, w, tpr)] = tiled_bits_from_row_order(bits);
+  }
+}
+
+// Packs each tile's kept codes at the start of its 2048-byte slot, one warp
+// per tile: lane L in order, row r0's then row r1's kept codes in ascending
+// channel order, zero padded to 16 bytes; res_bytes[t] = the padded size.
+// Every lane reads its 64 dense bytes before any lane writes (in place).
+__global__ void __launch_bounds__(256) k_sparse_compact(int T, sq_packed_weight pw) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * 8 + warp;
+  if (t >= T) return;
+  const int64_t lt = (int64_t)t * 32 + lane;
+  const uint32_t k0 = pw.keep_bits[lt * 2], k1 = pw.keep_bits[lt * 2 + 1];
+  uint32_t q[16];
+  const uint4* src = reinterpret_cast<const uint4*>(pw.res_q + lt * 64);
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    const uint4 v = src[m];
+    q[4 * m] = v.x;
+    q[4 * m + 1] = v.y;
+    q[4 * m + 2] = v.z;
+    q[4 * m + 3] = v.w;
+  }
+  const int n = __popc(k0) + __popc(k1);
+  int incl = n;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  const int total = __shfl_sync(0xffffffffu, incl, 31);
+  __syncwarp();
+  uint8_t* dst = reinterpret_cast<uint8_t*>(pw.res_q) + (int64_t)t * 2048;
+  int pos = incl - n;
+  for (int R = 0; R < 2; ++R) {
+    const uint32_t kb = R ? k1 : k0;
+    for (int w = 0; w < 8; ++w) {
+      // channels 4w .. 4w+3 of the lane's 32: keep bits 8c + w
+      const uint32_t nib = (((kb >> w) & 0x01010101u) * 0x01020408u) >> 24;
+      const uint32_t word = q[4 * (w >> 1) + 2 * (w & 1) + R];
+      for (int c = 0; c < 4; ++c)
+        if ((nib >> c) & 1u) dst[pos++] = (uint8_t)(word >> (8 * c));
+    }
+  }
+  const int padded = (total + 15) & ~15;
+  for (int b = total + lane; b < padded; b += 32) dst[b] = 0;
+  if (lane == 0) pw.res_bytes[t] = padded;
+}
+
 }  // namespace
+
+cudaError_t launch_sparsify_residual(const float* W, int N, int K, int Ps, const sq_packed_weight& pw,
+                                     cudaStream_t stream) {
+  const int64_t rows = tiles_rows(N);
+  k_sparse_residual<<<(int)rows, 256, 0, stream>>>(W, N, K, Ps, pw);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int64_t T = rows / kTileRows * (tiles_cols(K) / kTileK);
+  k_sparse_compact<<<(int)ceil_div(T, 8), 256, 0, stream>>>((int)T, pw);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_decompose_pack(const float* W, int N, int K, int P, const sq_packed_weight& pw,
                                   int32_t* status, cudaStream_t stream) {

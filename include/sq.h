@@ -56,7 +56,8 @@ typedef enum {
 #define SQ_LAUNCH_PDL 1u
 #define SQ_TRUNK_ONLY 2u
 /* SQ_TRUNK_ONLY (sq_linear, sq_quantize_linear, sq_linear_noalloc; weights in
- * SQ_LAYOUT_TILES only, else SQ_ERR_INVALID_ARG): the residual path is
+ * SQ_LAYOUT_TILES or SQ_LAYOUT_TILES_SPARSE only, else SQ_ERR_INVALID_ARG):
+ * the residual path is
  * skipped (m.lqnn.cn section 3.3: the 1-bit trunk first, the residual added
  * on demand; a request that tolerates a rougher answer skips it).  The
  * residual codes and scales are not read:
@@ -75,6 +76,7 @@ typedef enum {
 /* Packed-weight layouts (sq_packed_weight.layout). */
 #define SQ_LAYOUT_ROWS 0
 #define SQ_LAYOUT_TILES 1
+#define SQ_LAYOUT_TILES_SPARSE 2
 
 /*
  * Packed weight of one linear layer (N output rows, K input channels).
@@ -109,11 +111,25 @@ typedef enum {
  *   sign_stride = K128/32, res_stride = K128, scale_stride = K128/128
  *   (the padded row lengths).  K <= 131072.
  *
+ * SQ_LAYOUT_TILES_SPARSE (G = 128 only; written by sq_decompose_pack_sparse):
+ * SQ_LAYOUT_TILES with a sparse residual (m.lqnn.cn section 3.3: residual
+ * entries near zero are dropped and the rest stored sparsely).  Two arrays
+ * more, and res_q holds each tile's kept codes only:
+ *   keep_bits same shape and bit order as sign_bits: 1 = the residual entry
+ *             is kept, 0 = dropped (its code is 0)
+ *   res_q     tile t's slot of 2048 bytes at byte 2048*t holds the tile's
+ *             kept codes, packed: lane L = 0..31 in order, within a lane row
+ *             r0's 32 channels then row r1's, ascending channel; zero padded
+ *             to a multiple of 16 bytes; the rest of the slot is unused
+ *   res_bytes [T] i32, T = (N16/16)*(K128/128): the padded byte count of
+ *             each tile's kept codes (what the decode kernel reads)
+ * Every other array is that of SQ_LAYOUT_TILES.
+ *
  * The arrays may live in one allocation carved by sq_packed_view().
  */
 typedef struct {
   int32_t N, K, group_size;  /* group_size G: 32, 64 or 128 */
-  int32_t layout;            /* SQ_LAYOUT_ROWS or SQ_LAYOUT_TILES */
+  int32_t layout;            /* SQ_LAYOUT_ROWS, SQ_LAYOUT_TILES or SQ_LAYOUT_TILES_SPARSE */
   int32_t sign_stride;       /* u32 words per row of sign_bits / mask_bits */
   int32_t res_stride;        /* bytes per row of res_q */
   int32_t scale_stride;      /* floats per row of res_scale */
@@ -122,6 +138,8 @@ typedef struct {
   float *alpha;
   int8_t *res_q;
   float *res_scale;
+  uint32_t *keep_bits;       /* SQ_LAYOUT_TILES_SPARSE only, else NULL */
+  int32_t *res_bytes;        /* SQ_LAYOUT_TILES_SPARSE only, else NULL */
 } sq_packed_weight;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -160,6 +178,26 @@ sq_status sq_packed_view(void *base, int32_t N, int32_t K, int32_t group_size,
  */
 sq_status sq_decompose_pack(const float *W, int32_t N, int32_t K, int32_t trunk_percent,
                             const sq_packed_weight *out, int32_t *dev_status, void *stream);
+
+/*
+ * sq_decompose_pack with a sparse residual, into SQ_LAYOUT_TILES_SPARSE
+ * (m.lqnn.cn section 3.3: a small threshold zeroes the residual entries
+ * near zero, typically 50-70 % of them, and the residual is stored sparsely;
+ * the page gives no threshold rule).  Trunk, alpha and residual r as in
+ * sq_decompose_pack; then, per row, theta_r = the ceil(Ps*K/100)-th smallest
+ * |r| over the row's K channels (binary64; nearest rank, as the trunk
+ * threshold) and an entry is kept iff |r| > theta_r (ties dropped); group
+ * scales come from the kept entries only (s = float(max kept |r| / 127),
+ * 0 for a group with none kept) and a kept entry's code is
+ * clip(round_half_away(r / s), +-127).
+ *   residual_percent  Ps, 1..99
+ *   out               strides and pointers as from sq_packed_view() with
+ *                     layout SQ_LAYOUT_TILES_SPARSE; written in full.
+ * Non-finite W sets SQ_ERR_NONFINITE in dev_status.
+ */
+sq_status sq_decompose_pack_sparse(const float *W, int32_t N, int32_t K, int32_t trunk_percent,
+                                   int32_t residual_percent, const sq_packed_weight *out,
+                                   int32_t *dev_status, void *stream);
 
 /*
  * Outlier calibration (m.lqnn.cn section 2.2: detect the outlier channels once,
@@ -203,7 +241,7 @@ size_t sq_linear_workspace_bytes(const sq_packed_weight *w, int32_t M);
  * kernel; the outlier channels of section 2.2 at full precision).
  *   w           packed weight (device arrays)
  *   xq, sx, x_out, idx, n_out   as written by sq_quantize_act
- *   M           tokens, M >= 1.  A weight in SQ_LAYOUT_TILES runs on the
+ *   M           tokens, M >= 1.  A weight in SQ_LAYOUT_TILES (or _SPARSE) runs on the
  *               tensor cores (INT8 MMAs for the residual codes and for the
  *               trunk bits expanded to 0/-1 bytes), in passes of up to 8
  *               tokens; SQ_LAYOUT_ROWS runs on the CUDA cores (dp4a), in
@@ -238,7 +276,7 @@ sq_status sq_linear_accumulators(const sq_packed_weight *w, const int8_t *xq, co
 /*
  * The activation split and the linear layer in one kernel (m.lqnn.cn
  * sections 2.2, 2.3 and 3.3: the split, the two products and their sum in a
- * single fused step).  For a weight in SQ_LAYOUT_TILES.
+ * single fused step).  For a weight in SQ_LAYOUT_TILES or SQ_LAYOUT_TILES_SPARSE.
  *   x           [M][K] f32 activations, device
  *   idx, n_out  outlier channels, strictly ascending in [0, K) (checked on
  *               the device: a violation sets SQ_ERR_INVALID_ARG)
@@ -279,7 +317,7 @@ size_t sq_quantize_linear_workspace_bytes(const sq_packed_weight *w, int32_t M, 
 /*
  * Tokens per launch of sq_quantize_linear's fused kernel for this weight and
  * outlier count (1..8; 0 if not even one token fits, or for an invalid
- * weight or a weight not in SQ_LAYOUT_TILES).
+ * weight or a weight in SQ_LAYOUT_ROWS).
  */
 int32_t sq_quantize_linear_tokens_per_pass(const sq_packed_weight *w, int32_t n_out);
 

@@ -73,8 +73,13 @@ def unpack(pw: "sq.PackedWeight", rows=None) -> dict:
     sign_flat = pw.sign_bits().reshape(-1)
     scale_flat = pw.res_scale().reshape(-1)
     alpha_all = pw._arr("alpha", torch.float32, (pw.rows,))
-    q = _gather(code_flat, _tiled_code_offsets(rows, K128))
     wi = _tiled_word_index(rows, nwords)
+    keep = None
+    if pw.layout == sq.SQ_LAYOUT_TILES_SPARSE:
+        q, nbytes_ok = _unpack_sparse_codes(pw, rows, K128)
+        keep = _to_row_bit_order(_gather(pw.keep_bits().reshape(-1), wi).view(np.uint32))
+    else:
+        q = _gather(code_flat, _tiled_code_offsets(rows, K128))
     sign = _to_row_bit_order(_gather(sign_flat, wi).view(np.uint32))
     mask = None
     if pw.with_mask:
@@ -83,13 +88,61 @@ def unpack(pw: "sq.PackedWeight", rows=None) -> dict:
     si = ((rows[:, None] >> 4) * tpr + np.arange(tpr)[None, :]) * 16 + (rows[:, None] & 15)
     s = _gather(scale_flat, si)
     alpha = _gather(alpha_all, rows)
-    return {"sign": sign, "mask": mask, "alpha": alpha, "q": q, "s": s}
+    out = {"sign": sign, "mask": mask, "alpha": alpha, "q": q, "s": s}
+    if keep is not None:
+        out["keep"] = keep
+        out["res_bytes_ok"] = nbytes_ok
+    return out
+
+
+def _unpack_sparse_codes(pw, rows: np.ndarray, K128: int):
+    """Codes [n][K128] of the given rows from SQ_LAYOUT_TILES_SPARSE, as
+    include/sq.h describes it: tile t's slot at byte 2048*t holds its kept
+    codes packed lane by lane (lane L = 4*(row%8) + (channel%128)/32), within
+    a lane row r0's 32 channels then row r1's in ascending channel order; the
+    keep words are in the sign-bit layout.  Also whether res_bytes[t] is the
+    packed size rounded up to 16 for every tile read."""
+    tpr = K128 // 128
+    rb = np.unique(rows >> 4)
+    tiles = (rb[:, None] * tpr + np.arange(tpr)[None, :]).reshape(-1)           # [nt]
+    keep_flat = pw.keep_bits().reshape(-1)
+    lanes = np.arange(32)
+    kw = _gather(keep_flat, (tiles[:, None, None] * 32 + lanes[None, :, None]) * 2
+                 + np.arange(2)[None, None, :]).view(np.uint32)                  # [nt][32][2]
+    j = np.arange(32)
+    bitpos = (8 * (j % 4) + j // 4).astype(np.uint32)
+    kept = ((kw[:, :, :, None] >> bitpos[None, None, None, :]) & 1).astype(np.int64)  # [nt][32][2][32]
+    kept = kept.reshape(len(tiles), 32, 64)                                       # stream order
+    counts = kept.sum(axis=2)                                                     # [nt][32]
+    start = np.cumsum(counts, axis=1) - counts                                    # exclusive
+    byte_ix = start[:, :, None] + np.cumsum(kept, axis=2) - 1                    # [nt][32][64]
+    packed = _gather(pw.res_q().reshape(-1),
+                     tiles[:, None] * 2048 + np.arange(2048)[None, :])           # [nt][2048]
+    vals = np.take_along_axis(packed, np.clip(byte_ix.reshape(len(tiles), 2048), 0, 2047), axis=1)
+    vals = np.where(kept.astype(bool), vals.reshape(len(tiles), 32, 64), 0).astype(np.int8)
+    res_bytes = pw.res_bytes().cpu().numpy()[tiles]
+    nbytes_ok = bool(np.all(res_bytes == (counts.sum(axis=1) + 15) // 16 * 16))
+    # lane L, stream position R*32 + j -> row 8R + L//4, channel 32*(L%4) + j of the tile
+    blk = np.zeros((len(tiles), 16, 128), np.int8)
+    L = lanes[:, None, None]
+    R = np.arange(2)[None, :, None]
+    jj = j[None, None, :]
+    rr = (8 * R + L // 4) + 0 * jj                                                # [32][2][32]
+    cc = (32 * (L % 4) + jj) + 0 * R
+    blk[:, rr.reshape(-1), cc.reshape(-1)] = vals.reshape(len(tiles), 64 * 32)
+    tile_pos = {int(t): i for i, t in enumerate(tiles)}
+    q = np.zeros((len(rows), K128), np.int8)
+    for n, r in enumerate(rows):
+        for g in range(tpr):
+            q[n, 128 * g:128 * g + 128] = blk[tile_pos[int((r >> 4) * tpr + g)], r & 15]
+    return q, nbytes_ok
 
 
 def pad_rows_are_zero(pw: "sq.PackedWeight") -> bool:
     """The tiled layout's rows N..roundup(N,16) hold only zeros."""
-    if pw.layout != sq.SQ_LAYOUT_TILES or pw.rows == pw.N:
+    if not pw.tiled or pw.rows == pw.N:
         return True
     u = unpack(pw, rows=np.arange(pw.N, pw.rows))
-    parts = [u["sign"], u["alpha"], u["q"], u["s"]] + ([u["mask"]] if pw.with_mask else [])
+    parts = [u["sign"], u["alpha"], u["q"], u["s"]] + ([u["mask"]] if pw.with_mask else []) + \
+        ([u["keep"]] if "keep" in u else [])
     return all(not np.asarray(a).view(np.uint8).any() for a in parts)
