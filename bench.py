@@ -499,6 +499,13 @@ def layer_cases(workload: str):
     if workload == "threshold":
         L = wl.config4()
         return [("4096->14336 threshold trunk P=60", L, 1, -(-2 * L2_BYTES // L.packed_bytes))]
+    if workload == "asym":
+        out = []
+        for mid in range(4):
+            L = wl.config2_layer(0, mid)
+            out.append((f"{L.name.split('.')[-1]} {L.K}->{L.N} asymmetric residual",
+                        L.with_(residual_percent=-1), 1, -(-2 * L2_BYTES // L.packed_bytes)))
+        return out
     if workload == "sparse":
         out = []
         for Ps in (50, 60, 70):
@@ -559,9 +566,12 @@ def time_layer_case(L, M, copies, trunk, st, device, warmup, reps):
     import decode_matvec_sq_b200 as sq
     import synth.device as sdev
     W = sdev.fill_weights(L, torch.empty(L.N, L.K, device=device))
-    Ps = getattr(L, "residual_percent", None)
-    if Ps:
+    Ps = getattr(L, "residual_percent", 0)
+    if Ps > 0:
         pw = sq.decompose_pack_sparse(W, Ps, trunk_percent=L.trunk_percent, status=st)
+    elif Ps < 0:  # asymmetric residual groups
+        pw = sq.decompose_pack(W, trunk_percent=L.trunk_percent, layout=sq.SQ_LAYOUT_TILES_ASYM,
+                               status=st)
     else:
         pw = sq.decompose_pack(W, trunk_percent=L.trunk_percent, status=st)
     del W
@@ -584,7 +594,12 @@ def time_layer_case(L, M, copies, trunk, st, device, warmup, reps):
     for _ in range(warmup):
         launch()
     ms = _time_calls(launch, reps) / calls
-    wbytes = trunk_weight_bytes(L) if trunk else (sparse_weight_bytes(pw) if Ps else linear_weight_bytes(L))
+    if trunk:
+        wbytes = trunk_weight_bytes(L)
+    elif Ps > 0:
+        wbytes = sparse_weight_bytes(pw)
+    else:  # (an asymmetric residual adds its zero-points: 4 bytes per group)
+        wbytes = linear_weight_bytes(L) + (4 * pw.rows * pw.view.scale_stride if Ps < 0 else 0)
     nbytes = wbytes + M * (4 * L.K + 4 * L.N) + 4 * L.n_out
     launches = _fused_launches(pw, M, L)
     del pws, pw, ws
@@ -717,6 +732,9 @@ def run_layers(args, world, rank, local):
                           "W Laplace(0,0.02), x N(0,1) with 0.5% channels x30",
              "trunk": "trunk-only mode (residual path skipped) of the 7B-shaped stack's four "
                       "linears, batch 1, W Laplace(0,0.02), x N(0,1) with 0.5% channels x30",
+             "asym": "asymmetric residual groups (own min/max, scale, zero-point) on the "
+                     "7B-shaped stack's four linears, batch 1, W Laplace(0,0.02), "
+                     "x N(0,1) with 0.5% channels x30",
              "sparse": "sparse residual (per-row Ps-th percentile of |r| dropped, Ps 50/60/70) on "
                        "the 7B-shaped stack's four linears, batch 1, W Laplace(0,0.02), "
                        "x N(0,1) with 0.5% channels x30; GB/s on the bytes the kernel reads"}
@@ -915,7 +933,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["sq", "reference"], default="sq")
     ap.add_argument("--layers", type=int, default=32)
     ap.add_argument("--workload", choices=["decode", "prefill", "single", "mlp70b", "threshold",
-                                           "trunk", "sparse"],
+                                           "trunk", "sparse", "asym"],
                     default="decode",
                     help="decode: the 7B-shaped stack at batch 1 (default); prefill: "
                          "2048 tokens x 4096 -> 14336 on the tcgen05 kernel; single, mlp70b, "
@@ -940,7 +958,7 @@ def main(argv=None):
         return run_reference(args, world, rank)
     if args.workload == "prefill":
         return run_prefill(args, world, rank, local)
-    if args.workload in ("single", "mlp70b", "threshold", "trunk", "sparse"):
+    if args.workload in ("single", "mlp70b", "threshold", "trunk", "sparse", "asym"):
         return run_layers(args, world, rank, local)
     return run_gpu(args, world, rank, local)
 

@@ -26,6 +26,7 @@ SQ_TRUNK_ONLY = 2
 SQ_LAYOUT_ROWS = 0
 SQ_LAYOUT_TILES = 1
 SQ_LAYOUT_TILES_SPARSE = 2
+SQ_LAYOUT_TILES_ASYM = 3
 
 STATUS = {
     0: "SQ_OK", 1: "SQ_ERR_INVALID_ARG", 2: "SQ_ERR_SHAPE", 3: "SQ_ERR_ALIGN",
@@ -50,6 +51,7 @@ class SqPackedWeight(ctypes.Structure):
         ("sign_bits", ctypes.c_void_p), ("mask_bits", ctypes.c_void_p),
         ("alpha", ctypes.c_void_p), ("res_q", ctypes.c_void_p), ("res_scale", ctypes.c_void_p),
         ("keep_bits", ctypes.c_void_p), ("res_bytes", ctypes.c_void_p),
+        ("res_zero", ctypes.c_void_p),
     ]
 
 
@@ -74,6 +76,8 @@ def lib():
         "sq_packed_view": ([vp, i32, i32, i32, i32, i32, pw], ctypes.c_int),
         "sq_decompose_pack": ([vp, i32, i32, i32, pw, vp, vp], ctypes.c_int),
         "sq_decompose_pack_sparse": ([vp, i32, i32, i32, i32, pw, vp, vp], ctypes.c_int),
+        "sq_residual_errors_scratch_bytes": ([i32], sz),
+        "sq_residual_errors": ([vp, pw, vp, vp, sz, vp, vp], ctypes.c_int),
         "sq_calibrate_outliers": ([vp, i32, i32, i32, vp, vp, vp], ctypes.c_int),
         "sq_quantize_act": ([vp, i32, i32, vp, i32, vp, vp, vp, vp, u32, vp], ctypes.c_int),
         "sq_linear_workspace_bytes": ([pw, i32], sz),
@@ -148,7 +152,7 @@ class PackedWeight:
 
     @property
     def tiled(self) -> bool:
-        return self.layout in (SQ_LAYOUT_TILES, SQ_LAYOUT_TILES_SPARSE)
+        return self.layout in (SQ_LAYOUT_TILES, SQ_LAYOUT_TILES_SPARSE, SQ_LAYOUT_TILES_ASYM)
 
     @property
     def rows(self) -> int:
@@ -186,6 +190,13 @@ class PackedWeight:
     def res_scale(self):
         import torch
         return self._arr("res_scale", torch.float32, (self.rows, self.view.scale_stride))
+
+    def res_zero(self):
+        """Zero-points of the asymmetric residual, indexed like res_scale."""
+        import torch
+        if self.layout != SQ_LAYOUT_TILES_ASYM:
+            return None
+        return self._arr("res_zero", torch.int32, (self.rows, self.view.scale_stride))
 
     def keep_bits(self):
         import torch
@@ -247,6 +258,33 @@ def decompose_pack_sparse(W, residual_percent: int, trunk_percent: int = -1,
                                        ctypes.byref(out.view), _ptr(status), _stream(stream)),
         "sq_decompose_pack_sparse")
     return out
+
+
+def residual_errors(W, pw: PackedWeight, status=None, stream=None):
+    """(err_split, err_plain): sum over the layer of (W - What)^2 for the
+    packed weight and for plain symmetric INT8 groups of W (binary64, on the
+    device; include/sq.h sq_residual_errors).  Reads the two numbers back."""
+    import torch
+    err = torch.zeros(2, dtype=torch.float64, device=W.device)
+    nb = int(lib().sq_residual_errors_scratch_bytes(pw.N))
+    scratch = torch.empty(nb, dtype=torch.uint8, device=W.device)
+    _ck(lib().sq_residual_errors(_ptr(W), ctypes.byref(pw.view), _ptr(err), _ptr(scratch), nb,
+                                 _ptr(status), _stream(stream)), "sq_residual_errors")
+    e = err.cpu().tolist()
+    return e[0], e[1]
+
+
+def decompose_pack_auto(W, trunk_percent: int = -1, layout: int = None, status=None):
+    """The split with the per-layer fallback (m.lqnn.cn s2.3, last paragraph;
+    the rule of include/sq.h sq_residual_errors): when plain INT8 groups
+    reconstruct W at least as well as the split, the layer is packed with an
+    empty trunk (trunk_percent = 100), i.e. as plain INT8.  Returns
+    (packed weight, fell_back)."""
+    pw = decompose_pack(W, trunk_percent=trunk_percent, layout=layout, status=status)
+    e_split, e_plain = residual_errors(W, pw, status=status)
+    if e_plain <= e_split:
+        return decompose_pack(W, trunk_percent=100, layout=layout, status=status), True
+    return pw, False
 
 
 def calibrate_outliers(X, k: int, out=None, status=None, stream=None):

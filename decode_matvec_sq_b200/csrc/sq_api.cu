@@ -91,9 +91,12 @@ sq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? SQ_OK : SQ_ERR_CU
 constexpr int32_t kMaxTiledK = 131072;
 
 bool known_layout(int32_t layout) {
-  return layout == SQ_LAYOUT_ROWS || layout == SQ_LAYOUT_TILES || layout == SQ_LAYOUT_TILES_SPARSE;
+  return layout == SQ_LAYOUT_ROWS || layout == SQ_LAYOUT_TILES || layout == SQ_LAYOUT_TILES_SPARSE ||
+         layout == SQ_LAYOUT_TILES_ASYM;
 }
-bool tiled(int32_t layout) { return layout == SQ_LAYOUT_TILES || layout == SQ_LAYOUT_TILES_SPARSE; }
+bool tiled(int32_t layout) {
+  return layout == SQ_LAYOUT_TILES || layout == SQ_LAYOUT_TILES_SPARSE || layout == SQ_LAYOUT_TILES_ASYM;
+}
 
 bool valid_layout(int32_t layout, int32_t G, int32_t K) {
   if (layout == SQ_LAYOUT_ROWS) return true;
@@ -125,6 +128,10 @@ sq_status check_weight(const sq_packed_weight* w) {
     if (!w->keep_bits || !w->res_bytes) return SQ_ERR_INVALID_ARG;
     if (!aligned16(w->keep_bits) || !aligned16(w->res_bytes)) return SQ_ERR_ALIGN;
   }
+  if (w->layout == SQ_LAYOUT_TILES_ASYM) {
+    if (!w->res_zero) return SQ_ERR_INVALID_ARG;
+    if (!aligned16(w->res_zero)) return SQ_ERR_ALIGN;
+  }
   if (w->sign_stride != sign_stride_of(w->K, w->layout) ||
       w->res_stride != res_stride_of(w->K, w->layout) ||
       w->scale_stride != scale_stride_of(w->K, w->group_size, w->layout))
@@ -138,7 +145,7 @@ sq_status check_weight(const sq_packed_weight* w) {
 // Offsets of the five arrays inside one allocation, each 256-byte aligned.
 // alpha holds roundup(N, 8) (rows) or N16 (tiles) floats.
 struct Carve {
-  size_t sign, mask, alpha, res, scale, keep, count, total;
+  size_t sign, mask, alpha, res, scale, keep, count, zero, total;
 };
 
 Carve carve(int32_t N, int32_t K, int32_t G, int32_t with_mask, int32_t layout) {
@@ -155,11 +162,12 @@ Carve carve(int32_t N, int32_t K, int32_t G, int32_t with_mask, int32_t layout) 
   c.alpha = take((size_t)round_up(rows, 8) * 4);
   c.res = take((size_t)rows * res_stride_of(K, layout));
   c.scale = take((size_t)rows * scale_stride_of(K, G, layout) * 4);
-  c.keep = c.count = 0;
+  c.keep = c.count = c.zero = 0;
   if (layout == SQ_LAYOUT_TILES_SPARSE) {
     c.keep = take((size_t)rows * sign_stride_of(K, layout) * 4);
     c.count = take((size_t)tiles_of(N, K) * 4);
   }
+  if (layout == SQ_LAYOUT_TILES_ASYM) c.zero = take((size_t)rows * scale_stride_of(K, G, layout) * 4);
   c.total = off;
   return c;
 }
@@ -220,6 +228,7 @@ sq_status sq_packed_view(void* base, int32_t N, int32_t K, int32_t group_size, i
   const bool sparse = layout == SQ_LAYOUT_TILES_SPARSE;
   out->keep_bits = sparse ? reinterpret_cast<uint32_t*>(b + c.keep) : nullptr;
   out->res_bytes = sparse ? reinterpret_cast<int32_t*>(b + c.count) : nullptr;
+  out->res_zero = layout == SQ_LAYOUT_TILES_ASYM ? reinterpret_cast<int32_t*>(b + c.zero) : nullptr;
   return SQ_OK;
 }
 
@@ -265,6 +274,24 @@ sq_status sq_decompose_pack_sparse(const float* W, int32_t N, int32_t K, int32_t
   cudaError_t e = launch_decompose_pack(W, N, K, trunk_percent, dense, dev_status, s);
   if (e != cudaSuccess) return SQ_ERR_CUDA;
   return from_cuda(launch_sparsify_residual(W, N, K, residual_percent, *out, s));
+}
+
+size_t sq_residual_errors_scratch_bytes(int32_t N) {
+  return N < 1 ? 0 : (size_t)round_up(16 * (int64_t)N, 256);
+}
+
+sq_status sq_residual_errors(const float* W, const sq_packed_weight* w, double* err, void* scratch,
+                             size_t scratch_bytes, int32_t* dev_status, void* stream) {
+  if (!W || !err || !scratch) return SQ_ERR_INVALID_ARG;
+  sq_status st = check_weight(w);
+  if (st != SQ_OK) return st;
+  if (w->layout == SQ_LAYOUT_TILES_SPARSE) return SQ_ERR_INVALID_ARG;
+  if (scratch_bytes < sq_residual_errors_scratch_bytes(w->N)) return SQ_ERR_WORKSPACE;
+  if (!aligned16(W) || !aligned16(err) || !aligned16(scratch)) return SQ_ERR_ALIGN;
+  DeviceInfo d;
+  if ((st = check_device(&d)) != SQ_OK) return st;
+  return from_cuda(launch_residual_errors(W, *w, err, static_cast<double*>(scratch), dev_status,
+                                          static_cast<cudaStream_t>(stream)));
 }
 
 sq_status sq_calibrate_outliers(const float* X, int32_t T, int32_t K, int32_t k, int32_t* idx_out,

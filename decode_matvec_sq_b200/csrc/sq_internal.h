@@ -38,6 +38,11 @@ cudaError_t launch_decompose_pack(const float* W, int N, int K, int P, const sq_
 cudaError_t launch_sparsify_residual(const float* W, int N, int K, int Ps, const sq_packed_weight& pw,
                                      cudaStream_t stream);
 
+// Per-row squared reconstruction errors of w and of plain INT8 groups of W
+// into scratch[2N], then their sums in row order into err[2] (binary64).
+cudaError_t launch_residual_errors(const float* W, const sq_packed_weight& w, double* err,
+                                   double* scratch, int32_t* status, cudaStream_t stream);
+
 cudaError_t launch_calibrate(const float* X, int T, int K, int k, int32_t* idx_out,
                              int32_t* status, cudaStream_t stream);
 

@@ -66,6 +66,7 @@ struct Params {
   const float* scale;
   const uint32_t* keep;    // keep bits of a sparse residual (SQ_LAYOUT_TILES_SPARSE)
   const int32_t* nbytes;   // packed code bytes per tile (sparse)
+  const int32_t* zero;     // zero-points of an asymmetric residual (SQ_LAYOUT_TILES_ASYM)
   int N, K, tpr;    // rows, channels, tiles per row block
   int T;            // tiles = ceil(N / 16) * tpr
   int n_rb;         // row blocks = ceil(N / 16); CTA b owns [b*n_rb/grid, (b+1)*n_rb/grid)
@@ -133,6 +134,7 @@ struct Tile {
   uint32_t s[2];   // sign words of rows r0, r1
   uint32_t m[2];   // mask words (MASK only)
   float c[2];      // group scales of rows r0, r1
+  int z[2];        // zero-points of rows r0, r1 (asymmetric residual only)
 };
 
 // Streaming position of one lane: its part of the next tile to copy.
@@ -146,12 +148,14 @@ struct Cursor {
   const uint32_t* keep;
   const int32_t* nbytes;
   int nb, t, T;
-  template <bool SPARSE>
+  const int32_t* zero;   // asymmetric residual: the zero-point of row r0 (r1: + 8)
+  template <bool SPARSE, bool ASYM = false>
   __device__ __forceinline__ void advance() {
     code += 2048;
     sign += 64;
     mask += 64;
     scale += 16;
+    if constexpr (ASYM) zero += 16;
     if constexpr (SPARSE) {
       keep += 64;
       ++nbytes;
@@ -179,13 +183,15 @@ struct Cursor {
 // (then the 256 mask bytes), and the ring is kTrunkDepth slots deep.
 // A sparse residual (SPARSE) keeps the tile's packed codes, as they lie in
 // memory, in the code area and its keep words after the bit planes.
-template <bool MASK, bool RES = true, bool SPARSE = false>
+// An asymmetric residual (ASYM) keeps the lane's two zero-points after the scales.
+template <bool MASK, bool RES = true, bool SPARSE = false, bool ASYM = false>
 struct Slot {
   static constexpr int kSign = RES ? 2048 : 0;
   static constexpr int kMask = kSign + 256;  // (MASK only)
   static constexpr int kKeep = MASK ? kMask + 256 : kMask;  // (SPARSE only)
   static constexpr int kScale = SPARSE ? kKeep + 256 : kKeep;  // (RES only)
-  static constexpr int kBytes = kScale + (RES ? 256 : 0);
+  static constexpr int kZero = kScale + 256;  // (ASYM only)
+  static constexpr int kBytes = kScale + (RES ? 256 : 0) + (ASYM ? 256 : 0);
 };
 // Tiles in flight per warp in the trunk-only mode (small slots).
 constexpr int kTrunkDepth = 6;
@@ -210,9 +216,9 @@ __device__ __forceinline__ void cp_async_wait() {
 
 // RES = false (trunk only): the codes and scales are neither copied nor read.
 // SPARSE: only the tile's c.nb packed code bytes are copied, as they lie.
-template <bool MASK, bool RES, bool SPARSE = false>
+template <bool MASK, bool RES, bool SPARSE = false, bool ASYM = false>
 __device__ __forceinline__ void copy_tile(uint32_t slot, const Cursor& c, int lane) {
-  using SL = Slot<MASK, RES, SPARSE>;
+  using SL = Slot<MASK, RES, SPARSE, ASYM>;
   if constexpr (RES && SPARSE) {
 #pragma unroll
     for (int j = 0; j < 4; ++j)
@@ -230,6 +236,10 @@ __device__ __forceinline__ void copy_tile(uint32_t slot, const Cursor& c, int la
   if constexpr (RES) {
     cp_async4(slot + SL::kScale + lane * 8, c.scale);
     cp_async4(slot + SL::kScale + lane * 8 + 4, c.scale + 8);
+  }
+  if constexpr (ASYM) {
+    cp_async4(slot + SL::kZero + lane * 8, c.zero);
+    cp_async4(slot + SL::kZero + lane * 8 + 4, c.zero + 8);
   }
 }
 
@@ -273,10 +283,10 @@ __device__ __forceinline__ void expand_sparse(uint32_t (&q)[16], const uint8_t* 
   }
 }
 
-template <bool MASK, bool RES, bool SPARSE = false>
+template <bool MASK, bool RES, bool SPARSE = false, bool ASYM = false>
 __device__ __forceinline__ void read_tile(Tile<MASK>& t, const uint8_t* slot, int lane,
                                           const uint32_t* sel_lut = nullptr) {
-  using SL = Slot<MASK, RES, SPARSE>;
+  using SL = Slot<MASK, RES, SPARSE, ASYM>;
   if constexpr (RES && SPARSE) {
     const uint2 kv = *reinterpret_cast<const uint2*>(slot + SL::kKeep + lane * 8);
     expand_sparse(t.q, slot, kv.x, kv.y, lane, sel_lut);
@@ -303,6 +313,11 @@ __device__ __forceinline__ void read_tile(Tile<MASK>& t, const uint8_t* slot, in
     const float2 cv = *reinterpret_cast<const float2*>(slot + SL::kScale + lane * 8);
     t.c[0] = cv.x;
     t.c[1] = cv.y;
+  }
+  if constexpr (ASYM) {
+    const int2 zv = *reinterpret_cast<const int2*>(slot + SL::kZero + lane * 8);
+    t.z[0] = zv.x;
+    t.z[1] = zv.y;
   }
 }
 
@@ -522,9 +537,11 @@ __device__ __forceinline__ void split_activations(const Params& p, const uint32_
 // RES = false: the trunk-only mode (the residual path skipped: no codes or
 // scales read, no residual MMAs, outlier channels take the trunk weight).
 // SPARSE: the weight is in SQ_LAYOUT_TILES_SPARSE (packed kept codes).
-template <bool MASK, bool EMIT, bool FUSED, int D, bool RES, bool SPARSE>
+// ASYM: SQ_LAYOUT_TILES_ASYM: a group's residual term is s_g * (R_g - z_g * S_g)
+// with S_g the sum of the group's activation codes, exact in 64-bit integers.
+template <bool MASK, bool EMIT, bool FUSED, int D, bool RES, bool SPARSE, bool ASYM>
 __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
-  using SL = Slot<MASK, RES, SPARSE>;
+  using SL = Slot<MASK, RES, SPARSE, ASYM>;
   extern __shared__ __align__(16) uint8_t smem[];
   __shared__ uint32_t sel_lut[16];  // byte-permute selectors of the sparse expansion
   // shared: part [kWarps][2 slots][16 rows][M tokens] float4 | omask[nw] u32 |
@@ -553,6 +570,7 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
     cur.sign = p.sign + lt * 2;
     cur.mask = MASK ? p.mask + lt * 2 : p.sign;
     cur.scale = p.scale + (int64_t)t0 * 16 + gid;
+    if constexpr (ASYM) cur.zero = p.zero + (int64_t)t0 * 16 + gid;
     if constexpr (SPARSE) {
       cur.keep = p.keep + lt * 2;
       cur.nbytes = p.nbytes + t0;
@@ -573,9 +591,9 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
   constexpr int kEarly = FUSED ? kDepthEarly : D;
 #pragma unroll
   for (int d = 0; d < kEarly; ++d) {  // one commit group per tile, empty past the range
-    if (t0 + d < t1) copy_tile<MASK, RES, SPARSE>(ring_u + d * SL::kBytes, cur, lane);
+    if (t0 + d < t1) copy_tile<MASK, RES, SPARSE, ASYM>(ring_u + d * SL::kBytes, cur, lane);
     cp_async_commit();
-    cur.advance<SPARSE>();
+    cur.advance<SPARSE, ASYM>();
   }
 
   __syncthreads();  // omask zeroed (and the selector table written)
@@ -607,9 +625,9 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
     split_activations(p, omask, xq_s, xo_s, sx_s, reinterpret_cast<float*>(smem + p.off_red), jv, jp);
 #pragma unroll
     for (int d = kEarly; d < D; ++d) {
-      if (t0 + d < t1) copy_tile<MASK, RES, SPARSE>(ring_u + d * SL::kBytes, cur, lane);
+      if (t0 + d < t1) copy_tile<MASK, RES, SPARSE, ASYM>(ring_u + d * SL::kBytes, cur, lane);
       cp_async_commit();
-      cur.advance<SPARSE>();
+      cur.advance<SPARSE, ASYM>();
     }
   }
 
@@ -643,7 +661,7 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
     cp_async_wait<D - 1>();  // this lane's copies of the tile have landed
     __syncwarp();             // ... and every lane's
     Tile<MASK> tl;
-    read_tile<MASK, RES, SPARSE>(tl, ring_w + slot_i * SL::kBytes, lane, sel_lut);
+    read_tile<MASK, RES, SPARSE, ASYM>(tl, ring_w + slot_i * SL::kBytes, lane, sel_lut);
     // activation codes of this lane's 32 channels for its MMA column
     uint32_t xw[8];
     {
@@ -662,6 +680,10 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
     const uint32_t pb0 = MASK ? (tl.s[0] & tl.m[0]) : tl.s[0];
     const uint32_t pb1 = MASK ? (tl.s[1] & tl.m[1]) : tl.s[1];
     int R[4] = {0, 0, 0, 0};
+    // asymmetric residual: the tile's activation sum S_g per token, from the
+    // all-ones MMA (the growth of acc.S over the tile; with a mask, its own)
+    const int S0[4] = {acc.S[0], acc.S[1], acc.S[2], acc.S[3]};
+    int Sg[4] = {0, 0, 0, 0};
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
       const uint32_t b0 = xw[2 * m], b1 = xw[2 * m + 1];
@@ -674,14 +696,27 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
                bits_word(tl.m[0], 2 * m + 1), bits_word(tl.m[1], 2 * m + 1), b0, b1);
       else
         mma_s8(acc.S, kOnes, kOnes, kOnes, kOnes, b0, b1);
+      if constexpr (ASYM && MASK) mma_s8(Sg, kOnes, kOnes, kOnes, kOnes, b0, b1);
     }
     // promote the group sums: R[0..1] row r0, R[2..3] row r1
-    if constexpr (RES) {
+    if constexpr (ASYM) {
+      if constexpr (!MASK) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) Sg[i] = acc.S[i] - S0[i];
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const long long d = (long long)R[i] - (long long)tl.z[i >> 1] * (long long)Sg[i];
+        acc.F[i] = fmaf(tl.c[i >> 1], (float)d, acc.F[i]);
+      }
+    } else if constexpr (RES) {
       acc.F[0] = fmaf(tl.c[0], (float)R[0], acc.F[0]);
       acc.F[1] = fmaf(tl.c[0], (float)R[1], acc.F[1]);
       acc.F[2] = fmaf(tl.c[1], (float)R[2], acc.F[2]);
       acc.F[3] = fmaf(tl.c[1], (float)R[3], acc.F[3]);
     }
+    (void)S0;
+    (void)Sg;
     if (EMIT) {
       const int ng = p.tpr;
       const int r0 = rb * kTileRows + gid, r1 = r0 + 8;
@@ -715,7 +750,10 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
           const uint32_t m1 = MASK ? (tl.m[1] >> bit) & 1u : 1u;
           u0 = m0 ? (((tl.s[0] >> bit) & 1u) ? 1.0f : -1.0f) : 0.0f;
           u1 = m1 ? (((tl.s[1] >> bit) & 1u) ? 1.0f : -1.0f) : 0.0f;
-          if constexpr (RES) {
+          if constexpr (ASYM) {
+            w0 = tl.c[0] * (float)(tile_code<0>(tl.q, j) - tl.z[0]);
+            w1 = tl.c[1] * (float)(tile_code<1>(tl.q, j) - tl.z[1]);
+          } else if constexpr (RES) {
             w0 = tl.c[0] * (float)tile_code<0>(tl.q, j);
             w1 = tl.c[1] * (float)tile_code<1>(tl.q, j);
           }
@@ -750,9 +788,9 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
 
     // refill this slot with the tile D ahead, once no lane reads it
     __syncwarp();
-    if (t + D < t1) copy_tile<MASK, RES, SPARSE>(ring_u + slot_i * SL::kBytes, cur, lane);
+    if (t + D < t1) copy_tile<MASK, RES, SPARSE, ASYM>(ring_u + slot_i * SL::kBytes, cur, lane);
     cp_async_commit();
-    cur.advance<SPARSE>();
+    cur.advance<SPARSE, ASYM>();
     if (++slot_i == D) slot_i = 0;
 
     // end of a row block, or end of this warp's range
@@ -822,9 +860,10 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
   }
 }
 
-template <bool MASK, bool EMIT, bool FUSED, int D, bool RES = true, bool SPARSE = false>
+template <bool MASK, bool EMIT, bool FUSED, int D, bool RES = true, bool SPARSE = false,
+          bool ASYM = false>
 cudaError_t launch_one(const Params& p, int grid, int smem, bool pdl, cudaStream_t stream) {
-  auto* fn = k_linear_tc<MASK, EMIT, FUSED, D, RES, SPARSE>;
+  auto* fn = k_linear_tc<MASK, EMIT, FUSED, D, RES, SPARSE, ASYM>;
   cudaError_t e = ensure_smem_attr((const void*)fn, smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -840,27 +879,30 @@ cudaError_t launch_one(const Params& p, int grid, int smem, bool pdl, cudaStream
   return cudaLaunchKernelEx(&cfg, fn, p);
 }
 
+// kind: 0 dense symmetric residual, 1 sparse, 2 asymmetric.
 template <bool MASK, bool FUSED, int D>
-cudaError_t launch_plain(const Params& p, bool res, bool sparse, int grid, int smem, bool pdl,
+cudaError_t launch_plain(const Params& p, bool res, int kind, int grid, int smem, bool pdl,
                          cudaStream_t stream) {
   if (!res) return launch_one<MASK, false, FUSED, kTrunkDepth, false>(p, grid, smem, pdl, stream);
-  return sparse ? launch_one<MASK, false, FUSED, D, true, true>(p, grid, smem, pdl, stream)
-                : launch_one<MASK, false, FUSED, D, true, false>(p, grid, smem, pdl, stream);
+  if (kind == 1) return launch_one<MASK, false, FUSED, D, true, true>(p, grid, smem, pdl, stream);
+  if (kind == 2)
+    return launch_one<MASK, false, FUSED, D, true, false, true>(p, grid, smem, pdl, stream);
+  return launch_one<MASK, false, FUSED, D, true, false>(p, grid, smem, pdl, stream);
 }
 
 // Non-accumulator launch with a ring depth chosen at run time among Ds.
 template <int D0, int... Ds>
-cudaError_t launch_depth(int depth, bool mask, bool fused, bool res, bool sparse, const Params& p,
+cudaError_t launch_depth(int depth, bool mask, bool fused, bool res, int kind, const Params& p,
                          int grid, int smem, bool pdl, cudaStream_t stream) {
   if (depth == D0 || sizeof...(Ds) == 0) {
     if (fused)
-      return mask ? launch_plain<true, true, D0>(p, res, sparse, grid, smem, pdl, stream)
-                  : launch_plain<false, true, D0>(p, res, sparse, grid, smem, pdl, stream);
-    return mask ? launch_plain<true, false, D0>(p, res, sparse, grid, smem, pdl, stream)
-                : launch_plain<false, false, D0>(p, res, sparse, grid, smem, pdl, stream);
+      return mask ? launch_plain<true, true, D0>(p, res, kind, grid, smem, pdl, stream)
+                  : launch_plain<false, true, D0>(p, res, kind, grid, smem, pdl, stream);
+    return mask ? launch_plain<true, false, D0>(p, res, kind, grid, smem, pdl, stream)
+                : launch_plain<false, false, D0>(p, res, kind, grid, smem, pdl, stream);
   }
   if constexpr (sizeof...(Ds) > 0)
-    return launch_depth<Ds...>(depth, mask, fused, res, sparse, p, grid, smem, pdl, stream);
+    return launch_depth<Ds...>(depth, mask, fused, res, kind, p, grid, smem, pdl, stream);
   return cudaErrorInvalidValue;
 }
 
@@ -882,10 +924,16 @@ int outlier_table_bytes(const sq_packed_weight& w) { return (int)(tiles_cols(w.K
 int fused_token_bytes(const sq_packed_weight& w, int n_out) {
   return (int)tiles_cols(w.K) + (int)round_up(n_out, 4) * 4;
 }
-int ring_bytes(bool mask, int depth, bool sparse = false) {
-  const int slot = sparse ? (mask ? Slot<true, true, true>::kBytes : Slot<false, true, true>::kBytes)
-                          : (mask ? Slot<true>::kBytes : Slot<false>::kBytes);
+// kind: 0 dense symmetric residual, 1 sparse, 2 asymmetric.
+int ring_bytes(bool mask, int depth, int kind = 0) {
+  int slot;
+  if (kind == 1) slot = mask ? Slot<true, true, true>::kBytes : Slot<false, true, true>::kBytes;
+  else if (kind == 2) slot = mask ? Slot<true, true, false, true>::kBytes : Slot<false, true, false, true>::kBytes;
+  else slot = mask ? Slot<true>::kBytes : Slot<false>::kBytes;
   return kWarps * depth * slot;
+}
+int residual_kind(const sq_packed_weight& w) {
+  return w.layout == SQ_LAYOUT_TILES_SPARSE ? 1 : w.layout == SQ_LAYOUT_TILES_ASYM ? 2 : 0;
 }
 int trunk_ring_bytes(bool mask) {
   return kWarps * kTrunkDepth * (mask ? Slot<true, false>::kBytes : Slot<false, false>::kBytes);
@@ -894,7 +942,7 @@ int trunk_ring_bytes(bool mask) {
 
 int linear_tc_fused_tokens(const sq_packed_weight& w, int n_out) {
   // counted with the shallow ring; the deep one is used when it fits
-  const int fixed = ring_bytes(w.mask_bits != nullptr, kShallow, w.layout == SQ_LAYOUT_TILES_SPARSE) +
+  const int fixed = ring_bytes(w.mask_bits != nullptr, kShallow, residual_kind(w)) +
                     outlier_table_bytes(w) +
                     kCols * 4 + kWarps * kCols * 4 + 64;
   const int per = fused_token_bytes(w, n_out) + kSmemPartPerToken;
@@ -907,9 +955,14 @@ cudaError_t launch_linear_tc(const sq_packed_weight& w, int M, const int8_t* xq,
                              float* y, int32_t* T_out, int32_t* R_out, void* workspace,
                              size_t part_bytes, int sm_count, int32_t* status, bool pdl,
                              bool trunk_only, cudaStream_t stream) {
-  const bool sparse = w.layout == SQ_LAYOUT_TILES_SPARSE;
-  if (M < 1 || M > kCols || (w.layout != SQ_LAYOUT_TILES && !sparse)) return cudaErrorInvalidValue;
+  const int kind = residual_kind(w);
+  const bool sparse = kind == 1;
+  if (M < 1 || M > kCols) return cudaErrorInvalidValue;
+  if (w.layout != SQ_LAYOUT_TILES && w.layout != SQ_LAYOUT_TILES_SPARSE &&
+      w.layout != SQ_LAYOUT_TILES_ASYM)
+    return cudaErrorInvalidValue;
   if (sparse && (!w.keep_bits || !w.res_bytes)) return cudaErrorInvalidValue;
+  if (kind == 2 && !w.res_zero) return cudaErrorInvalidValue;
   if (trunk_only && T_out) return cudaErrorInvalidValue;
   const bool fused = x != nullptr;
   if (fused && (T_out || M > linear_tc_fused_tokens(w, n_out))) return cudaErrorInvalidValue;
@@ -921,6 +974,7 @@ cudaError_t launch_linear_tc(const sq_packed_weight& w, int M, const int8_t* xq,
   p.scale = w.res_scale;
   p.keep = w.keep_bits;
   p.nbytes = w.res_bytes;
+  p.zero = w.res_zero;
   p.N = w.N;
   p.K = w.K;
   p.tpr = (int)(tiles_cols(w.K) / kTileK);
@@ -966,18 +1020,21 @@ cudaError_t launch_linear_tc(const sq_packed_weight& w, int M, const int8_t* xq,
   // three tiles per warp above batch 2 where they fit, else two (the
   // accumulator mode, used to check the kernel, always takes two)
   const int depth =
-      (!emit && M > 2 && smem + ring_bytes(mask, kDeep, sparse) <= kSmemMax) ? kDeep : kShallow;
-  smem += trunk_only ? trunk_ring_bytes(mask) : ring_bytes(mask, depth, sparse);
+      (!emit && M > 2 && smem + ring_bytes(mask, kDeep, kind) <= kSmemMax) ? kDeep : kShallow;
+  smem += trunk_only ? trunk_ring_bytes(mask) : ring_bytes(mask, depth, kind);
   if (smem > kSmemMax) return cudaErrorInvalidValue;
   const int grid = (int)blocks;
   if (emit) {
     if (sparse)
       return mask ? launch_one<true, true, false, kShallow, true, true>(p, grid, smem, pdl, stream)
                   : launch_one<false, true, false, kShallow, true, true>(p, grid, smem, pdl, stream);
+    if (kind == 2)
+      return mask ? launch_one<true, true, false, kShallow, true, false, true>(p, grid, smem, pdl, stream)
+                  : launch_one<false, true, false, kShallow, true, false, true>(p, grid, smem, pdl, stream);
     return mask ? launch_one<true, true, false, kShallow>(p, grid, smem, pdl, stream)
                 : launch_one<false, true, false, kShallow>(p, grid, smem, pdl, stream);
   }
-  return launch_depth<kDeep, kShallow>(depth, mask, fused, !trunk_only, sparse, p, grid, smem, pdl,
+  return launch_depth<kDeep, kShallow>(depth, mask, fused, !trunk_only, kind, p, grid, smem, pdl,
                                        stream);
 }
 

@@ -91,8 +91,9 @@ __device__ __forceinline__ void load_tile(float* tile, int pitch, const float* _
 // ---- sign / mask bitplanes, alpha, residual codes and group scales --------
 // One thread per row.  TILED writes SQ_LAYOUT_TILES (rows padded to a
 // multiple of 16 and channels to a multiple of 128, pads zero); otherwise
-// SQ_LAYOUT_ROWS.
-template <bool TILED>
+// SQ_LAYOUT_ROWS.  ASYM (tiled): asymmetric residual groups with their own
+// min / max, scale and zero-point (SQ_LAYOUT_TILES_ASYM).
+template <bool TILED, bool ASYM>
 __global__ void __launch_bounds__(kPackRows) k_pack(const float* __restrict__ W, int N, int K,
                                                     int P, int G, sq_packed_weight pw,
                                                     int32_t* __restrict__ status) {
@@ -159,7 +160,42 @@ __global__ void __launch_bounds__(kPackRows) k_pack(const float* __restrict__ W,
     const int c0 = g * G;
     load_tile(tile, pitch2, W, N, K, r0, c0, G);
     __syncthreads();
-    if (live) {
+    if (live && ASYM) {
+      // asymmetric group: s = float((hi - lo) / 255), z = round(-lo/s - 128),
+      // code = clip(round(r/s + z), -128, 127), all binary64
+      const int ncols = valid ? min(G, K - c0) : 0;
+      const float* t = tile + threadIdx.x * pitch2;
+      auto resid = [&](int j) {
+        const float v = t[j];
+        const bool m = P < 0 ? true : (fabsf(v) > tau);
+        const double tr = m ? (v >= 0.0f ? (double)alpha : -(double)alpha) : 0.0;
+        return (double)v - tr;
+      };
+      double lo = 0.0, hi = 0.0;
+      for (int j = 0; j < ncols; ++j) {
+        const double r = resid(j);
+        if (j == 0 || r < lo) lo = r;
+        if (j == 0 || r > hi) hi = r;
+      }
+      const float s = ncols > 0 ? (float)((hi - lo) / 255.0) : 0.0f;
+      const int32_t z = s == 0.0f ? 0 : (int32_t)round(-lo / (double)s - 128.0);
+      pw.res_scale[tiled_scale_index(row, g, tpr)] = s;
+      pw.res_zero[tiled_scale_index(row, g, tpr)] = z;
+      for (int j0 = 0; j0 < G; j0 += 4) {
+        uint32_t word = 0;
+        for (int j = j0; j < j0 + 4 && j < ncols; ++j) {
+          int q = 0;
+          if (s != 0.0f) {
+            double v = round(resid(j) / (double)s + (double)z);
+            v = v > 127.0 ? 127.0 : v;
+            v = v < -128.0 ? -128.0 : v;
+            q = (int)v;
+          }
+          word |= ((uint32_t)(uint8_t)(int8_t)q) << (8 * (j - j0));
+        }
+        *reinterpret_cast<uint32_t*>(pw.res_q + tiled_code_offset(row, c0 + j0, tpr)) = word;
+      }
+    } else if (live) {
       const int ncols = valid ? min(G, K - c0) : 0;
       const float* t = tile + threadIdx.x * pitch2;
       double a = 0.0;
@@ -342,7 +378,95 @@ __global__ void __launch_bounds__(256) k_sparse_compact(int T, sq_packed_weight 
   if (lane == 0) pw.res_bytes[t] = padded;
 }
 
+// ---- per-layer fallback measure -------------------------------------------------
+// m.lqnn.cn section 2.3 (last paragraph): a layer that gains nothing from the
+// split falls back to plain 8-bit.  One thread per row: the squared
+// reconstruction error of the packed weight (What from its own arrays) and
+// of plain symmetric INT8 groups of W, binary64, channels ascending; then one
+// thread sums the rows in order.
+template <bool TILED, bool ASYM>
+__global__ void __launch_bounds__(128) k_row_errors(const float* __restrict__ W, sq_packed_weight pw,
+                                                    double* __restrict__ scratch) {
+  const int row = blockIdx.x * blockDim.x + threadIdx.x;
+  const int N = pw.N, K = pw.K, G = pw.group_size;
+  if (row >= N) return;
+  const int tpr = (int)(tiles_cols(K) / kTileK);
+  const float* wr = W + (int64_t)row * K;
+  const double al = (double)pw.alpha[row];
+  double e = 0.0;
+  for (int j = 0; j < K; ++j) {
+    const int g = j / G;
+    uint32_t sw, mw = 1u;
+    int bit;
+    int64_t ci, si;
+    if (TILED) {
+      const int64_t wi = tiled_bits_word(row, j >> 5, tpr);
+      bit = tiled_bit_of(j & 31);
+      sw = pw.sign_bits[wi];
+      if (pw.mask_bits) mw = pw.mask_bits[wi];
+      ci = tiled_code_offset(row, j, tpr);
+      si = tiled_scale_index(row, g, tpr);
+    } else {
+      const int64_t wi = (int64_t)row * pw.sign_stride + (j >> 5);
+      bit = j & 31;
+      sw = pw.sign_bits[wi];
+      if (pw.mask_bits) mw = pw.mask_bits[wi];
+      ci = (int64_t)row * pw.res_stride + j;
+      si = (int64_t)row * pw.scale_stride + g;
+    }
+    const bool m = pw.mask_bits ? ((mw >> bit) & 1u) != 0 : true;
+    const bool b = ((sw >> bit) & 1u) != 0;
+    const double t = m ? (b ? al : -al) : 0.0;
+    const int64_t z = ASYM ? (int64_t)pw.res_zero[si] : 0;
+    const double what = t + (double)pw.res_scale[si] * (double)((int64_t)pw.res_q[ci] - z);
+    const double d = (double)__ldg(wr + j) - what;
+    e += d * d;
+  }
+  double ep = 0.0;
+  for (int j0 = 0; j0 < K; j0 += G) {
+    const int j1 = min(K, j0 + G);
+    double a = 0.0;
+    for (int j = j0; j < j1; ++j) {
+      const double v = fabs((double)__ldg(wr + j));
+      a = v > a ? v : a;
+    }
+    const float sg = (float)(a / 127.0);
+    for (int j = j0; j < j1; ++j) {
+      const double w = (double)__ldg(wr + j);
+      const double d = w - (double)sg * (double)quantize_q(w, sg);
+      ep += d * d;
+    }
+  }
+  scratch[row] = e;
+  scratch[N + row] = ep;
+}
+
+__global__ void k_sum_errors(const double* __restrict__ scratch, int N, double* __restrict__ err) {
+  if (threadIdx.x != 0) return;
+  double a = 0.0, b = 0.0;
+  for (int r = 0; r < N; ++r) a += scratch[r];
+  for (int r = 0; r < N; ++r) b += scratch[N + r];
+  err[0] = a;
+  err[1] = b;
+}
+
 }  // namespace
+
+cudaError_t launch_residual_errors(const float* W, const sq_packed_weight& w, double* err,
+                                   double* scratch, int32_t* status, cudaStream_t stream) {
+  (void)status;
+  const int blocks = (int)ceil_div(w.N, 128);
+  if (w.layout == SQ_LAYOUT_TILES_ASYM)
+    k_row_errors<true, true><<<blocks, 128, 0, stream>>>(W, w, scratch);
+  else if (w.layout == SQ_LAYOUT_TILES)
+    k_row_errors<true, false><<<blocks, 128, 0, stream>>>(W, w, scratch);
+  else
+    k_row_errors<false, false><<<blocks, 128, 0, stream>>>(W, w, scratch);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  k_sum_errors<<<1, 32, 0, stream>>>(scratch, w.N, err);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_sparsify_residual(const float* W, int N, int K, int Ps, const sq_packed_weight& pw,
                                      cudaStream_t stream) {
@@ -363,17 +487,21 @@ cudaError_t launch_decompose_pack(const float* W, int N, int K, int P, const sq_
     if (e != cudaSuccess) return e;
   }
   const int G = pw.group_size;
-  const bool tiled = pw.layout == SQ_LAYOUT_TILES;
+  const bool asym = pw.layout == SQ_LAYOUT_TILES_ASYM;
+  const bool tiled = pw.layout == SQ_LAYOUT_TILES || asym;
   const size_t smem = (size_t)kPackRows * (G + 1) * sizeof(float);
-  const void* fn = tiled ? (const void*)k_pack<true> : (const void*)k_pack<false>;
+  const void* fn = asym ? (const void*)k_pack<true, true>
+                        : tiled ? (const void*)k_pack<true, false> : (const void*)k_pack<false, false>;
   cudaError_t e = ensure_smem_attr(fn, (int)smem);
   if (e != cudaSuccess) return e;
   const int64_t rows = tiled ? tiles_rows(N) : N;
   const int blocks = (int)ceil_div(rows, kPackRows);
-  if (tiled)
-    k_pack<true><<<blocks, kPackRows, smem, stream>>>(W, N, K, P, G, pw, status);
+  if (asym)
+    k_pack<true, true><<<blocks, kPackRows, smem, stream>>>(W, N, K, P, G, pw, status);
+  else if (tiled)
+    k_pack<true, false><<<blocks, kPackRows, smem, stream>>>(W, N, K, P, G, pw, status);
   else
-    k_pack<false><<<blocks, kPackRows, smem, stream>>>(W, N, K, P, G, pw, status);
+    k_pack<false, false><<<blocks, kPackRows, smem, stream>>>(W, N, K, P, G, pw, status);
   return cudaGetLastError();
 }
 

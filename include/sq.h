@@ -77,6 +77,7 @@ typedef enum {
 #define SQ_LAYOUT_ROWS 0
 #define SQ_LAYOUT_TILES 1
 #define SQ_LAYOUT_TILES_SPARSE 2
+#define SQ_LAYOUT_TILES_ASYM 3
 
 /*
  * Packed weight of one linear layer (N output rows, K input channels).
@@ -125,11 +126,19 @@ typedef enum {
  *             each tile's kept codes (what the decode kernel reads)
  * Every other array is that of SQ_LAYOUT_TILES.
  *
+ * SQ_LAYOUT_TILES_ASYM (G = 128 only): SQ_LAYOUT_TILES with an asymmetric
+ * residual (m.lqnn.cn section 2 pitfalls: the residual gets its own min/max,
+ * scale and zero-point; the asymmetric quantizer of the 2048ai.net
+ * explainer): codes in [-128, 127] and one more array,
+ *   res_zero  [tile][16] i32, indexed like res_scale: the zero-point z_g of
+ *             each (row, group); the dequantized residual is s_g*(q - z_g)
+ * Every other array is that of SQ_LAYOUT_TILES.
+ *
  * The arrays may live in one allocation carved by sq_packed_view().
  */
 typedef struct {
   int32_t N, K, group_size;  /* group_size G: 32, 64 or 128 */
-  int32_t layout;            /* SQ_LAYOUT_ROWS, SQ_LAYOUT_TILES or SQ_LAYOUT_TILES_SPARSE */
+  int32_t layout;            /* SQ_LAYOUT_ROWS, SQ_LAYOUT_TILES, _TILES_SPARSE or _TILES_ASYM */
   int32_t sign_stride;       /* u32 words per row of sign_bits / mask_bits */
   int32_t res_stride;        /* bytes per row of res_q */
   int32_t scale_stride;      /* floats per row of res_scale */
@@ -140,6 +149,7 @@ typedef struct {
   float *res_scale;
   uint32_t *keep_bits;       /* SQ_LAYOUT_TILES_SPARSE only, else NULL */
   int32_t *res_bytes;        /* SQ_LAYOUT_TILES_SPARSE only, else NULL */
+  int32_t *res_zero;         /* SQ_LAYOUT_TILES_ASYM only, else NULL */
 } sq_packed_weight;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -174,7 +184,11 @@ sq_status sq_packed_view(void *base, int32_t N, int32_t K, int32_t group_size,
  * in ascending channel order, cnt their number (0 -> alpha 0).  Residual
  * r = double(W) - m*(+-alpha) in binary64; group scale s = float(absmax/127);
  * code = clip(round_half_away(r / s), +-127) with a binary64 quotient (s == 0
- * gives 0).  Non-finite W sets SQ_ERR_NONFINITE in dev_status.
+ * gives 0).  Into SQ_LAYOUT_TILES_ASYM the residual groups are asymmetric:
+ * lo, hi = the group's min and max of r, s = float((hi - lo) / 255),
+ * z = round_half_away(-lo / s - 128), code = clip(round_half_away(r / s + z),
+ * -128, 127), all in binary64 (s == 0 gives z = 0 and codes 0).
+ * Non-finite W sets SQ_ERR_NONFINITE in dev_status.
  */
 sq_status sq_decompose_pack(const float *W, int32_t N, int32_t K, int32_t trunk_percent,
                             const sq_packed_weight *out, int32_t *dev_status, void *stream);
@@ -198,6 +212,29 @@ sq_status sq_decompose_pack(const float *W, int32_t N, int32_t K, int32_t trunk_
 sq_status sq_decompose_pack_sparse(const float *W, int32_t N, int32_t K, int32_t trunk_percent,
                                    int32_t residual_percent, const sq_packed_weight *out,
                                    int32_t *dev_status, void *stream);
+
+/*
+ * The per-layer fallback measure (m.lqnn.cn section 2.3, last paragraph: a
+ * layer that gains nothing from the split falls back to plain 8-bit).
+ *   W        [N][K] f32, device: the weight that `w` was decomposed from
+ *   w        packed weight of W (any layout but SQ_LAYOUT_TILES_SPARSE)
+ *   err      device, 2 doubles out:
+ *            err[0] = sum_r sum_j (W_rj - What_rj)^2 for w, What its
+ *                     dequantized weight (trunk + residual);
+ *            err[1] = the same for plain symmetric INT8 groups of W of w's
+ *                     group size (no trunk): What = s_g*Q(W, s_g),
+ *                     s_g = float(absmax_g |W| / 127);
+ *            each binary64, channels ascending within a row, rows in order.
+ *   scratch  device, sq_residual_errors_scratch_bytes(N) bytes
+ * The rule (this library's reading of the page): the layer falls back --
+ * it is packed with trunk_percent = 100, an empty trunk, i.e. plain INT8
+ * groups of W -- when err[1] <= err[0], that is when the split does not
+ * reconstruct W strictly better.
+ */
+size_t sq_residual_errors_scratch_bytes(int32_t N);
+sq_status sq_residual_errors(const float *W, const sq_packed_weight *w, double *err,
+                             void *scratch, size_t scratch_bytes, int32_t *dev_status,
+                             void *stream);
 
 /*
  * Outlier calibration (m.lqnn.cn section 2.2: detect the outlier channels once,

@@ -35,7 +35,7 @@ class Layer:
     out_factor: float = 50.0   # multiplier of the outlier channels in x
     trunk_percent: int = -1    # <0: full trunk; else per-row percentile
     group: int = 128
-    residual_percent: int = 0  # 0: dense residual; else the per-row percentile of |r| dropped
+    residual_percent: int = 0  # 0: dense residual; > 0: that per-row percentile of |r| dropped; < 0: asymmetric groups
 
     @property
     def seed(self) -> int:

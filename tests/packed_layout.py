@@ -89,6 +89,8 @@ def unpack(pw: "sq.PackedWeight", rows=None) -> dict:
     s = _gather(scale_flat, si)
     alpha = _gather(alpha_all, rows)
     out = {"sign": sign, "mask": mask, "alpha": alpha, "q": q, "s": s}
+    if pw.layout == sq.SQ_LAYOUT_TILES_ASYM:
+        out["z"] = _gather(pw.res_zero().reshape(-1), si)
     if keep is not None:
         out["keep"] = keep
         out["res_bytes_ok"] = nbytes_ok
@@ -144,5 +146,5 @@ def pad_rows_are_zero(pw: "sq.PackedWeight") -> bool:
         return True
     u = unpack(pw, rows=np.arange(pw.N, pw.rows))
     parts = [u["sign"], u["alpha"], u["q"], u["s"]] + ([u["mask"]] if pw.with_mask else []) + \
-        ([u["keep"]] if "keep" in u else [])
+        ([u["keep"]] if "keep" in u else []) + ([u["z"]] if "z" in u else [])
     return all(not np.asarray(a).view(np.uint8).any() for a in parts)

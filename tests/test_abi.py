@@ -57,7 +57,7 @@ def test_status_strings(L):
     (1, 1, 128, 0, 0), (7, 33, 32, 1, 0), (512, 512, 128, 0, 0), (12288, 4096, 128, 0, 0),
     (8192, 28672, 64, 1, 0), (1, 1, 128, 0, 1), (7, 33, 128, 1, 1), (12288, 4096, 128, 0, 1),
     (4096, 11008, 128, 1, 1), (8192, 28672, 128, 0, 1), (7, 33, 128, 0, 2), (12288, 4096, 128, 1, 2),
-    (4096, 11008, 128, 0, 2)])
+    (4096, 11008, 128, 0, 2), (7, 33, 128, 1, 3), (12288, 4096, 128, 0, 3)])
 def test_packed_view_layout(L, N, K, G, mask, layout):
     nbytes = L.sq_packed_bytes(N, K, G, mask, layout)
     assert nbytes > 0
@@ -85,6 +85,10 @@ def test_packed_view_layout(L, N, K, G, mask, layout):
         spans += [(v.keep_bits, rows * v.sign_stride * 4), (v.res_bytes, tiles * 4)]
     else:
         assert v.keep_bits is None and v.res_bytes is None
+    if layout == sq.SQ_LAYOUT_TILES_ASYM:
+        spans.append((v.res_zero, rows * v.scale_stride * 4))
+    else:
+        assert v.res_zero is None
     spans.sort()
     for (a, la), (b, _) in zip(spans, spans[1:]):
         assert a % 256 == 0 and a + la <= b
@@ -97,7 +101,7 @@ def test_packed_view_rejects(L):
     assert L.sq_packed_view(ctypes.c_void_p(1 << 40), 8, 8, 48, 0, 0, ctypes.byref(v)) == 2
     assert L.sq_packed_view(ctypes.c_void_p(1 << 40), 0, 8, 128, 0, 0, ctypes.byref(v)) == 2
     assert L.sq_packed_view(None, 8, 8, 128, 0, 0, ctypes.byref(v)) == 1
-    assert L.sq_packed_view(ctypes.c_void_p(1 << 40), 8, 8, 128, 0, 3, ctypes.byref(v)) == 1
+    assert L.sq_packed_view(ctypes.c_void_p(1 << 40), 8, 8, 128, 0, 4, ctypes.byref(v)) == 1
     # the sparse tiled layout: group size 128 only
     assert L.sq_packed_view(ctypes.c_void_p(1 << 40), 8, 8, 64, 0, 2, ctypes.byref(v)) == 2
     # the tiled layout: group size 128 only, K <= 131072
