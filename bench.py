@@ -544,17 +544,18 @@ def sparse_weight_bytes(pw) -> int:
     return rows * (4 * words * planes + 4 * groups + 4) + int(nb.sum().item()) + 4 * nb.numel()
 
 
-def _fused_launches(pw, M: int, L) -> int:
+def _fused_launches(pw, M: int, L, flags: int = 0) -> int:
     """Launches of one sq_quantize_linear call with a fused_workspace_bytes
-    workspace: the staged route (split + linear passes of 8) when M > 1 and
-    M * roundup(K, 128) > 16 KiB or when fused passes outnumber passes of 8,
-    else one fused launch per pass."""
+    workspace: the staged route (split + linear passes of sq_linear's pass
+    size) when M > 1 and M * roundup(K, 128) > 16 KiB or when fused passes
+    outnumber those passes, else one fused launch per pass."""
     import ctypes
     import decode_matvec_sq_b200 as sq
     kx = -(-L.K // 128) * 128
     per_pass = int(sq.lib().sq_quantize_linear_tokens_per_pass(ctypes.byref(pw.view), L.n_out))
-    staged = M > 1 and (M * kx > (16 << 10) or -(-M // per_pass) > -(-M // 8))
-    return 1 + -(-M // 8) if staged else -(-M // per_pass)
+    lin = int(sq.lib().sq_linear_tokens_per_pass(ctypes.byref(pw.view), flags))
+    staged = M > 1 and (M * kx > (16 << 10) or -(-M // per_pass) > -(-M // lin))
+    return 1 + -(-M // lin) if staged else -(-M // per_pass)
 
 
 def time_layer_case(L, M, copies, trunk, st, device, warmup, reps):
@@ -601,7 +602,7 @@ def time_layer_case(L, M, copies, trunk, st, device, warmup, reps):
     else:  # (an asymmetric residual adds its zero-points: 4 bytes per group)
         wbytes = linear_weight_bytes(L) + (4 * pw.rows * pw.view.scale_stride if Ps < 0 else 0)
     nbytes = wbytes + M * (4 * L.K + 4 * L.N) + 4 * L.n_out
-    launches = _fused_launches(pw, M, L)
+    launches = _fused_launches(pw, M, L, sq.SQ_TRUNK_ONLY if trunk else 0)
     del pws, pw, ws
     torch.cuda.empty_cache()
     return ms, nbytes, launches, calls
@@ -686,7 +687,8 @@ def run_layers(args, world, rank, local):
     """Single-layer workloads beside the stack: the 512 x 512 layer (hot and
     cold), the 70B-shaped MLP pair at batch 1..16 and the threshold-trunk layer.
     Each call is the one-launch fused entry point (activation split + linear;
-    batches above 8 take one launch per 8 tokens), timed as a CUDA graph of
+    larger batches take the split, then one decode launch per 16 tokens),
+    timed as a CUDA graph of
     calls rotating over the weight copies.  GB/s = algorithmic bytes (packed
     weights once + activations + y) / device time."""
     import torch

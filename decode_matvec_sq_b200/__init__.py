@@ -83,6 +83,7 @@ def lib():
         "sq_linear_workspace_bytes": ([pw, i32], sz),
         "sq_quantize_linear_workspace_bytes": ([pw, i32, i32], sz),
         "sq_quantize_linear_tokens_per_pass": ([pw, i32], i32),
+        "sq_linear_tokens_per_pass": ([pw, u32], i32),
         "sq_linear": ([pw, vp, vp, vp, vp, i32, i32, vp, vp, sz, vp, u32, vp], ctypes.c_int),
         "sq_linear_accumulators": ([pw, vp, vp, vp, vp, i32, i32, vp, vp, vp, vp, sz, vp, u32, vp],
                                    ctypes.c_int),

@@ -363,7 +363,7 @@ static sq_status linear_common(const sq_packed_weight* w, const int8_t* xq, cons
     return e == cudaSuccess ? SQ_OK : SQ_ERR_CUDA;
   }
   const bool tc = tiled(w->layout);
-  const int per_pass = tc ? kMaxTokensPerPassTc : kMaxTokensPerPass;
+  const int per_pass = tc ? linear_tc_pass_tokens(*w, trunk_only) : kMaxTokensPerPass;
   const int64_t xs = xq_stride_of(w->K);
   for (int t0 = 0; t0 < M; t0 += per_pass) {
     const int m = std::min(per_pass, M - t0);
@@ -433,6 +433,13 @@ size_t sq_quantize_linear_workspace_bytes(const sq_packed_weight* w, int32_t M, 
   return (size_t)round_up((int64_t)need, 256) + stage_bytes(*w, M, n_out);
 }
 
+int32_t sq_linear_tokens_per_pass(const sq_packed_weight* w, uint32_t flags) {
+  if (!w || check_weight(w) != SQ_OK || (flags & ~SQ_TRUNK_ONLY)) return 0;
+  const bool trunk_only = (flags & SQ_TRUNK_ONLY) != 0;
+  if (!tiled(w->layout)) return trunk_only ? 0 : kMaxTokensPerPass;
+  return linear_tc_pass_tokens(*w, trunk_only);
+}
+
 int32_t sq_quantize_linear_tokens_per_pass(const sq_packed_weight* w, int32_t n_out) {
   if (!w || check_weight(w) != SQ_OK || !tiled(w->layout)) return 0;
   if (n_out < 0 || n_out > kMaxOutliers || n_out > w->K) return 0;
@@ -462,7 +469,8 @@ sq_status sq_quantize_linear(const sq_packed_weight* w, const float* x, int32_t 
   const size_t part = linear_part_bytes(d.sm_count);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool staged_faster = M > 1 && ((int64_t)M * xq_stride_of(w->K) > kFusedMaxCodeBytes ||
-                                       ceil_div(M, per_pass) > ceil_div(M, kMaxTokensPerPassTc));
+                                       ceil_div(M, per_pass) >
+                                           ceil_div(M, linear_tc_pass_tokens(*w, (flags & SQ_TRUNK_ONLY) != 0)));
   const size_t base = (size_t)round_up((int64_t)need, 256);
   if (staged_faster && ws_bytes >= base + stage_bytes(*w, M, n_out)) {
     int8_t* xq = static_cast<int8_t*>(workspace) + base;

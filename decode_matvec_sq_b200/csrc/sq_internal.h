@@ -63,7 +63,6 @@ struct LinearPlan {
 };
 
 constexpr int kMaxTokensPerPass = 4;     // CUDA-core decode kernel
-constexpr int kMaxTokensPerPassTc = 8;   // tensor-core decode kernel
 constexpr int kMaxOutliers = 4096;
 
 // Plans a decode launch for M tokens (M <= kMaxTokensPerPass) on the current device.
@@ -80,10 +79,13 @@ cudaError_t launch_linear(const sq_packed_weight& w, const LinearPlan& plan, con
                           float* y, int32_t* T_out, int32_t* R_out, void* workspace,
                           size_t part_bytes, int32_t* status, bool pdl, cudaStream_t stream);
 
-// Tensor-core decode kernel (SQ_LAYOUT_TILES), up to kMaxTokensPerPassTc tokens.
-// With x != NULL (fused mode) it performs the activation split of x itself
-// (xq, sx, x_out unused) for at most linear_tc_fused_tokens() tokens.
+// Tensor-core decode kernel (tiled layouts), up to linear_tc_pass_tokens()
+// tokens (16 where their partial sums fit in shared memory, else 8): the
+// weights are read once per pass.  With x != NULL (fused mode) it performs the
+// activation split of x itself (xq, sx, x_out unused) for at most
+// linear_tc_fused_tokens() tokens.
 size_t linear_tc_part_bytes(int sm_count);
+int linear_tc_pass_tokens(const sq_packed_weight& w, bool trunk_only);
 int linear_tc_fused_tokens(const sq_packed_weight& w, int n_out);
 cudaError_t launch_linear_tc(const sq_packed_weight& w, int M, const int8_t* xq, const float* sx,
                              const float* x_out, const float* x, const int32_t* idx, int n_out,

@@ -191,7 +191,7 @@ struct Slot {
   static constexpr int kKeep = MASK ? kMask + 256 : kMask;  // (SPARSE only)
   static constexpr int kScale = SPARSE ? kKeep + 256 : kKeep;  // (RES only)
   static constexpr int kZero = kScale + 256;  // (ASYM only)
-  static constexpr int kBytes = kScale + (RES ? 256 : 0) + (ASYM ? 256 : 0);
+  static constexpr int kBytes = ASYM ? kZero + 256 : kScale + (RES ? 256 : 0);
 };
 // Tiles in flight per warp in the trunk-only mode (small slots).
 constexpr int kTrunkDepth = 6;
@@ -378,9 +378,9 @@ __device__ __forceinline__ void cell_add(float4& a, const float4& b) {
 // y = sx * (alpha * T + F) + (alpha * Ut + Ur).
 __device__ __forceinline__ void write_y(const Params& p, int rb, int gid, int tid4,
                                         const float4 (&v)[4], float al0, float al1, float sx0,
-                                        float sx1) {
+                                        float sx1, int tko) {
   const int r0 = rb * kTileRows + gid, r1 = r0 + 8;
-  const int tk0 = 2 * tid4, tk1 = tk0 + 1;
+  const int tk0 = 2 * tid4 + tko, tk1 = tk0 + 1;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int row = (i < 2) ? r0 : r1, tk = (i & 1) ? tk1 : tk0;
@@ -539,7 +539,9 @@ __device__ __forceinline__ void split_activations(const Params& p, const uint32_
 // SPARSE: the weight is in SQ_LAYOUT_TILES_SPARSE (packed kept codes).
 // ASYM: SQ_LAYOUT_TILES_ASYM: a group's residual term is s_g * (R_g - z_g * S_g)
 // with S_g the sum of the group's activation codes, exact in 64-bit integers.
-template <bool MASK, bool EMIT, bool FUSED, int D, bool RES, bool SPARSE, bool ASYM>
+// NT: groups of 8 tokens per pass (the MMA's N); every tile's weights serve
+// all of them, so a pass of 16 tokens reads the weights once.
+template <bool MASK, bool EMIT, bool FUSED, int D, bool RES, bool SPARSE, bool ASYM, int NT>
 __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
   using SL = Slot<MASK, RES, SPARSE, ASYM>;
   extern __shared__ __align__(16) uint8_t smem[];
@@ -631,22 +633,27 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
     }
   }
 
-  // tokens of this lane's accumulator columns; the B operand of this lane
-  // (MMA column gid) is token min(gid, M - 1): columns past M are not written
+  // tokens of this lane's accumulator columns in token group kg: tk0 + 8 kg
+  // and tk1 + 8 kg; the B operand of this lane (MMA column gid) is token
+  // min(gid + 8 kg, M - 1): columns past M are not written
   const int tk0 = 2 * tid4, tk1 = tk0 + 1;
-  float sx0, sx1;
-  if constexpr (FUSED) {
-    sx0 = tk0 < p.M ? sx_s[tk0] : 0.0f;
-    sx1 = tk1 < p.M ? sx_s[tk1] : 0.0f;
-  } else {
-    sx0 = tk0 < p.M ? __ldg(p.sx + tk0) : 0.0f;
-    sx1 = tk1 < p.M ? __ldg(p.sx + tk1) : 0.0f;
+  float sx0[NT], sx1[NT];
+  const int8_t* xrow[NT];
+  Acc acc[NT];
+#pragma unroll
+  for (int kg = 0; kg < NT; ++kg) {
+    const int a0 = tk0 + 8 * kg, a1 = tk1 + 8 * kg;
+    if constexpr (FUSED) {
+      sx0[kg] = a0 < p.M ? sx_s[a0] : 0.0f;
+      sx1[kg] = a1 < p.M ? sx_s[a1] : 0.0f;
+    } else {
+      sx0[kg] = a0 < p.M ? __ldg(p.sx + a0) : 0.0f;
+      sx1[kg] = a1 < p.M ? __ldg(p.sx + a1) : 0.0f;
+    }
+    const int tok = min(gid + 8 * kg, p.M - 1);
+    xrow[kg] = (FUSED ? xq_s + tok * p.xs : p.xq + (int64_t)tok * p.xs) + tid4 * 32;
+    acc_zero(acc[kg]);
   }
-  const int tok = min(gid, p.M - 1);
-  const int8_t* xrow = (FUSED ? xq_s + tok * p.xs : p.xq + (int64_t)tok * p.xs) + tid4 * 32;
-
-  Acc acc;
-  acc_zero(acc);
   int rb = t0 / p.tpr, cg = t0 - rb * p.tpr;
   bool rb_head = (cg == 0);  // this piece starts at the row block's first tile
   float al0 = 0.0f, al1 = 0.0f;
@@ -662,71 +669,76 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
     __syncwarp();             // ... and every lane's
     Tile<MASK> tl;
     read_tile<MASK, RES, SPARSE, ASYM>(tl, ring_w + slot_i * SL::kBytes, lane, sel_lut);
-    // activation codes of this lane's 32 channels for its MMA column
-    uint32_t xw[8];
-    {
-      const int4* xp = reinterpret_cast<const int4*>(xrow + cg * kTileK);
-      int4 a, b;
-      if constexpr (FUSED) {
-        a = xp[0];
-        b = xp[1];
-      } else {
-        a = __ldg(xp);
-        b = __ldg(xp + 1);
-      }
-      xw[0] = a.x; xw[1] = a.y; xw[2] = a.z; xw[3] = a.w;
-      xw[4] = b.x; xw[5] = b.y; xw[6] = b.z; xw[7] = b.w;
-    }
     const uint32_t pb0 = MASK ? (tl.s[0] & tl.m[0]) : tl.s[0];
     const uint32_t pb1 = MASK ? (tl.s[1] & tl.m[1]) : tl.s[1];
-    int R[4] = {0, 0, 0, 0};
-    // asymmetric residual: the tile's activation sum S_g per token, from the
-    // all-ones MMA (the growth of acc.S over the tile; with a mask, its own)
-    const int S0[4] = {acc.S[0], acc.S[1], acc.S[2], acc.S[3]};
-    int Sg[4] = {0, 0, 0, 0};
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      const uint32_t b0 = xw[2 * m], b1 = xw[2 * m + 1];
-      if constexpr (RES)
-        mma_s8(R, tl.q[4 * m], tl.q[4 * m + 1], tl.q[4 * m + 2], tl.q[4 * m + 3], b0, b1);
-      mma_s8(acc.Pn, bits_word(pb0, 2 * m), bits_word(pb1, 2 * m), bits_word(pb0, 2 * m + 1),
-             bits_word(pb1, 2 * m + 1), b0, b1);
-      if constexpr (MASK)
-        mma_s8(acc.S, bits_word(tl.m[0], 2 * m), bits_word(tl.m[1], 2 * m),
-               bits_word(tl.m[0], 2 * m + 1), bits_word(tl.m[1], 2 * m + 1), b0, b1);
-      else
-        mma_s8(acc.S, kOnes, kOnes, kOnes, kOnes, b0, b1);
-      if constexpr (ASYM && MASK) mma_s8(Sg, kOnes, kOnes, kOnes, kOnes, b0, b1);
-    }
-    // promote the group sums: R[0..1] row r0, R[2..3] row r1
-    if constexpr (ASYM) {
-      if constexpr (!MASK) {
+    for (int kg = 0; kg < NT; ++kg) {
+      Acc& ac = acc[kg];
+      // activation codes of this lane's 32 channels for its MMA column
+      uint32_t xw[8];
+      {
+        const int4* xp = reinterpret_cast<const int4*>(xrow[kg] + cg * kTileK);
+        int4 a, b;
+        if constexpr (FUSED) {
+          a = xp[0];
+          b = xp[1];
+        } else {
+          a = __ldg(xp);
+          b = __ldg(xp + 1);
+        }
+        xw[0] = a.x; xw[1] = a.y; xw[2] = a.z; xw[3] = a.w;
+        xw[4] = b.x; xw[5] = b.y; xw[6] = b.z; xw[7] = b.w;
+      }
+      int R[4] = {0, 0, 0, 0};
+      // asymmetric residual: the tile's activation sum S_g per token, from the
+      // all-ones MMA (the growth of ac.S over the tile; with a mask, its own)
+      const int S0[4] = {ac.S[0], ac.S[1], ac.S[2], ac.S[3]};
+      int Sg[4] = {0, 0, 0, 0};
 #pragma unroll
-        for (int i = 0; i < 4; ++i) Sg[i] = acc.S[i] - S0[i];
+      for (int m = 0; m < 4; ++m) {
+        const uint32_t b0 = xw[2 * m], b1 = xw[2 * m + 1];
+        if constexpr (RES)
+          mma_s8(R, tl.q[4 * m], tl.q[4 * m + 1], tl.q[4 * m + 2], tl.q[4 * m + 3], b0, b1);
+        mma_s8(ac.Pn, bits_word(pb0, 2 * m), bits_word(pb1, 2 * m), bits_word(pb0, 2 * m + 1),
+               bits_word(pb1, 2 * m + 1), b0, b1);
+        if constexpr (MASK)
+          mma_s8(ac.S, bits_word(tl.m[0], 2 * m), bits_word(tl.m[1], 2 * m),
+                 bits_word(tl.m[0], 2 * m + 1), bits_word(tl.m[1], 2 * m + 1), b0, b1);
+        else
+          mma_s8(ac.S, kOnes, kOnes, kOnes, kOnes, b0, b1);
+        if constexpr (ASYM && MASK) mma_s8(Sg, kOnes, kOnes, kOnes, kOnes, b0, b1);
       }
+      // promote the group sums: R[0..1] row r0, R[2..3] row r1
+      if constexpr (ASYM) {
+        if constexpr (!MASK) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const long long d = (long long)R[i] - (long long)tl.z[i >> 1] * (long long)Sg[i];
-        acc.F[i] = fmaf(tl.c[i >> 1], (float)d, acc.F[i]);
+          for (int i = 0; i < 4; ++i) Sg[i] = ac.S[i] - S0[i];
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const long long d = (long long)R[i] - (long long)tl.z[i >> 1] * (long long)Sg[i];
+          ac.F[i] = fmaf(tl.c[i >> 1], (float)d, ac.F[i]);
+        }
+      } else if constexpr (RES) {
+        ac.F[0] = fmaf(tl.c[0], (float)R[0], ac.F[0]);
+        ac.F[1] = fmaf(tl.c[0], (float)R[1], ac.F[1]);
+        ac.F[2] = fmaf(tl.c[1], (float)R[2], ac.F[2]);
+        ac.F[3] = fmaf(tl.c[1], (float)R[3], ac.F[3]);
       }
-    } else if constexpr (RES) {
-      acc.F[0] = fmaf(tl.c[0], (float)R[0], acc.F[0]);
-      acc.F[1] = fmaf(tl.c[0], (float)R[1], acc.F[1]);
-      acc.F[2] = fmaf(tl.c[1], (float)R[2], acc.F[2]);
-      acc.F[3] = fmaf(tl.c[1], (float)R[3], acc.F[3]);
-    }
-    (void)S0;
-    (void)Sg;
-    if (EMIT) {
-      const int ng = p.tpr;
-      const int r0 = rb * kTileRows + gid, r1 = r0 + 8;
-      if (tk0 < p.M) {
-        if (r0 < p.N) p.R_out[((int64_t)tk0 * p.N + r0) * ng + cg] = R[0];
-        if (r1 < p.N) p.R_out[((int64_t)tk0 * p.N + r1) * ng + cg] = R[2];
-      }
-      if (tk1 < p.M) {
-        if (r0 < p.N) p.R_out[((int64_t)tk1 * p.N + r0) * ng + cg] = R[1];
-        if (r1 < p.N) p.R_out[((int64_t)tk1 * p.N + r1) * ng + cg] = R[3];
+      (void)S0;
+      (void)Sg;
+      if (EMIT) {
+        const int ng = p.tpr;
+        const int r0 = rb * kTileRows + gid, r1 = r0 + 8;
+        const int a0 = tk0 + 8 * kg, a1 = tk1 + 8 * kg;
+        if (a0 < p.M) {
+          if (r0 < p.N) p.R_out[((int64_t)a0 * p.N + r0) * ng + cg] = R[0];
+          if (r1 < p.N) p.R_out[((int64_t)a0 * p.N + r1) * ng + cg] = R[2];
+        }
+        if (a1 < p.M) {
+          if (r0 < p.N) p.R_out[((int64_t)a1 * p.N + r0) * ng + cg] = R[1];
+          if (r1 < p.N) p.R_out[((int64_t)a1 * p.N + r1) * ng + cg] = R[3];
+        }
       }
     }
     // outlier channels of this tile (the same for every row): the lane
@@ -765,22 +777,27 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
         // (an index list that is not strictly ascending cannot push pos
         // past the list)
         if (pos >= 0 && pos < p.n_out) {
-          float x0, x1;
-          if constexpr (FUSED) {
-            x0 = tk0 < p.M ? xo_s[tk0 * p.n_pad + pos] : 0.0f;
-            x1 = tk1 < p.M ? xo_s[tk1 * p.n_pad + pos] : 0.0f;
-          } else {
-            x0 = tk0 < p.M ? __ldg(p.xout + (int64_t)tk0 * p.n_out + pos) : 0.0f;
-            x1 = tk1 < p.M ? __ldg(p.xout + (int64_t)tk1 * p.n_out + pos) : 0.0f;
+#pragma unroll
+          for (int kg = 0; kg < NT; ++kg) {
+            const int a0 = tk0 + 8 * kg, a1 = tk1 + 8 * kg;
+            float x0, x1;
+            if constexpr (FUSED) {
+              x0 = a0 < p.M ? xo_s[a0 * p.n_pad + pos] : 0.0f;
+              x1 = a1 < p.M ? xo_s[a1 * p.n_pad + pos] : 0.0f;
+            } else {
+              x0 = a0 < p.M ? __ldg(p.xout + (int64_t)a0 * p.n_out + pos) : 0.0f;
+              x1 = a1 < p.M ? __ldg(p.xout + (int64_t)a1 * p.n_out + pos) : 0.0f;
+            }
+            Acc& ac = acc[kg];
+            ac.Ut[0] = fmaf(u0, x0, ac.Ut[0]);
+            ac.Ut[1] = fmaf(u0, x1, ac.Ut[1]);
+            ac.Ut[2] = fmaf(u1, x0, ac.Ut[2]);
+            ac.Ut[3] = fmaf(u1, x1, ac.Ut[3]);
+            ac.Ur[0] = fmaf(w0, x0, ac.Ur[0]);
+            ac.Ur[1] = fmaf(w0, x1, ac.Ur[1]);
+            ac.Ur[2] = fmaf(w1, x0, ac.Ur[2]);
+            ac.Ur[3] = fmaf(w1, x1, ac.Ur[3]);
           }
-          acc.Ut[0] = fmaf(u0, x0, acc.Ut[0]);
-          acc.Ut[1] = fmaf(u0, x1, acc.Ut[1]);
-          acc.Ut[2] = fmaf(u1, x0, acc.Ut[2]);
-          acc.Ut[3] = fmaf(u1, x1, acc.Ut[3]);
-          acc.Ur[0] = fmaf(w0, x0, acc.Ur[0]);
-          acc.Ur[1] = fmaf(w0, x1, acc.Ur[1]);
-          acc.Ur[2] = fmaf(w1, x0, acc.Ur[2]);
-          acc.Ur[3] = fmaf(w1, x1, acc.Ur[3]);
         }
         ++pos;
       }
@@ -795,31 +812,36 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
 
     // end of a row block, or end of this warp's range
     if (cg == p.tpr - 1 || t + 1 == t1) {
-      float4 v[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        v[i] = cell(trunk_T<MASK>(acc, i), acc.F[i], acc.Ut[i], acc.Ur[i]);
-      if (EMIT) {
-        const int r0 = rb * kTileRows + gid, r1 = r0 + 8;
-        if (tk0 < p.M && r0 < p.N) atomicAdd(&p.T_out[(int64_t)tk0 * p.N + r0], trunk_T<MASK>(acc, 0));
-        if (tk1 < p.M && r0 < p.N) atomicAdd(&p.T_out[(int64_t)tk1 * p.N + r0], trunk_T<MASK>(acc, 1));
-        if (tk0 < p.M && r1 < p.N) atomicAdd(&p.T_out[(int64_t)tk0 * p.N + r1], trunk_T<MASK>(acc, 2));
-        if (tk1 < p.M && r1 < p.N) atomicAdd(&p.T_out[(int64_t)tk1 * p.N + r1], trunk_T<MASK>(acc, 3));
-      }
-      if (rb_head && cg == p.tpr - 1) {
-        write_y(p, rb, gid, tid4, v, al0, al1, sx0, sx1);
-      } else {
-        // a shared row block: slot 1 if this piece starts the row block
-        // (this range ends inside it), slot 0 if it continues one begun
-        // before this range
-        const int slot = rb_head ? 1 : 0;
+      for (int kg = 0; kg < NT; ++kg) {
+        const Acc& ac = acc[kg];
+        const int a0 = tk0 + 8 * kg, a1 = tk1 + 8 * kg;
+        float4 v[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int tk = (i & 1) ? tk1 : tk0;
-          if (tk < p.M) part_s[((warp * 2 + slot) * 16 + (i >> 1) * 8 + gid) * p.M + tk] = v[i];
+        for (int i = 0; i < 4; ++i) v[i] = cell(trunk_T<MASK>(ac, i), ac.F[i], ac.Ut[i], ac.Ur[i]);
+        if (EMIT) {
+          const int r0 = rb * kTileRows + gid, r1 = r0 + 8;
+          if (a0 < p.M && r0 < p.N) atomicAdd(&p.T_out[(int64_t)a0 * p.N + r0], trunk_T<MASK>(ac, 0));
+          if (a1 < p.M && r0 < p.N) atomicAdd(&p.T_out[(int64_t)a1 * p.N + r0], trunk_T<MASK>(ac, 1));
+          if (a0 < p.M && r1 < p.N) atomicAdd(&p.T_out[(int64_t)a0 * p.N + r1], trunk_T<MASK>(ac, 2));
+          if (a1 < p.M && r1 < p.N) atomicAdd(&p.T_out[(int64_t)a1 * p.N + r1], trunk_T<MASK>(ac, 3));
+        }
+        if (rb_head && cg == p.tpr - 1) {
+          write_y(p, rb, gid, tid4, v, al0, al1, sx0[kg], sx1[kg], 8 * kg);
+        } else {
+          // a shared row block: slot 1 if this piece starts the row block
+          // (this range ends inside it), slot 0 if it continues one begun
+          // before this range
+          const int slot = rb_head ? 1 : 0;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int tk = (i & 1) ? a1 : a0;
+            if (tk < p.M) part_s[((warp * 2 + slot) * 16 + (i >> 1) * 8 + gid) * p.M + tk] = v[i];
+          }
         }
       }
-      acc_zero(acc);
+#pragma unroll
+      for (int kg = 0; kg < NT; ++kg) acc_zero(acc[kg]);
       rb_head = true;
       if (cg == p.tpr - 1 && t + 1 < t1) {
         // the next row block starts: its row scales, needed at its end
@@ -842,28 +864,31 @@ __global__ void __launch_bounds__(kThreads, kBps) k_linear_tc(const Params p) {
   const int rb_last = (t1 - 1) / p.tpr;
   if (rb_last * p.tpr >= t0 && t1 % p.tpr != 0) {
     const int w_hi = tile_warp((rb_last + 1) * p.tpr - 1, T0c, T1c);
-    // (cells of tokens past M were never stored and are not written)
-    auto cell_at = [&](int w, int slot, int i) -> const float4& {
-      const int tk = min((i & 1) ? tk1 : tk0, p.M - 1);
-      return part_s[((w * 2 + slot) * 16 + (i >> 1) * 8 + gid) * p.M + tk];
-    };
-    float4 v[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) v[i] = cell_at(warp, 1, i);
-    for (int w = warp + 1; w <= w_hi; ++w) {
-      // a CTA with fewer tiles than warps has empty warps between its owners
-      if (warp_first_tile(w, T0c, T1c) == warp_first_tile(w + 1, T0c, T1c)) continue;
+    for (int kg = 0; kg < NT; ++kg) {
+      // (cells of tokens past M were never stored and are not written)
+      auto cell_at = [&](int w, int slot, int i) -> const float4& {
+        const int tk = min(((i & 1) ? tk1 : tk0) + 8 * kg, p.M - 1);
+        return part_s[((w * 2 + slot) * 16 + (i >> 1) * 8 + gid) * p.M + tk];
+      };
+      float4 v[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) cell_add(v[i], cell_at(w, 0, i));
+      for (int i = 0; i < 4; ++i) v[i] = cell_at(warp, 1, i);
+      for (int w = warp + 1; w <= w_hi; ++w) {
+        // a CTA with fewer tiles than warps has empty warps between its owners
+        if (warp_first_tile(w, T0c, T1c) == warp_first_tile(w + 1, T0c, T1c)) continue;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) cell_add(v[i], cell_at(w, 0, i));
+      }
+      write_y(p, rb_last, gid, tid4, v, al0, al1, sx0[kg], sx1[kg], 8 * kg);
     }
-    write_y(p, rb_last, gid, tid4, v, al0, al1, sx0, sx1);
   }
 }
 
 template <bool MASK, bool EMIT, bool FUSED, int D, bool RES = true, bool SPARSE = false,
-          bool ASYM = false>
+          bool ASYM = false, int NT = 1>
 cudaError_t launch_one(const Params& p, int grid, int smem, bool pdl, cudaStream_t stream) {
-  auto* fn = k_linear_tc<MASK, EMIT, FUSED, D, RES, SPARSE, ASYM>;
+  auto* fn = k_linear_tc<MASK, EMIT, FUSED, D, RES, SPARSE, ASYM, NT>;
   cudaError_t e = ensure_smem_attr((const void*)fn, smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -880,30 +905,52 @@ cudaError_t launch_one(const Params& p, int grid, int smem, bool pdl, cudaStream
 }
 
 // kind: 0 dense symmetric residual, 1 sparse, 2 asymmetric.
-template <bool MASK, bool FUSED, int D>
+template <bool MASK, bool FUSED, int D, int NT>
 cudaError_t launch_plain(const Params& p, bool res, int kind, int grid, int smem, bool pdl,
                          cudaStream_t stream) {
-  if (!res) return launch_one<MASK, false, FUSED, kTrunkDepth, false>(p, grid, smem, pdl, stream);
-  if (kind == 1) return launch_one<MASK, false, FUSED, D, true, true>(p, grid, smem, pdl, stream);
+  if (!res)
+    return launch_one<MASK, false, FUSED, kTrunkDepth, false, false, false, NT>(p, grid, smem, pdl,
+                                                                               stream);
+  if (kind == 1)
+    return launch_one<MASK, false, FUSED, D, true, true, false, NT>(p, grid, smem, pdl, stream);
   if (kind == 2)
-    return launch_one<MASK, false, FUSED, D, true, false, true>(p, grid, smem, pdl, stream);
-  return launch_one<MASK, false, FUSED, D, true, false>(p, grid, smem, pdl, stream);
+    return launch_one<MASK, false, FUSED, D, true, false, true, NT>(p, grid, smem, pdl, stream);
+  return launch_one<MASK, false, FUSED, D, true, false, false, NT>(p, grid, smem, pdl, stream);
 }
 
-// Non-accumulator launch with a ring depth chosen at run time among Ds.
+// Non-accumulator launch with a ring depth chosen at run time among Ds; two
+// token groups (NT = 2) only from global codes (the fused split stages at
+// most kCols tokens).
 template <int D0, int... Ds>
-cudaError_t launch_depth(int depth, bool mask, bool fused, bool res, int kind, const Params& p,
-                         int grid, int smem, bool pdl, cudaStream_t stream) {
+cudaError_t launch_depth(int depth, bool mask, bool fused, bool res, int kind, int nt,
+                         const Params& p, int grid, int smem, bool pdl, cudaStream_t stream) {
   if (depth == D0 || sizeof...(Ds) == 0) {
     if (fused)
-      return mask ? launch_plain<true, true, D0>(p, res, kind, grid, smem, pdl, stream)
-                  : launch_plain<false, true, D0>(p, res, kind, grid, smem, pdl, stream);
-    return mask ? launch_plain<true, false, D0>(p, res, kind, grid, smem, pdl, stream)
-                : launch_plain<false, false, D0>(p, res, kind, grid, smem, pdl, stream);
+      return mask ? launch_plain<true, true, D0, 1>(p, res, kind, grid, smem, pdl, stream)
+                  : launch_plain<false, true, D0, 1>(p, res, kind, grid, smem, pdl, stream);
+    if (nt == 2)
+      return mask ? launch_plain<true, false, D0, 2>(p, res, kind, grid, smem, pdl, stream)
+                  : launch_plain<false, false, D0, 2>(p, res, kind, grid, smem, pdl, stream);
+    return mask ? launch_plain<true, false, D0, 1>(p, res, kind, grid, smem, pdl, stream)
+                : launch_plain<false, false, D0, 1>(p, res, kind, grid, smem, pdl, stream);
   }
   if constexpr (sizeof...(Ds) > 0)
-    return launch_depth<Ds...>(depth, mask, fused, res, kind, p, grid, smem, pdl, stream);
+    return launch_depth<Ds...>(depth, mask, fused, res, kind, nt, p, grid, smem, pdl, stream);
   return cudaErrorInvalidValue;
+}
+
+// Accumulator-mode launch (two-tile ring).
+template <int NT>
+cudaError_t launch_emit(bool mask, int kind, const Params& p, int grid, int smem, bool pdl,
+                        cudaStream_t stream) {
+  if (kind == 1)
+    return mask ? launch_one<true, true, false, kShallow, true, true, false, NT>(p, grid, smem, pdl, stream)
+                : launch_one<false, true, false, kShallow, true, true, false, NT>(p, grid, smem, pdl, stream);
+  if (kind == 2)
+    return mask ? launch_one<true, true, false, kShallow, true, false, true, NT>(p, grid, smem, pdl, stream)
+                : launch_one<false, true, false, kShallow, true, false, true, NT>(p, grid, smem, pdl, stream);
+  return mask ? launch_one<true, true, false, kShallow, true, false, false, NT>(p, grid, smem, pdl, stream)
+              : launch_one<false, true, false, kShallow, true, false, false, NT>(p, grid, smem, pdl, stream);
 }
 
 }  // namespace
@@ -940,6 +987,15 @@ int trunk_ring_bytes(bool mask) {
 }
 }  // namespace
 
+int linear_tc_pass_tokens(const sq_packed_weight& w, bool trunk_only) {
+  // two token groups per pass where 2 kCols tokens' partial sums fit beside
+  // the shallow ring (every shape whose outlier table is small enough)
+  const int ring = trunk_only ? trunk_ring_bytes(w.mask_bits != nullptr)
+                              : ring_bytes(w.mask_bits != nullptr, kShallow, residual_kind(w));
+  const int need = kSmemPartPerToken * 2 * kCols + outlier_table_bytes(w) + 16 + ring;
+  return need <= kSmemMax ? 2 * kCols : kCols;
+}
+
 int linear_tc_fused_tokens(const sq_packed_weight& w, int n_out) {
   // counted with the shallow ring; the deep one is used when it fits
   const int fixed = ring_bytes(w.mask_bits != nullptr, kShallow, residual_kind(w)) +
@@ -957,7 +1013,7 @@ cudaError_t launch_linear_tc(const sq_packed_weight& w, int M, const int8_t* xq,
                              bool trunk_only, cudaStream_t stream) {
   const int kind = residual_kind(w);
   const bool sparse = kind == 1;
-  if (M < 1 || M > kCols) return cudaErrorInvalidValue;
+  if (M < 1 || M > linear_tc_pass_tokens(w, trunk_only)) return cudaErrorInvalidValue;
   if (w.layout != SQ_LAYOUT_TILES && w.layout != SQ_LAYOUT_TILES_SPARSE &&
       w.layout != SQ_LAYOUT_TILES_ASYM)
     return cudaErrorInvalidValue;
@@ -966,6 +1022,7 @@ cudaError_t launch_linear_tc(const sq_packed_weight& w, int M, const int8_t* xq,
   if (trunk_only && T_out) return cudaErrorInvalidValue;
   const bool fused = x != nullptr;
   if (fused && (T_out || M > linear_tc_fused_tokens(w, n_out))) return cudaErrorInvalidValue;
+  const int nt = M > kCols ? 2 : 1;
   Params p;
   p.res = w.res_q;
   p.sign = w.sign_bits;
@@ -1024,18 +1081,11 @@ cudaError_t launch_linear_tc(const sq_packed_weight& w, int M, const int8_t* xq,
   smem += trunk_only ? trunk_ring_bytes(mask) : ring_bytes(mask, depth, kind);
   if (smem > kSmemMax) return cudaErrorInvalidValue;
   const int grid = (int)blocks;
-  if (emit) {
-    if (sparse)
-      return mask ? launch_one<true, true, false, kShallow, true, true>(p, grid, smem, pdl, stream)
-                  : launch_one<false, true, false, kShallow, true, true>(p, grid, smem, pdl, stream);
-    if (kind == 2)
-      return mask ? launch_one<true, true, false, kShallow, true, false, true>(p, grid, smem, pdl, stream)
-                  : launch_one<false, true, false, kShallow, true, false, true>(p, grid, smem, pdl, stream);
-    return mask ? launch_one<true, true, false, kShallow>(p, grid, smem, pdl, stream)
-                : launch_one<false, true, false, kShallow>(p, grid, smem, pdl, stream);
-  }
-  return launch_depth<kDeep, kShallow>(depth, mask, fused, !trunk_only, kind, p, grid, smem, pdl,
-                                       stream);
+  if (emit)
+    return nt == 2 ? launch_emit<2>(mask, kind, p, grid, smem, pdl, stream)
+                   : launch_emit<1>(mask, kind, p, grid, smem, pdl, stream);
+  return launch_depth<kDeep, kShallow>(depth, mask, fused, !trunk_only, kind, nt, p, grid, smem,
+                                       pdl, stream);
 }
 
 }  // namespace sq

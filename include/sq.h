@@ -352,6 +352,16 @@ sq_status sq_quantize_linear(const sq_packed_weight *w, const float *x, int32_t 
 size_t sq_quantize_linear_workspace_bytes(const sq_packed_weight *w, int32_t M, int32_t n_out);
 
 /*
+ * Tokens that share one read of the weights in sq_linear's decode kernels for
+ * this weight and flags (SQ_TRUNK_ONLY or 0): for the tiled layouts 16 where
+ * the partial sums of 16 tokens fit in one CTA's shared memory beside its
+ * tile ring (every shape up to K = 28672 with the dense symmetric residual),
+ * else 8; for SQ_LAYOUT_ROWS 4 (below the prefill kernel's token count).  M
+ * tokens take ceil(M / this) launches.  0 for an invalid weight or flags.
+ */
+int32_t sq_linear_tokens_per_pass(const sq_packed_weight *w, uint32_t flags);
+
+/*
  * Tokens per launch of sq_quantize_linear's fused kernel for this weight and
  * outlier count (1..8; 0 if not even one token fits, or for an invalid
  * weight or a weight in SQ_LAYOUT_ROWS).

@@ -181,6 +181,29 @@ def test_fused_tokens_per_pass(L):
     assert L.sq_quantize_linear_tokens_per_pass(None, 0) == 0
 
 
+def test_linear_tokens_per_pass(L):
+    """Tokens per weight read of sq_linear follow the shared-memory arithmetic:
+    16 when 16 tokens' partial sums (8192 bytes each) + the outlier table
+    (roundup(K,128)/4 bytes) + 16 + a ring of two slots per warp (16 warps;
+    2560 bytes, 2816 with a mask or for the sparse / asymmetric residual,
+    3072 for both; six 256-byte slots, 512 with a mask, in the trunk-only
+    mode) fit in 227 KiB - 256; else 8.  The row layout: 4.  Host-only."""
+    def view(K, mask=False, layout=1):
+        v = sq.SqPackedWeight()
+        assert L.sq_packed_view(ctypes.c_void_p(1 << 40), 64, K, 128, int(mask), layout, ctypes.byref(v)) == 0
+        return v
+    for K, mask, layout, flags, want in [
+            (4096, False, 1, 0, 16), (28672, False, 1, 0, 16), (65536, False, 1, 0, 16),
+            (81920, False, 1, 0, 8), (43904, True, 1, 0, 16), (44032, True, 1, 0, 8),
+            (43904, False, 2, 0, 16), (44032, False, 3, 0, 8), (11008, True, 2, 0, 16),
+            (11264, True, 2, 0, 8), (11264, True, 3, 0, 8), (28672, True, 3, 0, 8),
+            (81920, True, 1, 2, 16), (4096, False, 0, 0, 4), (4096, False, 0, 2, 0)]:
+        assert L.sq_linear_tokens_per_pass(ctypes.byref(view(K, mask, layout)), flags) == want, \
+            (K, mask, layout, flags)
+    assert L.sq_linear_tokens_per_pass(ctypes.byref(view(4096)), 1) == 0  # PDL is not a pass flag
+    assert L.sq_linear_tokens_per_pass(None, 0) == 0
+
+
 def test_missing_library_fails_loudly():
     """Without the built CUDA library every entry point raises: there is no
     CPU fallback.  Run in a child process so this process keeps its loaded
