@@ -74,6 +74,18 @@ def _load():
             lib.sqo_abs_dot.argtypes = [i64, i64, i64, vp, vp, vp]
             lib.sqo_layer_sq_error.argtypes = [i64, i64, i32, vp, vp, vp, vp, vp, vp, vp, vp]
             lib.sqo_plain_sq_error.argtypes = [i64, i64, i32, vp, vp]
+            lib.sqo_e2m1_value.argtypes = [i32]
+            lib.sqo_e2m1_value.restype = dbl
+            lib.sqo_e2m1_round.argtypes = [dbl]
+            lib.sqo_e2m1_round.restype = i32
+            lib.sqo_ue4m3_value.argtypes = [i32]
+            lib.sqo_ue4m3_value.restype = dbl
+            lib.sqo_ue4m3_round.argtypes = [dbl]
+            lib.sqo_ue4m3_round.restype = i32
+            lib.sqo_nvfp4_quantize.argtypes = [vp, i64, i64, i32, vp, vp, vp]
+            lib.sqo_nvfp4_quantize.restype = i32
+            lib.sqo_nvfp4_linear.argtypes = [i64, i64, i64, vp, vp, ctypes.c_float, vp, vp, vp, vp]
+            lib.sqo_nvfp4_linear.restype = i32
             for name in ("sqo_quantize_groups", "sqo_trunk_threshold", "sqo_decompose",
                          "sqo_calibrate", "sqo_quantize_act", "sqo_accumulate",
                          "sqo_trunk_popcount", "sqo_linear", "sqo_linear_naive", "sqo_linear_trunk",
@@ -363,3 +375,50 @@ def choose_fallback(W, P: int = -1, G: int = 128) -> bool:
     nothing from the split falls back to plain 8-bit): fall back when plain
     INT8 groups reconstruct W at least as well as the split does."""
     return plain_sq_error(W, G) <= layer_sq_error(decompose(W, G=G, P=P), W)
+
+
+# ---- NVFP4 prefill format (the ISTA-DASLab page on separated quantization,
+# paragraphs 2-4: hardware-native NVFP4 for prefill).  The format's reading is
+# in sq_oracle.h.
+
+def e2m1_value(code: int) -> float:
+    return float(_load().sqo_e2m1_value(int(code)))
+
+
+def e2m1_round(v: float) -> int:
+    return int(_load().sqo_e2m1_round(float(v)))
+
+
+def ue4m3_value(code: int) -> float:
+    return float(_load().sqo_ue4m3_value(int(code)))
+
+
+def ue4m3_round(v: float) -> int:
+    return int(_load().sqo_ue4m3_round(float(v)))
+
+
+def nvfp4_quantize(X, per_row: bool):
+    """X [R][K] -> dict(codes [R][K] uint8 (one E2M1 code per byte), scales
+    [R][ceil(K/16)] uint8 (UE4M3), g [R] float32 (per row) or [1] (per
+    tensor))."""
+    X = _c(X, np.float32)
+    R, K = X.shape
+    codes = np.zeros((R, K), np.uint8)
+    scales = np.zeros((R, (K + 15) // 16), np.uint8)
+    g = np.zeros(R if per_row else 1, np.float32)
+    _ck(_load().sqo_nvfp4_quantize(_p(X), R, K, int(bool(per_row)), _p(codes), _p(scales), _p(g)),
+        "sqo_nvfp4_quantize")
+    return {"codes": codes, "scales": scales, "g": g}
+
+
+def nvfp4_linear(w, x):
+    """y [M][N] (binary64) = sum_j What_rj * xhat_tj for a per-tensor
+    quantized weight w and per-token quantized activations x."""
+    wc, ws = _c(w["codes"], np.uint8), _c(w["scales"], np.uint8)
+    xc, xs, gx = _c(x["codes"], np.uint8), _c(x["scales"], np.uint8), _c(x["g"], np.float32)
+    N, K = wc.shape
+    M = xc.shape[0]
+    y = np.zeros((M, N), np.float64)
+    _ck(_load().sqo_nvfp4_linear(M, N, K, _p(wc), _p(ws), float(w["g"][0]), _p(xc), _p(xs),
+                                 _p(gx), _p(y)), "sqo_nvfp4_linear")
+    return y

@@ -580,3 +580,126 @@ int sqo_plain_sq_error(int64_t N, int64_t K, int G, const float *W, double *err)
     *err = total;
     return SQO_OK;
 }
+
+/* ---- NVFP4: the prefill format of format separation ---------------------
+ * [P4] (the ISTA-DASLab page on separated quantization, paragraphs 2-4):
+ * prefill runs in the hardware's native quantized format, NVFP4, while
+ * decode keeps its own low-bit weight-only format.  The page names the
+ * format without defining it; the reading taken is the format as the
+ * Blackwell tensor cores consume it:
+ *   element  E2M1: sign, 2 exponent bits (bias 1), 1 mantissa bit; the
+ *            magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6 in code order 0..7, the
+ *            sign in bit 3; a value that rounds to 0 is stored as +0;
+ *   block    16 consecutive elements along K share one UE4M3 scale (no
+ *            sign, 4 exponent bits with bias 7, 3 mantissa bits; largest
+ *            finite 448, code 127 is NaN and never produced);
+ *   second   a binary32 scale g = amax / (6 * 448) per weight tensor, and
+ *   level    per token for activations.
+ * Quantization of x in block b: s_b = RNE_ue4m3(amax_b / (6 g)), then
+ * q = RNE_e2m1(x / (s_b g)), saturating at 6; ties go to the even code.  A
+ * zero g or s_b gives all-zero codes.  The dequantized value is
+ * e2m1(q) * s_b * g. */
+
+static const double kE2M1Mag[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+
+double sqo_e2m1_value(int code)
+{
+    double m = kE2M1Mag[code & 7];
+    return (code & 8) ? -m : m;
+}
+
+int sqo_e2m1_round(double v)
+{
+    double a = fabs(v);
+    int best = 0;
+    for (int c = 1; c < 8; ++c) {
+        double dc = fabs(a - kE2M1Mag[c]), db = fabs(a - kE2M1Mag[best]);
+        if (dc < db || (dc == db && (c & 1) == 0))
+            best = c;
+    }
+    if (best == 0)
+        return 0;
+    return v < 0.0 ? (best | 8) : best;
+}
+
+double sqo_ue4m3_value(int code)
+{
+    int e = (code >> 3) & 15, m = code & 7;
+    if (e == 0)
+        return ldexp((double)m, -9);
+    return ldexp(1.0 + (double)m / 8.0, e - 7);
+}
+
+int sqo_ue4m3_round(double v)
+{
+    int best = 0;
+    for (int c = 1; c < 127; ++c) {
+        double dc = fabs(v - sqo_ue4m3_value(c)), db = fabs(v - sqo_ue4m3_value(best));
+        if (dc < db || (dc == db && c % 2 == 0))
+            best = c;
+    }
+    return best;
+}
+
+int sqo_nvfp4_quantize(const float *X, int64_t R, int64_t K, int per_row, uint8_t *codes,
+                       uint8_t *scales, float *g)
+{
+    if (!X || !codes || !scales || !g || R < 1 || K < 1)
+        return SQO_BAD_ARG;
+    const int64_t nb = (K + 15) / 16;
+    for (int64_t i = 0; i < R * K; ++i)
+        if (!isfinite(X[i]))
+            return SQO_NONFINITE;
+    double amax_all = 0.0;
+    if (!per_row)
+        for (int64_t i = 0; i < R * K; ++i)
+            if (fabs((double)X[i]) > amax_all)
+                amax_all = fabs((double)X[i]);
+    if (!per_row)
+        g[0] = (float)(amax_all / 2688.0);
+    for (int64_t r = 0; r < R; ++r) {
+        const float *x = X + r * K;
+        if (per_row) {
+            double a = 0.0;
+            for (int64_t j = 0; j < K; ++j)
+                if (fabs((double)x[j]) > a)
+                    a = fabs((double)x[j]);
+            g[r] = (float)(a / 2688.0);
+        }
+        const double gr = (double)(per_row ? g[r] : g[0]);
+        for (int64_t b = 0; b < nb; ++b) {
+            int64_t j0 = 16 * b, j1 = j0 + 16 < K ? j0 + 16 : K;
+            double ab = 0.0;
+            for (int64_t j = j0; j < j1; ++j)
+                if (fabs((double)x[j]) > ab)
+                    ab = fabs((double)x[j]);
+            int sc = gr == 0.0 ? 0 : sqo_ue4m3_round(ab / (6.0 * gr));
+            scales[r * nb + b] = (uint8_t)sc;
+            double step = sqo_ue4m3_value(sc) * gr;
+            for (int64_t j = j0; j < j1; ++j)
+                codes[r * K + j] = (uint8_t)(step == 0.0 ? 0 : sqo_e2m1_round((double)x[j] / step));
+        }
+    }
+    return SQO_OK;
+}
+
+int sqo_nvfp4_linear(int64_t M, int64_t N, int64_t K, const uint8_t *wc, const uint8_t *ws,
+                     float gw, const uint8_t *xc, const uint8_t *xs, const float *gx, double *y)
+{
+    if (!wc || !ws || !xc || !xs || !gx || !y || M < 1 || N < 1 || K < 1)
+        return SQO_BAD_ARG;
+    const int64_t nb = (K + 15) / 16;
+    for (int64_t t = 0; t < M; ++t)
+        for (int64_t r = 0; r < N; ++r) {
+            double acc = 0.0;
+            for (int64_t j = 0; j < K; ++j) {
+                double w = sqo_e2m1_value(wc[r * K + j]) * sqo_ue4m3_value(ws[r * nb + j / 16]) *
+                           (double)gw;
+                double x = sqo_e2m1_value(xc[t * K + j]) * sqo_ue4m3_value(xs[t * nb + j / 16]) *
+                           (double)gx[t];
+                acc += w * x;
+            }
+            y[t * N + r] = acc;
+        }
+    return SQO_OK;
+}

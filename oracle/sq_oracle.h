@@ -185,6 +185,28 @@ int sqo_plain_sq_error(int64_t N, int64_t K, int G, const float *W, double *err)
 int sqo_abs_dot(int64_t M, int64_t N, int64_t K, const float *W,
                 const float *x, double *out);
 
+/* ---- NVFP4 prefill format ([P4], the ISTA-DASLab page on separated
+ * quantization, paragraphs 2-4: prefill in the hardware's native NVFP4,
+ * decode in its own weight-only format).  The page does not define the
+ * format; the reading taken (the format the Blackwell tensor cores read):
+ *   E2M1 elements (magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6; bit 3 = sign; a
+ *   value rounding to 0 is +0), blocks of 16 along K with a UE4M3 scale
+ *   (bias 7, 3 mantissa bits, largest 448), and a binary32 second-level
+ *   scale g = amax / (6 * 448): per tensor for weights, per token (row) for
+ *   activations.  s_b = RNE_ue4m3(amax_b / (6 g)); q = RNE_e2m1(x / (s_b g))
+ *   saturating at 6; ties to the even code; g = 0 or s_b = 0 -> codes 0.
+ *   Codes one per byte, [R][K]; scales [R][ceil(K/16)]. */
+double sqo_e2m1_value(int code);
+int sqo_e2m1_round(double v);
+double sqo_ue4m3_value(int code);
+int sqo_ue4m3_round(double v);  /* v >= 0 */
+int sqo_nvfp4_quantize(const float *X, int64_t R, int64_t K, int per_row, uint8_t *codes,
+                       uint8_t *scales, float *g);
+/* y_tr = sum_j What_rj * xhat_tj (binary64, ascending j) with
+ * What = e2m1(wc) * ue4m3(ws) * gw and xhat = e2m1(xc) * ue4m3(xs) * gx[t]. */
+int sqo_nvfp4_linear(int64_t M, int64_t N, int64_t K, const uint8_t *wc, const uint8_t *ws,
+                     float gw, const uint8_t *xc, const uint8_t *xs, const float *gx, double *y);
+
 #ifdef __cplusplus
 }
 #endif

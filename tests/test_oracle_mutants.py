@@ -83,6 +83,21 @@ MUTANTS = {
                                        "double t = mask[r * K + j] ? (sign[r * K + j] ? -(double)alpha[r] : (double)alpha[r]) : 0.0;\n            int64_t zz"),
     "plain_error_without_quantizer_clip": ("double d = w - (double)sg * (double)sqo_quantize(w, sg);",
                                            "double d = w - (double)sg * round(w / (double)sg * 1.001);"),
+    "e2m1_ties_to_odd": ("if (dc < db || (dc == db && (c & 1) == 0))",
+                         "if (dc < db || (dc == db && (c & 1) == 1))"),
+    "e2m1_negative_zero": ("    if (best == 0)\n        return 0;\n    return v < 0.0",
+                           "    return v < 0.0"),
+    "ue4m3_bias_8": ("return ldexp(1.0 + (double)m / 8.0, e - 7);",
+                     "return ldexp(1.0 + (double)m / 8.0, e - 8);"),
+    "ue4m3_ties_away": ("if (dc < db || (dc == db && c % 2 == 0))", "if (dc <= db)"),
+    "nvfp4_scale_without_six": ("sqo_ue4m3_round(ab / (6.0 * gr))", "sqo_ue4m3_round(ab / gr)"),
+    "nvfp4_tensor_scale_448": ("g[0] = (float)(amax_all / 2688.0);", "g[0] = (float)(amax_all / 448.0);"),
+    "nvfp4_row_scale_448": ("g[r] = (float)(a / 2688.0);", "g[r] = (float)(a / 448.0);"),
+    "nvfp4_block_drops_last": ("int64_t j0 = 16 * b, j1 = j0 + 16 < K ? j0 + 16 : K;",
+                               "int64_t j0 = 16 * b, j1 = j0 + 15 < K ? j0 + 15 : K;"),
+    "nvfp4_linear_drops_weight_scale": ("                           (double)gw;", "                           1.0;"),
+    "nvfp4_linear_token_scale_of_row": ("                           (double)gx[t];",
+                                        "                           (double)gx[0];"),
 }
 
 

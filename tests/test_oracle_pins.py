@@ -696,3 +696,177 @@ def test_generator_statistics():
     w3 = L3.weights(rows=np.arange(4))
     heavy = np.abs(w3) > 6 * 0.015
     assert 0.0003 < heavy.mean() < 0.003
+
+
+# ---- NVFP4 prefill format -------------------------------------------------------
+# The ISTA-DASLab page on separated quantization (paragraphs 2-4) names NVFP4
+# as the prefill format without defining it; the pins below follow from the
+# format's bit fields (E2M1: 1 sign, 2 exponent bits with bias 1, 1 mantissa
+# bit; UE4M3: 4 exponent bits with bias 7, 3 mantissa bits, code 127 NaN),
+# round-to-nearest-even and the two-level scale rule.
+
+def _e2m1_from_fields(code):
+    e, m = (code >> 1) & 3, code & 1
+    mag = m * 0.5 if e == 0 else (1.0 + m / 2.0) * 2.0 ** (e - 1)
+    return -mag if code & 8 else mag
+
+
+def test_e2m1_values_follow_the_bit_fields():
+    for c in range(16):
+        assert oracle.e2m1_value(c) == _e2m1_from_fields(c), c
+    assert sorted({abs(oracle.e2m1_value(c)) for c in range(16)}) == [0, 0.5, 1, 1.5, 2, 3, 4, 6]
+
+
+def test_ue4m3_values_known_points_and_spacing():
+    """1.0 at 0x38, 448 at 0x7E (largest finite), 2^-9 at 0x01, 2^-6 at 0x08
+    (smallest normal); strictly increasing; 8 values per binade above it."""
+    assert oracle.ue4m3_value(0x38) == 1.0
+    assert oracle.ue4m3_value(0x7E) == 448.0
+    assert oracle.ue4m3_value(0x01) == 2.0 ** -9
+    assert oracle.ue4m3_value(0x08) == 2.0 ** -6
+    assert oracle.ue4m3_value(0x07) == 7 * 2.0 ** -9
+    v = [oracle.ue4m3_value(c) for c in range(127)]
+    assert all(b > a for a, b in zip(v, v[1:]))
+    for e in range(1, 15):
+        assert sum(1 for x in v if 2.0 ** (e - 7) <= x < 2.0 ** (e - 6)) == 8
+
+
+def _nearest_even(v, grid, codes):
+    d = np.abs(np.asarray(grid) - v)
+    best = np.flatnonzero(d == d.min())
+    return [codes[i] for i in best if codes[i] % 2 == 0][0] if len(best) > 1 else codes[best[0]]
+
+
+def test_e2m1_round_ties_saturation_and_brute_force():
+    mags = [abs(_e2m1_from_fields(c)) for c in range(8)]
+    # ties: to the even code (mantissa bit 0)
+    for v, want in [(0.25, 0), (0.75, 2), (1.25, 2), (1.75, 4), (2.5, 4), (3.5, 6), (5.0, 6)]:
+        assert oracle.e2m1_round(v) == want, v
+        assert oracle.e2m1_round(-v) == (want | 8 if want else 0), -v
+    assert oracle.e2m1_round(100.0) == 7 and oracle.e2m1_round(-6.01) == 15
+    assert oracle.e2m1_round(-0.2) == 0 and oracle.e2m1_round(-0.0) == 0  # +0 for a zero result
+    rng = np.random.default_rng(5)
+    for v in np.concatenate([rng.uniform(-7, 7, 3000), np.array(mags), -np.array(mags)]):
+        c = oracle.e2m1_round(float(v))
+        want = _nearest_even(abs(v), mags, list(range(8)))
+        assert c == (want | 8 if (v < 0 and want) else want), v
+
+
+def test_ue4m3_round_ties_saturation_and_brute_force():
+    vals = [oracle.ue4m3_value(c) for c in range(127)]
+    rng = np.random.default_rng(6)
+    pts = np.concatenate([np.exp(rng.uniform(np.log(2.0 ** -11), np.log(500.0), 3000)),
+                          [(a + b) / 2 for a, b in zip(vals, vals[1:])], vals])
+    for v in pts:
+        assert oracle.ue4m3_round(float(v)) == _nearest_even(min(v, 1e9), vals, list(range(127))), v
+    assert oracle.ue4m3_round(1000.0) == 126
+    assert oracle.ue4m3_round(2.0 ** -10) == 0          # the tie between 0 and 2^-9
+    assert oracle.ue4m3_round(1.0 + 1.0 / 16) == 0x38   # the tie between 1 and 1.125: even
+    assert oracle.ue4m3_round(1.125 + 1.0 / 16) == 0x3A
+
+
+def _exact_nvfp4_rows(rng, R, nb, g):
+    """Rows whose every element is e2m1 * s_b * g exactly, each block holding
+    +-6 * s_b * g, and block 0 holding 6 * 448 * g: the quantizer must
+    reconstruct them exactly and find exactly these codes."""
+    scode = rng.integers(8, 127, size=(R, nb))
+    scode[:, 0] = 126
+    codes = rng.integers(0, 16, size=(R, nb * 16))
+    codes[codes == 8] = 0
+    for r in range(R):
+        for b in range(nb):
+            j = 16 * b + rng.integers(0, 16)
+            codes[r, j] = 7 | (8 * int(rng.integers(0, 2)))
+    X = np.zeros((R, nb * 16), np.float64)
+    for r in range(R):
+        for j in range(nb * 16):
+            X[r, j] = _e2m1_from_fields(codes[r, j]) * oracle.ue4m3_value(scode[r, j // 16]) * g[r]
+    return X.astype(np.float32), codes.astype(np.uint8), scode.astype(np.uint8)
+
+
+def test_nvfp4_exact_rows_reconstruct_exactly():
+    rng = np.random.default_rng(7)
+    g = 2.0 ** rng.integers(-12, -2, size=6)
+    X, codes, scode = _exact_nvfp4_rows(rng, 6, 5, g)
+    d = oracle.nvfp4_quantize(X, per_row=True)
+    assert np.array_equal(d["g"], g.astype(np.float32))
+    assert np.array_equal(d["scales"], scode)
+    assert np.array_equal(d["codes"], codes)
+    # per tensor: g is the largest row's, here the same for every row
+    Xs = X[:1].repeat(3, axis=0)
+    dt = oracle.nvfp4_quantize(Xs, per_row=False)
+    assert dt["g"].shape == (1,) and dt["g"][0] == np.float32(g[0])
+    assert np.array_equal(dt["codes"], codes[:1].repeat(3, axis=0))
+
+
+def test_nvfp4_scale_rule_and_block_maximum():
+    """g = float(amax / 2688) (per row, and per tensor = the largest row's);
+    the block scale is the nearest UE4M3 to amax_b / (6 g); with a normal
+    block scale the block's largest |x| gets the code of 6 (amax_b / (s_b g)
+    lies within 6 * [1/(1+2^-4), 1/(1-2^-4)], nearer 6 than 4); every code is
+    the nearest E2M1 level of x / (s_b g) (ties to even); a ragged last block
+    (K = 40) and an all-zero row."""
+    rng = np.random.default_rng(8)
+    X = (rng.standard_normal((7, 40)) * np.exp(rng.uniform(-3, 3, (7, 1)))).astype(np.float32)
+    X[:, 3] *= 20.0
+    X[4] = 0.0
+    d = oracle.nvfp4_quantize(X, per_row=True)
+    dt = oracle.nvfp4_quantize(X, per_row=False)
+    amax = np.abs(X.astype(np.float64)).max(axis=1)
+    assert np.array_equal(d["g"], (amax / 2688.0).astype(np.float32))
+    assert dt["g"][0] == np.float32(amax.max() / 2688.0)
+    vals = [oracle.ue4m3_value(c) for c in range(127)]
+    mags = [abs(_e2m1_from_fields(c)) for c in range(8)]
+    for q, gg in ((d, d["g"].astype(np.float64)), (dt, np.full(7, float(dt["g"][0])))):
+        assert q["scales"].shape == (7, 3)
+        assert not q["codes"][4].any() and not q["scales"][4].any()
+        for r in range(7):
+            for b in range(3):
+                blk = X[r, 16 * b: 16 * b + 16].astype(np.float64)
+                if gg[r] == 0:
+                    continue
+                ab = np.abs(blk).max()
+                sc = q["scales"][r, b]
+                assert sc == _nearest_even(ab / (6.0 * gg[r]), vals, list(range(127)))
+                step = vals[sc] * gg[r]
+                if vals[sc] >= 2.0 ** -6:
+                    assert q["codes"][r, 16 * b + int(np.abs(blk).argmax())] & 7 == 7
+                for j, v in enumerate(blk):
+                    c = int(q["codes"][r, 16 * b + j])
+                    want = _nearest_even(abs(v) / step, mags, list(range(8))) if step else 0
+                    assert c == (want | 8 if (v < 0 and want) else want)
+
+
+def test_nvfp4_linear_exact_and_second_route():
+    """Exact rows: y equals the exact dot products of the original values
+    (Fraction arithmetic).  Random rows: y equals the dequantized operands
+    (formed from the bit fields and scales in numpy) multiplied in binary64,
+    to 1e-12 of sum |What * xhat|."""
+    rng = np.random.default_rng(9)
+    gw = np.full(4, 2.0 ** -7)
+    Wx, _, _ = _exact_nvfp4_rows(rng, 4, 3, gw)
+    gx = 2.0 ** rng.integers(-9, -4, size=3)
+    Xx, _, _ = _exact_nvfp4_rows(rng, 3, 3, gx)
+    w = oracle.nvfp4_quantize(Wx, per_row=False)
+    x = oracle.nvfp4_quantize(Xx, per_row=True)
+    y = oracle.nvfp4_linear(w, x)
+    for t in range(3):
+        for r in range(4):
+            exact = sum(F(a) * F(b) for a, b in zip(Wx[r], Xx[t]))
+            assert Fraction(y[t, r]) == exact
+    L = wl.config2_layer(0, 0)
+    W = L.weights(rows=np.arange(12))[:, :300]
+    xa = L.activations(M=3)[:, :300]
+    w = oracle.nvfp4_quantize(W, per_row=False)
+    x = oracle.nvfp4_quantize(xa, per_row=True)
+    y = oracle.nvfp4_linear(w, x)
+    e2 = np.array([_e2m1_from_fields(c) for c in range(16)])
+    u4 = np.array([oracle.ue4m3_value(c) for c in range(127)])
+    Wh = e2[w["codes"]] * np.repeat(u4[w["scales"]], 16, axis=1)[:, :300] * float(w["g"][0])
+    Xh = e2[x["codes"]] * np.repeat(u4[x["scales"]], 16, axis=1)[:, :300] * \
+        x["g"].astype(np.float64)[:, None]
+    ref = Xh @ Wh.T
+    assert np.all(np.abs(y - ref) <= 1e-12 * (np.abs(Xh) @ np.abs(Wh).T))
+    # and it stays near the unquantized product (4-bit elements: a loose bound)
+    exact = xa.astype(np.float64) @ W.astype(np.float64).T
+    assert np.all(np.abs(y - exact) <= 0.1 * (np.abs(xa.astype(np.float64)) @ np.abs(W.astype(np.float64)).T))
