@@ -55,6 +55,14 @@ class SqPackedWeight(ctypes.Structure):
     ]
 
 
+class SqNvfp4Matrix(ctypes.Structure):
+    _fields_ = [
+        ("rows", ctypes.c_int32), ("K", ctypes.c_int32), ("per_row", ctypes.c_int32),
+        ("rows_pad", ctypes.c_int32), ("code_stride", ctypes.c_int32), ("sf_chunks", ctypes.c_int32),
+        ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("g", ctypes.c_void_p),
+    ]
+
+
 _lib = None
 
 
@@ -69,7 +77,12 @@ def lib():
     L = ctypes.CDLL(LIB_PATH)
     vp, i32, u32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_uint32, ctypes.c_size_t
     pw = ctypes.POINTER(SqPackedWeight)
+    nm = ctypes.POINTER(SqNvfp4Matrix)
     sig = {
+        "sq_nvfp4_bytes": ([i32, i32, i32], sz),
+        "sq_nvfp4_view": ([vp, i32, i32, i32, nm], ctypes.c_int),
+        "sq_nvfp4_quantize": ([vp, nm, vp, vp], ctypes.c_int),
+        "sq_nvfp4_linear": ([nm, nm, vp, vp, vp], ctypes.c_int),
         "sq_status_string": ([ctypes.c_int], ctypes.c_char_p),
         "sq_device_check": ([], ctypes.c_int),
         "sq_packed_bytes": ([i32, i32, i32, i32, i32], sz),
@@ -440,3 +453,74 @@ def linear_accumulators(pw: PackedWeight, xq, sx, x_out, idx, workspace=None, st
                                      workspace.numel(), _ptr(status), _flags(False),
                                      _stream(stream)), "sq_linear_accumulators")
     return y, T, R
+
+
+# ---- NVFP4 prefill (format separation; include/sq.h documents the format) ----
+
+@dataclass
+class Nvfp4Matrix:
+    """An NVFP4 matrix [rows][K] in one device allocation with its C view."""
+    rows: int
+    K: int
+    per_row: bool
+    buf: object                 # torch.uint8 device tensor
+    view: SqNvfp4Matrix
+
+    def _arr(self, field: str, dtype, count: int):
+        import torch
+        off = getattr(self.view, field) - self.buf.data_ptr()
+        itemsize = torch.empty(0, dtype=dtype).element_size()
+        return self.buf[off:off + count * itemsize].view(dtype)
+
+    def codes(self):
+        """[rows_pad][code_stride] uint8, two E2M1 codes a byte."""
+        import torch
+        v = self.view
+        return self._arr("codes", torch.uint8, v.rows_pad * v.code_stride).view(v.rows_pad,
+                                                                                v.code_stride)
+
+    def scales(self):
+        """The UE4M3 scale chunks, flat: [rows_pad/128 * sf_chunks * 512] uint8."""
+        import torch
+        v = self.view
+        return self._arr("scales", torch.uint8, (v.rows_pad // 128) * v.sf_chunks * 512)
+
+    def g(self):
+        """Second-level scales: [rows] (per row) or [1] (per tensor)."""
+        import torch
+        return self._arr("g", torch.float32, self.view.rows_pad if self.per_row else 1)[
+            :self.rows if self.per_row else 1]
+
+
+def alloc_nvfp4(rows: int, K: int, per_row: bool, device=None) -> Nvfp4Matrix:
+    import torch
+    nbytes = lib().sq_nvfp4_bytes(rows, K, int(per_row))
+    if nbytes == 0:
+        raise SQError(STATUS_CODE["SQ_ERR_SHAPE"], "sq_nvfp4_bytes")
+    buf = torch.empty(nbytes, dtype=torch.uint8, device=device or "cuda")
+    v = SqNvfp4Matrix()
+    _ck(lib().sq_nvfp4_view(_ptr(buf), rows, K, int(per_row), ctypes.byref(v)), "sq_nvfp4_view")
+    return Nvfp4Matrix(rows, K, bool(per_row), buf, v)
+
+
+def nvfp4_quantize(X, per_row: bool, out: Nvfp4Matrix = None, status=None,
+                   stream=None) -> Nvfp4Matrix:
+    """X[rows][K] (float32, device) -> NVFP4 (per tensor for a weight, per
+    row for activations)."""
+    rows, K = X.shape
+    if out is None:
+        out = alloc_nvfp4(rows, K, per_row, device=X.device)
+    _ck(lib().sq_nvfp4_quantize(_ptr(X), ctypes.byref(out.view), _ptr(status), _stream(stream)),
+        "sq_nvfp4_quantize")
+    return out
+
+
+def nvfp4_linear(w: Nvfp4Matrix, x: Nvfp4Matrix, y=None, status=None, stream=None):
+    """y [x.rows][w.rows] float32 = dequantized x @ dequantized w^T on the
+    block-scaled tensor cores."""
+    import torch
+    if y is None:
+        y = torch.empty(x.rows, w.rows, dtype=torch.float32, device=x.buf.device)
+    _ck(lib().sq_nvfp4_linear(ctypes.byref(w.view), ctypes.byref(x.view), _ptr(y), _ptr(status),
+                              _stream(stream)), "sq_nvfp4_linear")
+    return y

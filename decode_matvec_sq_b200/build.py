@@ -36,6 +36,7 @@ SOURCES = [
     ("sq_linear_tc.cu", []),
     ("sq_noalloc.cu", []),
     ("sq_prefill.cu", []),
+    ("sq_nvfp4.cu", ["-fmad=false"]),
 ]
 
 

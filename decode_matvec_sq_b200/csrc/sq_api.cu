@@ -493,6 +493,96 @@ sq_status sq_quantize_linear(const sq_packed_weight* w, const float* x, int32_t 
   return SQ_OK;
 }
 
+// ---- NVFP4 prefill ------------------------------------------------------------
+
+static bool nvfp4_shape(int32_t rows, int32_t K) {
+  return rows >= 1 && K >= 1 && rows <= (1 << 24) && K <= (1 << 20);
+}
+
+struct Nvfp4Carve {
+  size_t codes, scales, g, total;
+  int32_t rows_pad, code_stride, sf_chunks;
+};
+
+static Nvfp4Carve nvfp4_carve(int32_t rows, int32_t K, int32_t per_row) {
+  Nvfp4Carve c;
+  c.rows_pad = (int32_t)round_up(rows, 128);
+  const int64_t k256 = round_up(K, 256);
+  c.code_stride = (int32_t)(k256 / 2);
+  c.sf_chunks = (int32_t)(k256 / 64);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t at = off;
+    off = (size_t)round_up((int64_t)(off + bytes), 256);
+    return at;
+  };
+  c.codes = take((size_t)c.rows_pad * c.code_stride);
+  c.scales = take((size_t)(c.rows_pad / 128) * c.sf_chunks * 512);
+  c.g = take(per_row ? (size_t)c.rows_pad * 4 : 8);
+  c.total = off;
+  return c;
+}
+
+static sq_status check_nvfp4(const sq_nvfp4_matrix* m) {
+  if (!m || !m->codes || !m->scales || !m->g) return SQ_ERR_INVALID_ARG;
+  if (m->per_row != 0 && m->per_row != 1) return SQ_ERR_INVALID_ARG;
+  if (!nvfp4_shape(m->rows, m->K)) return SQ_ERR_SHAPE;
+  const Nvfp4Carve c = nvfp4_carve(m->rows, m->K, m->per_row);
+  if (m->rows_pad != c.rows_pad || m->code_stride != c.code_stride || m->sf_chunks != c.sf_chunks)
+    return SQ_ERR_SHAPE;
+  if (!aligned16(m->codes) || !aligned16(m->scales) || !aligned16(m->g)) return SQ_ERR_ALIGN;
+  return SQ_OK;
+}
+
+size_t sq_nvfp4_bytes(int32_t rows, int32_t K, int32_t per_row) {
+  if (!nvfp4_shape(rows, K) || (per_row != 0 && per_row != 1)) return 0;
+  return nvfp4_carve(rows, K, per_row).total;
+}
+
+sq_status sq_nvfp4_view(void* base, int32_t rows, int32_t K, int32_t per_row,
+                        sq_nvfp4_matrix* out) {
+  if (!base || !out || (per_row != 0 && per_row != 1)) return SQ_ERR_INVALID_ARG;
+  if (!nvfp4_shape(rows, K)) return SQ_ERR_SHAPE;
+  if ((reinterpret_cast<uintptr_t>(base) & 255u) != 0) return SQ_ERR_ALIGN;
+  const Nvfp4Carve c = nvfp4_carve(rows, K, per_row);
+  uint8_t* b = static_cast<uint8_t*>(base);
+  out->rows = rows;
+  out->K = K;
+  out->per_row = per_row;
+  out->rows_pad = c.rows_pad;
+  out->code_stride = c.code_stride;
+  out->sf_chunks = c.sf_chunks;
+  out->codes = b + c.codes;
+  out->scales = b + c.scales;
+  out->g = reinterpret_cast<float*>(b + c.g);
+  return SQ_OK;
+}
+
+sq_status sq_nvfp4_quantize(const float* X, const sq_nvfp4_matrix* out, int32_t* dev_status,
+                            void* stream) {
+  sq_status st = check_nvfp4(out);
+  if (st != SQ_OK) return st;
+  if (!X) return SQ_ERR_INVALID_ARG;
+  if (!aligned16(X)) return SQ_ERR_ALIGN;
+  DeviceInfo d;
+  if ((st = check_device(&d)) != SQ_OK) return st;
+  return from_cuda(launch_nvfp4_quantize(X, *out, dev_status, static_cast<cudaStream_t>(stream)));
+}
+
+sq_status sq_nvfp4_linear(const sq_nvfp4_matrix* w, const sq_nvfp4_matrix* x, float* y,
+                          int32_t* dev_status, void* stream) {
+  sq_status st = check_nvfp4(w);
+  if (st != SQ_OK) return st;
+  if ((st = check_nvfp4(x)) != SQ_OK) return st;
+  if (!y) return SQ_ERR_INVALID_ARG;
+  if (w->per_row != 0 || x->per_row != 1) return SQ_ERR_INVALID_ARG;
+  if (w->K != x->K) return SQ_ERR_SHAPE;
+  if (!aligned16(y)) return SQ_ERR_ALIGN;
+  DeviceInfo d;
+  if ((st = check_device(&d)) != SQ_OK) return st;
+  return from_cuda(launch_nvfp4_gemm(*w, *x, y, dev_status, static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"
 
 // ---- failure injection for the tests (include/sq_testing.h) -----------------------

@@ -99,6 +99,14 @@ constexpr int kPrefillMinTokens = 64;
 bool prefill_supported(const sq_packed_weight& w);
 // wait_ns bounds every wait of the kernel; skip_group >= 0 (tests only) never
 // requests that channel group's operands, so the kernel's waits run out.
+// NVFP4 prefill (sq_nvfp4.cu): the quantizer (per tensor: amax reduction,
+// then the quantizer; per row: one kernel) and the block-scaled tcgen05 GEMM.
+cudaError_t launch_nvfp4_quantize(const float* X, const sq_nvfp4_matrix& out, int32_t* status,
+                                  cudaStream_t stream);
+cudaError_t launch_nvfp4_gemm(const sq_nvfp4_matrix& w, const sq_nvfp4_matrix& x, float* y,
+                              int32_t* status, cudaStream_t stream,
+                              uint64_t wait_ns = 1000000000ull);
+
 cudaError_t launch_prefill(const sq_packed_weight& w, int M, const int8_t* xq, const float* sx,
                            const float* x_out, const int32_t* idx, int n_out, float* y,
                            int32_t* T_out, int32_t* R_out, int32_t* status, cudaStream_t stream,

@@ -28,15 +28,12 @@
 // commits to a last barrier and waits (bounded) until its MMAs are done, so
 // no copy still writes shared memory and no MMA still writes tensor memory
 // when the CTA frees it and exits.
-#include <cuda.h>
-#include <cudaTypedefs.h>
 #include <stdint.h>
 
 #include <algorithm>
-#include <mutex>
 
-#include "sq_common.cuh"
 #include "sq_internal.h"
+#include "sq_tcgen05.cuh"
 
 namespace sq {
 namespace {
@@ -92,24 +89,6 @@ struct Params {
   int skip_group;    // failure injection for tests: this group's operands are never requested (-1: none)
 };
 
-// ---- PTX wrappers ---------------------------------------------------------------
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
-                                            uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
-      "%3}], [%4];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
-      : "memory");
-}
-
-// K-major operand with 128-byte swizzle: rows of 128 bytes, 8-row atoms 1024
-// bytes apart (stride byte offset), leading byte offset 1 (unused by this
-// mode), descriptor version 1, layout type 2.
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t addr) {
-  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
-         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
-}
-
 // D (s32) += A (s8, K-major) * B (s8, K-major), M = 128, N = 64.
 constexpr uint32_t kIdesc = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                             ((uint32_t)(BM >> 4) << 24);
@@ -122,32 +101,13 @@ __device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t a, uint64_t b, 
       "l"(a), "l"(b), "r"(kIdesc), "r"(acc ? 1 : 0));
 }
 
-__device__ __forceinline__ void mma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   smem_u32(bar))
-               : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-
-// 32 consecutive TMEM columns of this thread's lane.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, int (&r)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
-      "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
-        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
-        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
+using tc05::fence_after;
+using tc05::fence_before;
+using tc05::make_map;
+using tc05::mma_commit;
+using tc05::sw128_desc;
+using tc05::tma_load_2d;
+using tc05::tmem_ld32;
 
 // int32 -> float for |r| < 2^22 (group sums are below 2^21, trunk sums below
 // 2^22 for K < 33000): the integer lands in the mantissa of 1.5 * 2^23.
@@ -219,9 +179,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int n = n0 + threadIdx.x - 128;
     aux->alpha[threadIdx.x - 128] = n < p.N ? __ldg(p.alpha + n) : 0.0f;
   }
-  tc_fence_before();
+  fence_before();
   __syncthreads();
-  tc_fence_after();
+  fence_after();
   const uint32_t tmem = aux->tmem_base;
 
   if (warp == 0) {
@@ -264,7 +224,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (kb >= kAccBufs &&
             !wait_or_abort(&aux->acce[b], ((uint32_t)(kb / kAccBufs) & 1u) ^ 1u, aux, p))
           break;
-        tc_fence_after();
+        fence_after();
         const uint32_t st = smem_u32(smem + s * kStageBytes);
 #pragma unroll
         for (int kk = 0; kk < BK / 32; ++kk) {
@@ -338,13 +298,13 @@ __global__ void __launch_bounds__(kThreads, 2)
                 wait_or_abort(&aux->accf[b], (uint32_t)(kb / kAccBufs) & 1u, aux, p);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) continue;
-      tc_fence_after();
+      fence_after();
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         int r[32];
         tmem_ld32(tmem + ((uint32_t)lb << 16) + 64 + 64 * b + 32 * h, r);
         if (h == 1) {
-          tc_fence_before();
+          fence_before();
           mbar_arrive(&aux->acce[b]);
         }
 #pragma unroll
@@ -371,7 +331,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     named_sync_epi();
     fin = !aborted(aux) && fin;
     if (fin) {
-      tc_fence_after();
+      fence_after();
       const float sxt = t < p.M ? __ldg(p.sx + t) : 0.0f;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
@@ -432,41 +392,13 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
     }
   }
-  tc_fence_before();
+  fence_before();
   __syncthreads();
   if (warp == 1) {
-    tc_fence_after();
+    fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
                  : "memory");
   }
-}
-
-// ---- host: tensor maps -------------------------------------------------------------
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
-
-bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int esize, const void* base, uint64_t inner,
-              uint64_t rows, uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows,
-              CUtensorMapSwizzle sw) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[2] = {inner, rows};
-  const cuuint64_t strides[1] = {row_bytes};
-  const cuuint32_t box[2] = {box_inner, box_rows};
-  const cuuint32_t es[2] = {1, 1};
-  (void)esize;
-  return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <bool MASK, bool EMIT>
@@ -482,7 +414,7 @@ cudaError_t launch_prefill_t(const CUtensorMap& a, const CUtensorMap& b, const C
 }  // namespace
 
 bool prefill_supported(const sq_packed_weight& w) {
-  return w.layout == SQ_LAYOUT_ROWS && w.group_size == BK && encode_fn() != nullptr;
+  return w.layout == SQ_LAYOUT_ROWS && w.group_size == BK && tc05::encode_fn() != nullptr;
 }
 
 cudaError_t launch_prefill(const sq_packed_weight& w, int M, const int8_t* xq, const float* sx,
@@ -492,15 +424,15 @@ cudaError_t launch_prefill(const sq_packed_weight& w, int M, const int8_t* xq, c
   if (!prefill_supported(w) || M < 1) return cudaErrorInvalidValue;
   const int64_t K128 = xq_stride_of(w.K);
   CUtensorMap ma, mb, ms, mm;
-  if (!make_map(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, xq, (uint64_t)K128, (uint64_t)M,
+  if (!make_map(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, (uint64_t)K128, (uint64_t)M,
                 (uint64_t)K128, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map(&mb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w.res_q, (uint64_t)w.res_stride,
+      !make_map(&mb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w.res_q, (uint64_t)w.res_stride,
                 (uint64_t)w.N, (uint64_t)w.res_stride, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map(&ms, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, w.sign_bits, (uint64_t)w.sign_stride,
+      !make_map(&ms, CU_TENSOR_MAP_DATA_TYPE_UINT32, w.sign_bits, (uint64_t)w.sign_stride,
                 (uint64_t)w.N, (uint64_t)w.sign_stride * 4, 4, BN, CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
   if (w.mask_bits) {
-    if (!make_map(&mm, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, w.mask_bits, (uint64_t)w.sign_stride,
+    if (!make_map(&mm, CU_TENSOR_MAP_DATA_TYPE_UINT32, w.mask_bits, (uint64_t)w.sign_stride,
                   (uint64_t)w.N, (uint64_t)w.sign_stride * 4, 4, BN, CU_TENSOR_MAP_SWIZZLE_NONE))
       return cudaErrorInvalidValue;
   } else {

@@ -394,6 +394,65 @@ sq_status sq_linear_noalloc(const sq_packed_weight *w, const int8_t *xq, const f
                             const float *x_out, const int32_t *idx, int32_t n_out, int32_t M,
                             float *y, int32_t *dev_status, uint32_t flags, void *stream);
 
+/* ---- NVFP4 prefill (format separation) ------------------------------------
+ * The ISTA-DASLab news page on separated quantization, paragraphs 2-4:
+ * prefill runs in the hardware's native quantized format, NVFP4, and decode
+ * keeps its own low-bit weight-only format (the packed weights above).  A
+ * layer then holds its weight twice: packed for decode and NVFP4 for
+ * prefill.  The page names NVFP4 without defining it; the format here is the
+ * one the B200 tensor cores read (tcgen05.mma kind::mxf4nvf4):
+ *   element  E2M1, two per byte (the lower channel in the low nibble), sign
+ *            in bit 3, magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6 in code order;
+ *   block    16 consecutive channels share a UE4M3 scale s_b (no sign, 4
+ *            exponent bits with bias 7, 3 mantissa bits, largest 448);
+ *   tensor   a float second-level scale g = amax / (6 * 448): one per weight
+ *            (per_row = 0), one per activation row, i.e. token (per_row = 1).
+ * Quantization: s_b = nearest UE4M3 to amax_b / (6 g), q = nearest E2M1 to
+ * x / (s_b g) saturating at +-6, ties to the even code, +0 for a zero
+ * result; g = 0 or s_b = 0 gives zero codes.  Dequantized: e2m1(q) s_b g.
+ *
+ * Layout of one matrix [rows][K] (sq_nvfp4_view carves one allocation):
+ *   codes   [rows_pad][code_stride] bytes, code_stride = roundup(K, 256) / 2,
+ *           rows_pad = roundup(rows, 128); pads are 0
+ *   scales  chunks of 512 bytes, chunk (rb, c) at byte 512 * (rb * sf_chunks
+ *           + c), sf_chunks = roundup(K, 256) / 64: byte 16 i + 4 w + s of
+ *           the chunk is the scale of row 128 rb + 32 w + i (i < 32, w < 4)
+ *           and block 4 c + s (the tensor core's scale-factor layout); pads 0
+ *   g       per_row: [rows_pad] floats (pads 0); else [2]: g, then a word the
+ *           quantizer uses as scratch
+ */
+typedef struct {
+  int32_t rows, K;
+  int32_t per_row;      /* 0: one second-level scale (a weight); 1: one per row */
+  int32_t rows_pad;     /* roundup(rows, 128) */
+  int32_t code_stride;  /* bytes per row of codes: roundup(K, 256) / 2 */
+  int32_t sf_chunks;    /* 64-channel scale chunks per 128-row block: roundup(K, 256) / 64 */
+  uint8_t *codes;
+  uint8_t *scales;
+  float *g;
+} sq_nvfp4_matrix;
+
+/* Bytes of one NVFP4 matrix (all three arrays, 256-byte aligned pieces);
+ * 0 for rows or K outside [1, 2^24] or [1, 2^20]. */
+size_t sq_nvfp4_bytes(int32_t rows, int32_t K, int32_t per_row);
+/* Carves `base` (sq_nvfp4_bytes of device memory, 256-byte aligned) into the
+ * arrays of *out.  No device access. */
+sq_status sq_nvfp4_view(void *base, int32_t rows, int32_t K, int32_t per_row,
+                        sq_nvfp4_matrix *out);
+/* Quantizes X [rows][K] (float, row-major) into *out (every array written,
+ * pads included).  Per tensor (per_row = 0) it reduces X's absolute maximum
+ * first (two kernels); per row it is one kernel.  Non-finite X sets
+ * SQ_ERR_NONFINITE in dev_status (the codes are then unspecified). */
+sq_status sq_nvfp4_quantize(const float *X, const sq_nvfp4_matrix *out, int32_t *dev_status,
+                            void *stream);
+/* y [x.rows][w.rows] (float, row-major) = sum_j What[n][j] * xhat[t][j] for
+ * a per-tensor weight w (N = w.rows) and per-row activations x (M = x.rows
+ * tokens) of the same K: one tcgen05 block-scaled GEMM launch, fp32
+ * accumulation in tensor memory, y = g_w * g_x[t] * D.  A bounded wait that
+ * runs out sets SQ_ERR_TIMEOUT in dev_status. */
+sq_status sq_nvfp4_linear(const sq_nvfp4_matrix *w, const sq_nvfp4_matrix *x, float *y,
+                          int32_t *dev_status, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -148,3 +148,25 @@ def pad_rows_are_zero(pw: "sq.PackedWeight") -> bool:
     parts = [u["sign"], u["alpha"], u["q"], u["s"]] + ([u["mask"]] if pw.with_mask else []) + \
         ([u["keep"]] if "keep" in u else []) + ([u["z"]] if "z" in u else [])
     return all(not np.asarray(a).view(np.uint8).any() for a in parts)
+
+
+def unpack_nvfp4(m: "sq.Nvfp4Matrix", rows=None) -> dict:
+    """An NVFP4 matrix read back as one E2M1 code per byte [rows][K256] and
+    one UE4M3 scale per 16-channel block [rows][K256/16], from the layout of
+    include/sq.h: codes two a byte, the lower channel in the low nibble;
+    scales in 512-byte chunks (rb, c), byte 16 i + 4 w + s = row
+    128 rb + 32 w + i, block 4 c + s.  rows=None: every padded row."""
+    v = m.view
+    if rows is None:
+        rows = np.arange(v.rows_pad)
+    rows = np.asarray(rows, dtype=np.int64)
+    cb = m.codes()[torch.as_tensor(rows, device=m.buf.device)].cpu().numpy()
+    codes = np.empty((len(rows), 2 * v.code_stride), np.uint8)
+    codes[:, 0::2] = cb & 15
+    codes[:, 1::2] = cb >> 4
+    nb = 2 * v.code_stride // 16
+    b = np.arange(nb, dtype=np.int64)[None, :]
+    r = rows[:, None]
+    off = ((r >> 7) * v.sf_chunks + (b >> 2)) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (b & 3)
+    scales = _gather(m.scales(), off)
+    return {"codes": codes, "scales": scales}

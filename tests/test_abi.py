@@ -204,6 +204,42 @@ def test_linear_tokens_per_pass(L):
     assert L.sq_linear_tokens_per_pass(None, 0) == 0
 
 
+def test_nvfp4_view_arithmetic(L):
+    """sq_nvfp4_bytes / sq_nvfp4_view: codes [roundup(rows,128)][roundup(K,256)/2],
+    scale chunks [rows_pad/128][roundup(K,256)/64][512], g [rows_pad] floats per
+    row or 2 per tensor, each piece 256-byte aligned; bad arguments refused.
+    Host-only: no device memory is touched."""
+    def r256(v):
+        return -(-v // 256) * 256
+    for rows, K, per_row in [(1, 16, 0), (130, 300, 1), (2048, 4096, 1), (14336, 4096, 0)]:
+        rp, k256 = -(-rows // 128) * 128, r256(K)
+        codes = r256(rp * k256 // 2)
+        scales = r256(rp // 128 * (k256 // 64) * 512)
+        gb = r256(rp * 4 if per_row else 8)
+        assert L.sq_nvfp4_bytes(rows, K, per_row) == codes + scales + gb
+        v = sq.SqNvfp4Matrix()
+        base = 1 << 40
+        assert L.sq_nvfp4_view(ctypes.c_void_p(base), rows, K, per_row, ctypes.byref(v)) == 0
+        assert (v.rows, v.K, v.per_row, v.rows_pad) == (rows, K, per_row, rp)
+        assert (v.code_stride, v.sf_chunks) == (k256 // 2, k256 // 64)
+        assert (v.codes, v.scales, v.g) == (base, base + codes, base + codes + scales)
+    v = sq.SqNvfp4Matrix()
+    assert L.sq_nvfp4_bytes(0, 16, 0) == 0 and L.sq_nvfp4_bytes(4, 16, 2) == 0
+    assert L.sq_nvfp4_view(ctypes.c_void_p((1 << 40) + 16), 4, 16, 0, ctypes.byref(v)) == 3
+    assert L.sq_nvfp4_view(None, 4, 16, 0, ctypes.byref(v)) == 1
+    assert L.sq_nvfp4_view(ctypes.c_void_p(1 << 40), 4, 0, 0, ctypes.byref(v)) == 2
+    # quantize / linear refuse bad views before any device work
+    assert L.sq_nvfp4_quantize(None, None, None, None) == 1
+    w, x = sq.SqNvfp4Matrix(), sq.SqNvfp4Matrix()
+    assert L.sq_nvfp4_view(ctypes.c_void_p(1 << 40), 64, 512, 0, ctypes.byref(w)) == 0
+    assert L.sq_nvfp4_view(ctypes.c_void_p(1 << 41), 8, 512, 1, ctypes.byref(x)) == 0
+    p = ctypes.c_void_p(1 << 42)
+    assert L.sq_nvfp4_linear(ctypes.byref(x), ctypes.byref(x), p, None, None) == 1  # weight per row
+    assert L.sq_nvfp4_linear(ctypes.byref(w), ctypes.byref(x), None, None, None) == 1
+    x.code_stride += 128
+    assert L.sq_nvfp4_linear(ctypes.byref(w), ctypes.byref(x), p, None, None) == 2
+
+
 def test_missing_library_fails_loudly():
     """Without the built CUDA library every entry point raises: there is no
     CPU fallback.  Run in a child process so this process keeps its loaded
