@@ -85,6 +85,21 @@ FALLBACK_BF16_TFLOPS = 1590.0
 INT8_PER_BF16 = 2.0  # nominal dense int8 : bf16 tensor throughput (4.5 : 2.25 P/s)
 
 
+FP4_PER_BF16 = 4.0  # nominal dense fp4 : bf16 tensor throughput (9 : 2.25 P/s)
+
+
+def load_fp4_peak():
+    """Dense NVFP4 tensor peak in TFLOP/s: the measured cuBLAS bf16 burst
+    figure times the nominal fp4/bf16 ratio."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]) * FP4_PER_BF16, "measured bf16 x nominal fp4/bf16 ratio"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS * FP4_PER_BF16, "fallback bf16 x nominal fp4/bf16 ratio"
+
+
 def load_int8_peak():
     """Dense int8 tensor peak in T int-ops/s: the measured cuBLAS bf16 burst
     figure times the nominal int8/bf16 ratio."""
@@ -649,6 +664,101 @@ def time_prefill_case(st, device, warmup, steps):
     return ms_step, ms_lin, 4 * L.M * L.N * L.K
 
 
+def time_nvfp4_prefill_case(st, device, warmup, steps):
+    """The prefill workload's shape (2048 tokens x 4096 -> 14336) in NVFP4
+    (format separation): the weight quantized once, then per step the
+    per-token activation quantizer and the block-scaled tcgen05 GEMM, with a
+    256 MB buffer written between steps (cold L2).  Device ms of the step and
+    of the GEMM alone, and the GEMM's 2*M*N*K flops."""
+    import torch
+    import decode_matvec_sq_b200 as sq
+    import synth.device as sdev
+    from synth import workloads as wl
+    L = wl.config5()
+    W = sdev.fill_weights(L, torch.empty(L.N, L.K, device=device))
+    w = sq.nvfp4_quantize(W, False, status=st)
+    del W
+    x = sdev.fill_activations(L, torch.empty(L.M, L.K, device=device))
+    a = sq.alloc_nvfp4(L.M, L.K, True, device=device)
+    y = torch.empty(L.M, L.N, device=device)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        sq.nvfp4_quantize(x, True, out=a, status=st)
+        sq.nvfp4_linear(w, a, y=y, status=st)
+    torch.cuda.synchronize()
+    ev = []
+    for _ in range(steps):
+        flush.fill_(1)
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        e[0].record(stream)
+        sq.nvfp4_quantize(x, True, out=a, status=st)
+        e[1].record(stream)
+        sq.nvfp4_linear(w, a, y=y, status=st)
+        e[2].record(stream)
+        ev.append(e)
+    torch.cuda.synchronize()
+    ms_step = sum(e[0].elapsed_time(e[2]) for e in ev) / len(ev)
+    ms_lin = sum(e[1].elapsed_time(e[2]) for e in ev) / len(ev)
+    del w, a, x, y, flush
+    torch.cuda.empty_cache()
+    return ms_step, ms_lin, 2 * L.M * L.N * L.K
+
+
+def run_prefill_nvfp4(args, world, rank, local):
+    """NVFP4 prefill (format separation) at the prefill workload's shape.
+    Tensor-bound: TFLOP/s of the GEMM's 2*M*N*K against the dense fp4 peak."""
+    import torch
+    import torch.distributed as dist
+    import decode_matvec_sq_b200 as sq
+    from decode_matvec_sq_b200 import build
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py: no CUDA device visible (the sq path has no CPU fallback)")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=device)
+    if rank == 0 or world == 1:
+        build.build_all()
+    barrier(world)
+    sq.device_check()
+    st = torch.zeros(1, dtype=torch.int32, device=device)
+    with ClockSampler(local) as clk:
+        barrier(world)
+        ms_step, ms_lin, flops = time_nvfp4_prefill_case(st, device, args.warmup, args.steps)
+        barrier(world)
+    clocks = clk.summary()
+    ms_step = max_over_ranks(ms_step, world, device)
+    ms_lin = max_over_ranks(ms_lin, world, device)
+    if st.item() != 0:
+        raise RuntimeError(f"device status {sq.STATUS.get(st.item())}")
+    peak, kind = load_fp4_peak()
+    achieved = flops / (ms_lin * 1e-3) / 1e12
+    if rank == 0:
+        print(json.dumps({
+            "metric": "prefill NVFP4 tensor TFLOP/s, 2048 tokens x 4096 -> 14336",
+            "value": round(world * flops / (ms_step * 1e-3) / 1e12, 1), "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic",
+            "config": {"workload": "prefill 2048 tokens x 4096 -> 14336 in NVFP4 (E2M1, UE4M3 "
+                                   "blocks of 16, per-tensor / per-token fp32 scales), W "
+                                   "Laplace(0,0.02), x N(0,1) with 0.5% channels x30",
+                       "l2": "a 256 MB buffer written between steps"},
+            "gpu_launches": 2 * args.steps,
+            "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak, 1),
+                         "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "peak_kind": kind,
+                         "traffic": None, "kernel": "k_nvfp4_gemm (tcgen05 kind::mxf4nvf4)",
+                         "us_per_launch": round(ms_lin * 1e3, 2)},
+            "clocks": clocks,
+        }), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
 def side_configs(device, warmup=3, reps=10):
     """Compact measurements of the other workloads, outside the headline's
     timed region: the 512 x 512 layer (hot and cold), the 70B-shaped MLP pair
@@ -678,6 +788,13 @@ def side_configs(device, warmup=3, reps=10):
                                        "t_intops_linear": round(ops / (ms_lin * 1e-3) / 1e12, 1),
                                        "frac_of_int8_peak": round(ops / (ms_lin * 1e-3) / 1e12 / peak, 4),
                                        "int8_peak_kind": kind}
+    ms_step, ms_lin, flops = time_nvfp4_prefill_case(st, device, warmup, reps)
+    peak, kind = load_fp4_peak()
+    out["prefill_nvfp4_2048x4096x14336"] = {"us_step": round(ms_step * 1e3, 1),
+                                             "us_gemm": round(ms_lin * 1e3, 1),
+                                             "tflops_gemm": round(flops / (ms_lin * 1e-3) / 1e12, 1),
+                                             "frac_of_fp4_peak": round(flops / (ms_lin * 1e-3) / 1e12 / peak, 4),
+                                             "fp4_peak_kind": kind}
     if st.item() != 0:
         raise RuntimeError(f"side configurations: device status {st.item()}")
     return out
@@ -934,11 +1051,12 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["sq", "reference"], default="sq")
     ap.add_argument("--layers", type=int, default=32)
-    ap.add_argument("--workload", choices=["decode", "prefill", "single", "mlp70b", "threshold",
-                                           "trunk", "sparse", "asym"],
+    ap.add_argument("--workload", choices=["decode", "prefill", "prefill_nvfp4", "single", "mlp70b",
+                                           "threshold", "trunk", "sparse", "asym"],
                     default="decode",
                     help="decode: the 7B-shaped stack at batch 1 (default); prefill: "
-                         "2048 tokens x 4096 -> 14336 on the tcgen05 kernel; single, mlp70b, "
+                         "2048 tokens x 4096 -> 14336 on the tcgen05 kernel; prefill_nvfp4: the "
+                         "same shape in NVFP4 (format separation); single, mlp70b, "
                          "threshold: single-layer workloads (512x512 hot/cold, the 70B-shaped "
                          "MLP pair at batch 1..16, the threshold-trunk layer); trunk: the "
                          "stack's four linears in the trunk-only mode")
@@ -960,6 +1078,8 @@ def main(argv=None):
         return run_reference(args, world, rank)
     if args.workload == "prefill":
         return run_prefill(args, world, rank, local)
+    if args.workload == "prefill_nvfp4":
+        return run_prefill_nvfp4(args, world, rank, local)
     if args.workload in ("single", "mlp70b", "threshold", "trunk", "sparse", "asym"):
         return run_layers(args, world, rank, local)
     return run_gpu(args, world, rank, local)

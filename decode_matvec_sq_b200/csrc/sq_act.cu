@@ -10,6 +10,8 @@
 // Built with -fmad=false.
 #include <stdint.h>
 
+#include <algorithm>
+
 #include "sq_common.cuh"
 #include "sq_internal.h"
 #include "sq_quant.cuh"
@@ -20,15 +22,17 @@ namespace {
 constexpr int kActThreads = 1024;
 constexpr int kCalThreads = 1024;
 
-// One CTA per token; warp w handles the 32-channel chunks w, w + 32, ...
-// with one channel per lane, keeping its x values in registers between the
-// absmax pass and the code pass (one global round trip).
-constexpr int kActRegs = 28;  // chunks per warp kept in registers: K <= 32*32*28
+// One CTA per token; with W warps, warp w handles the 32-channel chunks
+// w, w + W, ... with one channel per lane, keeping up to REGS of them in
+// registers between the absmax pass and the code pass (one global round
+// trip; chunks past W * REGS are read again).  A few tokens: 1024 threads
+// each (latency); many: CTAs sized to the row so that several fit an SM.
 
 __device__ __forceinline__ bool outlier_bit(const uint32_t* is_out, int j) {
   return (is_out[j >> 5] >> (j & 31)) & 1u;
 }
 
+template <int REGS>
 __global__ void __launch_bounds__(kActThreads) k_quantize_act(
     const float* __restrict__ x, int M, int K, int Kx, const int32_t* __restrict__ idx, int n_out,
     int8_t* __restrict__ xq, float* __restrict__ sx, float* __restrict__ x_out,
@@ -41,13 +45,14 @@ __global__ void __launch_bounds__(kActThreads) k_quantize_act(
   }
   const int t = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nw = blockDim.x >> 5;
   const int nchunk = (K + 31) >> 5;
   const float* xt = x + (int64_t)t * K;
   // x into registers (issued before anything else)
-  float v[kActRegs];
+  float v[REGS];
 #pragma unroll
-  for (int i = 0; i < kActRegs; ++i) {
-    const int j = (warp + 32 * i) * 32 + lane;
+  for (int i = 0; i < REGS; ++i) {
+    const int j = (warp + nw * i) * 32 + lane;
     v[i] = j < K ? __ldg(xt + j) : 0.0f;
   }
   for (int i = threadIdx.x; i < nchunk; i += blockDim.x) is_out[i] = 0u;
@@ -64,17 +69,17 @@ __global__ void __launch_bounds__(kActThreads) k_quantize_act(
 
   float a = 0.0f;
   bool nonfinite = false;
-  const bool big = nchunk > 32 * kActRegs;  // more chunks than registers: re-read x
+  const bool big = nchunk > nw * REGS;  // more chunks than registers: re-read x
 #pragma unroll
-  for (int i = 0; i < kActRegs; ++i) {
-    const int j = (warp + 32 * i) * 32 + lane;
+  for (int i = 0; i < REGS; ++i) {
+    const int j = (warp + nw * i) * 32 + lane;
     if (j < K) {
       nonfinite |= !isfinite(v[i]);
       if (!outlier_bit(is_out, j)) a = fmaxf(a, fabsf(v[i]));
     }
   }
   if (big) {
-    for (int c = warp + 32 * kActRegs; c < nchunk; c += 32) {
+    for (int c = warp + nw * REGS; c < nchunk; c += nw) {
       const int j = c * 32 + lane;
       if (j < K) {
         const float u = xt[j];
@@ -86,7 +91,7 @@ __global__ void __launch_bounds__(kActThreads) k_quantize_act(
   for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
   if (lane == 0) warp_max[warp] = a;
   __syncthreads();
-  a = warp_max[lane];
+  a = lane < nw ? warp_max[lane] : 0.0f;
   for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
 
   const float s = act_scale(a);
@@ -102,18 +107,18 @@ __global__ void __launch_bounds__(kActThreads) k_quantize_act(
     qt[j] = (int8_t)q;  // j < 32 * nchunk <= Kx
   };
 #pragma unroll
-  for (int i = 0; i < kActRegs; ++i) {
-    const int c = warp + 32 * i;
+  for (int i = 0; i < REGS; ++i) {
+    const int c = warp + nw * i;
     if (c < nchunk) emit(c, v[i]);
   }
   if (big) {
-    for (int c = warp + 32 * kActRegs; c < nchunk; c += 32) {
+    for (int c = warp + nw * REGS; c < nchunk; c += nw) {
       const int j = c * 32 + lane;
       emit(c, j < K ? xt[j] : 0.0f);
     }
   }
   // pad chunks up to the row stride (a multiple of 128 channels)
-  for (int c = nchunk + warp; c < (Kx >> 5); c += 32) qt[c * 32 + lane] = 0;
+  for (int c = nchunk + warp; c < (Kx >> 5); c += nw) qt[c * 32 + lane] = 0;
   if (nonfinite) set_status(status, SQ_ERR_NONFINITE);
   if (bad_idx) set_status(status, SQ_ERR_INVALID_ARG);
 }
@@ -195,16 +200,23 @@ __global__ void __launch_bounds__(kCalThreads) k_calibrate(const float* __restri
 
 }  // namespace
 
-cudaError_t launch_quantize_act(const float* x, int M, int K, const int32_t* idx, int n_out,
-                                int8_t* xq, float* sx, float* x_out, int32_t* status, bool pdl,
-                                cudaStream_t stream) {
-  const int Kx = (int)xq_stride_of(K);
-  const size_t smem = (size_t)ceil_div(K, 32) * sizeof(uint32_t);
-  cudaError_t e = ensure_smem_attr((const void*)k_quantize_act, (int)smem);
+namespace {
+// Register depths instantiated, and the launch shape for M tokens of K
+// channels: at least 2 tokens per SM -> warps = ceil(chunks / 16) (two
+// register rounds of 8 or more chunks per warp), else 1024 threads; the
+// depth is the smallest instantiated one covering the row, 28 at most.
+constexpr int kActDepths[] = {1, 2, 4, 8, 16, 28};
+
+template <int REGS>
+cudaError_t launch_act_t(const float* x, int M, int K, int Kx, const int32_t* idx, int n_out,
+                         int8_t* xq, float* sx, float* x_out, int32_t* status, bool pdl,
+                         int threads, size_t smem, cudaStream_t stream) {
+  auto* fn = k_quantize_act<REGS>;
+  cudaError_t e = ensure_smem_attr((const void*)fn, (int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(M);
-  cfg.blockDim = dim3(kActThreads);
+  cfg.blockDim = dim3(threads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -212,8 +224,36 @@ cudaError_t launch_quantize_act(const float* x, int M, int K, const int32_t* idx
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, k_quantize_act, x, M, K, Kx, idx, n_out, xq, sx, x_out, status,
-                            pdl ? 1 : 0);
+  return cudaLaunchKernelEx(&cfg, fn, x, M, K, Kx, idx, n_out, xq, sx, x_out, status, pdl ? 1 : 0);
+}
+}  // namespace
+
+cudaError_t launch_quantize_act(const float* x, int M, int K, const int32_t* idx, int n_out,
+                                int8_t* xq, float* sx, float* x_out, int32_t* status, bool pdl,
+                                cudaStream_t stream) {
+  const int Kx = (int)xq_stride_of(K);
+  const size_t smem = (size_t)ceil_div(K, 32) * sizeof(uint32_t);
+  const int nchunk = (int)ceil_div(K, 32);
+  DeviceInfo d;
+  const int sms = current_device(&d) ? d.sm_count : 148;
+  int warps = 32;
+  if (M >= 2 * sms) warps = std::min(32, std::max(1, (int)ceil_div(nchunk, 16)));
+  const int need = (int)ceil_div(nchunk, warps);
+  int regs = kActDepths[5];
+  for (int r : kActDepths)
+    if (r >= need) {
+      regs = r;
+      break;
+    }
+  const int threads = 32 * warps;
+  switch (regs) {
+    case 1: return launch_act_t<1>(x, M, K, Kx, idx, n_out, xq, sx, x_out, status, pdl, threads, smem, stream);
+    case 2: return launch_act_t<2>(x, M, K, Kx, idx, n_out, xq, sx, x_out, status, pdl, threads, smem, stream);
+    case 4: return launch_act_t<4>(x, M, K, Kx, idx, n_out, xq, sx, x_out, status, pdl, threads, smem, stream);
+    case 8: return launch_act_t<8>(x, M, K, Kx, idx, n_out, xq, sx, x_out, status, pdl, threads, smem, stream);
+    case 16: return launch_act_t<16>(x, M, K, Kx, idx, n_out, xq, sx, x_out, status, pdl, threads, smem, stream);
+    default: return launch_act_t<28>(x, M, K, Kx, idx, n_out, xq, sx, x_out, status, pdl, threads, smem, stream);
+  }
 }
 
 cudaError_t launch_calibrate(const float* X, int T, int K, int k, int32_t* idx_out,

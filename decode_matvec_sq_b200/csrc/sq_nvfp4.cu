@@ -22,18 +22,33 @@
 // code compares |x| with the seven E2M1 midpoints times s_b g, each product
 // exact in binary64.
 //
-// GEMM: CTA tile 128 tokens (MMA M, one TMEM lane each) x 128 weight rows
-// (MMA N), stages of 256 channels (128 bytes a row, 128-byte swizzle).
+// GEMM: a persistent kernel, one CTA per SM, looping over output tiles of
+// 128 tokens (MMA M, one TMEM lane each) x 128 weight rows (MMA N), token
+// tiles fastest so that concurrent CTAs share weight tiles in L2.  Stages of
+// 256 channels (128 bytes a row, 128-byte swizzle) run through a 5-stage
+// ring without draining between tiles.
 //   warp 0 (one lane): TMA of both code tiles, bulk copies of both scale
-//     chunks (2 KB each) into a 3-stage ring;
-//   warp 1 (one lane): per stage, tcgen05.cp of the 4 + 4 scale chunks into
-//     this stage's scale columns of tensor memory, then 4 block-scaled MMAs
-//     (K = 64 each) into the fp32 accumulator;
-//   warps 2-5: y = g_w g_x[t] * D read back with tcgen05.ld.
-// Two CTAs share an SM (256 TMEM columns each).  Every wait is bounded: a
+//     chunks (2 KB each) into the ring;
+//   warps 6-9 (one per tensor-memory lane quarter): per stage, the 4 + 4
+//     scale chunks from shared memory into that stage's scale columns
+//     (tcgen05.st, every quarter holding all of them: lane i of quarter q,
+//     column c = the scales of row 32 c + i), then arrive on the stage's
+//     scale barrier;
+//   warp 1 (one lane): per stage, 4 block-scaled MMAs (K = 64 each) into one
+//     of two fp32 accumulators (tiles alternate);
+//   warps 2-5: read an accumulator back (tcgen05.ld), free it for the tile
+//     after next, scale by g_w g_x[t], and write y through shared memory so
+//     that each store instruction covers whole 128-byte row segments.
+// The scales go in through the warps rather than tcgen05.cp: eight copies
+// per stage issued beside the MMAs took 131 us against 95 us per launch at
+// 2048 x 4096 -> 14336.
+// Tensor memory: accumulators at columns [0,128) and [128,256), the scales of
+// stage s at 256 + 32 s (A) and 272 + 32 s (B).  Every wait is bounded: a
 // wait that runs out sets SQ_ERR_TIMEOUT and the CTA drains its copies and
 // MMAs before it frees its tensor memory.
 #include <stdint.h>
+
+#include <algorithm>
 
 #include "sq_internal.h"
 #include "sq_tcgen05.cuh"
@@ -44,13 +59,14 @@ namespace {
 using tc05::fence_after;
 using tc05::fence_before;
 
-constexpr int BM = 128;          // tokens per CTA (MMA M)
-constexpr int BN = 128;          // weight rows per CTA (MMA N)
+constexpr int BM = 128;          // tokens per tile (MMA M)
+constexpr int BN = 128;          // weight rows per tile (MMA N)
 constexpr int kStageK = 256;     // channels per stage
 constexpr int kRowBytes = kStageK / 2;  // code bytes per row per stage
-constexpr int kStages = 3;
-constexpr int kThreads = 192;    // 6 warps
-constexpr uint32_t kTmemCols = 256;  // D [0,128); stage s scales: A at 128+32s, B at 144+32s
+constexpr int kStages = 5;
+constexpr int kThreads = 320;    // 10 warps
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kSfCol0 = 256;  // stage s scales: A at kSfCol0 + 32 s, B 16 columns on
 
 constexpr int kBytesA = BM * kRowBytes;  // 16 KB
 constexpr int kBytesB = BN * kRowBytes;  // 16 KB
@@ -58,16 +74,23 @@ constexpr int kBytesSf = 4 * 512;        // 4 chunks of 128 rows x 4 scales
 constexpr int kOffA = 0, kOffB = kBytesA, kOffSa = kOffB + kBytesB, kOffSb = kOffSa + kBytesSf;
 constexpr int kStageBytes = kOffSb + kBytesSf;  // 36 KB
 static_assert(kStageBytes % 1024 == 0, "stages must stay 1024-byte aligned");
+static_assert(kSfCol0 + 32 * kStages <= kTmemCols, "scale columns past the allocation");
+// y staging for the epilogue: per warp 32 rows x 32 floats, rows 36 floats
+// apart (16-byte stores of 8 consecutive lanes hit distinct banks).
+constexpr int kStageRow = 36;
+constexpr int kOffOut = kStages * kStageBytes;
+constexpr int kOutBytes = 4 * 32 * kStageRow * 4;  // 18 KB
 
 struct Aux {
-  uint64_t full[kStages], empty[kStages], tdone;
+  uint64_t full[kStages], empty[kStages], sfr[kStages], accf[2], acce[2], drain;
   uint32_t tmem_base;
   int abort;
 };
-constexpr int kSmemBytes = kStages * kStageBytes + (int)sizeof(Aux) + 1024;
+constexpr int kSmemBytes = kOffOut + kOutBytes + (int)sizeof(Aux) + 1024;
 
 struct Params {
-  int M, N, nk;  // nk = stages = K256 / 256
+  int M, N, nk;   // nk = stages per tile = K256 / 256
+  int nt_m, tiles;
   int sf_chunks;  // 64-channel scale chunks per 128-row block
   const uint8_t* sfa;  // activation scale chunks
   const uint8_t* sfb;  // weight scale chunks
@@ -93,11 +116,17 @@ __device__ __forceinline__ void mma_fp4(uint32_t d_tmem, uint64_t a, uint64_t b,
       "l"(a), "l"(b), "r"(kIdesc), "r"(acc ? 1 : 0), "r"(sfa), "r"(sfb));
 }
 
-// 32 rows x 16 bytes of shared memory into tensor-memory lanes 0-31 of 4
-// columns, replicated into all four lane quarters.
-__device__ __forceinline__ void sf_copy(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
-               : "memory");
+// 32 consecutive TMEM columns of this thread's lane.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&w)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+      "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7]),
+      "r"(w[8]), "r"(w[9]), "r"(w[10]), "r"(w[11]), "r"(w[12]), "r"(w[13]), "r"(w[14]), "r"(w[15]),
+      "r"(w[16]), "r"(w[17]), "r"(w[18]), "r"(w[19]), "r"(w[20]), "r"(w[21]), "r"(w[22]), "r"(w[23]),
+      "r"(w[24]), "r"(w[25]), "r"(w[26]), "r"(w[27]), "r"(w[28]), "r"(w[29]), "r"(w[30]), "r"(w[31])
+      : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Aux* aux,
@@ -111,23 +140,25 @@ __device__ __forceinline__ bool aborted(const Aux* aux) {
   return *reinterpret_cast<const volatile int*>(&aux->abort) != 0;
 }
 
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, 1)
     k_nvfp4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  Aux* aux = reinterpret_cast<Aux*>(smem + kStages * kStageBytes);
+  Aux* aux = reinterpret_cast<Aux*>(smem + kOffOut + kOutBytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nt_m = (p.M + BM - 1) / BM;
-  const int mt = blockIdx.x % nt_m, nt = blockIdx.x / nt_m;
-  const int m0 = mt * BM, n0 = nt * BN;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&aux->full[s], 1);
       mbar_init(&aux->empty[s], 1);
+      mbar_init(&aux->sfr[s], 128);
     }
-    mbar_init(&aux->tdone, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&aux->accf[b], 1);
+      mbar_init(&aux->acce[b], 128);
+    }
+    mbar_init(&aux->drain, 1);
     aux->abort = 0;
     fence_barrier_init();
   }
@@ -138,26 +169,31 @@ __global__ void __launch_bounds__(kThreads, 2)
   const uint32_t tmem = aux->tmem_base;
 
   if (warp == 0) {
-    // ---- producer
+    // ---- producer: every stage of every tile of this CTA, in order
     if (lane == 0) {
       int last_use[kStages];
 #pragma unroll
       for (int s = 0; s < kStages; ++s) last_use[s] = -1;
-      const uint8_t* sfa = p.sfa + (int64_t)mt * p.sf_chunks * 512;
-      const uint8_t* sfb = p.sfb + (int64_t)nt * p.sf_chunks * 512;
-      for (int kb = 0; kb < p.nk; ++kb) {
-        const int s = kb % kStages;
-        const uint32_t use = (uint32_t)(kb / kStages);
-        if (kb >= kStages && !wait_or_abort(&aux->empty[s], (use & 1u) ^ 1u, aux, p)) break;
-        if (aborted(aux)) break;
-        uint8_t* st = smem + s * kStageBytes;
-        mbar_arrive_expect_tx(&aux->full[s], kStageBytes);
-        tc05::tma_load_2d(st + kOffA, &tmA, kb * kRowBytes, m0, &aux->full[s]);
-        tc05::tma_load_2d(st + kOffB, &tmB, kb * kRowBytes, n0, &aux->full[s]);
-        tc05::bulk_load(st + kOffSa, sfa + (int64_t)kb * kBytesSf, kBytesSf, &aux->full[s]);
-        tc05::bulk_load(st + kOffSb, sfb + (int64_t)kb * kBytesSf, kBytesSf, &aux->full[s]);
-        last_use[s] = (int)use;
+      uint32_t g = 0;  // stages issued so far
+      for (int tile = blockIdx.x; tile < p.tiles && !aborted(aux); tile += gridDim.x) {
+        const int mt = tile % p.nt_m, nt = tile / p.nt_m;
+        const uint8_t* sfa = p.sfa + (int64_t)mt * p.sf_chunks * 512;
+        const uint8_t* sfb = p.sfb + (int64_t)nt * p.sf_chunks * 512;
+        for (int kb = 0; kb < p.nk; ++kb, ++g) {
+          const int s = (int)(g % kStages);
+          const uint32_t use = g / kStages;
+          if (g >= kStages && !wait_or_abort(&aux->empty[s], (use & 1u) ^ 1u, aux, p)) break;
+          if (aborted(aux)) break;
+          uint8_t* st = smem + s * kStageBytes;
+          mbar_arrive_expect_tx(&aux->full[s], kStageBytes);
+          tc05::tma_load_2d(st + kOffA, &tmA, kb * kRowBytes, mt * BM, &aux->full[s]);
+          tc05::tma_load_2d(st + kOffB, &tmB, kb * kRowBytes, nt * BN, &aux->full[s]);
+          tc05::bulk_load(st + kOffSa, sfa + (int64_t)kb * kBytesSf, kBytesSf, &aux->full[s]);
+          tc05::bulk_load(st + kOffSb, sfb + (int64_t)kb * kBytesSf, kBytesSf, &aux->full[s]);
+          last_use[s] = (int)use;
+        }
       }
+      // winding down after a timeout: every requested stage must have landed
       if (aborted(aux)) {
 #pragma unroll
         for (int s = 0; s < kStages; ++s)
@@ -167,54 +203,121 @@ __global__ void __launch_bounds__(kThreads, 2)
   } else if (warp == 1) {
     // ---- scale copies and MMAs
     if (lane == 0) {
-      for (int kb = 0; kb < p.nk; ++kb) {
-        const int s = kb % kStages;
-        const uint32_t use = (uint32_t)(kb / kStages);
-        if (!wait_or_abort(&aux->full[s], use & 1u, aux, p)) break;
+      uint32_t g = 0, n = 0;  // stages consumed, tiles started
+      for (int tile = blockIdx.x; tile < p.tiles; tile += gridDim.x, ++n) {
+        const uint32_t b = n & 1u;
+        if (n >= 2 && !wait_or_abort(&aux->acce[b], ((n >> 1) & 1u) ^ 1u, aux, p)) break;
         fence_after();
-        const uint32_t st = smem_u32(smem + s * kStageBytes);
-        const uint32_t ta = tmem + 128 + 32 * s, tb = ta + 16;
+        const uint32_t d = tmem + 128 * b;
+        bool ok = true;
+        for (int kb = 0; kb < p.nk; ++kb, ++g) {
+          const int s = (int)(g % kStages);
+          if (!wait_or_abort(&aux->full[s], (g / kStages) & 1u, aux, p) ||
+              !wait_or_abort(&aux->sfr[s], (g / kStages) & 1u, aux, p)) {
+            ok = false;
+            break;
+          }
+          fence_after();
+          const uint32_t st = smem_u32(smem + s * kStageBytes);
+          const uint32_t ta = tmem + kSfCol0 + 32 * s, tb = ta + 16;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_fp4(d, tc05::sw128_desc(st + kOffA + 32 * kk), tc05::sw128_desc(st + kOffB + 32 * kk),
+                    ta + 4 * kk, tb + 4 * kk, kb > 0 || kk > 0);
+          tc05::mma_commit(&aux->empty[s]);
+        }
+        if (!ok) break;
+        tc05::mma_commit(&aux->accf[b]);
+      }
+      // winding down after a timeout: the MMAs issued must be done before the
+      // tensor memory is freed
+      if (aborted(aux)) {
+        tc05::mma_commit(&aux->drain);  // tracks every MMA and copy issued before it
+        (void)mbar_wait(&aux->drain, 0u, p.wait_ns);
+      }
+    }
+  } else if (warp >= 6) {
+    // ---- scale factors into tensor memory: this warp's lane quarter
+    const int q = warp & 3;
+    uint32_t g = 0;
+    for (int tile = blockIdx.x; tile < p.tiles && !aborted(aux); tile += gridDim.x) {
+      bool ok = true;
+      for (int kb = 0; kb < p.nk; ++kb, ++g) {
+        const int s = (int)(g % kStages);
+        ok = wait_or_abort(&aux->full[s], (g / kStages) & 1u, aux, p);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        const uint8_t* st = smem + s * kStageBytes;
+        uint32_t w[32];
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          sf_copy(ta + 4 * kk, tc05::rows16_desc(st + kOffSa + 512 * kk));
-          sf_copy(tb + 4 * kk, tc05::rows16_desc(st + kOffSb + 512 * kk));
+          const uint4 a = *reinterpret_cast<const uint4*>(st + kOffSa + 512 * kk + 16 * lane);
+          const uint4 b = *reinterpret_cast<const uint4*>(st + kOffSb + 512 * kk + 16 * lane);
+          w[4 * kk] = a.x;
+          w[4 * kk + 1] = a.y;
+          w[4 * kk + 2] = a.z;
+          w[4 * kk + 3] = a.w;
+          w[16 + 4 * kk] = b.x;
+          w[16 + 4 * kk + 1] = b.y;
+          w[16 + 4 * kk + 2] = b.z;
+          w[16 + 4 * kk + 3] = b.w;
         }
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_fp4(tmem, tc05::sw128_desc(st + kOffA + 32 * kk), tc05::sw128_desc(st + kOffB + 32 * kk),
-                  ta + 4 * kk, tb + 4 * kk, kb > 0 || kk > 0);
-        tc05::mma_commit(&aux->empty[s]);
+        tmem_st32(tmem + ((uint32_t)(32 * q) << 16) + kSfCol0 + 32 * s, w);
+        fence_before();
+        mbar_arrive(&aux->sfr[s]);
       }
-      tc05::mma_commit(&aux->tdone);
-      if (aborted(aux)) (void)mbar_wait(&aux->tdone, 0u, p.wait_ns);
+      if (!ok) break;
     }
   } else {
     // ---- epilogue: one token (TMEM lane) per thread
-    const int lb = 32 * (warp & 3);
-    const int t = m0 + lb + lane;
-    bool ok = wait_or_abort(&aux->tdone, 0u, aux, p);
-    ok = __all_sync(0xffffffffu, ok) && !aborted(aux);
-    if (ok) {
+    const int q = warp & 3;  // TMEM lane quarter of this warp
+    float* stage_out = reinterpret_cast<float*>(smem + kOffOut) + q * 32 * kStageRow;
+    const float gw = __ldg(p.gw);
+    uint32_t n = 0;
+    for (int tile = blockIdx.x; tile < p.tiles; tile += gridDim.x, ++n) {
+      const uint32_t b = n & 1u;
+      const int m0 = (tile % p.nt_m) * BM + 32 * q, n0 = (tile / p.nt_m) * BN;
+      bool ok = !aborted(aux) && wait_or_abort(&aux->accf[b], (n >> 1) & 1u, aux, p);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
       fence_after();
-      const float sc = (t < p.M ? __ldg(p.gx + t) : 0.0f) * __ldg(p.gw);
-      float* yr = p.y + (int64_t)t * p.N + n0;
-      const bool full_row = n0 + BN <= p.N && (p.N & 3) == 0;
-#pragma unroll
+      const int t = m0 + lane;
+      const float sc = (t < p.M ? __ldg(p.gx + t) : 0.0f) * gw;
+#pragma unroll 1
       for (int h = 0; h < BN / 32; ++h) {
         int r[32];
-        tc05::tmem_ld32(tmem + ((uint32_t)lb << 16) + 32 * h, r);
-        if (t < p.M) {
-          if (full_row) {
+        tc05::tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + 128 * b + 32 * h, r);
+        if (h == BN / 32 - 1) {
+          fence_before();
+          mbar_arrive(&aux->acce[b]);
+        }
+        // this lane's row of the 32 x 32 block into shared memory
 #pragma unroll
-            for (int i = 0; i < 32; i += 4)
-              *reinterpret_cast<float4*>(yr + 32 * h + i) =
-                  make_float4(sc * __int_as_float(r[i]), sc * __int_as_float(r[i + 1]),
-                              sc * __int_as_float(r[i + 2]), sc * __int_as_float(r[i + 3]));
-          } else {
-            for (int i = 0; i < 32; ++i)
-              if (n0 + 32 * h + i < p.N) yr[32 * h + i] = sc * __int_as_float(r[i]);
+        for (int i = 0; i < 32; i += 4)
+          *reinterpret_cast<float4*>(stage_out + lane * kStageRow + i) =
+              make_float4(sc * __int_as_float(r[i]), sc * __int_as_float(r[i + 1]),
+                          sc * __int_as_float(r[i + 2]), sc * __int_as_float(r[i + 3]));
+        __syncwarp();
+        // four rows per store: lanes 8j .. 8j+7 write row 4i + j, 128 bytes
+        const int cn = n0 + 32 * h + 4 * (lane & 7);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int rr = 4 * i + (lane >> 3);
+          const int tt = m0 + rr;
+          const float4 v = *reinterpret_cast<const float4*>(stage_out + rr * kStageRow + 4 * (lane & 7));
+          if (tt < p.M) {
+            float* yp = p.y + (int64_t)tt * p.N + cn;
+            if (cn + 4 <= p.N && (p.N & 3) == 0) {
+              *reinterpret_cast<float4*>(yp) = v;
+            } else {
+              if (cn < p.N) yp[0] = v.x;
+              if (cn + 1 < p.N) yp[1] = v.y;
+              if (cn + 2 < p.N) yp[2] = v.z;
+              if (cn + 3 < p.N) yp[3] = v.w;
+            }
           }
         }
+        __syncwarp();
       }
     }
   }
@@ -320,11 +423,69 @@ __global__ void k_nvfp4_amax(const float* __restrict__ X, int64_t n, uint32_t* a
   if (threadIdx.x == 0) atomicMax(amax_bits, __float_as_uint(a));
 }
 
+// E2M1 code of x given the block's step s_b g: a binary32 estimate
+// v = |x| * (1 / step) (relative error below 3 * 2^-24) decides unless v lies
+// within 2^-19 of a midpoint (4 v within that of 1, 3, 5, 7, 10, 14 or 20);
+// then the exact binary64 comparison decides.
+__device__ __forceinline__ uint32_t e2m1_code_fast(float x, float inv, const E2m1Thresholds& th) {
+  const float v = fabsf(x) * inv;
+  const float u = 4.0f * v;
+  const float r = rintf(fminf(u, 31.0f));
+  const uint32_t ri = (uint32_t)r;
+  constexpr uint32_t kMid4 = (1u << 1) | (1u << 3) | (1u << 5) | (1u << 7) | (1u << 10) | (1u << 14) |
+                             (1u << 20);
+  if (((kMid4 >> ri) & 1u) && fabsf(u - r) <= u * 0x1p-19f) return e2m1_code(x, th);
+  const uint32_t c = (uint32_t)(v > 0.25f) + (uint32_t)(v > 0.75f) + (uint32_t)(v > 1.25f) +
+                     (uint32_t)(v > 1.75f) + (uint32_t)(v > 2.5f) + (uint32_t)(v > 3.5f) +
+                     (uint32_t)(v > 5.0f);
+  return (c != 0u && x < 0.0f) ? (c | 8u) : c;
+}
+
+// The codes (two words, channel 2i in the low nibble of byte i) and the
+// scale code of one 16-channel block under second-level scale g.
+__device__ __forceinline__ uint32_t quantize_block(const float (&v)[16], float gr, uint2& out) {
+  float ab = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) ab = fmaxf(ab, fabsf(v[i]));
+  const double gd = (double)gr;
+  const uint32_t sc = gr == 0.0f ? 0u : ue4m3_rne((double)ab / (6.0 * gd));
+  const double step = ue4m3_val(sc) * gd;
+  uint32_t w0 = 0u, w1 = 0u;
+  if (step != 0.0) {
+    const E2m1Thresholds th = e2m1_thresholds(step);
+    const float inv = __frcp_rn(__double2float_rn(step));
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w0 |= e2m1_code_fast(v[i], inv, th) << (4 * i);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w1 |= e2m1_code_fast(v[8 + i], inv, th) << (4 * i);
+  }
+  out = make_uint2(w0, w1);
+  return sc;
+}
+
+__device__ __forceinline__ void load_block(const float* x, int j0, int K, bool live, float (&v)[16]) {
+  if (live && j0 + 16 <= K && (K & 3) == 0) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float4 f = __ldg(reinterpret_cast<const float4*>(x + j0) + i);
+      v[4 * i] = f.x;
+      v[4 * i + 1] = f.y;
+      v[4 * i + 2] = f.z;
+      v[4 * i + 3] = f.w;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = (live && j0 + i < K) ? __ldg(x + j0 + i) : 0.0f;
+  }
+}
+
 // One CTA per row (rows_pad of them): every 16-channel block of the row up to
 // K256.  PER_ROW: g from the row's own amax (written to g[r]); else g from
-// the tensor amax in amax_bits (written to g[0] by CTA 0).
-template <bool PER_ROW>
-__global__ void __launch_bounds__(256) k_nvfp4_quantize(const float* __restrict__ X, int rows, int K,
+// the tensor amax in amax_bits (written to g[0] by CTA 0).  BPT > 0: each
+// thread holds its BPT blocks in registers between the amax and the codes
+// (one read of the row); BPT = 0: any K, the row is read twice.
+template <bool PER_ROW, int BPT>
+__global__ void __launch_bounds__(512) k_nvfp4_quantize(const float* __restrict__ X, int rows, int K,
                                                         int code_stride, int sf_chunks,
                                                         uint8_t* __restrict__ codes,
                                                         uint8_t* __restrict__ scales, float* g,
@@ -334,16 +495,30 @@ __global__ void __launch_bounds__(256) k_nvfp4_quantize(const float* __restrict_
   const bool live = r < rows;
   const float* x = X + (int64_t)(live ? r : 0) * K;
   const int nb = code_stride / 8;  // 16-channel blocks up to K256
+  constexpr int kHeld = BPT > 0 ? BPT : 1;
+  float v[kHeld][16];
+  float a = 0.0f;
+  bool bad = false;
+  if constexpr (BPT > 0) {
+#pragma unroll
+    for (int i = 0; i < BPT; ++i) {
+      const int b = threadIdx.x + i * blockDim.x;
+      load_block(x, 16 * b, K, live && b < nb, v[i]);
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        if (!isfinite(v[i][e])) bad = true;
+        a = fmaxf(a, fabsf(v[i][e]));
+      }
+    }
+  } else if (PER_ROW && live) {
+    for (int j = threadIdx.x; j < K; j += blockDim.x) {
+      const float t = __ldg(x + j);
+      if (!isfinite(t)) bad = true;
+      a = fmaxf(a, fabsf(t));
+    }
+  }
   float gr;
   if (PER_ROW) {
-    float a = 0.0f;
-    bool bad = false;
-    if (live)
-      for (int j = threadIdx.x; j < K; j += blockDim.x) {
-        const float v = __ldg(x + j);
-        if (!isfinite(v)) bad = true;
-        a = fmaxf(a, fabsf(v));
-      }
     if (bad) set_status(status, SQ_ERR_NONFINITE);
     a = absmax_reduce(a, red);
     gr = live ? __double2float_rn((double)a / 2688.0) : 0.0f;
@@ -352,54 +527,51 @@ __global__ void __launch_bounds__(256) k_nvfp4_quantize(const float* __restrict_
     gr = __double2float_rn((double)__uint_as_float(*amax_bits) / 2688.0);
     if (r == 0 && threadIdx.x == 0) g[0] = gr;
   }
-  const double gd = (double)gr;
   uint8_t* crow = codes + (int64_t)r * code_stride;
-  for (int b = threadIdx.x; b < nb; b += blockDim.x) {
-    const int j0 = 16 * b;
-    float v[16];
-    if (live && j0 + 16 <= K && (K & 3) == 0) {
+  if constexpr (BPT > 0) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float4 f = __ldg(reinterpret_cast<const float4*>(x + j0) + i);
-        v[4 * i] = f.x;
-        v[4 * i + 1] = f.y;
-        v[4 * i + 2] = f.z;
-        v[4 * i + 3] = f.w;
+    for (int i = 0; i < BPT; ++i) {
+      const int b = threadIdx.x + i * blockDim.x;
+      if (b < nb) {
+        uint2 w;
+        const uint32_t sc = quantize_block(v[i], gr, w);
+        *reinterpret_cast<uint2*>(crow + 8 * b) = w;
+        scales[sf_offset(r, b, sf_chunks)] = (uint8_t)sc;
       }
-    } else {
-#pragma unroll
-      for (int i = 0; i < 16; ++i) v[i] = (live && j0 + i < K) ? __ldg(x + j0 + i) : 0.0f;
     }
-    float ab = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) ab = fmaxf(ab, fabsf(v[i]));
-    const uint32_t sc = gr == 0.0f ? 0u : ue4m3_rne((double)ab / (6.0 * gd));
-    const double step = ue4m3_val(sc) * gd;
-    uint32_t w0 = 0u, w1 = 0u;
-    if (step != 0.0) {
-      const E2m1Thresholds th = e2m1_thresholds(step);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) w0 |= e2m1_code(v[i], th) << (4 * i);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) w1 |= e2m1_code(v[8 + i], th) << (4 * i);
+  } else {
+    for (int b = threadIdx.x; b < nb; b += blockDim.x) {
+      load_block(x, 16 * b, K, live, v[0]);
+      uint2 w;
+      const uint32_t sc = quantize_block(v[0], gr, w);
+      *reinterpret_cast<uint2*>(crow + 8 * b) = w;
+      scales[sf_offset(r, b, sf_chunks)] = (uint8_t)sc;
     }
-    *reinterpret_cast<uint2*>(crow + 8 * b) = make_uint2(w0, w1);
-    scales[sf_offset(r, b, sf_chunks)] = (uint8_t)sc;
   }
+}
+
+template <bool PER_ROW>
+cudaError_t launch_quantize_rows(const float* X, const sq_nvfp4_matrix& out, const uint32_t* amax,
+                                 int32_t* status, cudaStream_t stream) {
+  const int nb = out.code_stride / 8;
+  const int threads = nb <= 128 ? 128 : (nb <= 256 ? 256 : 512);
+  const int bpt = (nb + threads - 1) / threads;
+  auto go = [&](auto kern) {
+    kern<<<out.rows_pad, threads, 0, stream>>>(X, out.rows, out.K, out.code_stride, out.sf_chunks,
+                                               out.codes, out.scales, out.g, amax, status);
+    return cudaGetLastError();
+  };
+  if (bpt == 1) return go(k_nvfp4_quantize<PER_ROW, 1>);
+  if (bpt == 2) return go(k_nvfp4_quantize<PER_ROW, 2>);
+  if (bpt <= 4) return go(k_nvfp4_quantize<PER_ROW, 4>);
+  return go(k_nvfp4_quantize<PER_ROW, 0>);
 }
 
 }  // namespace
 
 cudaError_t launch_nvfp4_quantize(const float* X, const sq_nvfp4_matrix& out, int32_t* status,
                                   cudaStream_t stream) {
-  const int nb = out.code_stride / 8;
-  const int threads = nb >= 256 ? 256 : (nb >= 128 ? 128 : 64);
-  if (out.per_row) {
-    k_nvfp4_quantize<true><<<out.rows_pad, threads, 0, stream>>>(
-        X, out.rows, out.K, out.code_stride, out.sf_chunks, out.codes, out.scales, out.g, nullptr,
-        status);
-    return cudaGetLastError();
-  }
+  if (out.per_row) return launch_quantize_rows<true>(X, out, nullptr, status, stream);
   uint32_t* amax = reinterpret_cast<uint32_t*>(out.g + 1);
   cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(uint32_t), stream);
   if (e != cudaSuccess) return e;
@@ -408,10 +580,7 @@ cudaError_t launch_nvfp4_quantize(const float* X, const sq_nvfp4_matrix& out, in
   const int grid = (int)(want < 4096 ? want : 4096);
   k_nvfp4_amax<<<grid, 256, 0, stream>>>(X, n, amax, status);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  k_nvfp4_quantize<false><<<out.rows_pad, threads, 0, stream>>>(
-      X, out.rows, out.K, out.code_stride, out.sf_chunks, out.codes, out.scales, out.g, amax,
-      status);
-  return cudaGetLastError();
+  return launch_quantize_rows<false>(X, out, amax, status, stream);
 }
 
 cudaError_t launch_nvfp4_gemm(const sq_nvfp4_matrix& w, const sq_nvfp4_matrix& x, float* y,
@@ -430,6 +599,10 @@ cudaError_t launch_nvfp4_gemm(const sq_nvfp4_matrix& w, const sq_nvfp4_matrix& x
   p.M = x.rows;
   p.N = w.rows;
   p.nk = w.code_stride / kRowBytes;
+  p.nt_m = x.rows_pad / BM;
+  const int64_t tiles = (int64_t)p.nt_m * (w.rows_pad / BN);
+  if (tiles < 1 || tiles >= INT32_MAX) return cudaErrorInvalidValue;
+  p.tiles = (int)tiles;
   p.sf_chunks = w.sf_chunks;
   p.sfa = x.scales;
   p.sfb = w.scales;
@@ -438,11 +611,14 @@ cudaError_t launch_nvfp4_gemm(const sq_nvfp4_matrix& w, const sq_nvfp4_matrix& x
   p.y = y;
   p.status = status;
   p.wait_ns = wait_ns;
-  const int64_t grid = (int64_t)(x.rows_pad / BM) * (w.rows_pad / BN);
-  if (grid < 1 || grid >= INT32_MAX) return cudaErrorInvalidValue;
-  cudaError_t e = ensure_smem_attr((const void*)k_nvfp4_gemm, kSmemBytes);
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
-  k_nvfp4_gemm<<<(int)grid, kThreads, kSmemBytes, stream>>>(ma, mb, p);
+  const int grid = (int)std::min<int64_t>(tiles, sms);
+  e = ensure_smem_attr((const void*)k_nvfp4_gemm, kSmemBytes);
+  if (e != cudaSuccess) return e;
+  k_nvfp4_gemm<<<grid, kThreads, kSmemBytes, stream>>>(ma, mb, p);
   return cudaGetLastError();
 }
 

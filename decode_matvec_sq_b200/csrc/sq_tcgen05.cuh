@@ -45,14 +45,6 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t addr) {
          ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
 
-// K-major operand without swizzle whose rows are 16 bytes apart: core
-// matrices of 8 rows x 16 bytes, 128 bytes apart along the rows (stride byte
-// offset); one core matrix wide (leading byte offset 16, unused).
-__device__ __forceinline__ uint64_t rows16_desc(uint32_t addr) {
-  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(128 >> 4) << 32) |
-         ((uint64_t)1 << 46);
-}
-
 // Arrives on `bar` once every tcgen05 operation this thread issued is done.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(

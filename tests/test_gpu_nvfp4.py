@@ -59,7 +59,7 @@ def _rows_with_ties(rng, R, K):
 
 
 @pytest.mark.parametrize("R,K", [(1, 16), (5, 40), (130, 300), (128, 256), (257, 4096),
-                                 (64, 11008), (3, 1000)])
+                                 (64, 11008), (3, 1000), (3, 20000), (2, 40000)])
 @pytest.mark.parametrize("per_row", [False, True])
 def test_quantize_parity(R, K, per_row):
     rng = np.random.default_rng(R * 7 + K + per_row)
