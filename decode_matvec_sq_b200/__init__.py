@@ -91,6 +91,7 @@ def lib():
         "sq_decompose_pack_sparse": ([vp, i32, i32, i32, i32, pw, vp, vp], ctypes.c_int),
         "sq_residual_errors_scratch_bytes": ([i32], sz),
         "sq_residual_errors": ([vp, pw, vp, vp, sz, vp, vp], ctypes.c_int),
+        "sq_decompose_pack_auto": ([vp, i32, i32, i32, pw, vp, sz, vp, vp, vp, vp], ctypes.c_int),
         "sq_calibrate_outliers": ([vp, i32, i32, i32, vp, vp, vp], ctypes.c_int),
         "sq_quantize_act": ([vp, i32, i32, vp, i32, vp, vp, vp, vp, u32, vp], ctypes.c_int),
         "sq_linear_workspace_bytes": ([pw, i32], sz),
@@ -288,17 +289,23 @@ def residual_errors(W, pw: PackedWeight, status=None, stream=None):
     return e[0], e[1]
 
 
-def decompose_pack_auto(W, trunk_percent: int = -1, layout: int = None, status=None):
-    """The split with the per-layer fallback (m.lqnn.cn s2.3, last paragraph;
-    the rule of include/sq.h sq_residual_errors): when plain INT8 groups
-    reconstruct W at least as well as the split, the layer is packed with an
-    empty trunk (trunk_percent = 100), i.e. as plain INT8.  Returns
-    (packed weight, fell_back)."""
-    pw = decompose_pack(W, trunk_percent=trunk_percent, layout=layout, status=status)
-    e_split, e_plain = residual_errors(W, pw, status=status)
-    if e_plain <= e_split:
-        return decompose_pack(W, trunk_percent=100, layout=layout, status=status), True
-    return pw, False
+def decompose_pack_auto(W, trunk_percent: int = -1, layout: int = None, status=None, stream=None):
+    """The split with the per-layer fallback (include/sq.h
+    sq_decompose_pack_auto): plain INT8 groups (an empty trunk) when they
+    reconstruct W at least as well as the split.  Returns (packed weight,
+    fell_back).  Synchronous."""
+    import torch
+    N, K = W.shape
+    out = alloc_packed(N, K, 128, True, layout, device=W.device)
+    nb = int(lib().sq_residual_errors_scratch_bytes(N)) + 256
+    scratch = torch.empty(nb, dtype=torch.uint8, device=W.device)
+    fell = ctypes.c_int32(0)
+    _ck(lib().sq_decompose_pack_auto(_ptr(W), N, K, trunk_percent, ctypes.byref(out.view),
+                                     _ptr(scratch), nb, ctypes.byref(fell), None, _ptr(status),
+                                     _stream(stream)), "sq_decompose_pack_auto")
+    if not out.view.mask_bits:
+        out.with_mask = False
+    return out, bool(fell.value)
 
 
 def calibrate_outliers(X, k: int, out=None, status=None, stream=None):

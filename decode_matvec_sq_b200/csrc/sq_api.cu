@@ -294,6 +294,38 @@ sq_status sq_residual_errors(const float* W, const sq_packed_weight* w, double* 
                                           static_cast<cudaStream_t>(stream)));
 }
 
+sq_status sq_decompose_pack_auto(const float* W, int32_t N, int32_t K, int32_t trunk_percent,
+                                 sq_packed_weight* out, void* scratch, size_t scratch_bytes,
+                                 int32_t* fell_back, double* err_host, int32_t* dev_status,
+                                 void* stream) {
+  if (!W || !out || !scratch) return SQ_ERR_INVALID_ARG;
+  if (!out->mask_bits) return SQ_ERR_INVALID_ARG;  // the fallback needs an (empty) mask
+  sq_status st = check_weight(out);
+  if (st != SQ_OK) return st;
+  if (out->layout == SQ_LAYOUT_TILES_SPARSE) return SQ_ERR_INVALID_ARG;
+  if (scratch_bytes < sq_residual_errors_scratch_bytes(N) + 256) return SQ_ERR_WORKSPACE;
+  if (!aligned16(scratch)) return SQ_ERR_ALIGN;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((st = sq_decompose_pack(W, N, K, trunk_percent, out, dev_status, stream)) != SQ_OK) return st;
+  double* err = static_cast<double*>(scratch);
+  void* rest = static_cast<uint8_t*>(scratch) + 256;
+  if ((st = sq_residual_errors(W, out, err, rest, scratch_bytes - 256, dev_status, stream)) != SQ_OK)
+    return st;
+  double e[2];
+  if (cudaMemcpyAsync(e, err, sizeof(e), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return SQ_ERR_CUDA;
+  if (err_host) {
+    err_host[0] = e[0];
+    err_host[1] = e[1];
+  }
+  const bool fall = e[1] <= e[0];
+  if (fell_back) *fell_back = fall ? 1 : 0;
+  if (fall) return sq_decompose_pack(W, N, K, 100, out, dev_status, stream);
+  if (trunk_percent < 0) out->mask_bits = nullptr;
+  return SQ_OK;
+}
+
 sq_status sq_calibrate_outliers(const float* X, int32_t T, int32_t K, int32_t k, int32_t* idx_out,
                                 int32_t* dev_status, void* stream) {
   if (!X || !idx_out) return SQ_ERR_INVALID_ARG;

@@ -237,6 +237,26 @@ sq_status sq_residual_errors(const float *W, const sq_packed_weight *w, double *
                              void *stream);
 
 /*
+ * The split with the per-layer fallback applied (the rule above): decomposes
+ * W into *out with trunk_percent (as sq_decompose_pack), measures both
+ * errors and, when err[1] <= err[0], decomposes W again with
+ * trunk_percent = 100 (an empty trunk: plain INT8 groups of W).
+ *   out       packed weight with a mask array (layout SQ_LAYOUT_ROWS,
+ *             SQ_LAYOUT_TILES or SQ_LAYOUT_TILES_ASYM); on return
+ *             out->mask_bits is set to NULL when the split was kept with a
+ *             full trunk (trunk_percent < 0), whose all-ones mask the decode
+ *             kernels need not read (the array stays in the caller's buffer)
+ *   scratch   device, sq_residual_errors_scratch_bytes(N) + 256 bytes
+ *   fell_back host, may be NULL: 1 if the layer fell back, else 0
+ *   err_host  host, may be NULL: the two errors of the split, as err above
+ * Synchronous: it waits for `stream` to read the two errors back.
+ */
+sq_status sq_decompose_pack_auto(const float *W, int32_t N, int32_t K, int32_t trunk_percent,
+                                 sq_packed_weight *out, void *scratch, size_t scratch_bytes,
+                                 int32_t *fell_back, double *err_host, int32_t *dev_status,
+                                 void *stream);
+
+/*
  * Outlier calibration (m.lqnn.cn section 2.2: detect the outlier channels once,
  * cache their indices, look them up at run time).
  *   X        [T][K] f32 calibration activations, device

@@ -204,6 +204,26 @@ def test_linear_tokens_per_pass(L):
     assert L.sq_linear_tokens_per_pass(None, 0) == 0
 
 
+def test_decompose_pack_auto_host_checks(L):
+    """sq_decompose_pack_auto refuses, before any device work: a weight view
+    without a mask array (the fallback's empty trunk needs one), the sparse
+    layout, and a scratch below sq_residual_errors_scratch_bytes(N) + 256."""
+    p = ctypes.c_void_p(1 << 40)
+    def view(mask, layout=1):
+        v = sq.SqPackedWeight()
+        assert L.sq_packed_view(ctypes.c_void_p(1 << 41), 64, 512, 128, int(mask), layout, ctypes.byref(v)) == 0
+        return v
+    need = L.sq_residual_errors_scratch_bytes(64) + 256
+    fell = ctypes.c_int32(7)
+    assert L.sq_decompose_pack_auto(p, 64, 512, -1, ctypes.byref(view(False)), p, need, ctypes.byref(fell),
+                                    None, None, None) == 1
+    assert L.sq_decompose_pack_auto(p, 64, 512, -1, ctypes.byref(view(True, 2)), p, need, None, None, None,
+                                    None) == 1
+    assert L.sq_decompose_pack_auto(p, 64, 512, -1, ctypes.byref(view(True)), p, need - 1, None, None, None,
+                                    None) == 8
+    assert fell.value == 7  # untouched on a refusal
+
+
 def test_nvfp4_view_arithmetic(L):
     """sq_nvfp4_bytes / sq_nvfp4_view: codes [roundup(rows,128)][roundup(K,256)/2],
     scale chunks [rows_pad/128][roundup(K,256)/64][512], g [rows_pad] floats per
