@@ -83,6 +83,7 @@ def lib():
         "sq_nvfp4_view": ([vp, i32, i32, i32, nm], ctypes.c_int),
         "sq_nvfp4_quantize": ([vp, nm, vp, vp], ctypes.c_int),
         "sq_nvfp4_linear": ([nm, nm, vp, vp, vp], ctypes.c_int),
+        "sq_testing_nvfp4_stalled": ([nm, nm, vp, i32, ctypes.c_uint64, vp, vp], ctypes.c_int),
         "sq_status_string": ([ctypes.c_int], ctypes.c_char_p),
         "sq_device_check": ([], ctypes.c_int),
         "sq_packed_bytes": ([i32, i32, i32, i32, i32], sz),
@@ -531,3 +532,11 @@ def nvfp4_linear(w: Nvfp4Matrix, x: Nvfp4Matrix, y=None, status=None, stream=Non
     _ck(lib().sq_nvfp4_linear(ctypes.byref(w.view), ctypes.byref(x.view), _ptr(y), _ptr(status),
                               _stream(stream)), "sq_nvfp4_linear")
     return y
+
+
+def testing_nvfp4_stalled(w: Nvfp4Matrix, x: Nvfp4Matrix, y, skip_stage: int, wait_ns: int,
+                          status=None, stream=None):
+    """include/sq_testing.h: sq_nvfp4_linear with one channel stage never
+    requested and every wait limited to wait_ns (tests of the timeout path)."""
+    _ck(lib().sq_testing_nvfp4_stalled(ctypes.byref(w.view), ctypes.byref(x.view), _ptr(y), skip_stage,
+                                       wait_ns, _ptr(status), _stream(stream)), "sq_testing_nvfp4_stalled")

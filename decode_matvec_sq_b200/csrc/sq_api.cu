@@ -644,3 +644,21 @@ extern "C" sq_status sq_testing_prefill_stalled(const sq_packed_weight* w, const
   return from_cuda(launch_prefill(*w, M, xq, sx, x_out, idx, n_out, y, nullptr, nullptr, dev_status,
                                   static_cast<cudaStream_t>(stream), wait_ns, skip_group));
 }
+
+extern "C" sq_status sq_testing_nvfp4_stalled(const sq_nvfp4_matrix* w, const sq_nvfp4_matrix* x,
+                                              float* y, int32_t skip_stage, uint64_t wait_ns,
+                                              int32_t* dev_status, void* stream) {
+  sq_status st = check_nvfp4(w);
+  if (st != SQ_OK) return st;
+  if ((st = check_nvfp4(x)) != SQ_OK) return st;
+  if (!y) return SQ_ERR_INVALID_ARG;
+  if (w->per_row != 0 || x->per_row != 1) return SQ_ERR_INVALID_ARG;
+  if (w->K != x->K) return SQ_ERR_SHAPE;
+  if (skip_stage < -1 || skip_stage >= w->code_stride / 128) return SQ_ERR_INVALID_ARG;
+  if (wait_ns < 1 || wait_ns > 1000000000ull) return SQ_ERR_INVALID_ARG;
+  if (!aligned16(y)) return SQ_ERR_ALIGN;
+  DeviceInfo d;
+  if ((st = check_device(&d)) != SQ_OK) return st;
+  return from_cuda(launch_nvfp4_gemm(*w, *x, y, dev_status, static_cast<cudaStream_t>(stream),
+                                     wait_ns, skip_stage));
+}

@@ -105,7 +105,7 @@ cudaError_t launch_nvfp4_quantize(const float* X, const sq_nvfp4_matrix& out, in
                                   cudaStream_t stream);
 cudaError_t launch_nvfp4_gemm(const sq_nvfp4_matrix& w, const sq_nvfp4_matrix& x, float* y,
                               int32_t* status, cudaStream_t stream,
-                              uint64_t wait_ns = 1000000000ull);
+                              uint64_t wait_ns = 1000000000ull, int skip_stage = -1);
 
 cudaError_t launch_prefill(const sq_packed_weight& w, int M, const int8_t* xq, const float* sx,
                            const float* x_out, const int32_t* idx, int n_out, float* y,

@@ -99,6 +99,7 @@ struct Params {
   float* y;
   int32_t* status;
   uint64_t wait_ns;
+  int skip_stage;  // failure injection for tests: this stage is never requested (-1: none)
 };
 
 // D (f32) += A (E2M1, K-major) * B (E2M1, K-major) with UE4M3 block scales
@@ -184,6 +185,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t use = g / kStages;
           if (g >= kStages && !wait_or_abort(&aux->empty[s], (use & 1u) ^ 1u, aux, p)) break;
           if (aborted(aux)) break;
+          if (kb == p.skip_stage) continue;  // (tests only) never requested: its waits run out
           uint8_t* st = smem + s * kStageBytes;
           mbar_arrive_expect_tx(&aux->full[s], kStageBytes);
           tc05::tma_load_2d(st + kOffA, &tmA, kb * kRowBytes, mt * BM, &aux->full[s]);
@@ -352,8 +354,10 @@ __device__ __forceinline__ uint32_t ue4m3_rne(double q) {
 }
 
 __device__ __forceinline__ double ue4m3_val(uint32_t c) {
-  const int e = (int)(c >> 3), m = (int)(c & 7u);
-  return e == 0 ? (double)m * 0x1p-9 : ldexp(1.0 + (double)m * 0.125, e - 7);
+  const uint32_t e = c >> 3, m = c & 7u;
+  if (e == 0u) return (double)m * 0x1p-9;
+  // (1 + m/8) * 2^(e-7) from its binary64 fields
+  return __longlong_as_double((long long)(((uint64_t)(e - 7u + 1023u) << 52) | ((uint64_t)m << 49)));
 }
 
 // E2M1 code of x against the step s_b * g: the number of midpoints below
@@ -424,20 +428,21 @@ __global__ void k_nvfp4_amax(const float* __restrict__ X, int64_t n, uint32_t* a
 }
 
 // E2M1 code of x given the block's step s_b g: a binary32 estimate
-// v = |x| * (1 / step) (relative error below 3 * 2^-24) decides unless v lies
-// within 2^-19 of a midpoint (4 v within that of 1, 3, 5, 7, 10, 14 or 20);
-// then the exact binary64 comparison decides.
-__device__ __forceinline__ uint32_t e2m1_code_fast(float x, float inv, const E2m1Thresholds& th) {
-  const float v = fabsf(x) * inv;
-  const float u = 4.0f * v;
-  const float r = rintf(fminf(u, 31.0f));
-  const uint32_t ri = (uint32_t)r;
+// u = |x| * (4 / step) (relative error below 3 * 2^-24) decides unless u lies
+// within 2^-19 of one of the seven midpoints (4 x 0.25, 0.75, 1.25, 1.75, 2.5,
+// 3.5, 5 = 1, 3, 5, 7, 10, 14, 20); then the exact binary64 comparison
+// decides.  Away from them the code is the number of midpoints at or below
+// floor(u), one popcount.
+__device__ __forceinline__ uint32_t e2m1_code_fast(float x, float inv4, double step) {
+  const float u = fabsf(x) * inv4;
+  const float uc = fminf(u, 31.0f);
+  const float r = rintf(uc);
   constexpr uint32_t kMid4 = (1u << 1) | (1u << 3) | (1u << 5) | (1u << 7) | (1u << 10) | (1u << 14) |
                              (1u << 20);
-  if (((kMid4 >> ri) & 1u) && fabsf(u - r) <= u * 0x1p-19f) return e2m1_code(x, th);
-  const uint32_t c = (uint32_t)(v > 0.25f) + (uint32_t)(v > 0.75f) + (uint32_t)(v > 1.25f) +
-                     (uint32_t)(v > 1.75f) + (uint32_t)(v > 2.5f) + (uint32_t)(v > 3.5f) +
-                     (uint32_t)(v > 5.0f);
+  if (((kMid4 >> (uint32_t)r) & 1u) && fabsf(u - r) <= u * 0x1p-19f)
+    return e2m1_code(x, e2m1_thresholds(step));
+  const uint32_t k = (uint32_t)uc;  // floor: uc >= 0
+  const uint32_t c = (uint32_t)__popc(kMid4 & ((2u << k) - 1u));
   return (c != 0u && x < 0.0f) ? (c | 8u) : c;
 }
 
@@ -452,12 +457,11 @@ __device__ __forceinline__ uint32_t quantize_block(const float (&v)[16], float g
   const double step = ue4m3_val(sc) * gd;
   uint32_t w0 = 0u, w1 = 0u;
   if (step != 0.0) {
-    const E2m1Thresholds th = e2m1_thresholds(step);
-    const float inv = __frcp_rn(__double2float_rn(step));
+    const float inv4 = 4.0f * __frcp_rn(__double2float_rn(step));
 #pragma unroll
-    for (int i = 0; i < 8; ++i) w0 |= e2m1_code_fast(v[i], inv, th) << (4 * i);
+    for (int i = 0; i < 8; ++i) w0 |= e2m1_code_fast(v[i], inv4, step) << (4 * i);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) w1 |= e2m1_code_fast(v[8 + i], inv, th) << (4 * i);
+    for (int i = 0; i < 8; ++i) w1 |= e2m1_code_fast(v[8 + i], inv4, step) << (4 * i);
   }
   out = make_uint2(w0, w1);
   return sc;
@@ -584,7 +588,8 @@ cudaError_t launch_nvfp4_quantize(const float* X, const sq_nvfp4_matrix& out, in
 }
 
 cudaError_t launch_nvfp4_gemm(const sq_nvfp4_matrix& w, const sq_nvfp4_matrix& x, float* y,
-                              int32_t* status, cudaStream_t stream, uint64_t wait_ns) {
+                              int32_t* status, cudaStream_t stream, uint64_t wait_ns,
+                              int skip_stage) {
   if (w.K != x.K || w.code_stride != x.code_stride || w.per_row || !x.per_row)
     return cudaErrorInvalidValue;
   CUtensorMap ma, mb;
@@ -611,6 +616,7 @@ cudaError_t launch_nvfp4_gemm(const sq_nvfp4_matrix& w, const sq_nvfp4_matrix& x
   p.y = y;
   p.status = status;
   p.wait_ns = wait_ns;
+  p.skip_stage = skip_stage;
   int dev = 0, sms = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

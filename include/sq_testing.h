@@ -2,14 +2,14 @@
  * sq_testing.h -- failure injection for the tests of libsq.  Not part of the
  * decode path; the pages have no counterpart to it.
  *
- * The prefill kernel of sq_linear (many tokens, SQ_LAYOUT_ROWS, group size
- * 128) bounds every wait on its pipeline barriers.  When a wait runs out, the
+ * The prefill kernels -- sq_linear on many tokens (SQ_LAYOUT_ROWS, group size
+ * 128) and sq_nvfp4_linear -- bound every wait on their pipeline barriers.  When a wait runs out, the
  * kernel records SQ_ERR_TIMEOUT in the caller's status word and winds down:
  * it first waits (again bounded) for the operand copies it has requested and
  * for the tensor-core MMAs it has issued, then frees its tensor memory and
  * returns, so the context stays usable.  This entry point makes that happen
- * on purpose, without any fault: the operands of one channel group are
- * simply never requested, and every wait is limited to wait_ns.
+ * on purpose, without any fault: the operands of one channel group (stage)
+ * are simply never requested, and every wait is limited to wait_ns.
  */
 #ifndef SQ_TESTING_H
 #define SQ_TESTING_H
@@ -33,6 +33,18 @@ sq_status sq_testing_prefill_stalled(const sq_packed_weight *w, const int8_t *xq
                                      const float *x_out, const int32_t *idx, int32_t n_out,
                                      int32_t M, float *y, int32_t skip_group, uint64_t wait_ns,
                                      int32_t *dev_status, void *stream);
+
+/*
+ * sq_nvfp4_linear with its waits limited to wait_ns (1 .. 10^9 nanoseconds)
+ * and the operands of channel stage skip_stage (256 channels each,
+ * 0 <= skip_stage < roundup(K,256)/256) never requested for any tile;
+ * skip_stage = -1 requests everything and gives the result of
+ * sq_nvfp4_linear.  Arguments are those of sq_nvfp4_linear.  With a stage
+ * skipped, dev_status ends up SQ_ERR_TIMEOUT and y is unspecified.
+ */
+sq_status sq_testing_nvfp4_stalled(const sq_nvfp4_matrix *w, const sq_nvfp4_matrix *x, float *y,
+                                   int32_t skip_stage, uint64_t wait_ns, int32_t *dev_status,
+                                   void *stream);
 
 #ifdef __cplusplus
 }
