@@ -23,17 +23,18 @@
 // exact in binary64.
 //
 // GEMM: a persistent kernel, one CTA per SM, looping over output tiles of
-// 128 tokens (MMA M, one TMEM lane each) x 128 weight rows (MMA N), token
+// 128 tokens (MMA M, one TMEM lane each) x 192 weight rows (MMA N), token
 // tiles fastest so that concurrent CTAs share weight tiles in L2.  Stages of
-// 256 channels (128 bytes a row, 128-byte swizzle) run through a 5-stage
+// 256 channels (128 bytes a row, 128-byte swizzle) run through a 4-stage
 // ring without draining between tiles.
-//   warp 0 (one lane): TMA of both code tiles, bulk copies of both scale
-//     chunks (2 KB each) into the ring;
-//   warps 6-9 (one per tensor-memory lane quarter): per stage, the 4 + 4
-//     scale chunks from shared memory into that stage's scale columns
+//   warp 0 (one lane): TMA of both code tiles, bulk copies of the scale
+//     chunks (2 KB for the tokens, 2 x 2 KB for the two 128-row scale blocks
+//     the weight tile lies in) into the ring;
+//   warps 6-9 (one per tensor-memory lane quarter): per stage, the scales
+//     from shared memory into one of two scale sets of tensor memory
 //     (tcgen05.st, every quarter holding all of them: lane i of quarter q,
-//     column c = the scales of row 32 c + i), then arrive on the stage's
-//     scale barrier;
+//     word c = the scales of row 32 c + i; set g % 2, written once the MMAs
+//     of stage g - 2 are done), then arrive on the stage's scale barrier;
 //   warp 1 (one lane): per stage, 4 block-scaled MMAs (K = 64 each) into one
 //     of two fp32 accumulators (tiles alternate);
 //   warps 2-5: read an accumulator back (tcgen05.ld), free it for the tile
@@ -41,9 +42,10 @@
 //     that each store instruction covers whole 128-byte row segments.
 // The scales go in through the warps rather than tcgen05.cp: eight copies
 // per stage issued beside the MMAs took 131 us against 95 us per launch at
-// 2048 x 4096 -> 14336.
-// Tensor memory: accumulators at columns [0,128) and [128,256), the scales of
-// stage s at 256 + 32 s (A) and 272 + 32 s (B).  Every wait is bounded: a
+// 2048 x 4096 -> 14336 (then with 128-row weight tiles; 192 rows took the
+// launch from 99.9 to 94.0 us on one box: fewer shared-memory bytes per MAC).
+// Tensor memory: accumulators at columns [0,192) and [192,384), the scale
+// sets at 384 and 432 (A 16 columns, then B 32).  Every wait is bounded: a
 // wait that runs out sets SQ_ERR_TIMEOUT and the CTA drains its copies and
 // MMAs before it frees its tensor memory.
 #include <stdint.h>
@@ -60,21 +62,27 @@ using tc05::fence_after;
 using tc05::fence_before;
 
 constexpr int BM = 128;          // tokens per tile (MMA M)
-constexpr int BN = 128;          // weight rows per tile (MMA N)
+constexpr int BN = 192;          // weight rows per tile (MMA N)
 constexpr int kStageK = 256;     // channels per stage
 constexpr int kRowBytes = kStageK / 2;  // code bytes per row per stage
-constexpr int kStages = 5;
+constexpr int kStages = 4;
 constexpr int kThreads = 320;    // 10 warps
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kSfCol0 = 256;  // stage s scales: A at kSfCol0 + 32 s, B 16 columns on
+// tensor memory: accumulator b at columns [192 b, 192 b + 192); the scales of
+// stage g in set g % 2 at kSfCol0 + 48 (g % 2): A 16 columns, then B 32
+// (eight 32-row words per 64-channel chunk, as for 256 rows; words 6-7 zero)
+constexpr uint32_t kSfCol0 = 2 * BN;
+constexpr uint32_t kSfSet = 48;
 
 constexpr int kBytesA = BM * kRowBytes;  // 16 KB
-constexpr int kBytesB = BN * kRowBytes;  // 16 KB
-constexpr int kBytesSf = 4 * 512;        // 4 chunks of 128 rows x 4 scales
+constexpr int kBytesB = BN * kRowBytes;  // 24 KB
+constexpr int kBytesSf = 4 * 512;        // one 128-row block: 4 chunks of 128 rows x 4 scales
+// the weight tile's 192 rows start at a multiple of 64 and lie in two
+// consecutive 128-row scale blocks
 constexpr int kOffA = 0, kOffB = kBytesA, kOffSa = kOffB + kBytesB, kOffSb = kOffSa + kBytesSf;
-constexpr int kStageBytes = kOffSb + kBytesSf;  // 36 KB
+constexpr int kStageBytes = kOffSb + 2 * kBytesSf;  // 46 KB
 static_assert(kStageBytes % 1024 == 0, "stages must stay 1024-byte aligned");
-static_assert(kSfCol0 + 32 * kStages <= kTmemCols, "scale columns past the allocation");
+static_assert(kSfCol0 + 2 * kSfSet <= kTmemCols, "scale columns past the allocation");
 // y staging for the epilogue: per warp 32 rows x 32 floats, rows 36 floats
 // apart (16-byte stores of 8 consecutive lanes hit distinct banks).
 constexpr int kStageRow = 36;
@@ -92,6 +100,7 @@ struct Params {
   int M, N, nk;   // nk = stages per tile = K256 / 256
   int nt_m, tiles;
   int sf_chunks;  // 64-channel scale chunks per 128-row block
+  int nblk_b;     // 128-row scale blocks of the weight
   const uint8_t* sfa;  // activation scale chunks
   const uint8_t* sfb;  // weight scale chunks
   const float* gx;     // [M]
@@ -103,7 +112,7 @@ struct Params {
 };
 
 // D (f32) += A (E2M1, K-major) * B (E2M1, K-major) with UE4M3 block scales
-// of 16; M = 128, N = 128, K = 64.
+// of 16; M = 128, N = 192, K = 64.
 constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                             ((uint32_t)(BM >> 4) << 24);
 
@@ -117,7 +126,17 @@ __device__ __forceinline__ void mma_fp4(uint32_t d_tmem, uint64_t a, uint64_t b,
       "l"(a), "l"(b), "r"(kIdesc), "r"(acc ? 1 : 0), "r"(sfa), "r"(sfb));
 }
 
-// 32 consecutive TMEM columns of this thread's lane.
+// 16 consecutive TMEM columns of this thread's lane.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&w)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+      "%15,%16};" ::"r"(taddr),
+      "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7]),
+      "r"(w[8]), "r"(w[9]), "r"(w[10]), "r"(w[11]), "r"(w[12]), "r"(w[13]), "r"(w[14]), "r"(w[15])
+      : "memory");
+}
+
+// 32 consecutive TMEM columns of this thread's lane (waits for both stores).
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&w)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
@@ -178,8 +197,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t g = 0;  // stages issued so far
       for (int tile = blockIdx.x; tile < p.tiles && !aborted(aux); tile += gridDim.x) {
         const int mt = tile % p.nt_m, nt = tile / p.nt_m;
+        const int cb0 = (nt * BN) >> 7;  // first 128-row scale block of the tile
+        const bool two = cb0 + 1 < p.nblk_b;
         const uint8_t* sfa = p.sfa + (int64_t)mt * p.sf_chunks * 512;
-        const uint8_t* sfb = p.sfb + (int64_t)nt * p.sf_chunks * 512;
+        const uint8_t* sfb = p.sfb + (int64_t)cb0 * p.sf_chunks * 512;
         for (int kb = 0; kb < p.nk; ++kb, ++g) {
           const int s = (int)(g % kStages);
           const uint32_t use = g / kStages;
@@ -187,11 +208,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (aborted(aux)) break;
           if (kb == p.skip_stage) continue;  // (tests only) never requested: its waits run out
           uint8_t* st = smem + s * kStageBytes;
-          mbar_arrive_expect_tx(&aux->full[s], kStageBytes);
+          mbar_arrive_expect_tx(&aux->full[s], kStageBytes - (two ? 0 : kBytesSf));
           tc05::tma_load_2d(st + kOffA, &tmA, kb * kRowBytes, mt * BM, &aux->full[s]);
           tc05::tma_load_2d(st + kOffB, &tmB, kb * kRowBytes, nt * BN, &aux->full[s]);
           tc05::bulk_load(st + kOffSa, sfa + (int64_t)kb * kBytesSf, kBytesSf, &aux->full[s]);
           tc05::bulk_load(st + kOffSb, sfb + (int64_t)kb * kBytesSf, kBytesSf, &aux->full[s]);
+          if (two)
+            tc05::bulk_load(st + kOffSb + kBytesSf, sfb + ((int64_t)p.sf_chunks + 4 * kb) * 512,
+                            kBytesSf, &aux->full[s]);
           last_use[s] = (int)use;
         }
       }
@@ -210,7 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t b = n & 1u;
         if (n >= 2 && !wait_or_abort(&aux->acce[b], ((n >> 1) & 1u) ^ 1u, aux, p)) break;
         fence_after();
-        const uint32_t d = tmem + 128 * b;
+        const uint32_t d = tmem + BN * b;
         bool ok = true;
         for (int kb = 0; kb < p.nk; ++kb, ++g) {
           const int s = (int)(g % kStages);
@@ -221,11 +245,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           fence_after();
           const uint32_t st = smem_u32(smem + s * kStageBytes);
-          const uint32_t ta = tmem + kSfCol0 + 32 * s, tb = ta + 16;
+          const uint32_t ta = tmem + kSfCol0 + kSfSet * (g & 1u), tb = ta + 16;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             mma_fp4(d, tc05::sw128_desc(st + kOffA + 32 * kk), tc05::sw128_desc(st + kOffB + 32 * kk),
-                    ta + 4 * kk, tb + 4 * kk, kb > 0 || kk > 0);
+                    ta + 4 * kk, tb + 8 * kk, kb > 0 || kk > 0);
           tc05::mma_commit(&aux->empty[s]);
         }
         if (!ok) break;
@@ -239,32 +263,44 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp >= 6) {
-    // ---- scale factors into tensor memory: this warp's lane quarter
+    // ---- scale factors into tensor memory: this warp's lane quarter, in
+    // set g % 2 once the MMAs of stage g - 2 (the set's last readers) are done
     const int q = warp & 3;
     uint32_t g = 0;
     for (int tile = blockIdx.x; tile < p.tiles && !aborted(aux); tile += gridDim.x) {
+      const int n0 = (tile / p.nt_m) * BN;
+      const int cb0 = n0 >> 7;
+      const bool two = cb0 + 1 < p.nblk_b;
       bool ok = true;
       for (int kb = 0; kb < p.nk; ++kb, ++g) {
         const int s = (int)(g % kStages);
-        ok = wait_or_abort(&aux->full[s], (g / kStages) & 1u, aux, p);
+        ok = wait_or_abort(&aux->full[s], (g / kStages) & 1u, aux, p) &&
+             (g < 2 || wait_or_abort(&aux->empty[(g - 2) % kStages], ((g - 2) / kStages) & 1u, aux, p));
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         const uint8_t* st = smem + s * kStageBytes;
-        uint32_t w[32];
+        uint32_t wa[16], wb[32];
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
           const uint4 a = *reinterpret_cast<const uint4*>(st + kOffSa + 512 * kk + 16 * lane);
-          const uint4 b = *reinterpret_cast<const uint4*>(st + kOffSb + 512 * kk + 16 * lane);
-          w[4 * kk] = a.x;
-          w[4 * kk + 1] = a.y;
-          w[4 * kk + 2] = a.z;
-          w[4 * kk + 3] = a.w;
-          w[16 + 4 * kk] = b.x;
-          w[16 + 4 * kk + 1] = b.y;
-          w[16 + 4 * kk + 2] = b.z;
-          w[16 + 4 * kk + 3] = b.w;
+          wa[4 * kk] = a.x;
+          wa[4 * kk + 1] = a.y;
+          wa[4 * kk + 2] = a.z;
+          wa[4 * kk + 3] = a.w;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            // tile row 32 j + lane: global row n0 + 32 j + lane, in scale
+            // block cb0 + ((n0 & 127) + 32 j) / 128, word ((n0 & 127) / 32 + j) % 4
+            const int wq = ((n0 & 127) >> 5) + j;
+            const bool live = j < BN / 32 && (wq < 4 || two);
+            wb[8 * kk + j] = live ? *reinterpret_cast<const uint32_t*>(
+                                        st + kOffSb + (wq >> 2) * kBytesSf + 512 * kk + 16 * lane + 4 * (wq & 3))
+                                  : 0u;
+          }
         }
-        tmem_st32(tmem + ((uint32_t)(32 * q) << 16) + kSfCol0 + 32 * s, w);
+        const uint32_t ts = tmem + ((uint32_t)(32 * q) << 16) + kSfCol0 + kSfSet * (g & 1u);
+        tmem_st16(ts, wa);
+        tmem_st32(ts + 16, wb);
         fence_before();
         mbar_arrive(&aux->sfr[s]);
       }
@@ -288,7 +324,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
       for (int h = 0; h < BN / 32; ++h) {
         int r[32];
-        tc05::tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + 128 * b + 32 * h, r);
+        tc05::tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + BN * b + 32 * h, r);
         if (h == BN / 32 - 1) {
           fence_before();
           mbar_arrive(&aux->acce[b]);
@@ -605,7 +641,8 @@ cudaError_t launch_nvfp4_gemm(const sq_nvfp4_matrix& w, const sq_nvfp4_matrix& x
   p.N = w.rows;
   p.nk = w.code_stride / kRowBytes;
   p.nt_m = x.rows_pad / BM;
-  const int64_t tiles = (int64_t)p.nt_m * (w.rows_pad / BN);
+  p.nblk_b = w.rows_pad / 128;
+  const int64_t tiles = (int64_t)p.nt_m * ceil_div(w.rows, BN);
   if (tiles < 1 || tiles >= INT32_MAX) return cudaErrorInvalidValue;
   p.tiles = (int)tiles;
   p.sf_chunks = w.sf_chunks;
