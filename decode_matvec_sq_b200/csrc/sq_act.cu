@@ -123,6 +123,99 @@ __global__ void __launch_bounds__(kActThreads) k_quantize_act(
   if (bad_idx) set_status(status, SQ_ERR_INVALID_ARG);
 }
 
+// K % 4 == 0: the same split four channels per lane -- float4 loads, one
+// nibble of the outlier bitmap and one 32-bit store of four codes per lane
+// and chunk of 128 channels (a warp's 32 lanes); REGS chunks per warp held
+// in registers, any further ones read again.  Same codes as k_quantize_act
+// (the same quantizer decides them).
+template <int REGS>
+__global__ void __launch_bounds__(kActThreads) k_quantize_act4(
+    const float* __restrict__ x, int M, int K, int Kx, const int32_t* __restrict__ idx, int n_out,
+    int8_t* __restrict__ xq, float* __restrict__ sx, float* __restrict__ x_out,
+    int32_t* __restrict__ status, int pdl) {
+  extern __shared__ uint32_t is_out[];  // ceil(K/32) words
+  __shared__ float warp_max[kActThreads / 32];
+  if (pdl) {
+    pdl_launch_dependents();
+    pdl_wait();
+  }
+  const int t = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nw = blockDim.x >> 5;
+  const int K4 = K >> 2, Kx4 = Kx >> 2;
+  const int nch = (K4 + 31) >> 5;  // chunks of 128 channels
+  const float* xt = x + (int64_t)t * K;
+  const float4* xt4 = reinterpret_cast<const float4*>(xt);
+  // the first outlier entries and their values, issued with the x loads
+  const int j0 = threadIdx.x < n_out ? __ldg(idx + threadIdx.x) : -1;
+  const int jq0 = (threadIdx.x < n_out && threadIdx.x > 0) ? __ldg(idx + threadIdx.x - 1) : -1;
+  float4 v[REGS];
+#pragma unroll
+  for (int i = 0; i < REGS; ++i) {
+    const int j4 = (warp + nw * i) * 32 + lane;
+    v[i] = j4 < K4 ? __ldg(xt4 + j4) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  }
+  const float xo0 = (j0 >= 0 && j0 < K) ? __ldg(xt + j0) : 0.0f;
+  const int nwords = (K + 31) >> 5;
+  for (int i = threadIdx.x; i < nwords; i += blockDim.x) is_out[i] = 0u;
+  __syncthreads();
+  bool bad_idx = false;
+  for (int i = threadIdx.x; i < n_out; i += blockDim.x) {
+    const bool first = i < (int)blockDim.x;
+    const int j = first ? j0 : idx[i];
+    const int jq = first ? jq0 : idx[i - 1];
+    const bool ok = j >= 0 && j < K && (i == 0 || jq < j);
+    bad_idx |= !ok;
+    if (j >= 0 && j < K) atomicOr(&is_out[j >> 5], 1u << (j & 31));
+    x_out[(int64_t)t * n_out + i] = first ? xo0 : ((j >= 0 && j < K) ? xt[j] : 0.0f);
+  }
+  __syncthreads();
+
+  float a = 0.0f;
+  bool nonfinite = false;
+  const bool big = nch > nw * REGS;
+#pragma unroll
+  for (int i = 0; i < REGS; ++i) {
+    const int j4 = (warp + nw * i) * 32 + lane;
+    if (j4 < K4) a = absmax4(v[i], omask_nibble(is_out, j4), a, nonfinite);
+  }
+  if (big) {
+    for (int c = warp + nw * REGS; c < nch; c += nw) {
+      const int j4 = c * 32 + lane;
+      if (j4 < K4) a = absmax4(xt4[j4], omask_nibble(is_out, j4), a, nonfinite);
+    }
+  }
+  for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+  if (lane == 0) warp_max[warp] = a;
+  __syncthreads();
+  a = lane < nw ? warp_max[lane] : 0.0f;
+  for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+
+  const float s = act_scale(a);
+  const float rinv = act_rinv(s);
+  if (threadIdx.x == 0) sx[t] = s;
+  uint32_t* qt4 = reinterpret_cast<uint32_t*>(xq + (int64_t)t * Kx);
+  const bool fast = quantize_fast_ok(s, a);  // one branch per token
+#pragma unroll
+  for (int i = 0; i < REGS; ++i) {
+    const int j4 = (warp + nw * i) * 32 + lane;
+    if (j4 < K4) {
+      const uint32_t om = omask_nibble(is_out, j4);
+      qt4[j4] = fast ? pack_codes<true>(v[i], om, s, rinv) : pack_codes<false>(v[i], om, s, rinv);
+    }
+  }
+  if (big) {
+    for (int c = warp + nw * REGS; c < nch; c += nw) {
+      const int j4 = c * 32 + lane;
+      if (j4 < K4) qt4[j4] = pack_codes<false>(xt4[j4], omask_nibble(is_out, j4), s, rinv);
+    }
+  }
+  // pad words up to the row stride (a multiple of 128 channels)
+  for (int j4 = K4 + threadIdx.x; j4 < Kx4; j4 += blockDim.x) qt4[j4] = 0u;
+  if (nonfinite) set_status(status, SQ_ERR_NONFINITE);
+  if (bad_idx) set_status(status, SQ_ERR_INVALID_ARG);
+}
+
 // ---- calibration: per-channel max |X| over T tokens, top-k ------------------
 struct Cand {
   float mag;
@@ -207,11 +300,12 @@ namespace {
 // depth is the smallest instantiated one covering the row, 28 at most.
 constexpr int kActDepths[] = {1, 2, 4, 8, 16, 28};
 
-template <int REGS>
+template <int REGS, bool VEC>
 cudaError_t launch_act_t(const float* x, int M, int K, int Kx, const int32_t* idx, int n_out,
                          int8_t* xq, float* sx, float* x_out, int32_t* status, bool pdl,
                          int threads, size_t smem, cudaStream_t stream) {
   auto* fn = k_quantize_act<REGS>;
+  if constexpr (VEC) fn = k_quantize_act4<REGS>;
   cudaError_t e = ensure_smem_attr((const void*)fn, (int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -233,11 +327,13 @@ cudaError_t launch_quantize_act(const float* x, int M, int K, const int32_t* idx
                                 cudaStream_t stream) {
   const int Kx = (int)xq_stride_of(K);
   const size_t smem = (size_t)ceil_div(K, 32) * sizeof(uint32_t);
-  const int nchunk = (int)ceil_div(K, 32);
+  // chunks per lane-column: 32 channels (scalar kernel) or 128 (K % 4 == 0)
+  const bool vec = (K & 3) == 0;
+  const int nchunk = (int)ceil_div(K, vec ? 128 : 32);
   DeviceInfo d;
   const int sms = current_device(&d) ? d.sm_count : 148;
   int warps = 32;
-  if (M >= 2 * sms) warps = std::min(32, std::max(1, (int)ceil_div(nchunk, 16)));
+  if (M >= 2 * sms) warps = std::min(32, std::max(1, (int)ceil_div(nchunk, vec ? 4 : 16)));
   const int need = (int)ceil_div(nchunk, warps);
   int regs = kActDepths[5];
   for (int r : kActDepths)
@@ -245,15 +341,27 @@ cudaError_t launch_quantize_act(const float* x, int M, int K, const int32_t* idx
       regs = r;
       break;
     }
+  if (vec) regs = std::min(regs, 8);  // float4 chunks: at most 8 (32 registers) held
   const int threads = 32 * warps;
-  switch (regs) {
-    case 1: return launch_act_t<1>(x, M, K, Kx, idx, n_out, xq, sx, x_out, status, pdl, threads, smem, stream);
-    case 2: return launch_act_t<2>(x, M, K, Kx, idx, n_out, xq, sx, x_out, status, pdl, threads, smem, stream);
-    case 4: return launch_act_t<4>(x, M, K, Kx, idx, n_out, xq, sx, x_out, status, pdl, threads, smem, stream);
-    case 8: return launch_act_t<8>(x, M, K, Kx, idx, n_out, xq, sx, x_out, status, pdl, threads, smem, stream);
-    case 16: return launch_act_t<16>(x, M, K, Kx, idx, n_out, xq, sx, x_out, status, pdl, threads, smem, stream);
-    default: return launch_act_t<28>(x, M, K, Kx, idx, n_out, xq, sx, x_out, status, pdl, threads, smem, stream);
+#define SQ_ACT_LAUNCH(R, V) \
+  return launch_act_t<R, V>(x, M, K, Kx, idx, n_out, xq, sx, x_out, status, pdl, threads, smem, stream)
+  if (vec) {
+    switch (regs) {
+      case 1: SQ_ACT_LAUNCH(1, true);
+      case 2: SQ_ACT_LAUNCH(2, true);
+      case 4: SQ_ACT_LAUNCH(4, true);
+      default: SQ_ACT_LAUNCH(8, true);
+    }
   }
+  switch (regs) {
+    case 1: SQ_ACT_LAUNCH(1, false);
+    case 2: SQ_ACT_LAUNCH(2, false);
+    case 4: SQ_ACT_LAUNCH(4, false);
+    case 8: SQ_ACT_LAUNCH(8, false);
+    case 16: SQ_ACT_LAUNCH(16, false);
+    default: SQ_ACT_LAUNCH(28, false);
+  }
+#undef SQ_ACT_LAUNCH
 }
 
 cudaError_t launch_calibrate(const float* X, int T, int K, int k, int32_t* idx_out,

@@ -402,33 +402,6 @@ __device__ __forceinline__ void write_y(const Params& p, int rb, int gid, int ti
 // compiler spill registers in the fused kernels)
 constexpr int kXRegs = 8;
 
-__device__ __forceinline__ uint32_t omask_nibble(const uint32_t* omask, int j4) {
-  return (omask[j4 >> 3] >> ((j4 & 7) * 4)) & 0xFu;  // outlier bits of channels 4*j4 .. 4*j4+3
-}
-
-template <bool FAST>
-__device__ __forceinline__ int qcode(float v, float s, float rinv) {
-  return FAST ? quantize_fast(v, s, rinv) : quantize_exact(v, s, rinv);
-}
-template <bool FAST>
-__device__ __forceinline__ uint32_t pack_codes(float4 v, uint32_t om, float s, float rinv) {
-  const int q0 = (om & 1u) ? 0 : qcode<FAST>(v.x, s, rinv);
-  const int q1 = (om & 2u) ? 0 : qcode<FAST>(v.y, s, rinv);
-  const int q2 = (om & 4u) ? 0 : qcode<FAST>(v.z, s, rinv);
-  const int q3 = (om & 8u) ? 0 : qcode<FAST>(v.w, s, rinv);
-  return (uint32_t)(q0 & 0xFF) | ((uint32_t)(q1 & 0xFF) << 8) | ((uint32_t)(q2 & 0xFF) << 16) |
-         ((uint32_t)(q3 & 0xFF) << 24);
-}
-
-__device__ __forceinline__ float absmax4(float4 v, uint32_t om, float a, bool& nonfinite) {
-  nonfinite |= !isfinite(v.x) || !isfinite(v.y) || !isfinite(v.z) || !isfinite(v.w);
-  if (!(om & 1u)) a = fmaxf(a, fabsf(v.x));
-  if (!(om & 2u)) a = fmaxf(a, fabsf(v.y));
-  if (!(om & 4u)) a = fmaxf(a, fabsf(v.z));
-  if (!(om & 8u)) a = fmaxf(a, fabsf(v.w));
-  return a;
-}
-
 // jv, jp: this thread's entry of the outlier list and the one before it
 // (threads < n_out, loaded in the prologue).
 __device__ __forceinline__ void split_activations(const Params& p, const uint32_t* omask,
