@@ -100,6 +100,13 @@ def load_fp4_peak():
         return FALLBACK_BF16_TFLOPS * FP4_PER_BF16, "fallback bf16 x nominal fp4/bf16 ratio"
 
 
+def probe_peak(kind: int) -> float:
+    """The dense tensor-core rate measured on this device by the library's
+    probe (sq_testing_mma_peak): kind 0 int8, 1 NVFP4; T ops/s."""
+    import decode_matvec_sq_b200 as sq
+    return sq.testing_mma_peak(kind) / 1e12
+
+
 def load_int8_peak():
     """Dense int8 tensor peak in T int-ops/s: the measured cuBLAS bf16 burst
     figure times the nominal int8/bf16 ratio."""
@@ -444,6 +451,7 @@ def run_prefill(args, world, rank, local):
     if st.item() != 0:
         raise RuntimeError(f"device status {sq.STATUS.get(st.item())}")
     peak, kind = load_int8_peak()
+    probe = probe_peak(0)
     value = world * ops / (ms_step * 1e-3) / 1e12
     achieved = ops / (ms_lin * 1e-3) / 1e12
     if rank == 0:
@@ -459,7 +467,11 @@ def run_prefill(args, world, rank, local):
             "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak, 1),
                          "unit": "T int-ops/s", "frac": round(achieved / peak, 4), "peak_kind": kind,
                          "traffic": None, "kernel": "k_prefill (tcgen05 kind::i8)",
-                         "us_per_launch": round(ms_lin * 1e3, 2)},
+                         "us_per_launch": round(ms_lin * 1e3, 2),
+                         "probe_peak": round(probe, 1),
+                         "frac_of_probe": round(achieved / probe, 4),
+                         "probe_kind": "measured on this device: back-to-back kind::i8 MMAs "
+                                       "128x256x32 on every SM (sq_testing_mma_peak)"},
             "clocks": clocks,
         }), flush=True)
     if world > 1:
@@ -735,6 +747,7 @@ def run_prefill_nvfp4(args, world, rank, local):
     if st.item() != 0:
         raise RuntimeError(f"device status {sq.STATUS.get(st.item())}")
     peak, kind = load_fp4_peak()
+    probe = probe_peak(1)
     achieved = flops / (ms_lin * 1e-3) / 1e12
     if rank == 0:
         print(json.dumps({
@@ -751,7 +764,11 @@ def run_prefill_nvfp4(args, world, rank, local):
             "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak, 1),
                          "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "peak_kind": kind,
                          "traffic": None, "kernel": "k_nvfp4_gemm (tcgen05 kind::mxf4nvf4)",
-                         "us_per_launch": round(ms_lin * 1e3, 2)},
+                         "us_per_launch": round(ms_lin * 1e3, 2),
+                         "probe_peak": round(probe, 1),
+                         "frac_of_probe": round(achieved / probe, 4),
+                         "probe_kind": "measured on this device: back-to-back kind::mxf4nvf4 MMAs "
+                                       "128x256x64 on every SM (sq_testing_mma_peak)"},
             "clocks": clocks,
         }), flush=True)
     if world > 1:
@@ -787,14 +804,16 @@ def side_configs(device, warmup=3, reps=10):
                                        "us_linear": round(ms_lin * 1e3, 1),
                                        "t_intops_linear": round(ops / (ms_lin * 1e-3) / 1e12, 1),
                                        "frac_of_int8_peak": round(ops / (ms_lin * 1e-3) / 1e12 / peak, 4),
-                                       "int8_peak_kind": kind}
+                                       "int8_peak_kind": kind,
+                                       "frac_of_probe_int8_peak": round(ops / (ms_lin * 1e-3) / 1e12 / probe_peak(0), 4)}
     ms_step, ms_lin, flops = time_nvfp4_prefill_case(st, device, warmup, reps)
     peak, kind = load_fp4_peak()
     out["prefill_nvfp4_2048x4096x14336"] = {"us_step": round(ms_step * 1e3, 1),
                                              "us_gemm": round(ms_lin * 1e3, 1),
                                              "tflops_gemm": round(flops / (ms_lin * 1e-3) / 1e12, 1),
                                              "frac_of_fp4_peak": round(flops / (ms_lin * 1e-3) / 1e12 / peak, 4),
-                                             "fp4_peak_kind": kind}
+                                             "fp4_peak_kind": kind,
+                                             "frac_of_probe_fp4_peak": round(flops / (ms_lin * 1e-3) / 1e12 / probe_peak(1), 4)}
     if st.item() != 0:
         raise RuntimeError(f"side configurations: device status {st.item()}")
     return out

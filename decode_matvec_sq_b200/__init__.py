@@ -84,6 +84,7 @@ def lib():
         "sq_nvfp4_quantize": ([vp, nm, vp, vp], ctypes.c_int),
         "sq_nvfp4_linear": ([nm, nm, vp, vp, vp], ctypes.c_int),
         "sq_testing_nvfp4_stalled": ([nm, nm, vp, i32, ctypes.c_uint64, vp, vp], ctypes.c_int),
+        "sq_testing_mma_peak": ([i32, i32, ctypes.POINTER(ctypes.c_double), vp, vp], ctypes.c_int),
         "sq_status_string": ([ctypes.c_int], ctypes.c_char_p),
         "sq_device_check": ([], ctypes.c_int),
         "sq_packed_bytes": ([i32, i32, i32, i32, i32], sz),
@@ -540,3 +541,12 @@ def testing_nvfp4_stalled(w: Nvfp4Matrix, x: Nvfp4Matrix, y, skip_stage: int, wa
     requested and every wait limited to wait_ns (tests of the timeout path)."""
     _ck(lib().sq_testing_nvfp4_stalled(ctypes.byref(w.view), ctypes.byref(x.view), _ptr(y), skip_stage,
                                        wait_ns, _ptr(status), _stream(stream)), "sq_testing_nvfp4_stalled")
+
+
+def testing_mma_peak(kind: int, iters: int = 4000, status=None, stream=None) -> float:
+    """include/sq_testing.h: the measured dense tensor-core rate in ops/s
+    (kind 0: int8 MMA, 1: NVFP4 block-scaled MMA)."""
+    out = ctypes.c_double(0.0)
+    _ck(lib().sq_testing_mma_peak(kind, iters, ctypes.byref(out), _ptr(status), _stream(stream)),
+        "sq_testing_mma_peak")
+    return out.value

@@ -37,6 +37,7 @@ SOURCES = [
     ("sq_noalloc.cu", []),
     ("sq_prefill.cu", []),
     ("sq_nvfp4.cu", ["-fmad=false"]),
+    ("sq_probe.cu", []),
 ]
 
 

@@ -662,3 +662,13 @@ extern "C" sq_status sq_testing_nvfp4_stalled(const sq_nvfp4_matrix* w, const sq
   return from_cuda(launch_nvfp4_gemm(*w, *x, y, dev_status, static_cast<cudaStream_t>(stream),
                                      wait_ns, skip_stage));
 }
+
+extern "C" sq_status sq_testing_mma_peak(int32_t kind, int32_t iters, double* ops_per_s,
+                                         int32_t* dev_status, void* stream) {
+  if (!ops_per_s || (kind != 0 && kind != 1)) return SQ_ERR_INVALID_ARG;
+  if (iters < 1 || iters > 100000) return SQ_ERR_SHAPE;
+  DeviceInfo d;
+  sq_status st = check_device(&d);
+  if (st != SQ_OK) return st;
+  return from_cuda(run_mma_peak(kind, iters, ops_per_s, dev_status, static_cast<cudaStream_t>(stream)));
+}

@@ -107,6 +107,10 @@ cudaError_t launch_nvfp4_gemm(const sq_nvfp4_matrix& w, const sq_nvfp4_matrix& x
                               int32_t* status, cudaStream_t stream,
                               uint64_t wait_ns = 1000000000ull, int skip_stage = -1);
 
+// Tensor-core peak probe (sq_probe.cu; include/sq_testing.h).
+cudaError_t run_mma_peak(int kind, int iters, double* ops_per_s, int32_t* status,
+                         cudaStream_t stream);
+
 cudaError_t launch_prefill(const sq_packed_weight& w, int M, const int8_t* xq, const float* sx,
                            const float* x_out, const int32_t* idx, int n_out, float* y,
                            int32_t* T_out, int32_t* R_out, int32_t* status, cudaStream_t stream,

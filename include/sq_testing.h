@@ -46,6 +46,20 @@ sq_status sq_testing_nvfp4_stalled(const sq_nvfp4_matrix *w, const sq_nvfp4_matr
                                    int32_t skip_stage, uint64_t wait_ns, int32_t *dev_status,
                                    void *stream);
 
+/*
+ * Dense tensor-core throughput probe, the peak the prefill kernels are
+ * reported against: every SM issues `iters` x 4 back-to-back tcgen05.mma of
+ * one kind on operands resident in its shared memory (a fixed pseudo-random
+ * pattern; scales 1.0), accumulating in tensor memory.
+ *   kind 0: kind::i8, 128 x 256 x 32;  kind 1: kind::mxf4nvf4 (block 16),
+ *   128 x 256 x 64
+ *   ops_per_s  host: 2 x multiply-adds per second of device time (CUDA
+ *              events around one launch, after a warm-up launch)
+ * 1 <= iters <= 100000.  Synchronous on `stream`.
+ */
+sq_status sq_testing_mma_peak(int32_t kind, int32_t iters, double *ops_per_s, int32_t *dev_status,
+                              void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -187,3 +187,16 @@ def test_linear_rejects_mismatched_operands():
     for args in ((w, a), (a, a), (w, w)):
         with pytest.raises(sq.SQError):
             sq.nvfp4_linear(*args)
+
+
+def test_mma_peak_probe_is_plausible():
+    """The tensor-core probe the prefill fractions are reported against:
+    int8 and NVFP4 rates on this device, between a tenth of and twice the
+    nominal dense figures (4.5 and 9 P ops/s), NVFP4 above int8."""
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    i8 = sq.testing_mma_peak(0, status=st)
+    f4 = sq.testing_mma_peak(1, status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    assert 0.45e15 < i8 < 9e15 and 0.9e15 < f4 < 18e15
+    assert f4 > i8
