@@ -83,6 +83,7 @@ constexpr int kOffA = 0, kOffB = kBytesA, kOffSa = kOffB + kBytesB, kOffSb = kOf
 constexpr int kStageBytes = kOffSb + 2 * kBytesSf;  // 46 KB
 static_assert(kStageBytes % 1024 == 0, "stages must stay 1024-byte aligned");
 static_assert(kSfCol0 + 2 * kSfSet <= kTmemCols, "scale columns past the allocation");
+static_assert(BN % 64 == 0 && BN <= 192, "tiles start at 0 or 64 in a scale block and end in the next");
 // y staging for the epilogue: per warp 32 rows x 32 floats, rows 36 floats
 // apart (16-byte stores of 8 consecutive lanes hit distinct banks).
 constexpr int kStageRow = 36;
@@ -271,6 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int n0 = (tile / p.nt_m) * BN;
       const int cb0 = n0 >> 7;
       const bool two = cb0 + 1 < p.nblk_b;
+      const bool shifted = (n0 & 127) != 0;  // n0 % 128 is 0 or 64
       bool ok = true;
       for (int kb = 0; kb < p.nk; ++kb, ++g) {
         const int s = (int)(g % kStages);
@@ -279,6 +281,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         const uint8_t* st = smem + s * kStageBytes;
+        // Each lane reads its 16 bytes of every chunk (a 128-row block's four
+        // 32-row words for one 64-channel chunk) with one vector load; the
+        // tile's words are picked in registers.  Four-byte loads at a 16-byte
+        // lane stride would hit each bank four times, and the four warps'
+        // reads share the bandwidth with the copies and the MMAs.
         uint32_t wa[16], wb[32];
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
@@ -287,16 +294,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           wa[4 * kk + 1] = a.y;
           wa[4 * kk + 2] = a.z;
           wa[4 * kk + 3] = a.w;
+          const uint4 b0 = *reinterpret_cast<const uint4*>(st + kOffSb + 512 * kk + 16 * lane);
+          const uint4 b1 = two ? *reinterpret_cast<const uint4*>(st + kOffSb + kBytesSf + 512 * kk + 16 * lane)
+                               : make_uint4(0u, 0u, 0u, 0u);
+          const uint32_t w[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+          // tile row 32 j + lane is word j of the two blocks' words, or word
+          // j + 2 when the tile starts 64 rows into its first block
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            // tile row 32 j + lane: global row n0 + 32 j + lane, in scale
-            // block cb0 + ((n0 & 127) + 32 j) / 128, word ((n0 & 127) / 32 + j) % 4
-            const int wq = ((n0 & 127) >> 5) + j;
-            const bool live = j < BN / 32 && (wq < 4 || two);
-            wb[8 * kk + j] = live ? *reinterpret_cast<const uint32_t*>(
-                                        st + kOffSb + (wq >> 2) * kBytesSf + 512 * kk + 16 * lane + 4 * (wq & 3))
-                                  : 0u;
-          }
+          for (int j = 0; j < 8; ++j)
+            wb[8 * kk + j] = j < BN / 32 ? (shifted ? w[j + 2] : w[j]) : 0u;
         }
         const uint32_t ts = tmem + ((uint32_t)(32 * q) << 16) + kSfCol0 + kSfSet * (g & 1u);
         tmem_st16(ts, wa);
