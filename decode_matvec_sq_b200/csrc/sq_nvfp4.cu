@@ -84,11 +84,16 @@ constexpr int kStageBytes = kOffSb + 2 * kBytesSf;  // 46 KB
 static_assert(kStageBytes % 1024 == 0, "stages must stay 1024-byte aligned");
 static_assert(kSfCol0 + 2 * kSfSet <= kTmemCols, "scale columns past the allocation");
 static_assert(BN % 64 == 0 && BN <= 192, "tiles start at 0 or 64 in a scale block and end in the next");
-// y staging for the epilogue: per warp 32 rows x 32 floats, rows 36 floats
-// apart (16-byte stores of 8 consecutive lanes hit distinct banks).
+// y staging for the epilogue, per warp: two 32 x 32 float blocks in the
+// 128-byte-swizzled layout of a tensor store (16-byte chunk j of row r at
+// chunk j ^ (r % 8), so the 16-byte stores of 8 consecutive lanes hit distinct
+// banks); without the tensor store, one block with rows 36 floats apart.
 constexpr int kStageRow = 36;
 constexpr int kOffOut = kStages * kStageBytes;
-constexpr int kOutBytes = 4 * 32 * kStageRow * 4;  // 18 KB
+constexpr int kOutBlock = 32 * 32 * 4;         // 4 KB, 1024-byte aligned
+constexpr int kOutBytes = 4 * 2 * kOutBlock;   // 32 KB
+static_assert(kOffOut % 1024 == 0, "swizzled staging must be 1024-byte aligned");
+static_assert(4 * 32 * kStageRow * 4 <= kOutBytes, "padded staging past its area");
 
 struct Aux {
   uint64_t full[kStages], empty[kStages], sfr[kStages], accf[2], acce[2], drain;
@@ -161,9 +166,13 @@ __device__ __forceinline__ bool aborted(const Aux* aux) {
   return *reinterpret_cast<const volatile int*>(&aux->abort) != 0;
 }
 
+// TMA_Y: y leaves through tensor stores of the staged 32 x 32 blocks (y
+// 16-byte aligned and N % 4 = 0), else through 16-byte stores of whole
+// 128-byte row segments.
+template <bool TMA_Y>
 __global__ void __launch_bounds__(kThreads, 1)
     k_nvfp4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                 const Params p) {
+                 const __grid_constant__ CUtensorMap tmY, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Aux* aux = reinterpret_cast<Aux*>(smem + kOffOut + kOutBytes);
@@ -316,6 +325,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- epilogue: one token (TMEM lane) per thread
     const int q = warp & 3;  // TMEM lane quarter of this warp
     float* stage_out = reinterpret_cast<float*>(smem + kOffOut) + q * 32 * kStageRow;
+    uint8_t* blocks = smem + kOffOut + q * 2 * kOutBlock;  // TMA_Y: this warp's two blocks
+    uint32_t nb = 0;                                       // blocks stored so far
     const float gw = __ldg(p.gw);
     uint32_t n = 0;
     for (int tile = blockIdx.x; tile < p.tiles; tile += gridDim.x, ++n) {
@@ -335,35 +346,64 @@ __global__ void __launch_bounds__(kThreads, 1)
           fence_before();
           mbar_arrive(&aux->acce[b]);
         }
-        // this lane's row of the 32 x 32 block into shared memory
+        if constexpr (TMA_Y) {
+          const int x0 = n0 + 32 * h;
+          if (m0 >= p.M || x0 >= p.N) continue;  // the whole block is outside y
+          uint8_t* blk = blocks + (nb & 1u) * kOutBlock;
+          // the store that last read this block (two blocks ago) is done reading
+          if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+          __syncwarp();
 #pragma unroll
-        for (int i = 0; i < 32; i += 4)
-          *reinterpret_cast<float4*>(stage_out + lane * kStageRow + i) =
-              make_float4(sc * __int_as_float(r[i]), sc * __int_as_float(r[i + 1]),
-                          sc * __int_as_float(r[i + 2]), sc * __int_as_float(r[i + 3]));
-        __syncwarp();
-        // four rows per store: lanes 8j .. 8j+7 write row 4i + j, 128 bytes
-        const int cn = n0 + 32 * h + 4 * (lane & 7);
+          for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<float4*>(blk + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+                make_float4(sc * __int_as_float(r[4 * j]), sc * __int_as_float(r[4 * j + 1]),
+                            sc * __int_as_float(r[4 * j + 2]), sc * __int_as_float(r[4 * j + 3]));
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          __syncwarp();
+          if (lane == 0) {
+            // rows past M and columns past N are clipped by the tensor store
+            asm volatile(
+                "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                    reinterpret_cast<uint64_t>(&tmY)),
+                "r"(x0), "r"(m0), "r"(smem_u32(blk))
+                : "memory");
+            asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+          }
+          ++nb;
+        } else {
+          // this lane's row of the 32 x 32 block into shared memory
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int rr = 4 * i + (lane >> 3);
-          const int tt = m0 + rr;
-          const float4 v = *reinterpret_cast<const float4*>(stage_out + rr * kStageRow + 4 * (lane & 7));
-          if (tt < p.M) {
-            float* yp = p.y + (int64_t)tt * p.N + cn;
-            if (cn + 4 <= p.N && (p.N & 3) == 0) {
-              *reinterpret_cast<float4*>(yp) = v;
-            } else {
-              if (cn < p.N) yp[0] = v.x;
-              if (cn + 1 < p.N) yp[1] = v.y;
-              if (cn + 2 < p.N) yp[2] = v.z;
-              if (cn + 3 < p.N) yp[3] = v.w;
+          for (int i = 0; i < 32; i += 4)
+            *reinterpret_cast<float4*>(stage_out + lane * kStageRow + i) =
+                make_float4(sc * __int_as_float(r[i]), sc * __int_as_float(r[i + 1]),
+                            sc * __int_as_float(r[i + 2]), sc * __int_as_float(r[i + 3]));
+          __syncwarp();
+          // four rows per store: lanes 8j .. 8j+7 write row 4i + j, 128 bytes
+          const int cn = n0 + 32 * h + 4 * (lane & 7);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int rr = 4 * i + (lane >> 3);
+            const int tt = m0 + rr;
+            const float4 v = *reinterpret_cast<const float4*>(stage_out + rr * kStageRow + 4 * (lane & 7));
+            if (tt < p.M) {
+              float* yp = p.y + (int64_t)tt * p.N + cn;
+              if (cn + 4 <= p.N && (p.N & 3) == 0) {
+                *reinterpret_cast<float4*>(yp) = v;
+              } else {
+                if (cn < p.N) yp[0] = v.x;
+                if (cn + 1 < p.N) yp[1] = v.y;
+                if (cn + 2 < p.N) yp[2] = v.z;
+                if (cn + 3 < p.N) yp[3] = v.w;
+              }
             }
           }
+          __syncwarp();
         }
-        __syncwarp();
       }
     }
+    // the tensor stores have written y before the CTA leaves
+    if (TMA_Y && lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+    __syncwarp();
   }
   fence_before();
   __syncthreads();
@@ -665,9 +705,17 @@ cudaError_t launch_nvfp4_gemm(const sq_nvfp4_matrix& w, const sq_nvfp4_matrix& x
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
   const int grid = (int)std::min<int64_t>(tiles, sms);
-  e = ensure_smem_attr((const void*)k_nvfp4_gemm, kSmemBytes);
-  if (e != cudaSuccess) return e;
-  k_nvfp4_gemm<<<grid, kThreads, kSmemBytes, stream>>>(ma, mb, p);
+  CUtensorMap my;
+  const bool tma_y = (p.N & 3) == 0 && (reinterpret_cast<uintptr_t>(y) & 15u) == 0 &&
+                     tc05::make_map(&my, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, y, (uint64_t)p.N, (uint64_t)p.M,
+                                    (uint64_t)p.N * 4, 32, 32, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (tma_y) {
+    if ((e = ensure_smem_attr((const void*)k_nvfp4_gemm<true>, kSmemBytes)) != cudaSuccess) return e;
+    k_nvfp4_gemm<true><<<grid, kThreads, kSmemBytes, stream>>>(ma, mb, my, p);
+  } else {
+    if ((e = ensure_smem_attr((const void*)k_nvfp4_gemm<false>, kSmemBytes)) != cudaSuccess) return e;
+    k_nvfp4_gemm<false><<<grid, kThreads, kSmemBytes, stream>>>(ma, mb, ma, p);
+  }
   return cudaGetLastError();
 }
 
