@@ -38,8 +38,14 @@
 //   warp 1 (one lane): per stage, 4 block-scaled MMAs (K = 64 each) into one
 //     of two fp32 accumulators (tiles alternate);
 //   warps 2-5: read an accumulator back (tcgen05.ld), free it for the tile
-//     after next, scale by g_w g_x[t], and write y through shared memory so
-//     that each store instruction covers whole 128-byte row segments.
+//     after next, scale by g_w g_x[t], and stage y in shared memory in 32 x 32
+//     blocks that leave through tensor stores (else through stores of whole
+//     128-byte row segments; each thread storing its own row measured 117
+//     against 89 us).
+// Shared-memory bandwidth is the budget the roles share: per stage the copies
+// write 46 KB, the MMAs read 40 KB and the four scale warps each read the
+// stage's scales (16-byte loads: 4-byte loads at a 16-byte lane stride cost
+// four times the wavefronts and the launch 92 against 86 us).
 // The scales go in through the warps rather than tcgen05.cp: eight copies
 // per stage issued beside the MMAs took 131 us against 95 us per launch at
 // 2048 x 4096 -> 14336 (then with 128-row weight tiles; 192 rows took the
