@@ -351,24 +351,49 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
       // outlier channels: y += sum_i What[n][idx_i] * x_out[t][i], What from
       // the packed row (the dequantized weight); table in the free stage memory
+      // Thread et builds row nn = et % 64 of the table for the outliers
+      // i = et / 64 (mod 2), eight at a time: their channel indices first,
+      // then all their weight words, so that each batch costs two memory
+      // round trips instead of two per entry.
       float* wo = reinterpret_cast<float*>(smem);  // [64 outliers][BN]
+      static_assert(BN == 64, "two epilogue threads per weight row");
+      const int nn = et & (BN - 1), n = n0 + nn;
+      const bool live_row = n < p.N;
+      const int64_t nr = live_row ? n : 0;
       for (int i0 = 0; i0 < p.n_out; i0 += 64) {
         const int ni = min(64, p.n_out - i0);
         named_sync_epi();
-        for (int e = et; e < ni * BN; e += 128) {
-          const int i = e / BN, nn = e - i * BN, n = n0 + nn;
-          const int j = p.idx[i0 + i];
-          float w = 0.0f;
-          if (n < p.N && j >= 0 && j < p.K) {
-            const uint32_t bit = 1u << (j & 31);
-            const bool sgn = (p.sign[(int64_t)n * p.sign_stride + (j >> 5)] & bit) != 0;
-            const bool m = MASK ? (p.mask[(int64_t)n * p.sign_stride + (j >> 5)] & bit) != 0 : true;
-            const float al = aux->alpha[nn];
-            const float tr = m ? (sgn ? al : -al) : 0.0f;
-            w = fmaf(p.scale[(int64_t)n * p.scale_stride + (j >> 7)],
-                     (float)p.res[(int64_t)n * p.res_stride + j], tr);
+        for (int ib = et >> 6; ib < ni; ib += 16) {
+          int jj[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) jj[u] = ib + 2 * u < ni ? __ldg(p.idx + i0 + ib + 2 * u) : -1;
+          uint32_t sg[8], mk[8];
+          float sc[8];
+          int rs[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const bool ok = live_row && jj[u] >= 0 && jj[u] < p.K;
+            const int jc = ok ? jj[u] : 0;
+            sg[u] = ok ? __ldg(p.sign + nr * p.sign_stride + (jc >> 5)) : 0u;
+            mk[u] = (ok && MASK) ? __ldg(p.mask + nr * p.sign_stride + (jc >> 5)) : 0u;
+            sc[u] = ok ? __ldg(p.scale + nr * p.scale_stride + (jc >> 7)) : 0.0f;
+            rs[u] = ok ? (int)__ldg(p.res + nr * p.res_stride + jc) : 0;
           }
-          wo[i * BN + nn] = w;
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int i = ib + 2 * u, j = jj[u];
+            if (i >= ni) break;
+            float w = 0.0f;
+            if (live_row && j >= 0 && j < p.K) {
+              const uint32_t bit = 1u << (j & 31);
+              const bool sgn = (sg[u] & bit) != 0;
+              const bool m = MASK ? (mk[u] & bit) != 0 : true;
+              const float al = aux->alpha[nn];
+              const float tr = m ? (sgn ? al : -al) : 0.0f;
+              w = fmaf(sc[u], (float)rs[u], tr);
+            }
+            wo[i * BN + nn] = w;
+          }
         }
         named_sync_epi();
         if (t < p.M) {
