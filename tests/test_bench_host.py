@@ -117,3 +117,15 @@ def test_trunk_workload_cases():
         assert M == 1 and copies * bench.trunk_weight_bytes(L) >= 2 * bench.L2_BYTES
         # sign bits (1/8 byte per weight of the padded tile grid) + 4 bytes per padded row
         assert bench.trunk_weight_bytes(L) == (-(-L.N // 16) * 16) * (-(-L.K // 128) * 16 + 4)
+
+
+@pytest.mark.parametrize("n", [1, 4, 7, 8, 12, 20, 128, 129])
+def test_e2e_bounds_cover_every_linear_once(n):
+    """The end-to-end graph's chunks: strictly increasing starts from 0 to the
+    linear count, two-linear chunks first and last from 8 linears up."""
+    b = bench.e2e_bounds(n)
+    assert b[0] == 0 and b[-1] == n
+    assert all(x < y for x, y in zip(b, b[1:]))
+    if n >= 8:
+        assert b[1] == 2 and b[-2] == n - 2
+        assert all(y - x <= 16 for x, y in zip(b, b[1:]))
