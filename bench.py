@@ -100,6 +100,18 @@ def load_fp4_peak():
         return FALLBACK_BF16_TFLOPS * FP4_PER_BF16, "fallback bf16 x nominal fp4/bf16 ratio"
 
 
+def read_probe(device, nbytes: int = 2 << 30, iters: int = 10):
+    """The device's pure-read HBM rate in GB/s (sq_testing_read_peak over a
+    buffer 16x the L2), the decode kernels' second denominator."""
+    import torch
+    import decode_matvec_sq_b200 as sq
+    buf = torch.zeros(nbytes, dtype=torch.uint8, device=device)
+    gbs = sq.testing_read_peak(buf, iters=iters) / 1e9
+    del buf
+    torch.cuda.empty_cache()
+    return round(gbs, 1)
+
+
 def probe_peak(kind: int) -> float:
     """The dense tensor-core rate measured on this device by the library's
     probe (sq_testing_mma_peak): kind 0 int8, 1 NVFP4; T ops/s."""
@@ -1091,6 +1103,7 @@ def run_gpu(args, world, rank, local):
     side = None
     if rank == 0 and not args.no_side_configs:
         side = side_configs(device)
+    read_gbs = read_probe(device) if rank == 0 else None
 
     if rank == 0:
         line = {
@@ -1109,7 +1122,12 @@ def run_gpu(args, world, rank, local):
                                    if stack.fused else "k_linear_tc (decode linear, tensor cores)",
                          "bytes_per_launch": int(bytes_launch),
                          "us_per_launch": round(ms_launch * 1e3, 3),
-                         "timing": "timed PDL graph: step time / launches per step"},
+                         "timing": "timed PDL graph: step time / launches per step",
+                         "read_probe_peak": read_gbs,
+                         "frac_of_read_probe": round(achieved / read_gbs, 4) if read_gbs else None,
+                         "read_probe_kind": "measured on this device after the timed region: read-only "
+                                            "sweeps of a 2 GiB buffer, 16-byte coalesced loads "
+                                            "(sq_testing_read_peak)"},
             "clocks": clocks,
             "e2e": e2e,
             "cpu_baseline": cpu,

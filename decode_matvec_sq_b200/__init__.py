@@ -85,6 +85,7 @@ def lib():
         "sq_nvfp4_linear": ([nm, nm, vp, vp, vp], ctypes.c_int),
         "sq_testing_nvfp4_stalled": ([nm, nm, vp, i32, ctypes.c_uint64, vp, vp], ctypes.c_int),
         "sq_testing_mma_peak": ([i32, i32, ctypes.POINTER(ctypes.c_double), vp, vp], ctypes.c_int),
+        "sq_testing_read_peak": ([vp, ctypes.c_uint64, i32, ctypes.POINTER(ctypes.c_double), vp], ctypes.c_int),
         "sq_status_string": ([ctypes.c_int], ctypes.c_char_p),
         "sq_device_check": ([], ctypes.c_int),
         "sq_packed_bytes": ([i32, i32, i32, i32, i32], sz),
@@ -541,6 +542,18 @@ def testing_nvfp4_stalled(w: Nvfp4Matrix, x: Nvfp4Matrix, y, skip_stage: int, wa
     requested and every wait limited to wait_ns (tests of the timeout path)."""
     _ck(lib().sq_testing_nvfp4_stalled(ctypes.byref(w.view), ctypes.byref(x.view), _ptr(y), skip_stage,
                                        wait_ns, _ptr(status), _stream(stream)), "sq_testing_nvfp4_stalled")
+
+
+def testing_read_peak(buf, iters: int = 20, stream=None) -> float:
+    """include/sq_testing.h: bytes per second of read-only sweeps of a CUDA
+    tensor `buf` (contiguous, 16-byte aligned, size a multiple of 16)."""
+    if not buf.is_cuda or not buf.is_contiguous():
+        raise SQError(STATUS_CODE["SQ_ERR_INVALID_ARG"], "sq_testing_read_peak: a contiguous CUDA tensor")
+    out = ctypes.c_double(0.0)
+    nbytes = buf.numel() * buf.element_size()
+    _ck(lib().sq_testing_read_peak(buf.data_ptr(), nbytes, iters, ctypes.byref(out), _stream(stream)),
+        "sq_testing_read_peak")
+    return out.value
 
 
 def testing_mma_peak(kind: int, iters: int = 4000, status=None, stream=None) -> float:

@@ -672,3 +672,20 @@ extern "C" sq_status sq_testing_mma_peak(int32_t kind, int32_t iters, double* op
   if (st != SQ_OK) return st;
   return from_cuda(run_mma_peak(kind, iters, ops_per_s, dev_status, static_cast<cudaStream_t>(stream)));
 }
+
+namespace sq {
+// sq_probe.cu
+cudaError_t run_read_peak(const void* buf, size_t bytes, int iters, double* bytes_per_s,
+                          cudaStream_t stream);
+}  // namespace sq
+
+extern "C" sq_status sq_testing_read_peak(const void* buf, uint64_t bytes, int32_t iters,
+                                          double* bytes_per_s, void* stream) {
+  if (!buf || !bytes_per_s) return SQ_ERR_INVALID_ARG;
+  if (!aligned16(buf)) return SQ_ERR_ALIGN;
+  if (bytes < 16 || bytes % 16 != 0 || iters < 1 || iters > 1000) return SQ_ERR_SHAPE;
+  DeviceInfo d;
+  sq_status st = check_device(&d);
+  if (st != SQ_OK) return st;
+  return from_cuda(run_read_peak(buf, (size_t)bytes, iters, bytes_per_s, static_cast<cudaStream_t>(stream)));
+}

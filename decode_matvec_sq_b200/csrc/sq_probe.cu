@@ -1,7 +1,10 @@
-// sq_probe.cu -- the dense tensor-core peak the prefill kernels are measured
-// against, taken on the device itself: every SM issues back-to-back
-// tcgen05.mma of one kind on operands resident in its shared memory,
-// accumulating in tensor memory, with nothing else running.
+// sq_probe.cu -- the peaks the kernels are measured against, taken on the
+// device itself.
+// Tensor cores: every SM issues back-to-back tcgen05.mma of one kind on
+// operands resident in its shared memory, accumulating in tensor memory,
+// with nothing else running.
+// HBM reads: a read-only sweep of a caller's buffer larger than L2 (the
+// decode kernels only read weights; a copy also writes).
 //   kind 0: kind::i8 (s8 x s8 -> s32), M = 128, N = 256, K = 32
 //   kind 1: kind::mxf4nvf4 (E2M1 x E2M1, UE4M3 scales of 16), M = 128,
 //           N = 256, K = 64
@@ -97,7 +100,63 @@ __global__ void __launch_bounds__(kProbeThreads, 1) k_mma_peak(int iters, int32_
   }
 }
 
+// ---- pure-read sweep --------------------------------------------------------------
+constexpr int kReadThreads = 512, kReadUnroll = 8;
+__device__ int g_read_sink;
+
+// Every thread reads 16-byte words `stride` apart (consecutive threads,
+// consecutive words: one warp load covers 512 contiguous bytes), eight loads
+// in flight; the words are folded into one value so that no load is dead.
+__global__ void __launch_bounds__(kReadThreads) k_read_peak(const int4* __restrict__ p, size_t n4) {
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  int acc = 0;
+  for (; i + (kReadUnroll - 1) * stride < n4; i += kReadUnroll * stride) {
+    int4 v[kReadUnroll];
+#pragma unroll
+    for (int u = 0; u < kReadUnroll; ++u) v[u] = ldg_nc_v4(p + i + u * stride);
+#pragma unroll
+    for (int u = 0; u < kReadUnroll; ++u) acc ^= v[u].x ^ v[u].y ^ v[u].z ^ v[u].w;
+  }
+  for (; i < n4; i += stride) {
+    const int4 v = ldg_nc_v4(p + i);
+    acc ^= v.x ^ v.y ^ v.z ^ v.w;
+  }
+  if (acc == 0x5EED1234) g_read_sink = acc;  // (practically never taken)
+}
+
 }  // namespace
+
+// Bytes per second read by `iters` back-to-back sweeps of [buf, buf + bytes)
+// (bytes a multiple of 16), after one warm-up sweep.
+cudaError_t run_read_peak(const void* buf, size_t bytes, int iters, double* bytes_per_s,
+                          cudaStream_t stream) {
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  const int grid = 4 * sms;  // four 512-thread CTAs per SM
+  const int4* p = static_cast<const int4*>(buf);
+  const size_t n4 = bytes / 16;
+  cudaEvent_t a, b;
+  if ((e = cudaEventCreate(&a)) != cudaSuccess) return e;
+  if ((e = cudaEventCreate(&b)) != cudaSuccess) {
+    cudaEventDestroy(a);
+    return e;
+  }
+  k_read_peak<<<grid, kReadThreads, 0, stream>>>(p, n4);  // warm-up
+  cudaEventRecord(a, stream);
+  for (int it = 0; it < iters; ++it) k_read_peak<<<grid, kReadThreads, 0, stream>>>(p, n4);
+  cudaEventRecord(b, stream);
+  e = cudaEventSynchronize(b);
+  float ms = 0.0f;
+  if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, a, b);
+  cudaEventDestroy(a);
+  cudaEventDestroy(b);
+  if (e != cudaSuccess) return e;
+  *bytes_per_s = ms > 0.0f ? (double)bytes * iters / (ms * 1e-3) : 0.0;
+  return cudaGetLastError();
+}
 
 // Multiply-adds x 2 per second of one probe launch (iters x 4 MMAs per SM).
 cudaError_t run_mma_peak(int kind, int iters, double* ops_per_s, int32_t* status,

@@ -60,6 +60,21 @@ sq_status sq_testing_nvfp4_stalled(const sq_nvfp4_matrix *w, const sq_nvfp4_matr
 sq_status sq_testing_mma_peak(int32_t kind, int32_t iters, double *ops_per_s, int32_t *dev_status,
                               void *stream);
 
+/*
+ * Pure-read HBM probe, the second denominator of the decode kernels (which
+ * read weights and write almost nothing; a device copy also writes): `iters`
+ * back-to-back read-only sweeps of a caller's buffer, 16-byte coalesced
+ * loads, eight in flight per thread, four 512-thread CTAs per SM.
+ *   buf          device, 16-byte aligned, `bytes` readable bytes (contents
+ *                irrelevant); choose bytes well above the L2 size (126 MB)
+ *   bytes        a multiple of 16, >= 16
+ *   bytes_per_s  host: bytes x iters / device time (CUDA events around the
+ *                sweeps, after a warm-up sweep)
+ * 1 <= iters <= 1000.  Synchronous on `stream`.
+ */
+sq_status sq_testing_read_peak(const void *buf, uint64_t bytes, int32_t iters, double *bytes_per_s,
+                               void *stream);
+
 #ifdef __cplusplus
 }
 #endif
