@@ -21,6 +21,7 @@ from __future__ import annotations
 import argparse
 import json
 import os
+import platform
 import statistics
 import subprocess
 import sys
@@ -98,6 +99,20 @@ def load_fp4_peak():
         return float(d["bf16_tflops"]) * FP4_PER_BF16, "measured bf16 x nominal fp4/bf16 ratio"
     except Exception:
         return FALLBACK_BF16_TFLOPS * FP4_PER_BF16, "fallback bf16 x nominal fp4/bf16 ratio"
+
+
+def host_info():
+    """The host the oracle baseline ran on: logical CPUs and the CPU model."""
+    model = platform.processor() or ""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    model = ln.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"host_nproc": os.cpu_count(), "host_cpu": model}
 
 
 def read_probe(device, nbytes: int = 2 << 30, iters: int = 10):
@@ -298,7 +313,7 @@ def run_reference(args, world, rank):
         "vs_baseline": None, "dtype": "int8+f64", "data": "synthetic",
         "config": config_dict(args),
         "cpu_baseline": {"value": round(gbs, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": desc},
+                         "sample": desc, **host_info()},
         "e2e": {"value": round(gbs, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -1096,7 +1111,8 @@ def run_gpu(args, world, rank, local):
         cpu = {"value": round(gbs, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
                "sample": f"first {args.oracle_rows} rows of each linear of layer 0 "
                          f"({sbytes / 1e6:.1f} MB per pass, {passes} passes, "
-                         f"{per_pass * 1e3:.1f} ms per pass), quantize_act + linear"}
+                         f"{per_pass * 1e3:.1f} ms per pass), quantize_act + linear",
+               **host_info()}
         # the oracle's outputs for that sample against the timed graph's y
         parity = oracle_parity(sample, y_checked[:len(sample)])
 
