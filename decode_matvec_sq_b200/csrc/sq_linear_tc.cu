@@ -1012,7 +1012,13 @@ cudaError_t launch_linear_tc(const sq_packed_weight& w, int M, const int8_t* xq,
   if (T >= INT32_MAX / 2) return cudaErrorInvalidValue;
   p.T = (int)T;
   p.n_rb = (int)ceil_div(w.N, kTileRows);
-  const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((int64_t)sm_count * kBps, p.n_rb));
+  // The fewest CTAs with the largest share of row blocks that one CTA per SM
+  // gives: every CTA then streams the same number of row blocks (qkv: 128 x 6
+  // instead of 28 x 6 + 120 x 5) and none of them finishes alone with the
+  // memory system idle around it (7B-shaped stack on B200: 3798 -> 3896 GB/s).
+  const int64_t cap = std::max<int64_t>(1, std::min<int64_t>((int64_t)sm_count * kBps, p.n_rb));
+  const int64_t share = (p.n_rb + cap - 1) / cap;
+  const int64_t blocks = std::max<int64_t>(1, (p.n_rb + share - 1) / share);
   p.M = M;
   p.xq = xq;
   p.xs = (int)xq_stride_of(w.K);
