@@ -414,37 +414,37 @@ class Stack:
         return g
 
 
-def e2e_bounds(n: int, size: int = 16):
-    """Chunk starts for the end-to-end graph: the first and the last chunk two
-    linears each (the inputs that must arrive before any compute, the outputs
-    that return after all of it), chunks of `size` linears between them (the
-    last of them shorter); one linear per chunk for stacks under 8 linears.
-    Every chunk boundary costs a few microseconds of the step (measured on
-    B200, 7B-shaped stack: 8 equal chunks 3654-3685 GB/s, 16 equal 3638, 32
-    equal 3525; these bounds 3699)."""
-    if n < 8:
-        return list(range(n + 1))
-    b = [0, 2]
-    while b[-1] + size < n - 2:
-        b.append(b[-1] + size)
-    return b + [n - 2, n]
+def e2e_bounds(n: int):
+    """Where the end-to-end graph's copies join the compute stream.  Each join
+    costs the step time (measured on B200, 7B-shaped stack, with 16-byte copies
+    in the same graph shape: a wait of the compute stream for an input copy
+    about 4 us, a record that releases an output copy about 2 us), so there
+    are few of them:
+      inputs: linears [0, 2) first (the bytes that must land before any
+        compute), then [2, 12), then the rest, all on the copy stream from the
+        step's start; the compute stream waits before linears 0, 2 and 12;
+      outputs: back after every 32 linears and after the last two.
+    Returns (input group starts, output group starts), each from 0 to n."""
+    if n < 16:
+        return list(range(n + 1)), list(range(n + 1))
+    h2d = [0, 2, 12, n]
+    d2h = [0] + list(range(32, n - 2, 32)) + [n - 2, n]
+    return h2d, d2h
 
 
 def capture_e2e(stack, x_host, y_host, bounds=None):
     """One end-to-end step as a CUDA graph: the stack's inputs copied in from
-    pinned host memory and its outputs copied back, by chunks of linears on a
-    copy stream, so that a chunk's inputs arrive before its linears run and
-    its outputs go back while the later chunks compute.  Every byte of x and y
-    crosses each step; results are those of the plain step.  `bounds`: the
-    linears where chunks start (first 0, last the linear count), by default
-    e2e_bounds."""
+    pinned host memory and its outputs copied back on a copy stream, the inputs
+    by groups of linears issued at the step's start and each awaited before its
+    first linear, the outputs by groups sent back once their linears are done,
+    while the later linears compute.  Every byte of x and y crosses each step;
+    results are those of the plain step.  `bounds`: (input group starts,
+    output group starts), by default e2e_bounds."""
     import torch
     n = len(stack.pws)
-    if bounds is None:
-        bounds = e2e_bounds(n)
-    bounds = list(bounds)
-    chunks = len(bounds) - 1
-    assert bounds[0] == 0 and bounds[-1] == n and all(a < b for a, b in zip(bounds, bounds[1:]))
+    h2d, d2h = e2e_bounds(n) if bounds is None else bounds
+    for b in (h2d, d2h):
+        assert b[0] == 0 and b[-1] == n and all(x < y for x, y in zip(b, b[1:]))
     xoff, yoff = [0], [0]
     for L in stack.layers:
         xoff.append(xoff[-1] + L.K)
@@ -457,23 +457,28 @@ def capture_e2e(stack, x_host, y_host, bounds=None):
         fork = torch.cuda.Event()
         fork.record(s)
         sc.wait_event(fork)
-        x_in = []
-        for c in range(chunks):
-            a, b = xoff[bounds[c]], xoff[bounds[c + 1]]
+        x_in = {}
+        for c in range(len(h2d) - 1):
+            a, b = xoff[h2d[c]], xoff[h2d[c + 1]]
             with torch.cuda.stream(sc):
                 stack.x_all[a:b].copy_(x_host[a:b], non_blocking=True)
                 e = torch.cuda.Event()
                 e.record(sc)
-            x_in.append(e)
-        for c in range(chunks):
-            s.wait_event(x_in[c])
-            stack.step(lo=bounds[c], hi=bounds[c + 1])
-            done = torch.cuda.Event()
-            done.record(s)
-            sc.wait_event(done)
-            a, b = yoff[bounds[c]], yoff[bounds[c + 1]]
-            with torch.cuda.stream(sc):
-                y_host[a:b].copy_(stack.y_all[a:b], non_blocking=True)
+            x_in[h2d[c]] = e
+        ends = set(d2h[1:])
+        start = 0
+        for i in range(n):
+            if i in x_in:
+                s.wait_event(x_in[i])
+            stack.step(lo=i, hi=i + 1)
+            if i + 1 in ends:
+                done = torch.cuda.Event()
+                done.record(s)
+                sc.wait_event(done)
+                a, b = yoff[start], yoff[i + 1]
+                with torch.cuda.stream(sc):
+                    y_host[a:b].copy_(stack.y_all[a:b], non_blocking=True)
+                start = i + 1
         s.wait_stream(sc)
     torch.cuda.synchronize()
     return g, s
@@ -1099,9 +1104,10 @@ def run_gpu(args, world, rank, local):
                "us_per_token": round(ms_e2e * 1e3, 2),
                "h2d_bytes_per_step": int(stack.x_all.numel() * 4),
                "d2h_bytes_per_step": int(stack.y_all.numel() * 4),
-               "copies": "in the step's graph, by chunks of linears on a copy stream (two linears "
-                         "first and last, chunks of 16 between): a chunk's inputs in before its "
-                         "linears, its outputs back while later chunks run",
+               "copies": "in the step's graph on a copy stream: inputs issued at the step's start "
+                         "in three groups (linears 0-1, 2-11, the rest), each awaited before its "
+                         "first linear; outputs back after every 32 linears and after the last two, "
+                         "while later linears run",
                "outputs_equal_device": e2e_same}
 
     cpu, parity = None, None

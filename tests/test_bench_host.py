@@ -119,13 +119,16 @@ def test_trunk_workload_cases():
         assert bench.trunk_weight_bytes(L) == (-(-L.N // 16) * 16) * (-(-L.K // 128) * 16 + 4)
 
 
-@pytest.mark.parametrize("n", [1, 4, 7, 8, 12, 20, 128, 129])
+@pytest.mark.parametrize("n", [1, 4, 7, 8, 15, 16, 20, 40, 128, 129])
 def test_e2e_bounds_cover_every_linear_once(n):
-    """The end-to-end graph's chunks: strictly increasing starts from 0 to the
-    linear count, two-linear chunks first and last from 8 linears up."""
-    b = bench.e2e_bounds(n)
-    assert b[0] == 0 and b[-1] == n
-    assert all(x < y for x, y in zip(b, b[1:]))
-    if n >= 8:
-        assert b[1] == 2 and b[-2] == n - 2
-        assert all(y - x <= 16 for x, y in zip(b, b[1:]))
+    """The end-to-end graph's copy groups: for inputs and for outputs,
+    strictly increasing starts from 0 to the linear count; from 16 linears up
+    the first input group is two linears, the last output group two, and no
+    output group is longer than 32 linears."""
+    h2d, d2h = bench.e2e_bounds(n)
+    for b in (h2d, d2h):
+        assert b[0] == 0 and b[-1] == n
+        assert all(x < y for x, y in zip(b, b[1:]))
+    if n >= 16:
+        assert h2d[1] == 2 and d2h[-2] == n - 2
+        assert all(y - x <= 32 for x, y in zip(d2h, d2h[1:]))
