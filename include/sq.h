@@ -353,9 +353,9 @@ sq_status sq_linear_accumulators(const sq_packed_weight *w, const int8_t *xq, co
  * more fused passes than the decode kernel's passes of 8, and the workspace
  * is large enough, the call runs sq_quantize_act once into the workspace and
  * then sq_linear on its codes (two launches; y is the same bit for bit).
- * flags: SQ_LAUNCH_PDL (the kernel then reads x, idx and y-independent data
- * only after the previous kernel completes; the packed weights are streamed
- * before) and/or SQ_TRUNK_ONLY.
+ * flags: SQ_LAUNCH_PDL (the kernel then reads x and writes y only after the
+ * previous kernel completes; the packed weights and the index list are read
+ * before, as for every SQ_LAUNCH_PDL launch) and/or SQ_TRUNK_ONLY.
  */
 sq_status sq_quantize_linear(const sq_packed_weight *w, const float *x, int32_t M,
                              const int32_t *idx, int32_t n_out, float *y, void *workspace,
