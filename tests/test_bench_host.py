@@ -88,6 +88,8 @@ def test_reference_arm_under_torchrun_two_ranks():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["unit"] == "GB/s" and d["n_gpus"] == 2
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] == 1
+    assert d["cpu_baseline"]["host_nproc"] == os.cpu_count() >= 1
+    assert isinstance(d["cpu_baseline"]["host_cpu"], str)
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"] > 0
     assert d["metric"] == bench.METRIC and d["higher_is_better"] is True
 
