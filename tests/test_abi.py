@@ -322,3 +322,25 @@ def test_header_is_plain_c_and_links(tmp_path):
 
 def L_bytes() -> int:
     return sq.packed_bytes(64, 256, 128, False, sq.SQ_LAYOUT_TILES)
+
+
+def test_probe_host_checks(L):
+    """The peak probes refuse, before any device work: a null output or
+    buffer, a buffer not 16-byte aligned, a size that is not a positive
+    multiple of 16, an iteration count out of range, an unknown MMA kind."""
+    buf = ctypes.c_void_p(1 << 41)
+    out = ctypes.c_double(-1.0)
+    rp = L.sq_testing_read_peak
+    assert rp(None, 1 << 20, 10, ctypes.byref(out), None) == 1
+    assert rp(buf, 1 << 20, 10, None, None) == 1
+    assert rp(ctypes.c_void_p((1 << 41) + 8), 1 << 20, 10, ctypes.byref(out), None) == 3
+    for nbytes in (0, 8, 40):
+        assert rp(buf, nbytes, 10, ctypes.byref(out), None) == 2
+    for iters in (0, 1001):
+        assert rp(buf, 1 << 20, iters, ctypes.byref(out), None) == 2
+    mp = L.sq_testing_mma_peak
+    assert mp(2, 100, ctypes.byref(out), None, None) == 1
+    assert mp(0, 100, None, None, None) == 1
+    for iters in (0, 100001):
+        assert mp(1, iters, ctypes.byref(out), None, None) == 2
+    assert out.value == -1.0  # untouched on a refusal
